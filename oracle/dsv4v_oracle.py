@@ -1,0 +1,234 @@
+"""fp64 CPU oracle of the DeepSeek-V4-Flash vision tower forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's CPU-baseline leg
+may import this module.  The CUDA library never calls it, and it imports nothing from the CUDA
+path: it is a plain, slow restatement of what the pages define, in float64, with numpy's matmul
+as the only library primitive.  No blocking, fusion or reordering beyond the definitions.
+
+Sources (page title, then section):
+  [vision-API]  "nemo_automodel.components.models.deepseek_v4.vision" API reference
+                (classes DeepseekV4VisionRMSNorm / Attention / MLP / Block / Transformer /
+                Aligner, functions apply_vision_rotary, get_vision_cos_sin)
+  [model-API]   "nemo_automodel.components.models.deepseek_v4.model" API reference
+                (DeepseekV4Model.encode_image, merge_image_embeddings, the THD
+                cu_seqlens helpers)
+  [PR]          NeMo-Automodel pull request "Add native AutoModel support for
+                deepseek-ai/DeepSeek-V4-Flash-Vision-Exp", Changelog and Validation
+
+Where the pages leave a step open the function says "READING n"; the design notes list every
+reading.  Every function is pinned by the not-gpu tests (closed forms, invariants, brute force
+on tiny inputs, a hand-written aligner table) -- none is "parity unpinned" except that the
+*choice* among the readings themselves cannot be pinned without the released weights.
+
+Layouts: activations are packed varlen ``[P, D]`` (all images' patches back to back, patch
+``p = h * n_w + w`` row-major inside an image, READING 12); ``grids`` is a list of (n_h, n_w);
+weights are ``[out, in]``.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def cu_from_grids(grids) -> np.ndarray:
+    """Packed varlen offsets in the cu_seqlens form of [model-API, THD packing helpers]:
+    length n_images + 1, starting at 0, entry i+1 - entry i = n_h * n_w of image i."""
+    cu = [0]
+    for n_h, n_w in grids:
+        cu.append(cu[-1] + n_h * n_w)
+    return np.asarray(cu, dtype=np.int64)
+
+
+# --------------------------------------------------------------------------------------------
+# RMSNorm  [vision-API, DeepseekV4VisionRMSNorm]: RMSNorm over the last axis with an fp32
+# scale parameter, eps default 1e-6.  READING 3: y = w * x / sqrt(mean(x^2) + eps), with the
+# weight applied directly (not 1 + w).
+# --------------------------------------------------------------------------------------------
+def rmsnorm(x, weight, eps: float = 1e-6) -> np.ndarray:
+    x = _f64(x)
+    mean_sq = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(mean_sq + eps) * _f64(weight)
+
+
+# --------------------------------------------------------------------------------------------
+# 2D rotary table  [vision-API, get_vision_cos_sin]: the table for an n_h x n_w patch grid,
+# layout [n_h*n_w, 1, dim] on the page; the singleton head axis is dropped here.
+# READING 2: dim = head_dim / 2 (the table is what apply_vision_rotary consumes, whose cos/sin
+# layout is [patches, 1, head_dim/2]).
+# READING 1: the first dim/2 angles rotate by the patch's row index, the last dim/2 by its
+# column index; both halves share inv_freq_k = theta ** (-k / (dim/2)), k < dim/2; positions are
+# the integer grid coordinates of the patch inside its own image, starting at 0.
+# --------------------------------------------------------------------------------------------
+def vision_cos_sin(n_h: int, n_w: int, dim: int, theta: float):
+    if dim % 2:
+        raise ValueError("the 2D table needs an even width (head_dim % 4 == 0)")
+    quarter = dim // 2
+    inv_freq = np.asarray([theta ** (-k / quarter) for k in range(quarter)], dtype=np.float64)
+    angles = np.zeros((n_h * n_w, dim), dtype=np.float64)
+    for h in range(n_h):
+        for w in range(n_w):
+            p = h * n_w + w
+            angles[p, :quarter] = h * inv_freq
+            angles[p, quarter:] = w * inv_freq
+    return np.cos(angles), np.sin(angles)
+
+
+def packed_cos_sin(grids, dim: int, theta: float):
+    """Per-image tables stacked in packing order: row p of the result belongs to the patch in
+    row p of the packed activations (each image restarts at position (0, 0))."""
+    cs = [vision_cos_sin(h, w, dim, theta) for h, w in grids]
+    return np.concatenate([c for c, _ in cs]), np.concatenate([s for _, s in cs])
+
+
+# --------------------------------------------------------------------------------------------
+# Half-split rotation  [vision-API, apply_vision_rotary]: x [patches, heads, head_dim],
+# cos/sin [patches, 1, head_dim/2].  "Half-split": channel j pairs with channel j + head_dim/2
+# (the rotate-half convention); the pair is rotated by the angle of column j of the table.
+# --------------------------------------------------------------------------------------------
+def apply_vision_rotary(x, cos, sin) -> np.ndarray:
+    x = _f64(x)
+    half = x.shape[-1] // 2
+    c = _f64(cos)[:, None, :]
+    s = _f64(sin)[:, None, :]
+    first, second = x[..., :half], x[..., half:]
+    return np.concatenate([first * c - second * s, second * c + first * s], axis=-1)
+
+
+# --------------------------------------------------------------------------------------------
+# Attention  [vision-API, DeepseekV4VisionAttention / DeepseekV4VisionTransformer]: "full
+# bidirectional patch attention", "full attention over one image".  READING 6: scale
+# 1/sqrt(head_dim), no mask, no bias, no sinks.  READING 11: images of a packed batch never
+# attend to each other.
+# --------------------------------------------------------------------------------------------
+def attention_probs(q, k) -> np.ndarray:
+    """softmax(q k^T / sqrt(hd)) for one image and one head; q, k [N, hd] -> [N, N]."""
+    q, k = _f64(q), _f64(k)
+    scores = q @ k.T / math.sqrt(q.shape[-1])
+    scores = scores - scores.max(axis=1, keepdims=True)
+    e = np.exp(scores)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def attention_one_image(q, k, v) -> np.ndarray:
+    """q, k, v [N, H, hd] of one image -> [N, H*hd], heads concatenated in head order
+    (READING 5)."""
+    n, n_heads, hd = q.shape
+    out = np.zeros((n, n_heads, hd), dtype=np.float64)
+    for h in range(n_heads):
+        out[:, h, :] = attention_probs(q[:, h, :], k[:, h, :]) @ _f64(v[:, h, :])
+    return out.reshape(n, n_heads * hd)
+
+
+def attention_packed(q, k, v, grids) -> np.ndarray:
+    cu = cu_from_grids(grids)
+    return np.concatenate([attention_one_image(q[a:b], k[a:b], v[a:b])
+                           for a, b in zip(cu[:-1], cu[1:])])
+
+
+# --------------------------------------------------------------------------------------------
+# SwiGLU MLP  [vision-API, DeepseekV4VisionMLP]: "bias-free SwiGLU", [P, D] -> [P, D].
+# READING 7: silu(y Wg^T) * (y Wu^T), then Wd; silu(z) = z / (1 + exp(-z)); no clamp.
+# --------------------------------------------------------------------------------------------
+def silu(z) -> np.ndarray:
+    z = _f64(z)
+    return z / (1.0 + np.exp(-z))
+
+
+def mlp(y, w_gate, w_up, w_down) -> np.ndarray:
+    y = _f64(y)
+    return (silu(y @ _f64(w_gate).T) * (y @ _f64(w_up).T)) @ _f64(w_down).T
+
+
+def qkv_rope(y, wqkv, cos, sin, n_heads: int):
+    """The fused projection [vision-API, DeepseekV4VisionAttention.wqkv] followed by the
+    rotation of q and k.  READING 5: rows of wqkv are q | k | v blocks of D rows, head-major
+    inside each block.  READING 4: no bias.  Returns q, k, v as [P, H, hd]."""
+    y = _f64(y)
+    d = y.shape[1]
+    hd = d // n_heads
+    qkv = y @ _f64(wqkv).T
+    q = qkv[:, :d].reshape(-1, n_heads, hd)
+    k = qkv[:, d:2 * d].reshape(-1, n_heads, hd)
+    v = qkv[:, 2 * d:].reshape(-1, n_heads, hd)
+    return apply_vision_rotary(q, cos, sin), apply_vision_rotary(k, cos, sin), v
+
+
+# --------------------------------------------------------------------------------------------
+# Block  [vision-API, DeepseekV4VisionBlock]: pre-norm attention and MLP residual block,
+# x + attn(norm1(x)), then x + mlp(norm2(x)).  The output projection after attention has no
+# name on the pages (READING 4: bias-free, weight wo [D, D]).
+# --------------------------------------------------------------------------------------------
+def block_forward(x, layer: dict, cos, sin, grids, n_heads: int, eps: float = 1e-6) -> np.ndarray:
+    x = _f64(x)
+    y = rmsnorm(x, layer["norm1_w"], eps)
+    q, k, v = qkv_rope(y, layer["wqkv"], cos, sin, n_heads)
+    x = x + attention_packed(q, k, v, grids) @ _f64(layer["wo"]).T
+    y = rmsnorm(x, layer["norm2_w"], eps)
+    return x + mlp(y, layer["w_gate"], layer["w_up"], layer["w_down"])
+
+
+# --------------------------------------------------------------------------------------------
+# Tower  [vision-API, DeepseekV4VisionTransformer.forward]: blocks in order, then the tower's
+# `norm` (READING 8: applied after the last block; None skips it).  Starts from patch states
+# [P, D] (the patch embedding is outside this path).
+# --------------------------------------------------------------------------------------------
+def tower_forward(x, layers, final_norm_w, grids, n_heads: int, rope_theta: float = 10000.0,
+                  eps: float = 1e-6) -> np.ndarray:
+    x = _f64(x)
+    hd = x.shape[1] // n_heads
+    cos, sin = packed_cos_sin(grids, hd // 2, rope_theta)
+    for layer in layers:
+        x = block_forward(x, layer, cos, sin, grids, n_heads, eps)
+    if final_norm_w is not None:
+        x = rmsnorm(x, final_norm_w, eps)
+    return x
+
+
+# --------------------------------------------------------------------------------------------
+# Aligner  [vision-API, DeepseekV4VisionAligner]: spatially downsample each image's patch grid
+# by downsample_ratio in both directions and project to the LLM width.
+# READING 9: the grid is zero-padded at the bottom/right to a multiple of r; merged token
+# (i, j) is the concatenation, over a (outer) and b (inner) in [0, r), of the patch vector at
+# grid position (r*i + a, r*j + b) -> channel (a*r + b)*D + c; tokens are row-major over (i, j);
+# the projection is one bias-free linear r*r*D -> E.
+# --------------------------------------------------------------------------------------------
+def aligner_merge(x, grids, r: int):
+    """Returns the merged token matrix [T, r*r*D] and the token offsets [n_images + 1]."""
+    x = _f64(x)
+    d = x.shape[1]
+    cu = cu_from_grids(grids)
+    rows, cu_tok = [], [0]
+    for (n_h, n_w), start in zip(grids, cu[:-1]):
+        g_h, g_w = -(-n_h // r), -(-n_w // r)
+        padded = np.zeros((g_h * r, g_w * r, d), dtype=np.float64)
+        padded[:n_h, :n_w] = x[start:start + n_h * n_w].reshape(n_h, n_w, d)
+        for i in range(g_h):
+            for j in range(g_w):
+                parts = [padded[r * i + a, r * j + b] for a in range(r) for b in range(r)]
+                rows.append(np.concatenate(parts))
+        cu_tok.append(cu_tok[-1] + g_h * g_w)
+    return np.stack(rows), np.asarray(cu_tok, dtype=np.int64)
+
+
+def aligner_forward(x, w_align, grids, r: int):
+    merged, cu_tok = aligner_merge(x, grids, r)
+    return merged @ _f64(w_align).T, cu_tok
+
+
+def encode(inp, n_layers: int | None = None):
+    """Whole path for one drawn input set (vision_transformer_encoder_dsv4v_b200.synth.Inputs):
+    tower (first ``n_layers`` layers) then, if drawn, final norm and aligner.  Returns
+    (tower_out [P, D], aligner_out [T, E] or None)."""
+    wl = inp.wl
+    layers = [{k: (t.values if hasattr(t, "values") else t) for k, t in layer.items()}
+              for layer in inp.layers[:n_layers]]
+    out = tower_forward(inp.x.values, layers, inp.final_norm_w, wl.grids, wl.n_heads,
+                        wl.rope_theta, wl.eps)
+    if inp.w_align is None:
+        return out, None
+    return out, aligner_forward(out, inp.w_align.values, wl.grids, wl.downsample_ratio)[0]
