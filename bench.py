@@ -1,0 +1,412 @@
+"""Throughput of the vision-tower forward (32 bf16 blocks + final norm + aligner) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 4|5]
+
+One step = one pass of the whole path over one batch: copy the resident patch states into the
+working buffer, dsv4v_tower_forward, dsv4v_aligner_forward.  Default workload: one 28x28 image
+(784 patches, 196 tokens), seeded synthetic inputs and random-init weights of the tower's shape.
+Under torchrun each rank runs its own replica of the batch (images are independent, so the
+path shards by image with no collective; weak scaling); the reported time is the max over
+ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
+workload (the only other place this script runs the oracle besides the cpu_baseline leg).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from vision_transformer_encoder_dsv4v_b200 import synth  # noqa: E402
+
+METRIC = "ViT tower patches/sec and TFLOP/s (bf16, 1 B200) vs dense bf16 roofline"
+UNIT = "patches/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=4, choices=[4, 5])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def workload_desc(wl):
+    return {"workload": f"{wl.name}: {len(wl.grids)} image(s), {wl.n_patches} patches -> {wl.n_tokens} tokens, "
+                        f"D={wl.vision_dim} H={wl.n_heads} F={wl.mlp_hidden} r={wl.downsample_ratio} "
+                        f"E={wl.llm_dim} L={wl.n_layers}",
+            "grids": wl.grids, "patches_per_gpu": wl.n_patches, "tokens_per_gpu": wl.n_tokens,
+            "flops_per_gpu_step": synth.algorithmic_flops(wl)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle timing
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def time_oracle(wl, inp, budget_s):
+    """Runs the oracle on a bounded sample: whole layers of the tower (plus the aligner when the
+    budget allows), and scales to patches/s of the full workload by the counted work."""
+    from oracle import dsv4v_oracle as O
+    layers = [{k: (v.values if hasattr(v, "values") else v) for k, v in l.items()} for l in inp.layers]
+    cos, sin = O.packed_cos_sin(wl.grids, wl.head_dim // 2, wl.rope_theta)
+    x = inp.x.values.astype(np.float64)
+    t0 = time.perf_counter()
+    done = 0
+    while done < wl.n_layers:
+        x = O.block_forward(x, layers[done], cos, sin, wl.grids, wl.n_heads, wl.eps)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    t_layers = time.perf_counter() - t0
+    aligner_s = 0.0
+    if done == wl.n_layers:
+        t1 = time.perf_counter()
+        x = O.rmsnorm(x, inp.final_norm_w, wl.eps)
+        O.aligner_forward(x, inp.w_align.values, wl.grids, wl.downsample_ratio)
+        aligner_s = time.perf_counter() - t1
+    per_layer = t_layers / done
+    full_s = per_layer * wl.n_layers + (aligner_s if done == wl.n_layers else
+                                         per_layer * synth.algorithmic_flops(wl, 0, True) /
+                                         synth.algorithmic_flops(wl, 1, False))
+    sample = (f"{done} of {wl.n_layers} tower layers" + (" + final norm + aligner" if done == wl.n_layers else "") +
+              f" of the same workload in {t_layers + aligner_s:.1f} s; full step extrapolated by counted work")
+    return {"value": wl.n_patches / full_s, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": sample, "seconds_per_step_full": full_s}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = synth.workload(args.workload)
+    inp = synth.draw(wl)
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    last = None
+    for i in range(args.warmup + args.steps):
+        r = time_oracle(wl, inp, budget)
+        if i >= args.warmup:
+            vals.append(r["value"])
+        last = r
+    v = statistics.median(vals) if vals else last["value"]
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * wl.n_patches / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_desc(wl),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                             "sample": "each step: " + last["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+
+    from vision_transformer_encoder_dsv4v_b200 import build as B
+    from vision_transformer_encoder_dsv4v_b200 import dsv4v as A
+
+    B.build()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if dist is not None:
+            t = torch.ones(1, device="cuda")
+            dist.all_reduce(t)
+        torch.cuda.synchronize()
+
+    wl = synth.workload(args.workload)
+    inp = synth.draw(wl)
+    cfg = A.make_config(wl.vision_dim, wl.n_heads, wl.mlp_hidden, wl.downsample_ratio, wl.llm_dim, wl.n_layers,
+                        wl.eps, wl.rope_theta, A.DSV4V_BF16)
+    batch = A.BatchRef(wl.grids)
+
+    def dev(t):
+        return torch.from_numpy(t.bits.view(np.int16).copy()).view(torch.bfloat16).cuda()
+
+    layers = [{k: (torch.from_numpy(v).cuda() if isinstance(v, np.ndarray) else dev(v)) for k, v in l.items()}
+              for l in inp.layers]
+    lw = [A.block_weights(l) for l in layers]
+    fnw = torch.from_numpy(inp.final_norm_w).cuda()
+    wa = dev(inp.w_align)
+    x0 = dev(inp.x)
+    x = torch.empty_like(x0)
+    T = A.dsv4v_aligner_tokens(cfg, batch)
+    out = torch.empty(T, wl.llm_dim, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(A.dsv4v_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(s):
+        x.copy_(x0)
+        A.dsv4v_tower_forward(cfg, batch, lw, fnw, x, ws, stream=s.cuda_stream)
+        A.dsv4v_aligner_forward(cfg, batch, x, wa, out, ws, stream=s.cuda_stream)
+
+    # Capture one step (all kernels of the path, launched through the C ABI) in a CUDA graph.
+    with torch.cuda.stream(stream):
+        step(stream)  # warm the descriptor cache and function attributes
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(stream)
+    torch.cuda.synchronize()
+    if A.dsv4v_device_error() != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+    launches_per_step = 7 * wl.n_layers + 4  # per layer: 2 norms, 4 GEMMs, attention; rope table, final norm,
+    #                                          aligner index, aligner GEMM
+
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            graph.replay()
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            flush.zero_()  # L2 flush between steps, outside the timed interval
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+    stream.synchronize()
+    barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if A.dsv4v_device_error() != 0:
+        raise RuntimeError("device-side wait timed out")
+    ms = total_ms / args.steps
+    patches_all = wl.n_patches * world
+    value = patches_all * args.steps / (total_ms / 1e3)
+    tflops = synth.algorithmic_flops(wl) * world * args.steps / (total_ms / 1e3) / 1e12
+
+    # ---- kernel timing pass: the same step as component calls, with events around each launch
+    kern = kernel_timing(A, torch, cfg, batch, wl, layers, fnw, wa, x0, x, out, ws, stream, flush, args.steps)
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    x_host = x0.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            x.copy_(x_host, non_blocking=True)
+            A.dsv4v_tower_forward(cfg, batch, lw, fnw, x, ws, stream=stream.cuda_stream)
+            A.dsv4v_aligner_forward(cfg, batch, x, wa, out, ws, stream=stream.cuda_stream)
+            out_host.copy_(out, non_blocking=True)
+            b.record(stream)
+        stream.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_total = sum(e2e_ms)
+    if dist is not None:
+        t = torch.tensor([e2e_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = patches_all * args.steps / (e2e_total / 1e3)
+
+    peaks = load_peaks()
+    dom = kern["dominant"]
+    peak = peaks.get("bf16_tflops_sustained") or 1400.0
+    roof = {"bound": "tensor", "kernel": dom["name"], "achieved": dom["tflops"], "peak": peak, "unit": "TFLOP/s",
+            "frac": dom["tflops"] / peak, "traffic": None,
+            "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained (of measured)" if peaks else "fallback 1.4 PF",
+            "step_tflops": tflops, "step_frac": tflops / peak}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle(wl, inp, args.cpu_seconds)
+
+    if rank == 0:
+        cfgd = workload_desc(wl)
+        cfgd.update({"parallelism": f"replicas x{world} (image-parallel, no collective)",
+                     "l2": "flushed between timed steps (256 MB write outside the timed interval); "
+                           "weights (0.8 GB) exceed L2 anyway",
+                     "timing": "CUDA events per step around a CUDA-graph replay of the C-ABI calls",
+                     "graph": True})
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) patch states, N(0,0.02) "
+                "random-init weights of the tower's shape)", "config": cfgd,
+                "tflops": tflops, "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms),
+                "roofline": roof, "kernels": kern["all"], "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x0.numel() * 2,
+                        "d2h_bytes_per_step": out.numel() * 2,
+                        "path": "dsv4v_tower_forward + dsv4v_aligner_forward direct C-ABI calls (no graph), "
+                                "pinned host input/output copies inside the timed region"},
+                "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def kernel_timing(A, torch, cfg, batch, wl, layers, fnw, wa, x0, x, out, ws, stream, flush, steps):
+    """Per-launch device time of each kernel of the step, from CUDA events recorded on the
+    launching stream around every launch of the step issued as component calls (same kernels,
+    same plans as the tower entry point) inside one CUDA graph."""
+    D, F, P = wl.vision_dim, wl.mlp_hidden, wl.n_patches
+    hd2 = wl.head_dim // 2
+    cos = torch.empty(P, hd2, device="cuda")
+    sin = torch.empty_like(cos)
+    y = torch.empty(P, D, dtype=torch.bfloat16, device="cuda")
+    qkv = torch.empty(P, 3 * D, dtype=torch.bfloat16, device="cuda")
+    attn = torch.empty(P, D, dtype=torch.bfloat16, device="cuda")
+    h = torch.empty(P, F, dtype=torch.bfloat16, device="cuda")
+    s = stream.cuda_stream
+    names = ["rmsnorm", "gemm_qkv_rope", "attention", "gemm_out_resid", "gemm_swiglu", "gemm_down_resid"]
+    flops = {"gemm_qkv_rope": 2.0 * P * D * 3 * D, "gemm_out_resid": 2.0 * P * D * D,
+             "gemm_swiglu": 2.0 * P * D * 2 * F, "gemm_down_resid": 2.0 * P * F * D,
+             "attention": sum(4.0 * (a * b) ** 2 * D for a, b in wl.grids)}
+    events = {n: [] for n in names}
+
+    def timed(name, fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        events[name].append((a, b))
+
+    def one_step():
+        x.copy_(x0)
+        A.dsv4v_rope2d_table(cfg, batch, cos, sin, stream=s)
+        for l in layers:
+            timed("rmsnorm", lambda: A.dsv4v_rmsnorm(cfg, P, x, l["norm1_w"], y, stream=s))
+            timed("gemm_qkv_rope", lambda: A.dsv4v_qkv_rope(cfg, batch, y, l["wqkv"], cos, sin, qkv, ws, stream=s))
+            timed("attention", lambda: A.dsv4v_attention(cfg, batch, qkv, attn, stream=s))
+            timed("gemm_out_resid", lambda: A.dsv4v_linear_residual(cfg, P, D, attn, l["wo"], x, ws, stream=s))
+            timed("rmsnorm", lambda: A.dsv4v_rmsnorm(cfg, P, x, l["norm2_w"], y, stream=s))
+            timed("gemm_swiglu", lambda: A.dsv4v_swiglu(cfg, P, y, l["w_gate"], l["w_up"], h, ws, stream=s))
+            timed("gemm_down_resid", lambda: A.dsv4v_linear_residual(cfg, P, F, h, l["w_down"], x, ws, stream=s))
+
+    with torch.cuda.stream(stream):
+        one_step()
+    torch.cuda.synchronize()
+    for n in names:
+        events[n].clear()
+    for _ in range(steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            one_step()
+    torch.cuda.synchronize()
+    res = {}
+    for n in names:
+        ts = [a.elapsed_time(b) for a, b in events[n]]
+        avg_us = 1e3 * sum(ts) / len(ts)
+        r = {"launches": len(ts), "avg_us": avg_us, "total_ms": sum(ts)}
+        if n in flops:
+            r["tflops"] = flops[n] / (avg_us * 1e-6) / 1e12
+        if n == "rmsnorm":
+            r["gbs"] = 2.0 * P * D * 2 / (avg_us * 1e-6) / 1e9
+        res[n] = r
+    dom_name = max((n for n in names if n in flops), key=lambda n: res[n]["total_ms"])
+    return {"all": res, "dominant": {"name": dom_name, **res[dom_name]}}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return json.load(fh)
+    except Exception:
+        return {}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * dsv4v -- C ABI of a B200 (sm_100a) forward pass of the DeepSeek-V4-Flash vision tower
+ * and aligner.
+ *
+ * Sources (page title, then section):
+ *   [vision-API]  "nemo_automodel.components.models.deepseek_v4.vision" API reference
+ *   [model-API]   "nemo_automodel.components.models.deepseek_v4.model" API reference
+ *   [PR]          NeMo-Automodel pull request adding DeepSeek-V4-Flash-Vision-Exp
+ *                 (Changelog, Validation)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Packed varlen layout.  The patches of all images of a batch are stored back to back:
+ *    activations are row-major [P, vision_dim] with P = sum_i n_h[i] * n_w[i].  Inside an image
+ *    patch p = h * n_w + w (row-major over the grid, as the [n_h * n_w, vision_dim] layouts of
+ *    [vision-API, DeepseekV4VisionTransformer.forward] imply).  Offsets follow the cu_seqlens
+ *    form of [model-API, THD packing helpers]: int32, n_images + 1 entries, cu[0] = 0,
+ *    cu[i + 1] - cu[i] = n_h[i] * n_w[i].
+ *  - Images never interact: attention and the aligner merge stay inside an image, so packing
+ *    several images changes no result.
+ *  - Weights are row-major [out_features, in_features] (nn.Linear layout).  wqkv stacks the q,
+ *    k and v projections as three blocks of vision_dim rows, head-major inside each block.
+ *    RMSNorm scales are always fp32.  Every projection is bias-free.
+ *  - dtype DSV4V_BF16: activations, residual stream and projection weights are bf16; GEMMs
+ *    accumulate in fp32; RMSNorm, the rotary rotation, softmax and SiLU run in fp32 and round
+ *    once to bf16.  dtype DSV4V_F32: everything fp32 (CUDA-core path for small widths).
+ *  - The caller owns every buffer.  All device pointers must be on the current CUDA device.
+ *    The library allocates no device memory; scratch space is the caller's `workspace`
+ *    (size from dsv4v_workspace_size, 256-byte aligned).
+ *  - Every call is asynchronous and ordered on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Argument, shape and workspace errors are reported synchronously, before any
+ *    kernel is launched.  A bounded device-side wait that gives up records an error that
+ *    dsv4v_device_error() returns after synchronising the stream.
+ *  - Calls on the same workspace must not overlap on the GPU (put them on one stream).
+ *  - No call keeps device state between calls; each call may be captured in a CUDA graph
+ *    (the launch geometry is taken from the host copies of the grids and offsets, which must
+ *    equal the device copies).
+ */
+#ifndef DSV4V_H
+#define DSV4V_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSV4V_OK = 0,
+  DSV4V_ERR_INVALID_ARG = 1,   /* null pointer, bad grid/offset, inconsistent sizes */
+  DSV4V_ERR_UNSUPPORTED = 2,   /* shape outside the constraints listed at the config below */
+  DSV4V_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or smaller than required */
+  DSV4V_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  DSV4V_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (see dsv4v_device_error) */
+} dsv4v_status;
+
+typedef enum { DSV4V_F32 = 0, DSV4V_BF16 = 1 } dsv4v_dtype;
+
+/* Model dimensions ([vision-API] DeepseekV4VisionAttention: head_dim = vision_dim / n_heads;
+ * DeepseekV4VisionAligner: downsample_ratio; DeepseekV4VisionRMSNorm: eps default 1e-6;
+ * DeepseekV4VisionTransformer: rope_theta).
+ * Constraints: all sizes > 0; vision_dim % n_heads == 0; head_dim % 4 == 0 (the 2D table
+ * splits head_dim / 2 angles between rows and columns).
+ * DSV4V_BF16 additionally: head_dim == 64, vision_dim % 128 == 0, mlp_hidden % 128 == 0,
+ * llm_dim % 128 == 0.  Otherwise DSV4V_ERR_UNSUPPORTED. */
+typedef struct {
+  int vision_dim;        /* D */
+  int n_heads;           /* H */
+  int mlp_hidden;        /* F, SwiGLU hidden width */
+  int downsample_ratio;  /* r, aligner merges r x r patches */
+  int llm_dim;           /* E, aligner output width */
+  int n_layers;          /* L, blocks in the tower */
+  float eps;             /* RMSNorm epsilon (1e-6) */
+  float rope_theta;      /* rotary base (10000) */
+  dsv4v_dtype dtype;
+} dsv4v_config;
+
+/* One block's parameters ([vision-API] DeepseekV4VisionBlock: norm1, attn.wqkv, output
+ * projection, norm2, mlp).  Scales are fp32 [D]; projections are in the config dtype:
+ * wqkv [3D, D], wo [D, D], w_gate [F, D], w_up [F, D], w_down [D, F].  Device pointers, each
+ * 16-byte aligned. */
+typedef struct {
+  const float* norm1_w;
+  const float* norm2_w;
+  const void* wqkv;
+  const void* wo;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+} dsv4v_block_weights;
+
+/* A packed batch of images.  grid_hw: [n_images, 2] int32 (n_h, n_w), each >= 1.  cu_patches:
+ * [n_images + 1] int32 offsets (see above).  Both are needed on the host (launch geometry and
+ * validation) and on the device (read by the kernels); the two copies must hold the same
+ * values.  1 <= n_images <= DSV4V_MAX_IMAGES. */
+typedef struct {
+  int n_images;
+  const int32_t* grid_hw_host;
+  const int32_t* grid_hw_dev;
+  const int32_t* cu_patches_host;
+  const int32_t* cu_patches_dev;
+} dsv4v_batch;
+
+#define DSV4V_MAX_IMAGES 1024
+
+/* Bytes of device scratch that every call below needs for this config and batch (the maximum
+ * over the calls, so one workspace serves all of them).  0 if the arguments are invalid. */
+size_t dsv4v_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch);
+
+/* [vision-API, get_vision_cos_sin]: the 2D rotary table of every image of the batch, stacked
+ * in packing order: row p holds the table row of packed patch p.  Reading adopted: the table
+ * width is head_dim / 2; the first head_dim / 4 angles are h * theta^(-k / (head_dim/4)) and
+ * the last head_dim / 4 are w * theta^(-k / (head_dim/4)), k < head_dim / 4, with (h, w) the
+ * patch's grid position inside its own image.
+ * cos_out, sin_out: device fp32 [P, head_dim / 2], written. */
+dsv4v_status dsv4v_rope2d_table(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                float* cos_out, float* sin_out, void* stream);
+
+/* [vision-API, DeepseekV4VisionBlock.forward]: one pre-norm block on the packed batch,
+ *   x <- x + wo . attn(rope(wqkv . norm1(x)))   (attention within each image only)
+ *   x <- x + w_down . (silu(w_gate . norm2(x)) * (w_up . norm2(x)))
+ * cos, sin: device fp32 [P, head_dim / 2] (dsv4v_rope2d_table).  x_inout: device [P, D] in the
+ * config dtype, updated in place.  workspace: device scratch of ws_bytes bytes. */
+dsv4v_status dsv4v_block_forward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                 const dsv4v_block_weights* weights, const float* cos,
+                                 const float* sin, void* x_inout, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
+/* [vision-API, DeepseekV4VisionTransformer.forward] from patch states on: builds the rotary
+ * table, runs cfg->n_layers blocks (layers: host array of n_layers weight structs), then the
+ * tower's final RMSNorm with final_norm_w (device fp32 [D]; NULL skips it).  x_inout: device
+ * [P, D], updated in place.  The patch embedding is not part of this call. */
+dsv4v_status dsv4v_tower_forward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                 const dsv4v_block_weights* layers, const float* final_norm_w,
+                                 void* x_inout, void* workspace, size_t ws_bytes, void* stream);
+
+/* [vision-API, DeepseekV4VisionAligner.forward]: per image, zero-pad the grid at the
+ * bottom/right to a multiple of r (a stated assumption for odd grids), merge each r x r window
+ * into one token whose channel (a * r + b) * D + c holds channel c of the patch at window
+ * position (a, b) (a = row offset), order tokens row-major, and project with
+ * w_align [E, r*r*D] (bias-free).
+ * x: device [P, D]; out: device [T, E] with T = sum_i ceil(n_h/r) * ceil(n_w/r), both in the
+ * config dtype.  cu_tokens_host: optional host int32 [n_images + 1], filled with the token
+ * offsets of each image (NULL to skip). */
+dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                   const void* x, const void* w_align, void* out,
+                                   int32_t* cu_tokens_host, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* Number of aligner tokens T of the batch (host computation); -1 if the arguments are
+ * invalid. */
+int64_t dsv4v_aligner_tokens(const dsv4v_config* cfg, const dsv4v_batch* batch);
+
+/* ---- Component entry points: single steps of the block, for testing and profiling. ---- */
+
+/* RMSNorm [vision-API, DeepseekV4VisionRMSNorm]: y = w * x / sqrt(mean(x^2) + eps) per row,
+ * computed in fp32, cast to the config dtype.  x, y: device [rows, D]; w: device fp32 [D].
+ * y may equal x. */
+dsv4v_status dsv4v_rmsnorm(const dsv4v_config* cfg, int64_t rows, const void* x,
+                           const float* w, void* y, void* stream);
+
+/* Fused projection + rotation ([vision-API, DeepseekV4VisionAttention.wqkv] and
+ * apply_vision_rotary): qkv = y . wqkv^T, then q and k (columns [0, 2D)) rotated with the
+ * half-split rule x'_j = x_j cos_j - x_{j+hd/2} sin_j, x'_{j+hd/2} = x_{j+hd/2} cos_j +
+ * x_j sin_j.  y: device [P, D]; qkv: device [P, 3D], config dtype. */
+dsv4v_status dsv4v_qkv_rope(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* y,
+                            const void* wqkv, const float* cos, const float* sin, void* qkv,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* Full bidirectional attention within each image ([vision-API, DeepseekV4VisionAttention]):
+ * out[:, h*hd:(h+1)*hd] = softmax(q_h k_h^T / sqrt(hd)) v_h per image and head.
+ * qkv: device [P, 3D] (q | k | v, already rotated); out: device [P, D]. */
+dsv4v_status dsv4v_attention(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                             const void* qkv, void* out, void* stream);
+
+/* Projection with residual add: x <- x + a . w^T.  a: device [rows, K]; w: device [D, K];
+ * x: device [rows, D].  K is vision_dim or mlp_hidden. */
+dsv4v_status dsv4v_linear_residual(const dsv4v_config* cfg, int64_t rows, int k,
+                                   const void* a, const void* w, void* x, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
+/* SwiGLU gate/up ([vision-API, DeepseekV4VisionMLP]): h = silu(y . w_gate^T) * (y . w_up^T),
+ * silu(z) = z / (1 + exp(-z)).  y: device [rows, D]; h: device [rows, F]. */
+dsv4v_status dsv4v_swiglu(const dsv4v_config* cfg, int64_t rows, const void* y,
+                          const void* w_gate, const void* w_up, void* h, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and returns DSV4V_ERR_TIMEOUT if a kernel of this library recorded a
+ * bounded-wait timeout on the current device since the last call (and clears the record),
+ * DSV4V_ERR_CUDA if the stream reports an error, else DSV4V_OK. */
+dsv4v_status dsv4v_device_error(void* stream);
+
+/* Test hook for the bounded-wait machinery: launches one tiny kernel that waits on an
+ * mbarrier nothing ever signals, with a limit of `limit_ns` nanoseconds, and then records a
+ * timeout exactly as the production kernels do.  Nothing faults, traps or hangs. */
+dsv4v_status dsv4v_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
+const char* dsv4v_status_string(dsv4v_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSV4V_H */

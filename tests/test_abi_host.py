@@ -1,0 +1,109 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports every symbol the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from vision_transformer_encoder_dsv4v_b200 import build
+from vision_transformer_encoder_dsv4v_b200 import dsv4v as A
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return A.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "dsv4v.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\**\s+\**(dsv4v_[a-z0-9_]+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 14, names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(names) == sorted(A.EXPORTS)
+
+
+def test_status_strings(lib):
+    assert A.dsv4v_status_string(0) == "ok"
+    assert "workspace" in A.dsv4v_status_string(3)
+    assert A.dsv4v_status_string(99) == "unknown status"
+
+
+class HostBatch:
+    """A dsv4v_batch whose 'device' pointers are host buffers; only host validation reads them."""
+
+    def __init__(self, grids, cu=None):
+        self.grid = (ctypes.c_int32 * (2 * max(1, len(grids))))(*[v for g in grids for v in g])
+        if cu is None:
+            cu = [0]
+            for h, w in grids:
+                cu.append(cu[-1] + h * w)
+        self.cu = (ctypes.c_int32 * len(cu))(*cu)
+        self.c = A.Batch(len(grids), ctypes.addressof(self.grid), ctypes.addressof(self.grid),
+                         ctypes.addressof(self.cu), ctypes.addressof(self.cu))
+
+
+def cfg(**kw):
+    d = dict(vision_dim=1024, n_heads=16, mlp_hidden=2816, downsample_ratio=2, llm_dim=4096, n_layers=32,
+             dtype=A.DSV4V_BF16)
+    d.update(kw)
+    dt = d.pop("dtype")
+    return A.make_config(dtype=dt, **d)
+
+
+def test_workspace_size_and_tokens_host_only(lib):
+    b = HostBatch([(28, 28)])
+    n = lib.dsv4v_workspace_size(ctypes.byref(cfg()), ctypes.byref(b.c))
+    # at least the activations: y, qkv, attn (bf16) and h, plus the rotary table
+    assert n >= 784 * (1024 * 5 * 2 + 2816 * 2 + 32 * 8)
+    assert lib.dsv4v_aligner_tokens(ctypes.byref(cfg()), ctypes.byref(b.c)) == 196
+    b4 = HostBatch([(27, 37), (37, 27), (10, 78), (112, 7)])
+    assert lib.dsv4v_aligner_tokens(ctypes.byref(cfg()), ctypes.byref(b4.c)) == 266 + 266 + 195 + 224
+
+
+@pytest.mark.parametrize("case,status", [
+    ("null_cfg", 1), ("zero_images", 1), ("bad_cu", 1), ("bad_cu0", 1), ("zero_side", 1),
+    ("hd32_bf16", 2), ("dim_not_128", 2), ("hidden_not_128", 2), ("heads_not_dividing", 1), ("hd_odd_pairs", 2),
+    ("f32_hd_too_big", 2), ("too_many_images", 1),
+])
+def test_host_validation_rejects(lib, case, status):
+    c = cfg()
+    b = HostBatch([(4, 6), (3, 5)])
+    if case == "zero_images":
+        b.c.n_images = 0
+    elif case == "bad_cu":
+        b = HostBatch([(4, 6), (3, 5)], cu=[0, 24, 40])
+    elif case == "bad_cu0":
+        b = HostBatch([(4, 6)], cu=[1, 25])
+    elif case == "zero_side":
+        b = HostBatch([(4, 0)])
+    elif case == "hd32_bf16":
+        c = cfg(n_heads=32)
+    elif case == "dim_not_128":
+        c = cfg(vision_dim=1088, n_heads=17)
+    elif case == "hidden_not_128":
+        c = cfg(mlp_hidden=2800)
+    elif case == "heads_not_dividing":
+        c = cfg(n_heads=15)
+    elif case == "hd_odd_pairs":
+        c = cfg(vision_dim=36, n_heads=6, dtype=A.DSV4V_F32)
+    elif case == "f32_hd_too_big":
+        c = cfg(vision_dim=256, n_heads=2, dtype=A.DSV4V_F32)
+    elif case == "too_many_images":
+        b = HostBatch([(1, 1)] * (A.DSV4V_MAX_IMAGES + 1))
+    cp = None if case == "null_cfg" else ctypes.byref(c)
+    x = ctypes.c_void_p(4096)
+    w = A.BlockWeights(*([4096] * 7))
+    st = lib.dsv4v_block_forward(cp, ctypes.byref(b.c), ctypes.byref(w), x, x, x, x, 1 << 30, None)
+    assert st == status
+    assert lib.dsv4v_workspace_size(cp, ctypes.byref(b.c)) == 0
+    st = lib.dsv4v_aligner_forward(cp, ctypes.byref(b.c), x, x, x, None, x, 1 << 30, None)
+    assert st == status

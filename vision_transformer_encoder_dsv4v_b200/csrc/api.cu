@@ -1,0 +1,599 @@
+// C ABI of the vision-tower forward: argument validation, workspace layout, GEMM planning,
+// TMA descriptor construction and the launch sequence of each entry point.
+#include <string.h>
+
+#include <algorithm>
+
+#include <mutex>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/dsv4v.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsv4v {
+
+// Device word in which kernels record the first bounded-wait timeout.
+__device__ uint32_t g_dev_error;
+
+namespace {
+
+// ---------------------------------------------------------------------------- device info
+struct DeviceInfo {
+  int sms = 0;
+  uint32_t* err = nullptr;
+};
+
+bool device_info(DeviceInfo& out) {
+  static std::mutex mu;
+  static std::unordered_map<int, DeviceInfo> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) {
+    out = it->second;
+    return true;
+  }
+  DeviceInfo info;
+  if (cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) return false;
+  info.err = static_cast<uint32_t*>(p);
+  cache[dev] = info;
+  out = info;
+  return true;
+}
+
+// SM count used for planning when no device can be queried (sizing only).
+int planning_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+    return sms;
+  cudaGetLastError();
+  return 148;
+}
+
+// ---------------------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void* ptr;
+  int64_t rows, cols;
+  int box_rows;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = reinterpret_cast<size_t>(k.ptr);
+    h ^= static_cast<size_t>(k.rows) * 0x9E3779B97F4A7C15ull;
+    h ^= static_cast<size_t>(k.cols) * 0xC2B2AE3D27D4EB4Full + (h << 6);
+    h ^= static_cast<size_t>(k.box_rows) * 0x165667B19E3779F9ull + (h >> 2);
+    return h;
+  }
+};
+
+// bf16 row-major [rows, cols] matrix, boxes of 64 columns (128 B, 128-byte swizzle) x box_rows
+// rows; reads past the end return zeros.  Descriptors depend only on these values, so they are
+// cached per thread.
+bool bf16_map(const void* ptr, int64_t rows, int64_t cols, int box_rows, CUtensorMap* out) {
+  thread_local std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  MapKey key{ptr, rows, cols, box_rows};
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *out = it->second;
+    return true;
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMap m;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  if (cache.size() > 4096) cache.clear();
+  cache[key] = m;
+  *out = m;
+  return true;
+}
+
+// ---------------------------------------------------------------------------- validation
+struct Shape {
+  int D, H, hd, F, r, E, L;
+  bool bf16;
+  int64_t P, T;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dsv4v_status check_config(const dsv4v_config* c, Shape& s) {
+  if (!c) return DSV4V_ERR_INVALID_ARG;
+  if (c->vision_dim <= 0 || c->n_heads <= 0 || c->mlp_hidden <= 0 || c->downsample_ratio <= 0 || c->llm_dim <= 0 ||
+      c->n_layers < 0 || !(c->eps >= 0.0f) || !(c->rope_theta > 0.0f))
+    return DSV4V_ERR_INVALID_ARG;
+  if (c->dtype != DSV4V_F32 && c->dtype != DSV4V_BF16) return DSV4V_ERR_INVALID_ARG;
+  if (c->vision_dim % c->n_heads) return DSV4V_ERR_INVALID_ARG;
+  s.D = c->vision_dim;
+  s.H = c->n_heads;
+  s.hd = s.D / s.H;
+  s.F = c->mlp_hidden;
+  s.r = c->downsample_ratio;
+  s.E = c->llm_dim;
+  s.L = c->n_layers;
+  s.bf16 = c->dtype == DSV4V_BF16;
+  if (s.hd % 4) return DSV4V_ERR_UNSUPPORTED;
+  if (s.bf16) {
+    if (s.hd != 64 || s.D % 128 || s.F % 128 || s.E % 128) return DSV4V_ERR_UNSUPPORTED;
+  } else {
+    if (s.hd > 64) return DSV4V_ERR_UNSUPPORTED;
+  }
+  return DSV4V_OK;
+}
+
+dsv4v_status check_batch(const dsv4v_batch* b, Shape& s) {
+  if (!b || b->n_images < 1 || b->n_images > DSV4V_MAX_IMAGES) return DSV4V_ERR_INVALID_ARG;
+  if (!b->grid_hw_host || !b->cu_patches_host || !b->grid_hw_dev || !b->cu_patches_dev) return DSV4V_ERR_INVALID_ARG;
+  if (b->cu_patches_host[0] != 0) return DSV4V_ERR_INVALID_ARG;
+  int64_t p = 0, t = 0;
+  for (int i = 0; i < b->n_images; ++i) {
+    const int64_t n_h = b->grid_hw_host[2 * i], n_w = b->grid_hw_host[2 * i + 1];
+    if (n_h < 1 || n_w < 1) return DSV4V_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(b->cu_patches_host[i + 1]) - b->cu_patches_host[i] != n_h * n_w)
+      return DSV4V_ERR_INVALID_ARG;
+    p += n_h * n_w;
+    t += ((n_h + s.r - 1) / s.r) * ((n_w + s.r - 1) / s.r);
+    if (p > (1ll << 30)) return DSV4V_ERR_UNSUPPORTED;
+  }
+  s.P = p;
+  s.T = t;
+  return DSV4V_OK;
+}
+
+dsv4v_status check_all(const dsv4v_config* c, const dsv4v_batch* b, Shape& s) {
+  dsv4v_status st = check_config(c, s);
+  if (st != DSV4V_OK) return st;
+  return check_batch(b, s);
+}
+
+// ---------------------------------------------------------------------------- workspace
+struct Plans {
+  GemmPlan qkv, out, gateup, down, align;
+};
+
+Plans make_plans(const Shape& s, int sms) {
+  Plans p;
+  p.qkv = plan_gemm(EPI_QKV_ROPE, static_cast<int>(s.P), 3 * s.D, s.D, sms);
+  p.out = plan_gemm(EPI_RESID, static_cast<int>(s.P), s.D, s.D, sms);
+  p.gateup = plan_gemm(EPI_SWIGLU, static_cast<int>(s.P), s.F, s.D, sms);
+  p.down = plan_gemm(EPI_RESID, static_cast<int>(s.P), s.D, s.F, sms);
+  p.align = plan_gemm(EPI_STORE, static_cast<int>(s.T), s.E, s.r * s.r * s.D, sms);
+  return p;
+}
+
+struct Layout {
+  size_t cos, sin, y, qkv, attn, h, partials, counters, asrc, merged, total;
+  size_t counters_bytes;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Layout make_layout(const Shape& s, const Plans& pl) {
+  Layout l{};
+  const size_t es = s.bf16 ? 2 : 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off += up256(bytes);
+    return at;
+  };
+  l.cos = take(static_cast<size_t>(s.P) * (s.hd / 2) * 4);
+  l.sin = take(static_cast<size_t>(s.P) * (s.hd / 2) * 4);
+  l.y = take(static_cast<size_t>(s.P) * s.D * es);
+  l.qkv = take(static_cast<size_t>(s.P) * 3 * s.D * es);
+  l.attn = take(static_cast<size_t>(s.P) * s.D * es);
+  l.h = take(static_cast<size_t>(s.P) * s.F * es);
+  size_t part = 0;
+  int counters = 1;
+  if (s.bf16) {
+    const GemmPlan* all[5] = {&pl.qkv, &pl.out, &pl.gateup, &pl.down, &pl.align};
+    for (const GemmPlan* g : all) {
+      part = std::max(part, g->partial_bytes);
+      counters = std::max(counters, g->counters);
+    }
+  }
+  l.partials = take(part);
+  l.counters_bytes = up256(static_cast<size_t>(counters) * sizeof(int));
+  l.counters = take(l.counters_bytes);
+  l.asrc = take(static_cast<size_t>(s.T) * s.r * s.r * 4);
+  l.merged = take(s.bf16 ? 0 : static_cast<size_t>(s.T) * s.r * s.r * s.D * 4);
+  l.total = off;
+  return l;
+}
+
+struct Ctx {
+  Shape s;
+  float eps, theta;
+  Plans plans;
+  Layout lay;
+  DeviceInfo dev;
+  uint8_t* ws;
+  cudaStream_t stream;
+  template <class T>
+  T* at(size_t off) const {
+    return reinterpret_cast<T*>(ws + off);
+  }
+};
+
+dsv4v_status prepare(const dsv4v_config* c, const dsv4v_batch* b, void* workspace, size_t ws_bytes, void* stream,
+                     Ctx& ctx) {
+  dsv4v_status st = check_all(c, b, ctx.s);
+  if (st != DSV4V_OK) return st;
+  if (!device_info(ctx.dev)) return DSV4V_ERR_CUDA;
+  ctx.plans = make_plans(ctx.s, ctx.dev.sms);
+  ctx.lay = make_layout(ctx.s, ctx.plans);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < ctx.lay.total)
+    return DSV4V_ERR_WORKSPACE;
+  ctx.eps = c->eps;
+  ctx.theta = c->rope_theta;
+  ctx.ws = static_cast<uint8_t*>(workspace);
+  ctx.stream = static_cast<cudaStream_t>(stream);
+  return DSV4V_OK;
+}
+
+dsv4v_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSV4V_OK : DSV4V_ERR_CUDA; }
+
+#define DSV4V_TRY(expr)                           \
+  do {                                            \
+    dsv4v_status st_ = (expr);                    \
+    if (st_ != DSV4V_OK) return st_;              \
+  } while (0)
+
+// ---------------------------------------------------------------------------- bf16 steps
+dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* a, int64_t M, int K, const void* b,
+                       const void* b2, int n_out, void* out, const void* resid, const float* cos = nullptr,
+                       const float* sin = nullptr, bool gather = false, const int32_t* gsrc = nullptr,
+                       const void* gx = nullptr) {
+  if (M == 0) return DSV4V_OK;
+  const int box_b = epi == EPI_SWIGLU ? plan.bn / 2 : plan.bn;
+  CUtensorMap ta, tb, tb2;
+  if ((!gather && !bf16_map(a, M, K, 128, &ta)) || !bf16_map(b, n_out, K, box_b, &tb) ||
+      (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)))
+    return DSV4V_ERR_CUDA;
+  GemmArgs g{};
+  g.tm_a = gather ? nullptr : &ta;
+  g.tm_b = &tb;
+  g.tm_b2 = epi == EPI_SWIGLU ? &tb2 : nullptr;
+  g.M = static_cast<int>(M);
+  g.K = K;
+  g.n_out = n_out;
+  g.out = out;
+  g.ldo = n_out;
+  g.resid = resid;
+  g.cos = cos;
+  g.sin = sin;
+  g.rot_cols = 2 * c.s.D;
+  g.gather_src = gsrc;
+  g.gather_x = gx;
+  g.gather_r2 = c.s.r * c.s.r;
+  g.gather_d = c.s.D;
+  g.partials = c.at<float>(c.lay.partials);
+  g.counters = c.at<int>(c.lay.counters);
+  g.err = c.dev.err;
+  return cuda_status(launch_gemm_tc(epi, gather, plan, g, c.stream));
+}
+
+dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv, void* out) {
+  CUtensorMap tm;
+  if (!bf16_map(qkv, c.s.P, 3 * c.s.D, 128, &tm)) return DSV4V_ERR_CUDA;
+  thread_local AttnSchedule sched;
+  const int n = b->n_images;
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  // Longest image first: its CTAs cost the most (cost grows with the key count).
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
+    return b->cu_patches_host[x + 1] - b->cu_patches_host[x] > b->cu_patches_host[y + 1] - b->cu_patches_host[y];
+  });
+  sched.n_images = n;
+  int items = 0;
+  for (int k = 0; k < n; ++k) {
+    const int i = order[k];
+    const int len = b->cu_patches_host[i + 1] - b->cu_patches_host[i];
+    sched.item_start[k] = items;
+    sched.img_row0[k] = b->cu_patches_host[i];
+    sched.img_len[k] = len;
+    items += ((len + 127) / 128) * c.s.H;
+  }
+  sched.item_start[n] = items;
+  sched.n_items = items;
+  return cuda_status(launch_attention_tc(&tm, sched, c.s.H, c.s.D, out, c.dev.err, c.stream));
+}
+
+dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_weights* w, const float* cos,
+                        const float* sin, void* x) {
+  const Shape& s = c.s;
+  void* y = c.at<void>(c.lay.y);
+  void* qkv = c.at<void>(c.lay.qkv);
+  void* attn = c.at<void>(c.lay.attn);
+  void* h = c.at<void>(c.lay.h);
+  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm1_w, y, s.P, s.D, c.eps, c.stream)));
+  DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, y, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr, cos, sin));
+  DSV4V_TRY(attention_bf16(c, b, qkv, attn));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x));
+  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm2_w, y, s.P, s.D, c.eps, c.stream)));
+  DSV4V_TRY(gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, y, s.P, s.D, w->w_gate, w->w_up, s.F, h, nullptr));
+  return gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x);
+}
+
+// ---------------------------------------------------------------------------- fp32 steps
+dsv4v_status block_f32(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_weights* w, const float* cos,
+                       const float* sin, void* xv) {
+  const Shape& s = c.s;
+  float* x = static_cast<float*>(xv);
+  float* y = c.at<float>(c.lay.y);
+  float* qkv = c.at<float>(c.lay.qkv);
+  float* attn = c.at<float>(c.lay.attn);
+  float* h = c.at<float>(c.lay.h);
+  const int M = static_cast<int>(s.P);
+  DSV4V_TRY(cuda_status(launch_rmsnorm(false, x, w->norm1_w, y, s.P, s.D, c.eps, c.stream)));
+  DSV4V_TRY(cuda_status(launch_gemm_f32(EPI_STORE, y, static_cast<const float*>(w->wqkv), nullptr, qkv, nullptr, M,
+                                        3 * s.D, s.D, c.stream)));
+  DSV4V_TRY(cuda_status(launch_rope_apply_f32(qkv, cos, sin, s.P, s.D, s.H, c.stream)));
+  DSV4V_TRY(cuda_status(launch_attention_f32(qkv, attn, b->cu_patches_dev, b->n_images, s.P, s.D, s.H, c.stream)));
+  DSV4V_TRY(cuda_status(launch_gemm_f32(EPI_RESID, attn, static_cast<const float*>(w->wo), nullptr, x, x, M, s.D, s.D,
+                                        c.stream)));
+  DSV4V_TRY(cuda_status(launch_rmsnorm(false, x, w->norm2_w, y, s.P, s.D, c.eps, c.stream)));
+  DSV4V_TRY(cuda_status(launch_gemm_f32(EPI_SWIGLU, y, static_cast<const float*>(w->w_gate),
+                                        static_cast<const float*>(w->w_up), h, nullptr, M, s.F, s.D, c.stream)));
+  return cuda_status(launch_gemm_f32(EPI_RESID, h, static_cast<const float*>(w->w_down), nullptr, x, x, M, s.D, s.F,
+                                     c.stream));
+}
+
+bool weights_ok(const dsv4v_block_weights* w) {
+  return w && w->norm1_w && w->norm2_w && w->wqkv && w->wo && w->w_gate && w->w_up && w->w_down &&
+         aligned16(w->norm1_w) && aligned16(w->norm2_w) && aligned16(w->wqkv) && aligned16(w->wo) &&
+         aligned16(w->w_gate) && aligned16(w->w_up) && aligned16(w->w_down);
+}
+
+dsv4v_status reset_counters(const Ctx& c) {
+  if (!c.s.bf16) return DSV4V_OK;
+  return cuda_status(cudaMemsetAsync(c.ws + c.lay.counters, 0, c.lay.counters_bytes, c.stream));
+}
+
+dsv4v_status rope_table(const Ctx& c, const dsv4v_batch* b, float* cos, float* sin) {
+  return cuda_status(launch_rope_table(b->cu_patches_dev, b->grid_hw_dev, b->n_images, c.s.P, c.s.hd / 2, c.theta,
+                                       cos, sin, c.stream));
+}
+
+// Validation-only context for component calls that take a row count instead of a batch.
+dsv4v_status prepare_rows(const dsv4v_config* cfg, int64_t rows, void* workspace, size_t ws_bytes, void* stream,
+                          bool need_ws, Ctx& ctx) {
+  DSV4V_TRY(check_config(cfg, ctx.s));
+  if (rows < 0 || rows > (1ll << 30)) return DSV4V_ERR_INVALID_ARG;
+  ctx.s.P = rows;
+  ctx.s.T = 0;
+  if (!device_info(ctx.dev)) return DSV4V_ERR_CUDA;
+  ctx.plans = make_plans(ctx.s, ctx.dev.sms);
+  ctx.lay = make_layout(ctx.s, ctx.plans);
+  ctx.eps = cfg->eps;
+  ctx.theta = cfg->rope_theta;
+  ctx.stream = static_cast<cudaStream_t>(stream);
+  ctx.ws = static_cast<uint8_t*>(workspace);
+  if (need_ws && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < ctx.lay.total))
+    return DSV4V_ERR_WORKSPACE;
+  return DSV4V_OK;
+}
+
+}  // namespace
+}  // namespace dsv4v
+
+using namespace dsv4v;
+
+extern "C" {
+
+const char* dsv4v_status_string(dsv4v_status s) {
+  switch (s) {
+    case DSV4V_OK: return "ok";
+    case DSV4V_ERR_INVALID_ARG: return "invalid argument";
+    case DSV4V_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSV4V_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DSV4V_ERR_CUDA: return "CUDA error";
+    case DSV4V_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t dsv4v_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch) {
+  Shape s;
+  if (check_all(cfg, batch, s) != DSV4V_OK) return 0;
+  return make_layout(s, make_plans(s, planning_sms())).total;
+}
+
+int64_t dsv4v_aligner_tokens(const dsv4v_config* cfg, const dsv4v_batch* batch) {
+  Shape s;
+  if (check_all(cfg, batch, s) != DSV4V_OK) return -1;
+  return s.T;
+}
+
+dsv4v_status dsv4v_rope2d_table(const dsv4v_config* cfg, const dsv4v_batch* batch, float* cos_out, float* sin_out,
+                                void* stream) {
+  Shape s;
+  DSV4V_TRY(check_all(cfg, batch, s));
+  if (!cos_out || !sin_out) return DSV4V_ERR_INVALID_ARG;
+  return cuda_status(launch_rope_table(batch->cu_patches_dev, batch->grid_hw_dev, batch->n_images, s.P, s.hd / 2,
+                                       cfg->rope_theta, cos_out, sin_out, static_cast<cudaStream_t>(stream)));
+}
+
+dsv4v_status dsv4v_block_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const dsv4v_block_weights* w,
+                                 const float* cos, const float* sin, void* x_inout, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  Ctx c;
+  DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
+  if (!weights_ok(w) || !cos || !sin || !x_inout || !aligned16(x_inout) || !aligned16(cos) || !aligned16(sin))
+    return DSV4V_ERR_INVALID_ARG;
+  DSV4V_TRY(reset_counters(c));
+  return c.s.bf16 ? block_bf16(c, batch, w, cos, sin, x_inout) : block_f32(c, batch, w, cos, sin, x_inout);
+}
+
+dsv4v_status dsv4v_tower_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const dsv4v_block_weights* layers,
+                                 const float* final_norm_w, void* x_inout, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  Ctx c;
+  DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
+  if (!x_inout || !aligned16(x_inout) || (c.s.L > 0 && !layers)) return DSV4V_ERR_INVALID_ARG;
+  for (int l = 0; l < c.s.L; ++l)
+    if (!weights_ok(&layers[l])) return DSV4V_ERR_INVALID_ARG;
+  if (final_norm_w && !aligned16(final_norm_w)) return DSV4V_ERR_INVALID_ARG;
+  float* cos = c.at<float>(c.lay.cos);
+  float* sin = c.at<float>(c.lay.sin);
+  DSV4V_TRY(reset_counters(c));
+  DSV4V_TRY(rope_table(c, batch, cos, sin));
+  for (int l = 0; l < c.s.L; ++l)
+    DSV4V_TRY(c.s.bf16 ? block_bf16(c, batch, &layers[l], cos, sin, x_inout)
+                       : block_f32(c, batch, &layers[l], cos, sin, x_inout));
+  if (final_norm_w)
+    DSV4V_TRY(cuda_status(launch_rmsnorm(c.s.bf16, x_inout, final_norm_w, x_inout, c.s.P, c.s.D, c.eps, c.stream)));
+  return DSV4V_OK;
+}
+
+dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x,
+                                   const void* w_align, void* out, int32_t* cu_tokens_host, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  Ctx c;
+  DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
+  if (!x || !w_align || !out || !aligned16(x) || !aligned16(w_align) || !aligned16(out)) return DSV4V_ERR_INVALID_ARG;
+  if (cu_tokens_host) {
+    int64_t t = 0;
+    cu_tokens_host[0] = 0;
+    for (int i = 0; i < batch->n_images; ++i) {
+      const int n_h = batch->grid_hw_host[2 * i], n_w = batch->grid_hw_host[2 * i + 1];
+      t += static_cast<int64_t>((n_h + c.s.r - 1) / c.s.r) * ((n_w + c.s.r - 1) / c.s.r);
+      cu_tokens_host[i + 1] = static_cast<int32_t>(t);
+    }
+  }
+  const Shape& s = c.s;
+  int32_t* src = c.at<int32_t>(c.lay.asrc);
+  DSV4V_TRY(reset_counters(c));
+  DSV4V_TRY(cuda_status(
+      launch_aligner_index(batch->cu_patches_dev, batch->grid_hw_dev, batch->n_images, s.r, s.T, src, c.stream)));
+  const int K = s.r * s.r * s.D;
+  if (s.bf16)
+    return gemm_bf16(c, EPI_STORE, c.plans.align, nullptr, s.T, K, w_align, nullptr, s.E, out, nullptr, nullptr,
+                     nullptr, true, src, x);
+  float* merged = c.at<float>(c.lay.merged);
+  DSV4V_TRY(cuda_status(launch_gather_f32(static_cast<const float*>(x), src, merged, s.T, s.r * s.r, s.D, c.stream)));
+  return cuda_status(launch_gemm_f32(EPI_STORE, merged, static_cast<const float*>(w_align), nullptr,
+                                     static_cast<float*>(out), nullptr, static_cast<int>(s.T), s.E, K, c.stream));
+}
+
+dsv4v_status dsv4v_rmsnorm(const dsv4v_config* cfg, int64_t rows, const void* x, const float* w, void* y,
+                           void* stream) {
+  Shape s;
+  DSV4V_TRY(check_config(cfg, s));
+  if (rows < 0 || !x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return DSV4V_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_rmsnorm(s.bf16, x, w, y, rows, s.D, cfg->eps, static_cast<cudaStream_t>(stream)));
+}
+
+dsv4v_status dsv4v_qkv_rope(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* y, const void* wqkv,
+                            const float* cos, const float* sin, void* qkv, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  Ctx c;
+  DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
+  if (!y || !wqkv || !cos || !sin || !qkv || !aligned16(y) || !aligned16(wqkv) || !aligned16(cos) ||
+      !aligned16(sin) || !aligned16(qkv))
+    return DSV4V_ERR_INVALID_ARG;
+  const Shape& s = c.s;
+  if (!s.bf16) {
+    DSV4V_TRY(cuda_status(launch_gemm_f32(EPI_STORE, static_cast<const float*>(y), static_cast<const float*>(wqkv),
+                                          nullptr, static_cast<float*>(qkv), nullptr, static_cast<int>(s.P), 3 * s.D,
+                                          s.D, c.stream)));
+    return cuda_status(launch_rope_apply_f32(static_cast<float*>(qkv), cos, sin, s.P, s.D, s.H, c.stream));
+  }
+  DSV4V_TRY(reset_counters(c));
+  return gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, y, s.P, s.D, wqkv, nullptr, 3 * s.D, qkv, nullptr, cos, sin);
+}
+
+dsv4v_status dsv4v_attention(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* qkv, void* out,
+                             void* stream) {
+  Ctx c;
+  DSV4V_TRY(check_all(cfg, batch, c.s));
+  if (!qkv || !out || !aligned16(qkv) || !aligned16(out)) return DSV4V_ERR_INVALID_ARG;
+  if (!device_info(c.dev)) return DSV4V_ERR_CUDA;
+  c.stream = static_cast<cudaStream_t>(stream);
+  if (!c.s.bf16)
+    return cuda_status(launch_attention_f32(static_cast<const float*>(qkv), static_cast<float*>(out),
+                                            batch->cu_patches_dev, batch->n_images, c.s.P, c.s.D, c.s.H, c.stream));
+  return attention_bf16(c, batch, qkv, out);
+}
+
+dsv4v_status dsv4v_linear_residual(const dsv4v_config* cfg, int64_t rows, int k, const void* a, const void* w,
+                                   void* x, void* workspace, size_t ws_bytes, void* stream) {
+  Ctx c;
+  DSV4V_TRY(prepare_rows(cfg, rows, workspace, ws_bytes, stream, cfg && cfg->dtype == DSV4V_BF16, c));
+  if (!a || !w || !x || !aligned16(a) || !aligned16(w) || !aligned16(x)) return DSV4V_ERR_INVALID_ARG;
+  const Shape& s = c.s;
+  if (k != s.D && k != s.F) return DSV4V_ERR_INVALID_ARG;
+  if (!s.bf16)
+    return cuda_status(launch_gemm_f32(EPI_RESID, static_cast<const float*>(a), static_cast<const float*>(w), nullptr,
+                                       static_cast<float*>(x), static_cast<const float*>(x), static_cast<int>(rows),
+                                       s.D, k, c.stream));
+  DSV4V_TRY(reset_counters(c));
+  const GemmPlan& plan = k == s.D ? c.plans.out : c.plans.down;
+  return gemm_bf16(c, EPI_RESID, plan, a, rows, k, w, nullptr, s.D, x, x);
+}
+
+dsv4v_status dsv4v_swiglu(const dsv4v_config* cfg, int64_t rows, const void* y, const void* w_gate, const void* w_up,
+                          void* h, void* workspace, size_t ws_bytes, void* stream) {
+  Ctx c;
+  DSV4V_TRY(prepare_rows(cfg, rows, workspace, ws_bytes, stream, cfg && cfg->dtype == DSV4V_BF16, c));
+  if (!y || !w_gate || !w_up || !h || !aligned16(y) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h))
+    return DSV4V_ERR_INVALID_ARG;
+  const Shape& s = c.s;
+  if (!s.bf16)
+    return cuda_status(launch_gemm_f32(EPI_SWIGLU, static_cast<const float*>(y), static_cast<const float*>(w_gate),
+                                       static_cast<const float*>(w_up), static_cast<float*>(h), nullptr,
+                                       static_cast<int>(rows), s.F, s.D, c.stream));
+  DSV4V_TRY(reset_counters(c));
+  return gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, y, rows, s.D, w_gate, w_up, s.F, h, nullptr);
+}
+
+dsv4v_status dsv4v_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSV4V_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof(v)) != cudaSuccess) return DSV4V_ERR_CUDA;
+  if (v == 0) return DSV4V_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return DSV4V_ERR_CUDA;
+  return DSV4V_ERR_TIMEOUT;
+}
+
+dsv4v_status dsv4v_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  DeviceInfo d;
+  if (!device_info(d)) return DSV4V_ERR_CUDA;
+  if (limit_ns > 10000000000ull) return DSV4V_ERR_INVALID_ARG;
+  return cuda_status(launch_selftest_wait(limit_ns, d.err, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,552 @@
+// tcgen05 GEMM for the dense contractions of the vision block and the aligner:
+//   wqkv (+ 2D rotary epilogue), output projection (+ residual), SwiGLU gate/up (+ silu*mul),
+//   down projection (+ residual), aligner projection (A rows gathered from r x r windows).
+//
+// Structure (one persistent CTA per SM, 128 x BN output tiles, K in 64-element blocks):
+//   warp 0      TMA producer: A and B tiles (128-byte swizzle) into a STAGES-deep smem ring
+//   warp 1      TMEM owner + single-thread tcgen05.mma issuer (M=128, N=BN, K=16 per instr.)
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane = one output row
+//               per thread), fused epilogue math, bf16 stores
+//   warps 6..9  (aligner only) A-gather: cp.async rows of the patch matrix into the swizzled
+//               A tile, zero-filling padded window slots
+// The accumulator is double-buffered in TMEM so the epilogue of one tile overlaps the MMAs of
+// the next.  Split-K tiles are combined by the last-arriving contributor (ticket counter):
+// nobody waits on another CTA.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsv4v {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kSmemBudget = 225 * 1024;
+
+template <int BN>
+struct TileCfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES_FIT = (kSmemBudget - 2048) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : ((2 * BN <= 256) ? 256 : 512);
+  static constexpr int SMEM = 1024 + STAGES * STAGE + 512;
+};
+
+struct Params {
+  int M, K, n_out;
+  int tiles_m, splits, kb_total, work;
+  __nv_bfloat16* out;
+  int ldo;
+  const __nv_bfloat16* resid;
+  const float* cos;
+  const float* sin;
+  int rot_cols;
+  const int32_t* gsrc;
+  const __nv_bfloat16* gx;
+  int gr2, gd;
+  float* partials;
+  int* counters;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ void work_coords(const Params& p, int w, int& tile, int& m_tile, int& n_tile, int& kb0,
+                                            int& kb1) {
+  tile = w / p.splits;
+  const int split = w - tile * p.splits;
+  m_tile = tile % p.tiles_m;
+  n_tile = tile / p.tiles_m;
+  const int base = p.kb_total / p.splits, rem = p.kb_total % p.splits;
+  kb0 = split * base + min(split, rem);
+  kb1 = kb0 + base + (split < rem ? 1 : 0);
+}
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+
+// Epilogue of one 64-column accumulator group held in v[0..63] for output row `row`.
+//   STORE/RESID/QKV: v = accumulator columns [64g, 64g + 64) -> output columns n0 + 64g + j.
+//   SWIGLU: v[0..31] = gate columns, v[32..63] = up columns of output columns n0h + 32g + j.
+template <int EPI, int BN>
+__device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_tile, int g, float (&v)[64]) {
+  if (row >= p.M) return;
+  if constexpr (EPI == EPI_SWIGLU) {
+    const int col = n_tile * (BN / 2) + g * 32;
+    uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ldo + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 o;
+      o.x = pack_bf16x2(silu(v[8 * q + 0]) * v[32 + 8 * q + 0], silu(v[8 * q + 1]) * v[32 + 8 * q + 1]);
+      o.y = pack_bf16x2(silu(v[8 * q + 2]) * v[32 + 8 * q + 2], silu(v[8 * q + 3]) * v[32 + 8 * q + 3]);
+      o.z = pack_bf16x2(silu(v[8 * q + 4]) * v[32 + 8 * q + 4], silu(v[8 * q + 5]) * v[32 + 8 * q + 5]);
+      o.w = pack_bf16x2(silu(v[8 * q + 6]) * v[32 + 8 * q + 6], silu(v[8 * q + 7]) * v[32 + 8 * q + 7]);
+      dst[q] = o;
+    }
+  } else {
+    const int col = n_tile * BN + g * 64;
+    if constexpr (EPI == EPI_QKV_ROPE) {
+      if (col < p.rot_cols) {
+        const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(row) * 32);
+        const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(row) * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 c = c4[q], s = s4[q];
+          const float cc[4] = {c.x, c.y, c.z, c.w};
+          const float ss[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * q + e;
+            const float x1 = v[j], x2 = v[32 + j];
+            v[j] = x1 * cc[e] - x2 * ss[e];
+            v[32 + j] = x2 * cc[e] + x1 * ss[e];
+          }
+        }
+      }
+    }
+    if constexpr (EPI == EPI_RESID) {
+      const uint4* r4 = reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.ldo + col);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 r = r4[q];
+        v[8 * q + 0] += bf16_lo(r.x);
+        v[8 * q + 1] += bf16_hi(r.x);
+        v[8 * q + 2] += bf16_lo(r.y);
+        v[8 * q + 3] += bf16_hi(r.y);
+        v[8 * q + 4] += bf16_lo(r.z);
+        v[8 * q + 5] += bf16_hi(r.z);
+        v[8 * q + 6] += bf16_lo(r.w);
+        v[8 * q + 7] += bf16_hi(r.w);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ldo + col);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint4 o;
+      o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+      o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+      o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+      o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+      dst[q] = o;
+    }
+  }
+}
+
+// Accumulator chunks (32 columns each) that make up epilogue group g.
+template <int EPI, int BN>
+__device__ __forceinline__ void group_chunks(int g, int& c0, int& c1) {
+  if constexpr (EPI == EPI_SWIGLU) {
+    c0 = g;
+    c1 = BN / 64 + g;
+  } else {
+    c0 = 2 * g;
+    c1 = 2 * g + 1;
+  }
+}
+
+__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
+template <int BN, int EPI, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+              const __grid_constant__ CUtensorMap tm_b2, const Params p) {
+  using C = TileCfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* ticket = reinterpret_cast<volatile int*>(tmem_holder + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], GATHER ? 1 + 128 : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    if (!GATHER) tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+    if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tm_b2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_phase = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
+        int tile, m_tile, n_tile, kb0, kb1;
+        work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE;
+          uint8_t* sb = sa + C::A_BYTES;
+          if (GATHER) {
+            mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE);
+            tma_load_2d(sa, &tm_a, &full[stage], kb * BK, m_tile * BM);
+          }
+          if (EPI == EPI_SWIGLU) {
+            tma_load_2d(sb, &tm_b, &full[stage], kb * BK, n_tile * (BN / 2));
+            tma_load_2d(sb + (BN / 2) * 128, &tm_b2, &full[stage], kb * BK, n_tile * (BN / 2));
+          } else {
+            tma_load_2d(sb, &tm_b, &full[stage], kb * BK, n_tile * BN);
+          }
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Copies still in flight must land before the CTA may exit (error path only; in the
+      // normal path every issued stage was consumed already and these return at once).
+      volatile int never = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, &never, p.err, kErrTimeoutProducer);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, false);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
+        int tile, m_tile, n_tile, kb0, kb1;
+        work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma)) break;
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(smem + stage * C::STAGE);
+          const uint32_t b_addr = a_addr + C::A_BYTES;
+          const uint64_t adesc = sdesc_sw128(a_addr, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(b_addr, 16, 1024);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4).
+            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // Every MMA issued so far completes before TMEM may be released.
+      umma_commit(mma_done);
+      volatile int never = 0;
+      mbar_wait(mma_done, 0, &never, p.err, kErrTimeoutMma);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ epilogue
+    const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) belong to this warp
+    const int row_in_tile = quad * 32 + lane;
+    const int et = threadIdx.x - 64;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int w = blockIdx.x; w < p.work; w += gridDim.x) {
+      int tile, m_tile, n_tile, kb0, kb1;
+      work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
+      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
+      // All four epilogue warps continue or stop together (TMEM loads are warp-collective and
+      // the split-K path uses a named barrier).
+      if (!named_barrier_and(2, 128, got)) break;
+      tc_fence_after_sync();
+      const int row = m_tile * BM + row_in_tile;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      if (p.splits == 1) {
+#pragma unroll 1
+        for (int g = 0; g < BN / 64; ++g) {
+          int c0, c1;
+          group_chunks<EPI, BN>(g, c0, c1);
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_row + c0 * 32, r0);
+          tmem_ld32(t_row + c1 * 32, r1);
+          tmem_ld_wait(r0);
+          tmem_ld_wait(r1);
+          float v[64];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            v[j] = __uint_as_float(r0[j]);
+            v[32 + j] = __uint_as_float(r1[j]);
+          }
+          epilogue_group<EPI, BN>(p, row, n_tile, g, v);
+        }
+        tc_fence_before_sync();
+        mbar_arrive(&tempty[acc]);
+      } else {
+        // Write this contribution, then the last contributor of the tile sums all of them in
+        // split order (deterministic) and runs the epilogue.
+        float* slot = p.partials + (static_cast<size_t>(w) * BM + row_in_tile) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_row + c * 32, r);
+          tmem_ld_wait(r);
+          float4* dst = reinterpret_cast<float4*>(slot + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                                 __uint_as_float(r[4 * q + 3]));
+        }
+        tc_fence_before_sync();
+        mbar_arrive(&tempty[acc]);
+        __threadfence();
+        named_barrier_sync(1, 128);
+        if (et == 0) *ticket = atomicAdd(&p.counters[tile], 1);
+        named_barrier_sync(1, 128);
+        if (*ticket == p.splits - 1) {
+          __threadfence();
+#pragma unroll 1
+          for (int g = 0; g < BN / 64; ++g) {
+            int c0, c1;
+            group_chunks<EPI, BN>(g, c0, c1);
+            float v[64];
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] = 0.0f;
+#pragma unroll 1
+            for (int s = 0; s < p.splits; ++s) {
+              const float* src = p.partials + (static_cast<size_t>(tile * p.splits + s) * BM + row_in_tile) * BN;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 a = ld_cg_f4(src + c0 * 32 + 4 * q);
+                const float4 b = ld_cg_f4(src + c1 * 32 + 4 * q);
+                v[4 * q + 0] += a.x;
+                v[4 * q + 1] += a.y;
+                v[4 * q + 2] += a.z;
+                v[4 * q + 3] += a.w;
+                v[32 + 4 * q + 0] += b.x;
+                v[32 + 4 * q + 1] += b.y;
+                v[32 + 4 * q + 2] += b.z;
+                v[32 + 4 * q + 3] += b.w;
+              }
+            }
+            epilogue_group<EPI, BN>(p, row, n_tile, g, v);
+          }
+          if (et == 0) p.counters[tile] = 0;  // ready for the next launch
+        }
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  } else if constexpr (GATHER) {
+    // ------------------------------------------------------------------ A-gather (aligner)
+    const int r = threadIdx.x - 192;  // row of the A tile handled by this thread
+    const int blocks_per_slot = p.gd / BK;
+    int stage = 0, pending = -1;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
+      int tile, m_tile, n_tile, kb0, kb1;
+      work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
+      const int row = m_tile * BM + r;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutGather)) {
+          ok = false;
+          break;
+        }
+        const int slot = kb / blocks_per_slot;
+        const int c0 = (kb - slot * blocks_per_slot) * BK;
+        const int src = row < p.M ? p.gsrc[static_cast<size_t>(row) * p.gr2 + slot] : -1;
+        const uint32_t dst_row = smem_u32(smem + stage * C::STAGE) + r * 128;
+        const __nv_bfloat16* src_row = p.gx + (src >= 0 ? static_cast<size_t>(src) * p.gd + c0 : 0);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          cp_async_16(dst_row + ((c ^ (r & 7)) << 4), src_row + 8 * c, src >= 0 ? 16u : 0u);
+        cp_async_commit();
+        if (pending >= 0) {
+          cp_async_wait_1();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[pending]);
+        }
+        pending = stage;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    cp_async_wait_all();
+    if (pending >= 0) {
+      fence_proxy_async_smem();
+      mbar_arrive(&full[pending]);
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+template <int BN, int EPI, bool GATHER>
+cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
+  using C = TileCfg<BN>;
+  static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
+  auto kern = k_gemm_tc<BN, EPI, GATHER>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(attr_set_mask & (1ull << dev))) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set_mask |= 1ull << dev;
+  }
+  Params p;
+  p.M = a.M;
+  p.K = a.K;
+  p.n_out = a.n_out;
+  p.tiles_m = plan.tiles_m;
+  p.splits = plan.splits;
+  p.kb_total = plan.kb_total;
+  p.work = plan.work;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.ldo = a.ldo;
+  p.resid = static_cast<const __nv_bfloat16*>(a.resid);
+  p.cos = a.cos;
+  p.sin = a.sin;
+  p.rot_cols = a.rot_cols;
+  p.gsrc = a.gather_src;
+  p.gx = static_cast<const __nv_bfloat16*>(a.gather_x);
+  p.gr2 = a.gather_r2;
+  p.gd = a.gather_d;
+  p.partials = a.partials;
+  p.counters = a.counters;
+  p.err = a.err;
+  const CUtensorMap& ta = GATHER ? *a.tm_b : *a.tm_a;
+  const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
+  kern<<<plan.grid, GATHER ? 320 : 192, C::SMEM, s>>>(ta, *a.tm_b, tb2, p);
+  return cudaGetLastError();
+}
+
+template <int EPI, bool GATHER>
+cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
+  switch (plan.bn) {
+    case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
+    case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
+    case 192: return launch_one<192, EPI, GATHER>(plan, a, s);
+    case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Cycles of one 64-deep K block on one SM for an N-wide tile: the tensor pipe needs N/2 cycles
+// per K=16 step at M=128; shared memory must also deliver the A (4 KB) and B (N*32 B) slices
+// of the step at 128 B/cycle.
+double kblock_cycles(int bn) { return 4.0 * std::max(bn / 2.0, 32.0 + bn / 4.0); }
+
+}  // namespace
+
+GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms) {
+  GemmPlan best{};
+  double best_cost = 1e300;
+  const int kb_total = K / BK;
+  const int tiles_m = (M + BM - 1) / BM;
+  const int cands[4] = {256, 192, 128, 64};
+  for (int bn : cands) {
+    int n_cols_per_tile = (epi == EPI_SWIGLU) ? bn / 2 : bn;
+    if (n_out % n_cols_per_tile) continue;
+    const int tiles_n = n_out / n_cols_per_tile;
+    const int tiles = tiles_m * tiles_n;
+    for (int splits = 1; splits <= std::min(8, kb_total); ++splits) {
+      if (splits > 1 && tiles * splits > 2 * num_sms) break;
+      const int work = tiles * splits;
+      const int waves = (work + num_sms - 1) / num_sms;
+      const int kb_per = (kb_total + splits - 1) / splits;
+      double cost = waves * (kb_per * kblock_cycles(bn)) + 1500.0;
+      if (splits > 1) cost += 128.0 * bn * 4.0 * (splits + 1) / 64.0 + 800.0;  // partials through L2
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
+        best.bn = bn;
+        best.splits = splits;
+        best.tiles_m = tiles_m;
+        best.tiles_n = tiles_n;
+        best.kb_total = kb_total;
+        best.work = work;
+        best.grid = std::min(work, num_sms);
+        best.partial_bytes = splits > 1 ? static_cast<size_t>(work) * BM * bn * sizeof(float) : 0;
+        best.counters = splits > 1 ? tiles : 0;
+      }
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_gemm_tc(int epi, bool gather, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
+  if (gather) {
+    if (epi != EPI_STORE) return cudaErrorInvalidValue;
+    return launch_bn<EPI_STORE, true>(plan, a, s);
+  }
+  switch (epi) {
+    case EPI_STORE: return launch_bn<EPI_STORE, false>(plan, a, s);
+    case EPI_RESID: return launch_bn<EPI_RESID, false>(plan, a, s);
+    case EPI_QKV_ROPE: return launch_bn<EPI_QKV_ROPE, false>(plan, a, s);
+    case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(plan, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dsv4v

@@ -1,0 +1,88 @@
+// Host-side interface between the C ABI (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dsv4v {
+
+// ---------------------------------------------------------------------------- tcgen05 GEMM
+// C[M, n_out] = A[M, K] . B[n, K]^T with a fused epilogue; bf16 operands, fp32 accumulation.
+enum Epi : int {
+  EPI_STORE = 0,     // out = acc
+  EPI_RESID = 1,     // out = resid + acc          (out may alias resid)
+  EPI_QKV_ROPE = 2,  // out = acc, columns < rot_cols rotated pairwise (j, j + 32) per 64-wide head
+  EPI_SWIGLU = 3,    // out = silu(acc_gate) * acc_up; B = gate rows, B2 = up rows
+};
+
+struct GemmPlan {
+  int bn;        // MMA N per tile (SWIGLU: gate + up halves)
+  int splits;    // K splits per tile (fix-up by the last finisher)
+  int tiles_m, tiles_n, kb_total, work, grid;
+  size_t partial_bytes;  // fp32 scratch for split tiles
+  int counters;          // tile counters needed (split tiles only)
+};
+
+// Chooses tile width and split count for a GEMM of this shape on `num_sms` SMs.
+GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms);
+
+struct GemmArgs {
+  const CUtensorMap* tm_a;    // A [M, K], box 64 x 128 (ignored when gathering A)
+  const CUtensorMap* tm_b;    // B [n, K] (SWIGLU: w_gate), box 64 x bn (SWIGLU: bn / 2)
+  const CUtensorMap* tm_b2;   // SWIGLU: w_up, box 64 x bn / 2
+  int M, K, n_out;
+  void* out;
+  int ldo;
+  const void* resid;
+  const float* cos;
+  const float* sin;
+  int rot_cols;
+  // Aligner A-gather: row m of A, K-block slot s = x[src[m * r2 + s], :] (src < 0: zeros).
+  const int32_t* gather_src;
+  const void* gather_x;
+  int gather_r2;
+  int gather_d;
+  float* partials;
+  int* counters;
+  uint32_t* err;
+};
+
+cudaError_t launch_gemm_tc(int epi, bool gather, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------------------- attention
+constexpr int kMaxImages = 1024;
+
+// Images in the order they are scheduled (longest first); item_start is the prefix sum of
+// (query tiles x heads) in that order.
+struct AttnSchedule {
+  int n_images;
+  int n_items;
+  int item_start[kMaxImages + 1];
+  int img_row0[kMaxImages];
+  int img_len[kMaxImages];
+};
+
+cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& sched, int n_heads, int vision_dim,
+                                void* out, uint32_t* err, cudaStream_t s);
+
+// ---------------------------------------------------------------------------- small kernels
+cudaError_t launch_rope_table(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int64_t P, int half,
+                              float theta, float* cos_out, float* sin_out, cudaStream_t s);
+cudaError_t launch_rmsnorm(bool bf16, const void* x, const float* w, void* y, int64_t rows, int d, float eps,
+                           cudaStream_t s);
+cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int r,
+                                 int64_t n_tokens, int32_t* src_out, cudaStream_t s);
+cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
+
+// ---------------------------------------------------------------------------- fp32 CUDA-core path
+cudaError_t launch_gemm_f32(int epi, const float* a, const float* b, const float* b2, float* out, const float* resid,
+                            int M, int n_out, int K, cudaStream_t s);
+cudaError_t launch_rope_apply_f32(float* qkv, const float* cos, const float* sin, int64_t P, int d, int n_heads,
+                                  cudaStream_t s);
+cudaError_t launch_attention_f32(const float* qkv, float* out, const int32_t* cu_dev, int n_images, int64_t P,
+                                 int d, int n_heads, cudaStream_t s);
+cudaError_t launch_gather_f32(const float* x, const int32_t* src, float* merged, int64_t n_tokens, int r2, int d,
+                              cudaStream_t s);
+
+}  // namespace dsv4v

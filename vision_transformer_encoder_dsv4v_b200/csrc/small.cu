@@ -1,0 +1,191 @@
+// Memory-bound kernels of the path: the 2D rotary table, RMSNorm fused with the cast to the
+// activation dtype, the aligner's window index table, and the bounded-wait self test.
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsv4v {
+
+namespace {
+
+// Index of the image that packed row p belongs to: largest i with cu[i] <= p.
+__device__ __forceinline__ int image_of(const int32_t* cu, int n_images, int64_t p) {
+  int lo = 0, hi = n_images - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= p) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// cos/sin [P, half]: column k < half/2 turns by the patch row h, column k >= half/2 by the
+// patch column w, at inverse frequency theta^(-(k mod half/2) / (half/2)).
+__global__ void k_rope_table(const int32_t* __restrict__ cu, const int32_t* __restrict__ grid, int n_images,
+                             int64_t P, int half, float log2_theta, float* __restrict__ cos_out,
+                             float* __restrict__ sin_out) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= P * half) return;
+  const int64_t p = idx / half;
+  const int k = static_cast<int>(idx - p * half);
+  const int img = image_of(cu, n_images, p);
+  const int local = static_cast<int>(p - cu[img]);
+  const int n_w = grid[2 * img + 1];
+  const int h = local / n_w, w = local - h * n_w;
+  const int quarter = half >> 1;
+  const int kk = k < quarter ? k : k - quarter;
+  const float pos = static_cast<float>(k < quarter ? h : w);
+  const float inv_freq = exp2f(-static_cast<float>(kk) / static_cast<float>(quarter) * log2_theta);
+  float s, c;
+  sincosf(pos * inv_freq, &s, &c);
+  cos_out[idx] = c;
+  sin_out[idx] = s;
+}
+
+// One warp per row (y may alias x).  Pass 1 accumulates the sum of squares in fp32; pass 2 re-reads the row
+// (L1 hit), scales and casts.  bf16 rows are read and written 16 bytes per lane.
+template <bool BF16>
+__global__ void k_rmsnorm(const void* x, const float* __restrict__ w, void* y,
+                          int64_t rows, int d, float eps) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float ss = 0.0f;
+  if constexpr (BF16) {
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + row * d);
+    for (int c = lane; c < d / 8; c += 32) {
+      const uint4 v = xr[c];
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = bf16_lo(u[e]), b = bf16_hi(u[e]);
+        ss += a * a + b * b;
+      }
+    }
+  } else {
+    const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * d);
+    for (int c = lane; c < d / 4; c += 32) {
+      const float4 v = xr[c];
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
+  if constexpr (BF16) {
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + row * d);
+    uint4* yr = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(y) + row * d);
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    for (int c = lane; c < d / 8; c += 32) {
+      const uint4 v = xr[c];
+      const float4 wa = w4[2 * c], wb = w4[2 * c + 1];
+      uint4 o;
+      o.x = pack_bf16x2(bf16_lo(v.x) * inv * wa.x, bf16_hi(v.x) * inv * wa.y);
+      o.y = pack_bf16x2(bf16_lo(v.y) * inv * wa.z, bf16_hi(v.y) * inv * wa.w);
+      o.z = pack_bf16x2(bf16_lo(v.z) * inv * wb.x, bf16_hi(v.z) * inv * wb.y);
+      o.w = pack_bf16x2(bf16_lo(v.w) * inv * wb.z, bf16_hi(v.w) * inv * wb.w);
+      yr[c] = o;
+    }
+  } else {
+    const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * d);
+    float4* yr = reinterpret_cast<float4*>(static_cast<float*>(y) + row * d);
+    const float4* w4 = reinterpret_cast<const float4*>(w);
+    for (int c = lane; c < d / 4; c += 32) {
+      const float4 v = xr[c], ww = w4[c];
+      yr[c] = make_float4(v.x * inv * ww.x, v.y * inv * ww.y, v.z * inv * ww.z, v.w * inv * ww.w);
+    }
+  }
+}
+
+// src[t * r^2 + a * r + b] = packed row of the patch at window position (a, b) of token t, or
+// -1 where the window reaches into the zero padding.  Token offsets are rebuilt in shared
+// memory from the grids (one prefix sum per block).
+__global__ void k_aligner_index(const int32_t* __restrict__ cu, const int32_t* __restrict__ grid, int n_images,
+                                int r, int64_t n_tokens, int32_t* __restrict__ src) {
+  extern __shared__ int32_t tok_cu[];  // [n_images + 1]
+  if (threadIdx.x == 0) {
+    int32_t acc = 0;
+    tok_cu[0] = 0;
+    for (int i = 0; i < n_images; ++i) {
+      const int g_h = (grid[2 * i] + r - 1) / r, g_w = (grid[2 * i + 1] + r - 1) / r;
+      acc += g_h * g_w;
+      tok_cu[i + 1] = acc;
+    }
+  }
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= n_tokens) return;
+  const int img = image_of(tok_cu, n_images, t);
+  const int n_h = grid[2 * img], n_w = grid[2 * img + 1];
+  const int g_w = (n_w + r - 1) / r;
+  const int local = static_cast<int>(t - tok_cu[img]);
+  const int i = local / g_w, j = local - i * g_w;
+  for (int a = 0; a < r; ++a)
+    for (int b = 0; b < r; ++b) {
+      const int h = r * i + a, w = r * j + b;
+      src[t * r * r + a * r + b] = (h < n_h && w < n_w) ? cu[img] + h * n_w + w : -1;
+    }
+}
+
+// Waits on an mbarrier that nothing signals, with the production kernels' bounded wait.
+__global__ void k_selftest_wait(uint64_t limit_ns, uint32_t* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = global_timer_ns();
+    bool done = false;
+    while (!done) {
+      if (mbar_try_wait(&bar, 0)) break;
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicCAS(err, 0u, static_cast<uint32_t>(kErrTimeoutSelftest));
+        done = true;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_rope_table(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int64_t P, int half,
+                              float theta, float* cos_out, float* sin_out, cudaStream_t s) {
+  const int64_t n = P * half;
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (n + threads - 1) / threads;
+  k_rope_table<<<static_cast<unsigned>(blocks), threads, 0, s>>>(cu_dev, grid_dev, n_images, P, half, log2f(theta),
+                                                                 cos_out, sin_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm(bool bf16, const void* x, const float* w, void* y, int64_t rows, int d, float eps,
+                           cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  const int warps = 8;
+  const int64_t blocks = (rows + warps - 1) / warps;
+  if (bf16)
+    k_rmsnorm<true><<<static_cast<unsigned>(blocks), warps * 32, 0, s>>>(x, w, y, rows, d, eps);
+  else
+    k_rmsnorm<false><<<static_cast<unsigned>(blocks), warps * 32, 0, s>>>(x, w, y, rows, d, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int r,
+                                 int64_t n_tokens, int32_t* src_out, cudaStream_t s) {
+  if (n_tokens == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (n_tokens + threads - 1) / threads;
+  k_aligner_index<<<static_cast<unsigned>(blocks), threads, (n_images + 1) * sizeof(int32_t), s>>>(
+      cu_dev, grid_dev, n_images, r, n_tokens, src_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s) {
+  k_selftest_wait<<<1, 32, 0, s>>>(limit_ns, err);
+  return cudaGetLastError();
+}
+
+}  // namespace dsv4v

@@ -1,0 +1,204 @@
+"""Python binding of the dsv4v C ABI (include/dsv4v.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and passes raw device pointers
+of torch tensors plus the current CUDA stream; all arithmetic happens in the CUDA library.
+There is no fallback: if ``libdsv4v.so`` cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsv4v.so")
+
+DSV4V_F32 = 0
+DSV4V_BF16 = 1
+DSV4V_MAX_IMAGES = 1024
+
+STATUS = {0: "DSV4V_OK", 1: "DSV4V_ERR_INVALID_ARG", 2: "DSV4V_ERR_UNSUPPORTED", 3: "DSV4V_ERR_WORKSPACE",
+          4: "DSV4V_ERR_CUDA", 5: "DSV4V_ERR_TIMEOUT"}
+
+# Every symbol include/dsv4v.h declares.
+EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", "dsv4v_tower_forward",
+           "dsv4v_aligner_forward", "dsv4v_aligner_tokens", "dsv4v_rmsnorm", "dsv4v_qkv_rope", "dsv4v_attention",
+           "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
+           "dsv4v_status_string")
+
+
+class Dsv4vError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("vision_dim", ctypes.c_int), ("n_heads", ctypes.c_int), ("mlp_hidden", ctypes.c_int),
+                ("downsample_ratio", ctypes.c_int), ("llm_dim", ctypes.c_int), ("n_layers", ctypes.c_int),
+                ("eps", ctypes.c_float), ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int)]
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [("norm1_w", ctypes.c_void_p), ("norm2_w", ctypes.c_void_p), ("wqkv", ctypes.c_void_p),
+                ("wo", ctypes.c_void_p), ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
+                ("w_down", ctypes.c_void_p)]
+
+
+class Batch(ctypes.Structure):
+    _fields_ = [("n_images", ctypes.c_int), ("grid_hw_host", ctypes.c_void_p), ("grid_hw_dev", ctypes.c_void_p),
+                ("cu_patches_host", ctypes.c_void_p), ("cu_patches_dev", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libdsv4v.so (built by ``build.build()``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run vision_transformer_encoder_dsv4v_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64
+        cfg, bat, bw = ctypes.POINTER(Config), ctypes.POINTER(Batch), ctypes.POINTER(BlockWeights)
+        sig = {
+            "dsv4v_workspace_size": (SZ, [cfg, bat]),
+            "dsv4v_aligner_tokens": (I64, [cfg, bat]),
+            "dsv4v_rope2d_table": (I, [cfg, bat, P, P, P]),
+            "dsv4v_block_forward": (I, [cfg, bat, bw, P, P, P, P, SZ, P]),
+            "dsv4v_tower_forward": (I, [cfg, bat, bw, P, P, P, SZ, P]),
+            "dsv4v_aligner_forward": (I, [cfg, bat, P, P, P, P, P, SZ, P]),
+            "dsv4v_rmsnorm": (I, [cfg, I64, P, P, P, P]),
+            "dsv4v_qkv_rope": (I, [cfg, bat, P, P, P, P, P, P, SZ, P]),
+            "dsv4v_attention": (I, [cfg, bat, P, P, P]),
+            "dsv4v_linear_residual": (I, [cfg, I64, I, P, P, P, P, SZ, P]),
+            "dsv4v_swiglu": (I, [cfg, I64, P, P, P, P, P, SZ, P]),
+            "dsv4v_device_error": (I, [P]),
+            "dsv4v_selftest_bounded_wait": (I, [U64, P]),
+            "dsv4v_status_string": (ctypes.c_char_p, [I]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------------------ marshalling
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is not None:
+        return ctypes.c_void_p(stream)
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise Dsv4vError(status, where)
+
+
+def make_config(vision_dim, n_heads, mlp_hidden, downsample_ratio, llm_dim, n_layers, eps=1e-6, rope_theta=10000.0,
+                dtype=DSV4V_BF16) -> Config:
+    return Config(vision_dim, n_heads, mlp_hidden, downsample_ratio, llm_dim, n_layers, eps, rope_theta, dtype)
+
+
+class BatchRef:
+    """A dsv4v_batch plus the host and device int32 tensors it points to (kept alive here)."""
+
+    def __init__(self, grids, device="cuda"):
+        import torch
+        self.grids = [(int(h), int(w)) for h, w in grids]
+        cu = [0]
+        for h, w in self.grids:
+            cu.append(cu[-1] + h * w)
+        self.grid_host = torch.tensor(self.grids, dtype=torch.int32).reshape(-1, 2).contiguous()
+        self.cu_host = torch.tensor(cu, dtype=torch.int32)
+        self.grid_dev = self.grid_host.to(device)
+        self.cu_dev = self.cu_host.to(device)
+        self.n_patches = cu[-1]
+        self.c = Batch(len(self.grids), self.grid_host.data_ptr(), self.grid_dev.data_ptr(), self.cu_host.data_ptr(),
+                       self.cu_dev.data_ptr())
+
+
+def block_weights(layer: dict) -> BlockWeights:
+    """layer: dict of device tensors norm1_w, norm2_w (fp32) and wqkv, wo, w_gate, w_up, w_down."""
+    return BlockWeights(*(layer[k].data_ptr() for k in ("norm1_w", "norm2_w", "wqkv", "wo", "w_gate", "w_up", "w_down")))
+
+
+# ------------------------------------------------------------------------------ entry points
+def dsv4v_workspace_size(cfg: Config, batch: BatchRef) -> int:
+    return int(lib().dsv4v_workspace_size(ctypes.byref(cfg), ctypes.byref(batch.c)))
+
+
+def dsv4v_aligner_tokens(cfg: Config, batch: BatchRef) -> int:
+    return int(lib().dsv4v_aligner_tokens(ctypes.byref(cfg), ctypes.byref(batch.c)))
+
+
+def dsv4v_rope2d_table(cfg, batch, cos_out, sin_out, stream=None):
+    _check(lib().dsv4v_rope2d_table(ctypes.byref(cfg), ctypes.byref(batch.c), _ptr(cos_out), _ptr(sin_out),
+                                    _stream(stream)), "dsv4v_rope2d_table")
+
+
+def dsv4v_block_forward(cfg, batch, weights: BlockWeights, cos, sin, x_inout, workspace, stream=None):
+    _check(lib().dsv4v_block_forward(ctypes.byref(cfg), ctypes.byref(batch.c), ctypes.byref(weights), _ptr(cos),
+                                     _ptr(sin), _ptr(x_inout), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "dsv4v_block_forward")
+
+
+def dsv4v_tower_forward(cfg, batch, layers, final_norm_w, x_inout, workspace, stream=None):
+    arr = (BlockWeights * max(1, len(layers)))(*layers)
+    _check(lib().dsv4v_tower_forward(ctypes.byref(cfg), ctypes.byref(batch.c), arr, _ptr(final_norm_w),
+                                     _ptr(x_inout), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "dsv4v_tower_forward")
+
+
+def dsv4v_aligner_forward(cfg, batch, x, w_align, out, workspace, cu_tokens_host=None, stream=None):
+    buf = None
+    if cu_tokens_host is not None:
+        buf = cu_tokens_host.data_ptr()
+    _check(lib().dsv4v_aligner_forward(ctypes.byref(cfg), ctypes.byref(batch.c), _ptr(x), _ptr(w_align), _ptr(out),
+                                       buf, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "dsv4v_aligner_forward")
+
+
+def dsv4v_rmsnorm(cfg, rows, x, w, y, stream=None):
+    _check(lib().dsv4v_rmsnorm(ctypes.byref(cfg), rows, _ptr(x), _ptr(w), _ptr(y), _stream(stream)), "dsv4v_rmsnorm")
+
+
+def dsv4v_qkv_rope(cfg, batch, y, wqkv, cos, sin, qkv, workspace, stream=None):
+    _check(lib().dsv4v_qkv_rope(ctypes.byref(cfg), ctypes.byref(batch.c), _ptr(y), _ptr(wqkv), _ptr(cos), _ptr(sin),
+                                _ptr(qkv), _ptr(workspace), workspace.numel(), _stream(stream)), "dsv4v_qkv_rope")
+
+
+def dsv4v_attention(cfg, batch, qkv, out, stream=None):
+    _check(lib().dsv4v_attention(ctypes.byref(cfg), ctypes.byref(batch.c), _ptr(qkv), _ptr(out), _stream(stream)),
+           "dsv4v_attention")
+
+
+def dsv4v_linear_residual(cfg, rows, k, a, w, x, workspace, stream=None):
+    _check(lib().dsv4v_linear_residual(ctypes.byref(cfg), rows, k, _ptr(a), _ptr(w), _ptr(x), _ptr(workspace),
+                                       workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "dsv4v_linear_residual")
+
+
+def dsv4v_swiglu(cfg, rows, y, w_gate, w_up, h, workspace, stream=None):
+    _check(lib().dsv4v_swiglu(ctypes.byref(cfg), rows, _ptr(y), _ptr(w_gate), _ptr(w_up), _ptr(h), _ptr(workspace),
+                              workspace.numel() if workspace is not None else 0, _stream(stream)), "dsv4v_swiglu")
+
+
+def dsv4v_device_error(stream=None) -> int:
+    return int(lib().dsv4v_device_error(_stream(stream)))
+
+
+def dsv4v_selftest_bounded_wait(limit_ns: int, stream=None):
+    _check(lib().dsv4v_selftest_bounded_wait(limit_ns, _stream(stream)), "dsv4v_selftest_bounded_wait")
+
+
+def dsv4v_status_string(status: int) -> str:
+    return lib().dsv4v_status_string(status).decode()
