@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--workload", type=int, default=4, choices=[4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="run warm-up + steps as plain C-ABI calls (no graph, no extra passes) for ncu; "
+                         "prints no bench line")
     return ap.parse_args()
 
 
@@ -222,6 +225,15 @@ def run_ours(args):
         x.copy_(x0)
         A.dsv4v_tower_forward(cfg, batch, lw, fnw, x, ws, stream=s.cuda_stream)
         A.dsv4v_aligner_forward(cfg, batch, x, wa, out, ws, stream=s.cuda_stream)
+
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            with torch.cuda.stream(stream):
+                step(stream)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_run": True, "device_error": A.dsv4v_device_error(),
+                          "kernels_per_step": 7 * wl.n_layers + 4}), flush=True)
+        return
 
     # Capture one step (all kernels of the path, launched through the C ABI) in a CUDA graph.
     with torch.cuda.stream(stream):

@@ -54,7 +54,8 @@ def test_workload1_fp32_block_and_aligner():
     assert np.abs(to_np(out) - want_a).max() <= 1e-4
     # the tower entry point with one layer and no final norm is the same block
     x2 = dev(inp.x)
-    A.dsv4v_tower_forward(cfg, b, [A.block_weights(upload_layers(inp)[0])], None, x2, workspace(cfg, b))
+    layer = upload_layers(inp)[0]  # keep the device tensors alive across the call
+    A.dsv4v_tower_forward(cfg, b, [A.block_weights(layer)], None, x2, workspace(cfg, b))
     assert np.abs(to_np(x2) - want).max() <= 1e-4
 
 
