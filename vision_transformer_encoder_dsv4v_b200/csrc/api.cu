@@ -337,7 +337,9 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   void* qkv = c.at<void>(c.lay.qkv);
   void* attn = c.at<void>(c.lay.attn);
   void* h = c.at<void>(c.lay.h);
-  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm1_w, y, s.P, s.D, c.eps, c.stream)));
+  // The block's first kernel also clears the split-K tile counters of its GEMMs.
+  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm1_w, y, s.P, s.D, c.eps, c.stream, c.at<int>(c.lay.counters),
+                                       static_cast<int>(c.lay.counters_bytes / sizeof(int)))));
   DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, y, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr, cos, sin));
   DSV4V_TRY(attention_bf16(c, b, qkv, attn));
   DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x));
@@ -383,7 +385,8 @@ dsv4v_status reset_counters(const Ctx& c) {
 
 dsv4v_status rope_table(const Ctx& c, const dsv4v_batch* b, float* cos, float* sin) {
   return cuda_status(launch_rope_table(b->cu_patches_dev, b->grid_hw_dev, b->n_images, c.s.P, c.s.hd / 2, c.theta,
-                                       cos, sin, c.stream));
+                                       cos, sin, c.stream, c.s.bf16 ? c.at<int>(c.lay.counters) : nullptr,
+                                       c.s.bf16 ? static_cast<int>(c.lay.counters_bytes / sizeof(int)) : 0));
 }
 
 // Validation-only context for component calls that take a row count instead of a batch.
@@ -452,7 +455,6 @@ dsv4v_status dsv4v_block_forward(const dsv4v_config* cfg, const dsv4v_batch* bat
   DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
   if (!weights_ok(w) || !cos || !sin || !x_inout || !aligned16(x_inout) || !aligned16(cos) || !aligned16(sin))
     return DSV4V_ERR_INVALID_ARG;
-  DSV4V_TRY(reset_counters(c));
   return c.s.bf16 ? block_bf16(c, batch, w, cos, sin, x_inout) : block_f32(c, batch, w, cos, sin, x_inout);
 }
 
@@ -467,7 +469,6 @@ dsv4v_status dsv4v_tower_forward(const dsv4v_config* cfg, const dsv4v_batch* bat
   if (final_norm_w && !aligned16(final_norm_w)) return DSV4V_ERR_INVALID_ARG;
   float* cos = c.at<float>(c.lay.cos);
   float* sin = c.at<float>(c.lay.sin);
-  DSV4V_TRY(reset_counters(c));
   DSV4V_TRY(rope_table(c, batch, cos, sin));
   for (int l = 0; l < c.s.L; ++l)
     DSV4V_TRY(c.s.bf16 ? block_bf16(c, batch, &layers[l], cos, sin, x_inout)
@@ -494,9 +495,9 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
   }
   const Shape& s = c.s;
   int32_t* src = c.at<int32_t>(c.lay.asrc);
-  DSV4V_TRY(reset_counters(c));
-  DSV4V_TRY(cuda_status(
-      launch_aligner_index(batch->cu_patches_dev, batch->grid_hw_dev, batch->n_images, s.r, s.T, src, c.stream)));
+  DSV4V_TRY(cuda_status(launch_aligner_index(batch->cu_patches_dev, batch->grid_hw_dev, batch->n_images, s.r, s.T,
+                                             src, c.stream, s.bf16 ? c.at<int>(c.lay.counters) : nullptr,
+                                             s.bf16 ? static_cast<int>(c.lay.counters_bytes / sizeof(int)) : 0)));
   const int K = s.r * s.r * s.D;
   if (s.bf16)
     return gemm_bf16(c, EPI_STORE, c.plans.align, nullptr, s.T, K, w_align, nullptr, s.E, out, nullptr, nullptr,

@@ -42,6 +42,26 @@ struct Params {
   uint32_t* err;
 };
 
+// 2^x on the MUFU pipe (flushes results below 2^-126 to zero).
+__device__ __forceinline__ float ex2_mufu(float x) { return ex2_approx(x); }
+
+// 2^x for x <= 0 on the FMA pipe, used for a quarter of the softmax exponentials so that the
+// MUFU pipe is not the only one doing them.  Range reduction x = n + f with n = round(x) (the
+// 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2]; 2^f by a cubic fitted here for minimum
+// relative error on that interval (max 7.5e-5, far below the bf16 rounding of P); 2^n is added
+// to the exponent field.  Inputs below -125 (masked keys included) return 0.
+__device__ __forceinline__ float ex2_poly(float x) {
+  const float xc = fmaxf(x, -125.0f);
+  const float t = xc + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = xc - n;
+  const float p = fmaf(fmaf(fmaf(0.0551716573536396f, f, 0.2426111400127411f), f, 0.6932609677314758f), f,
+                       0.9999280571937561f);
+  const int ni = __float_as_int(t) - 0x4B400000;
+  const float r = __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<unsigned>(ni) << 23));
+  return x < -125.0f ? 0.0f : r;
+}
+
 __device__ __forceinline__ void find_item(const AttnSchedule& s, int item, int& img, int& local) {
   int lo = 0, hi = s.n_images - 1;
   while (lo < hi) {
@@ -114,9 +134,12 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_holder;
 
+  if (threadIdx.x == 0) launch_dependents();
+
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      grid_dependency_wait();
       const int col_q = head * HD, col_k = p.vision_dim + head * HD, col_v = 2 * p.vision_dim + head * HD;
       mbar_arrive_expect_tx(q_full, TILE_BYTES);
       tma_load_2d(smem + OFF_Q, &tm_qkv, q_full, col_q, q_row);
@@ -198,6 +221,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int c = 0; c < HD; ++c) o[c] = 0.0f;
     float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
     bool ok = true;
+    grid_dependency_wait();
     auto accumulate_pv = [&](int j, float alpha) -> bool {
       const bool got = mbar_wait(&pv_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
       if (!named_barrier_and(1, 128, got)) return false;
@@ -235,22 +259,36 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       const int valid = min(TK, len - j * TK);
-      float mx = -INFINITY;
+      if (valid < TK) {  // last tile of the image: keys past its end get -inf
 #pragma unroll
-      for (int c = 0; c < TK; ++c)
-        if (c < valid) mx = fmaxf(mx, __uint_as_float(s[c]));
+        for (int c = 0; c < TK; ++c)
+          if (c >= valid) s[c] = 0xFF800000u;
+      }
+      // Row max with eight independent chains.
+      float m8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) m8[u] = __uint_as_float(s[u]);
+#pragma unroll
+      for (int c = 8; c < TK; c += 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], __uint_as_float(s[c + u]));
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
-      const float alpha = exp2f(m_run - m_new);
-      float sum = 0.0f;
+      const float alpha = ex2_mufu(m_run - m_new);
+      const float neg_m = -m_new;
+      float l8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) l8[u] = 0.0f;
       uint8_t* prow = p_smem + (j & 1) * P_BYTES + r * 128;
 #pragma unroll
       for (int c16 = 0; c16 < TK / 8; ++c16) {
         float e[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int c = c16 * 8 + u;
-          e[u] = (c < valid) ? exp2f(__uint_as_float(s[c]) * p.scale_log2 - m_new) : 0.0f;
-          sum += e[u];
+          const float x = fmaf(__uint_as_float(s[c16 * 8 + u]), p.scale_log2, neg_m);
+          e[u] = (u >= 6) ? ex2_poly(x) : ex2_mufu(x);
+          l8[u] += e[u];
         }
         uint4 pk;
         pk.x = pack_bf16x2(e[0], e[1]);
@@ -260,6 +298,7 @@ __global__ void __launch_bounds__(192, 1)
         const int atom = c16 >> 3, chunk = c16 & 7;
         *reinterpret_cast<uint4*>(prow + atom * (TQ * 128) + ((chunk ^ (r & 7)) << 4)) = pk;
       }
+      const float sum = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       l_run = l_run * alpha + sum;
       m_run = m_new;
       fence_proxy_async_smem();  // generic-proxy P stores -> visible to the tensor core
@@ -316,8 +355,7 @@ cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& s
   p.scale_log2 = 1.4426950408889634f / 8.0f;  // log2(e) / sqrt(64)
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = err;
-  k_attn_tc<<<sched.n_items, 192, SMEM_BYTES, s>>>(*tm_qkv, sched, p);
-  return cudaGetLastError();
+  return launch_pdl(k_attn_tc, dim3(sched.n_items), dim3(192), SMEM_BYTES, s, *tm_qkv, sched, p);
 }
 
 }  // namespace dsv4v

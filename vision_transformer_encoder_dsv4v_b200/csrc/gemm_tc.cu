@@ -71,13 +71,15 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+// silu(z) = z / (1 + e^-z), from the MUFU exponential and reciprocal (ample for a bf16 result).
+__device__ __forceinline__ float silu(float z) { return z * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * z)); }
 
 // Epilogue of one 64-column accumulator group held in v[0..63] for output row `row`.
 //   STORE/RESID/QKV: v = accumulator columns [64g, 64g + 64) -> output columns n0 + 64g + j.
 //   SWIGLU: v[0..31] = gate columns, v[32..63] = up columns of output columns n0h + 32g + j.
-template <int EPI, int BN>
-__device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_tile, int g, float (&v)[64]) {
+template <int EPI, int BN, int NR>
+__device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_tile, int g, float (&v)[64],
+                                               const float (&rot_c)[NR], const float (&rot_s)[NR]) {
   if (row >= p.M) return;
   if constexpr (EPI == EPI_SWIGLU) {
     const int col = n_tile * (BN / 2) + g * 32;
@@ -95,20 +97,11 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
     const int col = n_tile * BN + g * 64;
     if constexpr (EPI == EPI_QKV_ROPE) {
       if (col < p.rot_cols) {
-        const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(row) * 32);
-        const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(row) * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 c = c4[q], s = s4[q];
-          const float cc[4] = {c.x, c.y, c.z, c.w};
-          const float ss[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * q + e;
-            const float x1 = v[j], x2 = v[32 + j];
-            v[j] = x1 * cc[e] - x2 * ss[e];
-            v[32 + j] = x2 * cc[e] + x1 * ss[e];
-          }
+        for (int j = 0; j < 32; ++j) {
+          const float x1 = v[j], x2 = v[32 + j];
+          v[j] = x1 * rot_c[j] - x2 * rot_s[j];
+          v[32 + j] = x2 * rot_c[j] + x1 * rot_s[j];
         }
       }
     }
@@ -206,6 +199,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_holder;
+  if (threadIdx.x == 0) launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -213,28 +207,52 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
       bool ok = true;
+      auto load_b = [&](uint8_t* sb, int kb, int n_tile, uint64_t* bar) {
+        if (EPI == EPI_SWIGLU) {
+          tma_load_2d(sb, &tm_b, bar, kb * BK, n_tile * (BN / 2));
+          tma_load_2d(sb + (BN / 2) * 128, &tm_b2, bar, kb * BK, n_tile * (BN / 2));
+        } else {
+          tma_load_2d(sb, &tm_b, bar, kb * BK, n_tile * BN);
+        }
+      };
+      // The weight tiles of the first stages do not depend on the previous kernel: start them
+      // before waiting for it, then add the activation tiles.
+      int pre = 0, pre_kb0 = 0, pre_m = 0;
+      if (static_cast<int>(blockIdx.x) < p.work) {
+        int tile, m_tile, n_tile, kb0, kb1;
+        work_coords(p, blockIdx.x, tile, m_tile, n_tile, kb0, kb1);
+        pre = min(STAGES, kb1 - kb0);
+        pre_kb0 = kb0;
+        pre_m = m_tile;
+        for (int i = 0; i < pre; ++i) {
+          uint8_t* sa = smem + i * C::STAGE;
+          mbar_arrive_expect_tx(&full[i], GATHER ? C::B_BYTES : C::STAGE);
+          load_b(sa + C::A_BYTES, kb0 + i, n_tile, &full[i]);
+          issued |= 1u << i;
+        }
+      }
+      grid_dependency_wait();
+      if (!GATHER)
+        for (int i = 0; i < pre; ++i)
+          tma_load_2d(smem + i * C::STAGE, &tm_a, &full[i], (pre_kb0 + i) * BK, pre_m * BM);
+      stage = pre % STAGES;
+      phase = (pre == STAGES) ? 1u : 0u;
       for (int w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
         int tile, m_tile, n_tile, kb0, kb1;
         work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = (w == static_cast<int>(blockIdx.x) ? kb0 + pre : kb0); kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutProducer)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * C::STAGE;
-          uint8_t* sb = sa + C::A_BYTES;
           if (GATHER) {
             mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::STAGE);
             tma_load_2d(sa, &tm_a, &full[stage], kb * BK, m_tile * BM);
           }
-          if (EPI == EPI_SWIGLU) {
-            tma_load_2d(sb, &tm_b, &full[stage], kb * BK, n_tile * (BN / 2));
-            tma_load_2d(sb + (BN / 2) * 128, &tm_b2, &full[stage], kb * BK, n_tile * (BN / 2));
-          } else {
-            tma_load_2d(sb, &tm_b, &full[stage], kb * BK, n_tile * BN);
-          }
+          load_b(sa + C::A_BYTES, kb, n_tile, &full[stage]);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -303,9 +321,23 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     const int et = threadIdx.x - 64;
     int acc = 0;
     uint32_t acc_phase = 0;
+    grid_dependency_wait();
     for (int w = blockIdx.x; w < p.work; w += gridDim.x) {
       int tile, m_tile, n_tile, kb0, kb1;
       work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
+      // The rotation table row of this thread's output row, fetched while the MMAs run.
+      float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
+      if constexpr (EPI == EPI_QKV_ROPE) {
+        const int prow = min(m_tile * BM + row_in_tile, p.M - 1);
+        const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(prow) * 32);
+        const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(prow) * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 c = c4[q], s = s4[q];
+          rot_c[4 * q] = c.x; rot_c[4 * q + 1] = c.y; rot_c[4 * q + 2] = c.z; rot_c[4 * q + 3] = c.w;
+          rot_s[4 * q] = s.x; rot_s[4 * q + 1] = s.y; rot_s[4 * q + 2] = s.z; rot_s[4 * q + 3] = s.w;
+        }
+      }
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
       // All four epilogue warps continue or stop together (TMEM loads are warp-collective and
       // the split-K path uses a named barrier).
@@ -329,7 +361,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             v[j] = __uint_as_float(r0[j]);
             v[32 + j] = __uint_as_float(r1[j]);
           }
-          epilogue_group<EPI, BN>(p, row, n_tile, g, v);
+          epilogue_group<EPI, BN>(p, row, n_tile, g, v, rot_c, rot_s);
         }
         tc_fence_before_sync();
         mbar_arrive(&tempty[acc]);
@@ -380,7 +412,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 v[32 + 4 * q + 3] += b.w;
               }
             }
-            epilogue_group<EPI, BN>(p, row, n_tile, g, v);
+            epilogue_group<EPI, BN>(p, row, n_tile, g, v, rot_c, rot_s);
           }
           if (et == 0) p.counters[tile] = 0;  // ready for the next launch
         }
@@ -394,6 +426,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     // ------------------------------------------------------------------ A-gather (aligner)
     const int r = threadIdx.x - 192;  // row of the A tile handled by this thread
     const int blocks_per_slot = p.gd / BK;
+    grid_dependency_wait();
     int stage = 0, pending = -1;
     uint32_t phase = 0;
     bool ok = true;
@@ -478,8 +511,7 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.err = a.err;
   const CUtensorMap& ta = GATHER ? *a.tm_b : *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
-  kern<<<plan.grid, GATHER ? 320 : 192, C::SMEM, s>>>(ta, *a.tm_b, tb2, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(plan.grid), dim3(GATHER ? 320 : 192), C::SMEM, s, ta, *a.tm_b, tb2, p);
 }
 
 template <int EPI, bool GATHER>

@@ -67,12 +67,16 @@ cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& s
                                 void* out, uint32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------------------- small kernels
+// The first kernel of an entry point also clears the GEMM tile counters of the call
+// (zero_ptr / zero_n; NULL / 0 when it has none to clear).
 cudaError_t launch_rope_table(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int64_t P, int half,
-                              float theta, float* cos_out, float* sin_out, cudaStream_t s);
+                              float theta, float* cos_out, float* sin_out, cudaStream_t s, int* zero_ptr = nullptr,
+                              int zero_n = 0);
 cudaError_t launch_rmsnorm(bool bf16, const void* x, const float* w, void* y, int64_t rows, int d, float eps,
-                           cudaStream_t s);
+                           cudaStream_t s, int* zero_ptr = nullptr, int zero_n = 0);
 cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int r,
-                                 int64_t n_tokens, int32_t* src_out, cudaStream_t s);
+                                 int64_t n_tokens, int32_t* src_out, cudaStream_t s, int* zero_ptr = nullptr,
+                                 int zero_n = 0);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------------------- fp32 CUDA-core path

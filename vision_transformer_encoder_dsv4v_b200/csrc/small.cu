@@ -7,6 +7,12 @@ namespace dsv4v {
 
 namespace {
 
+// Block 0 clears n ints (the GEMM tile counters of the call).
+__device__ __forceinline__ void zero_ints(int* ptr, int n) {
+  if (ptr && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n; i += blockDim.x) ptr[i] = 0;
+}
+
 // Index of the image that packed row p belongs to: largest i with cu[i] <= p.
 __device__ __forceinline__ int image_of(const int32_t* cu, int n_images, int64_t p) {
   int lo = 0, hi = n_images - 1;
@@ -22,7 +28,10 @@ __device__ __forceinline__ int image_of(const int32_t* cu, int n_images, int64_t
 // patch column w, at inverse frequency theta^(-(k mod half/2) / (half/2)).
 __global__ void k_rope_table(const int32_t* __restrict__ cu, const int32_t* __restrict__ grid, int n_images,
                              int64_t P, int half, float log2_theta, float* __restrict__ cos_out,
-                             float* __restrict__ sin_out) {
+                             float* __restrict__ sin_out, int* zero_ptr, int zero_n) {
+  grid_dependency_wait();
+  launch_dependents();
+  zero_ints(zero_ptr, zero_n);
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= P * half) return;
   const int64_t p = idx / half;
@@ -45,7 +54,10 @@ __global__ void k_rope_table(const int32_t* __restrict__ cu, const int32_t* __re
 // (L1 hit), scales and casts.  bf16 rows are read and written 16 bytes per lane.
 template <bool BF16>
 __global__ void k_rmsnorm(const void* x, const float* __restrict__ w, void* y,
-                          int64_t rows, int d, float eps) {
+                          int64_t rows, int d, float eps, int* zero_ptr, int zero_n) {
+  grid_dependency_wait();
+  launch_dependents();
+  zero_ints(zero_ptr, zero_n);
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -100,8 +112,11 @@ __global__ void k_rmsnorm(const void* x, const float* __restrict__ w, void* y,
 // -1 where the window reaches into the zero padding.  Token offsets are rebuilt in shared
 // memory from the grids (one prefix sum per block).
 __global__ void k_aligner_index(const int32_t* __restrict__ cu, const int32_t* __restrict__ grid, int n_images,
-                                int r, int64_t n_tokens, int32_t* __restrict__ src) {
+                                int r, int64_t n_tokens, int32_t* __restrict__ src, int* zero_ptr, int zero_n) {
   extern __shared__ int32_t tok_cu[];  // [n_images + 1]
+  grid_dependency_wait();
+  launch_dependents();
+  zero_ints(zero_ptr, zero_n);
   if (threadIdx.x == 0) {
     int32_t acc = 0;
     tok_cu[0] = 0;
@@ -151,36 +166,34 @@ __global__ void k_selftest_wait(uint64_t limit_ns, uint32_t* err) {
 }  // namespace
 
 cudaError_t launch_rope_table(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int64_t P, int half,
-                              float theta, float* cos_out, float* sin_out, cudaStream_t s) {
+                              float theta, float* cos_out, float* sin_out, cudaStream_t s, int* zero_ptr, int zero_n) {
   const int64_t n = P * half;
   if (n == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (n + threads - 1) / threads;
-  k_rope_table<<<static_cast<unsigned>(blocks), threads, 0, s>>>(cu_dev, grid_dev, n_images, P, half, log2f(theta),
-                                                                 cos_out, sin_out);
-  return cudaGetLastError();
+  return launch_pdl(k_rope_table, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, s, cu_dev, grid_dev,
+                    n_images, P, half, log2f(theta), cos_out, sin_out, zero_ptr, zero_n);
 }
 
 cudaError_t launch_rmsnorm(bool bf16, const void* x, const float* w, void* y, int64_t rows, int d, float eps,
-                           cudaStream_t s) {
+                           cudaStream_t s, int* zero_ptr, int zero_n) {
   if (rows == 0) return cudaSuccess;
   const int warps = 8;
-  const int64_t blocks = (rows + warps - 1) / warps;
+  const unsigned blocks = static_cast<unsigned>((rows + warps - 1) / warps);
   if (bf16)
-    k_rmsnorm<true><<<static_cast<unsigned>(blocks), warps * 32, 0, s>>>(x, w, y, rows, d, eps);
-  else
-    k_rmsnorm<false><<<static_cast<unsigned>(blocks), warps * 32, 0, s>>>(x, w, y, rows, d, eps);
+    return launch_pdl(k_rmsnorm<true>, dim3(blocks), dim3(warps * 32), 0, s, x, w, y, rows, d, eps, zero_ptr, zero_n);
+  k_rmsnorm<false><<<blocks, warps * 32, 0, s>>>(x, w, y, rows, d, eps, zero_ptr, zero_n);
   return cudaGetLastError();
 }
 
 cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int r,
-                                 int64_t n_tokens, int32_t* src_out, cudaStream_t s) {
+                                 int64_t n_tokens, int32_t* src_out, cudaStream_t s, int* zero_ptr, int zero_n) {
   if (n_tokens == 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (n_tokens + threads - 1) / threads;
-  k_aligner_index<<<static_cast<unsigned>(blocks), threads, (n_images + 1) * sizeof(int32_t), s>>>(
-      cu_dev, grid_dev, n_images, r, n_tokens, src_out);
-  return cudaGetLastError();
+  return launch_pdl(k_aligner_index, dim3(static_cast<unsigned>(blocks)), dim3(threads),
+                    (n_images + 1) * sizeof(int32_t), s, cu_dev, grid_dev, n_images, r, n_tokens, src_out, zero_ptr,
+                    zero_n);
 }
 
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s) {
