@@ -9,9 +9,18 @@
 //               per thread), fused epilogue math, bf16 stores
 //   warps 6..9  (aligner only) A-gather: cp.async rows of the patch matrix into the swizzled
 //               A tile, zero-filling padded window slots
-// The accumulator is double-buffered in TMEM so the epilogue of one tile overlaps the MMAs of
-// the next.  Split-K tiles are combined by the last-arriving contributor (ticket counter):
-// nobody waits on another CTA.
+//
+// Work split (stream-K): the GEMM is U = tiles x (K / 64) units of one 64-deep K block of one
+// output tile; CTA c of G owns units [c U / G, (c + 1) U / G), i.e. equal work per SM whatever
+// the tile count.  A CTA walks its range as segments (a tile and a K-block range).  A segment
+// that covers its whole tile is written directly.  A tile split between CTAs is finished by the
+// CTA that owns its first K block: for that CTA the tile is the last segment of its range, while
+// every other contributor meets the tile as its first segment, writes its fp32 partial to its
+// scratch slot early and bumps the tile's counter.  The finisher waits (bounded) for the counter,
+// adds the partials to its own accumulator in CTA order (deterministic) and runs the epilogue.
+// Only finishers wait, and only on contributors that never wait, so the waits cannot cycle.
+// The accumulator is double-buffered in TMEM so the epilogue of one segment overlaps the MMAs
+// of the next.
 #include <algorithm>
 
 #include "common.cuh"
@@ -38,7 +47,8 @@ struct TileCfg {
 
 struct Params {
   int M, K, n_out;
-  int tiles_m, splits, kb_total, work;
+  int tiles_m, kb_total;
+  long long units;  // tiles * kb_total
   __nv_bfloat16* out;
   int ldo;
   const __nv_bfloat16* resid;
@@ -48,21 +58,47 @@ struct Params {
   const int32_t* gsrc;
   const __nv_bfloat16* gx;
   int gr2, gd;
-  float* partials;
-  int* counters;
+  float* partials;  // [G][BN / 4][128][4] fp32: a contributor's partial of a split tile
+  int* counters;    // [tiles], zero between launches
   uint32_t* err;
 };
 
-__device__ __forceinline__ void work_coords(const Params& p, int w, int& tile, int& m_tile, int& n_tile, int& kb0,
-                                            int& kb1) {
-  tile = w / p.splits;
-  const int split = w - tile * p.splits;
-  m_tile = tile % p.tiles_m;
-  n_tile = tile / p.tiles_m;
-  const int base = p.kb_total / p.splits, rem = p.kb_total % p.splits;
-  kb0 = split * base + min(split, rem);
-  kb1 = kb0 + base + (split < rem ? 1 : 0);
+// ---------------------------------------------------------------------------- stream-K ranges
+__device__ __forceinline__ long long range_begin(const Params& p, int c) {
+  return static_cast<long long>(c) * p.units / gridDim.x;
 }
+// CTA owning unit u: the largest c with range_begin(c) <= u.
+__device__ __forceinline__ int unit_owner(const Params& p, long long u) {
+  return static_cast<int>(((u + 1) * gridDim.x - 1) / p.units);
+}
+
+struct Segment {
+  int tile, m_tile, n_tile, kb0, kb1;
+  bool first;  // first segment of this CTA's range
+};
+
+// Walks the segments of this CTA's unit range.
+struct SegmentWalker {
+  long long u, u_end;
+  bool first;
+  __device__ __forceinline__ explicit SegmentWalker(const Params& p) {
+    u = range_begin(p, blockIdx.x);
+    u_end = range_begin(p, blockIdx.x + 1);
+    first = true;
+  }
+  __device__ __forceinline__ bool next(const Params& p, Segment& s) {
+    if (u >= u_end) return false;
+    s.tile = static_cast<int>(u / p.kb_total);
+    s.kb0 = static_cast<int>(u - static_cast<long long>(s.tile) * p.kb_total);
+    s.kb1 = static_cast<int>(min(static_cast<long long>(p.kb_total), s.kb0 + (u_end - u)));
+    s.m_tile = s.tile % p.tiles_m;
+    s.n_tile = s.tile / p.tiles_m;
+    s.first = first;
+    first = false;
+    u += s.kb1 - s.kb0;
+    return true;
+  }
+};
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -72,7 +108,9 @@ __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // silu(z) = z / (1 + e^-z), from the MUFU exponential and reciprocal (ample for a bf16 result).
-__device__ __forceinline__ float silu(float z) { return z * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * z)); }
+__device__ __forceinline__ float silu(float z) {
+  return z * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * z));
+}
 
 // Epilogue of one 64-column accumulator group held in v[0..63] for output row `row`.
 //   STORE/RESID/QKV: v = accumulator columns [64g, 64g + 64) -> output columns n0 + 64g + j.
@@ -153,6 +191,38 @@ __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   return v;
 }
 
+// Scratch slot of CTA c (a contributor writes at most one partial: its first segment).
+// Layout [BN / 4][128 rows][4]: a warp's 32 rows of one 4-column group are 512 contiguous bytes.
+template <int BN>
+__device__ __forceinline__ float* partial_slot(const Params& p, int c) {
+  return p.partials + static_cast<size_t>(c) * BM * BN;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until *ctr reaches `target` (the other contributors of a split tile).
+__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort_flag, uint32_t* err) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if ((i & 63u) == 63u) {
+      if (*abort_flag) return false;
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        atomicCAS(err, 0u, static_cast<uint32_t>(kErrTimeoutEpilogue));
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 template <int BN, int EPI, bool GATHER>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -215,32 +285,29 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           tma_load_2d(sb, &tm_b, bar, kb * BK, n_tile * BN);
         }
       };
+      SegmentWalker walk(p);
+      Segment sg;
       // The weight tiles of the first stages do not depend on the previous kernel: start them
       // before waiting for it, then add the activation tiles.
-      int pre = 0, pre_kb0 = 0, pre_m = 0;
-      if (static_cast<int>(blockIdx.x) < p.work) {
-        int tile, m_tile, n_tile, kb0, kb1;
-        work_coords(p, blockIdx.x, tile, m_tile, n_tile, kb0, kb1);
-        pre = min(STAGES, kb1 - kb0);
-        pre_kb0 = kb0;
-        pre_m = m_tile;
+      int pre = 0;
+      Segment first{};
+      SegmentWalker peek = walk;
+      if (peek.next(p, first)) {
+        pre = min(STAGES, first.kb1 - first.kb0);
         for (int i = 0; i < pre; ++i) {
-          uint8_t* sa = smem + i * C::STAGE;
           mbar_arrive_expect_tx(&full[i], GATHER ? C::B_BYTES : C::STAGE);
-          load_b(sa + C::A_BYTES, kb0 + i, n_tile, &full[i]);
+          load_b(smem + i * C::STAGE + C::A_BYTES, first.kb0 + i, first.n_tile, &full[i]);
           issued |= 1u << i;
         }
       }
       grid_dependency_wait();
       if (!GATHER)
         for (int i = 0; i < pre; ++i)
-          tma_load_2d(smem + i * C::STAGE, &tm_a, &full[i], (pre_kb0 + i) * BK, pre_m * BM);
+          tma_load_2d(smem + i * C::STAGE, &tm_a, &full[i], (first.kb0 + i) * BK, first.m_tile * BM);
       stage = pre % STAGES;
       phase = (pre == STAGES) ? 1u : 0u;
-      for (int w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
-        int tile, m_tile, n_tile, kb0, kb1;
-        work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
-        for (int kb = (w == static_cast<int>(blockIdx.x) ? kb0 + pre : kb0); kb < kb1; ++kb) {
+      while (ok && walk.next(p, sg)) {
+        for (int kb = sg.first ? sg.kb0 + pre : sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutProducer)) {
             ok = false;
             break;
@@ -250,9 +317,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
           } else {
             mbar_arrive_expect_tx(&full[stage], C::STAGE);
-            tma_load_2d(sa, &tm_a, &full[stage], kb * BK, m_tile * BM);
+            tma_load_2d(sa, &tm_a, &full[stage], kb * BK, sg.m_tile * BM);
           }
-          load_b(sa + C::A_BYTES, kb, n_tile, &full[stage]);
+          load_b(sa + C::A_BYTES, kb, sg.n_tile, &full[stage]);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -274,13 +341,13 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
-        int tile, m_tile, n_tile, kb0, kb1;
-        work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
+      SegmentWalker walk(p);
+      Segment sg;
+      while (ok && walk.next(p, sg)) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutMma)) {
             ok = false;
             break;
@@ -293,7 +360,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4).
-            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -322,13 +389,13 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     grid_dependency_wait();
-    for (int w = blockIdx.x; w < p.work; w += gridDim.x) {
-      int tile, m_tile, n_tile, kb0, kb1;
-      work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
+    SegmentWalker walk(p);
+    Segment sg;
+    while (walk.next(p, sg)) {
       // The rotation table row of this thread's output row, fetched while the MMAs run.
       float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
       if constexpr (EPI == EPI_QKV_ROPE) {
-        const int prow = min(m_tile * BM + row_in_tile, p.M - 1);
+        const int prow = min(sg.m_tile * BM + row_in_tile, p.M - 1);
         const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(prow) * 32);
         const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(prow) * 32);
 #pragma unroll
@@ -340,12 +407,12 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       }
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
       // All four epilogue warps continue or stop together (TMEM loads are warp-collective and
-      // the split-K path uses a named barrier).
+      // the partial-tile path uses a named barrier).
       if (!named_barrier_and(2, 128, got)) break;
       tc_fence_after_sync();
-      const int row = m_tile * BM + row_in_tile;
+      const int row = sg.m_tile * BM + row_in_tile;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      if (p.splits == 1) {
+      if (sg.kb0 == 0 && sg.kb1 == p.kb_total) {
 #pragma unroll 1
         for (int g = 0; g < BN / 64; ++g) {
           int c0, c1;
@@ -361,60 +428,89 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             v[j] = __uint_as_float(r0[j]);
             v[32 + j] = __uint_as_float(r1[j]);
           }
-          epilogue_group<EPI, BN>(p, row, n_tile, g, v, rot_c, rot_s);
+          epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s);
         }
         tc_fence_before_sync();
         mbar_arrive(&tempty[acc]);
       } else {
-        // Write this contribution, then the last contributor of the tile sums all of them in
-        // split order (deterministic) and runs the epilogue.
-        float* slot = p.partials + (static_cast<size_t>(w) * BM + row_in_tile) * BN;
+        const long long u_first = static_cast<long long>(sg.tile) * p.kb_total;
+        const int c_first = unit_owner(p, u_first);
+        const int c_last = unit_owner(p, u_first + p.kb_total - 1);
+        if (static_cast<int>(blockIdx.x) != c_first) {
+          // Contributor: park the partial, release it, move on.
+          float* slot = partial_slot<BN>(p, blockIdx.x);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_row + c * 32, r);
-          tmem_ld_wait(r);
-          float4* dst = reinterpret_cast<float4*>(slot + c * 32);
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_row + c * 32, r);
+            tmem_ld_wait(r);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                                 __uint_as_float(r[4 * q + 3]));
-        }
-        tc_fence_before_sync();
-        mbar_arrive(&tempty[acc]);
-        __threadfence();
-        named_barrier_sync(1, 128);
-        if (et == 0) *ticket = atomicAdd(&p.counters[tile], 1);
-        named_barrier_sync(1, 128);
-        if (*ticket == p.splits - 1) {
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(slot + ((c * 8 + q) * BM + row_in_tile) * 4) =
+                  make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                              __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+          }
+          tc_fence_before_sync();
+          mbar_arrive(&tempty[acc]);
+          __threadfence();
+          named_barrier_sync(1, 128);
+          if (et == 0) atomicAdd(&p.counters[sg.tile], 1);
+        } else {
+          // Finisher: wait for the other contributors, add their partials (CTA order) to the
+          // accumulator and run the epilogue.
+          bool ready = true;
+          if (et == 0) {
+            ready = wait_counter(&p.counters[sg.tile], c_last - c_first, abort_flag, p.err);
+            *ticket = ready ? 1 : 0;
+          }
+          named_barrier_sync(1, 128);
+          if (!*ticket) {
+            tc_fence_before_sync();
+            mbar_arrive(&tempty[acc]);
+            break;
+          }
           __threadfence();
 #pragma unroll 1
           for (int g = 0; g < BN / 64; ++g) {
             int c0, c1;
             group_chunks<EPI, BN>(g, c0, c1);
+            uint32_t r0[32], r1[32];
+            tmem_ld32(t_row + c0 * 32, r0);
+            tmem_ld32(t_row + c1 * 32, r1);
+            tmem_ld_wait(r0);
+            tmem_ld_wait(r1);
             float v[64];
 #pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] = 0.0f;
-#pragma unroll 1
-            for (int s = 0; s < p.splits; ++s) {
-              const float* src = p.partials + (static_cast<size_t>(tile * p.splits + s) * BM + row_in_tile) * BN;
+            for (int j = 0; j < 32; ++j) {
+              v[j] = __uint_as_float(r0[j]);
+              v[32 + j] = __uint_as_float(r1[j]);
+            }
+#pragma unroll 2
+            for (int cc = c_first + 1; cc <= c_last; ++cc) {
+              const float* src = partial_slot<BN>(p, cc);
+              float4 a[8], b[8];
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
-                const float4 a = ld_cg_f4(src + c0 * 32 + 4 * q);
-                const float4 b = ld_cg_f4(src + c1 * 32 + 4 * q);
-                v[4 * q + 0] += a.x;
-                v[4 * q + 1] += a.y;
-                v[4 * q + 2] += a.z;
-                v[4 * q + 3] += a.w;
-                v[32 + 4 * q + 0] += b.x;
-                v[32 + 4 * q + 1] += b.y;
-                v[32 + 4 * q + 2] += b.z;
-                v[32 + 4 * q + 3] += b.w;
+                a[q] = ld_cg_f4(src + ((c0 * 8 + q) * BM + row_in_tile) * 4);
+                b[q] = ld_cg_f4(src + ((c1 * 8 + q) * BM + row_in_tile) * 4);
+              }
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                v[4 * q + 0] += a[q].x;
+                v[4 * q + 1] += a[q].y;
+                v[4 * q + 2] += a[q].z;
+                v[4 * q + 3] += a[q].w;
+                v[32 + 4 * q + 0] += b[q].x;
+                v[32 + 4 * q + 1] += b[q].y;
+                v[32 + 4 * q + 2] += b[q].z;
+                v[32 + 4 * q + 3] += b[q].w;
               }
             }
-            epilogue_group<EPI, BN>(p, row, n_tile, g, v, rot_c, rot_s);
+            epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s);
           }
-          if (et == 0) p.counters[tile] = 0;  // ready for the next launch
+          tc_fence_before_sync();
+          mbar_arrive(&tempty[acc]);
+          if (et == 0) p.counters[sg.tile] = 0;  // ready for the next launch
         }
       }
       if (++acc == 2) {
@@ -430,11 +526,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     int stage = 0, pending = -1;
     uint32_t phase = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
-      int tile, m_tile, n_tile, kb0, kb1;
-      work_coords(p, w, tile, m_tile, n_tile, kb0, kb1);
-      const int row = m_tile * BM + r;
-      for (int kb = kb0; kb < kb1; ++kb) {
+    SegmentWalker walk(p);
+    Segment sg;
+    while (ok && walk.next(p, sg)) {
+      const int row = sg.m_tile * BM + r;
+      for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutGather)) {
           ok = false;
           break;
@@ -493,9 +589,8 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.K = a.K;
   p.n_out = a.n_out;
   p.tiles_m = plan.tiles_m;
-  p.splits = plan.splits;
   p.kb_total = plan.kb_total;
-  p.work = plan.work;
+  p.units = static_cast<long long>(plan.tiles_m) * plan.tiles_n * plan.kb_total;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.ldo = a.ldo;
   p.resid = static_cast<const __nv_bfloat16*>(a.resid);
@@ -525,10 +620,35 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   }
 }
 
-// Cycles of one 64-deep K block on one SM for an N-wide tile: the tensor pipe needs N/2 cycles
-// per K=16 step at M=128; shared memory must also deliver the A (4 KB) and B (N*32 B) slices
-// of the step at 128 B/cycle.
-double kblock_cycles(int bn) { return 4.0 * std::max(bn / 2.0, 32.0 + bn / 4.0); }
+// Cost model (cycles) of one SM's share of a GEMM, used to pick the tile width and the grid.
+//  - one 64-deep K block of a 128 x bn tile: the larger of the tensor-pipe time (bn / 2 cycles
+//    per K=16 step) and the time to stream the A (16 KB) and B (bn * 128 B) tiles from L2 at
+//    ~72 B/cycle per SM, plus ~100 cycles of hand-off;
+//  - a split tile: its partial (128 x bn fp32) written once and read back by the finisher with
+//    the other contributors' partials, plus ~1500 cycles of fence and ticket;
+//  - per CTA: ~2000 cycles of set-up and first-load latency and ~12 cycles per output column.
+double kblock_cycles(int bn) { return std::max(2.0 * bn, (16384.0 + 128.0 * bn) / 72.0 + 100.0); }
+
+double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_out) {
+  const long long units = tiles * kb_total;
+  const long long per_cta = (units + grid - 1) / grid;
+  // Most contributors any tile has: ranges of per_cta units cut a tile of kb_total units.
+  int contrib = 1;
+  for (long long c = 0; c < grid; ++c) {
+    const long long b = c * units / grid, e = (c + 1) * units / grid;
+    if (b / kb_total != (e - 1) / kb_total || b % kb_total || e % kb_total) {
+      const long long t = b / kb_total;
+      const long long c0 = ((t * kb_total + 1) * grid - 1) / units;
+      const long long c1 = (((t + 1) * kb_total) * grid - 1) / units;
+      contrib = std::max<int>(contrib, static_cast<int>(c1 - c0 + 1));
+    }
+  }
+  *contrib_out = contrib;
+  const double slot = 128.0 * bn * 4.0 / 128.0;
+  double cost = per_cta * kblock_cycles(bn) + 2000.0 + 12.0 * bn;
+  if (contrib > 1) cost += 1000.0 + slot * contrib;
+  return cost;
+}
 
 }  // namespace
 
@@ -538,29 +658,34 @@ GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms) {
   const int kb_total = K / BK;
   const int tiles_m = (M + BM - 1) / BM;
   const int cands[4] = {256, 192, 128, 64};
+  if (kb_total <= 0 || tiles_m <= 0 || num_sms <= 0) return best;
   for (int bn : cands) {
-    int n_cols_per_tile = (epi == EPI_SWIGLU) ? bn / 2 : bn;
+    const int n_cols_per_tile = (epi == EPI_SWIGLU) ? bn / 2 : bn;
     if (n_out % n_cols_per_tile) continue;
     const int tiles_n = n_out / n_cols_per_tile;
-    const int tiles = tiles_m * tiles_n;
-    for (int splits = 1; splits <= std::min(8, kb_total); ++splits) {
-      if (splits > 1 && tiles * splits > 2 * num_sms) break;
-      const int work = tiles * splits;
-      const int waves = (work + num_sms - 1) / num_sms;
-      const int kb_per = (kb_total + splits - 1) / splits;
-      double cost = waves * (kb_per * kblock_cycles(bn)) + 1500.0;
-      if (splits > 1) cost += 128.0 * bn * 4.0 * (splits + 1) / 64.0 + 800.0;  // partials through L2
+    const long long tiles = static_cast<long long>(tiles_m) * tiles_n;
+    const long long units = tiles * kb_total;
+    // Grids: every SM; or s CTAs per tile (s = 1: one tile each, s > 1: split-K by s).
+    int grids[6];
+    int n_grids = 0;
+    grids[n_grids++] = static_cast<int>(std::min<long long>(num_sms, units));
+    for (int s = 1; s <= 4; ++s)
+      if (tiles * s <= num_sms && tiles * s <= units) grids[n_grids++] = static_cast<int>(tiles * s);
+    for (int gi = 0; gi < n_grids; ++gi) {
+      int contrib = 1;
+      const double cost = plan_cost(bn, tiles, kb_total, grids[gi], &contrib);
+      if (contrib > 8) continue;  // keep the finisher's read-back short
       if (cost < best_cost - 1e-9) {
         best_cost = cost;
         best.bn = bn;
-        best.splits = splits;
+        best.splits = contrib;
         best.tiles_m = tiles_m;
         best.tiles_n = tiles_n;
         best.kb_total = kb_total;
-        best.work = work;
-        best.grid = std::min(work, num_sms);
-        best.partial_bytes = splits > 1 ? static_cast<size_t>(work) * BM * bn * sizeof(float) : 0;
-        best.counters = splits > 1 ? tiles : 0;
+        best.work = static_cast<int>(tiles);
+        best.grid = grids[gi];
+        best.partial_bytes = contrib > 1 ? static_cast<size_t>(grids[gi]) * BM * bn * sizeof(float) : 0;
+        best.counters = contrib > 1 ? static_cast<int>(tiles) : 0;
       }
     }
   }
