@@ -232,7 +232,7 @@ def run_ours(args):
                 step(stream)
         torch.cuda.synchronize()
         print(json.dumps({"profile_run": True, "device_error": A.dsv4v_device_error(),
-                          "kernels_per_step": 7 * wl.n_layers + 4}), flush=True)
+                          "kernels_per_step": 5 * wl.n_layers + 5}), flush=True)
         return
 
     # Capture one step (all kernels of the path, launched through the C ABI) in a CUDA graph.
@@ -245,8 +245,9 @@ def run_ours(args):
     torch.cuda.synchronize()
     if A.dsv4v_device_error() != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
-    launches_per_step = 7 * wl.n_layers + 4  # per layer: 2 norms, 4 GEMMs, attention; rope table, final norm,
-    #                                          aligner index, aligner GEMM
+    # per layer: 4 GEMMs + attention; plus the rotary table, the first norm operand, the final
+    # norm, the aligner index and the aligner GEMM
+    launches_per_step = 5 * wl.n_layers + 5
 
     for _ in range(args.warmup):
         with torch.cuda.stream(stream):
@@ -281,7 +282,7 @@ def run_ours(args):
     tflops = synth.algorithmic_flops(wl) * world * args.steps / (total_ms / 1e3) / 1e12
 
     # ---- kernel timing pass: the same step as component calls, with events around each launch
-    kern = kernel_timing(A, torch, cfg, batch, wl, layers, fnw, wa, x0, x, out, ws, stream, flush, args.steps)
+    kern = kernel_timing(A, torch, cfg, batch, wl, lw, fnw, wa, x0, x, out, ws, stream, flush, args.steps)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     x_host = x0.cpu().pin_memory()
@@ -342,65 +343,49 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def kernel_timing(A, torch, cfg, batch, wl, layers, fnw, wa, x0, x, out, ws, stream, flush, steps):
-    """Per-launch device time of each kernel of the step, from CUDA events recorded on the
-    launching stream around every launch of the step issued as component calls (same kernels,
-    same plans as the tower entry point) inside one CUDA graph."""
+def kernel_timing(A, torch, cfg, batch, wl, lw, fnw, wa, x0, x, out, ws, stream, flush, steps):
+    """Per-launch device time of each GEMM class and the attention kernel, from CUDA events that
+    the library records on the launching stream around every launch of the step
+    (dsv4v_tower_forward_profiled, same kernels and plans as dsv4v_tower_forward), captured in
+    one CUDA graph and replayed `steps` times with an L2 flush between replays."""
     D, F, P = wl.vision_dim, wl.mlp_hidden, wl.n_patches
-    hd2 = wl.head_dim // 2
-    cos = torch.empty(P, hd2, device="cuda")
-    sin = torch.empty_like(cos)
-    y = torch.empty(P, D, dtype=torch.bfloat16, device="cuda")
-    qkv = torch.empty(P, 3 * D, dtype=torch.bfloat16, device="cuda")
-    attn = torch.empty(P, D, dtype=torch.bfloat16, device="cuda")
-    h = torch.empty(P, F, dtype=torch.bfloat16, device="cuda")
-    s = stream.cuda_stream
-    names = ["rmsnorm", "gemm_qkv_rope", "attention", "gemm_out_resid", "gemm_swiglu", "gemm_down_resid"]
-    flops = {"gemm_qkv_rope": 2.0 * P * D * 3 * D, "gemm_out_resid": 2.0 * P * D * D,
-             "gemm_swiglu": 2.0 * P * D * 2 * F, "gemm_down_resid": 2.0 * P * F * D,
-             "attention": sum(4.0 * (a * b) ** 2 * D for a, b in wl.grids)}
-    events = {n: [] for n in names}
-
-    def timed(name, fn):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fn()
-        b.record(stream)
-        events[name].append((a, b))
+    kinds = A.PROFILE_KINDS
+    flops = {"qkv": 2.0 * P * D * 3 * D, "out": 2.0 * P * D * D, "swiglu": 2.0 * P * D * 2 * F,
+             "down": 2.0 * P * F * D, "attention": sum(4.0 * (a * b) ** 2 * D for a, b in wl.grids)}
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(wl.n_layers * len(kinds) * 2)]
+    for e in events:  # creates the CUDA handles
+        e.record(stream)
+    torch.cuda.synchronize()
 
     def one_step():
         x.copy_(x0)
-        A.dsv4v_rope2d_table(cfg, batch, cos, sin, stream=s)
-        for l in layers:
-            timed("rmsnorm", lambda: A.dsv4v_rmsnorm(cfg, P, x, l["norm1_w"], y, stream=s))
-            timed("gemm_qkv_rope", lambda: A.dsv4v_qkv_rope(cfg, batch, y, l["wqkv"], cos, sin, qkv, ws, stream=s))
-            timed("attention", lambda: A.dsv4v_attention(cfg, batch, qkv, attn, stream=s))
-            timed("gemm_out_resid", lambda: A.dsv4v_linear_residual(cfg, P, D, attn, l["wo"], x, ws, stream=s))
-            timed("rmsnorm", lambda: A.dsv4v_rmsnorm(cfg, P, x, l["norm2_w"], y, stream=s))
-            timed("gemm_swiglu", lambda: A.dsv4v_swiglu(cfg, P, y, l["w_gate"], l["w_up"], h, ws, stream=s))
-            timed("gemm_down_resid", lambda: A.dsv4v_linear_residual(cfg, P, F, h, l["w_down"], x, ws, stream=s))
+        A.dsv4v_tower_forward_profiled(cfg, batch, lw, fnw, x, ws, events, stream=stream.cuda_stream)
+        A.dsv4v_aligner_forward(cfg, batch, x, wa, out, ws, stream=stream.cuda_stream)
 
     with torch.cuda.stream(stream):
         one_step()
     torch.cuda.synchronize()
-    for n in names:
-        events[n].clear()
-    for _ in range(steps):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_step()
+    times = {k: [] for k in kinds}
+    for i in range(steps + 2):
         with torch.cuda.stream(stream):
             flush.zero_()
-            one_step()
-    torch.cuda.synchronize()
+            g.replay()
+        stream.synchronize()
+        if i < 2:
+            continue
+        for l in range(wl.n_layers):
+            for ki, k in enumerate(kinds):
+                a, b = events[(l * len(kinds) + ki) * 2], events[(l * len(kinds) + ki) * 2 + 1]
+                times[k].append(a.elapsed_time(b))
     res = {}
-    for n in names:
-        ts = [a.elapsed_time(b) for a, b in events[n]]
+    for k in kinds:
+        ts = times[k]
         avg_us = 1e3 * sum(ts) / len(ts)
-        r = {"launches": len(ts), "avg_us": avg_us, "total_ms": sum(ts)}
-        if n in flops:
-            r["tflops"] = flops[n] / (avg_us * 1e-6) / 1e12
-        if n == "rmsnorm":
-            r["gbs"] = 2.0 * P * D * 2 / (avg_us * 1e-6) / 1e9
-        res[n] = r
-    dom_name = max((n for n in names if n in flops), key=lambda n: res[n]["total_ms"])
+        res[k] = {"launches": len(ts), "avg_us": avg_us, "total_ms": sum(ts), "tflops": flops[k] / (avg_us * 1e-6) / 1e12}
+    dom_name = max(kinds, key=lambda k: res[k]["total_ms"])
     return {"all": res, "dominant": {"name": dom_name, **res[dom_name]}}
 
 

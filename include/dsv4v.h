@@ -152,6 +152,27 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
  * invalid. */
 int64_t dsv4v_aligner_tokens(const dsv4v_config* cfg, const dsv4v_batch* batch);
 
+/* Kernel classes that dsv4v_tower_forward_profiled brackets with events. */
+enum {
+  DSV4V_PROFILE_QKV = 0,        /* fused projection + rotation GEMM (norm1 folded in) */
+  DSV4V_PROFILE_ATTENTION = 1,  /* varlen attention */
+  DSV4V_PROFILE_OUT = 2,        /* output projection + residual (prepares norm2) */
+  DSV4V_PROFILE_SWIGLU = 3,     /* gate/up GEMM + silu*mul (norm2 folded in) */
+  DSV4V_PROFILE_DOWN = 4,       /* down projection + residual (prepares the next norm1) */
+  DSV4V_PROFILE_KINDS = 5
+};
+
+/* dsv4v_tower_forward, recording CUDA events around the launches of every layer:
+ * events[(layer * DSV4V_PROFILE_KINDS + kind) * 2 + 0] before and [... + 1] after the kernel
+ * of that class (cudaEvent_t handles passed as void*, created by the caller; NULL entries are
+ * skipped).  The events sit between kernels, so the bracketed kernels cannot overlap their
+ * neighbours as in dsv4v_tower_forward; per-kernel durations from them are standalone
+ * durations.  Same results as dsv4v_tower_forward. */
+dsv4v_status dsv4v_tower_forward_profiled(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                          const dsv4v_block_weights* layers, const float* final_norm_w,
+                                          void* x_inout, void* workspace, size_t ws_bytes, void* stream,
+                                          void* const* events);
+
 /* ---- Component entry points: single steps of the block, for testing and profiling. ---- */
 
 /* RMSNorm [vision-API, DeepseekV4VisionRMSNorm]: y = w * x / sqrt(mean(x^2) + eps) per row,

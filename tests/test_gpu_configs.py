@@ -135,6 +135,27 @@ def run_tower_and_aligner(wl, inp):
     return to_np(x), to_np(out)
 
 
+def test_profiled_tower_matches_plain():
+    """dsv4v_tower_forward_profiled computes the same tower (bitwise) and records its events."""
+    wl = synth.workload(4)
+    inp = synth.draw(wl, n_layers=3)
+    cfg = config_of(wl, n_layers=3)
+    b = A.BatchRef(wl.grids)
+    ws = workspace(cfg, b)
+    layers = upload_layers(inp)
+    keep = [A.block_weights(l) for l in layers]
+    x1, x2 = dev(inp.x), dev(inp.x)
+    A.dsv4v_tower_forward(cfg, b, keep, None, x1, ws)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(3 * len(A.PROFILE_KINDS) * 2)]
+    for e in events:
+        e.record()
+    A.dsv4v_tower_forward_profiled(cfg, b, keep, None, x2, ws, events)
+    torch.cuda.synchronize()
+    assert torch.equal(x1, x2)
+    for i in range(0, len(events), 2):
+        assert events[i].elapsed_time(events[i + 1]) > 0.0
+
+
 def test_workload4_tower_aligner(workload4):
     wl, inp, tower_o, align_o = workload4
     tower_g, align_g = run_tower_and_aligner(wl, inp)

@@ -193,8 +193,9 @@ Plans make_plans(const Shape& s, int sms) {
 }
 
 struct Layout {
-  size_t cos, sin, y, qkv, attn, h, partials, counters, asrc, merged, total;
+  size_t cos, sin, y, qkv, attn, h, partials, counters, asrc, merged, ss1, ss2, total;
   size_t counters_bytes;
+  int ss_parts;  // row stride of ss1 / ss2: the most N tiles a residual GEMM can have
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -227,6 +228,9 @@ Layout make_layout(const Shape& s, const Plans& pl) {
   l.counters_bytes = up256(static_cast<size_t>(counters) * sizeof(int));
   l.counters = take(l.counters_bytes);
   l.asrc = take(static_cast<size_t>(s.T) * s.r * s.r * 4);
+  l.ss_parts = s.D / 64 > 0 ? s.D / 64 : 1;
+  l.ss1 = take(s.bf16 ? static_cast<size_t>(s.P) * l.ss_parts * 4 : 0);
+  l.ss2 = take(s.bf16 ? static_cast<size_t>(s.P) * l.ss_parts * 4 : 0);
   l.merged = take(s.bf16 ? 0 : static_cast<size_t>(s.T) * s.r * s.r * s.D * 4);
   l.total = off;
   return l;
@@ -271,17 +275,31 @@ dsv4v_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSV4V_OK : D
   } while (0)
 
 // ---------------------------------------------------------------------------- bf16 steps
+// Folded-RMSNorm operands of one GEMM launch (see GemmArgs); all NULL / 0 = none.
+struct NormFold {
+  const float* ss = nullptr;  // consumer: partial sums of x^2 per row, `parts` of them at row stride `stride`
+  int parts = 0;
+  int stride = 0;
+  void* xw_out = nullptr;     // producer: bf16(x * w) and its partial sums of x^2
+  const float* xw_w = nullptr;
+  float* ss_out = nullptr;
+  int ss_parts = 0;
+};
+
 dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* a, int64_t M, int K, const void* b,
                        const void* b2, int n_out, void* out, const void* resid, const float* cos = nullptr,
                        const float* sin = nullptr, bool gather = false, const int32_t* gsrc = nullptr,
-                       const void* gx = nullptr) {
+                       const void* gx = nullptr, const NormFold& nf = NormFold()) {
   if (M == 0) return DSV4V_OK;
   const int box_b = epi == EPI_SWIGLU ? plan.bn / 2 : plan.bn;
-  CUtensorMap ta, tb, tb2;
+  CUtensorMap ta, tb, tb2, t_out, t_xw;
   if ((!gather && !bf16_map(a, M, K, 128, &ta)) || !bf16_map(b, n_out, K, box_b, &tb) ||
-      (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)))
+      (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)) || !bf16_map(out, M, n_out, 32, &t_out) ||
+      (nf.xw_out && !bf16_map(nf.xw_out, M, n_out, 32, &t_xw)))
     return DSV4V_ERR_CUDA;
   GemmArgs g{};
+  g.tm_out = &t_out;
+  g.tm_xw = nf.xw_out ? &t_xw : nullptr;
   g.tm_a = gather ? nullptr : &ta;
   g.tm_b = &tb;
   g.tm_b2 = epi == EPI_SWIGLU ? &tb2 : nullptr;
@@ -301,6 +319,15 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.partials = c.at<float>(c.lay.partials);
   g.counters = c.at<int>(c.lay.counters);
   g.err = c.dev.err;
+  g.norm_ss = nf.ss;
+  g.norm_parts = nf.parts;
+  g.norm_stride = nf.stride;
+  g.norm_inv_d = 1.0f / static_cast<float>(c.s.D);
+  g.norm_eps = c.eps;
+  g.xw_out = nf.xw_out;
+  g.xw_w = nf.xw_w;
+  g.ss_out = nf.ss_out;
+  g.ss_parts = nf.ss_parts;
   return cuda_status(launch_gemm_tc(epi, gather, plan, g, c.stream));
 }
 
@@ -330,22 +357,77 @@ dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv,
   return cuda_status(launch_attention_tc(&tm, sched, c.s.H, c.s.D, out, c.dev.err, c.stream));
 }
 
+// One block on the bf16 path.  The two RMSNorms are folded into the GEMMs that consume them:
+// the residual epilogue before each norm also writes xw = bf16(x * w) and the row partial sums
+// of x^2, and the consuming GEMM (QKV, SwiGLU) reads xw and scales its rows by
+// 1/sqrt(mean(x^2) + eps).  The first norm of a block with no residual GEMM before it comes from
+// k_norm_prep.  next_norm_w: the norm1 weight of the following block, so that this block's last
+// epilogue prepares it (NULL for the last block).
+dsv4v_status record(void* const* ev, int kind, int which, cudaStream_t s) {
+  if (!ev || !ev[kind * 2 + which]) return DSV4V_OK;
+  cudaEvent_t e = static_cast<cudaEvent_t>(ev[kind * 2 + which]);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return DSV4V_ERR_CUDA;
+  // Inside a stream capture an external record becomes an event-record node of the graph.
+  return cuda_status(cap == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(e, s, cudaEventRecordExternal)
+                                                          : cudaEventRecord(e, s));
+}
+
 dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_weights* w, const float* cos,
-                        const float* sin, void* x) {
+                        const float* sin, void* x, bool first, const float* next_norm_w,
+                        void* const* ev = nullptr) {
   const Shape& s = c.s;
-  void* y = c.at<void>(c.lay.y);
+  void* xw = c.at<void>(c.lay.y);
   void* qkv = c.at<void>(c.lay.qkv);
   void* attn = c.at<void>(c.lay.attn);
   void* h = c.at<void>(c.lay.h);
-  // The block's first kernel also clears the split-K tile counters of its GEMMs.
-  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm1_w, y, s.P, s.D, c.eps, c.stream, c.at<int>(c.lay.counters),
-                                       static_cast<int>(c.lay.counters_bytes / sizeof(int)))));
-  DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, y, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr, cos, sin));
+  float* ss1 = c.at<float>(c.lay.ss1);
+  float* ss2 = c.at<float>(c.lay.ss2);
+  if (first) {
+    // The block's first kernel also clears the split-tile counters of its GEMMs.
+    DSV4V_TRY(cuda_status(launch_norm_prep(x, w->norm1_w, xw, ss1, c.lay.ss_parts, s.P, s.D, c.stream,
+                                           c.at<int>(c.lay.counters),
+                                           static_cast<int>(c.lay.counters_bytes / sizeof(int)))));
+  }
+  NormFold q;
+  q.ss = ss1;
+  q.parts = first ? 1 : c.plans.down.tiles_n;  // the prep kernel puts the whole row sum in slot 0
+  q.stride = c.lay.ss_parts;
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_QKV, 0, c.stream));
+  DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, xw, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr,
+                              cos, sin, false, nullptr, nullptr, q));
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_QKV, 1, c.stream));
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_ATTENTION, 0, c.stream));
   DSV4V_TRY(attention_bf16(c, b, qkv, attn));
-  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x));
-  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm2_w, y, s.P, s.D, c.eps, c.stream)));
-  DSV4V_TRY(gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, y, s.P, s.D, w->w_gate, w->w_up, s.F, h, nullptr));
-  return gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x);
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_ATTENTION, 1, c.stream));
+  NormFold o;
+  o.xw_out = xw;
+  o.xw_w = w->norm2_w;
+  o.ss_out = ss2;
+  o.ss_parts = c.lay.ss_parts;
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_OUT, 0, c.stream));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x, nullptr, nullptr,
+                              false, nullptr, nullptr, o));
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_OUT, 1, c.stream));
+  NormFold m;
+  m.ss = ss2;
+  m.parts = c.plans.out.tiles_n;
+  m.stride = c.lay.ss_parts;
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_SWIGLU, 0, c.stream));
+  DSV4V_TRY(gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, xw, s.P, s.D, w->w_gate, w->w_up, s.F, h, nullptr,
+                              nullptr, nullptr, false, nullptr, nullptr, m));
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_SWIGLU, 1, c.stream));
+  NormFold d;
+  if (next_norm_w) {
+    d.xw_out = xw;
+    d.xw_w = next_norm_w;
+    d.ss_out = ss1;
+    d.ss_parts = c.lay.ss_parts;
+  }
+  DSV4V_TRY(record(ev, DSV4V_PROFILE_DOWN, 0, c.stream));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x, nullptr, nullptr,
+                      false, nullptr, nullptr, d));
+  return record(ev, DSV4V_PROFILE_DOWN, 1, c.stream);
 }
 
 // ---------------------------------------------------------------------------- fp32 steps
@@ -455,12 +537,13 @@ dsv4v_status dsv4v_block_forward(const dsv4v_config* cfg, const dsv4v_batch* bat
   DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
   if (!weights_ok(w) || !cos || !sin || !x_inout || !aligned16(x_inout) || !aligned16(cos) || !aligned16(sin))
     return DSV4V_ERR_INVALID_ARG;
-  return c.s.bf16 ? block_bf16(c, batch, w, cos, sin, x_inout) : block_f32(c, batch, w, cos, sin, x_inout);
+  return c.s.bf16 ? block_bf16(c, batch, w, cos, sin, x_inout, true, nullptr)
+                   : block_f32(c, batch, w, cos, sin, x_inout);
 }
 
-dsv4v_status dsv4v_tower_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const dsv4v_block_weights* layers,
-                                 const float* final_norm_w, void* x_inout, void* workspace, size_t ws_bytes,
-                                 void* stream) {
+static dsv4v_status tower_impl(const dsv4v_config* cfg, const dsv4v_batch* batch, const dsv4v_block_weights* layers,
+                               const float* final_norm_w, void* x_inout, void* workspace, size_t ws_bytes,
+                               void* stream, void* const* events) {
   Ctx c;
   DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
   if (!x_inout || !aligned16(x_inout) || (c.s.L > 0 && !layers)) return DSV4V_ERR_INVALID_ARG;
@@ -471,11 +554,26 @@ dsv4v_status dsv4v_tower_forward(const dsv4v_config* cfg, const dsv4v_batch* bat
   float* sin = c.at<float>(c.lay.sin);
   DSV4V_TRY(rope_table(c, batch, cos, sin));
   for (int l = 0; l < c.s.L; ++l)
-    DSV4V_TRY(c.s.bf16 ? block_bf16(c, batch, &layers[l], cos, sin, x_inout)
+    DSV4V_TRY(c.s.bf16 ? block_bf16(c, batch, &layers[l], cos, sin, x_inout, l == 0,
+                                    l + 1 < c.s.L ? layers[l + 1].norm1_w : nullptr,
+                                    events ? events + static_cast<size_t>(l) * DSV4V_PROFILE_KINDS * 2 : nullptr)
                        : block_f32(c, batch, &layers[l], cos, sin, x_inout));
   if (final_norm_w)
     DSV4V_TRY(cuda_status(launch_rmsnorm(c.s.bf16, x_inout, final_norm_w, x_inout, c.s.P, c.s.D, c.eps, c.stream)));
   return DSV4V_OK;
+}
+
+dsv4v_status dsv4v_tower_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const dsv4v_block_weights* layers,
+                                 const float* final_norm_w, void* x_inout, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  return tower_impl(cfg, batch, layers, final_norm_w, x_inout, workspace, ws_bytes, stream, nullptr);
+}
+
+dsv4v_status dsv4v_tower_forward_profiled(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                          const dsv4v_block_weights* layers, const float* final_norm_w,
+                                          void* x_inout, void* workspace, size_t ws_bytes, void* stream,
+                                          void* const* events) {
+  return tower_impl(cfg, batch, layers, final_norm_w, x_inout, workspace, ws_bytes, stream, events);
 }
 
 dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x,

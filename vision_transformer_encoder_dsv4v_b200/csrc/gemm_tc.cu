@@ -22,6 +22,7 @@
 // The accumulator is double-buffered in TMEM so the epilogue of one segment overlaps the MMAs
 // of the next.
 #include <algorithm>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "internal.h"
@@ -32,17 +33,20 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kSmemBudget = 225 * 1024;
+constexpr int kMaxDynSmem = 232448;         // 227 KB per CTA
+constexpr int kStagingBytes = 4 * 2 * 4096;  // per epilogue warp: two 32-row x 128-byte staging boxes
 
 template <int BN>
 struct TileCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (kSmemBudget - 2048) / STAGE;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int RING_BUDGET = kMaxDynSmem - 1024 - 512 - kStagingBytes;
+  static constexpr int STAGES = RING_BUDGET / STAGE > 8 ? 8 : RING_BUDGET / STAGE;
   static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : ((2 * BN <= 256) ? 256 : 512);
-  static constexpr int SMEM = 1024 + STAGES * STAGE + 512;
+  static constexpr int OFF_STAGING = STAGES * STAGE;
+  static constexpr int OFF_BARRIERS = OFF_STAGING + kStagingBytes;
+  static constexpr int SMEM = 1024 + OFF_BARRIERS + 512;
 };
 
 struct Params {
@@ -61,6 +65,13 @@ struct Params {
   float* partials;  // [G][BN / 4][128][4] fp32: a contributor's partial of a split tile
   int* counters;    // [tiles], zero between launches
   uint32_t* err;
+  const float* norm_ss;  // folded RMSNorm, consumer side (see GemmArgs)
+  int norm_parts, norm_stride;
+  float norm_inv_d, norm_eps;
+  __nv_bfloat16* xw_out;  // folded RMSNorm, producer side
+  const float* xw_w;
+  float* ss_out;
+  int ss_parts;
 };
 
 // ---------------------------------------------------------------------------- stream-K ranges
@@ -112,16 +123,63 @@ __device__ __forceinline__ float silu(float z) {
   return z * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * z));
 }
 
-// Epilogue of one 64-column accumulator group held in v[0..63] for output row `row`.
+// Output staging of one epilogue warp: two boxes of 32 rows x 128 bytes (64 bf16 columns) in
+// the 128-byte-swizzled layout of the output tensor maps; lane i owns row i of a box.  Each box
+// is written to global memory by one TMA store; a box is reused only after the store issued
+// from it two stores ago has finished reading it.
+struct Stager {
+  uint8_t* base;
+  int lane, n;
+  __device__ __forceinline__ uint8_t* acquire() {
+    if (lane == 0 && n >= 2) bulk_wait_read_1();
+    __syncwarp();
+    return base + (n & 1) * 4096;
+  }
+  // Both boxes, once no earlier store still reads either.
+  __device__ __forceinline__ void acquire_both(uint8_t*& b0, uint8_t*& b1) {
+    if (lane == 0 && n >= 1) bulk_wait_read_0();
+    __syncwarp();
+    b0 = base + (n & 1) * 4096;
+    b1 = base + ((n + 1) & 1) * 4096;
+  }
+  // 16-byte chunk j (0..7) of this lane's row.
+  __device__ __forceinline__ void put(uint8_t* box, int j, uint4 v) {
+    *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+  }
+  // Stores the box to rows [y, y + 32) and columns [x, x + 64) of `map` (TMA clips rows past
+  // the end of the tensor; a box entirely past it is skipped).
+  __device__ __forceinline__ void store(uint8_t* box, const CUtensorMap* map, int x, int y, int rows) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && y < rows) {
+      tma_store_2d(map, box, x, y);
+      bulk_commit();
+    }
+    ++n;
+  }
+  __device__ __forceinline__ void drain() {
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+};
+
+// Epilogue math of one 64-column accumulator group v[0..63] of output row `row`; the result
+// goes to the warp's staging box (the caller stores it).
 //   STORE/RESID/QKV: v = accumulator columns [64g, 64g + 64) -> output columns n0 + 64g + j.
-//   SWIGLU: v[0..31] = gate columns, v[32..63] = up columns of output columns n0h + 32g + j.
+//   SWIGLU: v[0..31] = gate columns, v[32..63] = up columns of output columns n0h + 32g + j;
+//           written to chunks 4 (g & 1) .. 4 (g & 1) + 3 of the box.
+//   RESID with the next norm prepared: the second box receives bf16(x * w_next).
 template <int EPI, int BN, int NR>
 __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_tile, int g, float (&v)[64],
-                                               const float (&rot_c)[NR], const float (&rot_s)[NR]) {
+                                               const float (&rot_c)[NR], const float (&rot_s)[NR], float row_scale,
+                                               const uint4* resid, float& ss_acc, Stager& st, uint8_t* box,
+                                               uint8_t* box2) {
   if (row >= p.M) return;
+  if constexpr (EPI == EPI_SWIGLU || EPI == EPI_QKV_ROPE) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j) v[j] *= row_scale;
+  }
   if constexpr (EPI == EPI_SWIGLU) {
-    const int col = n_tile * (BN / 2) + g * 32;
-    uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ldo + col);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint4 o;
@@ -129,11 +187,11 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
       o.y = pack_bf16x2(silu(v[8 * q + 2]) * v[32 + 8 * q + 2], silu(v[8 * q + 3]) * v[32 + 8 * q + 3]);
       o.z = pack_bf16x2(silu(v[8 * q + 4]) * v[32 + 8 * q + 4], silu(v[8 * q + 5]) * v[32 + 8 * q + 5]);
       o.w = pack_bf16x2(silu(v[8 * q + 6]) * v[32 + 8 * q + 6], silu(v[8 * q + 7]) * v[32 + 8 * q + 7]);
-      dst[q] = o;
+      st.put(box, 4 * (g & 1) + q, o);
     }
   } else {
-    const int col = n_tile * BN + g * 64;
     if constexpr (EPI == EPI_QKV_ROPE) {
+      const int col = n_tile * BN + g * 64;
       if (col < p.rot_cols) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -144,10 +202,9 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
       }
     }
     if constexpr (EPI == EPI_RESID) {
-      const uint4* r4 = reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(row) * p.ldo + col);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const uint4 r = r4[q];
+        const uint4 r = resid[q];
         v[8 * q + 0] += bf16_lo(r.x);
         v[8 * q + 1] += bf16_hi(r.x);
         v[8 * q + 2] += bf16_lo(r.y);
@@ -158,17 +215,44 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
         v[8 * q + 7] += bf16_hi(r.w);
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ldo + col);
+    uint4 o[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      uint4 o;
-      o.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-      o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-      o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-      o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-      dst[q] = o;
+      o[q].x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+      o[q].y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+      o[q].z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+      o[q].w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+      st.put(box, q, o[q]);
+    }
+    if constexpr (EPI == EPI_RESID) {
+      if (p.xw_out) {
+        // Next RMSNorm's operand from the stored (bf16) x: bf16(x * w) and sum of x^2.
+        const float4* w4 = reinterpret_cast<const float4*>(p.xw_w + n_tile * BN + g * 64);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
+          const float x0 = bf16_lo(o[q].x), x1 = bf16_hi(o[q].x), x2 = bf16_lo(o[q].y), x3 = bf16_hi(o[q].y);
+          const float x4 = bf16_lo(o[q].z), x5 = bf16_hi(o[q].z), x6 = bf16_lo(o[q].w), x7 = bf16_hi(o[q].w);
+          ss_acc += ((x0 * x0 + x1 * x1) + (x2 * x2 + x3 * x3)) + ((x4 * x4 + x5 * x5) + (x6 * x6 + x7 * x7));
+          uint4 t;
+          t.x = pack_bf16x2(x0 * wa.x, x1 * wa.y);
+          t.y = pack_bf16x2(x2 * wa.z, x3 * wa.w);
+          t.z = pack_bf16x2(x4 * wb.x, x5 * wb.y);
+          t.w = pack_bf16x2(x6 * wb.z, x7 * wb.w);
+          st.put(box2, q, t);
+        }
+      }
     }
   }
+}
+
+// Folded-RMSNorm row scale of output row `row` (1 when the GEMM has no norm folded in).
+__device__ __forceinline__ float norm_row_scale(const Params& p, int row) {
+  if (!p.norm_ss) return 1.0f;
+  const float* s = p.norm_ss + static_cast<size_t>(min(row, p.M - 1)) * p.norm_stride;
+  float acc = 0.0f;
+  for (int i = 0; i < p.norm_parts; ++i) acc += s[i];
+  return 1.0f / sqrtf(acc * p.norm_inv_d + p.norm_eps);
 }
 
 // Accumulator chunks (32 columns each) that make up epilogue group g.
@@ -226,12 +310,13 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatil
 template <int BN, int EPI, bool GATHER>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-              const __grid_constant__ CUtensorMap tm_b2, const Params p) {
+              const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
+              const __grid_constant__ CUtensorMap tm_xw, const Params p) {
   using C = TileCfg<BN>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BARRIERS);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -260,6 +345,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     if (!GATHER) tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
     if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tm_b2);
+    tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -386,16 +472,25 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) belong to this warp
     const int row_in_tile = quad * 32 + lane;
     const int et = threadIdx.x - 64;
+    Stager st{smem + C::OFF_STAGING + (warp - 2) * 8192, lane, 0};
+    constexpr int NGROUPS = BN / 64;
     int acc = 0;
     uint32_t acc_phase = 0;
     grid_dependency_wait();
     SegmentWalker walk(p);
     Segment sg;
     while (walk.next(p, sg)) {
-      // The rotation table row of this thread's output row, fetched while the MMAs run.
+      const int row = sg.m_tile * BM + row_in_tile;
+      const int box_y = sg.m_tile * BM + quad * 32;
+      const bool finisher_or_full =
+          (sg.kb0 == 0 && sg.kb1 == p.kb_total) ||
+          static_cast<int>(blockIdx.x) == unit_owner(p, static_cast<long long>(sg.tile) * p.kb_total);
+      // Inputs of the epilogue math fetched while the MMAs run: the rotation table row and the
+      // residual row of this thread's output row, and the folded-norm row scale.
       float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
+      uint4 resid[EPI == EPI_RESID ? NGROUPS * 8 : 1];
       if constexpr (EPI == EPI_QKV_ROPE) {
-        const int prow = min(sg.m_tile * BM + row_in_tile, p.M - 1);
+        const int prow = min(row, p.M - 1);
         const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(prow) * 32);
         const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(prow) * 32);
 #pragma unroll
@@ -405,16 +500,62 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           rot_s[4 * q] = s.x; rot_s[4 * q + 1] = s.y; rot_s[4 * q + 2] = s.z; rot_s[4 * q + 3] = s.w;
         }
       }
+      if constexpr (EPI == EPI_RESID) {
+        if (finisher_or_full) {
+          const uint4* r4 =
+              reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(min(row, p.M - 1)) * p.ldo + sg.n_tile * BN);
+#pragma unroll
+          for (int q = 0; q < NGROUPS * 8; ++q) resid[q] = r4[q];
+        }
+      }
+      const float row_scale = norm_row_scale(p, row);
+      float ss_acc = 0.0f;
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
       // All four epilogue warps continue or stop together (TMEM loads are warp-collective and
       // the partial-tile path uses a named barrier).
       if (!named_barrier_and(2, 128, got)) break;
       tc_fence_after_sync();
-      const int row = sg.m_tile * BM + row_in_tile;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      if (sg.kb0 == 0 && sg.kb1 == p.kb_total) {
+      if (!finisher_or_full) {
+        // Contributor to a tile finished by another CTA: park the partial, release it, move on.
+        float* slot = partial_slot<BN>(p, blockIdx.x);
 #pragma unroll 1
-        for (int g = 0; g < BN / 64; ++g) {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_row + c * 32, r);
+          tmem_ld_wait(r);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(slot + ((c * 8 + q) * BM + row_in_tile) * 4) =
+                make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                            __uint_as_float(r[4 * q + 3]));
+        }
+        tc_fence_before_sync();
+        mbar_arrive(&tempty[acc]);
+        __threadfence();
+        named_barrier_sync(1, 128);
+        if (et == 0) atomicAdd(&p.counters[sg.tile], 1);
+      } else {
+        // Whole tile, or finisher of a split tile: wait for the other contributors (if any),
+        // add their partials in CTA order, run the epilogue math, stage and store.
+        const bool split = !(sg.kb0 == 0 && sg.kb1 == p.kb_total);
+        int c_first = 0, c_last = 0;
+        if (split) {
+          const long long u_first = static_cast<long long>(sg.tile) * p.kb_total;
+          c_first = unit_owner(p, u_first);
+          c_last = unit_owner(p, u_first + p.kb_total - 1);
+          if (et == 0) *ticket = wait_counter(&p.counters[sg.tile], c_last - c_first, abort_flag, p.err) ? 1 : 0;
+          named_barrier_sync(1, 128);
+          if (!*ticket) {
+            tc_fence_before_sync();
+            mbar_arrive(&tempty[acc]);
+            break;
+          }
+          __threadfence();
+        }
+        uint8_t* box = nullptr;
+#pragma unroll 1
+        for (int g = 0; g < NGROUPS; ++g) {
           int c0, c1;
           group_chunks<EPI, BN>(g, c0, c1);
           uint32_t r0[32], r1[32];
@@ -428,63 +569,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             v[j] = __uint_as_float(r0[j]);
             v[32 + j] = __uint_as_float(r1[j]);
           }
-          epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s);
-        }
-        tc_fence_before_sync();
-        mbar_arrive(&tempty[acc]);
-      } else {
-        const long long u_first = static_cast<long long>(sg.tile) * p.kb_total;
-        const int c_first = unit_owner(p, u_first);
-        const int c_last = unit_owner(p, u_first + p.kb_total - 1);
-        if (static_cast<int>(blockIdx.x) != c_first) {
-          // Contributor: park the partial, release it, move on.
-          float* slot = partial_slot<BN>(p, blockIdx.x);
-#pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(t_row + c * 32, r);
-            tmem_ld_wait(r);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              *reinterpret_cast<float4*>(slot + ((c * 8 + q) * BM + row_in_tile) * 4) =
-                  make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                              __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-          }
-          tc_fence_before_sync();
-          mbar_arrive(&tempty[acc]);
-          __threadfence();
-          named_barrier_sync(1, 128);
-          if (et == 0) atomicAdd(&p.counters[sg.tile], 1);
-        } else {
-          // Finisher: wait for the other contributors, add their partials (CTA order) to the
-          // accumulator and run the epilogue.
-          bool ready = true;
-          if (et == 0) {
-            ready = wait_counter(&p.counters[sg.tile], c_last - c_first, abort_flag, p.err);
-            *ticket = ready ? 1 : 0;
-          }
-          named_barrier_sync(1, 128);
-          if (!*ticket) {
-            tc_fence_before_sync();
-            mbar_arrive(&tempty[acc]);
-            break;
-          }
-          __threadfence();
-#pragma unroll 1
-          for (int g = 0; g < BN / 64; ++g) {
-            int c0, c1;
-            group_chunks<EPI, BN>(g, c0, c1);
-            uint32_t r0[32], r1[32];
-            tmem_ld32(t_row + c0 * 32, r0);
-            tmem_ld32(t_row + c1 * 32, r1);
-            tmem_ld_wait(r0);
-            tmem_ld_wait(r1);
-            float v[64];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              v[j] = __uint_as_float(r0[j]);
-              v[32 + j] = __uint_as_float(r1[j]);
-            }
+          if (split) {
 #pragma unroll 2
             for (int cc = c_first + 1; cc <= c_last; ++cc) {
               const float* src = partial_slot<BN>(p, cc);
@@ -506,18 +591,32 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                 v[32 + 4 * q + 3] += b[q].w;
               }
             }
-            epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s);
           }
-          tc_fence_before_sync();
-          mbar_arrive(&tempty[acc]);
-          if (et == 0) p.counters[sg.tile] = 0;  // ready for the next launch
+          uint8_t* box2 = nullptr;
+          if (EPI == EPI_RESID && p.xw_out) st.acquire_both(box, box2);
+          else if (EPI != EPI_SWIGLU || (g & 1) == 0) box = st.acquire();
+          epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s, row_scale,
+                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? g * 8 : 0) : nullptr, ss_acc, st,
+                                  box, box2);
+          if constexpr (EPI == EPI_SWIGLU) {
+            if ((g & 1) == 1 || g == NGROUPS - 1) st.store(box, &tm_out, sg.n_tile * (BN / 2) + (g >> 1) * 64, box_y, p.M);
+          } else {
+            st.store(box, &tm_out, sg.n_tile * BN + g * 64, box_y, p.M);
+            if (EPI == EPI_RESID && p.xw_out) st.store(box2, &tm_xw, sg.n_tile * BN + g * 64, box_y, p.M);
+          }
         }
+        tc_fence_before_sync();
+        mbar_arrive(&tempty[acc]);
+        if (EPI == EPI_RESID && p.xw_out && row < p.M)
+          p.ss_out[static_cast<size_t>(row) * p.ss_parts + sg.n_tile] = ss_acc;
+        if (split && et == 0) p.counters[sg.tile] = 0;  // ready for the next launch
       }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
       }
     }
+    st.drain();
   } else if constexpr (GATHER) {
     // ------------------------------------------------------------------ A-gather (aligner)
     const int r = threadIdx.x - 192;  // row of the A tile handled by this thread
@@ -604,19 +703,44 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.partials = a.partials;
   p.counters = a.counters;
   p.err = a.err;
+  p.norm_ss = a.norm_ss;
+  p.norm_parts = a.norm_parts;
+  p.norm_stride = a.norm_stride;
+  p.norm_inv_d = a.norm_inv_d;
+  p.norm_eps = a.norm_eps;
+  p.xw_out = static_cast<__nv_bfloat16*>(a.xw_out);
+  p.xw_w = a.xw_w;
+  p.ss_out = a.ss_out;
+  p.ss_parts = a.ss_parts;
   const CUtensorMap& ta = GATHER ? *a.tm_b : *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
-  return launch_pdl(kern, dim3(plan.grid), dim3(GATHER ? 320 : 192), C::SMEM, s, ta, *a.tm_b, tb2, p);
+  const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
+  return launch_pdl(kern, dim3(plan.grid), dim3(GATHER ? 320 : 192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
 }
 
+// Tile widths each epilogue supports (the planner only picks these).
 template <int EPI, bool GATHER>
 cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
-  switch (plan.bn) {
-    case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
-    case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
-    case 192: return launch_one<192, EPI, GATHER>(plan, a, s);
-    case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
-    default: return cudaErrorInvalidValue;
+  if constexpr (EPI == EPI_RESID) {
+    switch (plan.bn) {
+      case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
+      case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    switch (plan.bn) {
+      case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
+      case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    switch (plan.bn) {
+      case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
+      case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
+      case 192: return launch_one<192, EPI, GATHER>(plan, a, s);
+      case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
+      default: return cudaErrorInvalidValue;
+    }
   }
 }
 
@@ -652,7 +776,32 @@ double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_o
 
 }  // namespace
 
+GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms);
+
 GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms) {
+  // Plans depend only on the shape; each thread keeps the ones it has computed.
+  struct Key {
+    int epi, M, n_out, K, sms;
+    bool operator==(const Key& o) const {
+      return epi == o.epi && M == o.M && n_out == o.n_out && K == o.K && sms == o.sms;
+    }
+  };
+  struct KeyHash {
+    size_t operator()(const Key& k) const {
+      return (((static_cast<size_t>(k.M) * 1000003u + k.n_out) * 1000003u + k.K) * 31u + k.epi) * 1009u + k.sms;
+    }
+  };
+  thread_local std::unordered_map<Key, GemmPlan, KeyHash> cache;
+  const Key key{epi, M, n_out, K, num_sms};
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  if (cache.size() > 1024) cache.clear();
+  GemmPlan best = plan_gemm_uncached(epi, M, n_out, K, num_sms);
+  cache[key] = best;
+  return best;
+}
+
+GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms) {
   GemmPlan best{};
   double best_cost = 1e300;
   const int kb_total = K / BK;
@@ -660,6 +809,10 @@ GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms) {
   const int cands[4] = {256, 192, 128, 64};
   if (kb_total <= 0 || tiles_m <= 0 || num_sms <= 0) return best;
   for (int bn : cands) {
+    // Epilogue constraints: SwiGLU stores 64-column boxes of two 32-column groups (bn / 2 a
+    // multiple of 64); the residual epilogue keeps its residual row in registers (bn <= 128).
+    if (epi == EPI_SWIGLU && (bn / 2) % 64) continue;
+    if (epi == EPI_RESID && bn > 128) continue;
     const int n_cols_per_tile = (epi == EPI_SWIGLU) ? bn / 2 : bn;
     if (n_out % n_cols_per_tile) continue;
     const int tiles_n = n_out / n_cols_per_tile;
@@ -674,7 +827,7 @@ GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms) {
     for (int gi = 0; gi < n_grids; ++gi) {
       int contrib = 1;
       const double cost = plan_cost(bn, tiles, kb_total, grids[gi], &contrib);
-      if (contrib > 8) continue;  // keep the finisher's read-back short
+      if (contrib > 2) continue;  // more contributors leave straggling finishers (measured)
       if (cost < best_cost - 1e-9) {
         best_cost = cost;
         best.bn = bn;

@@ -28,6 +28,8 @@ struct GemmPlan {
 GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms);
 
 struct GemmArgs {
+  const CUtensorMap* tm_out;  // output [M, n_out] bf16, box 64 x 32 (TMA stores of the epilogue)
+  const CUtensorMap* tm_xw;   // RESID with the next norm prepared: xw_out [M, n_out], box 64 x 32
   const CUtensorMap* tm_a;    // A [M, K], box 64 x 128 (ignored when gathering A)
   const CUtensorMap* tm_b;    // B [n, K] (SWIGLU: w_gate), box 64 x bn (SWIGLU: bn / 2)
   const CUtensorMap* tm_b2;   // SWIGLU: w_up, box 64 x bn / 2
@@ -46,6 +48,19 @@ struct GemmArgs {
   float* partials;
   int* counters;
   uint32_t* err;
+  // RMSNorm folded into the GEMM (norm(x) W^T = r_p ((x * w) W^T), r_p = 1/sqrt(mean x_p^2 + eps)):
+  //  consumer side (QKV_ROPE, SWIGLU): A holds bf16(x * w); the epilogue scales row p by r_p,
+  //   computed from norm_ss[p * norm_stride + i], i < norm_parts (partial sums of x_p^2);
+  //   norm_ss == NULL: no scaling.
+  //  producer side (RESID): besides x, the epilogue writes xw_out = bf16(x * xw_w) and the
+  //   partial sums of x^2 of its columns to ss_out[p * ss_parts + n_tile]; xw_out == NULL: off.
+  const float* norm_ss;
+  int norm_parts, norm_stride;
+  float norm_inv_d, norm_eps;
+  void* xw_out;
+  const float* xw_w;
+  float* ss_out;
+  int ss_parts;
 };
 
 cudaError_t launch_gemm_tc(int epi, bool gather, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
@@ -78,6 +93,10 @@ cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev,
                                  int64_t n_tokens, int32_t* src_out, cudaStream_t s, int* zero_ptr = nullptr,
                                  int zero_n = 0);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
+// Norm operands of the first GEMM of a block: xw = bf16(x * w) and ss[p * parts] = sum_c x[p,c]^2
+// (the other parts of a row are zero-filled); also clears zero_n counters like the kernels above.
+cudaError_t launch_norm_prep(const void* x, const float* w, void* xw, float* ss, int parts, int64_t rows, int d,
+                             cudaStream_t s, int* zero_ptr = nullptr, int zero_n = 0);
 
 // ---------------------------------------------------------------------------- fp32 CUDA-core path
 cudaError_t launch_gemm_f32(int epi, const float* a, const float* b, const float* b2, float* out, const float* resid,

@@ -108,6 +108,38 @@ __global__ void k_rmsnorm(const void* x, const float* __restrict__ w, void* y,
   }
 }
 
+// First folded RMSNorm of a block (no residual GEMM precedes it): xw = bf16(x * w) and the row's
+// sum of squares in ss[p * parts] (the remaining parts zero).  One warp per row, bf16 rows.
+__global__ void k_norm_prep(const __nv_bfloat16* x, const float* __restrict__ w, __nv_bfloat16* xw, float* ss,
+                            int parts, int64_t rows, int d, int* zero_ptr, int zero_n) {
+  grid_dependency_wait();
+  launch_dependents();
+  zero_ints(zero_ptr, zero_n);
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * d);
+  uint4* yr = reinterpret_cast<uint4*>(xw + row * d);
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+  float acc = 0.0f;
+  for (int c = lane; c < d / 8; c += 32) {
+    const uint4 v = xr[c];
+    const float4 wa = w4[2 * c], wb = w4[2 * c + 1];
+    const float x0 = bf16_lo(v.x), x1 = bf16_hi(v.x), x2 = bf16_lo(v.y), x3 = bf16_hi(v.y);
+    const float x4 = bf16_lo(v.z), x5 = bf16_hi(v.z), x6 = bf16_lo(v.w), x7 = bf16_hi(v.w);
+    acc += ((x0 * x0 + x1 * x1) + (x2 * x2 + x3 * x3)) + ((x4 * x4 + x5 * x5) + (x6 * x6 + x7 * x7));
+    uint4 o;
+    o.x = pack_bf16x2(x0 * wa.x, x1 * wa.y);
+    o.y = pack_bf16x2(x2 * wa.z, x3 * wa.w);
+    o.z = pack_bf16x2(x4 * wb.x, x5 * wb.y);
+    o.w = pack_bf16x2(x6 * wb.z, x7 * wb.w);
+    yr[c] = o;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  for (int i = lane; i < parts; i += 32) ss[row * parts + i] = i == 0 ? acc : 0.0f;
+}
+
 // src[t * r^2 + a * r + b] = packed row of the patch at window position (a, b) of token t, or
 // -1 where the window reaches into the zero padding.  Token offsets are rebuilt in shared
 // memory from the grids (one prefix sum per block).
@@ -184,6 +216,15 @@ cudaError_t launch_rmsnorm(bool bf16, const void* x, const float* w, void* y, in
     return launch_pdl(k_rmsnorm<true>, dim3(blocks), dim3(warps * 32), 0, s, x, w, y, rows, d, eps, zero_ptr, zero_n);
   k_rmsnorm<false><<<blocks, warps * 32, 0, s>>>(x, w, y, rows, d, eps, zero_ptr, zero_n);
   return cudaGetLastError();
+}
+
+cudaError_t launch_norm_prep(const void* x, const float* w, void* xw, float* ss, int parts, int64_t rows, int d,
+                             cudaStream_t s, int* zero_ptr, int zero_n) {
+  if (rows == 0) return cudaSuccess;
+  const int warps = 8;
+  const unsigned blocks = static_cast<unsigned>((rows + warps - 1) / warps);
+  return launch_pdl(k_norm_prep, dim3(blocks), dim3(warps * 32), 0, s, static_cast<const __nv_bfloat16*>(x), w,
+                    static_cast<__nv_bfloat16*>(xw), ss, parts, rows, d, zero_ptr, zero_n);
 }
 
 cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int r,

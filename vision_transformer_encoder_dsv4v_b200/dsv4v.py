@@ -19,8 +19,11 @@ DSV4V_MAX_IMAGES = 1024
 STATUS = {0: "DSV4V_OK", 1: "DSV4V_ERR_INVALID_ARG", 2: "DSV4V_ERR_UNSUPPORTED", 3: "DSV4V_ERR_WORKSPACE",
           4: "DSV4V_ERR_CUDA", 5: "DSV4V_ERR_TIMEOUT"}
 
+PROFILE_KINDS = ("qkv", "attention", "out", "swiglu", "down")  # DSV4V_PROFILE_* order
+
 # Every symbol include/dsv4v.h declares.
 EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", "dsv4v_tower_forward",
+           "dsv4v_tower_forward_profiled",
            "dsv4v_aligner_forward", "dsv4v_aligner_tokens", "dsv4v_rmsnorm", "dsv4v_qkv_rope", "dsv4v_attention",
            "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
            "dsv4v_status_string")
@@ -67,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "dsv4v_rope2d_table": (I, [cfg, bat, P, P, P]),
             "dsv4v_block_forward": (I, [cfg, bat, bw, P, P, P, P, SZ, P]),
             "dsv4v_tower_forward": (I, [cfg, bat, bw, P, P, P, SZ, P]),
+            "dsv4v_tower_forward_profiled": (I, [cfg, bat, bw, P, P, P, SZ, P, P]),
             "dsv4v_aligner_forward": (I, [cfg, bat, P, P, P, P, P, SZ, P]),
             "dsv4v_rmsnorm": (I, [cfg, I64, P, P, P, P]),
             "dsv4v_qkv_rope": (I, [cfg, bat, P, P, P, P, P, P, SZ, P]),
@@ -156,6 +160,16 @@ def dsv4v_tower_forward(cfg, batch, layers, final_norm_w, x_inout, workspace, st
     _check(lib().dsv4v_tower_forward(ctypes.byref(cfg), ctypes.byref(batch.c), arr, _ptr(final_norm_w),
                                      _ptr(x_inout), _ptr(workspace), workspace.numel(), _stream(stream)),
            "dsv4v_tower_forward")
+
+
+def dsv4v_tower_forward_profiled(cfg, batch, layers, final_norm_w, x_inout, workspace, events, stream=None):
+    """events: sequence of n_layers * len(PROFILE_KINDS) * 2 torch.cuda.Event (or None), already
+    recorded once so that their CUDA handles exist; [(layer * kinds + kind) * 2 + 0/1]."""
+    arr = (BlockWeights * max(1, len(layers)))(*layers)
+    handles = (ctypes.c_void_p * len(events))(*[(e.cuda_event if e is not None else None) for e in events])
+    _check(lib().dsv4v_tower_forward_profiled(ctypes.byref(cfg), ctypes.byref(batch.c), arr, _ptr(final_norm_w),
+                                              _ptr(x_inout), _ptr(workspace), workspace.numel(), _stream(stream),
+                                              handles), "dsv4v_tower_forward_profiled")
 
 
 def dsv4v_aligner_forward(cfg, batch, x, w_align, out, workspace, cu_tokens_host=None, stream=None):
