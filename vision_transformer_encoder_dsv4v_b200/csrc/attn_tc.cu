@@ -12,7 +12,10 @@
 // Keys past the end of the image are masked; query rows past it are computed but not stored.
 //
 // Warp roles: warp 0 TMA producer (Q once, K/V rings), warp 1 TMEM owner + MMA issuer,
-// warps 2..5 softmax / output.
+// warps 2..9 softmax / output.  Warps w and w + 4 share the query rows of TMEM lane quadrant
+// w % 4: the first takes keys 0..63 of each S tile and output columns 0..31, the second keys
+// 64..127 and columns 32..63; they exchange row maxima (and at the end row sums) through shared
+// memory at a pair barrier.
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,8 +34,11 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + TILE_BYTES;
 constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
 constexpr int OFF_P = OFF_V + VS * TILE_BYTES;
-constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+constexpr int OFF_XCH = OFF_P + 2 * P_BYTES;  // [2 tiles][2 halves][128 rows] fp32 exchange
+constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 128 * 4;
 constexpr int SMEM_BYTES = 1024 + OFF_BAR + 512;
+constexpr int kSoftmaxWarps = 8;  // two per query row: one per 64-key half of each S tile
+constexpr int kThreads = 64 + kSoftmaxWarps * 32;
 constexpr int TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) PV0 [256,320) PV1 [320,384)
 
 struct Params {
@@ -73,7 +79,7 @@ __device__ __forceinline__ void find_item(const AttnSchedule& s, int item, int& 
   local = item - s.item_start[lo];
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ AttnSchedule sched,
               const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -116,9 +122,9 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&p_full[b], kSoftmaxWarps * 32);
       mbar_init(&pv_full[b], 1);
-      mbar_init(&pv_empty[b], 128);
+      mbar_init(&pv_empty[b], kSoftmaxWarps * 32);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -213,76 +219,77 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------------ softmax + output
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t pair_bar = 2 + quad;  // named barrier of warps (quad + 2 or quad + 6) and partner
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     uint8_t* p_smem = smem + OFF_P;
-    float o[HD];
+    float* xch = reinterpret_cast<float*>(smem + OFF_XCH);
+    float o[HD / 2];
 #pragma unroll
-    for (int c = 0; c < HD; ++c) o[c] = 0.0f;
+    for (int c = 0; c < HD / 2; ++c) o[c] = 0.0f;
     float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
     bool ok = true;
     grid_dependency_wait();
     auto accumulate_pv = [&](int j, float alpha) -> bool {
-      const bool got = mbar_wait(&pv_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
-      if (!named_barrier_and(1, 128, got)) return false;
+      bool got = mbar_wait(&pv_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
+      got = __all_sync(0xffffffffu, got);
+      if (!got) return false;
       tc_fence_after_sync();
-      uint32_t a[32], b[32];
-      const uint32_t t = t_lane + 256u + static_cast<uint32_t>((j & 1) * HD);
-      tmem_ld32(t, a);
-      tmem_ld32(t + 32, b);
+      uint32_t a[32];
+      tmem_ld32(t_lane + 256u + static_cast<uint32_t>((j & 1) * HD + half * 32), a);
       tmem_ld_wait(a);
-      tmem_ld_wait(b);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        o[c] = o[c] * alpha + __uint_as_float(a[c]);
-        o[32 + c] = o[32 + c] * alpha + __uint_as_float(b[c]);
-      }
+      for (int c = 0; c < 32; ++c) o[c] = o[c] * alpha + __uint_as_float(a[c]);
       tc_fence_before_sync();
       mbar_arrive(&pv_empty[j & 1]);
       return true;
     };
     for (int j = 0; j < n_kv; ++j) {
-      const bool got = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
-      if (!named_barrier_and(1, 128, got)) {
+      bool got = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
+      got = __all_sync(0xffffffffu, got);
+      uint32_t s[TK / 2];
+      float mx = -INFINITY;
+      if (got) {
+        tc_fence_after_sync();
+        const uint32_t ts = t_lane + static_cast<uint32_t>((j & 1) * TK + half * (TK / 2));
+        tmem_ld32(ts + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        const int valid = min(TK, len - j * TK) - half * (TK / 2);  // keys of this half inside the image
+        if (valid < TK / 2) {
+#pragma unroll
+          for (int c = 0; c < TK / 2; ++c)
+            if (c >= valid) s[c] = 0xFF800000u;  // -inf
+        }
+        // Row max over this half with eight independent chains.
+        float m8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m8[u] = __uint_as_float(s[u]);
+#pragma unroll
+        for (int c = 8; c < TK / 2; c += 8)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], __uint_as_float(s[c + u]));
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      }
+      float* xm = xch + (j & 1) * 256;  // double-buffered by tile parity
+      xm[half * 128 + r] = mx;
+      if (!named_barrier_and(pair_bar, 64, got)) {
         ok = false;
         break;
       }
-      tc_fence_after_sync();
-      uint32_t s[TK];
-      const uint32_t ts = t_lane + static_cast<uint32_t>((j & 1) * TK);
-      tmem_ld32(ts + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld32(ts + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld32(ts + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-      tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-      const int valid = min(TK, len - j * TK);
-      if (valid < TK) {  // last tile of the image: keys past its end get -inf
-#pragma unroll
-        for (int c = 0; c < TK; ++c)
-          if (c >= valid) s[c] = 0xFF800000u;
-      }
-      // Row max with eight independent chains.
-      float m8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) m8[u] = __uint_as_float(s[u]);
-#pragma unroll
-      for (int c = 8; c < TK; c += 8)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], __uint_as_float(s[c + u]));
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      mx = fmaxf(mx, xm[(1 - half) * 128 + r]);
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
       const float alpha = ex2_mufu(m_run - m_new);
       const float neg_m = -m_new;
       float l8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) l8[u] = 0.0f;
-      uint8_t* prow = p_smem + (j & 1) * P_BYTES + r * 128;
+      // This half's 64 keys are swizzle atom `half` of the P row.
+      uint8_t* prow = p_smem + (j & 1) * P_BYTES + half * (TQ * 128) + r * 128;
 #pragma unroll
-      for (int c16 = 0; c16 < TK / 8; ++c16) {
+      for (int c16 = 0; c16 < TK / 16; ++c16) {
         float e[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -295,8 +302,7 @@ __global__ void __launch_bounds__(192, 1)
         pk.y = pack_bf16x2(e[2], e[3]);
         pk.z = pack_bf16x2(e[4], e[5]);
         pk.w = pack_bf16x2(e[6], e[7]);
-        const int atom = c16 >> 3, chunk = c16 & 7;
-        *reinterpret_cast<uint4*>(prow + atom * (TQ * 128) + ((chunk ^ (r & 7)) << 4)) = pk;
+        *reinterpret_cast<uint4*>(prow + ((c16 ^ (r & 7)) << 4)) = pk;
       }
       const float sum = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
       l_run = l_run * alpha + sum;
@@ -311,12 +317,18 @@ __global__ void __launch_bounds__(192, 1)
       alpha_prev = alpha;
     }
     if (ok && n_kv > 0) ok = accumulate_pv(n_kv - 1, alpha_prev);
+    // Row sum = sum of the two halves' sums (both are relative to the same running max).
+    float* xl = xch + 512 - 256;  // reuse the exchange of tile parity 1 (its readers have passed)
+    named_barrier_sync(pair_bar, 64);
+    xl[half * 128 + r] = l_run;
+    named_barrier_sync(pair_bar, 64);
+    const float l_total = l_run + xl[(1 - half) * 128 + r];
     const int qi = q_tile * TQ + r;
     if (ok && qi < len) {
-      const float inv_l = 1.0f / l_run;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + qi) * p.vision_dim + head * HD);
+      const float inv_l = 1.0f / l_total;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + qi) * p.vision_dim + head * HD + half * 32);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 4; ++q) {
         uint4 v;
         v.x = pack_bf16x2(o[8 * q + 0] * inv_l, o[8 * q + 1] * inv_l);
         v.y = pack_bf16x2(o[8 * q + 2] * inv_l, o[8 * q + 3] * inv_l);
@@ -355,7 +367,7 @@ cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& s
   p.scale_log2 = 1.4426950408889634f / 8.0f;  // log2(e) / sqrt(64)
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = err;
-  return launch_pdl(k_attn_tc, dim3(sched.n_items), dim3(192), SMEM_BYTES, s, *tm_qkv, sched, p);
+  return launch_pdl(k_attn_tc, dim3(sched.n_items), dim3(kThreads), SMEM_BYTES, s, *tm_qkv, sched, p);
 }
 
 }  // namespace dsv4v
