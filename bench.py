@@ -31,6 +31,13 @@ sys.path.insert(0, ROOT)
 from vision_transformer_encoder_dsv4v_b200 import synth  # noqa: E402
 
 METRIC = "ViT tower patches/sec and TFLOP/s (bf16, 1 B200) vs dense bf16 roofline"
+
+# DRAM bytes per launch of each kernel class, from one ncu launch-list capture of the benchmark
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels as they are now; an entry is
+# removed when its kernel changes.
+TRAFFIC_BYTES = {
+    (4, "down"): 11.84e6, (4, "swiglu"): 13.24e6, (4, "qkv"): 8.20e6, (4, "out"): 5.37e6, (4, "attention"): 4.86e6,
+}
 UNIT = "patches/s"
 
 
@@ -311,8 +318,10 @@ def run_ours(args):
     peaks = load_peaks()
     dom = kern["dominant"]
     peak = peaks.get("bf16_tflops_sustained") or 1400.0
+    traffic = TRAFFIC_BYTES.get((args.workload, dom["name"]))
     roof = {"bound": "tensor", "kernel": dom["name"], "achieved": dom["tflops"], "peak": peak, "unit": "TFLOP/s",
-            "frac": dom["tflops"] / peak, "traffic": None,
+            "frac": dom["tflops"] / peak, "traffic": traffic,
+            "traffic_unit": "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, ncu)",
             "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained (of measured)" if peaks else "fallback 1.4 PF",
             "step_tflops": tflops, "step_frac": tflops / peak}
 
