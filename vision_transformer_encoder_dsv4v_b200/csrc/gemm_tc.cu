@@ -118,9 +118,11 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// silu(z) = z / (1 + e^-z), from the MUFU exponential and reciprocal (ample for a bf16 result).
+// silu(z) = z / (1 + e^-z) = (z / 2) (1 + tanh(z / 2)): one MUFU op per element, ample for a bf16
+// result.
 __device__ __forceinline__ float silu(float z) {
-  return z * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * z));
+  const float h = 0.5f * z;
+  return fmaf(h, tanh_approx(h), h);
 }
 
 // Output staging of one epilogue warp: two boxes of 32 rows x 128 bytes (64 bf16 columns) in
@@ -499,6 +501,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           rot_c[4 * q] = c.x; rot_c[4 * q + 1] = c.y; rot_c[4 * q + 2] = c.z; rot_c[4 * q + 3] = c.w;
           rot_s[4 * q] = s.x; rot_s[4 * q + 1] = s.y; rot_s[4 * q + 2] = s.z; rot_s[4 * q + 3] = s.w;
         }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          pin(rot_c[j]);
+          pin(rot_s[j]);
+        }
       }
       if constexpr (EPI == EPI_RESID) {
         if (finisher_or_full) {
@@ -506,9 +513,12 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
               reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(min(row, p.M - 1)) * p.ldo + sg.n_tile * BN);
 #pragma unroll
           for (int q = 0; q < NGROUPS * 8; ++q) resid[q] = r4[q];
+#pragma unroll
+          for (int q = 0; q < NGROUPS * 8; ++q) pin(resid[q]);
         }
       }
-      const float row_scale = norm_row_scale(p, row);
+      float row_scale = norm_row_scale(p, row);
+      pin(row_scale);
       float ss_acc = 0.0f;
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
       // All four epilogue warps continue or stop together (TMEM loads are warp-collective and
@@ -554,7 +564,8 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           __threadfence();
         }
         uint8_t* box = nullptr;
-#pragma unroll 1
+        // Unrolled for the residual epilogue so that its prefetched residual row stays in registers.
+#pragma unroll(EPI == EPI_RESID ? NGROUPS : 1)
         for (int g = 0; g < NGROUPS; ++g) {
           int c0, c1;
           group_chunks<EPI, BN>(g, c0, c1);
