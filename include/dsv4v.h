@@ -207,6 +207,22 @@ dsv4v_status dsv4v_swiglu(const dsv4v_config* cfg, int64_t rows, const void* y,
                           const void* w_gate, const void* w_up, void* h, void* workspace,
                           size_t ws_bytes, void* stream);
 
+/* x <- x + a . w^T exactly as dsv4v_linear_residual (bf16 configs only), for callers that
+ * cannot allocate device memory: code that runs where cudaMalloc is not allowed (inside a
+ * global-mode stream capture, on a fixed memory budget handed out at start-up, behind an
+ * allocator that cannot serve library scratch).  It takes no workspace and allocates nothing:
+ * the GEMM's split-tile scratch is a static device array of this library (10 MiB of partials
+ * and 16384 tile counters, held by every GPU that loads the library until the process exits).
+ * rows <= DSV4V_NOALLOC_MAX_ROWS; a larger call, or one whose GEMM plan needs more scratch than
+ * the array holds, returns DSV4V_ERR_UNSUPPORTED without launching anything.  The first call on
+ * a device looks the array's device address up (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  All calls on a device share the one array and each starts by
+ * clearing its counters on `stream`: calls that overlap on the GPU (different streams, no
+ * ordering) race on it.  The pages describe no counterpart of this call. */
+#define DSV4V_NOALLOC_MAX_ROWS 65536
+dsv4v_status dsv4v_linear_residual_noalloc(const dsv4v_config* cfg, int64_t rows, int k,
+                                           const void* a, const void* w, void* x, void* stream);
+
 /* Synchronises `stream` and returns DSV4V_ERR_TIMEOUT if a kernel of this library recorded a
  * bounded-wait timeout on the current device since the last call (and clears the record),
  * DSV4V_ERR_CUDA if the stream reports an error, else DSV4V_OK. */

@@ -491,6 +491,38 @@ dsv4v_status prepare_rows(const dsv4v_config* cfg, int64_t rows, void* workspace
 }
 
 }  // namespace
+
+// Residual GEMM x <- x + a . w^T on the bf16 path with split-tile scratch supplied by the caller
+// (partials: partial_cap bytes, counters: counter_cap ints, zero on entry).  Used by the entry
+// point whose scratch is a static device array.
+dsv4v_status linear_residual_with_scratch(const dsv4v_config* cfg, int64_t rows, int k, const void* a,
+                                          const void* w, void* x, float* partials, size_t partial_cap,
+                                          int* counters, int counter_cap, void* stream) {
+  Ctx c;
+  DSV4V_TRY(check_config(cfg, c.s));
+  if (!c.s.bf16) return DSV4V_ERR_UNSUPPORTED;
+  if (rows < 0 || rows > (1ll << 30) || !a || !w || !x || !aligned16(a) || !aligned16(w) || !aligned16(x))
+    return DSV4V_ERR_INVALID_ARG;
+  if (k != c.s.D && k != c.s.F) return DSV4V_ERR_INVALID_ARG;
+  if (rows == 0) return DSV4V_OK;
+  if (!device_info(c.dev)) return DSV4V_ERR_CUDA;
+  const GemmPlan plan = plan_gemm(EPI_RESID, static_cast<int>(rows), c.s.D, k, c.dev.sms);
+  if (plan.bn == 0) return DSV4V_ERR_UNSUPPORTED;
+  if (plan.partial_bytes > partial_cap || static_cast<size_t>(plan.counters) > static_cast<size_t>(counter_cap))
+    return DSV4V_ERR_UNSUPPORTED;
+  c.s.P = rows;
+  c.s.T = 0;
+  c.eps = cfg->eps;
+  c.theta = cfg->rope_theta;
+  c.stream = static_cast<cudaStream_t>(stream);
+  // gemm_bf16 addresses scratch as offsets from c.ws: point it at the partials, counters follow.
+  c.ws = reinterpret_cast<uint8_t*>(partials);
+  c.lay = Layout{};
+  c.lay.partials = 0;
+  c.lay.counters = static_cast<size_t>(reinterpret_cast<uint8_t*>(counters) - reinterpret_cast<uint8_t*>(partials));
+  return gemm_bf16(c, EPI_RESID, plan, a, rows, k, w, nullptr, c.s.D, x, x);
+}
+
 }  // namespace dsv4v
 
 using namespace dsv4v;

@@ -26,7 +26,9 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_tower_forward_profiled",
            "dsv4v_aligner_forward", "dsv4v_aligner_tokens", "dsv4v_rmsnorm", "dsv4v_qkv_rope", "dsv4v_attention",
            "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
-           "dsv4v_status_string")
+           "dsv4v_status_string", "dsv4v_linear_residual_noalloc")
+
+DSV4V_NOALLOC_MAX_ROWS = 65536
 
 
 class Dsv4vError(RuntimeError):
@@ -77,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "dsv4v_attention": (I, [cfg, bat, P, P, P]),
             "dsv4v_linear_residual": (I, [cfg, I64, I, P, P, P, P, SZ, P]),
             "dsv4v_swiglu": (I, [cfg, I64, P, P, P, P, P, SZ, P]),
+            "dsv4v_linear_residual_noalloc": (I, [cfg, I64, I, P, P, P, P]),
             "dsv4v_device_error": (I, [P]),
             "dsv4v_selftest_bounded_wait": (I, [U64, P]),
             "dsv4v_status_string": (ctypes.c_char_p, [I]),
@@ -199,6 +202,13 @@ def dsv4v_linear_residual(cfg, rows, k, a, w, x, workspace, stream=None):
     _check(lib().dsv4v_linear_residual(ctypes.byref(cfg), rows, k, _ptr(a), _ptr(w), _ptr(x), _ptr(workspace),
                                        workspace.numel() if workspace is not None else 0, _stream(stream)),
            "dsv4v_linear_residual")
+
+
+def dsv4v_linear_residual_noalloc(cfg, rows, k, a, w, x, stream=None):
+    """x <- x + a . w^T with no workspace: for callers that cannot allocate device memory (the
+    library's own static scratch is used; see include/dsv4v.h)."""
+    _check(lib().dsv4v_linear_residual_noalloc(ctypes.byref(cfg), rows, k, _ptr(a), _ptr(w), _ptr(x), _stream(stream)),
+           "dsv4v_linear_residual_noalloc")
 
 
 def dsv4v_swiglu(cfg, rows, y, w_gate, w_up, h, workspace, stream=None):
