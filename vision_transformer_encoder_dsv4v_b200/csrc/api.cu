@@ -8,7 +8,7 @@
 #include <unordered_map>
 #include <vector>
 
-#include "../../include/dsv4v.h"
+#include "dsv4v.h"
 #include "common.cuh"
 #include "internal.h"
 

@@ -68,6 +68,49 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return x < -125.0f ? 0.0f : r;
 }
 
+// Packed pairs of fp32 (one 64-bit register pair) for the sm_100 f32x2 arithmetic.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ex2_poly on two elements at once with packed arithmetic (same reduction and cubic).
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t xc = pk2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t magic = pk2(12582912.0f, 12582912.0f);
+  const uint64_t t = add2(xc, magic);
+  const uint64_t f = sub2(xc, sub2(t, magic));
+  uint64_t q = fma2(pk2(0.0551716573536396f, 0.0551716573536396f), f, pk2(0.2426111400127411f, 0.2426111400127411f));
+  q = fma2(q, f, pk2(0.6932609677314758f, 0.6932609677314758f));
+  q = fma2(q, f, pk2(0.9999280571937561f, 0.9999280571937561f));
+  float t0, t1, q0, q1;
+  upk2(t, t0, t1);
+  upk2(q, q0, q1);
+  const unsigned n0 = static_cast<unsigned>(__float_as_int(t0) - 0x4B400000);
+  const unsigned n1 = static_cast<unsigned>(__float_as_int(t1) - 0x4B400000);
+  y0 = x0 < -125.0f ? 0.0f : __int_as_float(__float_as_int(q0) + static_cast<int>(n0 << 23));
+  y1 = x1 < -125.0f ? 0.0f : __int_as_float(__float_as_int(q1) + static_cast<int>(n1 << 23));
+}
+
 __device__ __forceinline__ void find_item(const AttnSchedule& s, int item, int& img, int& local) {
   int lo = 0, hi = s.n_images - 1;
   while (lo < hi) {
@@ -239,8 +282,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t a[32];
       tmem_ld32(t_lane + 256u + static_cast<uint32_t>((j & 1) * HD + half * 32), a);
       tmem_ld_wait(a);
+      const uint64_t al2 = pk2(alpha, alpha);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) o[c] = o[c] * alpha + __uint_as_float(a[c]);
+      for (int c = 0; c < 32; c += 2) {
+        const uint64_t r2 = fma2(pk2(o[c], o[c + 1]), al2, pk2(__uint_as_float(a[c]), __uint_as_float(a[c + 1])));
+        upk2(r2, o[c], o[c + 1]);
+      }
       tc_fence_before_sync();
       mbar_arrive(&pv_empty[j & 1]);
       return true;
@@ -283,19 +330,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
       const float alpha = ex2_mufu(m_run - m_new);
       const float neg_m = -m_new;
-      float l8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) l8[u] = 0.0f;
-      // This half's 64 keys are swizzle atom `half` of the P row.
+      // This half's 64 keys are swizzle atom `half` of the P row.  One exponential pair in four
+      // runs on the FMA pipe, interleaved with the MUFU ones so that both pipes stay busy; the
+      // scale-subtract, the row sum and the cubic use packed f32x2 arithmetic.
       uint8_t* prow = p_smem + (j & 1) * P_BYTES + half * (TQ * 128) + r * 128;
+      const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(neg_m, neg_m);
+      uint64_t l2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c16 = 0; c16 < TK / 16; ++c16) {
         float e[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float x = fmaf(__uint_as_float(s[c16 * 8 + u]), p.scale_log2, neg_m);
-          e[u] = (u >= 6) ? ex2_poly(x) : ex2_mufu(x);
-          l8[u] += e[u];
+        for (int u = 0; u < 8; u += 2) {
+          float x0, x1;
+          upk2(fma2(pk2(__uint_as_float(s[c16 * 8 + u]), __uint_as_float(s[c16 * 8 + u + 1])), sc2, nm2), x0, x1);
+          if (u == 6) {
+            ex2_poly2(x0, x1, e[u], e[u + 1]);
+          } else {
+            e[u] = ex2_mufu(x0);
+            e[u + 1] = ex2_mufu(x1);
+          }
+          l2[u >> 1] = add2(l2[u >> 1], pk2(e[u], e[u + 1]));
         }
         uint4 pk;
         pk.x = pack_bf16x2(e[0], e[1]);
@@ -304,7 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk.w = pack_bf16x2(e[6], e[7]);
         *reinterpret_cast<uint4*>(prow + ((c16 ^ (r & 7)) << 4)) = pk;
       }
-      const float sum = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      float la, lb, lc, ld, le, lf, lg, lh;
+      upk2(l2[0], la, lb);
+      upk2(l2[1], lc, ld);
+      upk2(l2[2], le, lf);
+      upk2(l2[3], lg, lh);
+      const float sum = ((la + lb) + (lc + ld)) + ((le + lf) + (lg + lh));
       l_run = l_run * alpha + sum;
       m_run = m_new;
       fence_proxy_async_smem();  // generic-proxy P stores -> visible to the tensor core

@@ -4,7 +4,7 @@
 // instead, so the caller passes only its inputs and outputs.
 #include <mutex>
 
-#include "../../include/dsv4v.h"
+#include "dsv4v.h"
 #include "internal.h"
 
 namespace dsv4v {
