@@ -343,6 +343,14 @@ dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv,
     return b->cu_patches_host[x + 1] - b->cu_patches_host[x] > b->cu_patches_host[y + 1] - b->cu_patches_host[y];
   });
   sched.n_images = n;
+  // Two query tiles per CTA halve the K/V traffic and keep two softmax warps on every SM
+  // sub-partition; one per CTA when pairing would leave SMs idle.
+  int paired = 0;
+  for (int i = 0; i < n; ++i) {
+    const int len = b->cu_patches_host[i + 1] - b->cu_patches_host[i];
+    paired += ((len + 255) / 256) * c.s.H;
+  }
+  sched.pair = paired >= c.dev.sms ? 2 : 1;
   int items = 0;
   for (int k = 0; k < n; ++k) {
     const int i = order[k];
@@ -350,7 +358,8 @@ dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv,
     sched.item_start[k] = items;
     sched.img_row0[k] = b->cu_patches_host[i];
     sched.img_len[k] = len;
-    items += ((len + 127) / 128) * c.s.H;
+    const int qt = (len + 127) / 128;
+    items += ((qt + sched.pair - 1) / sched.pair) * c.s.H;
   }
   sched.item_start[n] = items;
   sched.n_items = items;

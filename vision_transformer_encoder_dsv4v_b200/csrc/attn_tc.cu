@@ -1,21 +1,29 @@
 // Varlen full (bidirectional) attention on tcgen05, head_dim 64.
 //
-// One CTA per work item (image, 128-query tile, head); items are scheduled longest image
-// first.  For each 128-key tile j of the image:
-//   S_j = Q K_j^T          tcgen05.mma M=128 N=128 K=64, fp32 into TMEM (two S buffers)
-//   P_j = exp2(S_j * log2(e)/sqrt(hd) - m_j)   softmax warps, one query row per thread, written
-//                          to smem as bf16 in the 128-byte-swizzled K-major layout
-//   PV_j = P_j V_j         tcgen05.mma M=128 N=64 K=128 (V read MN-major straight from the
-//                          natural [keys, hd] tile), fp32 into TMEM (two PV buffers)
-//   O = O * exp2(m_{j-1} - m_j) + PV_j     in registers, one tile behind, so the tensor core
-//                          computes S_{j+1} and PV_j while the softmax warps work on S_j.
+// One CTA per work item (image, one or two 128-query tiles A and B, head); items are scheduled
+// longest image first.  Both query tiles of an item share every K/V tile that the producer
+// loads.  For each 128-key tile j of the image and each query tile X of the item:
+//   S_X = Q_X K_j^T            tcgen05.mma M=128 N=128 K=64, fp32 into TMEM
+//   P_X = exp2(S_X c - m_X)    softmax warpgroup X, one query row per thread, written back to
+//                             TMEM as bf16 (two keys per 32-bit column)
+//   O_X += P_X V_j             tcgen05.mma M=128 N=64 K=128, A (= P) read from TMEM, V read
+//                             MN-major from the natural [keys, hd] smem tile; O_X stays in TMEM
+//                             for the whole key loop
+// The row max m_X is raised lazily: only when a row's running max exceeds m_X by more than
+// kRescaleLog2 (log2 units) are m_X, that row of O_X and its sum rescaled.  Otherwise the stale
+// max is kept, which bounds P by 2^kRescaleLog2 and changes nothing but rounding.
 // Keys past the end of the image are masked; query rows past it are computed but not stored.
 //
-// Warp roles: warp 0 TMA producer (Q once, K/V rings), warp 1 TMEM owner + MMA issuer,
-// warps 2..9 softmax / output.  Warps w and w + 4 share the query rows of TMEM lane quadrant
-// w % 4: the first takes keys 0..63 of each S tile and output columns 0..31, the second keys
-// 64..127 and columns 32..63; they exchange row maxima (and at the end row sums) through shared
-// memory at a pair barrier.
+// Warp roles: warp 0 TMA producer (Q once, K/V rings), warp 1 TMEM owner + MMA issuer of tile A,
+// warp 2 MMA issuer of tile B, warp 3 idle, warps 4..7 softmax of tile A, warps 8..11 softmax of
+// tile B.  Warp w reads TMEM lanes
+// 32 (w % 4) .. +31, so every softmax thread owns one full query row of its tile (128 scores in
+// registers).  The first warpgroup gives registers to the softmax warpgroups (setmaxnreg:
+// 128 x 56 + 256 x 224 = 384 x 168, the launch's total).  The two softmax warpgroups share no
+// barrier and drift apart, so that one's MUFU work overlaps the other's FMA work on each SM
+// sub-partition.
+//
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384) P_A [384,448) P_B [448,512).
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,25 +32,37 @@ namespace dsv4v {
 namespace {
 
 constexpr int HD = 64;
-constexpr int TQ = 128;                // queries per CTA
+constexpr int TQ = 128;                // queries per tile
 constexpr int TK = 128;                // keys per tile
-constexpr int KS = 3;                  // K ring depth
-constexpr int VS = 3;                  // V ring depth
+constexpr int KS = 4;                  // K ring depth
+constexpr int VS = 4;                  // V ring depth
 constexpr int TILE_BYTES = TK * HD * 2;  // 16 KB (Q, K or V tile)
-constexpr int P_BYTES = TQ * TK * 2;     // 32 KB
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE_BYTES;
+constexpr int OFF_Q = 0;               // Q_A, Q_B
+constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
 constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
-constexpr int OFF_P = OFF_V + VS * TILE_BYTES;
-constexpr int OFF_XCH = OFF_P + 2 * P_BYTES;  // [2 tiles][2 halves][128 rows] fp32 exchange
-constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 128 * 4;
+constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
 constexpr int SMEM_BYTES = 1024 + OFF_BAR + 512;
-constexpr int kSoftmaxWarps = 8;  // two per query row: one per 64-key half of each S tile
-constexpr int kThreads = 64 + kSoftmaxWarps * 32;
-constexpr int TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) PV0 [256,320) PV1 [320,384)
+constexpr int kSoftmaxWarps = 8;
+constexpr int kFirstSoftmaxWarp = 4;
+constexpr int kRegsControl = 56;    // warpgroup 0 after setmaxnreg
+constexpr int kRegsSoftmax = 224;   // softmax warpgroups after setmaxnreg
+constexpr int kThreads = (kFirstSoftmaxWarp + kSoftmaxWarps) * 32;
+constexpr int TMEM_COLS = 512;
+constexpr uint32_t T_S = 0, T_O = 256, T_P = 384;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr int kPolyPerEight = 1;    // exponential pairs per eight computed on the FMA pipe
+
+// Which exponential pairs (index i = column / 2) use the FMA-pipe polynomial.
+__host__ __device__ constexpr bool poly_pair(int i) {
+  return kPolyPerEight == 2   ? (i & 3) == 3
+         : kPolyPerEight == 3 ? ((i & 7) == 2 || (i & 7) == 5 || (i & 7) == 7)
+         : kPolyPerEight == 4 ? (i & 1) == 1
+         : kPolyPerEight == 1 ? (i & 7) == 7
+                              : false;
+}
 
 struct Params {
-  int n_heads, vision_dim;
+  int n_heads, vision_dim, pair;
   float scale_log2;
   __nv_bfloat16* out;
   uint32_t* err;
@@ -50,23 +70,6 @@ struct Params {
 
 // 2^x on the MUFU pipe (flushes results below 2^-126 to zero).
 __device__ __forceinline__ float ex2_mufu(float x) { return ex2_approx(x); }
-
-// 2^x for x <= 0 on the FMA pipe, used for a quarter of the softmax exponentials so that the
-// MUFU pipe is not the only one doing them.  Range reduction x = n + f with n = round(x) (the
-// 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2]; 2^f by a cubic fitted here for minimum
-// relative error on that interval (max 7.5e-5, far below the bf16 rounding of P); 2^n is added
-// to the exponent field.  Inputs below -125 (masked keys included) return 0.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float xc = fmaxf(x, -125.0f);
-  const float t = xc + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = xc - n;
-  const float p = fmaf(fmaf(fmaf(0.0551716573536396f, f, 0.2426111400127411f), f, 0.6932609677314758f), f,
-                       0.9999280571937561f);
-  const int ni = __float_as_int(t) - 0x4B400000;
-  const float r = __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<unsigned>(ni) << 23));
-  return x < -125.0f ? 0.0f : r;
-}
 
 // Packed pairs of fp32 (one 64-bit register pair) for the sm_100 f32x2 arithmetic.
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -92,8 +95,22 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
-// ex2_poly on two elements at once with packed arithmetic (same reduction and cubic).
+// 2^x for two x <= 0 at once on the FMA pipe, used for one softmax exponential in eight so
+// that the MUFU pipe is not the only one doing them.  Range reduction x = n + f with
+// n = round(x) (the 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2]; 2^f by a cubic fitted here
+// for minimum relative error on that interval (max 7.5e-5, far below the bf16 rounding of P);
+// 2^n is added to the exponent field.  Inputs below -125 (masked keys included) return 0.
 __device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& y1) {
   const uint64_t xc = pk2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
   const uint64_t magic = pk2(12582912.0f, 12582912.0f);
@@ -109,6 +126,69 @@ __device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& 
   const unsigned n1 = static_cast<unsigned>(__float_as_int(t1) - 0x4B400000);
   y0 = x0 < -125.0f ? 0.0f : __int_as_float(__float_as_int(q0) + static_cast<int>(n0 << 23));
   y1 = x1 < -125.0f ? 0.0f : __int_as_float(__float_as_int(q1) + static_cast<int>(n1 << 23));
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], bf16 inputs, fp32 accumulate; A holds M rows in TMEM lanes
+// with two K elements per 32-bit column.  One thread issues.
+__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Starts loading N x 32 columns of this thread's lane (complete after tmem_ld_wait_pin).
+template <int N>
+__device__ __forceinline__ void tmem_ld_issue(uint32_t taddr, uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) tmem_ld32(taddr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * i));
+}
+
+// Waits for this thread's TMEM loads, then pins N x 32 registers so that no use of them can be
+// scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait_pin(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32 * N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+// Loads N x 32 columns of this thread's lane with one wait, then pins the registers so that no
+// use of them can be scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) tmem_ld32(taddr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * i));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32 * N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+template <int R>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 __device__ __forceinline__ void find_item(const AttnSchedule& s, int item, int& img, int& local) {
@@ -133,12 +213,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + KS;
   uint64_t* v_full = k_empty + KS;
   uint64_t* v_empty = v_full + VS;
-  uint64_t* s_full = v_empty + VS;   // [2]
-  uint64_t* p_full = s_full + 2;     // [2]
-  uint64_t* pv_full = p_full + 2;    // [2]
-  uint64_t* pv_empty = pv_full + 2;  // [2]
-  uint64_t* mma_done = pv_empty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* s_full = v_empty + VS;   // [tile]
+  uint64_t* s_free = s_full + 2;     // [tile]
+  uint64_t* p_full = s_free + 2;     // [tile]
+  uint64_t* pv_done = p_full + 2;    // [tile]
+  uint64_t* mma_done = pv_done + 2;  // [tile]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -148,8 +228,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   find_item(sched, blockIdx.x, img, local);
   const int row0 = sched.img_row0[img];
   const int len = sched.img_len[img];
-  const int q_tile = local / p.n_heads;
-  const int head = local - q_tile * p.n_heads;
+  const int n_qt = (len + TQ - 1) / TQ;
+  const int q_pair = local / p.n_heads;
+  const int head = local - q_pair * p.n_heads;
+  const int q_tile = q_pair * p.pair;
+  const int n_tiles = min(p.pair, n_qt - q_tile);  // 1 or 2 query tiles in this item
   const int n_kv = (len + TK - 1) / TK;
   const int q_row = row0 + q_tile * TQ;
 
@@ -157,19 +240,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+      mbar_init(&k_empty[s], n_tiles);
     }
     for (int s = 0; s < VS; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+      mbar_init(&v_empty[s], n_tiles);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], kSoftmaxWarps * 32);
-      mbar_init(&pv_full[b], 1);
-      mbar_init(&pv_empty[b], kSoftmaxWarps * 32);
+      mbar_init(&s_free[b], 128);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -185,13 +269,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) launch_dependents();
 
+  static_assert(kThreads == 384 && 128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * 168,
+                "register split exceeds the launch's register total");
+  if (warp < kFirstSoftmaxWarp) {
+    regs_dec<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       grid_dependency_wait();
       const int col_q = head * HD, col_k = p.vision_dim + head * HD, col_v = 2 * p.vision_dim + head * HD;
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      tma_load_2d(smem + OFF_Q, &tm_qkv, q_full, col_q, q_row);
+      mbar_arrive_expect_tx(q_full, n_tiles * TILE_BYTES);
+      for (int x = 0; x < n_tiles; ++x)
+        tma_load_2d(smem + OFF_Q + x * TILE_BYTES, &tm_qkv, q_full, col_q, q_row + x * TQ);
       int issued_k = 0, issued_v = 0;
       for (int t = 0; t < n_kv; ++t) {
         if (!mbar_wait(&k_empty[t % KS], ((t / KS) & 1) ^ 1, abort_flag, p.err, kErrTimeoutProducer)) break;
@@ -211,189 +300,193 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = (issued_v > VS ? issued_v - VS : 0); t < issued_v; ++t)
         mbar_wait(&v_full[t % VS], (t / VS) & 1, &never, p.err, kErrTimeoutProducer);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp - 1 < n_tiles) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Warp 1 issues the products of tile A, warp 2 those of tile B, so that neither waits for
+    // the other's softmax; the K/V slots are released by one commit from each.
     if (lane == 0) {
+      const int x = warp - 1;
       constexpr uint32_t idesc_s = idesc_bf16(TQ, TK, false);
       constexpr uint32_t idesc_pv = idesc_bf16(TQ, HD, true);  // V is MN-major (hd contiguous)
-      const uint32_t q_addr = smem_u32(smem + OFF_Q);
-      const uint32_t p_addr = smem_u32(smem + OFF_P);
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.err, kErrTimeoutMma);
-      tc_fence_after_sync();
-      auto issue_s = [&](int j) -> bool {
-        if (!mbar_wait(&k_full[j % KS], (j / KS) & 1, abort_flag, p.err, kErrTimeoutMma)) return false;
-        tc_fence_after_sync();
-        const uint32_t k_addr = smem_u32(smem + OFF_K + (j % KS) * TILE_BYTES);
-        const uint64_t qd = sdesc_sw128(q_addr, 16, 1024);
-        const uint64_t kd = sdesc_sw128(k_addr, 16, 1024);
-        const uint32_t d = tmem_base + static_cast<uint32_t>((j & 1) * TK);
+      const uint64_t qd = sdesc_sw128(smem_u32(smem + OFF_Q + x * TILE_BYTES), 16, 1024);
+      const uint32_t d_s = tmem_base + T_S + static_cast<uint32_t>(x * TK);
+      const uint32_t d_o = tmem_base + T_O + static_cast<uint32_t>(x * HD);
+      const uint32_t a_p = tmem_base + T_P + static_cast<uint32_t>(x * (TK / 2));
+      auto issue_s = [&](int j) {
+        const uint64_t kd = sdesc_sw128(smem_u32(smem + OFF_K + (j % KS) * TILE_BYTES), 16, 1024);
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) umma_bf16(d, qd + 2 * k, kd + 2 * k, idesc_s, k > 0 ? 1u : 0u);
+        for (int k = 0; k < HD / 16; ++k) umma_bf16(d_s, qd + 2 * k, kd + 2 * k, idesc_s, k > 0 ? 1u : 0u);
+        umma_commit(&s_full[x]);
         umma_commit(&k_empty[j % KS]);
-        umma_commit(&s_full[j & 1]);
-        return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && n_kv > 1) ok = issue_s(1);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutMma)) break;
-        if (j >= 2 && !mbar_wait(&pv_empty[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.err, kErrTimeoutMma)) break;
-        if (!mbar_wait(&v_full[j % VS], (j / VS) & 1, abort_flag, p.err, kErrTimeoutMma)) break;
-        tc_fence_after_sync();
+      auto issue_pv = [&](int j) {
         const uint32_t v_addr = smem_u32(smem + OFF_V + (j % VS) * TILE_BYTES);
-        const uint32_t pj = p_addr + (j & 1) * P_BYTES;
-        const uint32_t d = tmem_base + 256u + static_cast<uint32_t>((j & 1) * HD);
 #pragma unroll
         for (int kk = 0; kk < TK / 16; ++kk) {
-          // P: two 64-key swizzle atoms of 16 KB; V: 16 keys = two 8-row groups of 1024 B.
-          const uint64_t pd = sdesc_sw128(pj + (kk >> 2) * (TQ * 128) + (kk & 3) * 32, 16, 1024);
+          // P: 16 keys = 8 TMEM columns; V: 16 keys = two 8-row groups of 1024 B.
           const uint64_t vd = sdesc_sw128(v_addr + kk * 2048, TILE_BYTES, 1024);
-          umma_bf16(d, pd, vd, idesc_pv, kk > 0 ? 1u : 0u);
+          umma_bf16_tmem_a(d_o, a_p + kk * 8, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
+        umma_commit(&pv_done[x]);
         umma_commit(&v_empty[j % VS]);
-        umma_commit(&pv_full[j & 1]);
-        if (j + 2 < n_kv) ok = issue_s(j + 2);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.err, kErrTimeoutMma);
+      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, p.err, kErrTimeoutMma);
+      if (ok) {
+        tc_fence_after_sync();
+        issue_s(0);
       }
-      umma_commit(mma_done);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv) {
+          // S(j+1) as soon as the softmax has S(j) in registers.
+          const int t = j + 1;
+          ok = mbar_wait(&k_full[t % KS], (t / KS) & 1, abort_flag, p.err, kErrTimeoutMma) &&
+               mbar_wait(&s_free[x], j & 1, abort_flag, p.err, kErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_s(t);
+        }
+        ok = mbar_wait(&v_full[j % VS], (j / VS) & 1, abort_flag, p.err, kErrTimeoutMma) &&
+             mbar_wait(&p_full[x], j & 1, abort_flag, p.err, kErrTimeoutMma);
+        if (!ok) break;
+        tc_fence_after_sync();
+        issue_pv(j);
+      }
+      umma_commit(&mma_done[x]);
       volatile int never = 0;
-      mbar_wait(mma_done, 0, &never, p.err, kErrTimeoutMma);
+      mbar_wait(&mma_done[x], 0, &never, p.err, kErrTimeoutMma);
     }
     __syncwarp();
-  } else {
+  }
+  } else if (regs_inc<kRegsSoftmax>(), (warp - kFirstSoftmaxWarp) / 4 < n_tiles) {
     // ------------------------------------------------------------------ softmax + output
+    const int x = (warp - kFirstSoftmaxWarp) >> 2;  // query tile of this warpgroup
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;  // query row within the tile = TMEM lane
-    const uint32_t pair_bar = 2 + quad;  // named barrier of warps (quad + 2 or quad + 6) and partner
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    uint8_t* p_smem = smem + OFF_P;
-    float* xch = reinterpret_cast<float*>(smem + OFF_XCH);
-    float o[HD / 2];
-#pragma unroll
-    for (int c = 0; c < HD / 2; ++c) o[c] = 0.0f;
-    float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
+    const uint32_t t_s = t_lane + T_S + static_cast<uint32_t>(x * TK);
+    const uint32_t t_o = t_lane + T_O + static_cast<uint32_t>(x * HD);
+    const uint32_t t_p = t_lane + T_P + static_cast<uint32_t>(x * (TK / 2));
+    float m_used = -INFINITY, l_run = 0.0f;
     bool ok = true;
     grid_dependency_wait();
-    auto accumulate_pv = [&](int j, float alpha) -> bool {
-      bool got = mbar_wait(&pv_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
-      got = __all_sync(0xffffffffu, got);
-      if (!got) return false;
-      tc_fence_after_sync();
-      uint32_t a[32];
-      tmem_ld32(t_lane + 256u + static_cast<uint32_t>((j & 1) * HD + half * 32), a);
-      tmem_ld_wait(a);
-      const uint64_t al2 = pk2(alpha, alpha);
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const uint64_t r2 = fma2(pk2(o[c], o[c + 1]), al2, pk2(__uint_as_float(a[c]), __uint_as_float(a[c + 1])));
-        upk2(r2, o[c], o[c + 1]);
-      }
-      tc_fence_before_sync();
-      mbar_arrive(&pv_empty[j & 1]);
-      return true;
-    };
     for (int j = 0; j < n_kv; ++j) {
-      bool got = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
-      got = __all_sync(0xffffffffu, got);
-      uint32_t s[TK / 2];
-      float mx = -INFINITY;
-      if (got) {
-        tc_fence_after_sync();
-        const uint32_t ts = t_lane + static_cast<uint32_t>((j & 1) * TK + half * (TK / 2));
-        tmem_ld32(ts + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld_wait(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        const int valid = min(TK, len - j * TK) - half * (TK / 2);  // keys of this half inside the image
-        if (valid < TK / 2) {
-#pragma unroll
-          for (int c = 0; c < TK / 2; ++c)
-            if (c >= valid) s[c] = 0xFF800000u;  // -inf
-        }
-        // Row max over this half with eight independent chains.
-        float m8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) m8[u] = __uint_as_float(s[u]);
-#pragma unroll
-        for (int c = 8; c < TK / 2; c += 8)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], __uint_as_float(s[c + u]));
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      }
-      float* xm = xch + (j & 1) * 256;  // double-buffered by tile parity
-      xm[half * 128 + r] = mx;
-      if (!named_barrier_and(pair_bar, 64, got)) {
+      bool got = mbar_wait(&s_full[x], j & 1, abort_flag, p.err, kErrTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
-      mx = fmaxf(mx, xm[(1 - half) * 128 + r]);
-      const float m_new = fmaxf(m_run, mx * p.scale_log2);
-      const float alpha = ex2_mufu(m_run - m_new);
-      const float neg_m = -m_new;
-      // This half's 64 keys are swizzle atom `half` of the P row.  One exponential pair in four
-      // runs on the FMA pipe, interleaved with the MUFU ones so that both pipes stay busy; the
-      // scale-subtract, the row sum and the cubic use packed f32x2 arithmetic.
-      uint8_t* prow = p_smem + (j & 1) * P_BYTES + half * (TQ * 128) + r * 128;
-      const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(neg_m, neg_m);
+      tc_fence_after_sync();
+      // Columns 0..63 first; 64..127 load while the first half's max is taken.
+      uint32_t s[TK];
+      tmem_ld_cols<2>(t_s, s);
+      tmem_ld_issue<2>(t_s + 64, s + 64);
+      const int valid = len - j * TK;
+      if (valid < TK / 2) {
+#pragma unroll
+        for (int c = 0; c < TK / 2; ++c)
+          if (c >= valid) s[c] = 0xFF800000u;  // -inf
+      }
+      // Row max with eight independent chains of three-input max.
+      float m8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) m8[u] = fmaxf(__uint_as_float(s[u]), __uint_as_float(s[8 + u]));
+#pragma unroll
+      for (int c = 16; c < TK / 2; c += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m8[u] = max3(m8[u], __uint_as_float(s[c + u]), __uint_as_float(s[c + 8 + u]));
+      tmem_ld_wait_pin<2>(s + 64);
+      tc_fence_before_sync();
+      mbar_arrive(&s_free[x]);  // S is in registers: the next S may overwrite it
+      if (valid < TK) {
+#pragma unroll
+        for (int c = TK / 2; c < TK; ++c)
+          if (c >= valid) s[c] = 0xFF800000u;
+      }
+#pragma unroll
+      for (int c = TK / 2; c < TK; c += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m8[u] = max3(m8[u], __uint_as_float(s[c + u]), __uint_as_float(s[c + 8 + u]));
+      const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+      const float m_cand = mx * p.scale_log2;
+      const bool raise = m_cand > m_used + kRescaleLog2;
+      const float m_new = raise ? m_cand : m_used;
+      const float alpha = raise ? ex2_mufu(m_used - m_new) : 1.0f;  // 0 on the first tile
+      m_used = m_new;
+      if (j > 0) {
+        // P_X and O_X are free once the previous P_X V product has completed.
+        got = mbar_wait(&pv_done[x], (j - 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        if (__any_sync(0xffffffffu, raise)) {
+          uint32_t o[HD];
+          tmem_ld_cols<HD / 32>(t_o, o);
+          const uint64_t al2 = pk2(alpha, alpha);
+#pragma unroll
+          for (int c = 0; c < HD; c += 2) {
+            float a0, a1;
+            upk2(mul2(pk2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), al2), a0, a1);
+            o[c] = __float_as_uint(a0);
+            o[c + 1] = __float_as_uint(a1);
+          }
+          tmem_st32(t_o, o);
+          tmem_st32(t_o + 32, o + 32);
+        }
+      }
+      // P = 2^(s c - m), some exponential pairs on the FMA pipe interleaved with the MUFU ones;
+      // the bf16 pairs are packed in place into s[0 .. TK/2) and each half of P goes to TMEM
+      // as soon as it is complete.
+      const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(-m_new, -m_new);
       uint64_t l2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c16 = 0; c16 < TK / 16; ++c16) {
-        float e[8];
-#pragma unroll
-        for (int u = 0; u < 8; u += 2) {
-          float x0, x1;
-          upk2(fma2(pk2(__uint_as_float(s[c16 * 8 + u]), __uint_as_float(s[c16 * 8 + u + 1])), sc2, nm2), x0, x1);
-          if (u == 6) {
-            ex2_poly2(x0, x1, e[u], e[u + 1]);
-          } else {
-            e[u] = ex2_mufu(x0);
-            e[u + 1] = ex2_mufu(x1);
-          }
-          l2[u >> 1] = add2(l2[u >> 1], pk2(e[u], e[u + 1]));
+      for (int c = 0; c < TK; c += 2) {
+        float x0, x1, e0, e1;
+        upk2(fma2(pk2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2), x0, x1);
+        if (poly_pair(c >> 1)) {
+          ex2_poly2(x0, x1, e0, e1);
+        } else {
+          e0 = ex2_mufu(x0);
+          e1 = ex2_mufu(x1);
         }
-        uint4 pk;
-        pk.x = pack_bf16x2(e[0], e[1]);
-        pk.y = pack_bf16x2(e[2], e[3]);
-        pk.z = pack_bf16x2(e[4], e[5]);
-        pk.w = pack_bf16x2(e[6], e[7]);
-        *reinterpret_cast<uint4*>(prow + ((c16 ^ (r & 7)) << 4)) = pk;
+        l2[(c >> 1) & 3] = add2(l2[(c >> 1) & 3], pk2(e0, e1));
+        s[c >> 1] = pack_bf16x2(e0, e1);
+        if (c == TK / 2 - 2) tmem_st32(t_p, s);
       }
+      tmem_st32(t_p + 32, s + 32);
       float la, lb, lc, ld, le, lf, lg, lh;
       upk2(l2[0], la, lb);
       upk2(l2[1], lc, ld);
       upk2(l2[2], le, lf);
       upk2(l2[3], lg, lh);
-      const float sum = ((la + lb) + (lc + ld)) + ((le + lf) + (lg + lh));
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-      fence_proxy_async_smem();  // generic-proxy P stores -> visible to the tensor core
+      l_run = l_run * alpha + (((la + lb) + (lc + ld)) + ((le + lf) + (lg + lh)));
+      tmem_st_wait();
       tc_fence_before_sync();
-      mbar_arrive(&p_full[j & 1]);
-      if (j >= 1 && !accumulate_pv(j - 1, alpha_prev)) {
-        ok = false;
-        break;
-      }
-      alpha_prev = alpha;
+      mbar_arrive(&p_full[x]);
     }
-    if (ok && n_kv > 0) ok = accumulate_pv(n_kv - 1, alpha_prev);
-    // Row sum = sum of the two halves' sums (both are relative to the same running max).
-    float* xl = xch + 512 - 256;  // reuse the exchange of tile parity 1 (its readers have passed)
-    named_barrier_sync(pair_bar, 64);
-    xl[half * 128 + r] = l_run;
-    named_barrier_sync(pair_bar, 64);
-    const float l_total = l_run + xl[(1 - half) * 128 + r];
-    const int qi = q_tile * TQ + r;
-    if (ok && qi < len) {
-      const float inv_l = 1.0f / l_total;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + qi) * p.vision_dim + head * HD + half * 32);
+    if (ok && n_kv > 0) {
+      const bool got = mbar_wait(&pv_done[x], (n_kv - 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
+      ok = __all_sync(0xffffffffu, got);
+    }
+    if (ok) {
+      tc_fence_after_sync();
+      uint32_t o[HD];
+      tmem_ld_cols<HD / 32>(t_o, o);
+      const int qi = (q_tile + x) * TQ + r;
+      if (qi < len) {
+        const float inv_l = 1.0f / l_run;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + qi) * p.vision_dim + head * HD);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 v;
-        v.x = pack_bf16x2(o[8 * q + 0] * inv_l, o[8 * q + 1] * inv_l);
-        v.y = pack_bf16x2(o[8 * q + 2] * inv_l, o[8 * q + 3] * inv_l);
-        v.z = pack_bf16x2(o[8 * q + 4] * inv_l, o[8 * q + 5] * inv_l);
-        v.w = pack_bf16x2(o[8 * q + 6] * inv_l, o[8 * q + 7] * inv_l);
-        dst[q] = v;
+        for (int q = 0; q < HD / 8; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+          dst[q] = v;
+        }
       }
     }
   }
@@ -415,14 +508,22 @@ cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& s
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(attr_set_mask & (1ull << dev))) {
+    // setmaxnreg.inc waits until the block has the registers it asks for: refuse to launch if
+    // the build gave the kernel fewer registers per thread than the split assumes.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, k_attn_tc);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * kThreads < 128 * kRegsControl + 256 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set_mask |= 1ull << dev;
   }
   if (sched.n_items <= 0) return cudaSuccess;
+  if (sched.pair != 1 && sched.pair != 2) return cudaErrorInvalidValue;
   Params p;
   p.n_heads = n_heads;
   p.vision_dim = vision_dim;
+  p.pair = sched.pair;
   p.scale_log2 = 1.4426950408889634f / 8.0f;  // log2(e) / sqrt(64)
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = err;

@@ -490,7 +490,10 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       // Inputs of the epilogue math fetched while the MMAs run: the rotation table row and the
       // residual row of this thread's output row, and the folded-norm row scale.
       float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
-      uint4 resid[EPI == EPI_RESID ? NGROUPS * 8 : 1];
+      // The residual epilogue keeps RG groups (64 columns each) of the residual row in
+      // registers and refills a slot RG groups ahead once its group is done.
+      constexpr int RG = NGROUPS < 2 ? NGROUPS : 2;
+      uint4 resid[EPI == EPI_RESID ? RG * 8 : 1];
       if constexpr (EPI == EPI_QKV_ROPE) {
         const int prow = min(row, p.M - 1);
         const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(prow) * 32);
@@ -512,9 +515,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           const uint4* r4 =
               reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(min(row, p.M - 1)) * p.ldo + sg.n_tile * BN);
 #pragma unroll
-          for (int q = 0; q < NGROUPS * 8; ++q) resid[q] = r4[q];
+          for (int q = 0; q < RG * 8; ++q) resid[q] = r4[q];
 #pragma unroll
-          for (int q = 0; q < NGROUPS * 8; ++q) pin(resid[q]);
+          for (int q = 0; q < RG * 8; ++q) pin(resid[q]);
         }
       }
       float row_scale = norm_row_scale(p, row);
@@ -607,8 +610,16 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           if (EPI == EPI_RESID && p.xw_out) st.acquire_both(box, box2);
           else if (EPI != EPI_SWIGLU || (g & 1) == 0) box = st.acquire();
           epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s, row_scale,
-                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? g * 8 : 0) : nullptr, ss_acc, st,
-                                  box, box2);
+                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? (g % RG) * 8 : 0) : nullptr, ss_acc,
+                                  st, box, box2);
+          if constexpr (EPI == EPI_RESID) {
+            if (g + RG < NGROUPS) {
+              const uint4* r4 = reinterpret_cast<const uint4*>(
+                  p.resid + static_cast<size_t>(min(row, p.M - 1)) * p.ldo + sg.n_tile * BN + (g + RG) * 64);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) resid[(g % RG) * 8 + q] = r4[q];
+            }
+          }
           if constexpr (EPI == EPI_SWIGLU) {
             if ((g & 1) == 1 || g == NGROUPS - 1) st.store(box, &tm_out, sg.n_tile * (BN / 2) + (g >> 1) * 64, box_y, p.M);
           } else {
@@ -736,6 +747,7 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
     switch (plan.bn) {
       case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
       case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
+      case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
       default: return cudaErrorInvalidValue;
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
@@ -821,9 +833,9 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms) {
   if (kb_total <= 0 || tiles_m <= 0 || num_sms <= 0) return best;
   for (int bn : cands) {
     // Epilogue constraints: SwiGLU stores 64-column boxes of two 32-column groups (bn / 2 a
-    // multiple of 64); the residual epilogue keeps its residual row in registers (bn <= 128).
+    // multiple of 64); the residual epilogue is built for bn in {64, 128, 256}.
     if (epi == EPI_SWIGLU && (bn / 2) % 64) continue;
-    if (epi == EPI_RESID && bn > 128) continue;
+    if (epi == EPI_RESID && bn == 192) continue;
     const int n_cols_per_tile = (epi == EPI_SWIGLU) ? bn / 2 : bn;
     if (n_out % n_cols_per_tile) continue;
     const int tiles_n = n_out / n_cols_per_tile;

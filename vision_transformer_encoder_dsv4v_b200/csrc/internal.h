@@ -70,9 +70,12 @@ constexpr int kMaxImages = 1024;
 
 // Images in the order they are scheduled (longest first); item_start is the prefix sum of
 // (query tiles x heads) in that order.
+// Work items of the attention kernel: for each image (longest first) and head, its query tiles
+// in groups of `pair` (1 or 2) 128-row tiles that share the K/V stream.
 struct AttnSchedule {
   int n_images;
   int n_items;
+  int pair;
   int item_start[kMaxImages + 1];
   int img_row0[kMaxImages];
   int img_len[kMaxImages];
