@@ -291,7 +291,7 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
                        const float* sin = nullptr, bool gather = false, const int32_t* gsrc = nullptr,
                        const void* gx = nullptr, const NormFold& nf = NormFold()) {
   if (M == 0) return DSV4V_OK;
-  const int box_b = epi == EPI_SWIGLU ? plan.bn / 2 : plan.bn;
+  const int box_b = (epi == EPI_SWIGLU || plan.pair) ? plan.bn / 2 : plan.bn;
   CUtensorMap ta, tb, tb2, t_out, t_xw;
   if ((!gather && !bf16_map(a, M, K, 128, &ta)) || !bf16_map(b, n_out, K, box_b, &tb) ||
       (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)) || !bf16_map(out, M, n_out, 32, &t_out) ||
@@ -515,7 +515,7 @@ dsv4v_status linear_residual_with_scratch(const dsv4v_config* cfg, int64_t rows,
   if (k != c.s.D && k != c.s.F) return DSV4V_ERR_INVALID_ARG;
   if (rows == 0) return DSV4V_OK;
   if (!device_info(c.dev)) return DSV4V_ERR_CUDA;
-  const GemmPlan plan = plan_gemm(EPI_RESID, static_cast<int>(rows), c.s.D, k, c.dev.sms);
+  const GemmPlan plan = plan_gemm(EPI_RESID, static_cast<int>(rows), c.s.D, k, c.dev.sms, partial_cap);
   if (plan.bn == 0) return DSV4V_ERR_UNSUPPORTED;
   if (plan.partial_bytes > partial_cap || static_cast<size_t>(plan.counters) > static_cast<size_t>(counter_cap))
     return DSV4V_ERR_UNSUPPORTED;

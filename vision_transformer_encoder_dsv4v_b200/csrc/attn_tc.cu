@@ -491,6 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  __syncwarp();  // every warp reconverged (role code ran on single lanes) before the CTA barrier
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 1) {

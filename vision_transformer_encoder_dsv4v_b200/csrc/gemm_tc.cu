@@ -36,10 +36,13 @@ constexpr int BK = 64;
 constexpr int kMaxDynSmem = 232448;         // 227 KB per CTA
 constexpr int kStagingBytes = 4 * 2 * 4096;  // per epilogue warp: two 32-row x 128-byte staging boxes
 
-template <int BN>
+// PAIR: the CTA is one half of a CTA pair that computes a 256 x BN tile (tcgen05 cta_group::2):
+// it holds 128 rows of A and BN / 2 rows of B per stage, and 128 x BN accumulators.
+template <int BN, bool PAIR = false>
 struct TileCfg {
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int RING_BUDGET = kMaxDynSmem - 1024 - 512 - kStagingBytes;
   static constexpr int STAGES = RING_BUDGET / STAGE > 8 ? 8 : RING_BUDGET / STAGE;
@@ -52,6 +55,7 @@ struct TileCfg {
 struct Params {
   int M, K, n_out;
   int tiles_m, kb_total;
+  int owners;       // unit owners: CTAs, or CTA pairs
   long long units;  // tiles * kb_total
   __nv_bfloat16* out;
   int ldo;
@@ -75,12 +79,13 @@ struct Params {
 };
 
 // ---------------------------------------------------------------------------- stream-K ranges
+// Units are owned by CTAs, or by CTA pairs (owner c = CTAs 2c and 2c + 1).
 __device__ __forceinline__ long long range_begin(const Params& p, int c) {
-  return static_cast<long long>(c) * p.units / gridDim.x;
+  return static_cast<long long>(c) * p.units / p.owners;
 }
-// CTA owning unit u: the largest c with range_begin(c) <= u.
+// Owner of unit u: the largest c with range_begin(c) <= u.
 __device__ __forceinline__ int unit_owner(const Params& p, long long u) {
-  return static_cast<int>(((u + 1) * gridDim.x - 1) / p.units);
+  return static_cast<int>(((u + 1) * p.owners - 1) / p.units);
 }
 
 struct Segment {
@@ -88,13 +93,13 @@ struct Segment {
   bool first;  // first segment of this CTA's range
 };
 
-// Walks the segments of this CTA's unit range.
+// Walks the segments of one owner's unit range.
 struct SegmentWalker {
   long long u, u_end;
   bool first;
-  __device__ __forceinline__ explicit SegmentWalker(const Params& p) {
-    u = range_begin(p, blockIdx.x);
-    u_end = range_begin(p, blockIdx.x + 1);
+  __device__ __forceinline__ SegmentWalker(const Params& p, int owner) {
+    u = range_begin(p, owner);
+    u_end = range_begin(p, owner + 1);
     first = true;
   }
   __device__ __forceinline__ bool next(const Params& p, Segment& s) {
@@ -309,12 +314,14 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatil
   }
 }
 
-template <int BN, int EPI, bool GATHER>
+template <int BN, int EPI, bool GATHER, bool PAIR>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
               const __grid_constant__ CUtensorMap tm_xw, const Params p) {
-  using C = TileCfg<BN>;
+  static_assert(!(GATHER && PAIR), "the A-gather runs on single CTAs");
+  using C = TileCfg<BN, PAIR>;
+  constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -329,6 +336,10 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // In a pair, rank 0 (the leader) issues the MMAs; its full and tempty barriers gather both
+  // CTAs' loads and epilogue releases, the other barriers are signalled in both CTAs at once.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int owner = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], PAIR ? 256 : 128);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -350,13 +361,27 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers are initialised before any remote use
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_holder;
+  if constexpr (PAIR) {
+    // The leader's MMAs write the same TMEM columns in both CTAs.
+    if (threadIdx.x == 0 &&
+        ld_shared_cluster_u32(mapa_shared(smem_u32(const_cast<uint32_t*>(tmem_holder)), rank ^ 1u)) != tmem_base) {
+      atomicCAS(p.err, 0u, static_cast<uint32_t>(kErrPairTmem));
+      *abort_flag = 1;
+    }
+  }
   if (threadIdx.x == 0) launch_dependents();
 
   if (warp == 0) {
@@ -365,15 +390,32 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
       bool ok = true;
-      auto load_b = [&](uint8_t* sb, int kb, int n_tile, uint64_t* bar) {
-        if (EPI == EPI_SWIGLU) {
-          tma_load_2d(sb, &tm_b, bar, kb * BK, n_tile * (BN / 2));
-          tma_load_2d(sb + (BN / 2) * 128, &tm_b2, bar, kb * BK, n_tile * (BN / 2));
+      // Stage s of both CTAs of a pair completes on the leader's full[s].
+      const uint32_t full_leader = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
+      const bool arrives = !PAIR || rank == 0;  // posts the expected bytes of the stage
+      constexpr uint32_t kStageTx = GATHER ? C::B_BYTES : (PAIR ? 2 * C::STAGE : C::STAGE);
+      auto load_a = [&](uint8_t* sa, int kb, int m_tile, int s) {
+        if constexpr (PAIR)
+          tma_load_2d_pair(sa, &tm_a, full_leader + 8u * s, kb * BK, m_tile * BMT + static_cast<int>(rank) * BM);
+        else
+          tma_load_2d(sa, &tm_a, &full[s], kb * BK, m_tile * BM);
+      };
+      auto load_b = [&](uint8_t* sb, int kb, int n_tile, int s) {
+        if constexpr (PAIR) {
+          // The MMA's B is split along N: rank 0 holds rows [0, BN/2), rank 1 rows [BN/2, BN)
+          // (SwiGLU: the gate rows and the up rows).
+          if (EPI == EPI_SWIGLU)
+            tma_load_2d_pair(sb, rank == 0 ? &tm_b : &tm_b2, full_leader + 8u * s, kb * BK, n_tile * (BN / 2));
+          else
+            tma_load_2d_pair(sb, &tm_b, full_leader + 8u * s, kb * BK, n_tile * BN + static_cast<int>(rank) * (BN / 2));
+        } else if (EPI == EPI_SWIGLU) {
+          tma_load_2d(sb, &tm_b, &full[s], kb * BK, n_tile * (BN / 2));
+          tma_load_2d(sb + (BN / 2) * 128, &tm_b2, &full[s], kb * BK, n_tile * (BN / 2));
         } else {
-          tma_load_2d(sb, &tm_b, bar, kb * BK, n_tile * BN);
+          tma_load_2d(sb, &tm_b, &full[s], kb * BK, n_tile * BN);
         }
       };
-      SegmentWalker walk(p);
+      SegmentWalker walk(p, owner);
       Segment sg;
       // The weight tiles of the first stages do not depend on the previous kernel: start them
       // before waiting for it, then add the activation tiles.
@@ -383,15 +425,14 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       if (peek.next(p, first)) {
         pre = min(STAGES, first.kb1 - first.kb0);
         for (int i = 0; i < pre; ++i) {
-          mbar_arrive_expect_tx(&full[i], GATHER ? C::B_BYTES : C::STAGE);
-          load_b(smem + i * C::STAGE + C::A_BYTES, first.kb0 + i, first.n_tile, &full[i]);
+          if (arrives) mbar_arrive_expect_tx(&full[i], kStageTx);
+          load_b(smem + i * C::STAGE + C::A_BYTES, first.kb0 + i, first.n_tile, i);
           issued |= 1u << i;
         }
       }
       grid_dependency_wait();
       if (!GATHER)
-        for (int i = 0; i < pre; ++i)
-          tma_load_2d(smem + i * C::STAGE, &tm_a, &full[i], (first.kb0 + i) * BK, first.m_tile * BM);
+        for (int i = 0; i < pre; ++i) load_a(smem + i * C::STAGE, first.kb0 + i, first.m_tile, i);
       stage = pre % STAGES;
       phase = (pre == STAGES) ? 1u : 0u;
       while (ok && walk.next(p, sg)) {
@@ -401,13 +442,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             break;
           }
           uint8_t* sa = smem + stage * C::STAGE;
-          if (GATHER) {
-            mbar_arrive_expect_tx(&full[stage], C::B_BYTES);
-          } else {
-            mbar_arrive_expect_tx(&full[stage], C::STAGE);
-            tma_load_2d(sa, &tm_a, &full[stage], kb * BK, sg.m_tile * BM);
-          }
-          load_b(sa + C::A_BYTES, kb, sg.n_tile, &full[stage]);
+          if (arrives) mbar_arrive_expect_tx(&full[stage], kStageTx);
+          if (!GATHER) load_a(sa, kb, sg.m_tile, stage);
+          load_b(sa + C::A_BYTES, kb, sg.n_tile, stage);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -417,22 +454,36 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         }
       }
       // Copies still in flight must land before the CTA may exit (error path only; in the
-      // normal path every issued stage was consumed already and these return at once).
+      // normal path every issued stage was consumed already and these return at once).  The
+      // second CTA of a pair has no full barrier of its own: it waits until the MMAs released
+      // each stage it filled.
       volatile int never = 0;
-      for (int s = 0; s < STAGES; ++s)
-        if (issued & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, &never, p.err, kErrTimeoutProducer);
+      for (int s = 0; s < STAGES; ++s) {
+        if (!(issued & (1u << s))) continue;
+        if (arrives) mbar_wait(&full[s], (issued_phase >> s) & 1u, &never, p.err, kErrTimeoutProducer);
+        else mbar_wait(&empty[s], (issued_phase >> s) & 1u, &never, p.err, kErrTimeoutProducer);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(BM, BN, false);
+    if (PAIR && rank != 0) {
+      // The second CTA of a pair issues nothing; its TMEM is written by the leader's MMAs until
+      // their final commit.
+      if (lane == 0) {
+        volatile int never = 0;
+        mbar_wait(mma_done, 0, &never, p.err, kErrTimeoutMma);
+      }
+    } else if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BMT, BN, false);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      SegmentWalker walk(p);
+      SegmentWalker walk(p, owner);
       Segment sg;
       while (ok && walk.next(p, sg)) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma)) break;
+        const bool free_acc = PAIR ? mbar_wait_cluster(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma)
+                                   : mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma);
+        if (!free_acc) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
@@ -448,23 +499,29 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4).
-            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
+            if constexpr (PAIR)
+              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (PAIR) umma_commit_pair(&empty[stage]);
+          else umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (PAIR) umma_commit_pair(&tfull[acc]);
+        else umma_commit(&tfull[acc]);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
       // Every MMA issued so far completes before TMEM may be released.
-      umma_commit(mma_done);
+      if constexpr (PAIR) umma_commit_pair(mma_done);
+      else umma_commit(mma_done);
       volatile int never = 0;
       mbar_wait(mma_done, 0, &never, p.err, kErrTimeoutMma);
     }
@@ -475,18 +532,26 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     const int row_in_tile = quad * 32 + lane;
     const int et = threadIdx.x - 64;
     Stager st{smem + C::OFF_STAGING + (warp - 2) * 8192, lane, 0};
+    // Hands an accumulator buffer back to the MMA issuer (the leader's barrier, in a pair).
+    const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
+    auto release_acc = [&](int buf) {
+      if constexpr (PAIR) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(buf));
+      else mbar_arrive(&tempty[buf]);
+    };
     constexpr int NGROUPS = BN / 64;
     int acc = 0;
     uint32_t acc_phase = 0;
     grid_dependency_wait();
-    SegmentWalker walk(p);
+    SegmentWalker walk(p, owner);
     Segment sg;
     while (walk.next(p, sg)) {
-      const int row = sg.m_tile * BM + row_in_tile;
-      const int box_y = sg.m_tile * BM + quad * 32;
+      const int row0 = sg.m_tile * BMT + static_cast<int>(rank) * BM;  // this CTA's rows of the tile
+      const int row = row0 + row_in_tile;
+      const int box_y = row0 + quad * 32;
+      const int ctr = PAIR ? 2 * sg.tile + static_cast<int>(rank) : sg.tile;  // split-tile counter
       const bool finisher_or_full =
           (sg.kb0 == 0 && sg.kb1 == p.kb_total) ||
-          static_cast<int>(blockIdx.x) == unit_owner(p, static_cast<long long>(sg.tile) * p.kb_total);
+          owner == unit_owner(p, static_cast<long long>(sg.tile) * p.kb_total);
       // Inputs of the epilogue math fetched while the MMAs run: the rotation table row and the
       // residual row of this thread's output row, and the folded-norm row scale.
       float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
@@ -544,10 +609,10 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                             __uint_as_float(r[4 * q + 3]));
         }
         tc_fence_before_sync();
-        mbar_arrive(&tempty[acc]);
+        release_acc(acc);
         __threadfence();
         named_barrier_sync(1, 128);
-        if (et == 0) atomicAdd(&p.counters[sg.tile], 1);
+        if (et == 0) atomicAdd(&p.counters[ctr], 1);
       } else {
         // Whole tile, or finisher of a split tile: wait for the other contributors (if any),
         // add their partials in CTA order, run the epilogue math, stage and store.
@@ -557,11 +622,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           const long long u_first = static_cast<long long>(sg.tile) * p.kb_total;
           c_first = unit_owner(p, u_first);
           c_last = unit_owner(p, u_first + p.kb_total - 1);
-          if (et == 0) *ticket = wait_counter(&p.counters[sg.tile], c_last - c_first, abort_flag, p.err) ? 1 : 0;
+          if (et == 0) *ticket = wait_counter(&p.counters[ctr], c_last - c_first, abort_flag, p.err) ? 1 : 0;
           named_barrier_sync(1, 128);
           if (!*ticket) {
             tc_fence_before_sync();
-            mbar_arrive(&tempty[acc]);
+            release_acc(acc);
             break;
           }
           __threadfence();
@@ -586,7 +651,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           if (split) {
 #pragma unroll 2
             for (int cc = c_first + 1; cc <= c_last; ++cc) {
-              const float* src = partial_slot<BN>(p, cc);
+              const float* src = partial_slot<BN>(p, PAIR ? 2 * cc + static_cast<int>(rank) : cc);
               float4 a[8], b[8];
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
@@ -628,10 +693,10 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           }
         }
         tc_fence_before_sync();
-        mbar_arrive(&tempty[acc]);
+        release_acc(acc);
         if (EPI == EPI_RESID && p.xw_out && row < p.M)
           p.ss_out[static_cast<size_t>(row) * p.ss_parts + sg.n_tile] = ss_acc;
-        if (split && et == 0) p.counters[sg.tile] = 0;  // ready for the next launch
+        if (split && et == 0) p.counters[ctr] = 0;  // ready for the next launch
       }
       if (++acc == 2) {
         acc = 0;
@@ -647,7 +712,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     int stage = 0, pending = -1;
     uint32_t phase = 0;
     bool ok = true;
-    SegmentWalker walk(p);
+    SegmentWalker walk(p, owner);
     Segment sg;
     while (ok && walk.next(p, sg)) {
       const int row = sg.m_tile * BM + r;
@@ -684,19 +749,24 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     }
   }
 
+  __syncwarp();  // every warp reconverged (role code ran on single lanes) before the CTA barrier
   tc_fence_before_sync();
   __syncthreads();
+  // Neither CTA of a pair leaves (or frees TMEM) while the other may still signal its barriers.
+  if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
-template <int BN, int EPI, bool GATHER>
+template <int BN, int EPI, bool GATHER, bool PAIR = false>
 cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
-  using C = TileCfg<BN>;
+  using C = TileCfg<BN, PAIR>;
   static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
-  auto kern = k_gemm_tc<BN, EPI, GATHER>;
+  auto kern = k_gemm_tc<BN, EPI, GATHER, PAIR>;
+  if (PAIR && (plan.grid & 1)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -711,6 +781,7 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.n_out = a.n_out;
   p.tiles_m = plan.tiles_m;
   p.kb_total = plan.kb_total;
+  p.owners = PAIR ? plan.grid / 2 : plan.grid;
   p.units = static_cast<long long>(plan.tiles_m) * plan.tiles_n * plan.kb_total;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.ldo = a.ldo;
@@ -737,12 +808,30 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   const CUtensorMap& ta = GATHER ? *a.tm_b : *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
   const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
-  return launch_pdl(kern, dim3(plan.grid), dim3(GATHER ? 320 : 192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
+  if constexpr (PAIR)
+    return launch_pdl_pair(kern, dim3(plan.grid), dim3(192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
+  else
+    return launch_pdl(kern, dim3(plan.grid), dim3(GATHER ? 320 : 192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
 }
 
 // Tile widths each epilogue supports (the planner only picks these).
 template <int EPI, bool GATHER>
 cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
+  if (plan.pair) {
+    // CTA pairs: 256-row tiles, no A-gather.
+    if constexpr (GATHER || EPI == EPI_STORE) {
+      return cudaErrorInvalidValue;
+    } else if constexpr (EPI == EPI_SWIGLU) {
+      if (plan.bn == 256) return launch_one<256, EPI, false, true>(plan, a, s);
+      return cudaErrorInvalidValue;
+    } else {
+      switch (plan.bn) {
+        case 128: return launch_one<128, EPI, false, true>(plan, a, s);
+        case 256: return launch_one<256, EPI, false, true>(plan, a, s);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+  }
   if constexpr (EPI == EPI_RESID) {
     switch (plan.bn) {
       case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
@@ -776,6 +865,13 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
 //  - per CTA: ~2000 cycles of set-up and first-load latency and ~12 cycles per output column.
 double kblock_cycles(int bn) { return std::max(2.0 * bn, (16384.0 + 128.0 * bn) / 72.0 + 100.0); }
 
+// CTA pairs (256 x 256 tiles, tcgen05 cta_group::2, one tile's B split between two SMs) are
+// taken when there are at least this many waves of pair tiles over the SM pairs.  Measured on
+// B200 (standalone, graph-replayed): at M = 25000 pairs beat 128 x 256 single-CTA tiles by 1-7 %
+// on all four GEMMs of the block (SwiGLU 235 -> 222 us, QKV 147 -> 137 us); at M = 3562 (1-4
+// waves) they lose by 1-60 %, mostly to split-tile fix-ups.
+constexpr int kPairMinWaves = 5;
+
 double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_out) {
   const long long units = tiles * kb_total;
   const long long per_cta = (units + grid - 1) / grid;
@@ -799,38 +895,66 @@ double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_o
 
 }  // namespace
 
-GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms);
+GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes);
 
-GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms) {
-  // Plans depend only on the shape; each thread keeps the ones it has computed.
+GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes) {
+  // Plans depend only on the shape (and the scratch cap); each thread keeps the ones it has
+  // computed.
   struct Key {
     int epi, M, n_out, K, sms;
+    size_t cap;
     bool operator==(const Key& o) const {
-      return epi == o.epi && M == o.M && n_out == o.n_out && K == o.K && sms == o.sms;
+      return epi == o.epi && M == o.M && n_out == o.n_out && K == o.K && sms == o.sms && cap == o.cap;
     }
   };
   struct KeyHash {
     size_t operator()(const Key& k) const {
-      return (((static_cast<size_t>(k.M) * 1000003u + k.n_out) * 1000003u + k.K) * 31u + k.epi) * 1009u + k.sms;
+      return ((((static_cast<size_t>(k.M) * 1000003u + k.n_out) * 1000003u + k.K) * 31u + k.epi) * 1009u + k.sms) *
+                 131u +
+             k.cap;
     }
   };
   thread_local std::unordered_map<Key, GemmPlan, KeyHash> cache;
-  const Key key{epi, M, n_out, K, num_sms};
+  const Key key{epi, M, n_out, K, num_sms, max_partial_bytes};
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   if (cache.size() > 1024) cache.clear();
-  GemmPlan best = plan_gemm_uncached(epi, M, n_out, K, num_sms);
+  GemmPlan best = plan_gemm_uncached(epi, M, n_out, K, num_sms, max_partial_bytes);
   cache[key] = best;
   return best;
 }
 
-GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms) {
+GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes) {
   GemmPlan best{};
-  double best_cost = 1e300;
   const int kb_total = K / BK;
+  if (kb_total <= 0 || M <= 0 || num_sms <= 0) return best;
+  // CTA pairs with 256-column tiles, stream-K over all SM pairs, when there is enough work.
+  if (epi != EPI_STORE && n_out % (epi == EPI_SWIGLU ? 128 : 256) == 0) {
+    const int tiles_m = (M + 2 * BM - 1) / (2 * BM);
+    const int tiles_n = n_out / (epi == EPI_SWIGLU ? 128 : 256);
+    const long long tiles = static_cast<long long>(tiles_m) * tiles_n;
+    const int pairs = num_sms / 2;
+    int contrib = 1;
+    plan_cost(256, tiles, kb_total, pairs, &contrib);
+    const size_t partial = contrib > 1 ? static_cast<size_t>(2 * pairs) * BM * 256 * sizeof(float) : 0;
+    if (pairs > 0 && tiles >= static_cast<long long>(kPairMinWaves) * pairs && contrib <= 2 &&
+        partial <= max_partial_bytes) {
+      best.bn = 256;
+      best.pair = 1;
+      best.splits = contrib;
+      best.tiles_m = tiles_m;
+      best.tiles_n = tiles_n;
+      best.kb_total = kb_total;
+      best.work = static_cast<int>(tiles);
+      best.grid = 2 * pairs;
+      best.partial_bytes = partial;
+      best.counters = contrib > 1 ? static_cast<int>(tiles) * 2 : 0;
+      return best;
+    }
+  }
+  double best_cost = 1e300;
   const int tiles_m = (M + BM - 1) / BM;
   const int cands[4] = {256, 192, 128, 64};
-  if (kb_total <= 0 || tiles_m <= 0 || num_sms <= 0) return best;
   for (int bn : cands) {
     // Epilogue constraints: SwiGLU stores 64-column boxes of two 32-column groups (bn / 2 a
     // multiple of 64); the residual epilogue is built for bn in {64, 128, 256}.
@@ -851,16 +975,19 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms) {
       int contrib = 1;
       const double cost = plan_cost(bn, tiles, kb_total, grids[gi], &contrib);
       if (contrib > 2) continue;  // more contributors leave straggling finishers (measured)
+      const size_t partial = contrib > 1 ? static_cast<size_t>(grids[gi]) * BM * bn * sizeof(float) : 0;
+      if (partial > max_partial_bytes) continue;
       if (cost < best_cost - 1e-9) {
         best_cost = cost;
         best.bn = bn;
+        best.pair = 0;
         best.splits = contrib;
         best.tiles_m = tiles_m;
         best.tiles_n = tiles_n;
         best.kb_total = kb_total;
         best.work = static_cast<int>(tiles);
         best.grid = grids[gi];
-        best.partial_bytes = contrib > 1 ? static_cast<size_t>(grids[gi]) * BM * bn * sizeof(float) : 0;
+        best.partial_bytes = partial;
         best.counters = contrib > 1 ? static_cast<int>(tiles) : 0;
       }
     }

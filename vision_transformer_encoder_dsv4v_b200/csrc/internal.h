@@ -18,20 +18,22 @@ enum Epi : int {
 
 struct GemmPlan {
   int bn;        // MMA N per tile (SWIGLU: gate + up halves)
+  int pair;      // 1: 256-row tiles on CTA pairs (tcgen05 cta_group::2), grid even; 0: 128-row tiles
   int splits;    // K splits per tile (fix-up by the last finisher)
   int tiles_m, tiles_n, kb_total, work, grid;
   size_t partial_bytes;  // fp32 scratch for split tiles
   int counters;          // tile counters needed (split tiles only)
 };
 
-// Chooses tile width and split count for a GEMM of this shape on `num_sms` SMs.
-GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms);
+// Chooses tile width, CTA pairing and split count for a GEMM of this shape on `num_sms` SMs;
+// plans whose split-tile partials exceed max_partial_bytes are not considered.
+GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes = SIZE_MAX);
 
 struct GemmArgs {
   const CUtensorMap* tm_out;  // output [M, n_out] bf16, box 64 x 32 (TMA stores of the epilogue)
   const CUtensorMap* tm_xw;   // RESID with the next norm prepared: xw_out [M, n_out], box 64 x 32
   const CUtensorMap* tm_a;    // A [M, K], box 64 x 128 (ignored when gathering A)
-  const CUtensorMap* tm_b;    // B [n, K] (SWIGLU: w_gate), box 64 x bn (SWIGLU: bn / 2)
+  const CUtensorMap* tm_b;    // B [n, K] (SWIGLU: w_gate), box 64 x bn (SWIGLU or pair: bn / 2)
   const CUtensorMap* tm_b2;   // SWIGLU: w_up, box 64 x bn / 2
   int M, K, n_out;
   void* out;
