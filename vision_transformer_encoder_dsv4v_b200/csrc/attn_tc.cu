@@ -218,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_free + 2;     // [tile]
   uint64_t* pv_done = p_full + 2;    // [tile]
   uint64_t* mma_done = pv_done + 2;  // [tile]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 2);
+  uint64_t* teardown = mma_done + 2;  // one arrival per warp once its role is done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
+    mbar_init(teardown, kThreads / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -491,9 +493,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  __syncwarp();  // every warp reconverged (role code ran on single lanes) before the CTA barrier
+  // Teardown: TMEM is released only after every warp has finished with it.  Role code ran on
+  // single lanes, so the warps meet on an mbarrier (one arrival per reconverged warp) rather than
+  // on a CTA-wide bar.sync.
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(teardown);
+  {
+    volatile int never = 0;
+    mbar_wait(teardown, 0, &never, p.err, kErrTimeoutEpilogue);
+  }
   if (warp == 1) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, TMEM_COLS);

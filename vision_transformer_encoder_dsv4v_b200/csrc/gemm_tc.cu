@@ -330,7 +330,8 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* teardown = mma_done + 1;  // one arrival per warp once its role is done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* ticket = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
@@ -351,6 +352,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       mbar_init(&tempty[a], PAIR ? 256 : 128);
     }
     mbar_init(mma_done, 1);
+    mbar_init(teardown, blockDim.x / 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -749,9 +751,16 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     }
   }
 
-  __syncwarp();  // every warp reconverged (role code ran on single lanes) before the CTA barrier
+  // Teardown: TMEM is released only after every warp has finished with it.  Role code ran on
+  // single lanes, so the warps meet on an mbarrier (one arrival per reconverged warp) rather than
+  // on a CTA-wide bar.sync.
   tc_fence_before_sync();
-  __syncthreads();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(teardown);
+  {
+    volatile int never = 0;
+    mbar_wait(teardown, 0, &never, p.err, kErrTimeoutEpilogue);
+  }
   // Neither CTA of a pair leaves (or frees TMEM) while the other may still signal its barriers.
   if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
