@@ -471,7 +471,8 @@ bool weights_ok(const dsv4v_block_weights* w) {
 
 dsv4v_status reset_counters(const Ctx& c) {
   if (!c.s.bf16) return DSV4V_OK;
-  return cuda_status(cudaMemsetAsync(c.ws + c.lay.counters, 0, c.lay.counters_bytes, c.stream));
+  return cuda_status(launch_zero_counters(c.at<int>(c.lay.counters), static_cast<int>(c.lay.counters_bytes / sizeof(int)),
+                                          c.stream));
 }
 
 dsv4v_status rope_table(const Ctx& c, const dsv4v_batch* b, float* cos, float* sin) {

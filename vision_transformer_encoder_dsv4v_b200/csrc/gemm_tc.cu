@@ -46,7 +46,13 @@ struct TileCfg {
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int RING_BUDGET = kMaxDynSmem - 1024 - 512 - kStagingBytes;
   static constexpr int STAGES = RING_BUDGET / STAGE > 8 ? 8 : RING_BUDGET / STAGE;
-  static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : ((2 * BN <= 256) ? 256 : 512);
+  // Independent accumulator chains per tile.  Consecutive K=16 MMAs into one accumulator cost
+  // at least ~97 cycles each (measured on B200: a 128 x N x 64 K block takes 387 cycles for
+  // N = 64 and 128, 513 for N = 256, i.e. full rate only at N = 256), so narrow tiles spread
+  // their K steps over CH accumulators (step k -> chain k % CH) and the epilogue sums them.
+  static constexpr int CH = BN >= 192 ? 1 : 256 / BN;
+  static constexpr int ACC_COLS = CH * BN;  // TMEM columns of one accumulator buffer
+  static constexpr int TMEM_COLS = (2 * ACC_COLS <= 128) ? 128 : ((2 * ACC_COLS <= 256) ? 256 : 512);
   static constexpr int OFF_STAGING = STAGES * STAGE;
   static constexpr int OFF_BARRIERS = OFF_STAGING + kStagingBytes;
   static constexpr int SMEM = 1024 + OFF_BARRIERS + 512;
@@ -487,7 +493,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                                    : mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma);
         if (!free_acc) break;
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::ACC_COLS);
         for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutMma)) {
             ok = false;
@@ -502,9 +508,10 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4).
             if constexpr (PAIR)
-              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
+              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);  // CH = 1
             else
-              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
+              umma_bf16(d_tmem + static_cast<uint32_t>((k % C::CH) * BN), adesc + 2 * k, bdesc + 2 * k, idesc,
+                        (kb > sg.kb0 || k >= C::CH) ? 1u : 0u);
           }
           if constexpr (PAIR) umma_commit_pair(&empty[stage]);
           else umma_commit(&empty[stage]);
@@ -595,7 +602,8 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       // the partial-tile path uses a named barrier).
       if (!named_barrier_and(2, 128, got)) break;
       tc_fence_after_sync();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::ACC_COLS);
       if (!finisher_or_full) {
         // Contributor to a tile finished by another CTA: park the partial, release it, move on.
         float* slot = partial_slot<BN>(p, blockIdx.x);
@@ -604,11 +612,20 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           uint32_t r[32];
           tmem_ld32(t_row + c * 32, r);
           tmem_ld_wait(r);
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+#pragma unroll
+          for (int ch = 1; ch < C::CH; ++ch) {
+            tmem_ld32(t_row + ch * BN + c * 32, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(r[j]);
+          }
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(slot + ((c * 8 + q) * BM + row_in_tile) * 4) =
-                make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                            __uint_as_float(r[4 * q + 3]));
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
         tc_fence_before_sync();
         release_acc(acc);
@@ -649,6 +666,18 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           for (int j = 0; j < 32; ++j) {
             v[j] = __uint_as_float(r0[j]);
             v[32 + j] = __uint_as_float(r1[j]);
+          }
+#pragma unroll
+          for (int ch = 1; ch < C::CH; ++ch) {
+            tmem_ld32(t_row + ch * BN + c0 * 32, r0);
+            tmem_ld32(t_row + ch * BN + c1 * 32, r1);
+            tmem_ld_wait(r0);
+            tmem_ld_wait(r1);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              v[j] += __uint_as_float(r0[j]);
+              v[32 + j] += __uint_as_float(r1[j]);
+            }
           }
           if (split) {
 #pragma unroll 2
@@ -866,20 +895,14 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
 }
 
 // Cost model (cycles) of one SM's share of a GEMM, used to pick the tile width and the grid.
-//  - one 64-deep K block of a 128 x bn tile: the larger of the tensor-pipe time (bn / 2 cycles
-//    per K=16 step) and the time to stream the A (16 KB) and B (bn * 128 B) tiles from L2 at
-//    ~72 B/cycle per SM, plus ~100 cycles of hand-off;
-//  - a split tile: its partial (128 x bn fp32) written once and read back by the finisher with
-//    the other contributors' partials, plus ~1500 cycles of fence and ticket;
+// Constants fitted to standalone, graph-replayed measurements on B200 (M = 784 and 3562, all four
+// block GEMMs, every candidate tile width and grid):
+//  - one 64-deep K block of a 128 x bn tile: ~600 cycles up to bn = 192 (the per-stage round trip
+//    of TMA load, MMA and release, not the tensor pipe) and ~3.1 cycles per column above;
+//  - a split tile: its partial (128 x bn fp32) written by each contributor and read back by the
+//    finisher, the counter hand-off and the finisher's late epilogue, ~4000 + 40 bn cycles;
 //  - per CTA: ~2000 cycles of set-up and first-load latency and ~12 cycles per output column.
-double kblock_cycles(int bn) { return std::max(2.0 * bn, (16384.0 + 128.0 * bn) / 72.0 + 100.0); }
-
-// CTA pairs (256 x 256 tiles, tcgen05 cta_group::2, one tile's B split between two SMs) are
-// taken when there are at least this many waves of pair tiles over the SM pairs.  Measured on
-// B200 (standalone, graph-replayed): at M = 25000 pairs beat 128 x 256 single-CTA tiles by 1-7 %
-// on all four GEMMs of the block (SwiGLU 235 -> 222 us, QKV 147 -> 137 us); at M = 3562 (1-4
-// waves) they lose by 1-60 %, mostly to split-tile fix-ups.
-constexpr int kPairMinWaves = 5;
+double kblock_cycles(int bn) { return std::max(600.0, 3.1 * bn); }
 
 double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_out) {
   const long long units = tiles * kb_total;
@@ -896,11 +919,17 @@ double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_o
     }
   }
   *contrib_out = contrib;
-  const double slot = 128.0 * bn * 4.0 / 128.0;
   double cost = per_cta * kblock_cycles(bn) + 2000.0 + 12.0 * bn;
-  if (contrib > 1) cost += 1000.0 + slot * contrib;
+  if (contrib > 1) cost += 4000.0 + 40.0 * bn;
   return cost;
 }
+
+// CTA pairs (256 x 256 tiles, tcgen05 cta_group::2, one tile's B split between two SMs) are
+// taken when there are at least this many waves of pair tiles over the SM pairs.  Measured on
+// B200 (standalone, graph-replayed): at M = 25000 pairs beat 128 x 256 single-CTA tiles by 1-7 %
+// on all four GEMMs of the block (SwiGLU 235 -> 222 us, QKV 147 -> 137 us); at M = 3562 (1-4
+// waves) they lose by 1-60 %, mostly to split-tile fix-ups.
+constexpr int kPairMinWaves = 5;
 
 }  // namespace
 
@@ -974,11 +1003,15 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
     const int tiles_n = n_out / n_cols_per_tile;
     const long long tiles = static_cast<long long>(tiles_m) * tiles_n;
     const long long units = tiles * kb_total;
-    // Grids: every SM; or s CTAs per tile (s = 1: one tile each, s > 1: split-K by s).
-    int grids[6];
+    // Grids: every SM; t whole tiles per CTA (t = 1..4); or s CTAs per tile (split-K by s).
+    int grids[9];
     int n_grids = 0;
     grids[n_grids++] = static_cast<int>(std::min<long long>(num_sms, units));
-    for (int s = 1; s <= 4; ++s)
+    for (int t = 1; t <= 4; ++t) {
+      const long long g = (tiles + t - 1) / t;
+      if (g <= num_sms) grids[n_grids++] = static_cast<int>(g);
+    }
+    for (int s = 2; s <= 4; ++s)
       if (tiles * s <= num_sms && tiles * s <= units) grids[n_grids++] = static_cast<int>(tiles * s);
     for (int gi = 0; gi < n_grids; ++gi) {
       int contrib = 1;

@@ -97,6 +97,7 @@ cudaError_t launch_rmsnorm(bool bf16, const void* x, const float* w, void* y, in
 cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev, int n_images, int r,
                                  int64_t n_tokens, int32_t* src_out, cudaStream_t s, int* zero_ptr = nullptr,
                                  int zero_n = 0);
+cudaError_t launch_zero_counters(int* ptr, int n, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
 // Norm operands of the first GEMM of a block: xw = bf16(x * w) and ss[p * parts] = sum_c x[p,c]^2
 // (the other parts of a row are zero-filled); also clears zero_n counters like the kernels above.

@@ -173,6 +173,14 @@ __global__ void k_aligner_index(const int32_t* __restrict__ cu, const int32_t* _
     }
 }
 
+// Clears the GEMM tile counters of a component call (one block; dependent launch, so that it
+// costs no more than a kernel boundary inside a graph, unlike a memset node).
+__global__ void k_zero_counters(int* ptr, int n) {
+  grid_dependency_wait();
+  launch_dependents();
+  zero_ints(ptr, n);
+}
+
 // Waits on an mbarrier that nothing signals, with the production kernels' bounded wait.
 __global__ void k_selftest_wait(uint64_t limit_ns, uint32_t* err) {
   __shared__ uint64_t bar;
@@ -235,6 +243,11 @@ cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev,
   return launch_pdl(k_aligner_index, dim3(static_cast<unsigned>(blocks)), dim3(threads),
                     (n_images + 1) * sizeof(int32_t), s, cu_dev, grid_dev, n_images, r, n_tokens, src_out, zero_ptr,
                     zero_n);
+}
+
+cudaError_t launch_zero_counters(int* ptr, int n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  return launch_pdl(k_zero_counters, dim3(1), dim3(256), 0, s, ptr, n);
 }
 
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s) {
