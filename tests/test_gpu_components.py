@@ -142,3 +142,63 @@ def test_aligner_bf16(grids):
     want, cu_o = O.aligner_forward(x.values, wa.values, grids, 2)
     assert list(cu_tok.numpy()) == list(cu_o)
     assert_bf16_close(to_np(out), want, abs_floor=2e-5)
+
+
+# Shapes large enough that the planner runs the block GEMMs on CTA pairs (256-row tiles split
+# between two SMs, tcgen05 cta_group::2).  The oracle is evaluated on sampled rows: both CTAs'
+# halves of several pair tiles, the pair-tile boundaries and the ragged tail.
+def _pair_rows(m, seed):
+    rng = np.random.default_rng(seed)
+    edges = [0, 1, 127, 128, 129, 255, 256, 257, 383, 384, 511, 512]
+    tail = [m - 1 - i for i in range(0, 260, 37)] + [(m // 256) * 256 - 1, (m // 256) * 256]
+    picks = rng.choice(m, size=64, replace=False).tolist()
+    return np.array(sorted({r for r in edges + tail + picks if 0 <= r < m}))
+
+
+@pytest.mark.parametrize("k", [1024, 2816])
+def test_linear_residual_pair_tiles(k):
+    rows = 25985
+    cfg = cfg_bf16()
+    a = random_bf16((rows, k), 1.0, seed=61)
+    w = random_bf16((1024, k), 0.02, seed=62)
+    x = random_bf16((rows, 1024), 1.0, seed=63)
+    xt = dev(x)
+    ws = torch.empty(A.dsv4v_workspace_size(cfg, A.BatchRef([(rows, 1)])), dtype=torch.uint8, device="cuda")
+    A.dsv4v_linear_residual(cfg, rows, k, dev(a), dev(w), xt, ws)
+    assert A.dsv4v_device_error() == 0
+    r = _pair_rows(rows, 64)
+    want = x.values[r].astype(np.float64) + a.values[r].astype(np.float64) @ w.values.astype(np.float64).T
+    assert_bf16_close(to_np(xt)[r], want, abs_floor=2e-5)
+
+
+def test_swiglu_pair_tiles():
+    rows = 9001
+    cfg = cfg_bf16()
+    y = random_bf16((rows, 1024), 1.0, seed=71)
+    wg = random_bf16((2816, 1024), 0.02, seed=72)
+    wu = random_bf16((2816, 1024), 0.02, seed=73)
+    h = torch.empty(rows, 2816, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(A.dsv4v_workspace_size(cfg, A.BatchRef([(rows, 1)])), dtype=torch.uint8, device="cuda")
+    A.dsv4v_swiglu(cfg, rows, dev(y), dev(wg), dev(wu), h, ws)
+    assert A.dsv4v_device_error() == 0
+    r = _pair_rows(rows, 74)
+    yy = y.values[r].astype(np.float64)
+    want = O.silu(yy @ wg.values.astype(np.float64).T) * (yy @ wu.values.astype(np.float64).T)
+    assert_bf16_close(to_np(h)[r], want, abs_floor=2e-5)
+
+
+def test_qkv_rope_pair_tiles():
+    grids = [(64, 64), (64, 64), (30, 31)]
+    b = A.BatchRef(grids)
+    cfg = cfg_bf16()
+    P = b.n_patches
+    y = random_bf16((P, 1024), 1.0, seed=81)
+    wqkv = random_bf16((3072, 1024), 0.02, seed=82)
+    c_o, s_o = O.packed_cos_sin(grids, 32, 10000.0)
+    qkv = torch.empty(P, 3072, dtype=torch.bfloat16, device="cuda")
+    A.dsv4v_qkv_rope(cfg, b, dev(y), dev(wqkv), f32(c_o), f32(s_o), qkv, workspace(cfg, b))
+    assert A.dsv4v_device_error() == 0
+    r = _pair_rows(P, 84)
+    q, k, v = O.qkv_rope(y.values[r], wqkv.values, c_o[r].astype(np.float32), s_o[r].astype(np.float32), 16)
+    want = np.concatenate([q.reshape(len(r), -1), k.reshape(len(r), -1), v.reshape(len(r), -1)], axis=1)
+    assert_bf16_close(to_np(qkv)[r], want, abs_floor=2e-5)
