@@ -400,7 +400,7 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   }
   NormFold q;
   q.ss = ss1;
-  q.parts = first ? 1 : c.plans.down.tiles_n;  // the prep kernel puts the whole row sum in slot 0
+  q.parts = first ? 1 : norm_parts_of(c.plans.down);  // the prep kernel puts the whole row sum in slot 0
   q.stride = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_QKV, 0, c.stream));
   DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, xw, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr,
@@ -420,7 +420,7 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   DSV4V_TRY(record(ev, DSV4V_PROFILE_OUT, 1, c.stream));
   NormFold m;
   m.ss = ss2;
-  m.parts = c.plans.out.tiles_n;
+  m.parts = norm_parts_of(c.plans.out);
   m.stride = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_SWIGLU, 0, c.stream));
   DSV4V_TRY(gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, xw, s.P, s.D, w->w_gate, w->w_up, s.F, h, nullptr,

@@ -46,13 +46,7 @@ struct TileCfg {
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int RING_BUDGET = kMaxDynSmem - 1024 - 512 - kStagingBytes;
   static constexpr int STAGES = RING_BUDGET / STAGE > 8 ? 8 : RING_BUDGET / STAGE;
-  // Independent accumulator chains per tile.  Consecutive K=16 MMAs into one accumulator cost
-  // at least ~97 cycles each (measured on B200: a 128 x N x 64 K block takes 387 cycles for
-  // N = 64 and 128, 513 for N = 256, i.e. full rate only at N = 256), so narrow tiles spread
-  // their K steps over CH accumulators (step k -> chain k % CH) and the epilogue sums them.
-  static constexpr int CH = BN >= 192 ? 1 : 256 / BN;
-  static constexpr int ACC_COLS = CH * BN;  // TMEM columns of one accumulator buffer
-  static constexpr int TMEM_COLS = (2 * ACC_COLS <= 128) ? 128 : ((2 * ACC_COLS <= 256) ? 256 : 512);
+  static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : ((2 * BN <= 256) ? 256 : 512);
   static constexpr int OFF_STAGING = STAGES * STAGE;
   static constexpr int OFF_BARRIERS = OFF_STAGING + kStagingBytes;
   static constexpr int SMEM = 1024 + OFF_BARRIERS + 512;
@@ -320,12 +314,14 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatil
   }
 }
 
-template <int BN, int EPI, bool GATHER, bool PAIR>
+template <int BN, int EPI, bool GATHER, bool PAIR, int KS>
 __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
               const __grid_constant__ CUtensorMap tm_xw, const Params p) {
   static_assert(!(GATHER && PAIR), "the A-gather runs on single CTAs");
+  static_assert(KS == 1 || (!GATHER && !PAIR && BN == 256 && EPI == EPI_RESID),
+                "cluster split-K is built for 256-column residual tiles");
   using C = TileCfg<BN, PAIR>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
   constexpr int STAGES = C::STAGES;
@@ -346,6 +342,10 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
   // In a pair, rank 0 (the leader) issues the MMAs; its full and tempty barriers gather both
   // CTAs' loads and epilogue releases, the other barriers are signalled in both CTAs at once.
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  // Cluster split-K (KS > 1): the KS CTAs of a cluster each run one K slice of the same tile and
+  // then reduce-scatter the accumulator through distributed shared memory; rank kslice finishes
+  // columns [kslice * BN / KS, (kslice + 1) * BN / KS).
+  const uint32_t kslice = KS > 1 ? cluster_ctarank() : 0u;
   const int owner = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
 
   if (threadIdx.x == 0) {
@@ -472,6 +472,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         else mbar_wait(&empty[s], (issued_phase >> s) & 1u, &never, p.err, kErrTimeoutProducer);
       }
     }
+    if constexpr (KS > 1) {
+      __syncwarp();
+      cluster_sync();  // the two reduce-scatter barriers of the epilogue
+      cluster_sync();
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (PAIR && rank != 0) {
@@ -493,7 +498,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
                                    : mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma);
         if (!free_acc) break;
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::ACC_COLS);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutMma)) {
             ok = false;
@@ -508,10 +513,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4).
             if constexpr (PAIR)
-              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);  // CH = 1
+              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
             else
-              umma_bf16(d_tmem + static_cast<uint32_t>((k % C::CH) * BN), adesc + 2 * k, bdesc + 2 * k, idesc,
-                        (kb > sg.kb0 || k >= C::CH) ? 1u : 0u);
+              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
           }
           if constexpr (PAIR) umma_commit_pair(&empty[stage]);
           else umma_commit(&empty[stage]);
@@ -535,6 +539,10 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       mbar_wait(mma_done, 0, &never, p.err, kErrTimeoutMma);
     }
     __syncwarp();
+    if constexpr (KS > 1) {
+      cluster_sync();  // the two reduce-scatter barriers of the epilogue (this CTA's MMAs are done)
+      cluster_sync();
+    }
   } else if (warp < 6) {
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) belong to this warp
@@ -553,7 +561,131 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     grid_dependency_wait();
     SegmentWalker walk(p, owner);
     Segment sg;
-    while (walk.next(p, sg)) {
+    if constexpr (KS > 1) {
+      // ------------------------------------------------ cluster split-K: one K slice of one tile
+      constexpr int GPR = NGROUPS / KS;  // 64-column groups finished by each rank
+      constexpr int SLOT_BYTES = GPR * 16 * BM * 16;
+      const int g0 = static_cast<int>(kslice) * GPR;
+      const bool have = walk.next(p, sg);
+      const int row = sg.m_tile * BM + row_in_tile;
+      const int box_y = sg.m_tile * BM + quad * 32;
+      float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
+      uint4 resid[EPI == EPI_RESID ? GPR * 8 : 1];
+      if constexpr (EPI == EPI_QKV_ROPE) {
+        const int prow = min(row, p.M - 1);
+        const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(prow) * 32);
+        const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(prow) * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 c = c4[q], s = s4[q];
+          rot_c[4 * q] = c.x; rot_c[4 * q + 1] = c.y; rot_c[4 * q + 2] = c.z; rot_c[4 * q + 3] = c.w;
+          rot_s[4 * q] = s.x; rot_s[4 * q + 1] = s.y; rot_s[4 * q + 2] = s.z; rot_s[4 * q + 3] = s.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          pin(rot_c[j]);
+          pin(rot_s[j]);
+        }
+      }
+      if constexpr (EPI == EPI_RESID) {
+        const uint4* r4 = reinterpret_cast<const uint4*>(p.resid + static_cast<size_t>(min(row, p.M - 1)) * p.ldo +
+                                                         sg.n_tile * BN + g0 * 64);
+#pragma unroll
+        for (int q = 0; q < GPR * 8; ++q) resid[q] = r4[q];
+#pragma unroll
+        for (int q = 0; q < GPR * 8; ++q) pin(resid[q]);
+      }
+      float row_scale = norm_row_scale(p, row);
+      pin(row_scale);
+      float ss_acc = 0.0f;
+      bool got = have && mbar_wait(&tfull[0], 0, abort_flag, p.err, kErrTimeoutEpilogue);
+      got = named_barrier_and(2, 128, got);
+      tc_fence_after_sync();
+      // Barrier 1: every CTA of the cluster has finished its MMAs, so their TMA rings are free
+      // to receive.  Rank j's ring holds, per sending rank (slot), its partial of j's groups in
+      // the layout [slot][group][16-byte column quad][row][4], conflict-free for a warp's rows.
+      cluster_sync();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+      if (got) {
+#pragma unroll 1
+        for (int j = 0; j < KS; ++j) {
+          if (j == static_cast<int>(kslice)) continue;
+          const int slot = static_cast<int>(kslice) < j ? static_cast<int>(kslice) : static_cast<int>(kslice) - 1;
+          const uint32_t dst_base = mapa_shared(smem_u32(smem), static_cast<uint32_t>(j)) +
+                                    static_cast<uint32_t>(slot * SLOT_BYTES + row_in_tile * 16);
+#pragma unroll 1
+          for (int gi = 0; gi < GPR; ++gi) {
+            int c0, c1;
+            group_chunks<EPI, BN>(j * GPR + gi, c0, c1);
+            uint32_t r0[32], r1[32];
+            tmem_ld32(t_row + c0 * 32, r0);
+            tmem_ld32(t_row + c1 * 32, r1);
+            tmem_ld_wait(r0);
+            tmem_ld_wait(r1);
+            const uint32_t dst = dst_base + static_cast<uint32_t>(gi * 16 * BM * 16);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              st_shared_cluster_v4(dst + q * (BM * 16),
+                                   make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
+                                               __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3])));
+              st_shared_cluster_v4(dst + (8 + q) * (BM * 16),
+                                   make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                                               __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3])));
+            }
+          }
+        }
+      }
+      cluster_sync();  // barrier 2: every partial slice has landed
+      if (got) {
+        uint8_t* box = nullptr;
+#pragma unroll
+        for (int gi = 0; gi < GPR; ++gi) {
+          const int g = g0 + gi;
+          int c0, c1;
+          group_chunks<EPI, BN>(g, c0, c1);
+          float v[64];
+#pragma unroll
+          for (int j = 0; j < 64; ++j) v[j] = 0.0f;
+          // Sum the K slices in rank order (deterministic).
+#pragma unroll 1
+          for (int src = 0; src < KS; ++src) {
+            if (src == static_cast<int>(kslice)) {
+              uint32_t r0[32], r1[32];
+              tmem_ld32(t_row + c0 * 32, r0);
+              tmem_ld32(t_row + c1 * 32, r1);
+              tmem_ld_wait(r0);
+              tmem_ld_wait(r1);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                v[j] += __uint_as_float(r0[j]);
+                v[32 + j] += __uint_as_float(r1[j]);
+              }
+            } else {
+              const int slot = src < static_cast<int>(kslice) ? src : src - 1;
+              const uint8_t* src_buf = smem + slot * SLOT_BYTES + gi * 16 * BM * 16 + row_in_tile * 16;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 lo = *reinterpret_cast<const float4*>(src_buf + q * (BM * 16));
+                const float4 hi = *reinterpret_cast<const float4*>(src_buf + (8 + q) * (BM * 16));
+                v[4 * q] += lo.x; v[4 * q + 1] += lo.y; v[4 * q + 2] += lo.z; v[4 * q + 3] += lo.w;
+                v[32 + 4 * q] += hi.x; v[32 + 4 * q + 1] += hi.y; v[32 + 4 * q + 2] += hi.z; v[32 + 4 * q + 3] += hi.w;
+              }
+            }
+          }
+          uint8_t* box2 = nullptr;
+          if (EPI == EPI_RESID && p.xw_out) st.acquire_both(box, box2);
+          else box = st.acquire();
+          epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s, row_scale,
+                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? gi * 8 : 0) : nullptr, ss_acc, st,
+                                  box, box2);
+          st.store(box, &tm_out, sg.n_tile * BN + g * 64, box_y, p.M);
+          if (EPI == EPI_RESID && p.xw_out) st.store(box2, &tm_xw, sg.n_tile * BN + g * 64, box_y, p.M);
+        }
+        if (EPI == EPI_RESID && p.xw_out && row < p.M)
+          p.ss_out[static_cast<size_t>(row) * p.ss_parts + sg.n_tile * KS + static_cast<int>(kslice)] = ss_acc;
+      }
+    }
+    while (KS == 1 && walk.next(p, sg)) {
       const int row0 = sg.m_tile * BMT + static_cast<int>(rank) * BM;  // this CTA's rows of the tile
       const int row = row0 + row_in_tile;
       const int box_y = row0 + quad * 32;
@@ -602,8 +734,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       // the partial-tile path uses a named barrier).
       if (!named_barrier_and(2, 128, got)) break;
       tc_fence_after_sync();
-      const uint32_t t_row =
-          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::ACC_COLS);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
       if (!finisher_or_full) {
         // Contributor to a tile finished by another CTA: park the partial, release it, move on.
         float* slot = partial_slot<BN>(p, blockIdx.x);
@@ -612,20 +743,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           uint32_t r[32];
           tmem_ld32(t_row + c * 32, r);
           tmem_ld_wait(r);
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-#pragma unroll
-          for (int ch = 1; ch < C::CH; ++ch) {
-            tmem_ld32(t_row + ch * BN + c * 32, r);
-            tmem_ld_wait(r);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(r[j]);
-          }
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(slot + ((c * 8 + q) * BM + row_in_tile) * 4) =
-                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                            __uint_as_float(r[4 * q + 3]));
         }
         tc_fence_before_sync();
         release_acc(acc);
@@ -667,18 +789,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             v[j] = __uint_as_float(r0[j]);
             v[32 + j] = __uint_as_float(r1[j]);
           }
-#pragma unroll
-          for (int ch = 1; ch < C::CH; ++ch) {
-            tmem_ld32(t_row + ch * BN + c0 * 32, r0);
-            tmem_ld32(t_row + ch * BN + c1 * 32, r1);
-            tmem_ld_wait(r0);
-            tmem_ld_wait(r1);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              v[j] += __uint_as_float(r0[j]);
-              v[32 + j] += __uint_as_float(r1[j]);
-            }
-          }
+
           if (split) {
 #pragma unroll 2
             for (int cc = c_first + 1; cc <= c_last; ++cc) {
@@ -799,12 +910,13 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
   }
 }
 
-template <int BN, int EPI, bool GATHER, bool PAIR = false>
+template <int BN, int EPI, bool GATHER, bool PAIR = false, int KS = 1>
 cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   using C = TileCfg<BN, PAIR>;
   static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
-  auto kern = k_gemm_tc<BN, EPI, GATHER, PAIR>;
+  auto kern = k_gemm_tc<BN, EPI, GATHER, PAIR, KS>;
   if (PAIR && (plan.grid & 1)) return cudaErrorInvalidValue;
+  if (KS > 1 && (plan.grid % KS || plan.kb_total % KS || plan.grid != plan.work * KS)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -846,8 +958,9 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   const CUtensorMap& ta = GATHER ? *a.tm_b : *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
   const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
-  if constexpr (PAIR)
-    return launch_pdl_pair(kern, dim3(plan.grid), dim3(192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
+  if constexpr (PAIR || KS > 1)
+    return launch_pdl_cluster(kern, dim3(plan.grid), dim3(192), C::SMEM, s, PAIR ? 2u : static_cast<unsigned>(KS), ta,
+                              *a.tm_b, tb2, *a.tm_out, txw, p);
   else
     return launch_pdl(kern, dim3(plan.grid), dim3(GATHER ? 320 : 192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
 }
@@ -855,6 +968,18 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
 // Tile widths each epilogue supports (the planner only picks these).
 template <int EPI, bool GATHER>
 cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
+  if (plan.ks > 1) {
+    // Cluster split-K: 256-column residual tiles.
+    if constexpr (!GATHER && EPI == EPI_RESID) {
+      if (plan.bn != 256 || plan.pair) return cudaErrorInvalidValue;
+      switch (plan.ks) {
+        case 2: return launch_one<256, EPI, false, false, 2>(plan, a, s);
+        case 4: return launch_one<256, EPI, false, false, 4>(plan, a, s);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+    return cudaErrorInvalidValue;
+  }
   if (plan.pair) {
     // CTA pairs: 256-row tiles, no A-gather.
     if constexpr (GATHER || EPI == EPI_STORE) {
@@ -931,6 +1056,13 @@ double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_o
 // waves) they lose by 1-60 %, mostly to split-tile fix-ups.
 constexpr int kPairMinWaves = 5;
 
+// Cost of one partial slice exchanged through distributed shared memory in a cluster split-K
+// (128 rows x 256 / ks fp32 written to a peer's ring and summed there, with the two cluster
+// barriers and the cluster launch).  Fitted on B200 at M = 784: 4-way split of the down
+// projection (K = 2816) 15.1 us vs 16.0 us for the best single-CTA plan; of the output
+// projection (K = 1024) 12.8 us vs 9.7 us.
+constexpr double kExchangeCycles = 4200.0;
+
 }  // namespace
 
 GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes);
@@ -979,6 +1111,7 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
         partial <= max_partial_bytes) {
       best.bn = 256;
       best.pair = 1;
+      best.ks = 1;
       best.splits = contrib;
       best.tiles_m = tiles_m;
       best.tiles_n = tiles_n;
@@ -1023,6 +1156,7 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
         best_cost = cost;
         best.bn = bn;
         best.pair = 0;
+        best.ks = 1;
         best.splits = contrib;
         best.tiles_m = tiles_m;
         best.tiles_n = tiles_n;
@@ -1031,6 +1165,30 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
         best.grid = grids[gi];
         best.partial_bytes = partial;
         best.counters = contrib > 1 ? static_cast<int>(tiles) : 0;
+      }
+    }
+  }
+  // Cluster split-K for 256-column residual tiles: full-rate N = 256 MMAs even when there are
+  // too few such tiles for the SMs, without the global-memory split-tile fix-up.
+  if (epi == EPI_RESID && n_out % 256 == 0) {
+    const long long tiles = static_cast<long long>(tiles_m) * (n_out / 256);
+    for (int ks : {2, 4}) {
+      if (kb_total % ks || tiles * ks > num_sms) continue;
+      const double cost =
+          (kb_total / ks) * kblock_cycles(256) + 2000.0 + 12.0 * (256 / ks) + kExchangeCycles * (ks - 1);
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
+        best.bn = 256;
+        best.pair = 0;
+        best.ks = ks;
+        best.splits = 1;
+        best.tiles_m = tiles_m;
+        best.tiles_n = n_out / 256;
+        best.kb_total = kb_total;
+        best.work = static_cast<int>(tiles);
+        best.grid = static_cast<int>(tiles * ks);
+        best.partial_bytes = 0;
+        best.counters = 0;
       }
     }
   }

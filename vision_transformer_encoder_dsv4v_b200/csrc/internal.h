@@ -19,11 +19,17 @@ enum Epi : int {
 struct GemmPlan {
   int bn;        // MMA N per tile (SWIGLU: gate + up halves)
   int pair;      // 1: 256-row tiles on CTA pairs (tcgen05 cta_group::2), grid even; 0: 128-row tiles
+  int ks;        // > 1 (residual epilogue only): each tile is split along K over a cluster of ks
+                 // CTAs, reduced through distributed shared memory (bn = 256; each CTA finishes
+                 // 256 / ks columns)
   int splits;    // K splits per tile (fix-up by the last finisher)
   int tiles_m, tiles_n, kb_total, work, grid;
   size_t partial_bytes;  // fp32 scratch for split tiles
   int counters;          // tile counters needed (split tiles only)
 };
+
+// Row partial sums of x^2 a residual GEMM with this plan writes per row (one per column slice).
+inline int norm_parts_of(const GemmPlan& p) { return p.tiles_n * (p.ks > 1 ? p.ks : 1); }
 
 // Chooses tile width, CTA pairing and split count for a GEMM of this shape on `num_sms` SMs;
 // plans whose split-tile partials exceed max_partial_bytes are not considered.
