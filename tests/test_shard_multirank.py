@@ -16,6 +16,13 @@ from vision_transformer_encoder_dsv4v_b200 import shard
 GRIDS = [(3, 5), (2, 2), (4, 6), (1, 7), (5, 1), (3, 3)]
 
 
+def test_token_ranges_follow_the_padded_windows():
+    assert shard.image_tokens(3, 5, 2) == 6 and shard.image_tokens(4, 6, 2) == 6
+    assert shard.image_tokens(1, 7, 2) == 4 and shard.image_tokens(28, 28, 2) == 196
+    rng = shard.token_ranges([(3, 5), (2, 2), (27, 37)], 2)
+    assert rng == [(0, 6), (6, 7), (7, 7 + 14 * 19)]
+
+
 def test_shard_covers_every_image_once_and_balances():
     for world in (1, 2, 3, 4, 8):
         parts = shard.shard_images(GRIDS, world, 16, 32)
@@ -54,10 +61,17 @@ def _worker(rank, world, port, out_q):
             for a, b, blk in part:
                 full[a:b] = blk
         ref = O.tower_forward(x, [layer], None, GRIDS, nh)
+        # aligner on each rank's images, then the library's all-gather(v) of the tokens
+        wa = 0.1 * rng.normal(size=(24, 4 * d))
+        za = O.aligner_forward(y, wa, my_grids, 2)[0] if my_grids else np.zeros((0, 24))
+        tok = shard.gather_tokens(torch.from_numpy(np.ascontiguousarray(za)), GRIDS, 2, world, rank,
+                                  vision_dim=d, mlp_hidden=f)
+        tok_ref = O.aligner_forward(ref, wa, GRIDS, 2)[0]
+        tok_err = float(np.abs(tok.numpy() - tok_ref).max())
         # the benchmark's max-over-ranks reduction of per-rank times
         t = torch.tensor([float(rank + 1)])
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        out_q.put((rank, float(np.abs(full - ref).max()), float(t.item())))
+        out_q.put((rank, max(float(np.abs(full - ref).max()), tok_err), float(t.item())))
     finally:
         dist.destroy_process_group()
 

@@ -35,3 +35,52 @@ def rank_batch(grids, world_size: int, rank: int, vision_dim: int = 1024, mlp_hi
     for h, w in grids:
         cu.append(cu[-1] + h * w)
     return [grids[i] for i in idx], [(cu[i], cu[i + 1]) for i in idx]
+
+
+def image_tokens(n_h: int, n_w: int, r: int) -> int:
+    """Aligner tokens of one image: the grid padded to multiples of r, one token per window."""
+    return -(-n_h // r) * -(-n_w // r)
+
+
+def token_ranges(grids, r: int):
+    """(start, end) of each image's tokens in the packed aligner output of the full batch."""
+    out, t = [], 0
+    for h, w in grids:
+        n = image_tokens(h, w, r)
+        out.append((t, t + n))
+        t += n
+    return out
+
+
+def gather_tokens(local, grids, r: int, world_size: int, rank: int, group=None,
+                  vision_dim: int = 1024, mlp_hidden: int = 2816):
+    """All-gather(v) of the per-rank aligner outputs into the full batch's packed token order.
+
+    `local` is this rank's [T_rank, E] output for the images `rank_batch` gave it (in that order);
+    the result is the [T, E] output of the whole batch on every rank.  One collective: each rank
+    pads its block to the largest rank's token count, `all_gather` moves the blocks (NCCL over
+    NVLink on GPUs, gloo on CPU), and each image's rows are copied to their place in image order.
+    """
+    import torch
+    import torch.distributed as dist
+
+    parts = shard_images(grids, world_size, vision_dim, mlp_hidden)
+    counts = [sum(image_tokens(*grids[i], r) for i in p) for p in parts]
+    if local.shape[0] != counts[rank]:
+        raise ValueError(f"rank {rank} holds {local.shape[0]} tokens, expected {counts[rank]}")
+    width = local.shape[1]
+    t_max = max(counts) if counts else 0
+    padded = local.new_zeros((t_max, width))
+    padded[: local.shape[0]] = local
+    blocks = [torch.empty_like(padded) for _ in range(world_size)]
+    dist.all_gather(blocks, padded, group=group)
+    ranges = token_ranges(grids, r)
+    total = ranges[-1][1] if ranges else 0
+    out = local.new_empty((total, width))
+    for k, p in enumerate(parts):
+        o = 0
+        for i in p:
+            a, b = ranges[i]
+            out[a:b] = blocks[k][o: o + (b - a)]
+            o += b - a
+    return out
