@@ -291,6 +291,9 @@ def run_ours(args):
     # ---- kernel timing pass: the same step as component calls, with events around each launch
     kern = kernel_timing(A, torch, cfg, batch, wl, lw, fnw, wa, x0, x, out, ws, stream, flush, args.steps)
 
+    # ---- the step before the tower: patch embedding of the same patches (14 x 14 RGB patches)
+    extras = {"patch_embed": patch_embed_timing(A, torch, cfg, wl, stream, flush, args.steps)}
+
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     x_host = x0.cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -341,7 +344,7 @@ def run_ours(args):
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) patch states, N(0,0.02) "
                 "random-init weights of the tower's shape)", "config": cfgd,
                 "tflops": tflops, "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms),
-                "roofline": roof, "kernels": kern["all"], "cpu_baseline": cpu,
+                "roofline": roof, "kernels": kern["all"], "extras": extras, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x0.numel() * 2,
                         "d2h_bytes_per_step": out.numel() * 2,
                         "path": "dsv4v_tower_forward + dsv4v_aligner_forward direct C-ABI calls (no graph), "
@@ -396,6 +399,44 @@ def kernel_timing(A, torch, cfg, batch, wl, lw, fnw, wa, x0, x, out, ws, stream,
         res[k] = {"launches": len(ts), "avg_us": avg_us, "total_ms": sum(ts), "tflops": flops[k] / (avg_us * 1e-6) / 1e12}
     dom_name = max(kinds, key=lambda k: res[k]["total_ms"])
     return {"all": res, "dominant": {"name": dom_name, **res[dom_name]}}
+
+
+def patch_embed_timing(A, torch, cfg, wl, stream, flush, steps, patch=14):
+    """dsv4v_patch_embed on the workload's patches (random bf16 pixels, 14 x 14 patches: K = 588
+    with rows padded to 592 elements, with a bias): CUDA events around a CUDA-graph replay of
+    20 calls, L2 flushed between replays.  Not part of the tower step above."""
+    P, D = wl.n_patches, wl.vision_dim
+    k = 3 * patch * patch
+    ld = (k + 7) // 8 * 8
+    g = torch.Generator(device="cuda").manual_seed(7)
+    pix = torch.randn(P, ld, device="cuda", generator=g).to(torch.bfloat16)
+    w = (torch.randn(D, ld, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    bias = torch.randn(D, device="cuda", generator=g)
+    out = torch.empty(P, D, dtype=torch.bfloat16, device="cuda")
+    reps = 20
+    with torch.cuda.stream(stream):
+        A.dsv4v_patch_embed(cfg, P, patch, patch, pix, w, bias, out, ld, ld, stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(reps):
+            A.dsv4v_patch_embed(cfg, P, patch, patch, pix, w, bias, out, ld, ld, stream=stream.cuda_stream)
+    times = []
+    for i in range(steps + 2):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+        stream.synchronize()
+        if i >= 2:
+            times.append(a.elapsed_time(b) / reps)
+    avg_ms = sum(times) / len(times)
+    flops = 2.0 * P * k * D
+    return {"avg_us": avg_ms * 1e3, "tflops": flops / (avg_ms * 1e-3) / 1e12, "patch": patch, "k": k, "ld": ld,
+            "bias": True, "launches_per_call": 1,
+            "note": "standalone, 20 calls per graph replay; the step before the tower, not in value"}
 
 
 def load_peaks():

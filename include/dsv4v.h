@@ -201,6 +201,22 @@ dsv4v_status dsv4v_linear_residual(const dsv4v_config* cfg, int64_t rows, int k,
                                    const void* a, const void* w, void* x, void* workspace,
                                    size_t ws_bytes, void* stream);
 
+/* Patch embedding ([vision-API, DeepseekV4VisionPatchEmbed]: a linear embedding of flattened
+ * RGB patches, [patches, 3, patch_h, patch_w] -> [patches, vision_dim], through its `proj`):
+ * x_out[p, :] = patches[p, :] . w_proj^T (+ bias), where row p of `patches` is the patch in its
+ * own (channel, row, column) order, K = 3 * patch_h * patch_w values.  The pages state neither
+ * the patch size nor whether `proj` has a bias: both are arguments (bias NULL = none).
+ *   patches: device [n_patches, ld_patches] (config dtype; columns >= K ignored);
+ *   w_proj:  device [vision_dim, ld_w], K columns used;  bias: device fp32 [vision_dim] or NULL;
+ *   x_out:   device [n_patches, vision_dim], config dtype.
+ *   ld_patches / ld_w: row strides in elements (0 = K).  The bf16 path needs them to be
+ *   multiples of 8 (16-byte rows for TMA; K = 588 for 14 x 14 patches, e.g. stride 592) and
+ *   returns DSV4V_ERR_UNSUPPORTED otherwise; the fp32 path needs them equal to K.
+ * Needs no workspace.  patch_h, patch_w in [1, 64]; all pointers 16-byte aligned. */
+dsv4v_status dsv4v_patch_embed(const dsv4v_config* cfg, int64_t n_patches, int patch_h, int patch_w,
+                               const void* patches, int64_t ld_patches, const void* w_proj,
+                               int64_t ld_w, const float* bias, void* x_out, void* stream);
+
 /* SwiGLU gate/up ([vision-API, DeepseekV4VisionMLP]): h = silu(y . w_gate^T) * (y . w_up^T),
  * silu(z) = z / (1 + exp(-z)).  y: device [rows, D]; h: device [rows, F]. */
 dsv4v_status dsv4v_swiglu(const dsv4v_config* cfg, int64_t rows, const void* y,

@@ -197,6 +197,20 @@ def tower_forward(x, layers, final_norm_w, grids, n_heads: int, rope_theta: floa
 # grid position (r*i + a, r*j + b) -> channel (a*r + b)*D + c; tokens are row-major over (i, j);
 # the projection is one bias-free linear r*r*D -> E.
 # --------------------------------------------------------------------------------------------
+def patch_embed(patches, w_proj, bias=None) -> np.ndarray:
+    """[vision-API, DeepseekV4VisionPatchEmbed]: a linear embedding of flattened RGB patches,
+    [patches, 3, patch_h, patch_w] -> [patches, vision_dim], through the module's `proj`.
+    READING 13: each patch is flattened in its own (channel, row, column) order, i.e. feature
+    index c * patch_h * patch_w + i * patch_w + j, and `proj` is a Linear [D, 3 * patch_h *
+    patch_w]; whether it has a bias is not stated, so the bias is optional (None = none)."""
+    p = _f64(patches)
+    flat = p.reshape(p.shape[0], -1)
+    y = flat @ _f64(w_proj).T
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return y
+
+
 def aligner_merge(x, grids, r: int):
     """Returns the merged token matrix [T, r*r*D] and the token offsets [n_images + 1]."""
     x = _f64(x)

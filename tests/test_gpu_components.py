@@ -202,3 +202,37 @@ def test_qkv_rope_pair_tiles():
     q, k, v = O.qkv_rope(y.values[r], wqkv.values, c_o[r].astype(np.float32), s_o[r].astype(np.float32), 16)
     want = np.concatenate([q.reshape(len(r), -1), k.reshape(len(r), -1), v.reshape(len(r), -1)], axis=1)
     assert_bf16_close(to_np(qkv)[r], want, abs_floor=2e-5)
+
+
+# Patch embedding (next step before the tower): flattened (3, p, p) patches through `proj`.
+@pytest.mark.parametrize("rows,patch,bias,ld", [(784, 16, True, 0), (784, 14, False, 592), (1, 14, True, 592),
+                                                (3562, 16, False, 0), (130, 14, True, 600)])
+def test_patch_embed_bf16(rows, patch, bias, ld):
+    cfg = cfg_bf16()
+    k = 3 * patch * patch
+    width = ld if ld else k
+    pix = random_bf16((rows, width), 1.0, seed=91)
+    w = random_bf16((1024, width), 0.02, seed=92)
+    if width > k:  # the padding past K must never be read: make it loud
+        for t in (pix, w):
+            t.bits[:, k:] = synth.bf16_bits(np.full((t.bits.shape[0], width - k), 1.0e4, dtype=np.float32))
+            t.values[:, k:] = 1.0e4
+    b = np.random.default_rng(93).normal(size=1024).astype(np.float32) if bias else None
+    out = torch.empty(rows, 1024, dtype=torch.bfloat16, device="cuda")
+    A.dsv4v_patch_embed(cfg, rows, patch, patch, dev(pix), dev(w), f32(b) if bias else None, out, ld, ld)
+    assert A.dsv4v_device_error() == 0
+    want = O.patch_embed(pix.values[:, :k].reshape(rows, 3, patch, patch), w.values[:, :k], b)
+    assert_bf16_close(to_np(out), want, abs_floor=2e-5)
+
+
+def test_patch_embed_f32():
+    cfg = A.make_config(64, 4, 128, 2, 128, 1, 1e-6, 10000.0, A.DSV4V_F32)
+    rows, patch = 24, 4
+    rng = np.random.default_rng(94)
+    pix = rng.normal(size=(rows, 3, patch, patch)).astype(np.float32)
+    w = (0.1 * rng.normal(size=(64, 3 * patch * patch))).astype(np.float32)
+    b = rng.normal(size=64).astype(np.float32)
+    out = torch.empty(rows, 64, dtype=torch.float32, device="cuda")
+    A.dsv4v_patch_embed(cfg, rows, patch, patch, f32(pix.reshape(rows, -1)), f32(w), f32(b), out)
+    want = O.patch_embed(pix, w, b)
+    assert np.abs(out.cpu().numpy().astype(np.float64) - want).max() < 1e-4

@@ -323,3 +323,26 @@ def test_aligner_projection_and_token_counts():
 
 def test_cu_from_grids():
     assert list(O.cu_from_grids([(27, 37), (37, 27), (10, 78), (112, 7)])) == [0, 999, 1998, 2778, 3562]
+
+
+def test_patch_embed_flatten_order_and_bias():
+    """One-hot pixels pin the flatten order (channel, row, column); zero pixels give the bias;
+    the map is linear."""
+    rng = np.random.default_rng(5)
+    ph, pw, d = 3, 4, 7
+    w = rng.normal(size=(d, 3 * ph * pw))
+    b = rng.normal(size=d)
+    for c, i, j in [(0, 0, 0), (1, 2, 3), (2, 1, 0), (2, 2, 3)]:
+        x = np.zeros((1, 3, ph, pw))
+        x[0, c, i, j] = 1.0
+        np.testing.assert_allclose(O.patch_embed(x, w)[0], w[:, c * ph * pw + i * pw + j], rtol=0, atol=0)
+        np.testing.assert_allclose(O.patch_embed(x, w, b)[0], w[:, c * ph * pw + i * pw + j] + b, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(O.patch_embed(np.zeros((2, 3, ph, pw)), w, b), np.stack([b, b]), rtol=0, atol=0)
+    x1, x2 = rng.normal(size=(5, 3, ph, pw)), rng.normal(size=(5, 3, ph, pw))
+    np.testing.assert_allclose(O.patch_embed(2.0 * x1 - x2, w), 2.0 * O.patch_embed(x1, w) - O.patch_embed(x2, w),
+                               rtol=1e-12, atol=1e-12)
+    # one patch written out by hand: 3 x 1 x 1 pixels (r, g, b) = (1, 2, 3), w = rows [1 0 0], [1 1 1]
+    np.testing.assert_allclose(O.patch_embed(np.array([[[[1.0]], [[2.0]], [[3.0]]]]),
+                                             np.array([[1.0, 0.0, 0.0], [1.0, 1.0, 1.0]]), np.array([0.5, -1.0])),
+                               [[1.5, 5.0]], rtol=0, atol=0)
+

@@ -75,10 +75,10 @@ EncodeTiledFn encode_fn() {
 
 struct MapKey {
   const void* ptr;
-  int64_t rows, cols;
+  int64_t rows, cols, ld;
   int box_rows;
   bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+    return ptr == o.ptr && rows == o.rows && cols == o.cols && ld == o.ld && box_rows == o.box_rows;
   }
 };
 struct MapKeyHash {
@@ -87,16 +87,19 @@ struct MapKeyHash {
     h ^= static_cast<size_t>(k.rows) * 0x9E3779B97F4A7C15ull;
     h ^= static_cast<size_t>(k.cols) * 0xC2B2AE3D27D4EB4Full + (h << 6);
     h ^= static_cast<size_t>(k.box_rows) * 0x165667B19E3779F9ull + (h >> 2);
+    h ^= static_cast<size_t>(k.ld) * 0x27D4EB2F165667C5ull + (h << 3);
     return h;
   }
 };
 
-// bf16 row-major [rows, cols] matrix, boxes of 64 columns (128 B, 128-byte swizzle) x box_rows
-// rows; reads past the end return zeros.  Descriptors depend only on these values, so they are
-// cached per thread.
-bool bf16_map(const void* ptr, int64_t rows, int64_t cols, int box_rows, CUtensorMap* out) {
+// bf16 row-major [rows, cols] matrix with row stride ld elements (0: cols; a multiple of 8),
+// boxes of 64 columns (128 B, 128-byte swizzle) x box_rows rows; reads past the end of a row or
+// of the matrix return zeros.  Descriptors depend only on these values, so they are cached per
+// thread.
+bool bf16_map(const void* ptr, int64_t rows, int64_t cols, int box_rows, CUtensorMap* out, int64_t ld = 0) {
   thread_local std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
-  MapKey key{ptr, rows, cols, box_rows};
+  if (ld == 0) ld = cols;
+  MapKey key{ptr, rows, cols, ld, box_rows};
   auto it = cache.find(key);
   if (it != cache.end()) {
     *out = it->second;
@@ -106,7 +109,7 @@ bool bf16_map(const void* ptr, int64_t rows, int64_t cols, int box_rows, CUtenso
   if (!fn) return false;
   CUtensorMap m;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -286,14 +289,20 @@ struct NormFold {
   int ss_parts = 0;
 };
 
+// Row strides of A and B when they are not K (0: K), and the STORE epilogue's bias.
+struct GemmExtra {
+  int64_t lda = 0, ldb = 0;
+  const float* bias = nullptr;
+};
+
 dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* a, int64_t M, int K, const void* b,
                        const void* b2, int n_out, void* out, const void* resid, const float* cos = nullptr,
                        const float* sin = nullptr, bool gather = false, const int32_t* gsrc = nullptr,
-                       const void* gx = nullptr, const NormFold& nf = NormFold()) {
+                       const void* gx = nullptr, const NormFold& nf = NormFold(), const GemmExtra& ex = GemmExtra()) {
   if (M == 0) return DSV4V_OK;
   const int box_b = (epi == EPI_SWIGLU || plan.pair) ? plan.bn / 2 : plan.bn;
   CUtensorMap ta, tb, tb2, t_out, t_xw;
-  if ((!gather && !bf16_map(a, M, K, 128, &ta)) || !bf16_map(b, n_out, K, box_b, &tb) ||
+  if ((!gather && !bf16_map(a, M, K, 128, &ta, ex.lda)) || !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
       (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)) || !bf16_map(out, M, n_out, 32, &t_out) ||
       (nf.xw_out && !bf16_map(nf.xw_out, M, n_out, 32, &t_xw)))
     return DSV4V_ERR_CUDA;
@@ -328,6 +337,7 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.xw_w = nf.xw_w;
   g.ss_out = nf.ss_out;
   g.ss_parts = nf.ss_parts;
+  g.bias = ex.bias;
   return cuda_status(launch_gemm_tc(epi, gather, plan, g, c.stream));
 }
 
@@ -718,6 +728,40 @@ dsv4v_status dsv4v_swiglu(const dsv4v_config* cfg, int64_t rows, const void* y, 
                                        static_cast<int>(rows), s.F, s.D, c.stream));
   DSV4V_TRY(reset_counters(c));
   return gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, y, rows, s.D, w_gate, w_up, s.F, h, nullptr);
+}
+
+dsv4v_status dsv4v_patch_embed(const dsv4v_config* cfg, int64_t n_patches, int patch_h, int patch_w,
+                               const void* patches, int64_t ld_patches, const void* w_proj, int64_t ld_w,
+                               const float* bias, void* x_out, void* stream) {
+  Ctx c;
+  DSV4V_TRY(prepare_rows(cfg, n_patches, nullptr, 0, stream, false, c));
+  if (patch_h <= 0 || patch_w <= 0 || patch_h > 64 || patch_w > 64) return DSV4V_ERR_INVALID_ARG;
+  const int K = 3 * patch_h * patch_w;
+  if (ld_patches == 0) ld_patches = K;
+  if (ld_w == 0) ld_w = K;
+  if (ld_patches < K || ld_w < K) return DSV4V_ERR_INVALID_ARG;
+  if (n_patches == 0) return DSV4V_OK;
+  if (!patches || !w_proj || !x_out || !aligned16(patches) || !aligned16(w_proj) || !aligned16(x_out) ||
+      (bias && !aligned16(bias)))
+    return DSV4V_ERR_INVALID_ARG;
+  const Shape& s = c.s;
+  if (!s.bf16) {
+    if (ld_patches != K || ld_w != K) return DSV4V_ERR_UNSUPPORTED;
+    return cuda_status(launch_gemm_f32(EPI_STORE, static_cast<const float*>(patches), static_cast<const float*>(w_proj),
+                                       nullptr, static_cast<float*>(x_out), nullptr, static_cast<int>(n_patches), s.D,
+                                       K, c.stream, bias));
+  }
+  // TMA rows start on 16-byte boundaries: strides in whole groups of 8 bf16.
+  if (ld_patches % 8 || ld_w % 8) return DSV4V_ERR_UNSUPPORTED;
+  // Whole tiles only (no split-tile scratch), so the call needs no workspace.
+  const GemmPlan plan = plan_gemm(EPI_STORE, static_cast<int>(n_patches), s.D, K, c.dev.sms, 0);
+  if (plan.bn == 0) return DSV4V_ERR_UNSUPPORTED;
+  GemmExtra ex;
+  ex.lda = ld_patches;
+  ex.ldb = ld_w;
+  ex.bias = bias;
+  return gemm_bf16(c, EPI_STORE, plan, patches, n_patches, K, w_proj, nullptr, s.D, x_out, nullptr, nullptr, nullptr,
+                   false, nullptr, nullptr, NormFold(), ex);
 }
 
 dsv4v_status dsv4v_device_error(void* stream) {

@@ -76,6 +76,7 @@ struct Params {
   const float* xw_w;
   float* ss_out;
   int ss_parts;
+  const float* bias;
 };
 
 // ---------------------------------------------------------------------------- stream-K ranges
@@ -205,6 +206,19 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
           const float x1 = v[j], x2 = v[32 + j];
           v[j] = x1 * rot_c[j] - x2 * rot_s[j];
           v[32 + j] = x2 * rot_c[j] + x1 * rot_s[j];
+        }
+      }
+    }
+    if constexpr (EPI == EPI_STORE) {
+      if (p.bias) {
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + n_tile * BN + g * 64);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float4 bq = b4[q];
+          v[4 * q] += bq.x;
+          v[4 * q + 1] += bq.y;
+          v[4 * q + 2] += bq.z;
+          v[4 * q + 3] += bq.w;
         }
       }
     }
@@ -955,6 +969,7 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.xw_w = a.xw_w;
   p.ss_out = a.ss_out;
   p.ss_parts = a.ss_parts;
+  p.bias = a.bias;
   const CUtensorMap& ta = GATHER ? *a.tm_b : *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
   const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
@@ -1096,7 +1111,7 @@ GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms, size_t max_par
 
 GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes) {
   GemmPlan best{};
-  const int kb_total = K / BK;
+  const int kb_total = (K + BK - 1) / BK;  // a ragged last K block reads zeros past the end
   if (kb_total <= 0 || M <= 0 || num_sms <= 0) return best;
   // CTA pairs with 256-column tiles, stream-K over all SM pairs, when there is enough work.
   if (epi != EPI_STORE && n_out % (epi == EPI_SWIGLU ? 128 : 256) == 0) {

@@ -69,6 +69,7 @@ struct GemmArgs {
   const float* xw_w;
   float* ss_out;
   int ss_parts;
+  const float* bias;  // STORE: per-column fp32 bias added before rounding (NULL: none)
 };
 
 cudaError_t launch_gemm_tc(int epi, bool gather, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
@@ -112,7 +113,7 @@ cudaError_t launch_norm_prep(const void* x, const float* w, void* xw, float* ss,
 
 // ---------------------------------------------------------------------------- fp32 CUDA-core path
 cudaError_t launch_gemm_f32(int epi, const float* a, const float* b, const float* b2, float* out, const float* resid,
-                            int M, int n_out, int K, cudaStream_t s);
+                            int M, int n_out, int K, cudaStream_t s, const float* bias = nullptr);
 cudaError_t launch_rope_apply_f32(float* qkv, const float* cos, const float* sin, int64_t P, int d, int n_heads,
                                   cudaStream_t s);
 cudaError_t launch_attention_f32(const float* qkv, float* out, const int32_t* cu_dev, int n_images, int64_t P,

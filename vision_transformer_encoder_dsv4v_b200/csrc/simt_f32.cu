@@ -13,7 +13,8 @@ constexpr int T = 32;  // output tile T x T, 256 threads, 4 outputs per thread
 template <int EPI>
 __global__ void __launch_bounds__(256) k_gemm_f32(const float* __restrict__ a, const float* __restrict__ b,
                                                   const float* __restrict__ b2, float* out,
-                                                  const float* resid, int M, int n_out, int K) {
+                                                  const float* resid, int M, int n_out, int K,
+                                                  const float* __restrict__ bias) {
   __shared__ float sa[T][T + 1];
   __shared__ float sb[T][T + 1];
   __shared__ float sb2[T][T + 1];
@@ -51,6 +52,7 @@ __global__ void __launch_bounds__(256) k_gemm_f32(const float* __restrict__ a, c
     float v = acc[q];
     if (EPI == EPI_SWIGLU) v = acc[q] / (1.0f + expf(-acc[q])) * acc2[q];
     if (EPI == EPI_RESID) v += resid[o];
+    if (EPI == EPI_STORE && bias) v += bias[c];
     out[o] = v;
   }
 }
@@ -129,13 +131,13 @@ __global__ void k_gather_f32(const float* __restrict__ x, const int32_t* __restr
 }  // namespace
 
 cudaError_t launch_gemm_f32(int epi, const float* a, const float* b, const float* b2, float* out, const float* resid,
-                            int M, int n_out, int K, cudaStream_t s) {
+                            int M, int n_out, int K, cudaStream_t s, const float* bias) {
   if (M == 0) return cudaSuccess;
   dim3 grid((n_out + T - 1) / T, (M + T - 1) / T);
   switch (epi) {
-    case EPI_STORE: k_gemm_f32<EPI_STORE><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K); break;
-    case EPI_RESID: k_gemm_f32<EPI_RESID><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K); break;
-    case EPI_SWIGLU: k_gemm_f32<EPI_SWIGLU><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K); break;
+    case EPI_STORE: k_gemm_f32<EPI_STORE><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K, bias); break;
+    case EPI_RESID: k_gemm_f32<EPI_RESID><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K, nullptr); break;
+    case EPI_SWIGLU: k_gemm_f32<EPI_SWIGLU><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K, nullptr); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

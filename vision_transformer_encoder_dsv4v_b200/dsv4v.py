@@ -26,7 +26,7 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_tower_forward_profiled",
            "dsv4v_aligner_forward", "dsv4v_aligner_tokens", "dsv4v_rmsnorm", "dsv4v_qkv_rope", "dsv4v_attention",
            "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
-           "dsv4v_status_string", "dsv4v_linear_residual_noalloc")
+           "dsv4v_status_string", "dsv4v_linear_residual_noalloc", "dsv4v_patch_embed")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "dsv4v_attention": (I, [cfg, bat, P, P, P]),
             "dsv4v_linear_residual": (I, [cfg, I64, I, P, P, P, P, SZ, P]),
             "dsv4v_swiglu": (I, [cfg, I64, P, P, P, P, P, SZ, P]),
+            "dsv4v_patch_embed": (I, [cfg, I64, I, I, P, I64, P, I64, P, P, P]),
             "dsv4v_linear_residual_noalloc": (I, [cfg, I64, I, P, P, P, P]),
             "dsv4v_device_error": (I, [P]),
             "dsv4v_selftest_bounded_wait": (I, [U64, P]),
@@ -214,6 +215,15 @@ def dsv4v_linear_residual_noalloc(cfg, rows, k, a, w, x, stream=None):
 def dsv4v_swiglu(cfg, rows, y, w_gate, w_up, h, workspace, stream=None):
     _check(lib().dsv4v_swiglu(ctypes.byref(cfg), rows, _ptr(y), _ptr(w_gate), _ptr(w_up), _ptr(h), _ptr(workspace),
                               workspace.numel() if workspace is not None else 0, _stream(stream)), "dsv4v_swiglu")
+
+
+def dsv4v_patch_embed(cfg, n_patches, patch_h, patch_w, patches, w_proj, bias, x_out, ld_patches=0, ld_w=0,
+                      stream=None):
+    """x_out = patches . w_proj^T (+ bias): rows of `patches` are flattened (3, patch_h, patch_w)
+    patches with row stride ld_patches (0: 3 * patch_h * patch_w); w_proj rows have stride ld_w."""
+    _check(lib().dsv4v_patch_embed(ctypes.byref(cfg), n_patches, patch_h, patch_w, _ptr(patches), ld_patches,
+                                   _ptr(w_proj), ld_w, _ptr(bias), _ptr(x_out), _stream(stream)),
+           "dsv4v_patch_embed")
 
 
 def dsv4v_device_error(stream=None) -> int:
