@@ -292,7 +292,8 @@ def run_ours(args):
     kern = kernel_timing(A, torch, cfg, batch, wl, lw, fnw, wa, x0, x, out, ws, stream, flush, args.steps)
 
     # ---- the step before the tower: patch embedding of the same patches (14 x 14 RGB patches)
-    extras = {"patch_embed": patch_embed_timing(A, torch, cfg, wl, stream, flush, args.steps)}
+    extras = {"patch_embed": patch_embed_timing(A, torch, cfg, wl, stream, flush, args.steps),
+              "patch_merger": patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, args.steps)}
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     x_host = x0.cpu().pin_memory()
@@ -437,6 +438,51 @@ def patch_embed_timing(A, torch, cfg, wl, stream, flush, steps, patch=14):
     return {"avg_us": avg_ms * 1e3, "tflops": flops / (avg_ms * 1e-3) / 1e12, "patch": patch, "k": k, "ld": ld,
             "bias": True, "launches_per_call": 1,
             "note": "standalone, 20 calls per graph replay; the step before the tower, not in value"}
+
+
+def patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, steps):
+    """dsv4v_patch_merger_forward (the PatchMerger projector: LayerNorm per patch, r x r merge,
+    Linear + GELU, Linear) on the workload's patches, timed like patch_embed_timing.  Not part of
+    the tower step above."""
+    P, D, E, r2 = wl.n_patches, wl.vision_dim, wl.llm_dim, wl.downsample_ratio ** 2
+    T = wl.n_tokens
+    g = torch.Generator(device="cuda").manual_seed(8)
+    x = torch.randn(P, D, device="cuda", generator=g).to(torch.bfloat16)
+    ln_w = 1 + 0.1 * torch.randn(D, device="cuda", generator=g)
+    ln_b = 0.1 * torch.randn(D, device="cuda", generator=g)
+    w1 = (torch.randn(r2 * D, r2 * D, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    b1 = 0.1 * torch.randn(r2 * D, device="cuda", generator=g)
+    w2 = (torch.randn(E, r2 * D, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    b2 = 0.1 * torch.randn(E, device="cuda", generator=g)
+    out = torch.empty(T, E, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(A.dsv4v_patch_merger_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    reps = 20
+
+    def call():
+        A.dsv4v_patch_merger_forward(cfg, batch, x, ln_w, ln_b, w1, b1, w2, b2, out, ws, stream=stream.cuda_stream)
+
+    with torch.cuda.stream(stream):
+        call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(reps):
+            call()
+    times = []
+    for i in range(steps + 2):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+        stream.synchronize()
+        if i >= 2:
+            times.append(a.elapsed_time(b) / reps)
+    avg_ms = sum(times) / len(times)
+    flops = 2.0 * T * (r2 * D) * (r2 * D) + 2.0 * T * (r2 * D) * E
+    return {"avg_us": avg_ms * 1e3, "tflops": flops / (avg_ms * 1e-3) / 1e12, "tokens": T, "launches_per_call": 4,
+            "note": "standalone, 20 calls per graph replay; the alternative projector, not in value"}
 
 
 def load_peaks():

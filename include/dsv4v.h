@@ -201,6 +201,26 @@ dsv4v_status dsv4v_linear_residual(const dsv4v_config* cfg, int64_t rows, int k,
                                    const void* a, const void* w, void* x, void* workspace,
                                    size_t ws_bytes, void* stream);
 
+/* PatchMerger projector (the second aligner the pages describe: [NVFP4 model card], a trained
+ * projector that merges each 2 x 2 group of patches and maps the 4 x 1152 = 4608-dimensional
+ * representation to the 4096-dimensional token space, 40,119,040 parameters).  The parameter
+ * count fixes the structure: a LayerNorm over each patch's D features (weight and bias, 2 D),
+ * then Linear r^2 D -> r^2 D with bias, then Linear r^2 D -> E with bias
+ * (2*1152 + (4608*4608 + 4608) + (4608*4096 + 4096) = 40,119,040).  The activation between the
+ * two Linears is not stated; this library uses the exact GELU, gelu(z) = z (1 + erf(z/sqrt 2))/2.
+ *   tokens:  merged windows exactly as dsv4v_aligner_forward (r x r, row-major, zero-padded grid;
+ *            a padding slot is a zero vector after the norm);
+ *   x: device [P, D]; ln_w, ln_b: device fp32 [D] (LayerNorm eps = cfg->eps);
+ *   w1: device [r^2 D, r^2 D], b1: device fp32 [r^2 D]; w2: device [E, r^2 D], b2: device fp32 [E];
+ *   out: device [T, E], config dtype.
+ * Workspace: dsv4v_patch_merger_workspace_size bytes, 256-byte aligned. */
+size_t dsv4v_patch_merger_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch);
+dsv4v_status dsv4v_patch_merger_forward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                        const void* x, const float* ln_w, const float* ln_b,
+                                        const void* w1, const float* b1, const void* w2,
+                                        const float* b2, void* out, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
 /* Patch embedding ([vision-API, DeepseekV4VisionPatchEmbed]: a linear embedding of flattened
  * RGB patches, [patches, 3, patch_h, patch_w] -> [patches, vision_dim], through its `proj`):
  * x_out[p, :] = patches[p, :] . w_proj^T (+ bias), where row p of `patches` is the patch in its

@@ -234,6 +234,42 @@ def aligner_forward(x, w_align, grids, r: int):
     return merged @ _f64(w_align).T, cu_tok
 
 
+def layer_norm(x, weight, bias, eps: float = 1e-6) -> np.ndarray:
+    """LayerNorm over the last axis: (x - mean) / sqrt(var + eps) * weight + bias, population
+    variance.  Used by the PatchMerger projector (see patch_merger)."""
+    x = _f64(x)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * _f64(weight) + _f64(bias)
+
+
+def gelu(z) -> np.ndarray:
+    """Exact GELU, z * Phi(z) = z (1 + erf(z / sqrt 2)) / 2."""
+    z = _f64(z)
+    return 0.5 * z * (1.0 + np.vectorize(math.erf)(z / math.sqrt(2.0)))
+
+
+def patch_merger_params(d: int, r: int, e: int) -> int:
+    """Parameter count of the PatchMerger structure below: LayerNorm(d) weight and bias, Linear
+    r^2 d -> r^2 d with bias, Linear r^2 d -> e with bias."""
+    h = r * r * d
+    return 2 * d + (h * h + h) + (h * e + e)
+
+
+def patch_merger(x, grids, r: int, ln_w, ln_b, w1, b1, w2, b2, eps: float = 1e-6) -> np.ndarray:
+    """The trained projector of [NVFP4 model card] ("merges each 2x2 group of patches and maps
+    the resulting 4608-dimensional representation into the 4096-dimensional token space", 40,119,040
+    parameters).  READING 14: the parameter count fixes a LayerNorm over each patch's d features,
+    then Linear r^2 d -> r^2 d (+ bias), then Linear r^2 d -> e (+ bias) (patch_merger_params);
+    the activation between the Linears is unstated and read as the exact GELU; the windows are
+    merged exactly as aligner_merge (READING 9), a padding slot being a zero vector after the
+    norm."""
+    xn = layer_norm(x, ln_w, ln_b, eps)
+    merged, cu_tok = aligner_merge(xn, grids, r)
+    h = gelu(merged @ _f64(w1).T + _f64(b1)[None, :])
+    return h @ _f64(w2).T + _f64(b2)[None, :], cu_tok
+
+
 def encode(inp, n_layers: int | None = None):
     """Whole path for one drawn input set (vision_transformer_encoder_dsv4v_b200.synth.Inputs):
     tower (first ``n_layers`` layers) then, if drawn, final norm and aligner.  Returns

@@ -236,3 +236,51 @@ def test_patch_embed_f32():
     A.dsv4v_patch_embed(cfg, rows, patch, patch, f32(pix.reshape(rows, -1)), f32(w), f32(b), out)
     want = O.patch_embed(pix, w, b)
     assert np.abs(out.cpu().numpy().astype(np.float64) - want).max() < 1e-4
+
+
+# PatchMerger projector (the second aligner on the pages): LayerNorm per patch, r x r merge,
+# Linear + GELU, Linear.  Two GEMMs with a bf16 intermediate: relative Frobenius error <= 1e-2
+# plus an element-wise bound.
+@pytest.mark.parametrize("grids", [[(28, 28)], [(3, 5), (1, 1), (4, 6)], [(27, 37), (37, 27), (10, 78), (112, 7)]])
+def test_patch_merger_bf16(grids):
+    cfg = cfg_bf16()
+    b = A.BatchRef(grids)
+    P = b.n_patches
+    rng = np.random.default_rng(55)
+    x = random_bf16((P, 1024), 1.0, seed=56)
+    ln_w = (1 + 0.1 * rng.normal(size=1024)).astype(np.float32)
+    ln_b = (0.1 * rng.normal(size=1024)).astype(np.float32)
+    w1 = random_bf16((4096, 4096), 0.02, seed=57)
+    b1 = (0.1 * rng.normal(size=4096)).astype(np.float32)
+    w2 = random_bf16((4096, 4096), 0.02, seed=58)
+    b2 = (0.1 * rng.normal(size=4096)).astype(np.float32)
+    T = A.dsv4v_aligner_tokens(cfg, b)
+    out = torch.empty(T, 4096, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(A.dsv4v_patch_merger_workspace_size(cfg, b), dtype=torch.uint8, device="cuda")
+    A.dsv4v_patch_merger_forward(cfg, b, dev(x), f32(ln_w), f32(ln_b), dev(w1), f32(b1), dev(w2), f32(b2), out, ws)
+    assert A.dsv4v_device_error() == 0
+    want, _ = O.patch_merger(x.values, grids, 2, ln_w, ln_b, w1.values, b1, w2.values, b2, eps=1e-6)
+    got = to_np(out)
+    assert rel_fro(got, want) < 1e-2
+    assert np.abs(got - want).max() < 3e-2 * max(1.0, np.abs(want).max())
+
+
+def test_patch_merger_f32():
+    cfg = A.make_config(64, 4, 128, 2, 128, 1, 1e-6, 10000.0, A.DSV4V_F32)
+    grids = [(4, 6), (3, 5)]
+    b = A.BatchRef(grids)
+    P = b.n_patches
+    rng = np.random.default_rng(59)
+    x = rng.normal(size=(P, 64)).astype(np.float32)
+    ln_w = (1 + 0.1 * rng.normal(size=64)).astype(np.float32)
+    ln_b = (0.1 * rng.normal(size=64)).astype(np.float32)
+    w1 = (0.05 * rng.normal(size=(256, 256))).astype(np.float32)
+    b1 = (0.1 * rng.normal(size=256)).astype(np.float32)
+    w2 = (0.05 * rng.normal(size=(128, 256))).astype(np.float32)
+    b2 = (0.1 * rng.normal(size=128)).astype(np.float32)
+    T = A.dsv4v_aligner_tokens(cfg, b)
+    out = torch.empty(T, 128, dtype=torch.float32, device="cuda")
+    ws = torch.empty(A.dsv4v_patch_merger_workspace_size(cfg, b), dtype=torch.uint8, device="cuda")
+    A.dsv4v_patch_merger_forward(cfg, b, f32(x), f32(ln_w), f32(ln_b), f32(w1), f32(b1), f32(w2), f32(b2), out, ws)
+    want, _ = O.patch_merger(x, grids, 2, ln_w, ln_b, w1, b1, w2, b2, eps=1e-6)
+    assert np.abs(out.cpu().numpy().astype(np.float64) - want).max() < 1e-4

@@ -346,3 +346,56 @@ def test_patch_embed_flatten_order_and_bias():
                                              np.array([[1.0, 0.0, 0.0], [1.0, 1.0, 1.0]]), np.array([0.5, -1.0])),
                                [[1.5, 5.0]], rtol=0, atol=0)
 
+
+def test_patch_merger_structure_matches_the_stated_parameter_count():
+    """The pages give 40,119,040 parameters for the projector that merges 2x2 groups of 1152-wide
+    patches (4608) into the 4096-wide token space: only LayerNorm(1152) + two biased Linears fits."""
+    assert O.patch_merger_params(1152, 2, 4096) == 40_119_040
+    assert 4 * 1152 == 4608
+    # the near alternatives do not fit: norm over the merged 4608, or no norm, or bias-free Linears
+    h = 4608
+    assert 2 * h + (h * h + h) + (h * 4096 + 4096) != 40_119_040
+    assert (h * h + h) + (h * 4096 + 4096) != 40_119_040
+    assert 2 * 1152 + h * h + h * 4096 != 40_119_040
+
+
+def test_layer_norm_closed_forms():
+    rng = np.random.default_rng(11)
+    x = rng.normal(size=(5, 40)) * 3 + 2
+    y = O.layer_norm(x, np.ones(40), np.zeros(40), eps=0.0)
+    np.testing.assert_allclose(y.mean(axis=1), 0, atol=1e-12)
+    np.testing.assert_allclose(y.var(axis=1), 1, rtol=1e-12)
+    b = rng.normal(size=40)
+    np.testing.assert_allclose(O.layer_norm(np.full((2, 40), 3.5), rng.normal(size=40), b), np.stack([b, b]), atol=1e-12)
+    # hand value: row (1, 3): mean 2, var 1 -> (-1, 1) / sqrt(1 + eps)
+    np.testing.assert_allclose(O.layer_norm(np.array([[1.0, 3.0]]), np.array([2.0, 1.0]), np.array([0.5, 0.0]), 0.0),
+                               [[-1.5, 1.0]], atol=1e-15)
+
+
+def test_gelu_values():
+    np.testing.assert_allclose(O.gelu(np.array([0.0, 1.0, -1.0])), [0.0, 0.8413447460685429, -0.15865525393145707],
+                               rtol=1e-15, atol=1e-16)
+    z = np.linspace(-6, 6, 61)
+    np.testing.assert_allclose(O.gelu(z) - O.gelu(-z), z, atol=1e-13)     # z Phi(z) - (-z) Phi(-z) = z
+    np.testing.assert_allclose(O.gelu(np.array([10.0])), [10.0], rtol=1e-15)
+
+
+def test_patch_merger_composition_and_padding():
+    rng = np.random.default_rng(12)
+    d, r, e = 3, 2, 5
+    grids = [(3, 5), (2, 2)]
+    x = rng.normal(size=(15 + 4, d))
+    lw, lb = 1 + 0.1 * rng.normal(size=d), 0.1 * rng.normal(size=d)
+    w1, b1 = rng.normal(size=(4 * d, 4 * d)), rng.normal(size=4 * d)
+    w2, b2 = rng.normal(size=(e, 4 * d)), rng.normal(size=e)
+    out, cu = O.patch_merger(x, grids, r, lw, lb, w1, b1, w2, b2)
+    assert out.shape == (6 + 1, e) and list(cu) == [0, 6, 7]
+    # written out step by step for token (0, 2) of image 0: patches (0,4), (1,4) and two padding slots
+    xn = O.layer_norm(x, lw, lb)
+    m = np.concatenate([xn[4], np.zeros(d), xn[5 + 4], np.zeros(d)])
+    np.testing.assert_allclose(out[2], O.gelu(w1 @ m + b1) @ w2.T + b2, rtol=1e-12, atol=1e-12)
+    # identity-like first layer: w1 = I, b1 = 0 gives w2 . gelu(merged) + b2
+    out_i, _ = O.patch_merger(x, grids, r, lw, lb, np.eye(4 * d), np.zeros(4 * d), w2, b2)
+    merged, _ = O.aligner_merge(xn, grids, r)
+    np.testing.assert_allclose(out_i, O.gelu(merged) @ w2.T + b2, rtol=1e-12, atol=1e-12)
+

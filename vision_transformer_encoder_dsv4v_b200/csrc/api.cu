@@ -658,6 +658,83 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
                                      static_cast<float*>(out), nullptr, static_cast<int>(s.T), s.E, K, c.stream));
 }
 
+// Scratch of the PatchMerger projector: window index [T, r^2] int32, merged rows and hidden rows
+// [T, r^2 D] in the activation dtype.
+namespace {
+struct MergerLayout {
+  size_t src, merged, hidden, total;
+};
+MergerLayout merger_layout(const Shape& s) {
+  MergerLayout l{};
+  const size_t es = s.bf16 ? 2 : 4;
+  const size_t rows = static_cast<size_t>(s.T) * s.r * s.r;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += up256(bytes);
+    return at;
+  };
+  l.src = take(rows * 4);
+  l.merged = take(rows * s.D * es);
+  l.hidden = take(rows * s.D * es);
+  l.total = off;
+  return l;
+}
+}  // namespace
+
+size_t dsv4v_patch_merger_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch) {
+  Shape s;
+  if (check_all(cfg, batch, s) != DSV4V_OK) return 0;
+  return merger_layout(s).total;
+}
+
+dsv4v_status dsv4v_patch_merger_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x,
+                                        const float* ln_w, const float* ln_b, const void* w1, const float* b1,
+                                        const void* w2, const float* b2, void* out, void* workspace, size_t ws_bytes,
+                                        void* stream) {
+  Ctx c;
+  DSV4V_TRY(check_all(cfg, batch, c.s));
+  if (!device_info(c.dev)) return DSV4V_ERR_CUDA;
+  const Shape& s = c.s;
+  for (const void* ptr : {x, static_cast<const void*>(ln_w), static_cast<const void*>(ln_b), w1,
+                          static_cast<const void*>(b1), w2, static_cast<const void*>(b2), static_cast<const void*>(out)})
+    if (!ptr || !aligned16(ptr)) return DSV4V_ERR_INVALID_ARG;
+  const MergerLayout l = merger_layout(s);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < l.total) return DSV4V_ERR_WORKSPACE;
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.eps = cfg->eps;
+  c.ws = static_cast<uint8_t*>(workspace);
+  c.lay = Layout{};  // the GEMMs below use no split-tile scratch
+  if (s.T == 0) return DSV4V_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* src = reinterpret_cast<int32_t*>(ws + l.src);
+  void* merged = ws + l.merged;
+  void* hidden = ws + l.hidden;
+  const int r2 = s.r * s.r, K = r2 * s.D;
+  DSV4V_TRY(cuda_status(launch_aligner_index(batch->cu_patches_dev, batch->grid_hw_dev, batch->n_images, s.r, s.T, src,
+                                             c.stream)));
+  DSV4V_TRY(cuda_status(launch_ln_merge(s.bf16, x, src, ln_w, ln_b, cfg->eps, merged, s.T, r2, s.D, c.stream)));
+  if (!s.bf16) {
+    DSV4V_TRY(cuda_status(launch_gemm_f32(EPI_GELU, static_cast<const float*>(merged), static_cast<const float*>(w1),
+                                          nullptr, static_cast<float*>(hidden), nullptr, static_cast<int>(s.T), K, K,
+                                          c.stream, b1)));
+    return cuda_status(launch_gemm_f32(EPI_STORE, static_cast<const float*>(hidden), static_cast<const float*>(w2),
+                                       nullptr, static_cast<float*>(out), nullptr, static_cast<int>(s.T), s.E, K,
+                                       c.stream, b2));
+  }
+  // Whole-tile plans only: no split-tile scratch.
+  const GemmPlan p1 = plan_gemm(EPI_GELU, static_cast<int>(s.T), K, K, c.dev.sms, 0);
+  const GemmPlan p2 = plan_gemm(EPI_STORE, static_cast<int>(s.T), s.E, K, c.dev.sms, 0);
+  if (p1.bn == 0 || p2.bn == 0) return DSV4V_ERR_UNSUPPORTED;
+  GemmExtra e1, e2;
+  e1.bias = b1;
+  e2.bias = b2;
+  DSV4V_TRY(gemm_bf16(c, EPI_GELU, p1, merged, s.T, K, w1, nullptr, K, hidden, nullptr, nullptr, nullptr, false,
+                      nullptr, nullptr, NormFold(), e1));
+  return gemm_bf16(c, EPI_STORE, p2, hidden, s.T, K, w2, nullptr, s.E, out, nullptr, nullptr, nullptr, false, nullptr,
+                   nullptr, NormFold(), e2);
+}
+
 dsv4v_status dsv4v_rmsnorm(const dsv4v_config* cfg, int64_t rows, const void* x, const float* w, void* y,
                            void* stream) {
   Shape s;

@@ -124,6 +124,9 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// gelu(z) = z (1 + erf(z / sqrt 2)) / 2, the exact (erf) form.
+__device__ __forceinline__ float gelu(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
+
 // silu(z) = z / (1 + e^-z) = (z / 2) (1 + tanh(z / 2)): one MUFU op per element, ample for a bf16
 // result.
 __device__ __forceinline__ float silu(float z) {
@@ -207,6 +210,17 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
           v[j] = x1 * rot_c[j] - x2 * rot_s[j];
           v[32 + j] = x2 * rot_c[j] + x1 * rot_s[j];
         }
+      }
+    }
+    if constexpr (EPI == EPI_GELU) {
+      const float4* b4 = reinterpret_cast<const float4*>(p.bias + n_tile * BN + g * 64);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float4 bq = b4[q];
+        v[4 * q] = gelu(v[4 * q] + bq.x);
+        v[4 * q + 1] = gelu(v[4 * q + 1] + bq.y);
+        v[4 * q + 2] = gelu(v[4 * q + 2] + bq.z);
+        v[4 * q + 3] = gelu(v[4 * q + 3] + bq.w);
       }
     }
     if constexpr (EPI == EPI_STORE) {
@@ -997,7 +1011,7 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   }
   if (plan.pair) {
     // CTA pairs: 256-row tiles, no A-gather.
-    if constexpr (GATHER || EPI == EPI_STORE) {
+    if constexpr (GATHER || EPI == EPI_STORE || EPI == EPI_GELU) {
       return cudaErrorInvalidValue;
     } else if constexpr (EPI == EPI_SWIGLU) {
       if (plan.bn == 256) return launch_one<256, EPI, false, true>(plan, a, s);
@@ -1114,7 +1128,7 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
   const int kb_total = (K + BK - 1) / BK;  // a ragged last K block reads zeros past the end
   if (kb_total <= 0 || M <= 0 || num_sms <= 0) return best;
   // CTA pairs with 256-column tiles, stream-K over all SM pairs, when there is enough work.
-  if (epi != EPI_STORE && n_out % (epi == EPI_SWIGLU ? 128 : 256) == 0) {
+  if ((epi == EPI_RESID || epi == EPI_QKV_ROPE || epi == EPI_SWIGLU) && n_out % (epi == EPI_SWIGLU ? 128 : 256) == 0) {
     const int tiles_m = (M + 2 * BM - 1) / (2 * BM);
     const int tiles_n = n_out / (epi == EPI_SWIGLU ? 128 : 256);
     const long long tiles = static_cast<long long>(tiles_m) * tiles_n;
@@ -1220,6 +1234,7 @@ cudaError_t launch_gemm_tc(int epi, bool gather, const GemmPlan& plan, const Gem
     case EPI_RESID: return launch_bn<EPI_RESID, false>(plan, a, s);
     case EPI_QKV_ROPE: return launch_bn<EPI_QKV_ROPE, false>(plan, a, s);
     case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(plan, a, s);
+    case EPI_GELU: return launch_bn<EPI_GELU, false>(plan, a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -14,6 +14,7 @@ enum Epi : int {
   EPI_RESID = 1,     // out = resid + acc          (out may alias resid)
   EPI_QKV_ROPE = 2,  // out = acc, columns < rot_cols rotated pairwise (j, j + 32) per 64-wide head
   EPI_SWIGLU = 3,    // out = silu(acc_gate) * acc_up; B = gate rows, B2 = up rows
+  EPI_GELU = 4,      // out = gelu(acc + bias), gelu(z) = z (1 + erf(z / sqrt 2)) / 2
 };
 
 struct GemmPlan {
@@ -105,6 +106,11 @@ cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev,
                                  int64_t n_tokens, int32_t* src_out, cudaStream_t s, int* zero_ptr = nullptr,
                                  int zero_n = 0);
 cudaError_t launch_zero_counters(int* ptr, int n, cudaStream_t s);
+// LayerNorm of each patch row (weight and bias, fp32 math) written into its slot of the merged
+// r x r window rows: merged[t, s * d : (s + 1) * d] = LN(x[src[t * r2 + s]]), zeros where
+// src < 0.  bf16 or fp32 activations.
+cudaError_t launch_ln_merge(bool bf16, const void* x, const int32_t* src, const float* w, const float* b, float eps,
+                            void* merged, int64_t n_tokens, int r2, int d, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
 // Norm operands of the first GEMM of a block: xw = bf16(x * w) and ss[p * parts] = sum_c x[p,c]^2
 // (the other parts of a row are zero-filled); also clears zero_n counters like the kernels above.

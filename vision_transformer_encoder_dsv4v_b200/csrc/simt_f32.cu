@@ -53,6 +53,10 @@ __global__ void __launch_bounds__(256) k_gemm_f32(const float* __restrict__ a, c
     if (EPI == EPI_SWIGLU) v = acc[q] / (1.0f + expf(-acc[q])) * acc2[q];
     if (EPI == EPI_RESID) v += resid[o];
     if (EPI == EPI_STORE && bias) v += bias[c];
+    if (EPI == EPI_GELU) {
+      const float z = v + bias[c];
+      v = 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+    }
     out[o] = v;
   }
 }
@@ -138,6 +142,7 @@ cudaError_t launch_gemm_f32(int epi, const float* a, const float* b, const float
     case EPI_STORE: k_gemm_f32<EPI_STORE><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K, bias); break;
     case EPI_RESID: k_gemm_f32<EPI_RESID><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K, nullptr); break;
     case EPI_SWIGLU: k_gemm_f32<EPI_SWIGLU><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K, nullptr); break;
+    case EPI_GELU: k_gemm_f32<EPI_GELU><<<grid, 256, 0, s>>>(a, b, b2, out, resid, M, n_out, K, bias); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -173,6 +173,45 @@ __global__ void k_aligner_index(const int32_t* __restrict__ cu, const int32_t* _
     }
 }
 
+// One warp per (token, slot) row of the merged output: LayerNorm of the source patch row (mean
+// and variance in fp32, two passes over the row), or zeros for a padding slot.
+template <bool BF16>
+__global__ void k_ln_merge(const void* __restrict__ x, const int32_t* __restrict__ src, const float* __restrict__ w,
+                           const float* __restrict__ b, float eps, void* merged, int64_t n_rows, int d) {
+  grid_dependency_wait();
+  launch_dependents();
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const int32_t s = src[row];
+  auto in = [&](int c) -> float {
+    if constexpr (BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(x)[static_cast<int64_t>(s) * d + c]);
+    else return static_cast<const float*>(x)[static_cast<int64_t>(s) * d + c];
+  };
+  auto put = [&](int c, float v) {
+    if constexpr (BF16) static_cast<__nv_bfloat16*>(merged)[row * d + c] = __float2bfloat16_rn(v);
+    else static_cast<float*>(merged)[row * d + c] = v;
+  };
+  if (s < 0) {
+    for (int c = lane; c < d; c += 32) put(c, 0.0f);
+    return;
+  }
+  float sum = 0.0f;
+  for (int c = lane; c < d; c += 32) sum += in(c);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum / static_cast<float>(d);
+  float var = 0.0f;
+  for (int c = lane; c < d; c += 32) {
+    const float t = in(c) - mean;
+    var += t * t;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) var += __shfl_xor_sync(0xffffffffu, var, o);
+  const float inv = rsqrtf(var / static_cast<float>(d) + eps);
+  for (int c = lane; c < d; c += 32) put(c, (in(c) - mean) * inv * w[c] + b[c]);
+}
+
 // Clears the GEMM tile counters of a component call (one block; dependent launch, so that it
 // costs no more than a kernel boundary inside a graph, unlike a memset node).
 __global__ void k_zero_counters(int* ptr, int n) {
@@ -243,6 +282,17 @@ cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev,
   return launch_pdl(k_aligner_index, dim3(static_cast<unsigned>(blocks)), dim3(threads),
                     (n_images + 1) * sizeof(int32_t), s, cu_dev, grid_dev, n_images, r, n_tokens, src_out, zero_ptr,
                     zero_n);
+}
+
+cudaError_t launch_ln_merge(bool bf16, const void* x, const int32_t* src, const float* w, const float* b, float eps,
+                            void* merged, int64_t n_tokens, int r2, int d, cudaStream_t s) {
+  const int64_t rows = n_tokens * r2;
+  if (rows == 0) return cudaSuccess;
+  const int64_t blocks = (rows * 32 + 255) / 256;
+  if (bf16) return launch_pdl(k_ln_merge<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, src, w, b, eps,
+                              merged, rows, d);
+  return launch_pdl(k_ln_merge<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, src, w, b, eps,
+                    merged, rows, d);
 }
 
 cudaError_t launch_zero_counters(int* ptr, int n, cudaStream_t s) {

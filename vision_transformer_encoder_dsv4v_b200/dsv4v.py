@@ -26,7 +26,8 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_tower_forward_profiled",
            "dsv4v_aligner_forward", "dsv4v_aligner_tokens", "dsv4v_rmsnorm", "dsv4v_qkv_rope", "dsv4v_attention",
            "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
-           "dsv4v_status_string", "dsv4v_linear_residual_noalloc", "dsv4v_patch_embed")
+           "dsv4v_status_string", "dsv4v_linear_residual_noalloc", "dsv4v_patch_embed",
+           "dsv4v_patch_merger_workspace_size", "dsv4v_patch_merger_forward")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
             "dsv4v_linear_residual": (I, [cfg, I64, I, P, P, P, P, SZ, P]),
             "dsv4v_swiglu": (I, [cfg, I64, P, P, P, P, P, SZ, P]),
             "dsv4v_patch_embed": (I, [cfg, I64, I, I, P, I64, P, I64, P, P, P]),
+            "dsv4v_patch_merger_workspace_size": (SZ, [cfg, bat]),
+            "dsv4v_patch_merger_forward": (I, [cfg, bat, P, P, P, P, P, P, P, P, P, SZ, P]),
             "dsv4v_linear_residual_noalloc": (I, [cfg, I64, I, P, P, P, P]),
             "dsv4v_device_error": (I, [P]),
             "dsv4v_selftest_bounded_wait": (I, [U64, P]),
@@ -224,6 +227,18 @@ def dsv4v_patch_embed(cfg, n_patches, patch_h, patch_w, patches, w_proj, bias, x
     _check(lib().dsv4v_patch_embed(ctypes.byref(cfg), n_patches, patch_h, patch_w, _ptr(patches), ld_patches,
                                    _ptr(w_proj), ld_w, _ptr(bias), _ptr(x_out), _stream(stream)),
            "dsv4v_patch_embed")
+
+
+def dsv4v_patch_merger_workspace_size(cfg, batch) -> int:
+    return int(lib().dsv4v_patch_merger_workspace_size(ctypes.byref(cfg), ctypes.byref(batch.c)))
+
+
+def dsv4v_patch_merger_forward(cfg, batch, x, ln_w, ln_b, w1, b1, w2, b2, out, workspace, stream=None):
+    """PatchMerger projector: LayerNorm per patch, r x r window merge, Linear + GELU, Linear."""
+    _check(lib().dsv4v_patch_merger_forward(ctypes.byref(cfg), ctypes.byref(batch.c), _ptr(x), _ptr(ln_w), _ptr(ln_b),
+                                            _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(out), _ptr(workspace),
+                                            workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "dsv4v_patch_merger_forward")
 
 
 def dsv4v_device_error(stream=None) -> int:
