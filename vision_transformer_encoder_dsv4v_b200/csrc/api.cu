@@ -234,7 +234,7 @@ Layout make_layout(const Shape& s, const Plans& pl) {
   l.ss_parts = s.D / 64 > 0 ? s.D / 64 : 1;
   l.ss1 = take(s.bf16 ? static_cast<size_t>(s.P) * l.ss_parts * 4 : 0);
   l.ss2 = take(s.bf16 ? static_cast<size_t>(s.P) * l.ss_parts * 4 : 0);
-  l.merged = take(s.bf16 ? 0 : static_cast<size_t>(s.T) * s.r * s.r * s.D * 4);
+  l.merged = take(static_cast<size_t>(s.T) * s.r * s.r * s.D * es);
   l.total = off;
   return l;
 }
@@ -649,9 +649,13 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
                                              src, c.stream, s.bf16 ? c.at<int>(c.lay.counters) : nullptr,
                                              s.bf16 ? static_cast<int>(c.lay.counters_bytes / sizeof(int)) : 0)));
   const int K = s.r * s.r * s.D;
-  if (s.bf16)
-    return gemm_bf16(c, EPI_STORE, c.plans.align, nullptr, s.T, K, w_align, nullptr, s.E, out, nullptr, nullptr,
-                     nullptr, true, src, x);
+  if (s.bf16) {
+    // Materialise the merged window rows, then a TMA GEMM (the weights stream once; the rows
+    // are a few MB).
+    void* merged = c.at<uint8_t>(c.lay.merged);
+    DSV4V_TRY(cuda_status(launch_merge_rows_bf16(x, src, merged, s.T, s.r * s.r, s.D, c.stream)));
+    return gemm_bf16(c, EPI_STORE, c.plans.align, merged, s.T, K, w_align, nullptr, s.E, out, nullptr);
+  }
   float* merged = c.at<float>(c.lay.merged);
   DSV4V_TRY(cuda_status(launch_gather_f32(static_cast<const float*>(x), src, merged, s.T, s.r * s.r, s.D, c.stream)));
   return cuda_status(launch_gemm_f32(EPI_STORE, merged, static_cast<const float*>(w_align), nullptr,
@@ -662,12 +666,14 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
 // [T, r^2 D] in the activation dtype.
 namespace {
 struct MergerLayout {
-  size_t src, merged, hidden, total;
+  GemmPlan p1, p2;  // Linear 1 (GELU epilogue) and Linear 2 (bias store)
+  size_t src, merged, hidden, partials, counters, counters_bytes, total;
 };
-MergerLayout merger_layout(const Shape& s) {
+MergerLayout merger_layout(const Shape& s, int sms) {
   MergerLayout l{};
   const size_t es = s.bf16 ? 2 : 4;
   const size_t rows = static_cast<size_t>(s.T) * s.r * s.r;
+  const int K = s.r * s.r * s.D;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -677,6 +683,17 @@ MergerLayout merger_layout(const Shape& s) {
   l.src = take(rows * 4);
   l.merged = take(rows * s.D * es);
   l.hidden = take(rows * s.D * es);
+  size_t part = 0;
+  int counters = 1;
+  if (s.bf16 && s.T > 0) {
+    l.p1 = plan_gemm(EPI_GELU, static_cast<int>(s.T), K, K, sms);
+    l.p2 = plan_gemm(EPI_STORE, static_cast<int>(s.T), s.E, K, sms);
+    part = std::max(l.p1.partial_bytes, l.p2.partial_bytes);
+    counters = std::max(counters, std::max(l.p1.counters, l.p2.counters));
+  }
+  l.partials = take(part);
+  l.counters_bytes = up256(static_cast<size_t>(counters) * sizeof(int));
+  l.counters = take(l.counters_bytes);
   l.total = off;
   return l;
 }
@@ -685,7 +702,7 @@ MergerLayout merger_layout(const Shape& s) {
 size_t dsv4v_patch_merger_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch) {
   Shape s;
   if (check_all(cfg, batch, s) != DSV4V_OK) return 0;
-  return merger_layout(s).total;
+  return merger_layout(s, planning_sms()).total;
 }
 
 dsv4v_status dsv4v_patch_merger_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x,
@@ -699,12 +716,15 @@ dsv4v_status dsv4v_patch_merger_forward(const dsv4v_config* cfg, const dsv4v_bat
   for (const void* ptr : {x, static_cast<const void*>(ln_w), static_cast<const void*>(ln_b), w1,
                           static_cast<const void*>(b1), w2, static_cast<const void*>(b2), static_cast<const void*>(out)})
     if (!ptr || !aligned16(ptr)) return DSV4V_ERR_INVALID_ARG;
-  const MergerLayout l = merger_layout(s);
+  const MergerLayout l = merger_layout(s, c.dev.sms);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < l.total) return DSV4V_ERR_WORKSPACE;
   c.stream = static_cast<cudaStream_t>(stream);
   c.eps = cfg->eps;
   c.ws = static_cast<uint8_t*>(workspace);
-  c.lay = Layout{};  // the GEMMs below use no split-tile scratch
+  c.lay = Layout{};
+  c.lay.partials = l.partials;  // split-tile scratch of the two GEMMs
+  c.lay.counters = l.counters;
+  c.lay.counters_bytes = l.counters_bytes;
   if (s.T == 0) return DSV4V_OK;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* src = reinterpret_cast<int32_t*>(ws + l.src);
@@ -722,10 +742,10 @@ dsv4v_status dsv4v_patch_merger_forward(const dsv4v_config* cfg, const dsv4v_bat
                                        nullptr, static_cast<float*>(out), nullptr, static_cast<int>(s.T), s.E, K,
                                        c.stream, b2));
   }
-  // Whole-tile plans only: no split-tile scratch.
-  const GemmPlan p1 = plan_gemm(EPI_GELU, static_cast<int>(s.T), K, K, c.dev.sms, 0);
-  const GemmPlan p2 = plan_gemm(EPI_STORE, static_cast<int>(s.T), s.E, K, c.dev.sms, 0);
+  const GemmPlan& p1 = l.p1;
+  const GemmPlan& p2 = l.p2;
   if (p1.bn == 0 || p2.bn == 0) return DSV4V_ERR_UNSUPPORTED;
+  DSV4V_TRY(reset_counters(c));  // the finishers of each GEMM leave the counters at zero again
   GemmExtra e1, e2;
   e1.bias = b1;
   e2.bias = b2;

@@ -348,8 +348,8 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
               const __grid_constant__ CUtensorMap tm_xw, const Params p) {
   static_assert(!(GATHER && PAIR), "the A-gather runs on single CTAs");
-  static_assert(KS == 1 || (!GATHER && !PAIR && BN == 256 && EPI == EPI_RESID),
-                "cluster split-K is built for 256-column residual tiles");
+  static_assert(KS == 1 || (!GATHER && !PAIR && BN == 256 && (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)),
+                "cluster split-K is built for 256-column residual, store and GELU tiles");
   using C = TileCfg<BN, PAIR>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
   constexpr int STAGES = C::STAGES;
@@ -998,8 +998,8 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
 template <int EPI, bool GATHER>
 cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   if (plan.ks > 1) {
-    // Cluster split-K: 256-column residual tiles.
-    if constexpr (!GATHER && EPI == EPI_RESID) {
+    // Cluster split-K: 256-column residual, store and GELU tiles.
+    if constexpr (!GATHER && (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)) {
       if (plan.bn != 256 || plan.pair) return cudaErrorInvalidValue;
       switch (plan.ks) {
         case 2: return launch_one<256, EPI, false, false, 2>(plan, a, s);
@@ -1165,14 +1165,20 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
     const int tiles_n = n_out / n_cols_per_tile;
     const long long tiles = static_cast<long long>(tiles_m) * tiles_n;
     const long long units = tiles * kb_total;
-    // Grids: every SM; t whole tiles per CTA (t = 1..4); or s CTAs per tile (split-K by s).
-    int grids[9];
+    // Grids: every SM; t whole tiles per CTA (t = 1..4); the largest divisor of the tile count
+    // that fits the SMs (equal whole tiles per CTA); or s CTAs per tile (split-K by s).
+    int grids[10];
     int n_grids = 0;
     grids[n_grids++] = static_cast<int>(std::min<long long>(num_sms, units));
     for (int t = 1; t <= 4; ++t) {
       const long long g = (tiles + t - 1) / t;
       if (g <= num_sms) grids[n_grids++] = static_cast<int>(g);
     }
+    for (long long g = std::min<long long>(num_sms, tiles); g >= 1; --g)
+      if (tiles % g == 0) {
+        grids[n_grids++] = static_cast<int>(g);
+        break;
+      }
     for (int s = 2; s <= 4; ++s)
       if (tiles * s <= num_sms && tiles * s <= units) grids[n_grids++] = static_cast<int>(tiles * s);
     for (int gi = 0; gi < n_grids; ++gi) {
@@ -1197,9 +1203,9 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
       }
     }
   }
-  // Cluster split-K for 256-column residual tiles: full-rate N = 256 MMAs even when there are
-  // too few such tiles for the SMs, without the global-memory split-tile fix-up.
-  if (epi == EPI_RESID && n_out % 256 == 0) {
+  // Cluster split-K for 256-column residual, store and GELU tiles: full-rate N = 256 MMAs even
+  // when there are too few such tiles for the SMs, without the global-memory split-tile fix-up.
+  if ((epi == EPI_RESID || epi == EPI_STORE || epi == EPI_GELU) && n_out % 256 == 0) {
     const long long tiles = static_cast<long long>(tiles_m) * (n_out / 256);
     for (int ks : {2, 4}) {
       if (kb_total % ks || tiles * ks > num_sms) continue;

@@ -20,7 +20,7 @@ enum Epi : int {
 struct GemmPlan {
   int bn;        // MMA N per tile (SWIGLU: gate + up halves)
   int pair;      // 1: 256-row tiles on CTA pairs (tcgen05 cta_group::2), grid even; 0: 128-row tiles
-  int ks;        // > 1 (residual epilogue only): each tile is split along K over a cluster of ks
+  int ks;        // > 1 (residual, store, GELU epilogues): each tile is split along K over a cluster of ks
                  // CTAs, reduced through distributed shared memory (bn = 256; each CTA finishes
                  // 256 / ks columns)
   int splits;    // K splits per tile (fix-up by the last finisher)
@@ -106,6 +106,10 @@ cudaError_t launch_aligner_index(const int32_t* cu_dev, const int32_t* grid_dev,
                                  int64_t n_tokens, int32_t* src_out, cudaStream_t s, int* zero_ptr = nullptr,
                                  int zero_n = 0);
 cudaError_t launch_zero_counters(int* ptr, int n, cudaStream_t s);
+// Merged r x r window rows of bf16 patch rows: merged[t, s * d : (s + 1) * d] = x[src[t * r2 + s]],
+// zeros where src < 0 (d a multiple of 8).
+cudaError_t launch_merge_rows_bf16(const void* x, const int32_t* src, void* merged, int64_t n_tokens, int r2, int d,
+                                   cudaStream_t s);
 // LayerNorm of each patch row (weight and bias, fp32 math) written into its slot of the merged
 // r x r window rows: merged[t, s * d : (s + 1) * d] = LN(x[src[t * r2 + s]]), zeros where
 // src < 0.  bf16 or fp32 activations.

@@ -212,6 +212,24 @@ __global__ void k_ln_merge(const void* __restrict__ x, const int32_t* __restrict
   for (int c = lane; c < d; c += 32) put(c, (in(c) - mean) * inv * w[c] + b[c]);
 }
 
+// One warp per (token, slot) row: a 16-byte-vector copy of the source patch row, or zeros.
+__global__ void k_merge_rows_bf16(const uint4* __restrict__ x, const int32_t* __restrict__ src, uint4* merged,
+                                  int64_t n_rows, int d8) {
+  grid_dependency_wait();
+  launch_dependents();
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const int32_t s = src[row];
+  uint4* dst = merged + row * d8;
+  if (s < 0) {
+    for (int c = lane; c < d8; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const uint4* in = x + static_cast<int64_t>(s) * d8;
+  for (int c = lane; c < d8; c += 32) dst[c] = in[c];
+}
+
 // Clears the GEMM tile counters of a component call (one block; dependent launch, so that it
 // costs no more than a kernel boundary inside a graph, unlike a memset node).
 __global__ void k_zero_counters(int* ptr, int n) {
@@ -293,6 +311,15 @@ cudaError_t launch_ln_merge(bool bf16, const void* x, const int32_t* src, const 
                               merged, rows, d);
   return launch_pdl(k_ln_merge<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, src, w, b, eps,
                     merged, rows, d);
+}
+
+cudaError_t launch_merge_rows_bf16(const void* x, const int32_t* src, void* merged, int64_t n_tokens, int r2, int d,
+                                   cudaStream_t s) {
+  const int64_t rows = n_tokens * r2;
+  if (rows == 0) return cudaSuccess;
+  const int64_t blocks = (rows * 32 + 255) / 256;
+  return launch_pdl(k_merge_rows_bf16, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                    static_cast<const uint4*>(x), src, static_cast<uint4*>(merged), rows, d / 8);
 }
 
 cudaError_t launch_zero_counters(int* ptr, int n, cudaStream_t s) {
