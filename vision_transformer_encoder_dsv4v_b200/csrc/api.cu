@@ -297,19 +297,18 @@ struct GemmExtra {
 
 dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* a, int64_t M, int K, const void* b,
                        const void* b2, int n_out, void* out, const void* resid, const float* cos = nullptr,
-                       const float* sin = nullptr, bool gather = false, const int32_t* gsrc = nullptr,
-                       const void* gx = nullptr, const NormFold& nf = NormFold(), const GemmExtra& ex = GemmExtra()) {
+                       const float* sin = nullptr, const NormFold& nf = NormFold(), const GemmExtra& ex = GemmExtra()) {
   if (M == 0) return DSV4V_OK;
   const int box_b = (epi == EPI_SWIGLU || plan.pair) ? plan.bn / 2 : plan.bn;
   CUtensorMap ta, tb, tb2, t_out, t_xw;
-  if ((!gather && !bf16_map(a, M, K, 128, &ta, ex.lda)) || !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
+  if (!bf16_map(a, M, K, 128, &ta, ex.lda) || !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
       (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)) || !bf16_map(out, M, n_out, 32, &t_out) ||
       (nf.xw_out && !bf16_map(nf.xw_out, M, n_out, 32, &t_xw)))
     return DSV4V_ERR_CUDA;
   GemmArgs g{};
   g.tm_out = &t_out;
   g.tm_xw = nf.xw_out ? &t_xw : nullptr;
-  g.tm_a = gather ? nullptr : &ta;
+  g.tm_a = &ta;
   g.tm_b = &tb;
   g.tm_b2 = epi == EPI_SWIGLU ? &tb2 : nullptr;
   g.M = static_cast<int>(M);
@@ -321,10 +320,6 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.cos = cos;
   g.sin = sin;
   g.rot_cols = 2 * c.s.D;
-  g.gather_src = gsrc;
-  g.gather_x = gx;
-  g.gather_r2 = c.s.r * c.s.r;
-  g.gather_d = c.s.D;
   g.partials = c.at<float>(c.lay.partials);
   g.counters = c.at<int>(c.lay.counters);
   g.err = c.dev.err;
@@ -338,7 +333,7 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.ss_out = nf.ss_out;
   g.ss_parts = nf.ss_parts;
   g.bias = ex.bias;
-  return cuda_status(launch_gemm_tc(epi, gather, plan, g, c.stream));
+  return cuda_status(launch_gemm_tc(epi, plan, g, c.stream));
 }
 
 dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv, void* out) {
@@ -413,8 +408,8 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   q.parts = first ? 1 : norm_parts_of(c.plans.down);  // the prep kernel puts the whole row sum in slot 0
   q.stride = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_QKV, 0, c.stream));
-  DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, xw, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr,
-                              cos, sin, false, nullptr, nullptr, q));
+  DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, xw, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr, cos,
+                      sin, q));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_QKV, 1, c.stream));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_ATTENTION, 0, c.stream));
   DSV4V_TRY(attention_bf16(c, b, qkv, attn));
@@ -425,16 +420,15 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   o.ss_out = ss2;
   o.ss_parts = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_OUT, 0, c.stream));
-  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x, nullptr, nullptr,
-                              false, nullptr, nullptr, o));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x, nullptr, nullptr, o));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_OUT, 1, c.stream));
   NormFold m;
   m.ss = ss2;
   m.parts = norm_parts_of(c.plans.out);
   m.stride = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_SWIGLU, 0, c.stream));
-  DSV4V_TRY(gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, xw, s.P, s.D, w->w_gate, w->w_up, s.F, h, nullptr,
-                              nullptr, nullptr, false, nullptr, nullptr, m));
+  DSV4V_TRY(gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, xw, s.P, s.D, w->w_gate, w->w_up, s.F, h, nullptr, nullptr,
+                      nullptr, m));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_SWIGLU, 1, c.stream));
   NormFold d;
   if (next_norm_w) {
@@ -444,8 +438,7 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
     d.ss_parts = c.lay.ss_parts;
   }
   DSV4V_TRY(record(ev, DSV4V_PROFILE_DOWN, 0, c.stream));
-  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x, nullptr, nullptr,
-                      false, nullptr, nullptr, d));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x, nullptr, nullptr, d));
   return record(ev, DSV4V_PROFILE_DOWN, 1, c.stream);
 }
 
@@ -749,10 +742,9 @@ dsv4v_status dsv4v_patch_merger_forward(const dsv4v_config* cfg, const dsv4v_bat
   GemmExtra e1, e2;
   e1.bias = b1;
   e2.bias = b2;
-  DSV4V_TRY(gemm_bf16(c, EPI_GELU, p1, merged, s.T, K, w1, nullptr, K, hidden, nullptr, nullptr, nullptr, false,
-                      nullptr, nullptr, NormFold(), e1));
-  return gemm_bf16(c, EPI_STORE, p2, hidden, s.T, K, w2, nullptr, s.E, out, nullptr, nullptr, nullptr, false, nullptr,
-                   nullptr, NormFold(), e2);
+  DSV4V_TRY(gemm_bf16(c, EPI_GELU, p1, merged, s.T, K, w1, nullptr, K, hidden, nullptr, nullptr, nullptr, NormFold(),
+                      e1));
+  return gemm_bf16(c, EPI_STORE, p2, hidden, s.T, K, w2, nullptr, s.E, out, nullptr, nullptr, nullptr, NormFold(), e2);
 }
 
 dsv4v_status dsv4v_rmsnorm(const dsv4v_config* cfg, int64_t rows, const void* x, const float* w, void* y,
@@ -858,7 +850,7 @@ dsv4v_status dsv4v_patch_embed(const dsv4v_config* cfg, int64_t n_patches, int p
   ex.ldb = ld_w;
   ex.bias = bias;
   return gemm_bf16(c, EPI_STORE, plan, patches, n_patches, K, w_proj, nullptr, s.D, x_out, nullptr, nullptr, nullptr,
-                   false, nullptr, nullptr, NormFold(), ex);
+                   NormFold(), ex);
 }
 
 dsv4v_status dsv4v_device_error(void* stream) {

@@ -1,14 +1,12 @@
 // tcgen05 GEMM for the dense contractions of the vision block and the aligner:
 //   wqkv (+ 2D rotary epilogue), output projection (+ residual), SwiGLU gate/up (+ silu*mul),
-//   down projection (+ residual), aligner projection (A rows gathered from r x r windows).
+//   down projection (+ residual), aligner projection, patch embedding, PatchMerger projector.
 //
 // Structure (one persistent CTA per SM, 128 x BN output tiles, K in 64-element blocks):
 //   warp 0      TMA producer: A and B tiles (128-byte swizzle) into a STAGES-deep smem ring
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer (M=128, N=BN, K=16 per instr.)
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane = one output row
 //               per thread), fused epilogue math, bf16 stores
-//   warps 6..9  (aligner only) A-gather: cp.async rows of the patch matrix into the swizzled
-//               A tile, zero-filling padded window slots
 //
 // Work split (stream-K): the GEMM is U = tiles x (K / 64) units of one 64-deep K block of one
 // output tile; CTA c of G owns units [c U / G, (c + 1) U / G), i.e. equal work per SM whatever
@@ -63,9 +61,6 @@ struct Params {
   const float* cos;
   const float* sin;
   int rot_cols;
-  const int32_t* gsrc;
-  const __nv_bfloat16* gx;
-  int gr2, gd;
   float* partials;  // [G][BN / 4][128][4] fp32: a contributor's partial of a split tile
   int* counters;    // [tiles], zero between launches
   uint32_t* err;
@@ -116,13 +111,6 @@ struct SegmentWalker {
     return true;
   }
 };
-
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // gelu(z) = z (1 + erf(z / sqrt 2)) / 2, the exact (erf) form.
 __device__ __forceinline__ float gelu(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
@@ -342,13 +330,12 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatil
   }
 }
 
-template <int BN, int EPI, bool GATHER, bool PAIR, int KS>
-__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
+template <int BN, int EPI, bool PAIR, int KS>
+__global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
               const __grid_constant__ CUtensorMap tm_xw, const Params p) {
-  static_assert(!(GATHER && PAIR), "the A-gather runs on single CTAs");
-  static_assert(KS == 1 || (!GATHER && !PAIR && BN == 256 && (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)),
+  static_assert(KS == 1 || (!PAIR && BN == 256 && (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)),
                 "cluster split-K is built for 256-column residual, store and GELU tiles");
   using C = TileCfg<BN, PAIR>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
@@ -378,7 +365,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], GATHER ? 1 + 128 : 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -391,7 +378,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    if (!GATHER) tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
     if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tm_b2);
     tma_prefetch_desc(&tm_out);
@@ -429,7 +416,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       // Stage s of both CTAs of a pair completes on the leader's full[s].
       const uint32_t full_leader = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
       const bool arrives = !PAIR || rank == 0;  // posts the expected bytes of the stage
-      constexpr uint32_t kStageTx = GATHER ? C::B_BYTES : (PAIR ? 2 * C::STAGE : C::STAGE);
+      constexpr uint32_t kStageTx = PAIR ? 2 * C::STAGE : C::STAGE;
       auto load_a = [&](uint8_t* sa, int kb, int m_tile, int s) {
         if constexpr (PAIR)
           tma_load_2d_pair(sa, &tm_a, full_leader + 8u * s, kb * BK, m_tile * BMT + static_cast<int>(rank) * BM);
@@ -467,8 +454,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
         }
       }
       grid_dependency_wait();
-      if (!GATHER)
-        for (int i = 0; i < pre; ++i) load_a(smem + i * C::STAGE, first.kb0 + i, first.m_tile, i);
+      for (int i = 0; i < pre; ++i) load_a(smem + i * C::STAGE, first.kb0 + i, first.m_tile, i);
       stage = pre % STAGES;
       phase = (pre == STAGES) ? 1u : 0u;
       while (ok && walk.next(p, sg)) {
@@ -479,7 +465,7 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
           }
           uint8_t* sa = smem + stage * C::STAGE;
           if (arrives) mbar_arrive_expect_tx(&full[stage], kStageTx);
-          if (!GATHER) load_a(sa, kb, sg.m_tile, stage);
+          load_a(sa, kb, sg.m_tile, stage);
           load_b(sa + C::A_BYTES, kb, sg.n_tile, stage);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -874,49 +860,6 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       }
     }
     st.drain();
-  } else if constexpr (GATHER) {
-    // ------------------------------------------------------------------ A-gather (aligner)
-    const int r = threadIdx.x - 192;  // row of the A tile handled by this thread
-    const int blocks_per_slot = p.gd / BK;
-    grid_dependency_wait();
-    int stage = 0, pending = -1;
-    uint32_t phase = 0;
-    bool ok = true;
-    SegmentWalker walk(p, owner);
-    Segment sg;
-    while (ok && walk.next(p, sg)) {
-      const int row = sg.m_tile * BM + r;
-      for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutGather)) {
-          ok = false;
-          break;
-        }
-        const int slot = kb / blocks_per_slot;
-        const int c0 = (kb - slot * blocks_per_slot) * BK;
-        const int src = row < p.M ? p.gsrc[static_cast<size_t>(row) * p.gr2 + slot] : -1;
-        const uint32_t dst_row = smem_u32(smem + stage * C::STAGE) + r * 128;
-        const __nv_bfloat16* src_row = p.gx + (src >= 0 ? static_cast<size_t>(src) * p.gd + c0 : 0);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          cp_async_16(dst_row + ((c ^ (r & 7)) << 4), src_row + 8 * c, src >= 0 ? 16u : 0u);
-        cp_async_commit();
-        if (pending >= 0) {
-          cp_async_wait_1();
-          fence_proxy_async_smem();
-          mbar_arrive(&full[pending]);
-        }
-        pending = stage;
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-    }
-    cp_async_wait_all();
-    if (pending >= 0) {
-      fence_proxy_async_smem();
-      mbar_arrive(&full[pending]);
-    }
   }
 
   // Teardown: TMEM is released only after every warp has finished with it.  Role code ran on
@@ -938,11 +881,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
   }
 }
 
-template <int BN, int EPI, bool GATHER, bool PAIR = false, int KS = 1>
+template <int BN, int EPI, bool PAIR = false, int KS = 1>
 cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   using C = TileCfg<BN, PAIR>;
   static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
-  auto kern = k_gemm_tc<BN, EPI, GATHER, PAIR, KS>;
+  auto kern = k_gemm_tc<BN, EPI, PAIR, KS>;
   if (PAIR && (plan.grid & 1)) return cudaErrorInvalidValue;
   if (KS > 1 && (plan.grid % KS || plan.kb_total % KS || plan.grid != plan.work * KS)) return cudaErrorInvalidValue;
   int dev = 0;
@@ -967,10 +910,6 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.cos = a.cos;
   p.sin = a.sin;
   p.rot_cols = a.rot_cols;
-  p.gsrc = a.gather_src;
-  p.gx = static_cast<const __nv_bfloat16*>(a.gather_x);
-  p.gr2 = a.gather_r2;
-  p.gd = a.gather_d;
   p.partials = a.partials;
   p.counters = a.counters;
   p.err = a.err;
@@ -984,65 +923,65 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.ss_out = a.ss_out;
   p.ss_parts = a.ss_parts;
   p.bias = a.bias;
-  const CUtensorMap& ta = GATHER ? *a.tm_b : *a.tm_a;
+  const CUtensorMap& ta = *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
   const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
   if constexpr (PAIR || KS > 1)
     return launch_pdl_cluster(kern, dim3(plan.grid), dim3(192), C::SMEM, s, PAIR ? 2u : static_cast<unsigned>(KS), ta,
                               *a.tm_b, tb2, *a.tm_out, txw, p);
   else
-    return launch_pdl(kern, dim3(plan.grid), dim3(GATHER ? 320 : 192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
+    return launch_pdl(kern, dim3(plan.grid), dim3(192), C::SMEM, s, ta, *a.tm_b, tb2, *a.tm_out, txw, p);
 }
 
 // Tile widths each epilogue supports (the planner only picks these).
-template <int EPI, bool GATHER>
+template <int EPI>
 cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   if (plan.ks > 1) {
     // Cluster split-K: 256-column residual, store and GELU tiles.
-    if constexpr (!GATHER && (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)) {
+    if constexpr (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU) {
       if (plan.bn != 256 || plan.pair) return cudaErrorInvalidValue;
       switch (plan.ks) {
-        case 2: return launch_one<256, EPI, false, false, 2>(plan, a, s);
-        case 4: return launch_one<256, EPI, false, false, 4>(plan, a, s);
+        case 2: return launch_one<256, EPI, false, 2>(plan, a, s);
+        case 4: return launch_one<256, EPI, false, 4>(plan, a, s);
         default: return cudaErrorInvalidValue;
       }
     }
     return cudaErrorInvalidValue;
   }
   if (plan.pair) {
-    // CTA pairs: 256-row tiles, no A-gather.
-    if constexpr (GATHER || EPI == EPI_STORE || EPI == EPI_GELU) {
+    // CTA pairs: 256-row tiles.
+    if constexpr (EPI == EPI_STORE || EPI == EPI_GELU) {
       return cudaErrorInvalidValue;
     } else if constexpr (EPI == EPI_SWIGLU) {
-      if (plan.bn == 256) return launch_one<256, EPI, false, true>(plan, a, s);
+      if (plan.bn == 256) return launch_one<256, EPI, true>(plan, a, s);
       return cudaErrorInvalidValue;
     } else {
       switch (plan.bn) {
-        case 128: return launch_one<128, EPI, false, true>(plan, a, s);
-        case 256: return launch_one<256, EPI, false, true>(plan, a, s);
+        case 128: return launch_one<128, EPI, true>(plan, a, s);
+        case 256: return launch_one<256, EPI, true>(plan, a, s);
         default: return cudaErrorInvalidValue;
       }
     }
   }
   if constexpr (EPI == EPI_RESID) {
     switch (plan.bn) {
-      case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
-      case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
-      case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
+      case 64: return launch_one<64, EPI>(plan, a, s);
+      case 128: return launch_one<128, EPI>(plan, a, s);
+      case 256: return launch_one<256, EPI>(plan, a, s);
       default: return cudaErrorInvalidValue;
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
     switch (plan.bn) {
-      case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
-      case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
+      case 128: return launch_one<128, EPI>(plan, a, s);
+      case 256: return launch_one<256, EPI>(plan, a, s);
       default: return cudaErrorInvalidValue;
     }
   } else {
     switch (plan.bn) {
-      case 64: return launch_one<64, EPI, GATHER>(plan, a, s);
-      case 128: return launch_one<128, EPI, GATHER>(plan, a, s);
-      case 192: return launch_one<192, EPI, GATHER>(plan, a, s);
-      case 256: return launch_one<256, EPI, GATHER>(plan, a, s);
+      case 64: return launch_one<64, EPI>(plan, a, s);
+      case 128: return launch_one<128, EPI>(plan, a, s);
+      case 192: return launch_one<192, EPI>(plan, a, s);
+      case 256: return launch_one<256, EPI>(plan, a, s);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -1230,17 +1169,13 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
   return best;
 }
 
-cudaError_t launch_gemm_tc(int epi, bool gather, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
-  if (gather) {
-    if (epi != EPI_STORE) return cudaErrorInvalidValue;
-    return launch_bn<EPI_STORE, true>(plan, a, s);
-  }
+cudaError_t launch_gemm_tc(int epi, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   switch (epi) {
-    case EPI_STORE: return launch_bn<EPI_STORE, false>(plan, a, s);
-    case EPI_RESID: return launch_bn<EPI_RESID, false>(plan, a, s);
-    case EPI_QKV_ROPE: return launch_bn<EPI_QKV_ROPE, false>(plan, a, s);
-    case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(plan, a, s);
-    case EPI_GELU: return launch_bn<EPI_GELU, false>(plan, a, s);
+    case EPI_STORE: return launch_bn<EPI_STORE>(plan, a, s);
+    case EPI_RESID: return launch_bn<EPI_RESID>(plan, a, s);
+    case EPI_QKV_ROPE: return launch_bn<EPI_QKV_ROPE>(plan, a, s);
+    case EPI_SWIGLU: return launch_bn<EPI_SWIGLU>(plan, a, s);
+    case EPI_GELU: return launch_bn<EPI_GELU>(plan, a, s);
     default: return cudaErrorInvalidValue;
   }
 }

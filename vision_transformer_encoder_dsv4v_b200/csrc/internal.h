@@ -39,7 +39,7 @@ GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms, size_t max_par
 struct GemmArgs {
   const CUtensorMap* tm_out;  // output [M, n_out] bf16, box 64 x 32 (TMA stores of the epilogue)
   const CUtensorMap* tm_xw;   // RESID with the next norm prepared: xw_out [M, n_out], box 64 x 32
-  const CUtensorMap* tm_a;    // A [M, K], box 64 x 128 (ignored when gathering A)
+  const CUtensorMap* tm_a;    // A [M, K], box 64 x 128
   const CUtensorMap* tm_b;    // B [n, K] (SWIGLU: w_gate), box 64 x bn (SWIGLU or pair: bn / 2)
   const CUtensorMap* tm_b2;   // SWIGLU: w_up, box 64 x bn / 2
   int M, K, n_out;
@@ -49,11 +49,6 @@ struct GemmArgs {
   const float* cos;
   const float* sin;
   int rot_cols;
-  // Aligner A-gather: row m of A, K-block slot s = x[src[m * r2 + s], :] (src < 0: zeros).
-  const int32_t* gather_src;
-  const void* gather_x;
-  int gather_r2;
-  int gather_d;
   float* partials;
   int* counters;
   uint32_t* err;
@@ -73,7 +68,7 @@ struct GemmArgs {
   const float* bias;  // STORE: per-column fp32 bias added before rounding (NULL: none)
 };
 
-cudaError_t launch_gemm_tc(int epi, bool gather, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_gemm_tc(int epi, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------- attention
 constexpr int kMaxImages = 1024;
