@@ -29,8 +29,8 @@
  *    (size from dsv4v_workspace_size, 256-byte aligned).
  *  - Every call is asynchronous and ordered on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  Argument, shape and workspace errors are reported synchronously, before any
- *    kernel is launched.  A bounded device-side wait that gives up records an error that
- *    dsv4v_device_error() returns after synchronising the stream.
+ *    kernel is launched.  A device-side check that fails (a bounded wait that gives up)
+ *    records an error that dsv4v_device_error() returns after synchronising the stream.
  *  - Calls on the same workspace must not overlap on the GPU (put them on one stream).
  *  - No call keeps device state between calls; each call may be captured in a CUDA graph
  *    (the launch geometry is taken from the host copies of the grids and offsets, which must
@@ -52,7 +52,9 @@ typedef enum {
   DSV4V_ERR_UNSUPPORTED = 2,   /* shape outside the constraints listed at the config below */
   DSV4V_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or smaller than required */
   DSV4V_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
-  DSV4V_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (see dsv4v_device_error) */
+  DSV4V_ERR_TIMEOUT = 5        /* a device-side check failed: a bounded wait gave up, or the two
+                                  CTAs of a GEMM CTA pair got different TMEM addresses (see
+                                  dsv4v_device_error) */
 } dsv4v_status;
 
 typedef enum { DSV4V_F32 = 0, DSV4V_BF16 = 1 } dsv4v_dtype;
@@ -260,8 +262,9 @@ dsv4v_status dsv4v_linear_residual_noalloc(const dsv4v_config* cfg, int64_t rows
                                            const void* a, const void* w, void* x, void* stream);
 
 /* Synchronises `stream` and returns DSV4V_ERR_TIMEOUT if a kernel of this library recorded a
- * bounded-wait timeout on the current device since the last call (and clears the record),
- * DSV4V_ERR_CUDA if the stream reports an error, else DSV4V_OK. */
+ * device-side failure on the current device since the last call (a bounded wait that gave up,
+ * or a CTA pair whose TMEM allocations differ), and clears the record; DSV4V_ERR_CUDA if the
+ * stream reports an error; else DSV4V_OK. */
 dsv4v_status dsv4v_device_error(void* stream);
 
 /* Test hook for the bounded-wait machinery: launches one tiny kernel that waits on an
