@@ -10,8 +10,9 @@ Sources (page title, then section):
                 (classes DeepseekV4VisionRMSNorm / Attention / MLP / Block / Transformer /
                 Aligner, functions apply_vision_rotary, get_vision_cos_sin)
   [model-API]   "nemo_automodel.components.models.deepseek_v4.model" API reference
-                (DeepseekV4Model.encode_image, merge_image_embeddings, the THD
-                cu_seqlens helpers)
+                (DeepseekV4Model.encode_image, merge_image_embeddings and the sentinel
+                parameters image_start / image_end / image_newline / image_pad,
+                apply_deepseek_v4_image_visibility, the THD cu_seqlens helpers)
   [PR]          NeMo-Automodel pull request "Add native AutoModel support for
                 deepseek-ai/DeepSeek-V4-Flash-Vision-Exp", Changelog and Validation
 
@@ -268,6 +269,105 @@ def patch_merger(x, grids, r: int, ln_w, ln_b, w1, b1, w2, b2, eps: float = 1e-6
     merged, cu_tok = aligner_merge(xn, grids, r)
     h = gelu(merged @ _f64(w1).T + _f64(b1)[None, :])
     return h @ _f64(w2).T + _f64(b2)[None, :], cu_tok
+
+
+# --------------------------------------------------------------------------------------------
+# Image-token bridge: [model-API, DeepseekV4Model] (sentinel parameters image_start, image_end,
+# image_newline, image_pad; merge_image_embeddings; apply_deepseek_v4_image_visibility).
+# READING 15: the integer codes of the pseudo-token types are not printed; -1 = text is stated.
+# Taken: 0 = an image feature position, 1 = image_start, 2 = image_end, 3 = image_newline,
+# 4 = image_pad.  The N-layout of one image of g_h x g_w aligner tokens is image_start, then
+# each token row followed by image_newline, then image_end.  image_pad never appears in that
+# layout; a caller may place it (e.g. to fill a bucket) and the merge gives it its sentinel.
+# --------------------------------------------------------------------------------------------
+TOK_TEXT, TOK_IMAGE, TOK_START, TOK_END, TOK_NEWLINE, TOK_PAD = -1, 0, 1, 2, 3, 4
+SENTINEL_ORDER = (TOK_START, TOK_END, TOK_NEWLINE, TOK_PAD)  # rows of the sentinel matrix
+
+
+def image_layout(n_h: int, n_w: int, r: int) -> np.ndarray:
+    """Pseudo-token types of one image of an n_h x n_w patch grid (READING 15): the aligner gives
+    ceil(n_h / r) rows of ceil(n_w / r) tokens (READING 9); each row is closed by a newline and
+    the whole image is enclosed by start and end."""
+    g_h, g_w = -(-n_h // r), -(-n_w // r)
+    types = [TOK_START]
+    for _ in range(g_h):
+        types.extend([TOK_IMAGE] * g_w)
+        types.append(TOK_NEWLINE)
+    types.append(TOK_END)
+    return np.asarray(types, dtype=np.int32)
+
+
+def merge_image_embeddings(embeds, types, image_tokens, sentinels, tokens_per_image):
+    """[model-API, DeepseekV4Model.merge_image_embeddings]: every pseudo-token row of the text
+    embeddings is replaced; text rows (-1) are kept.
+
+    embeds: [batch, seq, E]; types: [batch, seq]; image_tokens: [T, E], the aligner output of
+    all images in packing order; sentinels: [4, E] in SENTINEL_ORDER; tokens_per_image: aligner
+    tokens of each image in packing order.
+    READING 16: the spans (image_spans, per sequence) taken in batch-major order are the images
+    in packing order; the j-th span's feature positions take image j's tokens in order, and it
+    must hold exactly that many.  Raises ValueError when the types do not fit the images."""
+    out = np.array(embeds, copy=True)
+    types = np.asarray(types)
+    cu = np.concatenate([[0], np.cumsum(tokens_per_image)]).astype(np.int64)
+    j = 0
+    for b in range(types.shape[0]):
+        spans = image_spans(types[b])
+        for p, t in enumerate(types[b]):
+            if t not in (TOK_TEXT, TOK_IMAGE) and t not in SENTINEL_ORDER:
+                raise ValueError(f"unknown pseudo-token type {t} at ({b}, {p})")
+        for a, e in spans:
+            if j >= len(tokens_per_image):
+                raise ValueError(f"more image spans than the {len(tokens_per_image)} images")
+            k = cu[j]
+            for p in range(a, e + 1):
+                t = types[b, p]
+                if t == TOK_IMAGE:
+                    if k >= cu[j + 1]:
+                        raise ValueError(f"span {j} holds more than {cu[j + 1] - cu[j]} features")
+                    out[b, p] = image_tokens[k]
+                    k += 1
+                else:
+                    out[b, p] = sentinels[SENTINEL_ORDER.index(t)]
+            if k != cu[j + 1]:
+                raise ValueError(f"span {j} holds {k - cu[j]} features, image {j} has {cu[j + 1] - cu[j]}")
+            j += 1
+    if j != len(tokens_per_image):
+        raise ValueError(f"{j} image spans for {len(tokens_per_image)} images")
+    return out
+
+
+def image_spans(types_row):
+    """Image spans of one sequence as inclusive (start, end) pairs.  READING 17: a span runs from
+    an image_start to the next image_end; a pseudo token outside such a pair, an image_start
+    inside an open span or a span left open at the end is an error (ValueError)."""
+    spans, open_at = [], None
+    for p, t in enumerate(types_row):
+        if t == TOK_START:
+            if open_at is not None:
+                raise ValueError(f"image_start at {p} inside the span opened at {open_at}")
+            open_at = p
+        elif t == TOK_END:
+            if open_at is None:
+                raise ValueError(f"image_end at {p} outside a span")
+            spans.append((open_at, p))
+            open_at = None
+        elif t != TOK_TEXT and open_at is None:
+            raise ValueError(f"pseudo token {t} at {p} outside a span")
+    if open_at is not None:
+        raise ValueError(f"span opened at {open_at} is not closed")
+    return spans
+
+
+def image_visibility(mask, types):
+    """[model-API, apply_deepseek_v4_image_visibility]: every pair of positions inside one image
+    span becomes visible (additive 0); all other entries are kept.  mask: [batch, seq, seq]
+    additive (the pages' [batch, 1, seq, seq] without the head axis); types: [batch, seq]."""
+    out = np.array(mask, copy=True)
+    for b in range(out.shape[0]):
+        for a, e in image_spans(types[b]):
+            out[b, a:e + 1, a:e + 1] = 0
+    return out
 
 
 def encode(inp, n_layers: int | None = None):

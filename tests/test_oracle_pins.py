@@ -399,3 +399,109 @@ def test_patch_merger_composition_and_padding():
     merged, _ = O.aligner_merge(xn, grids, r)
     np.testing.assert_allclose(out_i, O.gelu(merged) @ w2.T + b2, rtol=1e-12, atol=1e-12)
 
+
+
+# ------------------------------------------------------------------------ image-token bridge
+def _golden_rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def test_image_layout_hand_table_and_length():
+    # hand-written layout of a 3x5 grid at r = 2; catches a missing newline, a swapped
+    # start/end or a token row of the wrong width.
+    want = [int(v) for v in _golden_rows("image_layout_3x5_r2.txt")[0]]
+    assert O.image_layout(3, 5, 2).tolist() == want
+    # closed form: 2 + g_h (g_w + 1) entries, g_h g_w of them features; the pages' grids.
+    for n_h, n_w in [(28, 28), (27, 37), (37, 27), (10, 78), (112, 7), (1, 1)]:
+        for r in (1, 2, 3):
+            g_h, g_w = -(-n_h // r), -(-n_w // r)
+            lay = O.image_layout(n_h, n_w, r)
+            assert len(lay) == 2 + g_h * (g_w + 1)
+            assert int((lay == O.TOK_IMAGE).sum()) == g_h * g_w
+            assert int((lay == O.TOK_NEWLINE).sum()) == g_h
+            # each newline closes a row: it sits g_w + 1 after the previous one
+            nl = np.flatnonzero(lay == O.TOK_NEWLINE)
+            assert (np.diff(np.concatenate([[0], nl])) == g_w + 1).all()
+
+
+def _bridge_case():
+    # two sequences of 24 holding three images (3x5 -> 6 tokens, 1x1 -> 1, 4x4 -> 4 at r = 2)
+    # with text around and between them, and one image_pad inside the last span.
+    lay = [O.image_layout(3, 5, 2), O.image_layout(1, 1, 2), O.image_layout(4, 4, 2)]
+    last = np.concatenate([lay[2][:-1], [O.TOK_PAD], lay[2][-1:]])
+    s0 = np.concatenate([[-1, -1], lay[0], [-1], lay[1], [-1] * 7])
+    s1 = np.concatenate([[-1] * 3, last, [-1] * 12])
+    assert len(s0) == 24 and len(s1) == 24
+    return np.stack([s0, s1]).astype(np.int32), [6, 1, 4]
+
+
+def test_merge_image_embeddings_encoded_rows():
+    # rows carry their own identity: text rows 1000 + position, token k -> k, sentinel i ->
+    # -(i + 1).  Catches a wrong token order, a skipped or repeated token, a sentinel mix-up and
+    # a text row that is touched.
+    types, per_image = _bridge_case()
+    b, s = types.shape
+    e = 3
+    embeds = (1000.0 + np.arange(b * s, dtype=np.float64)).repeat(e).reshape(b, s, e)
+    toks = np.arange(sum(per_image), dtype=np.float64).repeat(e).reshape(-1, e)
+    sent = -(1.0 + np.arange(4, dtype=np.float64)).repeat(e).reshape(4, e)
+    out = O.merge_image_embeddings(embeds, types, toks, sent, per_image)
+    flat_t, flat_o, flat_in = types.reshape(-1), out.reshape(-1, e), embeds.reshape(-1, e)
+    feats = flat_o[flat_t == O.TOK_IMAGE, 0]
+    assert feats.tolist() == list(range(sum(per_image)))
+    for code, row in zip(O.SENTINEL_ORDER, range(4)):
+        assert (flat_o[flat_t == code] == -(row + 1.0)).all()
+    np.testing.assert_array_equal(flat_o[flat_t == O.TOK_TEXT], flat_in[flat_t == O.TOK_TEXT])
+    assert int((flat_t == O.TOK_PAD).sum()) == 1
+
+
+@pytest.mark.parametrize("mutate", ["drop_feature", "extra_feature", "open_span", "stray_pad",
+                                    "nested_start", "bad_code", "few_images"])
+def test_merge_image_embeddings_rejects_layouts_that_do_not_fit(mutate):
+    types, per_image = _bridge_case()
+    t = types.copy()
+    f0 = int(np.flatnonzero(t[0] == O.TOK_IMAGE)[0])
+    if mutate == "drop_feature":
+        t[0, f0] = O.TOK_PAD
+    elif mutate == "extra_feature":
+        t[1, int(np.flatnonzero(t[1] == O.TOK_PAD)[0])] = O.TOK_IMAGE
+    elif mutate == "open_span":
+        t[1, int(np.flatnonzero(t[1] == O.TOK_END)[0])] = O.TOK_NEWLINE
+    elif mutate == "stray_pad":
+        t[0, 0] = O.TOK_PAD
+    elif mutate == "nested_start":
+        t[0, f0] = O.TOK_START
+    elif mutate == "bad_code":
+        t[0, 0] = 7
+    elif mutate == "few_images":
+        per_image = per_image + [1]
+    z = np.zeros(t.shape + (2,))
+    with pytest.raises(ValueError):
+        O.merge_image_embeddings(z, t, np.zeros((sum(per_image), 2)), np.zeros((4, 2)), per_image)
+
+
+def test_image_visibility_hand_table():
+    rows = _golden_rows("image_visibility_12.txt")
+    types = np.array([[int(v) for v in rows[0]]])
+    n = types.shape[1]
+    causal = np.where(np.arange(n)[None, :] > np.arange(n)[:, None], -np.inf, 0.0)[None]
+    want = np.array([[0.0 if c == "." else -np.inf for c in row] for row in rows[1:]])
+    np.testing.assert_array_equal(O.image_visibility(causal, types)[0], want)
+    assert O.image_spans(types[0]) == [(2, 6), (8, 11)]
+
+
+def test_image_visibility_keeps_text_and_other_samples():
+    # random additive mask: entries outside the spans are untouched, the spans' blocks are 0,
+    # and a sample without images is unchanged; catches a span leaking across samples.
+    types, _ = _bridge_case()
+    types = np.concatenate([types, np.full((1, types.shape[1]), -1, np.int32)])
+    m = RNG.normal(size=(3, 24, 24))
+    out = O.image_visibility(m, types)
+    inside = np.zeros_like(m, dtype=bool)
+    for b in range(3):
+        for a, e in O.image_spans(types[b]):
+            inside[b, a:e + 1, a:e + 1] = True
+    assert inside[0].sum() == 10 ** 2 + 4 ** 2 and inside[1].sum() == 9 ** 2 and not inside[2].any()
+    assert (out[inside] == 0).all()
+    np.testing.assert_array_equal(out[~inside], m[~inside])
