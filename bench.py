@@ -239,7 +239,7 @@ def run_ours(args):
                 step(stream)
         torch.cuda.synchronize()
         print(json.dumps({"profile_run": True, "device_error": A.dsv4v_device_error(),
-                          "kernels_per_step": 5 * wl.n_layers + 5}), flush=True)
+                          "kernels_per_step": 5 * wl.n_layers + 6}), flush=True)
         return
 
     # Capture one step (all kernels of the path, launched through the C ABI) in a CUDA graph.
@@ -253,8 +253,8 @@ def run_ours(args):
     if A.dsv4v_device_error() != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
     # per layer: 4 GEMMs + attention; plus the rotary table, the first norm operand, the final
-    # norm, the aligner index and the aligner GEMM
-    launches_per_step = 5 * wl.n_layers + 5
+    # norm, and the aligner's window index, merged-row copy and GEMM
+    launches_per_step = 5 * wl.n_layers + 6
 
     for _ in range(args.warmup):
         with torch.cuda.stream(stream):
