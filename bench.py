@@ -293,7 +293,8 @@ def run_ours(args):
 
     # ---- the step before the tower: patch embedding of the same patches (14 x 14 RGB patches)
     extras = {"patch_embed": patch_embed_timing(A, torch, cfg, wl, stream, flush, args.steps),
-              "patch_merger": patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, args.steps)}
+              "patch_merger": patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, args.steps),
+              "bridge": bridge_timing(A, torch, cfg, stream, flush, args.steps)}
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     x_host = x0.cpu().pin_memory()
@@ -483,6 +484,67 @@ def patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, steps):
     flops = 2.0 * T * (r2 * D) * (r2 * D) + 2.0 * T * (r2 * D) * E
     return {"avg_us": avg_ms * 1e3, "tflops": flops / (avg_ms * 1e-3) / 1e12, "tokens": T, "launches_per_call": 4,
             "note": "standalone, 20 calls per graph replay; the alternative projector, not in value"}
+
+
+def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
+    """The image-token bridge on a language batch of n_seqs x seq_len positions holding the 16
+    images of the high-resolution batch (N-layouts from dsv4v_image_layout, placed by
+    synth.place_spans with text gaps, one image_pad in every fourth span), E = llm_dim bf16:
+    dsv4v_merge_image_embeddings (2 launches) and dsv4v_image_visibility on an fp32
+    [n_seqs, seq_len, seq_len] mask (1 launch).  Each timed call is preceded by an L2 flush
+    outside its events.  Not part of the tower step above."""
+    import numpy as np
+    grids = synth.workload(5).grids
+    r, E = cfg.downsample_ratio, cfg.llm_dim
+    layouts = [A.dsv4v_image_layout(h, w, r) for h, w in grids]
+    types_np = synth.place_spans(layouts, n_seqs, seq_len, seed=21, pad_every=4, balance=True)
+    b = A.BatchRef(grids)
+    T = A.dsv4v_aligner_tokens(cfg, b)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    types = torch.from_numpy(types_np).cuda()
+    embeds = torch.randn(n_seqs, seq_len, E, device="cuda", generator=g).to(torch.bfloat16)
+    toks = torch.randn(T, E, device="cuda", generator=g).to(torch.bfloat16)
+    sent = torch.randn(4, E, device="cuda", generator=g).to(torch.bfloat16)
+    ws = torch.empty(A.dsv4v_merge_workspace_size(n_seqs * seq_len), dtype=torch.uint8, device="cuda")
+    mask = torch.full((n_seqs, seq_len, seq_len), float("-inf"), device="cuda")
+
+    def timed(fn):
+        out = []
+        for i in range(steps + 3):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ev0.record(stream)
+                fn()
+                ev1.record(stream)
+            stream.synchronize()
+            if i >= 3:
+                out.append(ev0.elapsed_time(ev1))
+        return sum(out) / len(out)
+
+    merge_ms = timed(lambda: A.dsv4v_merge_image_embeddings(cfg, b, types, toks, sent, embeds, ws,
+                                                            stream=stream.cuda_stream))
+    vis_ms = timed(lambda: A.dsv4v_image_visibility(types, mask, stream=stream.cuda_stream))
+    if A.dsv4v_device_error(stream.cuda_stream) != 0:
+        raise RuntimeError("bridge layout rejected on the device")
+    n = n_seqs * seq_len
+    pseudo = int((types_np != -1).sum())
+    merge_bytes = 2.0 * pseudo * E * 2 + 2.0 * n * 4  # each pseudo row read and written; types read twice
+    span_cells = 0
+    for row in types_np:
+        starts, ends = np.flatnonzero(row == 1), np.flatnonzero(row == 2)
+        span_cells += int(((ends - starts + 1) ** 2).sum())
+    vis_bytes = span_cells * 4.0  # the span blocks written; the type scans stay in L1/L2
+    hbm = load_peaks().get("hbm_gbs")
+    merge_gbs = merge_bytes / (merge_ms * 1e-3) / 1e9
+    return {"workload": f"{len(grids)} images ({T} tokens) in {n_seqs} x {seq_len} positions, E={E} bf16",
+            "pseudo_tokens": pseudo,
+            "merge": {"avg_us": merge_ms * 1e3, "bytes": merge_bytes, "gbs": merge_gbs,
+                      "frac_hbm": merge_gbs / hbm if hbm else None, "launches_per_call": 2},
+            "visibility": {"avg_us": vis_ms * 1e3, "bytes_written": vis_bytes,
+                           "gbs": vis_bytes / (vis_ms * 1e-3) / 1e9, "launches_per_call": 1},
+            "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if hbm else None,
+            "note": "standalone, one call per timed interval after an L2 flush; not in value"}
 
 
 def load_peaks():

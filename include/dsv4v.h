@@ -52,9 +52,12 @@ typedef enum {
   DSV4V_ERR_UNSUPPORTED = 2,   /* shape outside the constraints listed at the config below */
   DSV4V_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or smaller than required */
   DSV4V_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
-  DSV4V_ERR_TIMEOUT = 5        /* a device-side check failed: a bounded wait gave up, or the two
+  DSV4V_ERR_TIMEOUT = 5,       /* a device-side check failed: a bounded wait gave up, or the two
                                   CTAs of a GEMM CTA pair got different TMEM addresses (see
                                   dsv4v_device_error) */
+  DSV4V_ERR_LAYOUT = 6         /* pseudo-token types that do not fit the images, found on the
+                                  device by dsv4v_merge_image_embeddings or
+                                  dsv4v_image_visibility (see dsv4v_device_error) */
 } dsv4v_status;
 
 typedef enum { DSV4V_F32 = 0, DSV4V_BF16 = 1 } dsv4v_dtype;
@@ -261,10 +264,11 @@ dsv4v_status dsv4v_swiglu(const dsv4v_config* cfg, int64_t rows, const void* y,
 dsv4v_status dsv4v_linear_residual_noalloc(const dsv4v_config* cfg, int64_t rows, int k,
                                            const void* a, const void* w, void* x, void* stream);
 
-/* Synchronises `stream` and returns DSV4V_ERR_TIMEOUT if a kernel of this library recorded a
- * device-side failure on the current device since the last call (a bounded wait that gave up,
- * or a CTA pair whose TMEM allocations differ), and clears the record; DSV4V_ERR_CUDA if the
- * stream reports an error; else DSV4V_OK. */
+/* Synchronises `stream` and returns the first device-side failure that a kernel of this library
+ * recorded on the current device since the last call, and clears the record:
+ * DSV4V_ERR_LAYOUT for pseudo-token types that do not fit the images (the bridge calls below),
+ * DSV4V_ERR_TIMEOUT for any other (a bounded wait that gave up, or a CTA pair whose TMEM
+ * allocations differ).  DSV4V_ERR_CUDA if the stream reports an error; else DSV4V_OK. */
 dsv4v_status dsv4v_device_error(void* stream);
 
 /* Test hook for the bounded-wait machinery: launches one tiny kernel that waits on an
@@ -273,6 +277,69 @@ dsv4v_status dsv4v_device_error(void* stream);
 dsv4v_status dsv4v_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 const char* dsv4v_status_string(dsv4v_status s);
+
+/* ---------------------------------------------------------------- image-token bridge
+ * [model-API, DeepseekV4Model]: the sentinel parameters image_start, image_end, image_newline
+ * and image_pad; merge_image_embeddings; apply_deepseek_v4_image_visibility.
+ * Pseudo-token types, one int32 per sequence position.  The pages state only -1 = text; the
+ * other codes are a reading.  A span runs from an image_start to the next image_end of the
+ * same sequence, and every other pseudo token must lie inside one. */
+enum {
+  DSV4V_TOKEN_TEXT = -1,
+  DSV4V_TOKEN_IMAGE = 0,    /* takes the next aligner token of its image */
+  DSV4V_TOKEN_START = 1,    /* image_start sentinel (sentinel row 0) */
+  DSV4V_TOKEN_END = 2,      /* image_end sentinel (row 1) */
+  DSV4V_TOKEN_NEWLINE = 3,  /* image_newline sentinel (row 2) */
+  DSV4V_TOKEN_PAD = 4       /* image_pad sentinel (row 3) */
+};
+
+/* The N-layout of one image (host computation, reading adopted): image_start, then each of the
+ * ceil(grid_h / r) rows of ceil(grid_w / r) aligner tokens followed by image_newline, then
+ * image_end: 2 + rows * (cols + 1) types.  *length_out (if non-NULL) receives that length.
+ * types_out: host int32 array of `capacity` entries, written if non-NULL.
+ * DSV4V_ERR_INVALID_ARG for a grid or r below 1, or types_out with capacity below the length
+ * (nothing is written then). */
+dsv4v_status dsv4v_image_layout(int grid_h, int grid_w, int downsample_ratio, int32_t* types_out,
+                                int64_t capacity, int64_t* length_out);
+
+/* Bytes of device scratch dsv4v_merge_image_embeddings needs for n_positions positions
+ * (16 bytes per 256 positions, rounded up to 256 bytes); 0 if n_positions < 1. */
+size_t dsv4v_merge_workspace_size(int64_t n_positions);
+
+/* [model-API, DeepseekV4Model.merge_image_embeddings]: replaces every pseudo-token row of the
+ * text embeddings; text rows are not touched.  Reading adopted: the image spans, in batch-major
+ * order, are the batch's images in packing order; the feature positions of the j-th span take
+ * image j's aligner tokens in order, and the span must hold exactly that many.
+ *   token_types:  device int32 [n_seqs * seq_len], batch-major.
+ *   image_tokens: device [T, E] in the config dtype (dsv4v_aligner_forward's output; T and the
+ *                 per-image counts follow from cfg->downsample_ratio and the batch's grids).
+ *   sentinels:    device [4, E] in the config dtype: image_start, image_end, image_newline,
+ *                 image_pad.
+ *   embeds:       device [n_seqs, seq_len, E] in the config dtype, updated in place; must not
+ *                 overlap image_tokens or sentinels.
+ * E = cfg->llm_dim; E times the element size must be a multiple of 16 bytes, and the three
+ * matrices 16-byte aligned (else DSV4V_ERR_UNSUPPORTED / DSV4V_ERR_INVALID_ARG).
+ * n_seqs * seq_len < 2^31.  workspace: device, 256-byte aligned, at least
+ * dsv4v_merge_workspace_size(n_seqs * seq_len) bytes.  Types that do not fit the images (an
+ * unknown code, a pseudo token outside a span, an unclosed or nested span, a span whose
+ * feature count differs from its image's, more or fewer spans than images) are found on the
+ * device: the offending rows are left as they were, and the next dsv4v_device_error returns
+ * DSV4V_ERR_LAYOUT. */
+dsv4v_status dsv4v_merge_image_embeddings(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                          int64_t n_seqs, int64_t seq_len,
+                                          const int32_t* token_types, const void* image_tokens,
+                                          const void* sentinels, void* embeds, void* workspace,
+                                          size_t ws_bytes, void* stream);
+
+/* [model-API, apply_deepseek_v4_image_visibility]: every pair of positions inside one image
+ * span becomes visible (entry set to 0); every other entry is kept.
+ *   token_types: device int32 [n_seqs * seq_len], batch-major.
+ *   mask:        device additive mask [n_seqs, seq_len, seq_len] (the pages' [batch, 1, seq,
+ *                seq]) of elem_bytes 2 (bf16 / fp16) or 4 (fp32) per entry, updated in place.
+ * A row of a pseudo token that is not inside a well-formed span is left as it was, and the next
+ * dsv4v_device_error returns DSV4V_ERR_LAYOUT. */
+dsv4v_status dsv4v_image_visibility(int64_t n_seqs, int64_t seq_len, const int32_t* token_types,
+                                    void* mask, int elem_bytes, void* stream);
 
 #ifdef __cplusplus
 }

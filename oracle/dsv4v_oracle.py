@@ -312,11 +312,7 @@ def merge_image_embeddings(embeds, types, image_tokens, sentinels, tokens_per_im
     cu = np.concatenate([[0], np.cumsum(tokens_per_image)]).astype(np.int64)
     j = 0
     for b in range(types.shape[0]):
-        spans = image_spans(types[b])
-        for p, t in enumerate(types[b]):
-            if t not in (TOK_TEXT, TOK_IMAGE) and t not in SENTINEL_ORDER:
-                raise ValueError(f"unknown pseudo-token type {t} at ({b}, {p})")
-        for a, e in spans:
+        for a, e in image_spans(types[b]):
             if j >= len(tokens_per_image):
                 raise ValueError(f"more image spans than the {len(tokens_per_image)} images")
             k = cu[j]
@@ -339,11 +335,17 @@ def merge_image_embeddings(embeds, types, image_tokens, sentinels, tokens_per_im
 
 def image_spans(types_row):
     """Image spans of one sequence as inclusive (start, end) pairs.  READING 17: a span runs from
-    an image_start to the next image_end; a pseudo token outside such a pair, an image_start
-    inside an open span or a span left open at the end is an error (ValueError)."""
+    an image_start to the next image_end and holds pseudo tokens only; a pseudo token outside
+    such a pair, text inside one, an image_start inside an open span, a span left open at the
+    end or an unknown type code is an error (ValueError)."""
     spans, open_at = [], None
     for p, t in enumerate(types_row):
-        if t == TOK_START:
+        if t != TOK_TEXT and t != TOK_IMAGE and t not in SENTINEL_ORDER:
+            raise ValueError(f"unknown pseudo-token type {t} at {p}")
+        if t == TOK_TEXT:
+            if open_at is not None:
+                raise ValueError(f"text at {p} inside the span opened at {open_at}")
+        elif t == TOK_START:
             if open_at is not None:
                 raise ValueError(f"image_start at {p} inside the span opened at {open_at}")
             open_at = p
@@ -352,7 +354,7 @@ def image_spans(types_row):
                 raise ValueError(f"image_end at {p} outside a span")
             spans.append((open_at, p))
             open_at = None
-        elif t != TOK_TEXT and open_at is None:
+        elif open_at is None:
             raise ValueError(f"pseudo token {t} at {p} outside a span")
     if open_at is not None:
         raise ValueError(f"span opened at {open_at} is not closed")

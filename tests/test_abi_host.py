@@ -107,3 +107,51 @@ def test_host_validation_rejects(lib, case, status):
     assert lib.dsv4v_workspace_size(cp, ctypes.byref(b.c)) == 0
     st = lib.dsv4v_aligner_forward(cp, ctypes.byref(b.c), x, x, x, None, x, 1 << 30, None)
     assert st == status
+
+
+# ------------------------------------------------------------------------ image-token bridge
+def test_image_layout_host_matches_oracle(lib):
+    # the library's host N-layout against the oracle's, on the pages' grids and edge grids
+    import numpy as np
+    from oracle import dsv4v_oracle as O
+    for n_h, n_w in [(28, 28), (27, 37), (37, 27), (10, 78), (112, 7), (1, 1), (1, 9), (9, 1)]:
+        for r in (1, 2, 3, 4):
+            np.testing.assert_array_equal(A.dsv4v_image_layout(n_h, n_w, r), O.image_layout(n_h, n_w, r))
+
+
+def test_image_layout_argument_checks(lib):
+    n = ctypes.c_int64(-1)
+    assert lib.dsv4v_image_layout(0, 5, 2, None, 0, ctypes.byref(n)) == 1
+    assert lib.dsv4v_image_layout(3, 5, 0, None, 0, ctypes.byref(n)) == 1
+    assert lib.dsv4v_image_layout(3, 5, 2, None, 0, ctypes.byref(n)) == 0 and n.value == 10
+    buf = (ctypes.c_int32 * 9)(*([77] * 9))
+    assert lib.dsv4v_image_layout(3, 5, 2, ctypes.addressof(buf), 9, None) == 1  # too small
+    assert list(buf) == [77] * 9  # nothing written
+
+
+def test_merge_workspace_size(lib):
+    assert A.dsv4v_merge_workspace_size(0) == 0
+    assert A.dsv4v_merge_workspace_size(1) == 256
+    assert A.dsv4v_merge_workspace_size(256 * 16) == 256
+    assert A.dsv4v_merge_workspace_size(256 * 16 + 1) == 512
+
+
+def test_bridge_host_validation_rejects(lib):
+    # every rejection below happens on the host, before any CUDA call
+    b = HostBatch([(3, 5)])
+    c = cfg()
+    al = 4096  # a 16-byte aligned fake address; never dereferenced
+    ws = 1 << 20
+    merge = lib.dsv4v_merge_image_embeddings
+    assert merge(ctypes.byref(c), ctypes.byref(b.c), 0, 8, al, al, al, al, al, ws, None) == 1  # no sequences
+    assert merge(ctypes.byref(c), ctypes.byref(b.c), 1, 8, None, al, al, al, al, ws, None) == 1  # no types
+    assert merge(ctypes.byref(c), ctypes.byref(b.c), 1, 8, al, al + 8, al, al, al, ws, None) == 1  # misaligned
+    assert merge(ctypes.byref(c), ctypes.byref(b.c), 1, 8, al, al, al, al, al, 0, None) == 3  # workspace
+    assert merge(ctypes.byref(c), ctypes.byref(b.c), 1 << 20, 1 << 12, al, al, al, al, al, ws, None) == 1  # > 2^31
+    f32 = cfg(dtype=A.DSV4V_F32, llm_dim=6, vision_dim=64, n_heads=4, mlp_hidden=96)
+    assert merge(ctypes.byref(f32), ctypes.byref(b.c), 1, 8, al, al, al, al, al, ws, None) == 2  # 24-byte rows
+    vis = lib.dsv4v_image_visibility
+    assert vis(1, 8, al, al, 3, None) == 1  # element size
+    assert vis(1, 8, al, al + 2, 4, None) == 1  # misaligned fp32 mask
+    assert vis(0, 8, al, al, 4, None) == 1
+    assert vis(1, 8, None, al, 4, None) == 1

@@ -457,7 +457,7 @@ def test_merge_image_embeddings_encoded_rows():
 
 
 @pytest.mark.parametrize("mutate", ["drop_feature", "extra_feature", "open_span", "stray_pad",
-                                    "nested_start", "bad_code", "few_images"])
+                                    "nested_start", "bad_code", "few_images", "text_in_span"])
 def test_merge_image_embeddings_rejects_layouts_that_do_not_fit(mutate):
     types, per_image = _bridge_case()
     t = types.copy()
@@ -476,6 +476,8 @@ def test_merge_image_embeddings_rejects_layouts_that_do_not_fit(mutate):
         t[0, 0] = 7
     elif mutate == "few_images":
         per_image = per_image + [1]
+    elif mutate == "text_in_span":  # feature counts intact, one newline turned into text
+        t[0, int(np.flatnonzero(t[0] == O.TOK_NEWLINE)[0])] = O.TOK_TEXT
     z = np.zeros(t.shape + (2,))
     with pytest.raises(ValueError):
         O.merge_image_embeddings(z, t, np.zeros((sum(per_image), 2)), np.zeros((4, 2)), per_image)

@@ -549,7 +549,8 @@ const char* dsv4v_status_string(dsv4v_status s) {
     case DSV4V_ERR_UNSUPPORTED: return "unsupported shape";
     case DSV4V_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case DSV4V_ERR_CUDA: return "CUDA error";
-    case DSV4V_ERR_TIMEOUT: return "device wait timed out";
+    case DSV4V_ERR_TIMEOUT: return "device-side check failed (wait timed out)";
+    case DSV4V_ERR_LAYOUT: return "pseudo-token types do not fit the images";
   }
   return "unknown status";
 }
@@ -860,7 +861,69 @@ dsv4v_status dsv4v_device_error(void* stream) {
   if (v == 0) return DSV4V_OK;
   const uint32_t zero = 0;
   if (cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return DSV4V_ERR_CUDA;
-  return DSV4V_ERR_TIMEOUT;
+  return v == kErrBridgeLayout ? DSV4V_ERR_LAYOUT : DSV4V_ERR_TIMEOUT;
+}
+
+// ---------------------------------------------------------------------------- image-token bridge
+dsv4v_status dsv4v_image_layout(int grid_h, int grid_w, int downsample_ratio, int32_t* types_out, int64_t capacity,
+                                int64_t* length_out) {
+  if (grid_h < 1 || grid_w < 1 || downsample_ratio < 1) return DSV4V_ERR_INVALID_ARG;
+  const int64_t rows = (grid_h + downsample_ratio - 1) / downsample_ratio;
+  const int64_t cols = (grid_w + downsample_ratio - 1) / downsample_ratio;
+  const int64_t len = 2 + rows * (cols + 1);
+  if (length_out) *length_out = len;
+  if (!types_out) return DSV4V_OK;
+  if (capacity < len) return DSV4V_ERR_INVALID_ARG;
+  int64_t q = 0;
+  types_out[q++] = DSV4V_TOKEN_START;
+  for (int64_t i = 0; i < rows; ++i) {
+    for (int64_t j = 0; j < cols; ++j) types_out[q++] = DSV4V_TOKEN_IMAGE;
+    types_out[q++] = DSV4V_TOKEN_NEWLINE;
+  }
+  types_out[q++] = DSV4V_TOKEN_END;
+  return DSV4V_OK;
+}
+
+size_t dsv4v_merge_workspace_size(int64_t n_positions) {
+  if (n_positions < 1) return 0;
+  const size_t chunks = static_cast<size_t>((n_positions + kBridgeChunk - 1) / kBridgeChunk);
+  return up256(chunks * sizeof(int4));
+}
+
+dsv4v_status dsv4v_merge_image_embeddings(const dsv4v_config* cfg, const dsv4v_batch* batch, int64_t n_seqs,
+                                          int64_t seq_len, const int32_t* token_types, const void* image_tokens,
+                                          const void* sentinels, void* embeds, void* workspace, size_t ws_bytes,
+                                          void* stream) {
+  Shape s;
+  DSV4V_TRY(check_all(cfg, batch, s));
+  if (n_seqs < 1 || seq_len < 1 || n_seqs > (int64_t{1} << 31) / seq_len) return DSV4V_ERR_INVALID_ARG;
+  const int64_t n = n_seqs * seq_len;
+  if (n >= (int64_t{1} << 31)) return DSV4V_ERR_INVALID_ARG;
+  if (!token_types || (reinterpret_cast<uintptr_t>(token_types) & 3u)) return DSV4V_ERR_INVALID_ARG;
+  for (const void* ptr : {image_tokens, sentinels, static_cast<const void*>(embeds)})
+    if (!ptr || !aligned16(ptr)) return DSV4V_ERR_INVALID_ARG;
+  const size_t row_bytes = static_cast<size_t>(s.E) * (s.bf16 ? 2 : 4);
+  if (row_bytes % 16) return DSV4V_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < dsv4v_merge_workspace_size(n))
+    return DSV4V_ERR_WORKSPACE;
+  DeviceInfo d;
+  if (!device_info(d)) return DSV4V_ERR_CUDA;
+  return cuda_status(launch_bridge_merge(token_types, n, seq_len, static_cast<int4*>(workspace), batch->grid_hw_dev,
+                                         batch->n_images, s.r, s.T, image_tokens, sentinels, embeds,
+                                         static_cast<int>(row_bytes / 16), d.err, static_cast<cudaStream_t>(stream)));
+}
+
+dsv4v_status dsv4v_image_visibility(int64_t n_seqs, int64_t seq_len, const int32_t* token_types, void* mask,
+                                    int elem_bytes, void* stream) {
+  if (n_seqs < 1 || seq_len < 1 || n_seqs > (int64_t{1} << 31) / seq_len) return DSV4V_ERR_INVALID_ARG;
+  if (elem_bytes != 2 && elem_bytes != 4) return DSV4V_ERR_INVALID_ARG;
+  if (!token_types || (reinterpret_cast<uintptr_t>(token_types) & 3u)) return DSV4V_ERR_INVALID_ARG;
+  if (!mask || (reinterpret_cast<uintptr_t>(mask) & static_cast<uintptr_t>(elem_bytes - 1)))
+    return DSV4V_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (!device_info(d)) return DSV4V_ERR_CUDA;
+  return cuda_status(launch_image_visibility(token_types, n_seqs, seq_len, mask, elem_bytes, d.err,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 dsv4v_status dsv4v_selftest_bounded_wait(uint64_t limit_ns, void* stream) {

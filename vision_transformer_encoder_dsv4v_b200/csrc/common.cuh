@@ -21,6 +21,7 @@ enum : uint32_t {
   kErrTimeoutGather = 0x400,
   kErrTimeoutSelftest = 0x500,
   kErrPairTmem = 0x600,  // the two CTAs of a pair received different TMEM addresses
+  kErrBridgeLayout = 0x700,  // pseudo-token types that do not fit the images (image-token bridge)
 };
 
 // A wait that exceeds this many nanoseconds gives up, records an error and lets the kernel

@@ -111,6 +111,14 @@ cudaError_t launch_merge_rows_bf16(const void* x, const int32_t* src, void* merg
 cudaError_t launch_ln_merge(bool bf16, const void* x, const int32_t* src, const float* w, const float* b, float eps,
                             void* merged, int64_t n_tokens, int r2, int d, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
+// Image-token bridge (bridge.cu).  Positions per CTA of the merge; counts holds one int4 per
+// chunk of that many positions.
+constexpr int kBridgeChunk = 256;
+cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, int4* counts, const int32_t* grid_dev,
+                                int n_images, int r, int64_t n_tokens, const void* image_tokens, const void* sentinels,
+                                void* embeds, int row_vec, uint32_t* err, cudaStream_t s);
+cudaError_t launch_image_visibility(const int32_t* types, int64_t batch, int64_t seq, void* mask, int elem_bytes,
+                                    uint32_t* err, cudaStream_t s);
 // Norm operands of the first GEMM of a block: xw = bf16(x * w) and ss[p * parts] = sum_c x[p,c]^2
 // (the other parts of a row are zero-filled); also clears zero_n counters like the kernels above.
 cudaError_t launch_norm_prep(const void* x, const float* w, void* xw, float* ss, int parts, int64_t rows, int d,

@@ -17,7 +17,12 @@ DSV4V_BF16 = 1
 DSV4V_MAX_IMAGES = 1024
 
 STATUS = {0: "DSV4V_OK", 1: "DSV4V_ERR_INVALID_ARG", 2: "DSV4V_ERR_UNSUPPORTED", 3: "DSV4V_ERR_WORKSPACE",
-          4: "DSV4V_ERR_CUDA", 5: "DSV4V_ERR_TIMEOUT"}
+          4: "DSV4V_ERR_CUDA", 5: "DSV4V_ERR_TIMEOUT", 6: "DSV4V_ERR_LAYOUT"}
+DSV4V_ERR_TIMEOUT = 5
+DSV4V_ERR_LAYOUT = 6
+
+# Pseudo-token types of the image-token bridge (DSV4V_TOKEN_*); sentinel rows follow types 1..4.
+TOKEN_TEXT, TOKEN_IMAGE, TOKEN_START, TOKEN_END, TOKEN_NEWLINE, TOKEN_PAD = -1, 0, 1, 2, 3, 4
 
 PROFILE_KINDS = ("qkv", "attention", "out", "swiglu", "down")  # DSV4V_PROFILE_* order
 
@@ -27,7 +32,8 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_aligner_forward", "dsv4v_aligner_tokens", "dsv4v_rmsnorm", "dsv4v_qkv_rope", "dsv4v_attention",
            "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
            "dsv4v_status_string", "dsv4v_linear_residual_noalloc", "dsv4v_patch_embed",
-           "dsv4v_patch_merger_workspace_size", "dsv4v_patch_merger_forward")
+           "dsv4v_patch_merger_workspace_size", "dsv4v_patch_merger_forward", "dsv4v_image_layout",
+           "dsv4v_merge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -84,6 +90,10 @@ def lib() -> ctypes.CDLL:
             "dsv4v_patch_merger_workspace_size": (SZ, [cfg, bat]),
             "dsv4v_patch_merger_forward": (I, [cfg, bat, P, P, P, P, P, P, P, P, P, SZ, P]),
             "dsv4v_linear_residual_noalloc": (I, [cfg, I64, I, P, P, P, P]),
+            "dsv4v_image_layout": (I, [I, I, I, P, I64, ctypes.POINTER(ctypes.c_int64)]),
+            "dsv4v_merge_workspace_size": (SZ, [I64]),
+            "dsv4v_merge_image_embeddings": (I, [cfg, bat, I64, I64, P, P, P, P, P, SZ, P]),
+            "dsv4v_image_visibility": (I, [I64, I64, P, P, I, P]),
             "dsv4v_device_error": (I, [P]),
             "dsv4v_selftest_bounded_wait": (I, [U64, P]),
             "dsv4v_status_string": (ctypes.c_char_p, [I]),
@@ -239,6 +249,43 @@ def dsv4v_patch_merger_forward(cfg, batch, x, ln_w, ln_b, w1, b1, w2, b2, out, w
                                             _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(out), _ptr(workspace),
                                             workspace.numel() if workspace is not None else 0, _stream(stream)),
            "dsv4v_patch_merger_forward")
+
+
+def dsv4v_image_layout(grid_h: int, grid_w: int, downsample_ratio: int):
+    """N-layout of one image as a host numpy int32 array (computed by the C library)."""
+    import numpy as np
+    n = ctypes.c_int64(0)
+    _check(lib().dsv4v_image_layout(grid_h, grid_w, downsample_ratio, None, 0, ctypes.byref(n)), "dsv4v_image_layout")
+    out = np.empty(n.value, dtype=np.int32)
+    _check(lib().dsv4v_image_layout(grid_h, grid_w, downsample_ratio, out.ctypes.data_as(ctypes.c_void_p), n.value,
+                                    None), "dsv4v_image_layout")
+    return out
+
+
+def dsv4v_merge_workspace_size(n_positions: int) -> int:
+    return int(lib().dsv4v_merge_workspace_size(n_positions))
+
+
+def dsv4v_merge_image_embeddings(cfg, batch, token_types, image_tokens, sentinels, embeds, workspace, stream=None):
+    """embeds [n_seqs, seq_len, E] (updated in place) <- image tokens and sentinels at the
+    pseudo-token positions of token_types [n_seqs, seq_len] (int32)."""
+    n_seqs, seq_len = int(embeds.shape[0]), int(embeds.shape[1])
+    _check(lib().dsv4v_merge_image_embeddings(ctypes.byref(cfg), ctypes.byref(batch.c), n_seqs, seq_len,
+                                              _ptr(token_types), _ptr(image_tokens), _ptr(sentinels), _ptr(embeds),
+                                              _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                              _stream(stream)),
+           "dsv4v_merge_image_embeddings")
+
+
+def dsv4v_image_visibility(token_types, mask, stream=None):
+    """mask [n_seqs, seq_len, seq_len] (or with a unit head axis), updated in place: every pair
+    inside one image span of token_types [n_seqs, seq_len] becomes 0."""
+    n_seqs, seq_len = int(token_types.shape[0]), int(token_types.shape[1])
+    if mask.numel() != n_seqs * seq_len * seq_len:
+        raise ValueError(f"mask has {mask.numel()} entries, expected {n_seqs} x {seq_len} x {seq_len}")
+    _check(lib().dsv4v_image_visibility(n_seqs, seq_len, _ptr(token_types), _ptr(mask), mask.element_size(),
+                                        _stream(stream)),
+           "dsv4v_image_visibility")
 
 
 def dsv4v_device_error(stream=None) -> int:

@@ -180,3 +180,33 @@ def algorithmic_flops(wl: Workload, n_layers: int | None = None, aligner: bool |
         r = wl.downsample_ratio
         total += 2.0 * wl.n_tokens * r * r * D * wl.llm_dim
     return total
+
+
+def place_spans(layouts, n_seqs: int, seq_len: int, seed: int, max_gap: int = 40, pad_every: int = 0,
+                balance: bool = False) -> np.ndarray:
+    """A seeded [n_seqs, seq_len] int32 pseudo-token type array: the given per-image layouts
+    (int32 arrays, in image order) placed left to right into text (-1) sequences, each preceded
+    by a text gap drawn uniformly from 0..max_gap.  By default an image moves to the next
+    sequence when it does not fit; with balance=True image i goes to sequence
+    floor(i * n_seqs / n_images), so the sequences hold contiguous, near-equal groups.  With
+    pad_every = k > 0, every k-th image gets one type-4 entry inserted before its last entry (a
+    filler inside the span).  Raises ValueError if the images do not fit."""
+    rng = np.random.default_rng(seed)
+    out = np.full((n_seqs, seq_len), -1, dtype=np.int32)
+    s, pos = 0, 0
+    n_img = len(layouts)
+    for i, lay in enumerate(layouts):
+        lay = np.asarray(lay, dtype=np.int32)
+        if pad_every and i % pad_every == pad_every - 1:
+            lay = np.concatenate([lay[:-1], np.array([4], np.int32), lay[-1:]])
+        gap = int(rng.integers(0, max_gap + 1))
+        target = i * n_seqs // n_img if balance else s
+        if target != s:
+            s, pos = target, 0
+        elif not balance and pos + gap + len(lay) > seq_len:
+            s, pos = s + 1, 0
+        if s >= n_seqs or pos + gap + len(lay) > seq_len:
+            raise ValueError(f"image {i} ({len(lay)} positions) does not fit")
+        out[s, pos + gap: pos + gap + len(lay)] = lay
+        pos += gap + len(lay)
+    return out
