@@ -491,7 +491,7 @@ def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
     images of the high-resolution batch (N-layouts from dsv4v_image_layout, placed by
     synth.place_spans with text gaps, one image_pad in every fourth span), E = llm_dim bf16:
     dsv4v_merge_image_embeddings (2 launches) and dsv4v_image_visibility on an fp32
-    [n_seqs, seq_len, seq_len] mask (1 launch).  Each timed call is preceded by an L2 flush
+    [n_seqs, seq_len, seq_len] mask (3 launches).  Each timed call is preceded by an L2 flush
     outside its events.  Not part of the tower step above."""
     import numpy as np
     grids = synth.workload(5).grids
@@ -505,7 +505,7 @@ def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
     embeds = torch.randn(n_seqs, seq_len, E, device="cuda", generator=g).to(torch.bfloat16)
     toks = torch.randn(T, E, device="cuda", generator=g).to(torch.bfloat16)
     sent = torch.randn(4, E, device="cuda", generator=g).to(torch.bfloat16)
-    ws = torch.empty(A.dsv4v_merge_workspace_size(n_seqs * seq_len), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(A.dsv4v_bridge_workspace_size(n_seqs * seq_len), dtype=torch.uint8, device="cuda")
     mask = torch.full((n_seqs, seq_len, seq_len), float("-inf"), device="cuda")
 
     def timed(fn):
@@ -524,7 +524,7 @@ def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
 
     merge_ms = timed(lambda: A.dsv4v_merge_image_embeddings(cfg, b, types, toks, sent, embeds, ws,
                                                             stream=stream.cuda_stream))
-    vis_ms = timed(lambda: A.dsv4v_image_visibility(types, mask, stream=stream.cuda_stream))
+    vis_ms = timed(lambda: A.dsv4v_image_visibility(types, mask, ws, stream=stream.cuda_stream))
     if A.dsv4v_device_error(stream.cuda_stream) != 0:
         raise RuntimeError("bridge layout rejected on the device")
     n = n_seqs * seq_len
@@ -542,7 +542,7 @@ def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
             "merge": {"avg_us": merge_ms * 1e3, "bytes": merge_bytes, "gbs": merge_gbs,
                       "frac_hbm": merge_gbs / hbm if hbm else None, "launches_per_call": 2},
             "visibility": {"avg_us": vis_ms * 1e3, "bytes_written": vis_bytes,
-                           "gbs": vis_bytes / (vis_ms * 1e-3) / 1e9, "launches_per_call": 1},
+                           "gbs": vis_bytes / (vis_ms * 1e-3) / 1e9, "launches_per_call": 3},
             "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if hbm else None,
             "note": "standalone, one call per timed interval after an L2 flush; not in value"}
 

@@ -302,9 +302,10 @@ enum {
 dsv4v_status dsv4v_image_layout(int grid_h, int grid_w, int downsample_ratio, int32_t* types_out,
                                 int64_t capacity, int64_t* length_out);
 
-/* Bytes of device scratch dsv4v_merge_image_embeddings needs for n_positions positions
- * (16 bytes per 256 positions, rounded up to 256 bytes); 0 if n_positions < 1. */
-size_t dsv4v_merge_workspace_size(int64_t n_positions);
+/* Bytes of device scratch that dsv4v_merge_image_embeddings and dsv4v_image_visibility need for
+ * n_positions = n_seqs * seq_len positions (16 bytes per 256 positions plus 12 bytes per
+ * position, each part rounded up to 256 bytes); 0 unless 1 <= n_positions < 2^31. */
+size_t dsv4v_bridge_workspace_size(int64_t n_positions);
 
 /* [model-API, DeepseekV4Model.merge_image_embeddings]: replaces every pseudo-token row of the
  * text embeddings; text rows are not touched.  Reading adopted: the image spans, in batch-major
@@ -320,7 +321,7 @@ size_t dsv4v_merge_workspace_size(int64_t n_positions);
  * E = cfg->llm_dim; E times the element size must be a multiple of 16 bytes, and the three
  * matrices 16-byte aligned (else DSV4V_ERR_UNSUPPORTED / DSV4V_ERR_INVALID_ARG).
  * n_seqs * seq_len < 2^31.  workspace: device, 256-byte aligned, at least
- * dsv4v_merge_workspace_size(n_seqs * seq_len) bytes.  Types that do not fit the images (an
+ * dsv4v_bridge_workspace_size(n_seqs * seq_len) bytes.  Types that do not fit the images (an
  * unknown code, a pseudo token outside a span, an unclosed or nested span, a span whose
  * feature count differs from its image's, more or fewer spans than images) are found on the
  * device: the offending rows are left as they were, and the next dsv4v_device_error returns
@@ -335,11 +336,17 @@ dsv4v_status dsv4v_merge_image_embeddings(const dsv4v_config* cfg, const dsv4v_b
  * span becomes visible (entry set to 0); every other entry is kept.
  *   token_types: device int32 [n_seqs * seq_len], batch-major.
  *   mask:        device additive mask [n_seqs, seq_len, seq_len] (the pages' [batch, 1, seq,
- *                seq]) of elem_bytes 2 (bf16 / fp16) or 4 (fp32) per entry, updated in place.
- * A row of a pseudo token that is not inside a well-formed span is left as it was, and the next
- * dsv4v_device_error returns DSV4V_ERR_LAYOUT. */
+ *                seq]) of elem_bytes 2 (bf16 / fp16) or 4 (fp32) per entry, elem_bytes-aligned,
+ *                updated in place.
+ *   workspace:   device, 256-byte aligned, at least dsv4v_bridge_workspace_size(n_seqs *
+ *                seq_len) bytes.
+ * Types that are not well formed (see dsv4v_merge_image_embeddings) are found on the device:
+ * the next dsv4v_device_error returns DSV4V_ERR_LAYOUT, and the mask may then hold zeros in
+ * some rows of the malformed spans; rows of text and entries outside each row's own sequence
+ * are never written. */
 dsv4v_status dsv4v_image_visibility(int64_t n_seqs, int64_t seq_len, const int32_t* token_types,
-                                    void* mask, int elem_bytes, void* stream);
+                                    void* mask, int elem_bytes, void* workspace, size_t ws_bytes,
+                                    void* stream);
 
 #ifdef __cplusplus
 }

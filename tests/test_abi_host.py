@@ -129,11 +129,12 @@ def test_image_layout_argument_checks(lib):
     assert list(buf) == [77] * 9  # nothing written
 
 
-def test_merge_workspace_size(lib):
-    assert A.dsv4v_merge_workspace_size(0) == 0
-    assert A.dsv4v_merge_workspace_size(1) == 256
-    assert A.dsv4v_merge_workspace_size(256 * 16) == 256
-    assert A.dsv4v_merge_workspace_size(256 * 16 + 1) == 512
+def test_bridge_workspace_size(lib):
+    assert A.dsv4v_bridge_workspace_size(0) == 0
+    assert A.dsv4v_bridge_workspace_size(1 << 31) == 0
+    assert A.dsv4v_bridge_workspace_size(1) == 256 * 4  # counts + three int32 tables
+    n = 256 * 16 + 1  # 17 chunks of counts (272 bytes -> 512), tables of 16388 bytes (-> 16640)
+    assert A.dsv4v_bridge_workspace_size(n) == 512 + 3 * 16640
 
 
 def test_bridge_host_validation_rejects(lib):
@@ -151,7 +152,9 @@ def test_bridge_host_validation_rejects(lib):
     f32 = cfg(dtype=A.DSV4V_F32, llm_dim=6, vision_dim=64, n_heads=4, mlp_hidden=96)
     assert merge(ctypes.byref(f32), ctypes.byref(b.c), 1, 8, al, al, al, al, al, ws, None) == 2  # 24-byte rows
     vis = lib.dsv4v_image_visibility
-    assert vis(1, 8, al, al, 3, None) == 1  # element size
-    assert vis(1, 8, al, al + 2, 4, None) == 1  # misaligned fp32 mask
-    assert vis(0, 8, al, al, 4, None) == 1
-    assert vis(1, 8, None, al, 4, None) == 1
+    assert vis(1, 8, al, al, 3, al, ws, None) == 1  # element size
+    assert vis(1, 8, al, al + 2, 4, al, ws, None) == 1  # misaligned fp32 mask
+    assert vis(0, 8, al, al, 4, al, ws, None) == 1
+    assert vis(1, 8, None, al, 4, al, ws, None) == 1
+    assert vis(1, 8, al, al, 4, al + 16, ws, None) == 3  # workspace not 256-byte aligned
+    assert vis(1, 8, al, al, 4, al, 100, None) == 3  # workspace too small

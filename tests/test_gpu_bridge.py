@@ -44,10 +44,14 @@ def raw(t):
     return t.cpu().view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32).numpy()
 
 
+def bridge_ws(types):
+    return torch.empty(A.dsv4v_bridge_workspace_size(types.size), dtype=torch.uint8, device="cuda")
+
+
 def run_merge(cfg, grids, types, embeds_bits, tok_bits, sent_bits, dtype):
     b = A.BatchRef(grids)
     embeds = to_dev(embeds_bits, dtype)
-    ws = torch.empty(A.dsv4v_merge_workspace_size(types.size), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(A.dsv4v_bridge_workspace_size(types.size), dtype=torch.uint8, device="cuda")
     A.dsv4v_merge_image_embeddings(cfg, b, torch.from_numpy(types).cuda(), to_dev(tok_bits, dtype),
                                    to_dev(sent_bits, dtype), embeds, ws)
     return embeds, A.dsv4v_device_error()
@@ -148,7 +152,7 @@ def test_image_visibility_bit_exact(elem, case):
     mask = torch.from_numpy(m).cuda()
     if elem == 2:
         mask = mask.to(torch.bfloat16)
-    A.dsv4v_image_visibility(torch.from_numpy(types).cuda(), mask)
+    A.dsv4v_image_visibility(torch.from_numpy(types).cuda(), mask, bridge_ws(types))
     assert A.dsv4v_device_error() == 0
     want = O.image_visibility(m.astype(np.float64), types)
     got = mask.float().cpu().numpy().astype(np.float64)
@@ -171,7 +175,7 @@ def test_image_visibility_reports_layout_errors(bad):
     with pytest.raises(ValueError):
         O.image_spans(types[0])
     mask = torch.zeros(1, 70, 70, device="cuda")
-    A.dsv4v_image_visibility(torch.from_numpy(types).cuda(), mask)
+    A.dsv4v_image_visibility(torch.from_numpy(types).cuda(), mask, bridge_ws(types))
     assert A.dsv4v_device_error() == A.DSV4V_ERR_LAYOUT
 
 
@@ -191,7 +195,7 @@ def test_bridge_full_size_stream():
     np.testing.assert_array_equal(raw(got), O.merge_image_embeddings(emb, types, tok, sent, per))
     del got
     mask = torch.full((4, 8192, 8192), float("-inf"), device="cuda")
-    A.dsv4v_image_visibility(torch.from_numpy(types).cuda(), mask)
+    A.dsv4v_image_visibility(torch.from_numpy(types).cuda(), mask, bridge_ws(types))
     assert A.dsv4v_device_error() == 0
     rng = np.random.default_rng(25)
     pseudo = np.argwhere(types != O.TOK_TEXT)

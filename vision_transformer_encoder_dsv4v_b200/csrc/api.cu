@@ -884,10 +884,27 @@ dsv4v_status dsv4v_image_layout(int grid_h, int grid_w, int downsample_ratio, in
   return DSV4V_OK;
 }
 
-size_t dsv4v_merge_workspace_size(int64_t n_positions) {
-  if (n_positions < 1) return 0;
-  const size_t chunks = static_cast<size_t>((n_positions + kBridgeChunk - 1) / kBridgeChunk);
-  return up256(chunks * sizeof(int4));
+// Bridge scratch: per-chunk counts, then (visibility only) the span tables and the span number
+// of every position.
+struct BridgeLayout {
+  size_t counts, span_first, span_last, span_of, total;
+};
+
+BridgeLayout bridge_layout(int64_t n) {
+  BridgeLayout l{};
+  const size_t chunks = static_cast<size_t>((n + kBridgeChunk - 1) / kBridgeChunk);
+  const size_t ints = up256(static_cast<size_t>(n) * sizeof(int32_t));
+  l.counts = 0;
+  l.span_first = up256(chunks * sizeof(int4));
+  l.span_last = l.span_first + ints;
+  l.span_of = l.span_last + ints;
+  l.total = l.span_of + ints;
+  return l;
+}
+
+size_t dsv4v_bridge_workspace_size(int64_t n_positions) {
+  if (n_positions < 1 || n_positions >= (int64_t{1} << 31)) return 0;
+  return bridge_layout(n_positions).total;
 }
 
 dsv4v_status dsv4v_merge_image_embeddings(const dsv4v_config* cfg, const dsv4v_batch* batch, int64_t n_seqs,
@@ -904,7 +921,7 @@ dsv4v_status dsv4v_merge_image_embeddings(const dsv4v_config* cfg, const dsv4v_b
     if (!ptr || !aligned16(ptr)) return DSV4V_ERR_INVALID_ARG;
   const size_t row_bytes = static_cast<size_t>(s.E) * (s.bf16 ? 2 : 4);
   if (row_bytes % 16) return DSV4V_ERR_UNSUPPORTED;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < dsv4v_merge_workspace_size(n))
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < dsv4v_bridge_workspace_size(n))
     return DSV4V_ERR_WORKSPACE;
   DeviceInfo d;
   if (!device_info(d)) return DSV4V_ERR_CUDA;
@@ -914,16 +931,24 @@ dsv4v_status dsv4v_merge_image_embeddings(const dsv4v_config* cfg, const dsv4v_b
 }
 
 dsv4v_status dsv4v_image_visibility(int64_t n_seqs, int64_t seq_len, const int32_t* token_types, void* mask,
-                                    int elem_bytes, void* stream) {
+                                    int elem_bytes, void* workspace, size_t ws_bytes, void* stream) {
   if (n_seqs < 1 || seq_len < 1 || n_seqs > (int64_t{1} << 31) / seq_len) return DSV4V_ERR_INVALID_ARG;
+  const int64_t n = n_seqs * seq_len;
+  if (n >= (int64_t{1} << 31)) return DSV4V_ERR_INVALID_ARG;
   if (elem_bytes != 2 && elem_bytes != 4) return DSV4V_ERR_INVALID_ARG;
   if (!token_types || (reinterpret_cast<uintptr_t>(token_types) & 3u)) return DSV4V_ERR_INVALID_ARG;
   if (!mask || (reinterpret_cast<uintptr_t>(mask) & static_cast<uintptr_t>(elem_bytes - 1)))
     return DSV4V_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < dsv4v_bridge_workspace_size(n))
+    return DSV4V_ERR_WORKSPACE;
   DeviceInfo d;
   if (!device_info(d)) return DSV4V_ERR_CUDA;
-  return cuda_status(launch_image_visibility(token_types, n_seqs, seq_len, mask, elem_bytes, d.err,
-                                             static_cast<cudaStream_t>(stream)));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const BridgeLayout l = bridge_layout(n);
+  return cuda_status(launch_image_visibility(
+      token_types, n_seqs, seq_len, mask, elem_bytes, reinterpret_cast<int4*>(ws + l.counts),
+      reinterpret_cast<int32_t*>(ws + l.span_first), reinterpret_cast<int32_t*>(ws + l.span_last),
+      reinterpret_cast<int32_t*>(ws + l.span_of), d.err, static_cast<cudaStream_t>(stream)));
 }
 
 dsv4v_status dsv4v_selftest_bounded_wait(uint64_t limit_ns, void* stream) {

@@ -3,10 +3,19 @@
 // the image-span visibility of the additive attention mask (apply_deepseek_v4_image_visibility).
 //
 // Pseudo-token types: -1 text, 0 image feature, 1 image_start, 2 image_end, 3 image_newline,
-// 4 image_pad.  A span runs from an image_start to the next image_end of the same sequence;
-// every other pseudo token lies inside one.  Both operations are copies, so they are bound by
-// HBM: the merge moves each pseudo-token row once (read the source row, write the embedding
-// row); the visibility call writes only the span blocks of the mask.
+// 4 image_pad.  A span runs from an image_start to the next image_end of the same sequence and
+// holds pseudo tokens only; every pseudo token lies inside one.
+//
+// Both calls start with the same two steps over chunks of kBridgeChunk positions: a count of
+// features, starts and ends per chunk, then, per chunk, the exclusive prefix of those counts
+// over the chunks before it plus a ballot scan inside the chunk.  That gives every position its
+// feature index and its span index without any serial pass, and checks the span structure.
+// The data movement that follows is bound by HBM:
+//  * merge: each pseudo-token row is read once (aligner token or sentinel) and written once.
+//    The pseudo rows of a batch gather in few chunks (images sit together in a sequence), so
+//    every chunk is served by `slices` CTAs, each moving its own column slice of the rows.
+//  * visibility: the scan records each span's first and last position; then one warp per mask
+//    row writes the zeros of its span block with 16-byte stores.
 #include "common.cuh"
 #include "internal.h"
 
@@ -15,37 +24,122 @@ namespace dsv4v {
 namespace {
 
 constexpr int kTypeText = -1, kTypeImage = 0, kTypeStart = 1, kTypeEnd = 2, kTypePad = 4;
+constexpr int kWarps = kBridgeChunk / 32;
 
 __device__ __forceinline__ void record(uint32_t* err) { atomicCAS(err, 0u, static_cast<uint32_t>(kErrBridgeLayout)); }
 
-// counts[c] = (features, image_starts, image_ends) among positions [c*kBridgeChunk, ...).
+// counts[c] = (features, image_starts, image_ends) among positions [c*kBridgeChunk, ...).  With
+// span tables (visibility), also marks every span slot of this chunk's positions as unset.
 __global__ void __launch_bounds__(kBridgeChunk) k_bridge_count(const int32_t* __restrict__ types, int64_t n,
-                                                               int4* __restrict__ counts, uint32_t* err) {
+                                                               int4* __restrict__ counts, int32_t* span_first,
+                                                               int32_t* span_last, uint32_t* err) {
   grid_dependency_wait();
   launch_dependents();
   const int64_t p = static_cast<int64_t>(blockIdx.x) * kBridgeChunk + threadIdx.x;
   const int t = p < n ? types[p] : kTypeText;
   if (t < kTypeText || t > kTypePad) record(err);
+  if (span_first && p < n) {
+    span_first[p] = -1;
+    span_last[p] = -1;
+  }
   const int c_img = __syncthreads_count(t == kTypeImage);
   const int c_start = __syncthreads_count(t == kTypeStart);
   const int c_end = __syncthreads_count(t == kTypeEnd);
   if (threadIdx.x == 0) counts[blockIdx.x] = make_int4(c_img, c_start, c_end, 0);
 }
 
-// One CTA per chunk of kBridgeChunk positions.  Each CTA rebuilds the exclusive prefix of the
-// three counts over the chunks before it, scans its own chunk with warp ballots, checks the
-// span structure and the per-image feature counts, then its warps copy the pseudo-token rows
-// (row_vec 16-byte vectors each).
+// What the scan tells one position of the chunk.
+struct PosScan {
+  int64_t p;            // position
+  int t;                // its type (text past the end)
+  int64_t k_img;        // features before p
+  int64_t starts_incl;  // image_starts at or before p
+  int64_t ends_excl;    // image_ends before p
+  bool bad;             // violates the span structure
+  int64_t total[3];     // features, starts, ends up to the end of this chunk
+};
+
+struct ScanSmem {
+  int part[3][kWarps];
+  int64_t base[3];
+};
+
+// Prefix over the previous chunks and ballot scan inside this one; checks that the type is
+// known, that a sequence starts with every span closed, that text lies outside spans and that
+// every other pseudo token lies inside exactly one.  Must be called by all threads of the CTA.
+__device__ __forceinline__ PosScan chunk_scan(const int32_t* __restrict__ types, int64_t n, int64_t seq,
+                                              const int4* __restrict__ counts, ScanSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int64_t acc[3] = {0, 0, 0};
+  for (int c = tid; c < static_cast<int>(blockIdx.x); c += kBridgeChunk) {
+    const int4 v = counts[c];
+    acc[0] += v.x;
+    acc[1] += v.y;
+    acc[2] += v.z;
+  }
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
+  }
+  if (lane == 0)
+    for (int k = 0; k < 3; ++k) sm.part[k][warp] = static_cast<int>(acc[k]);  // fewer than 2^31 positions
+  __syncthreads();
+  if (tid < 3) {
+    int64_t s = 0;
+    for (int w = 0; w < kWarps; ++w) s += sm.part[tid][w];
+    sm.base[tid] = s;
+  }
+  __syncthreads();
+
+  PosScan r;
+  r.p = static_cast<int64_t>(blockIdx.x) * kBridgeChunk + tid;
+  r.t = r.p < n ? types[r.p] : kTypeText;
+  const unsigned lt = (1u << lane) - 1u;
+  const unsigned b_img = __ballot_sync(0xffffffffu, r.t == kTypeImage);
+  const unsigned b_st = __ballot_sync(0xffffffffu, r.t == kTypeStart);
+  const unsigned b_en = __ballot_sync(0xffffffffu, r.t == kTypeEnd);
+  if (lane == 0) {  // sm.part was last read before the barrier above
+    sm.part[0][warp] = __popc(b_img);
+    sm.part[1][warp] = __popc(b_st);
+    sm.part[2][warp] = __popc(b_en);
+  }
+  __syncthreads();
+  int64_t before[3] = {sm.base[0], sm.base[1], sm.base[2]};
+  for (int k = 0; k < 3; ++k) r.total[k] = sm.base[k];
+  for (int w = 0; w < kWarps; ++w)
+    for (int k = 0; k < 3; ++k) {
+      if (w < warp) before[k] += sm.part[k][w];
+      r.total[k] += sm.part[k][w];
+    }
+  __syncthreads();  // sm.part is free again when this returns
+  r.k_img = before[0] + __popc(b_img & lt);
+  r.starts_incl = before[1] + __popc(b_st & (lt | (1u << lane)));
+  r.ends_excl = before[2] + __popc(b_en & lt);
+  const bool in_span = r.starts_incl - r.ends_excl == 1;
+  r.bad = r.t < kTypeText || r.t > kTypePad;
+  if (r.p < n) {
+    if (r.p % seq == 0 && r.starts_incl - (r.t == kTypeStart) != r.ends_excl) r.bad = true;
+    if (r.t == kTypeText ? in_span : !in_span) r.bad = true;
+  }
+  return r;
+}
+
+// grid (chunks, slices).  Every CTA of a chunk scans it; the one of slice 0 reports layout
+// errors.  Each CTA then copies columns [s * vs, (s + 1) * vs) (16-byte vectors, vs = row_vec /
+// slices) of the chunk's pseudo rows: aligner token rows for features, sentinel rows for the
+// other pseudo types.
 __global__ void __launch_bounds__(kBridgeChunk)
     k_bridge_merge(const int32_t* __restrict__ types, int64_t n, int64_t seq, const int4* __restrict__ counts,
                    const int32_t* __restrict__ grid, int n_images, int r, int64_t n_tokens,
-                   const uint4* __restrict__ image_tokens, const uint4* __restrict__ sentinels, uint4* embeds,
-                   int row_vec, uint32_t* err) {
-  constexpr int kWarps = kBridgeChunk / 32;
+                   const uint4* __restrict__ image_tokens, const uint4* __restrict__ sentinels,
+                   uint4* __restrict__ embeds, int row_vec, uint32_t* err) {
   extern __shared__ int32_t tok_cu[];  // [n_images + 1] aligner-token offsets of the images
-  __shared__ int part[3][kWarps];      // per-warp partial sums / counts
-  __shared__ int64_t base[3];          // features, starts, ends before this chunk
-  __shared__ int64_t src[kBridgeChunk];
+  __shared__ ScanSmem sm;
+  __shared__ int warp_copies[kWarps];
+  __shared__ int n_list;
+  __shared__ int list_pos[kBridgeChunk];      // chunk offsets of the pseudo rows
+  __shared__ int64_t list_src[kBridgeChunk];  // >= 0: aligner token; <= -2: sentinel row -s - 2
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   grid_dependency_wait();
   launch_dependents();
@@ -66,154 +160,132 @@ __global__ void __launch_bounds__(kBridgeChunk)
       carry += __shfl_sync(0xffffffffu, v, 31);
     }
   }
+  const PosScan ps = chunk_scan(types, n, seq, counts, sm);  // its barriers publish tok_cu
 
-  // prefix over the previous chunks
-  int64_t acc[3] = {0, 0, 0};
-  for (int c = tid; c < static_cast<int>(blockIdx.x); c += kBridgeChunk) {
-    const int4 v = counts[c];
-    acc[0] += v.x;
-    acc[1] += v.y;
-    acc[2] += v.z;
-  }
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
-  }
-  if (lane == 0)
-    for (int k = 0; k < 3; ++k) part[k][warp] = static_cast<int>(acc[k]);  // < 2^31 positions
-  __syncthreads();
-  if (tid < 3) {
-    int64_t s = 0;
-    for (int w = 0; w < kWarps; ++w) s += part[tid][w];
-    base[tid] = s;
-  }
-  __syncthreads();
-
-  // in-chunk scan
-  const int64_t p = static_cast<int64_t>(blockIdx.x) * kBridgeChunk + tid;
-  const int t = p < n ? types[p] : kTypeText;
-  const unsigned lt = (1u << lane) - 1u;
-  const unsigned b_img = __ballot_sync(0xffffffffu, t == kTypeImage);
-  const unsigned b_st = __ballot_sync(0xffffffffu, t == kTypeStart);
-  const unsigned b_en = __ballot_sync(0xffffffffu, t == kTypeEnd);
-  if (lane == 0) {
-    part[0][warp] = __popc(b_img);
-    part[1][warp] = __popc(b_st);
-    part[2][warp] = __popc(b_en);
-  }
-  __syncthreads();
-  int64_t before[3] = {base[0], base[1], base[2]};
-  int64_t chunk_tot[3] = {0, 0, 0};
-  for (int w = 0; w < kWarps; ++w)
-    for (int k = 0; k < 3; ++k) {
-      if (w < warp) before[k] += part[k][w];
-      chunk_tot[k] += part[k][w];
-    }
-  const int64_t k_img = before[0] + __popc(b_img & lt);              // features before p
-  const int64_t starts_incl = before[1] + __popc(b_st & (lt | (1u << lane)));  // starts at or before p
-  const int64_t ends_excl = before[2] + __popc(b_en & lt);           // ends before p
-
-  bool bad = t < kTypeText || t > kTypePad;
-  // a sequence starts with every span closed
-  if (p < n && p % seq == 0 && starts_incl - (t == kTypeStart) != ends_excl) bad = true;
-  // a span holds pseudo tokens only
-  if (p < n && t == kTypeText && starts_incl - ends_excl == 1) bad = true;
-  int64_t s = -1;  // -1: keep the row; >= 0: aligner token; <= -2: sentinel row -s - 2
-  if (!bad && t != kTypeText && p < n) {
-    if (starts_incl - ends_excl != 1) {
-      bad = true;  // outside a span, or a start inside an open one
-    } else if (t == kTypeImage) {
-      const int64_t j = starts_incl - 1;
-      if (j >= n_images || k_img < tok_cu[j] || k_img >= tok_cu[j + 1]) bad = true;
-      else s = k_img;
+  bool bad = ps.bad;
+  int64_t s = -1;  // -1: keep the row
+  if (!bad && ps.t != kTypeText && ps.p < n) {
+    if (ps.t == kTypeImage) {
+      const int64_t j = ps.starts_incl - 1;
+      if (j >= n_images || ps.k_img < tok_cu[j] || ps.k_img >= tok_cu[j + 1]) bad = true;
+      else s = ps.k_img;
     } else {
-      s = -static_cast<int64_t>(t) - 1;  // type 1..4 -> sentinel row 0..3
+      s = -static_cast<int64_t>(ps.t) - 1;  // type 1..4 -> sentinel row 0..3
     }
   }
-  if (bad) record(err);
-  src[tid] = bad ? -1 : s;
-  if (blockIdx.x == gridDim.x - 1 && tid == 0) {
-    const int64_t f = base[0] + chunk_tot[0], st = base[1] + chunk_tot[1], en = base[2] + chunk_tot[2];
-    if (f != n_tokens || st != n_images || st != en) record(err);
+  if (blockIdx.y == 0) {
+    if (bad) record(err);
+    if (blockIdx.x == gridDim.x - 1 && tid == 0 &&
+        (ps.total[0] != n_tokens || ps.total[1] != n_images || ps.total[1] != ps.total[2]))
+      record(err);
   }
+  // compact this chunk's rows to copy, in position order
+  const bool copy = !bad && s != -1;
+  const unsigned b_copy = __ballot_sync(0xffffffffu, copy);
+  if (lane == 0) warp_copies[warp] = __popc(b_copy);
+  __syncthreads();
+  int slot = __popc(b_copy & ((1u << lane) - 1u));
+  for (int w = 0; w < warp; ++w) slot += warp_copies[w];
+  if (copy) {
+    list_pos[slot] = tid;
+    list_src[slot] = s;
+  }
+  if (tid == kBridgeChunk - 1) n_list = slot + (copy ? 1 : 0);
   __syncthreads();
 
-  for (int i = warp; i < kBridgeChunk; i += kWarps) {
-    const int64_t si = src[i];
-    if (si == -1) continue;
-    const uint4* from = si >= 0 ? image_tokens + si * row_vec : sentinels + (-si - 2) * row_vec;
-    uint4* to = embeds + (static_cast<int64_t>(blockIdx.x) * kBridgeChunk + i) * row_vec;
-    int v = lane;
-    for (; v + 96 < row_vec; v += 128) {
-      const uint4 a0 = __ldg(from + v), a1 = __ldg(from + v + 32), a2 = __ldg(from + v + 64),
-                  a3 = __ldg(from + v + 96);
-      to[v] = a0;
-      to[v + 32] = a1;
-      to[v + 64] = a2;
-      to[v + 96] = a3;
+  const int vs = row_vec / static_cast<int>(gridDim.y);
+  const int col0 = static_cast<int>(blockIdx.y) * vs;
+  const int64_t items = static_cast<int64_t>(n_list) * vs;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kBridgeChunk;
+  constexpr int kUnroll = 4;
+  for (int64_t it0 = tid; it0 < items; it0 += kBridgeChunk * kUnroll) {
+    uint4 v[kUnroll];
+    uint4* dst[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t it = it0 + u * kBridgeChunk;
+      dst[u] = nullptr;
+      if (it < items) {
+        const int j = static_cast<int>(it / vs);
+        const int c = col0 + static_cast<int>(it - static_cast<int64_t>(j) * vs);
+        const int64_t si = list_src[j];
+        const uint4* from = si >= 0 ? image_tokens + si * row_vec : sentinels + (-si - 2) * row_vec;
+        v[u] = __ldg(from + c);
+        dst[u] = embeds + (row0 + list_pos[j]) * row_vec + c;
+      }
     }
-    for (; v < row_vec; v += 32) to[v] = __ldg(from + v);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (dst[u]) *dst[u] = v[u];
   }
 }
 
-// Nearest image_start / image_end at or before `from` (dir = -1) or at or after it (dir = +1)
-// inside [lo, hi); returns its type, or kTypeText if there is none.  *text_between tells
-// whether a text position lies between `from` and that marker (or the range's end).
-__device__ __forceinline__ int nearest_marker(const int32_t* __restrict__ types, int64_t from, int dir, int64_t lo,
-                                              int64_t hi, int64_t* at, bool* text_between) {
-  const int lane = threadIdx.x & 31;
-  bool text = false;
-  for (int64_t q0 = from; q0 >= lo && q0 < hi; q0 += 32 * dir) {
-    const int64_t q = q0 + dir * lane;
-    const bool in = q >= lo && q < hi;
-    const int t = in ? types[q] : kTypeText;
-    const unsigned m = __ballot_sync(0xffffffffu, in && (t == kTypeStart || t == kTypeEnd));
-    const unsigned tx = __ballot_sync(0xffffffffu, in && t == kTypeText);
-    if (m) {
-      const int first = __ffs(m) - 1;  // the lowest lane is the nearest position
-      *at = q0 + dir * first;
-      *text_between = text || (tx & ((1u << first) - 1u)) != 0;
-      return __shfl_sync(0xffffffffu, t, first);
-    }
-    text = text || tx != 0;
-  }
-  *text_between = text;
-  return kTypeText;
+// Visibility, step 2: per chunk, the scan; each valid image_start / image_end stores its
+// position in the span tables (index = span number), and every position its span number (-1
+// for text or a bad position).
+__global__ void __launch_bounds__(kBridgeChunk)
+    k_span_scan(const int32_t* __restrict__ types, int64_t n, int64_t seq, const int4* __restrict__ counts,
+                int32_t* __restrict__ span_first, int32_t* __restrict__ span_last, int32_t* __restrict__ span_of,
+                uint32_t* err) {
+  __shared__ ScanSmem sm;
+  grid_dependency_wait();
+  launch_dependents();
+  const PosScan ps = chunk_scan(types, n, seq, counts, sm);
+  if (ps.bad) record(err);
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0 && ps.total[1] != ps.total[2]) record(err);
+  if (ps.p >= n) return;
+  const bool pseudo = !ps.bad && ps.t != kTypeText;
+  const int32_t j = static_cast<int32_t>(ps.starts_incl - 1);
+  span_of[ps.p] = pseudo ? j : -1;
+  if (pseudo && ps.t == kTypeStart) span_first[j] = static_cast<int32_t>(ps.p);
+  if (pseudo && ps.t == kTypeEnd) span_last[j] = static_cast<int32_t>(ps.p);
 }
 
-// One warp per mask row (b, i).  A pseudo token's span is bounded by the nearest image_start at
-// or before it (strictly before an image_end) and the nearest image_end at or after it
-// (strictly after an image_start); anything else is a layout error and the row is left as is.
-// The image_start row also checks that no text lies inside its span.
-template <typename E>
-__global__ void __launch_bounds__(256) k_image_visibility(const int32_t* __restrict__ types, int64_t rows, int64_t seq,
-                                                          E* mask, uint32_t* err) {
+// Visibility, step 3: one warp per mask row (b, i) of a pseudo token: zero the columns of its
+// span, when both ends of the span were found inside the row's own sequence.
+__global__ void __launch_bounds__(256)
+    k_visibility_fill(const int32_t* __restrict__ span_of, const int32_t* __restrict__ span_first,
+                      const int32_t* __restrict__ span_last, int64_t rows, int64_t seq, char* mask, int elem,
+                      uint32_t* err) {
   grid_dependency_wait();
   launch_dependents();
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  const int t = types[row];
-  if (t == kTypeText) return;
-  if (t < kTypeText || t > kTypePad) {
+  const int32_t j = span_of[row];
+  if (j < 0) return;
+  const int64_t a = span_first[j], e = span_last[j], lo = row - row % seq;
+  if (a < lo || e >= lo + seq || a > row || e < row) {  // the span is not closed in this sequence
     if (lane == 0) record(err);
     return;
   }
-  const int64_t lo = row - row % seq, hi = lo + seq;
-  int64_t a = -1, e = -1;
-  bool text_back, text_fwd;
-  const int back = nearest_marker(types, t == kTypeEnd ? row - 1 : row, -1, lo, hi, &a, &text_back);
-  const int fwd = nearest_marker(types, t == kTypeStart ? row + 1 : row, +1, lo, hi, &e, &text_fwd);
-  if (back != kTypeStart || fwd != kTypeEnd || (t == kTypeStart && text_fwd)) {
-    if (lane == 0) record(err);
-    return;
+  char* beg = mask + (row * seq + (a - lo)) * elem;
+  char* end = mask + (row * seq + (e - lo) + 1) * elem;
+  char* body = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(beg) + 15) & ~uintptr_t(15));
+  if (body > end) body = end;
+  char* tail = reinterpret_cast<char*>(reinterpret_cast<uintptr_t>(end) & ~uintptr_t(15));
+  if (tail < body) tail = body;
+  const int64_t head_n = (body - beg) / elem, tail_n = (end - tail) / elem;
+  if (elem == 4) {
+    for (int64_t k = lane; k < head_n; k += 32) reinterpret_cast<uint32_t*>(beg)[k] = 0u;
+    for (int64_t k = lane; k < tail_n; k += 32) reinterpret_cast<uint32_t*>(tail)[k] = 0u;
+  } else {
+    for (int64_t k = lane; k < head_n; k += 32) reinterpret_cast<uint16_t*>(beg)[k] = 0;
+    for (int64_t k = lane; k < tail_n; k += 32) reinterpret_cast<uint16_t*>(tail)[k] = 0;
   }
-  E* out = mask + row * seq;  // columns are positions inside the sequence
-  for (int64_t c = a - lo + lane; c <= e - lo; c += 32) out[c] = E(0);
+  const int64_t vecs = (tail - body) / 16;
+  for (int64_t k = lane; k < vecs; k += 32) reinterpret_cast<uint4*>(body)[k] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 }  // namespace
+
+// CTAs per chunk of the merge: as many column slices of at least 32 vectors (one per lane) as
+// divide the row, up to 16.
+int bridge_slices(int row_vec) {
+  int s = 1;
+  while (s < 16 && row_vec % (2 * s) == 0 && row_vec / (2 * s) >= 32) s *= 2;
+  return s;
+}
 
 cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, int4* counts, const int32_t* grid_dev,
                                 int n_images, int r, int64_t n_tokens, const void* image_tokens, const void* sentinels,
@@ -221,24 +293,31 @@ cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, in
   const int64_t chunks = (n + kBridgeChunk - 1) / kBridgeChunk;
   if (chunks == 0) return cudaSuccess;
   cudaError_t e = launch_pdl(k_bridge_count, dim3(static_cast<unsigned>(chunks)), dim3(kBridgeChunk), 0, s, types, n,
-                             counts, err);
+                             counts, static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr), err);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_bridge_merge, dim3(static_cast<unsigned>(chunks)), dim3(kBridgeChunk),
-                    (n_images + 1) * sizeof(int32_t), s, types, n, seq, static_cast<const int4*>(counts), grid_dev,
-                    n_images, r, n_tokens, static_cast<const uint4*>(image_tokens),
-                    static_cast<const uint4*>(sentinels), static_cast<uint4*>(embeds), row_vec, err);
+  const int slices = bridge_slices(row_vec);
+  return launch_pdl(k_bridge_merge, dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(slices)),
+                    dim3(kBridgeChunk), (n_images + 1) * sizeof(int32_t), s, types, n, seq,
+                    static_cast<const int4*>(counts), grid_dev, n_images, r, n_tokens,
+                    static_cast<const uint4*>(image_tokens), static_cast<const uint4*>(sentinels),
+                    static_cast<uint4*>(embeds), row_vec, err);
 }
 
 cudaError_t launch_image_visibility(const int32_t* types, int64_t batch, int64_t seq, void* mask, int elem_bytes,
+                                    int4* counts, int32_t* span_first, int32_t* span_last, int32_t* span_of,
                                     uint32_t* err, cudaStream_t s) {
-  const int64_t rows = batch * seq;
-  if (rows == 0) return cudaSuccess;
-  const dim3 grid(static_cast<unsigned>((rows * 32 + 255) / 256));
-  if (elem_bytes == 4)
-    return launch_pdl(k_image_visibility<uint32_t>, grid, dim3(256), 0, s, types, rows, seq,
-                      static_cast<uint32_t*>(mask), err);
-  return launch_pdl(k_image_visibility<uint16_t>, grid, dim3(256), 0, s, types, rows, seq,
-                    static_cast<uint16_t*>(mask), err);
+  const int64_t n = batch * seq;
+  const int64_t chunks = (n + kBridgeChunk - 1) / kBridgeChunk;
+  if (chunks == 0) return cudaSuccess;
+  cudaError_t e = launch_pdl(k_bridge_count, dim3(static_cast<unsigned>(chunks)), dim3(kBridgeChunk), 0, s, types, n,
+                             counts, span_first, span_last, err);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(k_span_scan, dim3(static_cast<unsigned>(chunks)), dim3(kBridgeChunk), 0, s, types, n, seq,
+                 static_cast<const int4*>(counts), span_first, span_last, span_of, err);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_visibility_fill, dim3(static_cast<unsigned>((n * 32 + 255) / 256)), dim3(256), 0, s,
+                    static_cast<const int32_t*>(span_of), static_cast<const int32_t*>(span_first),
+                    static_cast<const int32_t*>(span_last), n, seq, static_cast<char*>(mask), elem_bytes, err);
 }
 
 }  // namespace dsv4v

@@ -118,6 +118,7 @@ cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, in
                                 int n_images, int r, int64_t n_tokens, const void* image_tokens, const void* sentinels,
                                 void* embeds, int row_vec, uint32_t* err, cudaStream_t s);
 cudaError_t launch_image_visibility(const int32_t* types, int64_t batch, int64_t seq, void* mask, int elem_bytes,
+                                    int4* counts, int32_t* span_first, int32_t* span_last, int32_t* span_of,
                                     uint32_t* err, cudaStream_t s);
 // Norm operands of the first GEMM of a block: xw = bf16(x * w) and ss[p * parts] = sum_c x[p,c]^2
 // (the other parts of a row are zero-filled); also clears zero_n counters like the kernels above.

@@ -33,7 +33,7 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
            "dsv4v_status_string", "dsv4v_linear_residual_noalloc", "dsv4v_patch_embed",
            "dsv4v_patch_merger_workspace_size", "dsv4v_patch_merger_forward", "dsv4v_image_layout",
-           "dsv4v_merge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility")
+           "dsv4v_bridge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -91,9 +91,9 @@ def lib() -> ctypes.CDLL:
             "dsv4v_patch_merger_forward": (I, [cfg, bat, P, P, P, P, P, P, P, P, P, SZ, P]),
             "dsv4v_linear_residual_noalloc": (I, [cfg, I64, I, P, P, P, P]),
             "dsv4v_image_layout": (I, [I, I, I, P, I64, ctypes.POINTER(ctypes.c_int64)]),
-            "dsv4v_merge_workspace_size": (SZ, [I64]),
+            "dsv4v_bridge_workspace_size": (SZ, [I64]),
             "dsv4v_merge_image_embeddings": (I, [cfg, bat, I64, I64, P, P, P, P, P, SZ, P]),
-            "dsv4v_image_visibility": (I, [I64, I64, P, P, I, P]),
+            "dsv4v_image_visibility": (I, [I64, I64, P, P, I, P, SZ, P]),
             "dsv4v_device_error": (I, [P]),
             "dsv4v_selftest_bounded_wait": (I, [U64, P]),
             "dsv4v_status_string": (ctypes.c_char_p, [I]),
@@ -262,8 +262,8 @@ def dsv4v_image_layout(grid_h: int, grid_w: int, downsample_ratio: int):
     return out
 
 
-def dsv4v_merge_workspace_size(n_positions: int) -> int:
-    return int(lib().dsv4v_merge_workspace_size(n_positions))
+def dsv4v_bridge_workspace_size(n_positions: int) -> int:
+    return int(lib().dsv4v_bridge_workspace_size(n_positions))
 
 
 def dsv4v_merge_image_embeddings(cfg, batch, token_types, image_tokens, sentinels, embeds, workspace, stream=None):
@@ -277,13 +277,14 @@ def dsv4v_merge_image_embeddings(cfg, batch, token_types, image_tokens, sentinel
            "dsv4v_merge_image_embeddings")
 
 
-def dsv4v_image_visibility(token_types, mask, stream=None):
+def dsv4v_image_visibility(token_types, mask, workspace, stream=None):
     """mask [n_seqs, seq_len, seq_len] (or with a unit head axis), updated in place: every pair
     inside one image span of token_types [n_seqs, seq_len] becomes 0."""
     n_seqs, seq_len = int(token_types.shape[0]), int(token_types.shape[1])
     if mask.numel() != n_seqs * seq_len * seq_len:
         raise ValueError(f"mask has {mask.numel()} entries, expected {n_seqs} x {seq_len} x {seq_len}")
     _check(lib().dsv4v_image_visibility(n_seqs, seq_len, _ptr(token_types), _ptr(mask), mask.element_size(),
+                                        _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                         _stream(stream)),
            "dsv4v_image_visibility")
 
