@@ -294,7 +294,8 @@ def run_ours(args):
     # ---- the step before the tower: patch embedding of the same patches (14 x 14 RGB patches)
     extras = {"patch_embed": patch_embed_timing(A, torch, cfg, wl, stream, flush, args.steps),
               "patch_merger": patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, args.steps),
-              "bridge": bridge_timing(A, torch, cfg, stream, flush, args.steps)}
+              "bridge": bridge_timing(A, torch, cfg, stream, flush, args.steps),
+              "block_backward": block_backward_timing(A, torch, cfg, batch, wl, lw, stream, flush, args.steps)}
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     x_host = x0.cpu().pin_memory()
@@ -545,6 +546,48 @@ def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
                            "gbs": vis_bytes / (vis_ms * 1e-3) / 1e9, "launches_per_call": 3},
             "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if hbm else None,
             "note": "standalone, one call per timed interval after an L2 flush; not in value"}
+
+
+def block_backward_timing(A, torch, cfg, batch, wl, lw, stream, flush, steps):
+    """dsv4v_block_backward of the first block on the workload's patches (random input and output
+    gradient): CUDA events around one call after an L2 flush.  The call recomputes the block's
+    forward, then runs the backward; 'tflops' counts the backward's algorithmic work only (two
+    GEMMs per forward GEMM, 8 N^2 D for the attention), without the recompute.  Not part of the
+    tower step above."""
+    P, D, F, H = wl.n_patches, wl.vision_dim, wl.mlp_hidden, wl.n_heads
+    g = torch.Generator(device="cuda").manual_seed(10)
+    x = torch.randn(P, D, device="cuda", generator=g).to(torch.bfloat16)
+    do = torch.randn(P, D, device="cuda", generator=g).to(torch.bfloat16)
+    dx = torch.empty(P, D, dtype=torch.bfloat16, device="cuda")
+    gb = {"norm1_w": torch.empty(D, device="cuda"), "norm2_w": torch.empty(D, device="cuda"),
+          "wqkv": torch.empty(3 * D, D, dtype=torch.bfloat16, device="cuda"),
+          "wo": torch.empty(D, D, dtype=torch.bfloat16, device="cuda"),
+          "w_gate": torch.empty(F, D, dtype=torch.bfloat16, device="cuda"),
+          "w_up": torch.empty(F, D, dtype=torch.bfloat16, device="cuda"),
+          "w_down": torch.empty(D, F, dtype=torch.bfloat16, device="cuda")}
+    grads = A.block_grads(gb["norm1_w"], gb["norm2_w"], gb["wqkv"], gb["wo"], gb["w_gate"], gb["w_up"], gb["w_down"])
+    cos = torch.empty(P, D // H // 2, device="cuda")
+    sin = torch.empty_like(cos)
+    A.dsv4v_rope2d_table(cfg, batch, cos, sin, stream=stream.cuda_stream)
+    ws = torch.empty(A.dsv4v_backward_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
+    times = []
+    for i in range(steps + 3):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            A.dsv4v_block_backward(cfg, batch, lw[0], cos, sin, x, do, dx, grads, ws, stream=stream.cuda_stream)
+            ev1.record(stream)
+        stream.synchronize()
+        if i >= 3:
+            times.append(ev0.elapsed_time(ev1))
+    if A.dsv4v_device_error(stream.cuda_stream) != 0:
+        raise RuntimeError("device-side check failed in the block backward")
+    ms = sum(times) / len(times)
+    flops = 2.0 * P * (8 * D * D + 6 * D * F) + sum(8.0 * (h * w) ** 2 * D for h, w in wl.grids)
+    return {"avg_us": ms * 1e3, "tflops": flops / (ms * 1e-3) / 1e12, "patches": P,
+            "note": "standalone, one call per timed interval after an L2 flush; recompute + backward of one "
+                    "block; attention backward on CUDA cores; not in value"}
 
 
 def load_peaks():

@@ -278,6 +278,80 @@ dsv4v_status dsv4v_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 const char* dsv4v_status_string(dsv4v_status s);
 
+/* ---------------------------------------------------------------- backward
+ * The gradient of the tower ([PR], Validation: the pages train the tower and test "ragged grids
+ * and backward"; no backward is printed, so each call is the chain rule through the forward
+ * above).  bf16 configs only (DSV4V_ERR_UNSUPPORTED otherwise): activations and gradients are
+ * bf16, norm weights and their gradients fp32, GEMMs accumulate in fp32.  Every call takes the
+ * scratch of dsv4v_backward_workspace_size and writes its outputs (gradients are not
+ * accumulated into the destination). */
+
+/* Weight gradients of one block, laid out like dsv4v_block_weights: norm1_w, norm2_w fp32 [D];
+ * wqkv [3D, D], wo [D, D], w_gate [F, D], w_up [F, D], w_down [D, F] bf16.  Device pointers,
+ * 16-byte aligned, written. */
+typedef struct {
+  float* norm1_w;
+  float* norm2_w;
+  void* wqkv;
+  void* wo;
+  void* w_gate;
+  void* w_up;
+  void* w_down;
+} dsv4v_block_grads;
+
+/* Bytes of device scratch every backward call below needs for this config and batch; 0 if the
+ * arguments are invalid or the config is not bf16. */
+size_t dsv4v_backward_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch);
+
+/* Gradient of the attention ([vision-API, DeepseekV4VisionAttention]; see dsv4v_attention):
+ * per image and head, dv = P^T do, dS = P * (do v^T - rowsum(do * o)), dq = dS k / sqrt(hd),
+ * dk = dS^T q / sqrt(hd), with P the softmax of the forward.
+ *   qkv: device [P, 3D], the forward's input (q and k already rotated); out: device [P, D], the
+ *   forward's output; d_out: device [P, D]; dqkv: device [P, 3D], written: the gradients with
+ *   respect to the rotated q, k and to v. */
+dsv4v_status dsv4v_attention_backward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                      const void* qkv, const void* out, const void* d_out,
+                                      void* dqkv, void* workspace, size_t ws_bytes, void* stream);
+
+/* Gradient of RMSNorm ([vision-API, DeepseekV4VisionRMSNorm], y = w * x * r,
+ * r = 1 / sqrt(mean(x^2) + eps)): dx = r (dy * w) - x r^3 ((dy * w) . x) / D, plus d_in if
+ * non-NULL (a residual gradient to add); dw = sum over rows of dy * x * r.
+ *   x, dy, d_in, dx: device [P, D] (P = the batch's patches); dx may equal d_in.
+ *   w: device fp32 [D]; dw: device fp32 [D], written. */
+dsv4v_status dsv4v_rmsnorm_backward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                    const void* x, const float* w, const void* dy,
+                                    const void* d_in, void* dx, float* dw, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
+/* Gradient of one block ([vision-API, DeepseekV4VisionBlock.forward], see
+ * dsv4v_block_forward) with respect to its input and its weights, for the output gradient
+ * d_out.  The block's intermediates are recomputed from x; then the MLP branch, norm2, the
+ * output projection, attention, the inverse rotation, the fused projection and norm1 are
+ * differentiated in turn, with the residual gradients added.
+ *   x: device [P, D], the block's input; d_out: device [P, D]; dx: device [P, D], written
+ *   (must not overlap x or d_out); cos, sin: the rotation table of dsv4v_rope2d_table;
+ *   grads: host struct of device outputs. */
+dsv4v_status dsv4v_block_backward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                  const dsv4v_block_weights* weights, const float* cos,
+                                  const float* sin, const void* x, const void* d_out, void* dx,
+                                  const dsv4v_block_grads* grads, void* workspace,
+                                  size_t ws_bytes, void* stream);
+
+/* Gradient of the tower ([vision-API, DeepseekV4VisionTransformer.forward], see
+ * dsv4v_tower_forward): the final norm's backward (if final_norm_w is non-NULL), then every
+ * block's backward from the last to the first.  The caller keeps the forward's activations:
+ *   layer_inputs: host array of cfg->n_layers device pointers, the input [P, D] of each block;
+ *   x_last: device [P, D], the last block's output (the final norm's input; unused without a
+ *   final norm); d_out: device [P, D], the gradient of the tower's output; dx: device [P, D],
+ *   written; layer_grads: host array of cfg->n_layers gradient structs; d_final_norm_w: device
+ *   fp32 [D], written (unused without a final norm). */
+dsv4v_status dsv4v_tower_backward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                  const dsv4v_block_weights* layers, const float* final_norm_w,
+                                  const void* const* layer_inputs, const void* x_last,
+                                  const void* d_out, void* dx,
+                                  const dsv4v_block_grads* layer_grads, float* d_final_norm_w,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- image-token bridge
  * [model-API, DeepseekV4Model]: the sentinel parameters image_start, image_end, image_newline
  * and image_pad; merge_image_embeddings; apply_deepseek_v4_image_visibility.

@@ -158,3 +158,19 @@ def test_bridge_host_validation_rejects(lib):
     assert vis(1, 8, None, al, 4, al, ws, None) == 1
     assert vis(1, 8, al, al, 4, al + 16, ws, None) == 3  # workspace not 256-byte aligned
     assert vis(1, 8, al, al, 4, al, 100, None) == 3  # workspace too small
+
+
+def test_backward_host_checks(lib):
+    # sizing is host-only; fp32 configs are rejected before any CUDA call
+    b = HostBatch([(28, 28)])
+    assert lib.dsv4v_backward_workspace_size(ctypes.byref(cfg()), ctypes.byref(b.c)) > 0
+    f32 = cfg(dtype=A.DSV4V_F32, vision_dim=64, n_heads=4, mlp_hidden=128, llm_dim=128)
+    assert lib.dsv4v_backward_workspace_size(ctypes.byref(f32), ctypes.byref(b.c)) == 0
+    assert lib.dsv4v_attention_backward(ctypes.byref(f32), ctypes.byref(b.c), None, None, None, None, None, 0,
+                                        None) == 2
+    assert lib.dsv4v_block_backward(ctypes.byref(f32), ctypes.byref(b.c), None, None, None, None, None, None, None,
+                                    None, 0, None) == 2
+    # the scratch grows with the patches: every activation, gradient and transpose is kept
+    small = lib.dsv4v_backward_workspace_size(ctypes.byref(cfg()), ctypes.byref(HostBatch([(3, 5)]).c))
+    big = lib.dsv4v_backward_workspace_size(ctypes.byref(cfg()), ctypes.byref(b.c))
+    assert 0 < small < big

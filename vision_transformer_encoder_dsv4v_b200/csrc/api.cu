@@ -958,4 +958,285 @@ dsv4v_status dsv4v_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
   return cuda_status(launch_selftest_wait(limit_ns, d.err, static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------------------- backward
+namespace {
+
+constexpr int kNormParts = 512;  // most CTAs of one RMSNorm backward (each leaves a [D] partial)
+
+// Scratch of the backward calls, after the forward layout (whose split-tile scratch and
+// rotation tables the recompute reuses).  Activations and gradients are bf16 [P, width];
+// transposed operands of the weight-gradient GEMMs are bf16 [width, ldp] (ldp = P rounded up to
+// a multiple of 8, 16-byte TMA rows); transposed weights; fp32 attention row statistics and
+// RMSNorm partials.
+struct BwdLayout {
+  int64_t ldp;
+  size_t y1, qkv, att, x2, y2, g, u, h, dh, dgu, dy2, dx2, datt, dqkv, dy1, dcur0, dcur1;
+  size_t dout_t, h_t, dgu_t, y2_t, dx2_t, att_t, dqkv_t, y1_t;
+  size_t wd_t, wgu_t, wo_t, wqkv_t, lse, rowdot, norm_parts, total;
+};
+
+BwdLayout bwd_layout(const Shape& s, size_t fwd_total) {
+  BwdLayout l{};
+  const size_t P = static_cast<size_t>(s.P), D = s.D, F = s.F;
+  l.ldp = (s.P + 7) / 8 * 8;
+  if (l.ldp < 8) l.ldp = 8;
+  const size_t ldp = static_cast<size_t>(l.ldp);
+  size_t off = up256(fwd_total);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += up256(bytes);
+    return at;
+  };
+  l.y1 = take(P * D * 2);
+  l.qkv = take(P * 3 * D * 2);
+  l.att = take(P * D * 2);
+  l.x2 = take(P * D * 2);
+  l.y2 = take(P * D * 2);
+  l.g = take(P * F * 2);
+  l.u = take(P * F * 2);
+  l.h = take(P * F * 2);
+  l.dh = take(P * F * 2);
+  l.dgu = take(P * 2 * F * 2);
+  l.dy2 = take(P * D * 2);
+  l.dx2 = take(P * D * 2);
+  l.datt = take(P * D * 2);
+  l.dqkv = take(P * 3 * D * 2);
+  l.dy1 = take(P * D * 2);
+  l.dcur0 = take(P * D * 2);
+  l.dcur1 = take(P * D * 2);
+  l.dout_t = take(D * ldp * 2);
+  l.h_t = take(F * ldp * 2);
+  l.dgu_t = take(2 * F * ldp * 2);
+  l.y2_t = take(D * ldp * 2);
+  l.dx2_t = take(D * ldp * 2);
+  l.att_t = take(D * ldp * 2);
+  l.dqkv_t = take(3 * D * ldp * 2);
+  l.y1_t = take(D * ldp * 2);
+  l.wd_t = take(F * D * 2);
+  l.wgu_t = take(D * 2 * F * 2);
+  l.wo_t = take(D * D * 2);
+  l.wqkv_t = take(D * 3 * D * 2);
+  l.lse = take(P * s.H * 4);
+  l.rowdot = take(P * s.H * 4);
+  l.norm_parts = take(static_cast<size_t>(kNormParts) * D * 4);
+  l.total = off;
+  return l;
+}
+
+// The backward calls are bf16 only and need a grid that the transposes can cover.
+dsv4v_status bwd_prepare(const dsv4v_config* cfg, const dsv4v_batch* batch, void* workspace, size_t ws_bytes,
+                         void* stream, Ctx& c, BwdLayout& bl) {
+  DSV4V_TRY(check_all(cfg, batch, c.s));
+  if (!c.s.bf16) return DSV4V_ERR_UNSUPPORTED;
+  if ((c.s.P + 31) / 32 > 65535) return DSV4V_ERR_UNSUPPORTED;
+  DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
+  bl = bwd_layout(c.s, c.lay.total);
+  if (ws_bytes < bl.total) return DSV4V_ERR_WORKSPACE;
+  return DSV4V_OK;
+}
+
+int norm_parts_for(const Ctx& c, int64_t rows) {
+  const int64_t want = std::min<int64_t>((rows + 7) / 8, 2 * static_cast<int64_t>(c.dev.sms));
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, kNormParts)));
+}
+
+// out[M, n_out] = a[M, K] . b[n_out, K]^T with row strides lda / ldb (0 = K): whole tiles only,
+// so no split-tile scratch is used.
+dsv4v_status gemm_store(const Ctx& c, const void* a, int64_t M, int K, int64_t lda, const void* b, int64_t ldb,
+                        int n_out, void* out) {
+  const GemmPlan plan = plan_gemm(EPI_STORE, static_cast<int>(M), n_out, K, c.dev.sms, 0);
+  if (plan.bn == 0) return DSV4V_ERR_UNSUPPORTED;
+  GemmExtra ex;
+  ex.lda = lda;
+  ex.ldb = ldb;
+  return gemm_bf16(c, EPI_STORE, plan, a, M, K, b, nullptr, n_out, out, nullptr, nullptr, nullptr, NormFold(), ex);
+}
+
+dsv4v_status transpose(const Ctx& c, const void* in, int64_t rows, int cols, void* out, int64_t ld_out,
+                       int64_t col0 = 0) {
+  return cuda_status(launch_transpose_bf16(in, rows, cols, cols, out, ld_out, col0, c.stream));
+}
+
+int attention_blocks(const dsv4v_batch* b) {
+  int64_t n = 0;
+  for (int i = 0; i < b->n_images; ++i) n += (b->cu_patches_host[i + 1] - b->cu_patches_host[i] + 63) / 64;
+  return static_cast<int>(n);
+}
+
+dsv4v_status attention_bwd(const Ctx& c, const BwdLayout& bl, const dsv4v_batch* b, const void* qkv, const void* out,
+                           const void* dout, void* dqkv) {
+  return cuda_status(launch_attention_bwd(qkv, out, dout, dqkv, c.at<float>(bl.lse), c.at<float>(bl.rowdot),
+                                          b->cu_patches_dev, b->n_images, attention_blocks(b), c.s.D, c.s.H,
+                                          c.stream));
+}
+
+dsv4v_status rmsnorm_bwd(const Ctx& c, const BwdLayout& bl, const void* x, const float* w, const void* dy,
+                         const void* d_in, void* dx, float* dw) {
+  return cuda_status(launch_rmsnorm_bwd(x, w, dy, d_in, dx, c.at<float>(bl.norm_parts), norm_parts_for(c, c.s.P), dw,
+                                        c.s.P, c.s.D, c.eps, c.stream));
+}
+
+bool grads_ok(const dsv4v_block_grads* g) {
+  if (!g) return false;
+  const void* ptrs[] = {g->norm1_w, g->wqkv, g->wo, g->norm2_w, g->w_gate, g->w_up, g->w_down};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return false;
+  return true;
+}
+
+// One block backward (see dsv4v_block_backward): recompute, then the MLP branch, norm2, the
+// output projection, attention, the rotation and projection, norm1.
+dsv4v_status block_backward_bf16(const Ctx& c, const BwdLayout& bl, const dsv4v_batch* batch,
+                                 const dsv4v_block_weights* w, const float* cos, const float* sin, const void* x,
+                                 const void* dout, void* dx, const dsv4v_block_grads* gr) {
+  const Shape& s = c.s;
+  const int64_t P = s.P, ldp = bl.ldp;
+  const int D = s.D, F = s.F;
+  void* y1 = c.at<void>(bl.y1);
+  void* qkv = c.at<void>(bl.qkv);
+  void* att = c.at<void>(bl.att);
+  void* x2 = c.at<void>(bl.x2);
+  void* y2 = c.at<void>(bl.y2);
+  void* g = c.at<void>(bl.g);
+  void* u = c.at<void>(bl.u);
+  void* h = c.at<void>(bl.h);
+  void* dh = c.at<void>(bl.dh);
+  uint8_t* dgu = c.at<uint8_t>(bl.dgu);
+  void* dy2 = c.at<void>(bl.dy2);
+  void* dx2 = c.at<void>(bl.dx2);
+  void* datt = c.at<void>(bl.datt);
+  void* dqkv = c.at<void>(bl.dqkv);
+  void* dy1 = c.at<void>(bl.dy1);
+  uint8_t* dgu_t = c.at<uint8_t>(bl.dgu_t);
+  // transposed weights: the input-gradient GEMMs read W^T rows
+  DSV4V_TRY(transpose(c, w->w_down, D, F, c.at<void>(bl.wd_t), D));
+  DSV4V_TRY(transpose(c, w->w_gate, F, D, c.at<void>(bl.wgu_t), 2 * F, 0));
+  DSV4V_TRY(transpose(c, w->w_up, F, D, c.at<void>(bl.wgu_t), 2 * F, F));
+  DSV4V_TRY(transpose(c, w->wo, D, D, c.at<void>(bl.wo_t), D));
+  DSV4V_TRY(transpose(c, w->wqkv, 3 * D, D, c.at<void>(bl.wqkv_t), 3 * D));
+  // recompute the block's intermediates
+  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm1_w, y1, P, D, c.eps, c.stream)));
+  DSV4V_TRY(reset_counters(c));
+  DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, y1, P, D, w->wqkv, nullptr, 3 * D, qkv, nullptr, cos, sin));
+  DSV4V_TRY(attention_bf16(c, batch, qkv, att));
+  DSV4V_TRY(cuda_status(cudaMemcpyAsync(x2, x, static_cast<size_t>(P) * D * 2, cudaMemcpyDeviceToDevice, c.stream)));
+  DSV4V_TRY(reset_counters(c));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, att, P, D, w->wo, nullptr, D, x2, x2));
+  DSV4V_TRY(cuda_status(launch_rmsnorm(true, x2, w->norm2_w, y2, P, D, c.eps, c.stream)));
+  DSV4V_TRY(gemm_store(c, y2, P, D, 0, w->w_gate, 0, F, g));
+  DSV4V_TRY(gemm_store(c, y2, P, D, 0, w->w_up, 0, F, u));
+  // MLP branch
+  DSV4V_TRY(gemm_store(c, dout, P, D, 0, c.at<void>(bl.wd_t), 0, F, dh));
+  DSV4V_TRY(cuda_status(launch_swiglu_bwd(g, u, dh, dgu, h, P, F, c.dev.sms, c.stream)));
+  DSV4V_TRY(transpose(c, dout, P, D, c.at<void>(bl.dout_t), ldp));
+  DSV4V_TRY(transpose(c, h, P, F, c.at<void>(bl.h_t), ldp));
+  DSV4V_TRY(gemm_store(c, c.at<void>(bl.dout_t), D, static_cast<int>(P), ldp, c.at<void>(bl.h_t), ldp, F, gr->w_down));
+  DSV4V_TRY(gemm_store(c, dgu, P, 2 * F, 0, c.at<void>(bl.wgu_t), 0, D, dy2));
+  DSV4V_TRY(transpose(c, dgu, P, 2 * F, dgu_t, ldp));
+  DSV4V_TRY(transpose(c, y2, P, D, c.at<void>(bl.y2_t), ldp));
+  DSV4V_TRY(gemm_store(c, dgu_t, F, static_cast<int>(P), ldp, c.at<void>(bl.y2_t), ldp, D, gr->w_gate));
+  DSV4V_TRY(gemm_store(c, dgu_t + static_cast<size_t>(F) * ldp * 2, F, static_cast<int>(P), ldp,
+                       c.at<void>(bl.y2_t), ldp, D, gr->w_up));
+  // norm2 and the residual
+  DSV4V_TRY(rmsnorm_bwd(c, bl, x2, w->norm2_w, dy2, dout, dx2, gr->norm2_w));
+  // output projection
+  DSV4V_TRY(gemm_store(c, dx2, P, D, 0, c.at<void>(bl.wo_t), 0, D, datt));
+  DSV4V_TRY(transpose(c, dx2, P, D, c.at<void>(bl.dx2_t), ldp));
+  DSV4V_TRY(transpose(c, att, P, D, c.at<void>(bl.att_t), ldp));
+  DSV4V_TRY(gemm_store(c, c.at<void>(bl.dx2_t), D, static_cast<int>(P), ldp, c.at<void>(bl.att_t), ldp, D, gr->wo));
+  // attention, rotation, fused projection
+  DSV4V_TRY(attention_bwd(c, bl, batch, qkv, att, datt, dqkv));
+  DSV4V_TRY(cuda_status(launch_rotary_bwd(dqkv, cos, sin, P, D, s.hd, c.dev.sms, c.stream)));
+  DSV4V_TRY(gemm_store(c, dqkv, P, 3 * D, 0, c.at<void>(bl.wqkv_t), 0, D, dy1));
+  DSV4V_TRY(transpose(c, dqkv, P, 3 * D, c.at<void>(bl.dqkv_t), ldp));
+  DSV4V_TRY(transpose(c, y1, P, D, c.at<void>(bl.y1_t), ldp));
+  DSV4V_TRY(gemm_store(c, c.at<void>(bl.dqkv_t), 3 * D, static_cast<int>(P), ldp, c.at<void>(bl.y1_t), ldp, D,
+                       gr->wqkv));
+  // norm1 and the residual
+  return rmsnorm_bwd(c, bl, x, w->norm1_w, dy1, dx2, dx, gr->norm1_w);
+}
+
+}  // namespace
+
+size_t dsv4v_backward_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch) {
+  Shape s;
+  if (check_all(cfg, batch, s) != DSV4V_OK || !s.bf16) return 0;
+  DeviceInfo d;
+  const int sms = device_info(d) ? d.sms : planning_sms();
+  return bwd_layout(s, make_layout(s, make_plans(s, sms)).total).total;
+}
+
+dsv4v_status dsv4v_attention_backward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* qkv,
+                                      const void* out, const void* d_out, void* dqkv, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  Ctx c;
+  BwdLayout bl;
+  DSV4V_TRY(bwd_prepare(cfg, batch, workspace, ws_bytes, stream, c, bl));
+  for (const void* p : {qkv, out, d_out, static_cast<const void*>(dqkv)})
+    if (!p || !aligned16(p)) return DSV4V_ERR_INVALID_ARG;
+  return attention_bwd(c, bl, batch, qkv, out, d_out, dqkv);
+}
+
+dsv4v_status dsv4v_rmsnorm_backward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x, const float* w,
+                                    const void* dy, const void* d_in, void* dx, float* dw, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  Ctx c;
+  BwdLayout bl;
+  DSV4V_TRY(bwd_prepare(cfg, batch, workspace, ws_bytes, stream, c, bl));
+  for (const void* p : {x, static_cast<const void*>(w), dy, static_cast<const void*>(dx), static_cast<const void*>(dw)})
+    if (!p || !aligned16(p)) return DSV4V_ERR_INVALID_ARG;
+  if (d_in && !aligned16(d_in)) return DSV4V_ERR_INVALID_ARG;
+  return rmsnorm_bwd(c, bl, x, w, dy, d_in, dx, dw);
+}
+
+dsv4v_status dsv4v_block_backward(const dsv4v_config* cfg, const dsv4v_batch* batch,
+                                  const dsv4v_block_weights* weights, const float* cos, const float* sin, const void* x,
+                                  const void* d_out, void* dx, const dsv4v_block_grads* grads, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  Ctx c;
+  BwdLayout bl;
+  DSV4V_TRY(bwd_prepare(cfg, batch, workspace, ws_bytes, stream, c, bl));
+  if (!weights_ok(weights) || !grads_ok(grads) || !cos || !sin || !aligned16(cos) || !aligned16(sin))
+    return DSV4V_ERR_INVALID_ARG;
+  for (const void* p : {x, d_out, static_cast<const void*>(dx)})
+    if (!p || !aligned16(p)) return DSV4V_ERR_INVALID_ARG;
+  return block_backward_bf16(c, bl, batch, weights, cos, sin, x, d_out, dx, grads);
+}
+
+dsv4v_status dsv4v_tower_backward(const dsv4v_config* cfg, const dsv4v_batch* batch, const dsv4v_block_weights* layers,
+                                  const float* final_norm_w, const void* const* layer_inputs, const void* x_last,
+                                  const void* d_out, void* dx, const dsv4v_block_grads* layer_grads,
+                                  float* d_final_norm_w, void* workspace, size_t ws_bytes, void* stream) {
+  Ctx c;
+  BwdLayout bl;
+  DSV4V_TRY(bwd_prepare(cfg, batch, workspace, ws_bytes, stream, c, bl));
+  const int L = c.s.L;
+  if (L < 1 || !layers || !layer_inputs || !layer_grads || !d_out || !dx || !aligned16(d_out) || !aligned16(dx))
+    return DSV4V_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l)
+    if (!weights_ok(&layers[l]) || !grads_ok(&layer_grads[l]) || !layer_inputs[l] || !aligned16(layer_inputs[l]))
+      return DSV4V_ERR_INVALID_ARG;
+  if (final_norm_w && (!aligned16(final_norm_w) || !x_last || !aligned16(x_last) || !d_final_norm_w ||
+                       !aligned16(d_final_norm_w)))
+    return DSV4V_ERR_INVALID_ARG;
+  float* cos = c.at<float>(c.lay.cos);
+  float* sin = c.at<float>(c.lay.sin);
+  DSV4V_TRY(rope_table(c, batch, cos, sin));
+  const void* d = d_out;
+  void* bufs[2] = {c.at<void>(bl.dcur0), c.at<void>(bl.dcur1)};
+  int next = 0;
+  if (final_norm_w) {
+    DSV4V_TRY(rmsnorm_bwd(c, bl, x_last, final_norm_w, d_out, nullptr, bufs[next], d_final_norm_w));
+    d = bufs[next];
+    next ^= 1;
+  }
+  for (int l = L - 1; l >= 0; --l) {
+    void* target = l == 0 ? dx : bufs[next];
+    DSV4V_TRY(block_backward_bf16(c, bl, batch, &layers[l], cos, sin, layer_inputs[l], d, target, &layer_grads[l]));
+    d = target;
+    next ^= 1;
+  }
+  return DSV4V_OK;
+}
+
 }  // extern "C"

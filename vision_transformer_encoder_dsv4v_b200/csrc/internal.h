@@ -111,6 +111,19 @@ cudaError_t launch_merge_rows_bf16(const void* x, const int32_t* src, void* merg
 cudaError_t launch_ln_merge(bool bf16, const void* x, const int32_t* src, const float* w, const float* b, float eps,
                             void* merged, int64_t n_tokens, int r2, int d, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
+// Backward of the block (backward.cu).  All bf16 except the fp32 norm weights, their gradients,
+// the rotation tables and the attention row statistics.
+cudaError_t launch_transpose_bf16(const void* in, int64_t rows, int cols, int64_t ld_in, void* out, int64_t ld_out,
+                                  int64_t col0, cudaStream_t s);
+cudaError_t launch_rmsnorm_bwd(const void* x, const float* w, const void* dy, const void* d_in, void* dx,
+                               float* partial, int parts, float* dw, int64_t rows, int d, float eps, cudaStream_t s);
+cudaError_t launch_swiglu_bwd(const void* g, const void* u, const void* dh, void* dgu, void* h, int64_t rows, int f,
+                              int sms, cudaStream_t s);
+cudaError_t launch_rotary_bwd(void* dqkv, const float* cos, const float* sin, int64_t P, int D, int hd, int sms,
+                              cudaStream_t s);
+cudaError_t launch_attention_bwd(const void* qkv, const void* out, const void* dout, void* dqkv, float* lse,
+                                 float* rowdot, const int32_t* cu_dev, int n_images, int total_blocks, int D, int H,
+                                 cudaStream_t s);
 // Image-token bridge (bridge.cu).  Positions per CTA of the merge; counts holds one int4 per
 // chunk of that many positions.
 constexpr int kBridgeChunk = 256;

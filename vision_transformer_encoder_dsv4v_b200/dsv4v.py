@@ -33,7 +33,9 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_linear_residual", "dsv4v_swiglu", "dsv4v_device_error", "dsv4v_selftest_bounded_wait",
            "dsv4v_status_string", "dsv4v_linear_residual_noalloc", "dsv4v_patch_embed",
            "dsv4v_patch_merger_workspace_size", "dsv4v_patch_merger_forward", "dsv4v_image_layout",
-           "dsv4v_bridge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility")
+           "dsv4v_bridge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility",
+           "dsv4v_backward_workspace_size", "dsv4v_attention_backward", "dsv4v_rmsnorm_backward",
+           "dsv4v_block_backward", "dsv4v_tower_backward")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -51,6 +53,12 @@ class Config(ctypes.Structure):
 
 
 class BlockWeights(ctypes.Structure):
+    _fields_ = [("norm1_w", ctypes.c_void_p), ("norm2_w", ctypes.c_void_p), ("wqkv", ctypes.c_void_p),
+                ("wo", ctypes.c_void_p), ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
+                ("w_down", ctypes.c_void_p)]
+
+
+class BlockGrads(ctypes.Structure):
     _fields_ = [("norm1_w", ctypes.c_void_p), ("norm2_w", ctypes.c_void_p), ("wqkv", ctypes.c_void_p),
                 ("wo", ctypes.c_void_p), ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
                 ("w_down", ctypes.c_void_p)]
@@ -91,6 +99,11 @@ def lib() -> ctypes.CDLL:
             "dsv4v_patch_merger_forward": (I, [cfg, bat, P, P, P, P, P, P, P, P, P, SZ, P]),
             "dsv4v_linear_residual_noalloc": (I, [cfg, I64, I, P, P, P, P]),
             "dsv4v_image_layout": (I, [I, I, I, P, I64, ctypes.POINTER(ctypes.c_int64)]),
+            "dsv4v_backward_workspace_size": (SZ, [cfg, bat]),
+            "dsv4v_attention_backward": (I, [cfg, bat, P, P, P, P, P, SZ, P]),
+            "dsv4v_rmsnorm_backward": (I, [cfg, bat, P, P, P, P, P, P, P, SZ, P]),
+            "dsv4v_block_backward": (I, [cfg, bat, bw, P, P, P, P, P, ctypes.POINTER(BlockGrads), P, SZ, P]),
+            "dsv4v_tower_backward": (I, [cfg, bat, bw, P, P, P, P, P, ctypes.POINTER(BlockGrads), P, P, SZ, P]),
             "dsv4v_bridge_workspace_size": (SZ, [I64]),
             "dsv4v_merge_image_embeddings": (I, [cfg, bat, I64, I64, P, P, P, P, P, SZ, P]),
             "dsv4v_image_visibility": (I, [I64, I64, P, P, I, P, SZ, P]),
@@ -287,6 +300,55 @@ def dsv4v_image_visibility(token_types, mask, workspace, stream=None):
                                         _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                         _stream(stream)),
            "dsv4v_image_visibility")
+
+
+# ------------------------------------------------------------------------------ backward
+def block_grads(norm1_w, norm2_w, wqkv, wo, w_gate, w_up, w_down) -> BlockGrads:
+    """A dsv4v_block_grads of the given device tensors (the caller keeps them alive)."""
+    return BlockGrads(*[t.data_ptr() for t in (norm1_w, norm2_w, wqkv, wo, w_gate, w_up, w_down)])
+
+
+def dsv4v_backward_workspace_size(cfg, batch) -> int:
+    return int(lib().dsv4v_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(batch.c)))
+
+
+def _ws(workspace):
+    return _ptr(workspace), workspace.numel() if workspace is not None else 0
+
+
+def dsv4v_attention_backward(cfg, batch, qkv, out, d_out, dqkv, workspace, stream=None):
+    """dqkv [P, 3D] <- gradients of the attention w.r.t. its (rotated) q, k and v."""
+    _check(lib().dsv4v_attention_backward(ctypes.byref(cfg), ctypes.byref(batch.c), _ptr(qkv), _ptr(out), _ptr(d_out),
+                                          _ptr(dqkv), *_ws(workspace), _stream(stream)),
+           "dsv4v_attention_backward")
+
+
+def dsv4v_rmsnorm_backward(cfg, batch, x, w, dy, d_in, dx, dw, workspace, stream=None):
+    _check(lib().dsv4v_rmsnorm_backward(ctypes.byref(cfg), ctypes.byref(batch.c), _ptr(x), _ptr(w), _ptr(dy),
+                                        _ptr(d_in), _ptr(dx), _ptr(dw), *_ws(workspace), _stream(stream)),
+           "dsv4v_rmsnorm_backward")
+
+
+def dsv4v_block_backward(cfg, batch, weights, cos, sin, x, d_out, dx, grads, workspace, stream=None):
+    """weights: BlockWeights; grads: BlockGrads (see block_grads)."""
+    _check(lib().dsv4v_block_backward(ctypes.byref(cfg), ctypes.byref(batch.c), ctypes.byref(weights), _ptr(cos),
+                                      _ptr(sin), _ptr(x), _ptr(d_out), _ptr(dx), ctypes.byref(grads), *_ws(workspace),
+                                      _stream(stream)),
+           "dsv4v_block_backward")
+
+
+def dsv4v_tower_backward(cfg, batch, layers, final_norm_w, layer_inputs, x_last, d_out, dx, layer_grads,
+                         d_final_norm_w, workspace, stream=None):
+    """layers: list of BlockWeights; layer_inputs: list of device tensors (each block's input);
+    layer_grads: list of BlockGrads."""
+    n = len(layer_inputs)
+    arr = (BlockWeights * n)(*layers)
+    inputs = (ctypes.c_void_p * n)(*[t.data_ptr() for t in layer_inputs])
+    grads = (BlockGrads * n)(*layer_grads)
+    _check(lib().dsv4v_tower_backward(ctypes.byref(cfg), ctypes.byref(batch.c), arr, _ptr(final_norm_w), inputs,
+                                      _ptr(x_last), _ptr(d_out), _ptr(dx), grads, _ptr(d_final_norm_w),
+                                      *_ws(workspace), _stream(stream)),
+           "dsv4v_tower_backward")
 
 
 def dsv4v_device_error(stream=None) -> int:
