@@ -570,22 +570,35 @@ def block_backward_timing(A, torch, cfg, batch, wl, lw, stream, flush, steps):
     sin = torch.empty_like(cos)
     A.dsv4v_rope2d_table(cfg, batch, cos, sin, stream=stream.cuda_stream)
     ws = torch.empty(A.dsv4v_backward_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
-    times = []
-    for i in range(steps + 3):
-        with torch.cuda.stream(stream):
-            flush.zero_()
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ev0.record(stream)
-            A.dsv4v_block_backward(cfg, batch, lw[0], cos, sin, x, do, dx, grads, ws, stream=stream.cuda_stream)
-            ev1.record(stream)
-        stream.synchronize()
-        if i >= 3:
-            times.append(ev0.elapsed_time(ev1))
+    def timed(fn):
+        out = []
+        for i in range(steps + 3):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ev0.record(stream)
+                fn()
+                ev1.record(stream)
+            stream.synchronize()
+            if i >= 3:
+                out.append(ev0.elapsed_time(ev1))
+        return sum(out) / len(out)
+
+    ms = timed(lambda: A.dsv4v_block_backward(cfg, batch, lw[0], cos, sin, x, do, dx, grads, ws,
+                                              stream=stream.cuda_stream))
+    # the attention backward alone, on the same shapes (its share of the call above)
+    qkv = torch.randn(P, 3 * D, device="cuda", generator=g).to(torch.bfloat16)
+    att = torch.empty(P, D, dtype=torch.bfloat16, device="cuda")
+    dqkv = torch.empty(P, 3 * D, dtype=torch.bfloat16, device="cuda")
+    A.dsv4v_attention(cfg, batch, qkv, att, stream=stream.cuda_stream)
+    attn_ms = timed(lambda: A.dsv4v_attention_backward(cfg, batch, qkv, att, do, dqkv, ws, stream=stream.cuda_stream))
     if A.dsv4v_device_error(stream.cuda_stream) != 0:
         raise RuntimeError("device-side check failed in the block backward")
-    ms = sum(times) / len(times)
-    flops = 2.0 * P * (8 * D * D + 6 * D * F) + sum(8.0 * (h * w) ** 2 * D for h, w in wl.grids)
+    attn_flops = sum(8.0 * (h * w) ** 2 * D for h, w in wl.grids)
+    flops = 2.0 * P * (8 * D * D + 6 * D * F) + attn_flops
     return {"avg_us": ms * 1e3, "tflops": flops / (ms * 1e-3) / 1e12, "patches": P,
+            "attention_backward": {"avg_us": attn_ms * 1e3, "tflops": attn_flops / (attn_ms * 1e-3) / 1e12,
+                                   "launches_per_call": 2},
             "note": "standalone, one call per timed interval after an L2 flush; recompute + backward of one "
                     "block; attention backward on CUDA cores; not in value"}
 
