@@ -26,6 +26,7 @@ GRIDS = {
     "28x28": [(28, 28)],
     "ragged4": [(27, 37), (37, 27), (10, 78), (112, 7)],
     "small": [(3, 5), (1, 1), (9, 14)],
+    "one_patch": [(1, 1)],  # the weight gradients reduce over K = P = 1
 }
 
 
@@ -88,11 +89,15 @@ def test_attention_backward(name):
     dq, dk, dv = G.attention_backward(q, k, v, do.values, grids)
     got = to_np(dqkv)
     for i, want in enumerate((dq, dk, dv)):
-        err = rel_fro(got[:, i * D:(i + 1) * D], want.reshape(P, D))
+        w, g = want.reshape(P, D), got[:, i * D:(i + 1) * D]
+        if not w.any():  # one key: the softmax is exactly 1, so dq = dk = 0 up to fp32 rounding
+            assert np.linalg.norm(g) <= 1e-3 * np.linalg.norm(do.values), i
+            continue
+        err = rel_fro(g, w)
         assert err < 1e-2, (i, err)
 
 
-@pytest.mark.parametrize("name", ["28x28", "small"])
+@pytest.mark.parametrize("name", ["28x28", "small", "one_patch"])
 def test_rmsnorm_backward(name):
     cfg = cfg_bf16()
     b = A.BatchRef(GRIDS[name])
