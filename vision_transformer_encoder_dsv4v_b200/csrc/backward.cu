@@ -23,7 +23,8 @@ namespace dsv4v {
 namespace {
 
 // ------------------------------------------------------------------------------ transpose
-// out[(col0 + c) ... ]: out[c * ld_out + col0 + r] = in[r * ld_in + c] for r < rows, c < cols.
+// out[c * ld_out + col0 + r] = in[r * ld_in + c] for r < rows, c < cols: a 32 x 32 tile per CTA
+// through shared memory, so that both the reads and the writes run along rows.
 __global__ void __launch_bounds__(256)
     k_transpose_bf16(const __nv_bfloat16* __restrict__ in, int64_t rows, int cols, int64_t ld_in,
                      __nv_bfloat16* __restrict__ out, int64_t ld_out, int64_t col0) {
