@@ -450,7 +450,9 @@ def test_merge_image_embeddings_encoded_rows():
     flat_t, flat_o, flat_in = types.reshape(-1), out.reshape(-1, e), embeds.reshape(-1, e)
     feats = flat_o[flat_t == O.TOK_IMAGE, 0]
     assert feats.tolist() == list(range(sum(per_image)))
-    for code, row in zip(O.SENTINEL_ORDER, range(4)):
+    # the sentinel rows are image_start, image_end, image_newline, image_pad (types 1, 2, 3, 4),
+    # written out here rather than read from the oracle
+    for code, row in ((1, 0), (2, 1), (3, 2), (4, 3)):
         assert (flat_o[flat_t == code] == -(row + 1.0)).all()
     np.testing.assert_array_equal(flat_o[flat_t == O.TOK_TEXT], flat_in[flat_t == O.TOK_TEXT])
     assert int((flat_t == O.TOK_PAD).sum()) == 1
@@ -481,6 +483,19 @@ def test_merge_image_embeddings_rejects_layouts_that_do_not_fit(mutate):
     z = np.zeros(t.shape + (2,))
     with pytest.raises(ValueError):
         O.merge_image_embeddings(z, t, np.zeros((sum(per_image), 2)), np.zeros((4, 2)), per_image)
+
+
+@pytest.mark.parametrize("row", [[1, 0, -1, 0, 2],      # text inside a span
+                                 [1, 0, 1, 0, 2, 2],    # a start inside an open span
+                                 [0, 1, 0, 2],          # a feature before any span
+                                 [1, 0, 3],             # a span never closed
+                                 [2, 1, 0, 2],          # an end outside a span
+                                 [1, 5, 2]])            # an unknown code
+def test_image_spans_rejects_malformed_rows(row):
+    with pytest.raises(ValueError):
+        O.image_spans(np.array(row))
+    with pytest.raises(ValueError):
+        O.image_visibility(np.zeros((1, len(row), len(row))), np.array([row]))
 
 
 def test_image_visibility_hand_table():
