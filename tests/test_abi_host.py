@@ -174,3 +174,11 @@ def test_backward_host_checks(lib):
     small = lib.dsv4v_backward_workspace_size(ctypes.byref(cfg()), ctypes.byref(HostBatch([(3, 5)]).c))
     big = lib.dsv4v_backward_workspace_size(ctypes.byref(cfg()), ctypes.byref(b.c))
     assert 0 < small < big
+
+
+def test_backward_rejects_batches_past_the_transpose_grid(lib):
+    # the transposes cover P rows in 32-row CTAs along grid.y (at most 65535): a 1500 x 1500 image
+    # (2.25 M patches) is refused on the host, before any CUDA call
+    b = HostBatch([(1500, 1500)])
+    assert lib.dsv4v_block_backward(ctypes.byref(cfg()), ctypes.byref(b.c), None, None, None, None, None, None, None,
+                                    None, 0, None) == 2
