@@ -182,3 +182,21 @@ def test_backward_rejects_batches_past_the_transpose_grid(lib):
     b = HostBatch([(1500, 1500)])
     assert lib.dsv4v_block_backward(ctypes.byref(cfg()), ctypes.byref(b.c), None, None, None, None, None, None, None,
                                     None, 0, None) == 2
+
+
+def test_header_compiles_as_c99_and_links(lib, tmp_path):
+    # the public header is plain C: a C99 program includes it, links the library and runs the
+    # calls that need no GPU
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_host_check"
+    libdir = os.path.dirname(A.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_host_check.c"), "-o", str(exe), "-L", libdir, "-ldsv4v",
+                    f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert "c abi ok" in r.stdout
