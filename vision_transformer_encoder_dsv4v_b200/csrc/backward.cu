@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------------------ attention backward
 constexpr int kAB = 64;   // rows of a tile (queries or keys) and the head dim
-constexpr int kLd = 65;   // shared-memory row stride in floats
+constexpr int kLd = 68;   // shared-memory row stride in floats (16-byte rows for vector access)
 constexpr int kTile = kAB * kLd;
 
 // Block-count offsets of the images (ceil(N_i / 64) blocks each), by one warp; then the image
@@ -226,40 +226,62 @@ __device__ __forceinline__ int image_of_block(const int32_t* blk_cu, int n_image
   return lo;
 }
 
+// Eight channels [col0 + 8v, col0 + 8v + 8) of row `row` (zeros past row_end), as floats.
+__device__ __forceinline__ void load8(const __nv_bfloat16* __restrict__ src, int64_t ld, int64_t row, int64_t row_end,
+                                      int64_t col0, int v, float out[8]) {
+  if (row < row_end) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(src + row * ld + col0 + v * 8);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      out[2 * k] = __low2float(h2[k]);
+      out[2 * k + 1] = __high2float(h2[k]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) out[k] = 0.0f;
+  }
+}
+
 // dst[r][c] = src[(row0 + r) * ld + col0 + c] for r < 64, c < 64, zero for rows >= row_end.
 __device__ __forceinline__ void load_tile(float* dst, const __nv_bfloat16* __restrict__ src, int64_t ld, int64_t row0,
                                           int64_t row_end, int64_t col0) {
   for (int i = threadIdx.x; i < kAB * 8; i += blockDim.x) {
     const int r = i >> 3, v = i & 7;
-    const int64_t row = row0 + r;
-    float* d = dst + r * kLd + v * 8;
-    if (row < row_end) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(src + row * ld + col0 + v * 8);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    float f[8];
+    load8(src, ld, row0 + r, row_end, col0, v, f);
+    float4* d = reinterpret_cast<float4*>(dst + r * kLd + v * 8);
+    d[0] = make_float4(f[0], f[1], f[2], f[3]);
+    d[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+// The transpose: dst[c][r] = src[(row0 + r) * ld + col0 + c].  Consecutive lanes take
+// consecutive rows, so the shared-memory stores of a warp hit consecutive banks.
+__device__ __forceinline__ void load_tile_t(float* dst, const __nv_bfloat16* __restrict__ src, int64_t ld,
+                                            int64_t row0, int64_t row_end, int64_t col0) {
+  for (int i = threadIdx.x; i < kAB * 8; i += blockDim.x) {
+    const int r = i & (kAB - 1), v = i >> 6;
+    float f[8];
+    load8(src, ld, row0 + r, row_end, col0, v, f);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        d[2 * k] = __low2float(h2[k]);
-        d[2 * k + 1] = __high2float(h2[k]);
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) d[k] = 0.0f;
-    }
+    for (int k = 0; k < 8; ++k) dst[(v * 8 + k) * kLd + r] = f[k];
   }
 }
 
 // acc[a][b] += sum over t < 64 of A(r0 + a, t) * B(t, s0 + b), with A(r, t) = A[r * ars + t * ats]
-// and B(t, s) = B[t * bts + s * bss] in shared memory.
-__device__ __forceinline__ void mm64(const float* A, int ars, int ats, const float* B, int bts, int bss, int r0, int s0,
+// and B(t, s) = B[t * bts + s] in shared memory.  B is read as one 16-byte vector per t (the 16
+// column groups of a half-warp cover 256 contiguous bytes); A's four values are shared by the
+// half-warp and broadcast.
+__device__ __forceinline__ void mm64(const float* A, int ars, int ats, const float* B, int bts, int r0, int s0,
                                      float acc[4][4]) {
 #pragma unroll 4
   for (int t = 0; t < kAB; ++t) {
-    float a[4], b[4];
+    float a[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      a[i] = A[(r0 + i) * ars + t * ats];
-      b[i] = B[t * bts + (s0 + i) * bss];
-    }
+    for (int i = 0; i < 4; ++i) a[i] = A[(r0 + i) * ars + t * ats];
+    const float4 bv = *reinterpret_cast<const float4*>(B + t * bts + s0);
+    const float b[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -290,11 +312,12 @@ struct AttnBwdArgs {
 // s0..s0+3 (s0 = (t % 16) * 4); the 16 threads of a row group are 16 consecutive lanes.
 __global__ void __launch_bounds__(256) k_attn_bwd_dq(AttnBwdArgs a) {
   extern __shared__ float sm[];
-  float* sQ = sm;
-  float* sDO = sQ + kTile;
-  float* sK = sDO + kTile;
-  float* sV = sK + kTile;
-  float* sS = sV + kTile;
+  float* sQ = sm;            // [query][channel]
+  float* sDO = sQ + kTile;   // [query][channel]
+  float* sKt = sDO + kTile;  // [channel][key]
+  float* sVt = sKt + kTile;  // [channel][key]
+  float* sK = sVt + kTile;   // [key][channel]
+  float* sS = sK + kTile;    // [query][key]: dS
   float* sRowDot = sS + kTile;                              // [64]
   int32_t* blk_cu = reinterpret_cast<int32_t*>(sRowDot + kAB);  // [n_images + 1]
   grid_dependency_wait();
@@ -327,11 +350,11 @@ __global__ void __launch_bounds__(256) k_attn_bwd_dq(AttnBwdArgs a) {
   }
   for (int kb = 0; kb < n_kb; ++kb) {
     const int64_t k0 = beg + static_cast<int64_t>(kb) * kAB;
-    load_tile(sK, a.qkv, ld3, k0, end, D + static_cast<int64_t>(h) * kAB);
+    load_tile_t(sKt, a.qkv, ld3, k0, end, D + static_cast<int64_t>(h) * kAB);
     __syncthreads();
     float acc[4][4];
     zero44(acc);
-    mm64(sQ, kLd, 1, sK, 1, kLd, r0, s0, acc);
+    mm64(sQ, kLd, 1, sKt, kLd, r0, s0, acc);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -365,23 +388,27 @@ __global__ void __launch_bounds__(256) k_attn_bwd_dq(AttnBwdArgs a) {
   zero44(dq);
   for (int kb = 0; kb < n_kb; ++kb) {
     const int64_t k0 = beg + static_cast<int64_t>(kb) * kAB;
+    load_tile_t(sKt, a.qkv, ld3, k0, end, D + static_cast<int64_t>(h) * kAB);
+    load_tile_t(sVt, a.qkv, ld3, k0, end, 2 * D + static_cast<int64_t>(h) * kAB);
     load_tile(sK, a.qkv, ld3, k0, end, D + static_cast<int64_t>(h) * kAB);
-    load_tile(sV, a.qkv, ld3, k0, end, 2 * D + static_cast<int64_t>(h) * kAB);
     __syncthreads();
     float s[4][4], dp[4][4];
     zero44(s);
     zero44(dp);
-    mm64(sQ, kLd, 1, sK, 1, kLd, r0, s0, s);
-    mm64(sDO, kLd, 1, sV, 1, kLd, r0, s0, dp);
+    mm64(sQ, kLd, 1, sKt, kLd, r0, s0, s);
+    mm64(sDO, kLd, 1, sVt, kLd, r0, s0, dp);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
+      float ds[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float p = k0 + s0 + j < end ? expf(s[i][j] * a.scale - lse[i]) : 0.0f;
-        sS[(r0 + i) * kLd + s0 + j] = p * (dp[i][j] - sRowDot[r0 + i]);
+        ds[j] = p * (dp[i][j] - sRowDot[r0 + i]);
       }
+      *reinterpret_cast<float4*>(sS + (r0 + i) * kLd + s0) = make_float4(ds[0], ds[1], ds[2], ds[3]);
+    }
     __syncthreads();
-    mm64(sS, kLd, 1, sK, kLd, 1, r0, s0, dq);
+    mm64(sS, kLd, 1, sK, kLd, r0, s0, dq);
     __syncthreads();
   }
 
@@ -400,12 +427,12 @@ __global__ void __launch_bounds__(256) k_attn_bwd_dq(AttnBwdArgs a) {
 
 __global__ void __launch_bounds__(256) k_attn_bwd_dkdv(AttnBwdArgs a) {
   extern __shared__ float sm[];
-  float* sK = sm;
-  float* sV = sK + kTile;
-  float* sQ = sV + kTile;
-  float* sDO = sQ + kTile;
-  float* sP = sDO + kTile;
-  float* sDS = sP + kTile;
+  float* sKt = sm;            // [channel][key]
+  float* sVt = sKt + kTile;   // [channel][key]
+  float* sQ = sVt + kTile;    // [query][channel]
+  float* sDO = sQ + kTile;    // [query][channel]
+  float* sP = sDO + kTile;    // [query][key]
+  float* sDS = sP + kTile;    // [query][key]
   float* sLse = sDS + kTile;                                // [64]
   float* sRowDot = sLse + kAB;                              // [64]
   int32_t* blk_cu = reinterpret_cast<int32_t*>(sRowDot + kAB);  // [n_images + 1]
@@ -419,8 +446,8 @@ __global__ void __launch_bounds__(256) k_attn_bwd_dkdv(AttnBwdArgs a) {
   const int64_t k0 = beg + static_cast<int64_t>(blockIdx.x - blk_cu[img]) * kAB;
   const int n_qb = static_cast<int>((end - beg + kAB - 1) / kAB);
 
-  load_tile(sK, a.qkv, ld3, k0, end, D + static_cast<int64_t>(h) * kAB);
-  load_tile(sV, a.qkv, ld3, k0, end, 2 * D + static_cast<int64_t>(h) * kAB);
+  load_tile_t(sKt, a.qkv, ld3, k0, end, D + static_cast<int64_t>(h) * kAB);
+  load_tile_t(sVt, a.qkv, ld3, k0, end, 2 * D + static_cast<int64_t>(h) * kAB);
   float dk[4][4], dv[4][4];
   zero44(dk);
   zero44(dv);
@@ -437,20 +464,23 @@ __global__ void __launch_bounds__(256) k_attn_bwd_dkdv(AttnBwdArgs a) {
     float s[4][4], dp[4][4];
     zero44(s);
     zero44(dp);
-    mm64(sQ, kLd, 1, sK, 1, kLd, r0, s0, s);    // rows: queries, columns: keys
-    mm64(sDO, kLd, 1, sV, 1, kLd, r0, s0, dp);
+    mm64(sQ, kLd, 1, sKt, kLd, r0, s0, s);    // rows: queries, columns: keys
+    mm64(sDO, kLd, 1, sVt, kLd, r0, s0, dp);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
+      float pv[4], ds[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const bool ok = q0 + r0 + i < end && k0 + s0 + j < end;
-        const float p = ok ? expf(s[i][j] * a.scale - sLse[r0 + i]) : 0.0f;
-        sP[(r0 + i) * kLd + s0 + j] = p;
-        sDS[(r0 + i) * kLd + s0 + j] = p * (dp[i][j] - sRowDot[r0 + i]);
+        pv[j] = ok ? expf(s[i][j] * a.scale - sLse[r0 + i]) : 0.0f;
+        ds[j] = pv[j] * (dp[i][j] - sRowDot[r0 + i]);
       }
+      *reinterpret_cast<float4*>(sP + (r0 + i) * kLd + s0) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+      *reinterpret_cast<float4*>(sDS + (r0 + i) * kLd + s0) = make_float4(ds[0], ds[1], ds[2], ds[3]);
+    }
     __syncthreads();
-    mm64(sP, 1, kLd, sDO, kLd, 1, r0, s0, dv);   // rows: keys, columns: channels
-    mm64(sDS, 1, kLd, sQ, kLd, 1, r0, s0, dk);
+    mm64(sP, 1, kLd, sDO, kLd, r0, s0, dv);   // rows: keys, columns: channels
+    mm64(sDS, 1, kLd, sQ, kLd, r0, s0, dk);
     __syncthreads();
   }
 #pragma unroll
@@ -507,7 +537,7 @@ cudaError_t launch_rotary_bwd(void* dqkv, const float* cos, const float* sin, in
 }
 
 size_t attn_bwd_smem(int kernel, int n_images) {
-  const size_t tiles = kernel == 0 ? 5 : 6;
+  const size_t tiles = 6;
   const size_t vecs = kernel == 0 ? 1 : 2;
   return tiles * kTile * sizeof(float) + vecs * kAB * sizeof(float) + (n_images + 1) * sizeof(int32_t);
 }
