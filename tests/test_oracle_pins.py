@@ -128,6 +128,98 @@ def test_rotary_relative_position_property():
     assert abs(dot(0, 1) - dot(0, 2)) > 1e-6
 
 
+# ------------------------------------------------------------------------------- fused projection + rotation
+def _qkv_rope_checks(qkv_rope):
+    """Facts about the projection-plus-rotation of one 6x6 image that hold for the stated
+    definition [vision-API, DeepseekV4VisionAttention, apply_vision_rotary]; returns the names of
+    the ones that fail.  (a) with one y row shared by every patch, q_p . k_p' of each head depends
+    only on (h - h', w - w'): fails when q or k is left unrotated; (b) with that shared row every
+    v row is equal: fails when v is rotated; (c) with distinct random y, q and k equal the
+    rotation, written out by hand below, of y . W[0:D]^T and y . W[D:2D]^T and v equals
+    y . W[2D:3D]^T: fails on a swap or reorder of the q | k | v blocks."""
+    n, d, nh = 6, 16, 2
+    hd = d // nh
+    rng = np.random.default_rng(77)
+    cos, sin = O.vision_cos_sin(n, n, hd // 2, 100.0)
+    w = rng.normal(size=(3 * d, d))
+    failed = []
+    y_same = np.tile(rng.normal(size=(1, d)), (n * n, 1))
+    q, k, v = qkv_rope(y_same, w, cos, sin, nh)
+
+    def dot(h, p, pp):
+        return float(np.dot(q[p, h], k[pp, h]))
+
+    rel_ok = True
+    for h in range(nh):
+        for (a, b, a2, b2, dh, dw) in [(0, 1, 3, 4, 2, 1), (5, 0, 3, 2, -3, 3), (2, 4, 0, 5, 1, -4),
+                                       (1, 3, 4, 0, 1, 2)]:
+            assert all(0 <= t < n for t in (a + dh, a2 + dh, b + dw, b2 + dw))
+            x0 = dot(h, a * n + b, a2 * n + b2)
+            x1 = dot(h, (a + dh) * n + (b + dw), (a2 + dh) * n + (b2 + dw))
+            rel_ok &= abs(x0 - x1) < 1e-10 * max(1.0, abs(x0))
+    if not rel_ok:
+        failed.append("relative position")
+    if not np.allclose(v, v[:1], rtol=0, atol=1e-12):
+        failed.append("v rows equal")
+    y = rng.normal(size=(n * n, d))
+    q, k, v = qkv_rope(y, w, cos, sin, nh)
+    blocks_ok = True
+    for p in range(n * n):
+        for h in range(nh):
+            for which, got in ((0, q), (1, k)):
+                lin = [sum(y[p, c] * w[which * d + h * hd + j, c] for c in range(d)) for j in range(hd)]
+                for j in range(hd // 2):
+                    c_, s_ = cos[p, j], sin[p, j]
+                    want_lo = lin[j] * c_ - lin[j + hd // 2] * s_
+                    want_hi = lin[j + hd // 2] * c_ + lin[j] * s_
+                    blocks_ok &= abs(got[p, h, j] - want_lo) < 1e-11 and abs(got[p, h, j + hd // 2] - want_hi) < 1e-11
+            for j in range(hd):
+                want_v = sum(y[p, c] * w[2 * d + h * hd + j, c] for c in range(d))
+                blocks_ok &= abs(v[p, h, j] - want_v) < 1e-11
+    if not blocks_ok:
+        failed.append("q | k | v blocks")
+    return failed
+
+
+def test_qkv_rope_rotates_q_and_k_in_block_order():
+    assert _qkv_rope_checks(O.qkv_rope) == []
+
+
+def _planted(kind):
+    """Copies of the oracle's projection with one plausible mistake each (planted here, on the
+    CPU, to show that the checks above catch it)."""
+    def f(y, wqkv, cos, sin, n_heads):
+        y = np.asarray(y, dtype=np.float64)
+        d = y.shape[1]
+        hd = d // n_heads
+        qkv = y @ np.asarray(wqkv, dtype=np.float64).T
+        q = qkv[:, :d].reshape(-1, n_heads, hd)
+        k = qkv[:, d:2 * d].reshape(-1, n_heads, hd)
+        v = qkv[:, 2 * d:].reshape(-1, n_heads, hd)
+        rot = lambda t: O.apply_vision_rotary(t, cos, sin)
+        if kind == "rotate q only":
+            return rot(q), k, v
+        if kind == "rotate k only":
+            return q, rot(k), v
+        if kind == "swap q and k":
+            return rot(k), rot(q), v
+        if kind == "rotate v too":
+            return rot(q), rot(k), rot(v)
+        if kind == "k and v blocks swapped":
+            return rot(q), rot(v), k
+        raise ValueError(kind)
+    return f
+
+
+@pytest.mark.parametrize("kind,caught_by", [("rotate q only", "relative position"),
+                                            ("rotate k only", "relative position"),
+                                            ("swap q and k", "q | k | v blocks"),
+                                            ("rotate v too", "v rows equal"),
+                                            ("k and v blocks swapped", "q | k | v blocks")])
+def test_qkv_rope_checks_catch_planted_mistakes(kind, caught_by):
+    assert caught_by in _qkv_rope_checks(_planted(kind))
+
+
 # ------------------------------------------------------------------------------- attention
 def _naive_attention(q, k, v):
     """Pure-Python loops, exp without max subtraction, scale 1/sqrt(hd)."""
