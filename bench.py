@@ -163,7 +163,9 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        return parse_clock_lines(self.lines)
+        # the reader thread ends at EOF of the pipe; parse only once it has appended every line
+        self.thread.join(timeout=5)
+        return parse_clock_lines(list(self.lines))
 
 
 def parse_clock_lines(lines):

@@ -257,9 +257,11 @@ dsv4v_status dsv4v_swiglu(const dsv4v_config* cfg, int64_t rows, const void* y,
  * rows <= DSV4V_NOALLOC_MAX_ROWS; a larger call, or one whose GEMM plan needs more scratch than
  * the array holds, returns DSV4V_ERR_UNSUPPORTED without launching anything.  The first call on
  * a device looks the array's device address up (cudaGetSymbolAddress); make that first call
- * before any stream capture.  All calls on a device share the one array and each starts by
- * clearing its counters on `stream`: calls that overlap on the GPU (different streams, no
- * ordering) race on it.  The pages describe no counterpart of this call. */
+ * before any stream capture.  All calls on a device share the one array.  A call that is
+ * accepted clears, on `stream` and just before its GEMM, the counters its plan uses; a call that
+ * is refused (any error status) puts nothing on the stream.  Calls that overlap on the GPU
+ * (different streams, no ordering) race on the array.  The pages describe no counterpart of
+ * this call. */
 #define DSV4V_NOALLOC_MAX_ROWS 65536
 dsv4v_status dsv4v_linear_residual_noalloc(const dsv4v_config* cfg, int64_t rows, int k,
                                            const void* a, const void* w, void* x, void* stream);

@@ -165,10 +165,12 @@ def test_workload4_tower_aligner(workload4):
 
 
 # ------------------------------------------------------------------------------ workload 5
-def test_workload5_sampled_images():
-    """Full 16-image batch on the GPU in the benchmark's launch configuration; the oracle runs
-    on the three smallest images alone (images never interact, so their rows of the packed
-    result are exactly what the oracle computes for them)."""
+def test_workload5_images_against_oracle():
+    """Full 16-image batch on the GPU in the benchmark's launch configuration.  Images never
+    interact, so each image's rows of the packed result are exactly what the oracle computes for
+    that image alone; the oracle runs, alone, on the three smallest images, the two closest to
+    1000 patches (the size class of the pages' validation grids), the largest odd (zero-padded)
+    grid and the 64x64 image (4096 patches: 32 key tiles, paired query tiles)."""
     wl = synth.workload(5)
     inp = synth.draw(wl)
     tower_g, align_g = run_tower_and_aligner(wl, inp)
@@ -176,7 +178,13 @@ def test_workload5_sampled_images():
     r = wl.downsample_ratio
     tok = np.cumsum([0] + [-(-h // r) * -(-w // r) for h, w in wl.grids])
     sizes = [h * w for h, w in wl.grids]
-    for i in sorted(range(len(sizes)), key=lambda k: sizes[k])[:3]:
+    by_size = sorted(range(len(sizes)), key=lambda k: sizes[k])
+    near_1000 = sorted(range(len(sizes)), key=lambda k: abs(sizes[k] - 1000))[:2]
+    odd = [k for k in by_size if wl.grids[k][0] % r or wl.grids[k][1] % r]
+    square64 = [k for k in range(len(sizes)) if wl.grids[k] == (64, 64)]
+    assert len(square64) == 1 and odd
+    chosen = sorted(set(by_size[:3]) | set(near_1000) | {odd[-1]} | set(square64), key=lambda k: sizes[k])
+    for i in chosen:
         sub = synth.Inputs(wl, synth.Tensor(inp.x.values[cu[i]:cu[i + 1]]), inp.layers, inp.final_norm_w,
                            inp.w_align)
         sub.wl = synth.Workload(wl.name, wl.dtype, wl.vision_dim, wl.n_heads, wl.mlp_hidden, r, wl.llm_dim,

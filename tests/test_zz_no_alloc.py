@@ -42,3 +42,35 @@ def test_noalloc_rejects_sizes_beyond_its_limit():
     with pytest.raises(A.Dsv4vError) as e:
         A.dsv4v_linear_residual_noalloc(cfg, A.DSV4V_NOALLOC_MAX_ROWS + 1, 1024, a, a, a)
     assert e.value.status == 2   # DSV4V_ERR_UNSUPPORTED, nothing launched
+
+
+def test_noalloc_rejected_calls_enqueue_nothing():
+    """A call the entry point refuses (an fp32 config, a K that is neither D nor F, too many rows)
+    returns its error before putting any work on the stream: captured into a graph, it leaves
+    the graph empty (so it cannot clear counters that a call on another stream is using)."""
+    from cuda.bindings import runtime as rt
+
+    cfg_bf16 = A.make_config(1024, 16, 2816, 2, 4096, 1)
+    cfg_f32 = A.make_config(1024, 16, 2816, 2, 4096, 1, dtype=A.DSV4V_F32)
+    a = _bf16((784, 1024), 1.0, 1)
+    w = _bf16((1024, 1024), 0.02, 2)
+    x = _bf16((784, 1024), 1.0, 3)
+    A.dsv4v_linear_residual_noalloc(cfg_bf16, 784, 1024, a, w, x)  # first call on the device: outside capture
+    torch.cuda.synchronize()
+    err, s = rt.cudaStreamCreateWithFlags(rt.cudaStreamNonBlocking)
+    assert err == rt.cudaError_t.cudaSuccess
+    try:
+        for cfg, rows, k, status in [(cfg_f32, 784, 1024, 2), (cfg_bf16, 784, 1000, 1),
+                                     (cfg_bf16, A.DSV4V_NOALLOC_MAX_ROWS + 1, 1024, 2)]:
+            (err,) = rt.cudaStreamBeginCapture(s, rt.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
+            assert err == rt.cudaError_t.cudaSuccess
+            with pytest.raises(A.Dsv4vError) as e:
+                A.dsv4v_linear_residual_noalloc(cfg, rows, k, a, w, x, stream=int(s))
+            err, graph = rt.cudaStreamEndCapture(s)
+            assert err == rt.cudaError_t.cudaSuccess
+            err, _, n_nodes = rt.cudaGraphGetNodes(graph, 0)
+            assert err == rt.cudaError_t.cudaSuccess
+            rt.cudaGraphDestroy(graph)
+            assert e.value.status == status and n_nodes == 0
+    finally:
+        rt.cudaStreamDestroy(s)

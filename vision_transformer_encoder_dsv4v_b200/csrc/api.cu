@@ -293,6 +293,7 @@ struct NormFold {
 struct GemmExtra {
   int64_t lda = 0, ldb = 0;
   const float* bias = nullptr;
+  int clear_counters = 0;  // zero this many split-tile counters on the stream right before the launch
 };
 
 dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* a, int64_t M, int K, const void* b,
@@ -333,6 +334,9 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.ss_out = nf.ss_out;
   g.ss_parts = nf.ss_parts;
   g.bias = ex.bias;
+  if (ex.clear_counters > 0 &&
+      cudaMemsetAsync(g.counters, 0, static_cast<size_t>(ex.clear_counters) * sizeof(int), c.stream) != cudaSuccess)
+    return DSV4V_ERR_CUDA;
   return cuda_status(launch_gemm_tc(epi, plan, g, c.stream));
 }
 
@@ -506,8 +510,10 @@ dsv4v_status prepare_rows(const dsv4v_config* cfg, int64_t rows, void* workspace
 }  // namespace
 
 // Residual GEMM x <- x + a . w^T on the bf16 path with split-tile scratch supplied by the caller
-// (partials: partial_cap bytes, counters: counter_cap ints, zero on entry).  Used by the entry
-// point whose scratch is a static device array.
+// (partials: partial_cap bytes, counters: counter_cap ints).  Used by the entry point whose
+// scratch is a static device array: that array keeps the last call's contents, so the counters
+// the plan uses are cleared on the stream, but only once every argument and the plan have been
+// accepted (a rejected call enqueues nothing).
 dsv4v_status linear_residual_with_scratch(const dsv4v_config* cfg, int64_t rows, int k, const void* a,
                                           const void* w, void* x, float* partials, size_t partial_cap,
                                           int* counters, int counter_cap, void* stream) {
@@ -533,7 +539,9 @@ dsv4v_status linear_residual_with_scratch(const dsv4v_config* cfg, int64_t rows,
   c.lay = Layout{};
   c.lay.partials = 0;
   c.lay.counters = static_cast<size_t>(reinterpret_cast<uint8_t*>(counters) - reinterpret_cast<uint8_t*>(partials));
-  return gemm_bf16(c, EPI_RESID, plan, a, rows, k, w, nullptr, c.s.D, x, x);
+  GemmExtra ex;
+  ex.clear_counters = plan.counters;
+  return gemm_bf16(c, EPI_RESID, plan, a, rows, k, w, nullptr, c.s.D, x, x, nullptr, nullptr, NormFold(), ex);
 }
 
 }  // namespace dsv4v

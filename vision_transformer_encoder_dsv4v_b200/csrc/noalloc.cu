@@ -52,9 +52,8 @@ extern "C" dsv4v_status dsv4v_linear_residual_noalloc(const dsv4v_config* cfg, i
   if (st != DSV4V_OK) return st;
   float* partials = static_cast<float*>(base);
   int* counters = reinterpret_cast<int*>(static_cast<unsigned char*>(base) + kPartialBytes);
-  // The array keeps the previous call's contents; the tile counters must start at zero.
-  if (rows > 0 && cudaMemsetAsync(counters, 0, kCounters * sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return DSV4V_ERR_CUDA;
+  // The array keeps the previous call's contents; the tile counters the plan uses are cleared
+  // on the stream after the call has been accepted, just before the GEMM.
   return dsv4v::linear_residual_with_scratch(cfg, rows, k, a, w, x, partials, kPartialBytes, counters, kCounters,
                                              stream);
 }
