@@ -164,13 +164,40 @@ enum {
   DSV4V_PROFILE_OUT = 2,        /* output projection + residual (prepares norm2) */
   DSV4V_PROFILE_SWIGLU = 3,     /* gate/up GEMM + silu*mul (norm2 folded in) */
   DSV4V_PROFILE_DOWN = 4,       /* down projection + residual (prepares the next norm1) */
-  DSV4V_PROFILE_KINDS = 5
+  DSV4V_PROFILE_CHAIN = 5,      /* chained GEMMs of one block in one persistent launch (output
+                                   projection, SwiGLU, down projection and the next block's
+                                   q|k|v projection); see dsv4v_tower_path */
+  DSV4V_PROFILE_KINDS = 6
 };
+
+/* Launch sequence of the bf16 blocks (no effect on fp32 configs).  Both compute the same
+ * block, with the same roundings: they differ in how the GEMMs' K dimension is split, so sums
+ * of fp32 products may be added in another order.
+ *  DSV4V_PATH_KERNELS: one kernel per GEMM of the block (plus attention).
+ *  DSV4V_PATH_CHAIN:   per block, attention plus one persistent launch that runs the output
+ *                      projection, SwiGLU, the down projection and the next block's q|k|v
+ *                      projection with per-128-row-tile dependencies between them.
+ *  DSV4V_PATH_AUTO:    the sequence measured faster for the batch's size (at present one kernel
+ *                      per GEMM at every size). */
+enum { DSV4V_PATH_AUTO = 0, DSV4V_PATH_KERNELS = 1, DSV4V_PATH_CHAIN = 2 };
+
+/* Sets the launch sequence for the calls that follow, process-wide (host state only; the
+ * default is DSV4V_PATH_AUTO).  Workspace sizes depend on it: size the workspace after setting
+ * it.  Returns DSV4V_ERR_INVALID_ARG for an unknown value. */
+dsv4v_status dsv4v_set_tower_path(int path);
+
+/* The launch sequence dsv4v_block_forward / dsv4v_tower_forward use for this config and
+ * batch under the current setting: DSV4V_PATH_KERNELS or DSV4V_PATH_CHAIN; -1 if the arguments
+ * are invalid. */
+int dsv4v_tower_path(const dsv4v_config* cfg, const dsv4v_batch* batch);
 
 /* dsv4v_tower_forward, recording CUDA events around the launches of every layer:
  * events[(layer * DSV4V_PROFILE_KINDS + kind) * 2 + 0] before and [... + 1] after the kernel
  * of that class (cudaEvent_t handles passed as void*, created by the caller; NULL entries are
- * skipped).  The events sit between kernels, so the bracketed kernels cannot overlap their
+ * skipped).  With DSV4V_PATH_KERNELS the kinds QKV, ATTENTION, OUT, SWIGLU and DOWN are
+ * recorded; with DSV4V_PATH_CHAIN, ATTENTION and CHAIN (layer l's CHAIN launch runs its output
+ * projection, SwiGLU and down projection and layer l + 1's q|k|v projection; layer 0's q|k|v
+ * projection is a launch of its own that is not bracketed).  The events sit between kernels, so the bracketed kernels cannot overlap their
  * neighbours as in dsv4v_tower_forward; per-kernel durations from them are standalone
  * durations.  Same results as dsv4v_tower_forward. */
 dsv4v_status dsv4v_tower_forward_profiled(const dsv4v_config* cfg, const dsv4v_batch* batch,
@@ -310,7 +337,11 @@ size_t dsv4v_backward_workspace_size(const dsv4v_config* cfg, const dsv4v_batch*
  * dk = dS^T q / sqrt(hd), with P the softmax of the forward.
  *   qkv: device [P, 3D], the forward's input (q and k already rotated); out: device [P, D], the
  *   forward's output; d_out: device [P, D]; dqkv: device [P, 3D], written: the gradients with
- *   respect to the rotated q, k and to v. */
+ *   respect to the rotated q, k and to v.
+ * P is rebuilt from each row's log-sum-exp, which this call recomputes with the forward
+ * attention kernel (into scratch); dsv4v_block_backward takes it from its own forward
+ * recompute.  Every output row is written by exactly one CTA (no atomics): the result does not
+ * depend on the schedule. */
 dsv4v_status dsv4v_attention_backward(const dsv4v_config* cfg, const dsv4v_batch* batch,
                                       const void* qkv, const void* out, const void* d_out,
                                       void* dqkv, void* workspace, size_t ws_bytes, void* stream);

@@ -200,3 +200,22 @@ def test_header_compiles_as_c99_and_links(lib, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     assert "c abi ok" in r.stdout
+
+
+def test_tower_path_choice_and_validation():
+    """The launch-sequence setting and its automatic choice (host logic only: no kernel runs)."""
+    from vision_transformer_encoder_dsv4v_b200 import dsv4v as A
+    try:
+        with pytest.raises(A.Dsv4vError):
+            A.dsv4v_set_tower_path(7)
+        cfg = A.make_config(1024, 16, 2816, 2, 4096, 1)
+        A.dsv4v_set_tower_path(A.PATH_AUTO)
+        assert A.dsv4v_tower_path(cfg, A.BatchRef([(64, 64), (8, 8)], device=None)) == A.PATH_KERNELS
+        A.dsv4v_set_tower_path(A.PATH_KERNELS)
+        assert A.dsv4v_tower_path(cfg, A.BatchRef([(28, 28)], device=None)) == A.PATH_KERNELS
+        A.dsv4v_set_tower_path(A.PATH_CHAIN)
+        assert A.dsv4v_tower_path(cfg, A.BatchRef([(64, 64), (8, 8)], device=None)) == A.PATH_CHAIN
+        cfg32 = A.make_config(64, 4, 128, 2, 128, 1, dtype=A.DSV4V_F32)
+        assert A.dsv4v_tower_path(cfg32, A.BatchRef([(4, 6)], device=None)) == A.PATH_KERNELS
+    finally:
+        A.dsv4v_set_tower_path(A.PATH_AUTO)

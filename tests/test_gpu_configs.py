@@ -135,25 +135,36 @@ def run_tower_and_aligner(wl, inp):
     return to_np(x), to_np(out)
 
 
-def test_profiled_tower_matches_plain():
-    """dsv4v_tower_forward_profiled computes the same tower (bitwise) and records its events."""
-    wl = synth.workload(4)
-    inp = synth.draw(wl, n_layers=3)
-    cfg = config_of(wl, n_layers=3)
-    b = A.BatchRef(wl.grids)
-    ws = workspace(cfg, b)
-    layers = upload_layers(inp)
-    keep = [A.block_weights(l) for l in layers]
-    x1, x2 = dev(inp.x), dev(inp.x)
-    A.dsv4v_tower_forward(cfg, b, keep, None, x1, ws)
-    events = [torch.cuda.Event(enable_timing=True) for _ in range(3 * len(A.PROFILE_KINDS) * 2)]
-    for e in events:
-        e.record()
-    A.dsv4v_tower_forward_profiled(cfg, b, keep, None, x2, ws, events)
-    torch.cuda.synchronize()
-    assert torch.equal(x1, x2)
-    for i in range(0, len(events), 2):
-        assert events[i].elapsed_time(events[i + 1]) > 0.0
+@pytest.mark.parametrize("path", [A.PATH_KERNELS, A.PATH_CHAIN])
+def test_profiled_tower_matches_plain(path):
+    """dsv4v_tower_forward_profiled computes the same tower (bitwise) and records the events of
+    the kernel classes of the launch sequence in use."""
+    A.dsv4v_set_tower_path(path)
+    try:
+        wl = synth.workload(4)
+        inp = synth.draw(wl, n_layers=3)
+        cfg = config_of(wl, n_layers=3)
+        b = A.BatchRef(wl.grids)
+        ws = workspace(cfg, b)
+        layers = upload_layers(inp)
+        keep = [A.block_weights(l) for l in layers]
+        x1, x2 = dev(inp.x), dev(inp.x)
+        A.dsv4v_tower_forward(cfg, b, keep, None, x1, ws)
+        kinds = A.PROFILE_KINDS
+        events = [torch.cuda.Event(enable_timing=True) for _ in range(3 * len(kinds) * 2)]
+        for e in events:
+            e.record()
+        torch.cuda.synchronize()
+        A.dsv4v_tower_forward_profiled(cfg, b, keep, None, x2, ws, events)
+        torch.cuda.synchronize()
+        assert torch.equal(x1, x2)
+        active = ("attention", "chain") if path == A.PATH_CHAIN else ("qkv", "attention", "out", "swiglu", "down")
+        for l in range(3):
+            for k in active:
+                i = (l * len(kinds) + kinds.index(k)) * 2
+                assert events[i].elapsed_time(events[i + 1]) > 0.0
+    finally:
+        A.dsv4v_set_tower_path(A.PATH_AUTO)
 
 
 def test_workload4_tower_aligner(workload4):

@@ -3,6 +3,8 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
+#include <cmath>
 
 #include <mutex>
 #include <unordered_map>
@@ -180,9 +182,85 @@ dsv4v_status check_all(const dsv4v_config* c, const dsv4v_batch* b, Shape& s) {
   return check_batch(b, s);
 }
 
+// ---------------------------------------------------------------------------- chain plan
+// Which launch sequence the bf16 blocks use: one kernel per GEMM, or the persistent chain kernel
+// (chain.cu) that runs the output projection, SwiGLU, down projection and the next block's q|k|v
+// projection in one launch per block.  Automatic choice: the chain for batches of at most
+// kChainMaxRows patches (none at present: measured on B200, the chain does not yet beat one
+// kernel per GEMM at 784 patches).
+std::atomic<int> g_tower_path{DSV4V_PATH_AUTO};
+constexpr int64_t kChainMaxRows = 0;
+
+struct ChainStagePlan {
+  int bn = 0, splits = 1, tiles_n = 0, kb = 0;
+};
+struct ChainPlan {
+  bool use = false;
+  int tiles_m = 0;
+  ChainStagePlan st[4];  // output projection, SwiGLU, down projection, q|k|v projection
+};
+enum { CS_OUT = 0, CS_GATEUP = 1, CS_DOWN = 2, CS_QKV = 3 };
+
+// Estimated cycles of one stage (fitted constants, B200): a 64-deep K block of a 128 x bn tile
+// costs ~390 cycles at bn = 128 (the MMA instruction floor), ~478 at bn = 192 and ~574 at
+// bn = 256 (the rate at which an SM takes in 48 KB of operands); tasks of one stage run in waves
+// over the SMs; a split tile adds its partials' round trip through L2 and the epilogue ~8 cycles
+// per column.
+double chain_stage_cycles(int bn, int kb, int tasks, int splits, int sms) {
+  const double kb_cyc = bn >= 256 ? 574.0 : (bn >= 192 ? 478.0 : 390.0);
+  const int waves = (tasks + sms - 1) / sms;
+  const int kb_per = (kb + splits - 1) / splits;
+  double c = waves * kb_per * kb_cyc + 8.0 * bn;
+  if (splits > 1) c += 1500.0 + (splits - 1) * 6.0 * bn;
+  return c;
+}
+
+ChainStagePlan plan_chain_stage(int stage, const Shape& s, int tiles_m, int sms) {
+  ChainStagePlan best;
+  double best_c = 1e300;
+  const int K = stage == CS_DOWN ? s.F : s.D;
+  const int kb = (K + 63) / 64;
+  const int n_cols = stage == CS_GATEUP ? s.F : s.D;
+  const int bns[2] = {256, 128};
+  for (int bi = 0; bi < (stage == CS_QKV ? 1 : 2); ++bi) {
+    const int bn = stage == CS_QKV ? 192 : bns[bi];
+    const int cols = stage == CS_QKV ? 64 : (stage == CS_GATEUP ? bn / 2 : bn);
+    if (n_cols % cols) continue;
+    const int tiles_n = n_cols / cols;
+    // SwiGLU and the q|k|v projection finish whole tiles; the residual GEMMs may split K.
+    const int max_splits = (stage == CS_OUT || stage == CS_DOWN) ? 4 : 1;
+    for (int sp = 1; sp <= max_splits && sp <= kb; ++sp) {
+      const double c = chain_stage_cycles(bn, kb, tiles_m * tiles_n * sp, sp, sms);
+      if (c < best_c - 1e-9) {
+        best_c = c;
+        best.bn = bn;
+        best.splits = sp;
+        best.tiles_n = tiles_n;
+        best.kb = kb;
+      }
+    }
+  }
+  return best;
+}
+
+ChainPlan make_chain_plan(const Shape& s, int sms) {
+  ChainPlan cp;
+  if (!s.bf16 || s.P <= 0) return cp;
+  const int path = g_tower_path.load();
+  if (path == DSV4V_PATH_KERNELS || (path == DSV4V_PATH_AUTO && s.P > kChainMaxRows)) return cp;
+  if (s.hd != 64 || s.D % 256 || s.F % 128) return cp;
+  cp.tiles_m = static_cast<int>((s.P + 127) / 128);
+  for (int st = 0; st < 4; ++st) cp.st[st] = plan_chain_stage(st, s, cp.tiles_m, sms);
+  for (int st = 0; st < 4; ++st)
+    if (cp.st[st].bn == 0) return ChainPlan{};
+  cp.use = true;
+  return cp;
+}
+
 // ---------------------------------------------------------------------------- workspace
 struct Plans {
   GemmPlan qkv, out, gateup, down, align;
+  ChainPlan chain;
 };
 
 Plans make_plans(const Shape& s, int sms) {
@@ -192,6 +270,7 @@ Plans make_plans(const Shape& s, int sms) {
   p.gateup = plan_gemm(EPI_SWIGLU, static_cast<int>(s.P), s.F, s.D, sms);
   p.down = plan_gemm(EPI_RESID, static_cast<int>(s.P), s.D, s.F, sms);
   p.align = plan_gemm(EPI_STORE, static_cast<int>(s.T), s.E, s.r * s.r * s.D, sms);
+  p.chain = make_chain_plan(s, sms);
   return p;
 }
 
@@ -199,7 +278,17 @@ struct Layout {
   size_t cos, sin, y, qkv, attn, h, partials, counters, asrc, merged, ss1, ss2, total;
   size_t counters_bytes;
   int ss_parts;  // row stride of ss1 / ss2: the most N tiles a residual GEMM can have
+  // chain kernel: fp32 split partials of each stage, and (inside the counters region, which the
+  // first kernel of every call clears) per launch a ticket and per stage and row tile a
+  // finished-tile counter, then per stage the split arrival counters
+  size_t chain_partials[4];
+  int chain_launches;   // launches the counters are laid out for
+  int chain_ctr_off;    // int offset of the chain counters inside the counters region
+  int chain_arr_off[4]; // int offsets of each stage's arrival counters
 };
+
+// Chain counters of launch `l`: [ticket][stage 0 done x tiles_m][stage 1 ...] ... [stage 3].
+inline int chain_launch_ints(const ChainPlan& cp) { return 1 + 4 * cp.tiles_m; }
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -228,7 +317,24 @@ Layout make_layout(const Shape& s, const Plans& pl) {
     }
   }
   l.partials = take(part);
-  l.counters_bytes = up256(static_cast<size_t>(counters) * sizeof(int));
+  int n_ints = counters;
+  if (pl.chain.use) {
+    const ChainPlan& cp = pl.chain;
+    for (int st = 0; st < 4; ++st) {
+      const ChainStagePlan& sp = cp.st[st];
+      l.chain_partials[st] = take(sp.splits > 1 ? static_cast<size_t>(cp.tiles_m) * sp.tiles_n * (sp.splits - 1) *
+                                                          128 * sp.bn * sizeof(float)
+                                                    : 0);
+    }
+    l.chain_launches = std::max(2, s.L + 1);
+    l.chain_ctr_off = counters;
+    n_ints = counters + l.chain_launches * chain_launch_ints(cp);
+    for (int st = 0; st < 4; ++st) {
+      l.chain_arr_off[st] = n_ints;
+      n_ints += cp.st[st].splits > 1 ? cp.tiles_m * cp.st[st].tiles_n : 0;
+    }
+  }
+  l.counters_bytes = up256(static_cast<size_t>(n_ints) * sizeof(int));
   l.counters = take(l.counters_bytes);
   l.asrc = take(static_cast<size_t>(s.T) * s.r * s.r * 4);
   l.ss_parts = s.D / 64 > 0 ? s.D / 64 : 1;
@@ -340,26 +446,19 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   return cuda_status(launch_gemm_tc(epi, plan, g, c.stream));
 }
 
-dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv, void* out) {
-  CUtensorMap tm;
-  if (!bf16_map(qkv, c.s.P, 3 * c.s.D, 128, &tm)) return DSV4V_ERR_CUDA;
-  thread_local AttnSchedule sched;
+// Work items of the attention kernels: images longest first, per image its 128-row tiles in
+// groups of `pair` (item_start, img_row0, img_len in that order).
+void attention_schedule(const dsv4v_batch* b, int pair, int heads_per_item, AttnSchedule& sched) {
   const int n = b->n_images;
   std::vector<int> order(n);
   for (int i = 0; i < n; ++i) order[i] = i;
-  // Longest image first: its CTAs cost the most (cost grows with the key count).
+  // Longest image first: its items cost the most (cost grows with the key count).
   std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
     return b->cu_patches_host[x + 1] - b->cu_patches_host[x] > b->cu_patches_host[y + 1] - b->cu_patches_host[y];
   });
   sched.n_images = n;
-  // Two query tiles per CTA halve the K/V traffic and keep two softmax warps on every SM
-  // sub-partition; one per CTA when pairing would leave SMs idle.
-  int paired = 0;
-  for (int i = 0; i < n; ++i) {
-    const int len = b->cu_patches_host[i + 1] - b->cu_patches_host[i];
-    paired += ((len + 255) / 256) * c.s.H;
-  }
-  sched.pair = paired >= c.dev.sms ? 2 : 1;
+  sched.pair = pair;
+  sched.split = 0;
   int items = 0;
   for (int k = 0; k < n; ++k) {
     const int i = order[k];
@@ -368,11 +467,28 @@ dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv,
     sched.img_row0[k] = b->cu_patches_host[i];
     sched.img_len[k] = len;
     const int qt = (len + 127) / 128;
-    items += ((qt + sched.pair - 1) / sched.pair) * c.s.H;
+    items += ((qt + pair - 1) / pair) * heads_per_item;
   }
   sched.item_start[n] = items;
   sched.n_items = items;
-  return cuda_status(launch_attention_tc(&tm, sched, c.s.H, c.s.D, out, c.dev.err, c.stream));
+}
+
+dsv4v_status attention_bf16(const Ctx& c, const dsv4v_batch* b, const void* qkv, void* out, float* lse = nullptr) {
+  CUtensorMap tm;
+  if (!bf16_map(qkv, c.s.P, 3 * c.s.D, 128, &tm)) return DSV4V_ERR_CUDA;
+  thread_local AttnSchedule sched;
+  // Two query tiles per CTA halve the K/V traffic and keep two softmax warps on every SM
+  // sub-partition; one per CTA when pairing would leave SMs idle.
+  int paired = 0;
+  for (int i = 0; i < b->n_images; ++i) {
+    const int len = b->cu_patches_host[i + 1] - b->cu_patches_host[i];
+    paired += ((len + 255) / 256) * c.s.H;
+  }
+  attention_schedule(b, paired >= c.dev.sms ? 2 : 1, c.s.H, sched);
+  // Unpaired items (fewer than the SMs): both softmax warpgroups of a CTA work on its query tile,
+  // each on every other key tile, so that each SM sub-partition runs two softmax warps.
+  sched.split = sched.pair == 1 ? 1 : 0;
+  return cuda_status(launch_attention_tc(&tm, sched, c.s.H, c.s.D, out, c.dev.err, c.stream, lse, c.s.P));
 }
 
 // One block on the bf16 path.  The two RMSNorms are folded into the GEMMs that consume them:
@@ -444,6 +560,155 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   DSV4V_TRY(record(ev, DSV4V_PROFILE_DOWN, 0, c.stream));
   DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x, nullptr, nullptr, d));
   return record(ev, DSV4V_PROFILE_DOWN, 1, c.stream);
+}
+
+// ---------------------------------------------------------------------------- chain path
+// Tensor maps of one chain launch, shared between stages that use the same tensor and box.
+struct ChainBuilder {
+  ChainParams p{};
+  const void* key_ptr[kChainMaxMaps] = {};
+  int key_box[kChainMaxMaps] = {};
+  bool ok = true;
+  int map(const void* ptr, int64_t rows, int64_t cols, int box) {
+    for (int i = 0; i < p.n_maps; ++i)
+      if (key_ptr[i] == ptr && key_box[i] == box) return i;
+    if (p.n_maps >= kChainMaxMaps || !bf16_map(ptr, rows, cols, box, &p.maps[p.n_maps])) {
+      ok = false;
+      return 0;
+    }
+    key_ptr[p.n_maps] = ptr;
+    key_box[p.n_maps] = box;
+    return p.n_maps++;
+  }
+};
+
+// One chain launch: the output projection, SwiGLU and down projection of block `cur` (NULL:
+// none) followed by the q|k|v projection of block `next` (NULL: none).  `launch` selects this
+// launch's ticket and row-tile counters.  next_norm1_w: the norm1 weight of `next`, which the
+// down projection's epilogue prepares (NULL when `cur` is the last block); the q|k|v projection
+// of a launch without `cur` takes its norm operand from k_norm_prep (whole row sum in slot 0).
+dsv4v_status run_chain(const Ctx& c, int launch, const dsv4v_block_weights* cur, const dsv4v_block_weights* next,
+                       const float* next_norm1_w, const float* cos, const float* sin, void* x) {
+  const Shape& s = c.s;
+  const ChainPlan& cp = c.plans.chain;
+  if (launch >= c.lay.chain_launches) return DSV4V_ERR_UNSUPPORTED;
+  void* xw = c.at<void>(c.lay.y);
+  void* qkv = c.at<void>(c.lay.qkv);
+  void* attn = c.at<void>(c.lay.attn);
+  void* h = c.at<void>(c.lay.h);
+  float* ss1 = c.at<float>(c.lay.ss1);
+  float* ss2 = c.at<float>(c.lay.ss2);
+  int* ctr = c.at<int>(c.lay.counters);
+  int* base = ctr + c.lay.chain_ctr_off + launch * chain_launch_ints(cp);
+  ChainBuilder b;
+  ChainParams& p = b.p;
+  p.ticket = base;
+  p.err = c.dev.err;
+  p.norm_inv_d = 1.0f / static_cast<float>(s.D);
+  p.norm_eps = c.eps;
+  int task = 0;
+  auto stage = [&](int cs) -> ChainStage& {
+    ChainStage& d = p.st[p.n_stages++];
+    d = ChainStage{};
+    const ChainStagePlan& sp = cp.st[cs];
+    d.bn = sp.bn;
+    d.kb_total = sp.kb;
+    d.tiles_m = cp.tiles_m;
+    d.tiles_n = sp.tiles_n;
+    d.splits = sp.splits;
+    d.task_base = task;
+    task += d.tiles_m * d.tiles_n * d.splits;
+    d.dep_stage = -1;
+    d.map_b2 = -1;
+    d.map_xw = -1;
+    d.M = static_cast<int>(s.P);
+    d.D = s.D;
+    d.done = base + 1 + cs * cp.tiles_m;
+    if (sp.splits > 1) {
+      d.partials = c.at<float>(c.lay.chain_partials[cs]);
+      d.arrivals = ctr + c.lay.chain_arr_off[cs];
+    }
+    return d;
+  };
+  if (cur) {
+    ChainStage& o = stage(CS_OUT);
+    o.epi = CHAIN_RESID;
+    o.map_a = b.map(attn, s.P, s.D, 128);
+    o.map_b = b.map(cur->wo, s.D, s.D, o.bn);
+    o.map_out = b.map(x, s.P, s.D, 32);
+    o.map_xw = b.map(xw, s.P, s.D, 32);
+    o.resid = x;
+    o.ldr = s.D;
+    o.xw_w = cur->norm2_w;
+    o.ss_out = ss2;
+    o.ss_parts = c.lay.ss_parts;
+    ChainStage& g = stage(CS_GATEUP);
+    g.epi = CHAIN_SWIGLU;
+    g.dep_stage = 0;
+    g.dep_target = p.st[0].tiles_n;
+    g.map_a = b.map(xw, s.P, s.D, 128);
+    g.map_b = b.map(cur->w_gate, s.F, s.D, g.bn / 2);
+    g.map_b2 = b.map(cur->w_up, s.F, s.D, g.bn / 2);
+    g.map_out = b.map(h, s.P, s.F, 32);
+    g.norm_ss = ss2;
+    g.norm_parts = p.st[0].tiles_n;
+    g.norm_stride = c.lay.ss_parts;
+    ChainStage& dn = stage(CS_DOWN);
+    dn.epi = CHAIN_RESID;
+    dn.dep_stage = 1;
+    dn.dep_target = p.st[1].tiles_n;
+    dn.map_a = b.map(h, s.P, s.F, 128);
+    dn.map_b = b.map(cur->w_down, s.D, s.F, dn.bn);
+    dn.map_out = b.map(x, s.P, s.D, 32);
+    dn.resid = x;
+    dn.ldr = s.D;
+    if (next_norm1_w) {
+      dn.map_xw = b.map(xw, s.P, s.D, 32);
+      dn.xw_w = next_norm1_w;
+      dn.ss_out = ss1;
+      dn.ss_parts = c.lay.ss_parts;
+    }
+  }
+  if (next) {
+    ChainStage& q = stage(CS_QKV);
+    q.epi = CHAIN_QKV_HEADS;
+    q.dep_stage = cur ? 2 : -1;
+    q.dep_target = cur ? p.st[2].tiles_n : 0;
+    q.map_a = b.map(xw, s.P, s.D, 128);
+    q.map_b = b.map(next->wqkv, 3 * s.D, s.D, 64);
+    q.map_out = b.map(qkv, s.P, 3 * s.D, 32);
+    q.cos = cos;
+    q.sin = sin;
+    q.norm_ss = ss1;
+    q.norm_parts = cur ? p.st[2].tiles_n : 1;
+    q.norm_stride = c.lay.ss_parts;
+  }
+  if (!b.ok) return DSV4V_ERR_CUDA;
+  p.total_tasks = task;
+  return cuda_status(launch_chain(p, c.dev.sms, c.stream));
+}
+
+// Blocks [0, L) on the chain path: the first norm operand, layer 0's q|k|v projection, then per
+// layer attention and one chain launch (layer l's remaining GEMMs and layer l + 1's q|k|v).
+// The first kernel clears every counter of the call.  ev: DSV4V_PROFILE_* event pairs per layer.
+dsv4v_status blocks_chain(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_weights* layers, int L,
+                          const float* cos, const float* sin, void* x, void* const* ev) {
+  const Shape& s = c.s;
+  DSV4V_TRY(cuda_status(launch_norm_prep(x, layers[0].norm1_w, c.at<void>(c.lay.y), c.at<float>(c.lay.ss1),
+                                         c.lay.ss_parts, s.P, s.D, c.stream, c.at<int>(c.lay.counters),
+                                         static_cast<int>(c.lay.counters_bytes / sizeof(int)))));
+  DSV4V_TRY(run_chain(c, 0, nullptr, &layers[0], nullptr, cos, sin, x));
+  for (int l = 0; l < L; ++l) {
+    void* const* e = ev ? ev + static_cast<size_t>(l) * DSV4V_PROFILE_KINDS * 2 : nullptr;
+    DSV4V_TRY(record(e, DSV4V_PROFILE_ATTENTION, 0, c.stream));
+    DSV4V_TRY(attention_bf16(c, b, c.at<void>(c.lay.qkv), c.at<void>(c.lay.attn)));
+    DSV4V_TRY(record(e, DSV4V_PROFILE_ATTENTION, 1, c.stream));
+    DSV4V_TRY(record(e, DSV4V_PROFILE_CHAIN, 0, c.stream));
+    DSV4V_TRY(run_chain(c, l + 1, &layers[l], l + 1 < L ? &layers[l + 1] : nullptr,
+                        l + 1 < L ? layers[l + 1].norm1_w : nullptr, cos, sin, x));
+    DSV4V_TRY(record(e, DSV4V_PROFILE_CHAIN, 1, c.stream));
+  }
+  return DSV4V_OK;
 }
 
 // ---------------------------------------------------------------------------- fp32 steps
@@ -563,6 +828,19 @@ const char* dsv4v_status_string(dsv4v_status s) {
   return "unknown status";
 }
 
+dsv4v_status dsv4v_set_tower_path(int path) {
+  if (path != DSV4V_PATH_AUTO && path != DSV4V_PATH_KERNELS && path != DSV4V_PATH_CHAIN)
+    return DSV4V_ERR_INVALID_ARG;
+  g_tower_path.store(path);
+  return DSV4V_OK;
+}
+
+int dsv4v_tower_path(const dsv4v_config* cfg, const dsv4v_batch* batch) {
+  Shape s;
+  if (check_all(cfg, batch, s) != DSV4V_OK) return -1;
+  return make_chain_plan(s, planning_sms()).use ? DSV4V_PATH_CHAIN : DSV4V_PATH_KERNELS;
+}
+
 size_t dsv4v_workspace_size(const dsv4v_config* cfg, const dsv4v_batch* batch) {
   Shape s;
   if (check_all(cfg, batch, s) != DSV4V_OK) return 0;
@@ -591,6 +869,7 @@ dsv4v_status dsv4v_block_forward(const dsv4v_config* cfg, const dsv4v_batch* bat
   DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
   if (!weights_ok(w) || !cos || !sin || !x_inout || !aligned16(x_inout) || !aligned16(cos) || !aligned16(sin))
     return DSV4V_ERR_INVALID_ARG;
+  if (c.s.bf16 && c.plans.chain.use) return blocks_chain(c, batch, w, 1, cos, sin, x_inout, nullptr);
   return c.s.bf16 ? block_bf16(c, batch, w, cos, sin, x_inout, true, nullptr)
                    : block_f32(c, batch, w, cos, sin, x_inout);
 }
@@ -607,11 +886,15 @@ static dsv4v_status tower_impl(const dsv4v_config* cfg, const dsv4v_batch* batch
   float* cos = c.at<float>(c.lay.cos);
   float* sin = c.at<float>(c.lay.sin);
   DSV4V_TRY(rope_table(c, batch, cos, sin));
+  if (c.s.bf16 && c.plans.chain.use && c.s.L > 0) {
+    DSV4V_TRY(blocks_chain(c, batch, layers, c.s.L, cos, sin, x_inout, events));
+  } else {
   for (int l = 0; l < c.s.L; ++l)
     DSV4V_TRY(c.s.bf16 ? block_bf16(c, batch, &layers[l], cos, sin, x_inout, l == 0,
                                     l + 1 < c.s.L ? layers[l + 1].norm1_w : nullptr,
                                     events ? events + static_cast<size_t>(l) * DSV4V_PROFILE_KINDS * 2 : nullptr)
                        : block_f32(c, batch, &layers[l], cos, sin, x_inout));
+  }
   if (final_norm_w)
     DSV4V_TRY(cuda_status(launch_rmsnorm(c.s.bf16, x_inout, final_norm_w, x_inout, c.s.P, c.s.D, c.eps, c.stream)));
   return DSV4V_OK;
@@ -1065,17 +1348,21 @@ dsv4v_status transpose(const Ctx& c, const void* in, int64_t rows, int cols, voi
   return cuda_status(launch_transpose_bf16(in, rows, cols, cols, out, ld_out, col0, c.stream));
 }
 
-int attention_blocks(const dsv4v_batch* b) {
-  int64_t n = 0;
-  for (int i = 0; i < b->n_images; ++i) n += (b->cu_patches_host[i + 1] - b->cu_patches_host[i] + 63) / 64;
-  return static_cast<int>(n);
-}
 
+// Attention backward on tcgen05.  lse_ready: bl.lse already holds the forward's per-row
+// log-sum-exp ([H, P], written by the forward recompute); otherwise the forward runs once more
+// into scratch to produce it.
 dsv4v_status attention_bwd(const Ctx& c, const BwdLayout& bl, const dsv4v_batch* b, const void* qkv, const void* out,
-                           const void* dout, void* dqkv) {
-  return cuda_status(launch_attention_bwd(qkv, out, dout, dqkv, c.at<float>(bl.lse), c.at<float>(bl.rowdot),
-                                          b->cu_patches_dev, b->n_images, attention_blocks(b), c.s.D, c.s.H,
-                                          c.stream));
+                           const void* dout, void* dqkv, bool lse_ready) {
+  if (!lse_ready) DSV4V_TRY(attention_bf16(c, b, qkv, c.at<void>(c.lay.attn), c.at<float>(bl.lse)));
+  CUtensorMap tm_qkv, tm_do;
+  if (!bf16_map(qkv, c.s.P, 3 * c.s.D, 128, &tm_qkv) || !bf16_map(dout, c.s.P, c.s.D, 128, &tm_do))
+    return DSV4V_ERR_CUDA;
+  thread_local AttnSchedule sched;
+  attention_schedule(b, 1, 1, sched);
+  return cuda_status(launch_attention_bwd_tc(&tm_qkv, &tm_do, sched, sched, out, dout, c.at<float>(bl.lse),
+                                             c.at<float>(bl.rowdot), c.s.P, dqkv, c.s.P, c.s.H, c.s.D, c.dev.err,
+                                             c.stream));
 }
 
 dsv4v_status rmsnorm_bwd(const Ctx& c, const BwdLayout& bl, const void* x, const float* w, const void* dy,
@@ -1126,7 +1413,7 @@ dsv4v_status block_backward_bf16(const Ctx& c, const BwdLayout& bl, const dsv4v_
   DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm1_w, y1, P, D, c.eps, c.stream)));
   DSV4V_TRY(reset_counters(c));
   DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, y1, P, D, w->wqkv, nullptr, 3 * D, qkv, nullptr, cos, sin));
-  DSV4V_TRY(attention_bf16(c, batch, qkv, att));
+  DSV4V_TRY(attention_bf16(c, batch, qkv, att, c.at<float>(bl.lse)));
   DSV4V_TRY(cuda_status(cudaMemcpyAsync(x2, x, static_cast<size_t>(P) * D * 2, cudaMemcpyDeviceToDevice, c.stream)));
   DSV4V_TRY(reset_counters(c));
   DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, att, P, D, w->wo, nullptr, D, x2, x2));
@@ -1153,7 +1440,7 @@ dsv4v_status block_backward_bf16(const Ctx& c, const BwdLayout& bl, const dsv4v_
   DSV4V_TRY(transpose(c, att, P, D, c.at<void>(bl.att_t), ldp));
   DSV4V_TRY(gemm_store(c, c.at<void>(bl.dx2_t), D, static_cast<int>(P), ldp, c.at<void>(bl.att_t), ldp, D, gr->wo));
   // attention, rotation, fused projection
-  DSV4V_TRY(attention_bwd(c, bl, batch, qkv, att, datt, dqkv));
+  DSV4V_TRY(attention_bwd(c, bl, batch, qkv, att, datt, dqkv, true));
   DSV4V_TRY(cuda_status(launch_rotary_bwd(dqkv, cos, sin, P, D, s.hd, c.dev.sms, c.stream)));
   DSV4V_TRY(gemm_store(c, dqkv, P, 3 * D, 0, c.at<void>(bl.wqkv_t), 0, D, dy1));
   DSV4V_TRY(transpose(c, dqkv, P, 3 * D, c.at<void>(bl.dqkv_t), ldp));
@@ -1182,7 +1469,7 @@ dsv4v_status dsv4v_attention_backward(const dsv4v_config* cfg, const dsv4v_batch
   DSV4V_TRY(bwd_prepare(cfg, batch, workspace, ws_bytes, stream, c, bl));
   for (const void* p : {qkv, out, d_out, static_cast<const void*>(dqkv)})
     if (!p || !aligned16(p)) return DSV4V_ERR_INVALID_ARG;
-  return attention_bwd(c, bl, batch, qkv, out, d_out, dqkv);
+  return attention_bwd(c, bl, batch, qkv, out, d_out, dqkv, false);
 }
 
 dsv4v_status dsv4v_rmsnorm_backward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x, const float* w,

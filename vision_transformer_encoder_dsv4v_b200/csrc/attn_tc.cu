@@ -41,7 +41,8 @@ constexpr int OFF_Q = 0;               // Q_A, Q_B
 constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
 constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
-constexpr int SMEM_BYTES = 1024 + OFF_BAR + 512;
+constexpr int OFF_XCHG = OFF_BAR + 512;  // split mode: the second warpgroup's row max and sum (128 x 2 floats)
+constexpr int SMEM_BYTES = 1024 + OFF_XCHG + 1024;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kFirstSoftmaxWarp = 4;
 constexpr int kRegsControl = 56;    // warpgroup 0 after setmaxnreg
@@ -63,8 +64,11 @@ __host__ __device__ constexpr bool poly_pair(int i) {
 
 struct Params {
   int n_heads, vision_dim, pair;
+  int split;  // one query tile per item: its key tiles alternate between the two warpgroups
   float scale_log2;
   __nv_bfloat16* out;
+  float* lse;       // optional [H, lse_ld]: log2 of each row's softmax denominator, in the units of
+  int64_t lse_ld;   // s * scale_log2 (so that P = 2^(s scale_log2 - lse)); NULL: not written
   uint32_t* err;
 };
 
@@ -128,60 +132,6 @@ __device__ __forceinline__ void ex2_poly2(float x0, float x1, float& y0, float& 
   y1 = x1 < -125.0f ? 0.0f : __int_as_float(__float_as_int(q1) + static_cast<int>(n1 << 23));
 }
 
-// D[tmem] (+)= A[tmem] * B[smem], bf16 inputs, fp32 accumulate; A holds M rows in TMEM lanes
-// with two K elements per 32-bit column.  One thread issues.
-__device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Starts loading N x 32 columns of this thread's lane (complete after tmem_ld_wait_pin).
-template <int N>
-__device__ __forceinline__ void tmem_ld_issue(uint32_t taddr, uint32_t* r) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) tmem_ld32(taddr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * i));
-}
-
-// Waits for this thread's TMEM loads, then pins N x 32 registers so that no use of them can be
-// scheduled before the wait.
-template <int N>
-__device__ __forceinline__ void tmem_ld_wait_pin(uint32_t* r) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32 * N; ++i) asm volatile("" : "+r"(r[i]));
-}
-
-// Loads N x 32 columns of this thread's lane with one wait, then pins the registers so that no
-// use of them can be scheduled before the wait.
-template <int N>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) tmem_ld32(taddr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * i));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32 * N; ++i) asm volatile("" : "+r"(r[i]));
-}
-
 template <int R>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
@@ -236,16 +186,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tiles = min(p.pair, n_qt - q_tile);  // 1 or 2 query tiles in this item
   const int n_kv = (len + TK - 1) / TK;
   const int q_row = row0 + q_tile * TQ;
+  // Split mode: one query tile; issuer/warpgroup x takes key tiles x, x + 2, x + 4, ... with its
+  // own S, P and O in TMEM and its own running max and sum, and the two partial results are
+  // combined at the end.  Otherwise group x owns query tile x and every key tile.
+  const bool split = p.split != 0 && n_tiles == 1;
+  const int n_groups = split ? 2 : n_tiles;
+  const int kv_step = split ? 2 : 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], n_tiles);
+      mbar_init(&k_empty[s], split ? 1 : n_tiles);  // released by every issuer that reads the slot
     }
     for (int s = 0; s < VS; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], n_tiles);
+      mbar_init(&v_empty[s], split ? 1 : n_tiles);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -302,15 +258,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = (issued_v > VS ? issued_v - VS : 0); t < issued_v; ++t)
         mbar_wait(&v_full[t % VS], (t / VS) & 1, &never, p.err, kErrTimeoutProducer);
     }
-  } else if (warp - 1 < n_tiles) {
+  } else if (warp - 1 < n_groups) {
     // ------------------------------------------------------------------ MMA issuers
-    // Warp 1 issues the products of tile A, warp 2 those of tile B, so that neither waits for
-    // the other's softmax; the K/V slots are released by one commit from each.
+    // Warp 1 issues the products of group A, warp 2 those of group B, so that neither waits for
+    // the other's softmax; the K/V slots are released by one commit from each issuer that
+    // reads them.
     if (lane == 0) {
       const int x = warp - 1;
       constexpr uint32_t idesc_s = idesc_bf16(TQ, TK, false);
       constexpr uint32_t idesc_pv = idesc_bf16(TQ, HD, true);  // V is MN-major (hd contiguous)
-      const uint64_t qd = sdesc_sw128(smem_u32(smem + OFF_Q + x * TILE_BYTES), 16, 1024);
+      const uint64_t qd = sdesc_sw128(smem_u32(smem + OFF_Q + (split ? 0 : x) * TILE_BYTES), 16, 1024);
       const uint32_t d_s = tmem_base + T_S + static_cast<uint32_t>(x * TK);
       const uint32_t d_o = tmem_base + T_O + static_cast<uint32_t>(x * HD);
       const uint32_t a_p = tmem_base + T_P + static_cast<uint32_t>(x * (TK / 2));
@@ -321,38 +278,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&s_full[x]);
         umma_commit(&k_empty[j % KS]);
       };
-      auto issue_pv = [&](int j) {
+      // it: this group's iteration (its it-th key tile, global key tile j = x0 + it * kv_step).
+      auto issue_pv = [&](int j, int it) {
         const uint32_t v_addr = smem_u32(smem + OFF_V + (j % VS) * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < TK / 16; ++kk) {
           // P: 16 keys = 8 TMEM columns; V: 16 keys = two 8-row groups of 1024 B.
           const uint64_t vd = sdesc_sw128(v_addr + kk * 2048, TILE_BYTES, 1024);
-          umma_bf16_tmem_a(d_o, a_p + kk * 8, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(d_o, a_p + kk * 8, vd, idesc_pv, (it > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[x]);
         umma_commit(&v_empty[j % VS]);
       };
+      const int x0 = split ? x : 0;
       bool ok = mbar_wait(q_full, 0, abort_flag, p.err, kErrTimeoutMma);
-      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, p.err, kErrTimeoutMma);
-      if (ok) {
-        tc_fence_after_sync();
-        issue_s(0);
+      if (ok && x0 < n_kv) {
+        ok = mbar_wait(&k_full[x0 % KS], (x0 / KS) & 1, abort_flag, p.err, kErrTimeoutMma);
+        if (ok) {
+          tc_fence_after_sync();
+          issue_s(x0);
+        }
       }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv) {
-          // S(j+1) as soon as the softmax has S(j) in registers.
-          const int t = j + 1;
+      for (int j = x0, it = 0; j < n_kv && ok; j += kv_step, ++it) {
+        if (j + kv_step < n_kv) {
+          // S of the next key tile as soon as the softmax has this one's in registers.
+          const int t = j + kv_step;
           ok = mbar_wait(&k_full[t % KS], (t / KS) & 1, abort_flag, p.err, kErrTimeoutMma) &&
-               mbar_wait(&s_free[x], j & 1, abort_flag, p.err, kErrTimeoutMma);
+               mbar_wait(&s_free[x], it & 1, abort_flag, p.err, kErrTimeoutMma);
           if (!ok) break;
           tc_fence_after_sync();
           issue_s(t);
         }
         ok = mbar_wait(&v_full[j % VS], (j / VS) & 1, abort_flag, p.err, kErrTimeoutMma) &&
-             mbar_wait(&p_full[x], j & 1, abort_flag, p.err, kErrTimeoutMma);
+             mbar_wait(&p_full[x], it & 1, abort_flag, p.err, kErrTimeoutMma);
         if (!ok) break;
         tc_fence_after_sync();
-        issue_pv(j);
+        issue_pv(j, it);
       }
       umma_commit(&mma_done[x]);
       volatile int never = 0;
@@ -360,9 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
-  } else if (regs_inc<kRegsSoftmax>(), (warp - kFirstSoftmaxWarp) / 4 < n_tiles) {
+  } else if (regs_inc<kRegsSoftmax>(), (warp - kFirstSoftmaxWarp) / 4 < n_groups) {
     // ------------------------------------------------------------------ softmax + output
-    const int x = (warp - kFirstSoftmaxWarp) >> 2;  // query tile of this warpgroup
+    const int x = (warp - kFirstSoftmaxWarp) >> 2;  // group of this warpgroup
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
@@ -372,7 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY, l_run = 0.0f;
     bool ok = true;
     grid_dependency_wait();
-    for (int j = 0; j < n_kv; ++j) {
+    const int x0 = split ? x : 0;
+    int n_it = 0;  // key tiles this group processed
+    for (int kt = x0; kt < n_kv; kt += kv_step, ++n_it) {
+      const int j = n_it;  // this group's iteration (barrier phases)
       bool got = mbar_wait(&s_full[x], j & 1, abort_flag, p.err, kErrTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
@@ -383,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t s[TK];
       tmem_ld_cols<2>(t_s, s);
       tmem_ld_issue<2>(t_s + 64, s + 64);
-      const int valid = len - j * TK;
+      const int valid = len - kt * TK;
       if (valid < TK / 2) {
 #pragma unroll
         for (int c = 0; c < TK / 2; ++c)
@@ -468,17 +432,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before_sync();
       mbar_arrive(&p_full[x]);
     }
-    if (ok && n_kv > 0) {
-      const bool got = mbar_wait(&pv_done[x], (n_kv - 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
+    if (ok && n_it > 0) {
+      const bool got = mbar_wait(&pv_done[x], (n_it - 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
       ok = __all_sync(0xffffffffu, got);
+    }
+    float* xchg = reinterpret_cast<float*>(smem + OFF_XCHG);
+    if (split) {
+      // The second group hands its row max and sum to the first through shared memory; its O
+      // stays in TMEM, where the first group's thread of the same row (same TMEM lane) reads it.
+      if (x == 1) {
+        xchg[r] = ok ? m_used : -INFINITY;
+        xchg[128 + r] = ok && n_it > 0 ? l_run : 0.0f;
+        tc_fence_before_sync();
+      }
+      named_barrier_sync(3, 256);
+      if (x == 1) ok = false;  // the first group writes the output
+      else tc_fence_after_sync();
     }
     if (ok) {
       tc_fence_after_sync();
       uint32_t o[HD];
       tmem_ld_cols<HD / 32>(t_o, o);
-      const int qi = (q_tile + x) * TQ + r;
+      float l_tot = l_run;
+      if (split) {
+        const float m_b = xchg[r], l_b = xchg[128 + r];
+        if (l_b > 0.0f) {
+          // O = O_A 2^(m_A - m) + O_B 2^(m_B - m), l = l_A 2^(m_A - m) + l_B 2^(m_B - m)
+          const float m = fmaxf(m_used, m_b);
+          const float fa = n_it > 0 ? ex2_mufu(m_used - m) : 0.0f, fb = ex2_mufu(m_b - m);
+          uint32_t ob[HD];
+          tmem_ld_cols<HD / 32>(t_lane + T_O + static_cast<uint32_t>(HD), ob);
+#pragma unroll
+          for (int c = 0; c < HD; ++c)
+            o[c] = __float_as_uint((n_it > 0 ? __uint_as_float(o[c]) * fa : 0.0f) + __uint_as_float(ob[c]) * fb);
+          l_tot = (n_it > 0 ? l_run * fa : 0.0f) + l_b * fb;
+        }
+      }
+      const int qi = (q_tile + (split ? 0 : x)) * TQ + r;
+      if (qi < len && p.lse) {
+        // reference max of O's accumulation: the combined max in split mode, else m_used
+        float m_ref = m_used;
+        if (split) {
+          const float m_b = xchg[r], l_b = xchg[128 + r];
+          if (l_b > 0.0f) m_ref = fmaxf(m_used, m_b);
+        }
+        p.lse[static_cast<int64_t>(head) * p.lse_ld + row0 + qi] = m_ref + __log2f(l_tot);
+      }
       if (qi < len) {
-        const float inv_l = 1.0f / l_run;
+        const float inv_l = 1.0f / l_tot;
         uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + qi) * p.vision_dim + head * HD);
 #pragma unroll
         for (int q = 0; q < HD / 8; ++q) {
@@ -512,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& sched, int n_heads, int vision_dim,
-                                void* out, uint32_t* err, cudaStream_t s) {
+                                void* out, uint32_t* err, cudaStream_t s, float* lse, int64_t lse_ld) {
   static unsigned long long attr_set_mask = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -534,8 +535,11 @@ cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& s
   p.n_heads = n_heads;
   p.vision_dim = vision_dim;
   p.pair = sched.pair;
+  p.split = sched.split;
   p.scale_log2 = 1.4426950408889634f / 8.0f;  // log2(e) / sqrt(64)
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.lse_ld = lse_ld;
   p.err = err;
   return launch_pdl(k_attn_tc, dim3(sched.n_items), dim3(kThreads), SMEM_BYTES, s, *tm_qkv, sched, p);
 }

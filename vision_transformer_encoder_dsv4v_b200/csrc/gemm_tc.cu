@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tile_util.cuh"
 
 namespace dsv4v {
 
@@ -112,55 +113,7 @@ struct SegmentWalker {
   }
 };
 
-// gelu(z) = z (1 + erf(z / sqrt 2)) / 2, the exact (erf) form.
-__device__ __forceinline__ float gelu(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
 
-// silu(z) = z / (1 + e^-z) = (z / 2) (1 + tanh(z / 2)): one MUFU op per element, ample for a bf16
-// result.
-__device__ __forceinline__ float silu(float z) {
-  const float h = 0.5f * z;
-  return fmaf(h, tanh_approx(h), h);
-}
-
-// Output staging of one epilogue warp: two boxes of 32 rows x 128 bytes (64 bf16 columns) in
-// the 128-byte-swizzled layout of the output tensor maps; lane i owns row i of a box.  Each box
-// is written to global memory by one TMA store; a box is reused only after the store issued
-// from it two stores ago has finished reading it.
-struct Stager {
-  uint8_t* base;
-  int lane, n;
-  __device__ __forceinline__ uint8_t* acquire() {
-    if (lane == 0 && n >= 2) bulk_wait_read_1();
-    __syncwarp();
-    return base + (n & 1) * 4096;
-  }
-  // Both boxes, once no earlier store still reads either.
-  __device__ __forceinline__ void acquire_both(uint8_t*& b0, uint8_t*& b1) {
-    if (lane == 0 && n >= 1) bulk_wait_read_0();
-    __syncwarp();
-    b0 = base + (n & 1) * 4096;
-    b1 = base + ((n + 1) & 1) * 4096;
-  }
-  // 16-byte chunk j (0..7) of this lane's row.
-  __device__ __forceinline__ void put(uint8_t* box, int j, uint4 v) {
-    *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
-  }
-  // Stores the box to rows [y, y + 32) and columns [x, x + 64) of `map` (TMA clips rows past
-  // the end of the tensor; a box entirely past it is skipped).
-  __device__ __forceinline__ void store(uint8_t* box, const CUtensorMap* map, int x, int y, int rows) {
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0 && y < rows) {
-      tma_store_2d(map, box, x, y);
-      bulk_commit();
-    }
-    ++n;
-  }
-  __device__ __forceinline__ void drain() {
-    if (lane == 0) bulk_wait_all();
-    __syncwarp();
-  }
-};
 
 // Epilogue math of one 64-column accumulator group v[0..63] of output row `row`; the result
 // goes to the warp's staging box (the caller stores it).
@@ -290,13 +243,6 @@ __device__ __forceinline__ void group_chunks(int g, int& c0, int& c1) {
   }
 }
 
-__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
-  float4 v;
-  asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "l"(p));
-  return v;
-}
 
 // Scratch slot of CTA c (a contributor writes at most one partial: its first segment).
 // Layout [BN / 4][128 rows][4]: a warp's 32 rows of one 4-column group are 512 contiguous bytes.
@@ -305,30 +251,7 @@ __device__ __forceinline__ float* partial_slot(const Params& p, int c) {
   return p.partials + static_cast<size_t>(c) * BM * BN;
 }
 
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 
-// Bounded wait until *ctr reaches `target` (the other contributors of a split tile).
-__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort_flag, uint32_t* err) {
-  uint64_t t0 = 0;
-  for (uint32_t i = 0;; ++i) {
-    if (ld_acquire_gpu(ctr) >= target) return true;
-    if ((i & 63u) == 63u) {
-      if (*abort_flag) return false;
-      const uint64_t now = global_timer_ns();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > kWaitLimitNs) {
-        atomicCAS(err, 0u, static_cast<uint32_t>(kErrTimeoutEpilogue));
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
 
 template <int BN, int EPI, bool PAIR, int KS>
 __global__ void __launch_bounds__(192, 1)

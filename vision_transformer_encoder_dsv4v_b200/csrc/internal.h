@@ -70,6 +70,46 @@ struct GemmArgs {
 
 cudaError_t launch_gemm_tc(int epi, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
 
+// ---------------------------------------------------------------------------- chain kernel
+// Several dependent GEMM stages of the block in one persistent launch (chain.cu).  Stage tiles
+// are 128 rows x bn columns, K in 64-element blocks, optionally split along K; a stage waits per
+// 128-row tile for an earlier stage of the same launch (dep_stage), or for the kernels before
+// the launch (dep_stage < 0).
+constexpr int kChainMaxStages = 4;
+constexpr int kChainMaxMaps = 20;
+enum ChainEpi : int {
+  CHAIN_RESID = 0,      // out = resid + acc; optionally xw = bf16(out * xw_w) and row sums of out^2
+  CHAIN_SWIGLU = 1,     // out = silu(r acc_gate) * (r acc_up); B = gate rows, B2 = up rows (bn / 2 each)
+  CHAIN_QKV_HEADS = 2,  // bn = 192: the q, k, v rows of head n; rows scaled by r, q and k rotated
+};
+struct ChainStage {
+  int epi, bn, kb_total, tiles_m, tiles_n, splits, task_base;
+  int dep_stage, dep_target;                   // counters of an earlier stage of the launch (-1: none)
+  int map_a, map_b, map_b2, map_out, map_xw;   // indices into ChainParams::maps (-1: unused)
+  int M, D;                                    // rows; vision_dim (head-blocked q|k|v output columns)
+  const void* resid;                           // CHAIN_RESID: bf16 residual rows, row stride ldr
+  int ldr;
+  const float* cos;                            // CHAIN_QKV_HEADS: rotation tables [M, 32]
+  const float* sin;
+  const float* norm_ss;                        // folded norm, consumer side (NULL: r = 1)
+  int norm_parts, norm_stride;
+  const float* xw_w;                           // folded norm, producer side (map_xw >= 0)
+  float* ss_out;
+  int ss_parts;
+  float* partials;                             // splits > 1: [tiles][splits - 1][128 * bn] fp32
+  int* arrivals;                               // splits > 1: [tiles], zero between launches
+  int* done;                                   // [tiles_m]: finished tiles per row tile, zero before the launch
+};
+struct ChainParams {
+  CUtensorMap maps[kChainMaxMaps];
+  ChainStage st[kChainMaxStages];
+  int n_stages, n_maps, total_tasks;
+  float norm_inv_d, norm_eps;
+  int* ticket;  // zero before the launch
+  uint32_t* err;
+};
+cudaError_t launch_chain(const ChainParams& p, int grid, cudaStream_t s);
+
 // ---------------------------------------------------------------------------- attention
 constexpr int kMaxImages = 1024;
 
@@ -81,13 +121,24 @@ struct AttnSchedule {
   int n_images;
   int n_items;
   int pair;
+  int split;  // pair == 1 only: the two softmax warpgroups of a CTA share its query tile's key tiles
   int item_start[kMaxImages + 1];
   int img_row0[kMaxImages];
   int img_len[kMaxImages];
 };
 
+// lse (optional, [n_heads, lse_ld] fp32): per row and head, log2 of the softmax denominator in
+// the units of the scaled scores, P = 2^(q.k log2(e) / sqrt(hd) - lse).
 cudaError_t launch_attention_tc(const CUtensorMap* tm_qkv, const AttnSchedule& sched, int n_heads, int vision_dim,
-                                void* out, uint32_t* err, cudaStream_t s);
+                                void* out, uint32_t* err, cudaStream_t s, float* lse = nullptr, int64_t lse_ld = 0);
+
+// Attention backward on tcgen05 (attn_bwd_tc.cu): rowdot[h, p] = rowsum(dout * out) per head,
+// then dK/dV (one CTA per key tile and head, kv_sched) and dQ (one CTA per query tile and head,
+// q_sched) into dqkv [P, 3D].  lse / rowdot: [H, lse_ld] fp32, lse from launch_attention_tc.
+cudaError_t launch_attention_bwd_tc(const CUtensorMap* tm_qkv, const CUtensorMap* tm_do, const AttnSchedule& kv_sched,
+                                    const AttnSchedule& q_sched, const void* out, const void* dout, const float* lse,
+                                    float* rowdot, int64_t lse_ld, void* dqkv, int64_t P, int H, int D, uint32_t* err,
+                                    cudaStream_t s);
 
 // ---------------------------------------------------------------------------- small kernels
 // The first kernel of an entry point also clears the GEMM tile counters of the call
@@ -121,9 +172,6 @@ cudaError_t launch_swiglu_bwd(const void* g, const void* u, const void* dh, void
                               int sms, cudaStream_t s);
 cudaError_t launch_rotary_bwd(void* dqkv, const float* cos, const float* sin, int64_t P, int D, int hd, int sms,
                               cudaStream_t s);
-cudaError_t launch_attention_bwd(const void* qkv, const void* out, const void* dout, void* dqkv, float* lse,
-                                 float* rowdot, const int32_t* cu_dev, int n_images, int total_blocks, int D, int H,
-                                 cudaStream_t s);
 // Image-token bridge (bridge.cu).  Positions per CTA of the merge; counts holds one int4 per
 // chunk of that many positions.
 constexpr int kBridgeChunk = 256;

@@ -24,7 +24,10 @@ DSV4V_ERR_LAYOUT = 6
 # Pseudo-token types of the image-token bridge (DSV4V_TOKEN_*); sentinel rows follow types 1..4.
 TOKEN_TEXT, TOKEN_IMAGE, TOKEN_START, TOKEN_END, TOKEN_NEWLINE, TOKEN_PAD = -1, 0, 1, 2, 3, 4
 
-PROFILE_KINDS = ("qkv", "attention", "out", "swiglu", "down")  # DSV4V_PROFILE_* order
+PROFILE_KINDS = ("qkv", "attention", "out", "swiglu", "down", "chain")  # DSV4V_PROFILE_* order
+
+# Launch sequences of the bf16 blocks (DSV4V_PATH_*).
+PATH_AUTO, PATH_KERNELS, PATH_CHAIN = 0, 1, 2
 
 # Every symbol include/dsv4v.h declares.
 EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", "dsv4v_tower_forward",
@@ -35,7 +38,7 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_patch_merger_workspace_size", "dsv4v_patch_merger_forward", "dsv4v_image_layout",
            "dsv4v_bridge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility",
            "dsv4v_backward_workspace_size", "dsv4v_attention_backward", "dsv4v_rmsnorm_backward",
-           "dsv4v_block_backward", "dsv4v_tower_backward")
+           "dsv4v_block_backward", "dsv4v_tower_backward", "dsv4v_set_tower_path", "dsv4v_tower_path")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -110,6 +113,8 @@ def lib() -> ctypes.CDLL:
             "dsv4v_device_error": (I, [P]),
             "dsv4v_selftest_bounded_wait": (I, [U64, P]),
             "dsv4v_status_string": (ctypes.c_char_p, [I]),
+            "dsv4v_set_tower_path": (I, [I]),
+            "dsv4v_tower_path": (I, [cfg, bat]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -190,6 +195,20 @@ def dsv4v_tower_forward(cfg, batch, layers, final_norm_w, x_inout, workspace, st
     _check(lib().dsv4v_tower_forward(ctypes.byref(cfg), ctypes.byref(batch.c), arr, _ptr(final_norm_w),
                                      _ptr(x_inout), _ptr(workspace), workspace.numel(), _stream(stream)),
            "dsv4v_tower_forward")
+
+
+def dsv4v_set_tower_path(path):
+    """Process-wide choice of the bf16 blocks' launch sequence (PATH_AUTO, PATH_KERNELS or
+    PATH_CHAIN) for the calls that follow; size workspaces after setting it."""
+    _check(lib().dsv4v_set_tower_path(int(path)), "dsv4v_set_tower_path")
+
+
+def dsv4v_tower_path(cfg, batch):
+    """PATH_KERNELS or PATH_CHAIN: the sequence the block and tower calls use for this batch."""
+    r = lib().dsv4v_tower_path(ctypes.byref(cfg), ctypes.byref(batch.c))
+    if r < 0:
+        raise Dsv4vError(DSV4V_ERR_INVALID_ARG, "dsv4v_tower_path")
+    return r
 
 
 def dsv4v_tower_forward_profiled(cfg, batch, layers, final_norm_w, x_inout, workspace, events, stream=None):
