@@ -35,13 +35,15 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kRing = 4;                      // operand ring depth
-constexpr int kStageBytes = 48 * 1024;        // A (16 KB) + B (up to 256 rows, 32 KB)
+// Operand ring: a byte arena of kRingBytes holding up to kRingMax stages of each one's own size
+// (A + B of one K block), so that narrow tiles keep as many bytes in flight as wide ones.
+constexpr int kRingBytes = 208 * 1024;
+constexpr int kRingMax = 8;
 constexpr int kABytes = BM * BK * 2;
-constexpr int kStagingBytes = 4 * 8192;       // per epilogue warp: two 32-row x 64-column bf16 boxes
+constexpr int kStagingBytes = 4 * 4096;       // per epilogue warp: one 32-row x 64-column bf16 box
 constexpr int kTaskSlots = 4;
 constexpr int kThreads = 192;
-constexpr int OFF_STAGING = kRing * kStageBytes;
+constexpr int OFF_STAGING = kRingBytes;
 constexpr int OFF_BAR = OFF_STAGING + kStagingBytes;
 constexpr int kBarBytes = 1024;
 constexpr int SMEM = 1024 + OFF_BAR + kBarBytes;
@@ -141,64 +143,170 @@ __device__ __forceinline__ void load_acc(uint32_t t_row, int c0, int c1, float (
   }
 }
 
-// Finisher epilogue of one tile.  CHAIN_RESID: x <- x + acc on columns [n BN, (n + 1) BN),
-// optionally also bf16(x * w) and the row's partial sum of x^2 over these columns.  CHAIN_SWIGLU:
-// accumulator = gate columns then up columns of output columns [n BN/2, (n + 1) BN/2); h =
-// silu(r gate) * (r up) with r the folded norm's row scale.  CHAIN_QKV_HEADS: accumulator = the
-// q, k and v columns of head n (64 each); rows scaled by r, q and k rotated, each 64-column group
-// stored at column g D + 64 n.
+// Output staging of one epilogue warp: one box of 32 rows x 64 bf16 columns in the 128-byte
+// swizzled layout of the output tensor maps (lane i owns row i); each box goes out by one TMA
+// store and is reused once that store has read it.
+struct Stager1 {
+  uint8_t* box;
+  int lane, n;
+  __device__ __forceinline__ uint8_t* acquire() {
+    if (lane == 0 && n >= 1) bulk_wait_read_0();
+    __syncwarp();
+    return box;
+  }
+  __device__ __forceinline__ void put(int j, uint4 v) {
+    *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+  }
+  __device__ __forceinline__ void store(const CUtensorMap* map, int x, int y, int rows) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && y < rows) {
+      tma_store_2d(map, box, x, y);
+      bulk_commit();
+    }
+    ++n;
+  }
+};
+
+__device__ __forceinline__ void pack8(const float* v, uint4 (&o)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    o[q].x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    o[q].y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    o[q].z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    o[q].w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+  }
+}
+
+// One task of the epilogue warps.  The inputs of the epilogue math (folded-norm row scale,
+// rotation tables, residual row) are fetched before the accumulator is waited for, so that their
+// L2 round trips overlap the MMAs.  An earlier split parks its fp32 partial; the finisher adds
+// the partials (split order), runs the epilogue math, stores, and releases the row tile's counter
+// once its stores are complete.
+//   CHAIN_RESID: x <- x + acc on columns [n BN, (n + 1) BN), optionally also bf16(x * w) and the
+//     row's partial sum of x^2 over these columns.
+//   CHAIN_SWIGLU: accumulator = gate columns then up columns of output columns
+//     [n BN/2, (n + 1) BN/2); h = silu(r gate) * (r up), r the folded norm's row scale.
+//   CHAIN_QKV_HEADS: accumulator = the q, k and v columns of head n (64 each); rows scaled by r,
+//     q and k rotated, each 64-column group stored at column g D + 64 n.
+// Returns false when a bounded wait gave up.
 template <int EPI>
-__device__ __forceinline__ void finish_tile(const ChainParams& p, const ChainStage& d, const Task& k, uint32_t t_row,
-                                            int quad, int lane, Stager& st) {
+__device__ __forceinline__ bool epilogue_task(const ChainParams& p, const ChainStage& d, const Task& k,
+                                              uint32_t t_row, uint64_t* tfull_acc, uint64_t* tempty_acc,
+                                              uint32_t acc_phase, int quad, int lane, int et, Stager1& st,
+                                              volatile int* abort_flag, volatile int* ticket_ok) {
   const int row_in_tile = quad * 32 + lane;
   const int row = k.m * BM + row_in_tile;
+  const int prow = min(row, d.M - 1);
   const int box_y = k.m * BM + quad * 32;
   const int tile = k.m * d.tiles_n + k.n;
-  const CUtensorMap* m_out = &p.maps[d.map_out];
+  const bool finisher = k.split + 1 == d.splits;
   const int ngroups = d.bn / 64;
+  // ---- inputs fetched while the MMAs run
+  float scale = 1.0f;
+  float rc[EPI == CHAIN_QKV_HEADS ? 32 : 1], rs[EPI == CHAIN_QKV_HEADS ? 32 : 1];
+  uint4 res[EPI == CHAIN_RESID ? 16 : 1];  // residual: the first two 64-column groups
+  const uint4* rrow = nullptr;
+  if (finisher) {
+    if constexpr (EPI != CHAIN_RESID) {
+      scale = chain_row_scale(p, d, row);
+      pin(scale);
+    }
+    if constexpr (EPI == CHAIN_QKV_HEADS) {
+      const float4* c4 = reinterpret_cast<const float4*>(d.cos + static_cast<size_t>(prow) * 32);
+      const float4* s4 = reinterpret_cast<const float4*>(d.sin + static_cast<size_t>(prow) * 32);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 c = c4[q], sv = s4[q];
+        rc[4 * q] = c.x; rc[4 * q + 1] = c.y; rc[4 * q + 2] = c.z; rc[4 * q + 3] = c.w;
+        rs[4 * q] = sv.x; rs[4 * q + 1] = sv.y; rs[4 * q + 2] = sv.z; rs[4 * q + 3] = sv.w;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        pin(rc[j]);
+        pin(rs[j]);
+      }
+    }
+    if constexpr (EPI == CHAIN_RESID) {
+      rrow = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(d.resid) +
+                                            static_cast<size_t>(prow) * d.ldr + k.n * d.bn);
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (q < 8 * ngroups) res[q] = rrow[q];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) pin(res[q]);
+    }
+  }
+  const bool got = mbar_wait(tfull_acc, acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
+  if (!named_barrier_and(2, 128, got)) return false;
+  tc_fence_after_sync();
+  if (!finisher) {
+    // An earlier split of the tile: park the fp32 partial, release it, move on.
+    float* part = d.partials + (static_cast<size_t>(tile) * (d.splits - 1) + k.split) * BM * d.bn;
+    for (int c = 0; c < d.bn / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(t_row + c * 32, r);
+      tmem_ld_wait(r);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(part + ((c * 8 + q) * BM + row_in_tile) * 4) =
+            make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                        __uint_as_float(r[4 * q + 3]));
+    }
+    tc_fence_before_sync();
+    mbar_arrive(tempty_acc);
+    __threadfence();
+    named_barrier_sync(1, 128);
+    if (et == 0) atomicAdd(d.arrivals + tile, 1);
+    return true;
+  }
+  if (d.splits > 1) {
+    if (et == 0)
+      *ticket_ok = wait_counter_backoff(d.arrivals + tile, d.splits - 1, abort_flag, p.err, kErrTimeoutEpilogue) ? 1
+                                                                                                                 : 0;
+    named_barrier_sync(1, 128);
+    if (!*ticket_ok) {
+      tc_fence_before_sync();
+      mbar_arrive(tempty_acc);
+      return false;
+    }
+    __threadfence();
+  }
+  const CUtensorMap* m_out = &p.maps[d.map_out];
   if constexpr (EPI == CHAIN_RESID) {
     const CUtensorMap* m_xw = d.map_xw >= 0 ? &p.maps[d.map_xw] : nullptr;
     float ss_acc = 0.0f;
-    const uint4* rrow = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(d.resid) +
-                                                       static_cast<size_t>(min(row, d.M - 1)) * d.ldr + k.n * d.bn);
-    uint4 res[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) res[q] = rrow[q];
-    for (int g = 0; g < ngroups; ++g) {
+    // Group g uses the residual slot r (8 x 16 bytes: 64 columns), refilled two groups ahead.
+    auto group = [&](int g, uint4* r) {
       float v[64];
       load_acc(t_row, 2 * g, 2 * g + 1, v);
       add_partials(d, tile, row_in_tile, 2 * g, 2 * g + 1, v);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        v[8 * q + 0] += bf16_lo(res[q].x);
-        v[8 * q + 1] += bf16_hi(res[q].x);
-        v[8 * q + 2] += bf16_lo(res[q].y);
-        v[8 * q + 3] += bf16_hi(res[q].y);
-        v[8 * q + 4] += bf16_lo(res[q].z);
-        v[8 * q + 5] += bf16_hi(res[q].z);
-        v[8 * q + 6] += bf16_lo(res[q].w);
-        v[8 * q + 7] += bf16_hi(res[q].w);
+        const uint4 x = r[q];
+        v[8 * q + 0] += bf16_lo(x.x);
+        v[8 * q + 1] += bf16_hi(x.x);
+        v[8 * q + 2] += bf16_lo(x.y);
+        v[8 * q + 3] += bf16_hi(x.y);
+        v[8 * q + 4] += bf16_lo(x.z);
+        v[8 * q + 5] += bf16_hi(x.z);
+        v[8 * q + 6] += bf16_lo(x.w);
+        v[8 * q + 7] += bf16_hi(x.w);
       }
-      if (g + 1 < ngroups) {
+      if (g + 2 < ngroups) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) res[q] = rrow[8 * (g + 1) + q];
+        for (int q = 0; q < 8; ++q) r[q] = rrow[8 * (g + 2) + q];
       }
-      uint8_t* box = nullptr;
-      uint8_t* box2 = nullptr;
-      if (m_xw) st.acquire_both(box, box2);
-      else box = st.acquire();
       uint4 o[8];
+      pack8(v, o);
+      st.acquire();
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        o[q].x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-        o[q].y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-        o[q].z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-        o[q].w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-        if (row < d.M) st.put(box, q, o[q]);
-      }
-      if (m_xw && row < d.M) {
+      for (int q = 0; q < 8; ++q) st.put(q, o[q]);
+      st.store(m_out, k.n * d.bn + g * 64, box_y, d.M);
+      if (m_xw) {
         // The next norm's operand from the stored (bf16) x: bf16(x * w) and the sum of x^2.
         const float4* w4 = reinterpret_cast<const float4*>(d.xw_w + k.n * d.bn + g * 64);
+        st.acquire();
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
@@ -210,38 +318,53 @@ __device__ __forceinline__ void finish_tile(const ChainParams& p, const ChainSta
           t.y = pack_bf16x2(x2 * wa.z, x3 * wa.w);
           t.z = pack_bf16x2(x4 * wb.x, x5 * wb.y);
           t.w = pack_bf16x2(x6 * wb.z, x7 * wb.w);
-          st.put(box2, q, t);
+          st.put(q, t);
         }
+        st.store(m_xw, k.n * d.bn + g * 64, box_y, d.M);
       }
-      st.store(box, m_out, k.n * d.bn + g * 64, box_y, d.M);
-      if (m_xw) st.store(box2, m_xw, k.n * d.bn + g * 64, box_y, d.M);
+    };
+    for (int g = 0; g < ngroups; g += 2) {
+      group(g, res);
+      if (g + 1 < ngroups) group(g + 1, res + 8);
     }
     if (m_xw && row < d.M) d.ss_out[static_cast<size_t>(row) * d.ss_parts + k.n] = ss_acc;
   } else if constexpr (EPI == CHAIN_SWIGLU) {
-    const float scale = chain_row_scale(p, d, row);
-    uint8_t* box = nullptr;
+    uint4 h2[4];
     for (int g = 0; g < ngroups; ++g) {
       float v[64];
       load_acc(t_row, g, ngroups + g, v);
       add_partials(d, tile, row_in_tile, g, ngroups + g, v);
-      if ((g & 1) == 0) box = st.acquire();
+      uint4 h4[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float h[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) h[e] = silu(scale * v[8 * q + e]) * (scale * v[32 + 8 * q + e]);
-        uint4 o;
-        o.x = pack_bf16x2(h[0], h[1]);
-        o.y = pack_bf16x2(h[2], h[3]);
-        o.z = pack_bf16x2(h[4], h[5]);
-        o.w = pack_bf16x2(h[6], h[7]);
-        st.put(box, 4 * (g & 1) + q, o);
+        h4[q].x = pack_bf16x2(h[0], h[1]);
+        h4[q].y = pack_bf16x2(h[2], h[3]);
+        h4[q].z = pack_bf16x2(h[4], h[5]);
+        h4[q].w = pack_bf16x2(h[6], h[7]);
       }
-      if ((g & 1) == 1 || g == ngroups - 1) st.store(box, m_out, k.n * (d.bn / 2) + (g >> 1) * 64, box_y, d.M);
+      if ((g & 1) == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) h2[q] = h4[q];
+      }
+      if ((g & 1) == 1 || g == ngroups - 1) {
+        st.acquire();
+        if ((g & 1) == 1) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            st.put(q, h2[q]);
+            st.put(4 + q, h4[q]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) st.put(q, h4[q]);
+        }
+        st.store(m_out, k.n * (d.bn / 2) + (g >> 1) * 64, box_y, d.M);
+      }
     }
   } else {  // CHAIN_QKV_HEADS
-    const float scale = chain_row_scale(p, d, row);
-    const int prow = min(row, d.M - 1);
     for (int g = 0; g < ngroups; ++g) {
       float v[64];
       load_acc(t_row, 2 * g, 2 * g + 1, v);
@@ -249,22 +372,14 @@ __device__ __forceinline__ void finish_tile(const ChainParams& p, const ChainSta
 #pragma unroll
       for (int j = 0; j < 64; ++j) v[j] *= scale;
       if (g < 2) {
-        const float4* c4 = reinterpret_cast<const float4*>(d.cos + static_cast<size_t>(prow) * 32);
-        const float4* s4 = reinterpret_cast<const float4*>(d.sin + static_cast<size_t>(prow) * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 c = c4[q], s = s4[q];
-          const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * q + e;
-            const float x1 = v[j], x2 = v[32 + j];
-            v[j] = x1 * cc[e] - x2 * ss[e];
-            v[32 + j] = x2 * cc[e] + x1 * ss[e];
-          }
+        for (int j = 0; j < 32; ++j) {
+          const float x1 = v[j], x2 = v[32 + j];
+          v[j] = x1 * rc[j] - x2 * rs[j];
+          v[32 + j] = x2 * rc[j] + x1 * rs[j];
         }
       }
-      uint8_t* box = st.acquire();
+      st.acquire();
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         uint4 o;
@@ -272,19 +387,36 @@ __device__ __forceinline__ void finish_tile(const ChainParams& p, const ChainSta
         o.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
         o.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
         o.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-        st.put(box, q, o);
+        st.put(q, o);
       }
-      st.store(box, m_out, g * d.D + k.n * 64, box_y, d.M);
+      st.store(m_out, g * d.D + k.n * 64, box_y, d.M);
     }
   }
+  tc_fence_before_sync();
+  mbar_arrive(tempty_acc);
+  if (d.splits > 1 && et == 0) d.arrivals[tile] = 0;  // ready for the next launch
+  // Completion: this warp's TMA stores have written global memory, then one release per tile on
+  // the row tile's counter.
+  if (lane == 0) {
+    bulk_wait_all();
+    fence_proxy_async_global();
+  }
+  __syncwarp();
+  __threadfence();
+  named_barrier_sync(1, 128);
+  if (et == 0) {
+    __threadfence();
+    atomicAdd(d.done + k.m, 1);
+  }
+  return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ ChainParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* empty = full + kRing;
-  uint64_t* tfull = empty + kRing;
+  uint64_t* empty = full + kRingMax;
+  uint64_t* tfull = empty + kRingMax;
   uint64_t* tempty = tfull + 2;
   uint64_t* task_full = tempty + 2;
   uint64_t* task_empty = task_full + kTaskSlots;
@@ -294,12 +426,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tasks + kTaskSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* ticket_ok = reinterpret_cast<volatile int*>(tmem_holder + 2);
+  uint32_t* stage_off = tmem_holder + 4;  // [kRingMax]: byte offset in the ring of each stage slot
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRing; ++s) {
+    for (int s = 0; s < kRingMax; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -334,13 +467,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
     // ------------------------------------------------------------------ tickets + TMA producer
     if (lane == 0) {
       grid_dependency_wait();  // earlier kernels of the stream (their outputs are the first operands)
-      int stage = 0;
-      uint32_t phase = 0, issued = 0, issued_phase = 0;
+      // Operand ring as a byte arena: stage i (barrier slot i % kRingMax) takes the next
+      // kABytes + BN * 128 bytes after the previous stage, wrapping to offset 0 when it would not
+      // fit before the end; it is allocated once no in-flight stage overlaps it (stages are
+      // released in order by the MMA issuer's commits).
+      int sseq = 0, rel = 0;
+      uint32_t head = 0;
+      uint32_t s_off[kRingMax], s_size[kRingMax];
       bool ok = true;
-      auto next_stage = [&]() {
-        if (++stage == kRing) {
-          stage = 0;
-          phase ^= 1;
+      auto alloc = [&](uint32_t size) -> int {
+        for (;;) {
+          uint32_t off = head;
+          if (off + size > static_cast<uint32_t>(kRingBytes)) off = 0;
+          bool fits = sseq - rel < kRingMax;
+          for (int i = rel; fits && i < sseq; ++i) {
+            const uint32_t o = s_off[i % kRingMax], e = o + s_size[i % kRingMax];
+            if (off < e && o < off + size) fits = false;
+          }
+          if (fits) {
+            const int slot = sseq % kRingMax;
+            s_off[slot] = off;
+            s_size[slot] = size;
+            stage_off[slot] = off;
+            head = off + size;
+            ++sseq;
+            return slot;
+          }
+          if (!mbar_wait(&empty[rel % kRingMax], static_cast<uint32_t>(rel / kRingMax) & 1u, abort_flag, p.err,
+                         kErrTimeoutProducer))
+            return -1;
+          ++rel;
         }
       };
       for (int seq = 0; ok; ++seq) {
@@ -373,36 +529,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
         const CUtensorMap* ma = &p.maps[d.map_a];
         const CUtensorMap* mb = &p.maps[d.map_b];
         const CUtensorMap* mb2 = d.map_b2 >= 0 ? &p.maps[d.map_b2] : mb;
-        const uint32_t stage_tx = static_cast<uint32_t>(kABytes + d.bn * 128);
-        auto load_b = [&](int s, int kb) {
-          uint8_t* sb = smem + s * kStageBytes + kABytes;
+        const uint32_t stage_bytes = static_cast<uint32_t>(kABytes + d.bn * 128);
+        auto load_b = [&](int rs, int kb) {
+          uint8_t* sb = smem + s_off[rs] + kABytes;
           if (d.epi == CHAIN_SWIGLU) {
-            tma_load_2d(sb, mb, &full[s], kb * BK, k.n * (d.bn / 2));
-            tma_load_2d(sb + (d.bn / 2) * 128, mb2, &full[s], kb * BK, k.n * (d.bn / 2));
+            tma_load_2d(sb, mb, &full[rs], kb * BK, k.n * (d.bn / 2));
+            tma_load_2d(sb + (d.bn / 2) * 128, mb2, &full[rs], kb * BK, k.n * (d.bn / 2));
           } else if (d.epi == CHAIN_QKV_HEADS) {
             // q, k and v rows of head n: three 64-row boxes of wqkv
-            tma_load_2d(sb, mb, &full[s], kb * BK, k.n * 64);
-            tma_load_2d(sb + 64 * 128, mb, &full[s], kb * BK, d.D + k.n * 64);
-            tma_load_2d(sb + 128 * 128, mb, &full[s], kb * BK, 2 * d.D + k.n * 64);
+            tma_load_2d(sb, mb, &full[rs], kb * BK, k.n * 64);
+            tma_load_2d(sb + 64 * 128, mb, &full[rs], kb * BK, d.D + k.n * 64);
+            tma_load_2d(sb + 128 * 128, mb, &full[rs], kb * BK, 2 * d.D + k.n * 64);
           } else {
-            tma_load_2d(sb, mb, &full[s], kb * BK, k.n * d.bn);
+            tma_load_2d(sb, mb, &full[rs], kb * BK, k.n * d.bn);
           }
         };
-        auto load_a = [&](int s, int kb) { tma_load_2d(smem + s * kStageBytes, ma, &full[s], kb * BK, k.m * BM); };
+        auto load_a = [&](int rs, int kb) { tma_load_2d(smem + s_off[rs], ma, &full[rs], kb * BK, k.m * BM); };
         // Weight tiles of the first stages: they depend on nothing.
         const int nkb = k.kb1 - k.kb0;
-        const int pre = nkb < kRing ? nkb : kRing;
-        const int first_stage = stage;
+        const int pre = nkb < 4 ? nkb : 4;
+        int pre_slot[4];
         for (int i = 0; i < pre && ok; ++i) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutProducer)) {
+          const int rs = alloc(stage_bytes);
+          if (rs < 0) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], stage_tx);
-          load_b(stage, k.kb0 + i);
-          issued |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          next_stage();
+          pre_slot[i] = rs;
+          mbar_arrive_expect_tx(&full[rs], stage_bytes);
+          load_b(rs, k.kb0 + i);
         }
         // The activation rows: wait until the stage producing them has finished this row tile.
         if (ok && d.dep_stage >= 0) {
@@ -417,31 +572,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
         }
         tasks[slot] = k;
         mbar_arrive(&task_full[slot]);
-        for (int i = 0; i < pre; ++i) load_a((first_stage + i) % kRing, k.kb0 + i);
+        for (int i = 0; i < pre; ++i) load_a(pre_slot[i], k.kb0 + i);
         for (int kb = k.kb0 + pre; kb < k.kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.err, kErrTimeoutProducer)) {
+          const int rs = alloc(stage_bytes);
+          if (rs < 0) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], stage_tx);
-          load_a(stage, kb);
-          load_b(stage, kb);
-          issued |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          next_stage();
+          mbar_arrive_expect_tx(&full[rs], stage_bytes);
+          load_a(rs, kb);
+          load_b(rs, kb);
         }
       }
       // Copies still in flight must land before the CTA may exit (error path; in the normal path
       // every issued stage has been consumed and these return at once).
       volatile int never = 0;
-      for (int s = 0; s < kRing; ++s)
-        if (issued & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, &never, p.err, kErrTimeoutProducer);
+      for (int i = rel; i < sseq; ++i)
+        mbar_wait(&full[i % kRingMax], static_cast<uint32_t>(i / kRingMax) & 1u, &never, p.err, kErrTimeoutProducer);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int mseq = 0, acc = 0;  // stages consumed; accumulator buffer
+      uint32_t acc_phase = 0;
       bool ok = true;
       for (int seq = 0; ok; ++seq) {
         const int slot = seq % kTaskSlots;
@@ -456,22 +609,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
         for (int kb = k.kb0; kb < k.kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutMma)) {
+          const int rs = mseq % kRingMax;
+          if (!mbar_wait(&full[rs], static_cast<uint32_t>(mseq / kRingMax) & 1u, abort_flag, p.err, kErrTimeoutMma)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+          const uint32_t a_addr = smem_u32(smem + stage_off[rs]);
           const uint64_t adesc = sdesc_sw128(a_addr, 16, 1024);
           const uint64_t bdesc = sdesc_sw128(a_addr + kABytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > k.kb0 || kk > 0) ? 1u : 0u);
-          umma_commit(&empty[stage]);
-          if (++stage == kRing) {
-            stage = 0;
-            phase ^= 1;
-          }
+          umma_commit(&empty[rs]);
+          ++mseq;
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
@@ -490,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
     const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
     const int row_in_tile = quad * 32 + lane;
     const int et = threadIdx.x - 64;
-    Stager st{smem + OFF_STAGING + (warp - 2) * 8192, lane, 0};
+    Stager1 st{smem + OFF_STAGING + (warp - 2) * 4096, lane, 0};
     grid_dependency_wait();
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -504,70 +655,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
       if (lane == 0) mbar_arrive(&task_empty[slot]);
       if (k.done) break;
       const ChainStage& d = p.st[k.stage];
-      const int tile = k.m * d.tiles_n + k.n;
-      const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
-      if (!named_barrier_and(2, 128, got)) break;
-      tc_fence_after_sync();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
-      if (k.split + 1 < d.splits) {
-        // An earlier split of the tile: park the fp32 partial, release it, move on.
-        float* part = d.partials + (static_cast<size_t>(tile) * (d.splits - 1) + k.split) * BM * d.bn;
-        for (int c = 0; c < d.bn / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_row + c * 32, r);
-          tmem_ld_wait(r);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(part + ((c * 8 + q) * BM + row_in_tile) * 4) =
-                make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                            __uint_as_float(r[4 * q + 3]));
-        }
-        tc_fence_before_sync();
-        mbar_arrive(&tempty[acc]);
-        __threadfence();
-        named_barrier_sync(1, 128);
-        if (et == 0) atomicAdd(d.arrivals + tile, 1);
-      } else {
-        if (d.splits > 1) {
-          if (et == 0)
-            *ticket_ok = wait_counter_backoff(d.arrivals + tile, d.splits - 1, abort_flag, p.err, kErrTimeoutEpilogue)
-                             ? 1 : 0;
-          named_barrier_sync(1, 128);
-          if (!*ticket_ok) {
-            tc_fence_before_sync();
-            mbar_arrive(&tempty[acc]);
-            break;
-          }
-          __threadfence();
-        }
-        switch (d.epi) {
-          case CHAIN_RESID: finish_tile<CHAIN_RESID>(p, d, k, t_row, quad, lane, st); break;
-          case CHAIN_SWIGLU: finish_tile<CHAIN_SWIGLU>(p, d, k, t_row, quad, lane, st); break;
-          default: finish_tile<CHAIN_QKV_HEADS>(p, d, k, t_row, quad, lane, st); break;
-        }
-        tc_fence_before_sync();
-        mbar_arrive(&tempty[acc]);
-        if (d.splits > 1 && et == 0) d.arrivals[tile] = 0;  // ready for the next launch
-        // Completion: this warp's TMA stores have written global memory, then one release per
-        // tile on the row tile's counter.
-        if (lane == 0) {
-          bulk_wait_all();
-          fence_proxy_async_global();
-        }
-        __syncwarp();
-        __threadfence();
-        named_barrier_sync(1, 128);
-        if (et == 0) {
-          __threadfence();
-          atomicAdd(d.done + k.m, 1);
-        }
+      bool ok;
+      switch (d.epi) {
+        case CHAIN_RESID:
+          ok = epilogue_task<CHAIN_RESID>(p, d, k, t_row, &tfull[acc], &tempty[acc], acc_phase, quad, lane, et, st,
+                                          abort_flag, ticket_ok);
+          break;
+        case CHAIN_SWIGLU:
+          ok = epilogue_task<CHAIN_SWIGLU>(p, d, k, t_row, &tfull[acc], &tempty[acc], acc_phase, quad, lane, et, st,
+                                           abort_flag, ticket_ok);
+          break;
+        default:
+          ok = epilogue_task<CHAIN_QKV_HEADS>(p, d, k, t_row, &tfull[acc], &tempty[acc], acc_phase, quad, lane, et,
+                                              st, abort_flag, ticket_ok);
+          break;
       }
+      if (!ok) break;
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
       }
     }
-    st.drain();
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // Teardown: TMEM is released only after every warp has finished with it (role code ran on
@@ -600,11 +711,13 @@ cudaError_t launch_chain(const ChainParams& p, int grid, cudaStream_t s) {
   if (p.total_tasks <= 0) return cudaSuccess;
   if (p.n_stages < 1 || p.n_stages > kChainMaxStages || p.n_maps > kChainMaxMaps || grid <= 0)
     return cudaErrorInvalidValue;
+
   for (int i = 0; i < p.n_stages; ++i) {
     const ChainStage& d = p.st[i];
     if (d.bn <= 0 || d.bn > kAccCols || d.bn % 64 || d.splits < 1 || d.splits > d.kb_total ||
         (d.epi == CHAIN_QKV_HEADS && d.bn != 192) || (d.epi == CHAIN_SWIGLU && d.bn % 128) ||
-        d.dep_stage >= i || (d.splits > 1 && (!d.partials || !d.arrivals)) || !d.done)
+        d.dep_stage >= i || (d.splits > 1 && (!d.partials || !d.arrivals)) || !d.done ||
+        kABytes + d.bn * 128 > kRingBytes / 2)
       return cudaErrorInvalidValue;
   }
   return launch_pdl(k_chain, dim3(grid), dim3(kThreads), SMEM, s, p);
