@@ -190,6 +190,7 @@ dsv4v_status check_all(const dsv4v_config* c, const dsv4v_batch* b, Shape& s) {
 // kernel per GEMM at 784 patches).
 std::atomic<int> g_tower_path{DSV4V_PATH_AUTO};
 constexpr int64_t kChainMaxRows = 0;
+constexpr int kChainRingSlotsMax = 8;  // operand ring slots of the chain kernel (at most)
 
 struct ChainStagePlan {
   int bn = 0, splits = 1, tiles_n = 0, kb = 0;
@@ -221,8 +222,10 @@ ChainStagePlan plan_chain_stage(int stage, const Shape& s, int tiles_m, int sms)
   const int K = stage == CS_DOWN ? s.F : s.D;
   const int kb = (K + 63) / 64;
   const int n_cols = stage == CS_GATEUP ? s.F : s.D;
+  // SwiGLU takes 256-column tiles (128 gate + 128 up): measured on B200 at 784 rows, two waves of
+  // them finish ~8 us sooner than three waves of 128-column tiles.
   const int bns[2] = {256, 128};
-  for (int bi = 0; bi < (stage == CS_QKV ? 1 : 2); ++bi) {
+  for (int bi = 0; bi < (stage == CS_QKV || stage == CS_GATEUP ? 1 : 2); ++bi) {
     const int bn = stage == CS_QKV ? 192 : bns[bi];
     const int cols = stage == CS_QKV ? 64 : (stage == CS_GATEUP ? bn / 2 : bn);
     if (n_cols % cols) continue;
@@ -685,6 +688,11 @@ dsv4v_status run_chain(const Ctx& c, int launch, const dsv4v_block_weights* cur,
   }
   if (!b.ok) return DSV4V_ERR_CUDA;
   p.total_tasks = task;
+  // Ring slots as large as the launch's largest stage (A + B tile of one K block), as many as fit.
+  int stage_bytes = 0;
+  for (int i = 0; i < p.n_stages; ++i) stage_bytes = std::max(stage_bytes, 128 * 64 * 2 + p.st[i].bn * 128);
+  p.slot_bytes = (stage_bytes + 8191) / 8192 * 8192;
+  p.ring_slots = std::min(kChainRingSlotsMax, chain_ring_bytes() / p.slot_bytes);
   return cuda_status(launch_chain(p, c.dev.sms, c.stream));
 }
 

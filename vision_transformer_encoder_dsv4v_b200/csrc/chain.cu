@@ -35,8 +35,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-// Operand ring: a byte arena of kRingBytes holding up to kRingMax stages of each one's own size
-// (A + B of one K block), so that narrow tiles keep as many bytes in flight as wide ones.
+// Operand ring: kRingBytes split into ChainParams::ring_slots slots of slot_bytes (the launch's
+// largest stage, A + B of one K block), at most kRingMax of them.
 constexpr int kRingBytes = 208 * 1024;
 constexpr int kRingMax = 8;
 constexpr int kABytes = BM * BK * 2;
@@ -426,7 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tasks + kTaskSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* ticket_ok = reinterpret_cast<volatile int*>(tmem_holder + 2);
-  uint32_t* stage_off = tmem_holder + 4;  // [kRingMax]: byte offset in the ring of each stage slot
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -467,37 +466,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
     // ------------------------------------------------------------------ tickets + TMA producer
     if (lane == 0) {
       grid_dependency_wait();  // earlier kernels of the stream (their outputs are the first operands)
-      // Operand ring as a byte arena: stage i (barrier slot i % kRingMax) takes the next
-      // kABytes + BN * 128 bytes after the previous stage, wrapping to offset 0 when it would not
-      // fit before the end; it is allocated once no in-flight stage overlaps it (stages are
-      // released in order by the MMA issuer's commits).
-      int sseq = 0, rel = 0;
-      uint32_t head = 0;
-      uint32_t s_off[kRingMax], s_size[kRingMax];
+      // Operand ring: ring_slots slots of slot_bytes (chosen per launch for its largest stage);
+      // stage i uses slot i % ring_slots.
+      const int n_ring = p.ring_slots;
+      int sseq = 0;
       bool ok = true;
-      auto alloc = [&](uint32_t size) -> int {
-        for (;;) {
-          uint32_t off = head;
-          if (off + size > static_cast<uint32_t>(kRingBytes)) off = 0;
-          bool fits = sseq - rel < kRingMax;
-          for (int i = rel; fits && i < sseq; ++i) {
-            const uint32_t o = s_off[i % kRingMax], e = o + s_size[i % kRingMax];
-            if (off < e && o < off + size) fits = false;
-          }
-          if (fits) {
-            const int slot = sseq % kRingMax;
-            s_off[slot] = off;
-            s_size[slot] = size;
-            stage_off[slot] = off;
-            head = off + size;
-            ++sseq;
-            return slot;
-          }
-          if (!mbar_wait(&empty[rel % kRingMax], static_cast<uint32_t>(rel / kRingMax) & 1u, abort_flag, p.err,
-                         kErrTimeoutProducer))
-            return -1;
-          ++rel;
-        }
+      auto alloc = [&](uint32_t) -> int {
+        const int slot = sseq % n_ring;
+        if (sseq >= n_ring &&
+            !mbar_wait(&empty[slot], static_cast<uint32_t>(sseq / n_ring - 1) & 1u, abort_flag, p.err,
+                       kErrTimeoutProducer))
+          return -1;
+        ++sseq;
+        return slot;
       };
       for (int seq = 0; ok; ++seq) {
         const int slot = seq % kTaskSlots;
@@ -531,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
         const CUtensorMap* mb2 = d.map_b2 >= 0 ? &p.maps[d.map_b2] : mb;
         const uint32_t stage_bytes = static_cast<uint32_t>(kABytes + d.bn * 128);
         auto load_b = [&](int rs, int kb) {
-          uint8_t* sb = smem + s_off[rs] + kABytes;
+          uint8_t* sb = smem + rs * p.slot_bytes + kABytes;
           if (d.epi == CHAIN_SWIGLU) {
             tma_load_2d(sb, mb, &full[rs], kb * BK, k.n * (d.bn / 2));
             tma_load_2d(sb + (d.bn / 2) * 128, mb2, &full[rs], kb * BK, k.n * (d.bn / 2));
@@ -544,10 +525,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
             tma_load_2d(sb, mb, &full[rs], kb * BK, k.n * d.bn);
           }
         };
-        auto load_a = [&](int rs, int kb) { tma_load_2d(smem + s_off[rs], ma, &full[rs], kb * BK, k.m * BM); };
-        // Weight tiles of the first stages: they depend on nothing.
+        auto load_a = [&](int rs, int kb) { tma_load_2d(smem + rs * p.slot_bytes, ma, &full[rs], kb * BK, k.m * BM); };
+        // Weight tiles of the first stages: they depend on nothing.  The task is published (and
+        // its stages consumed) only after its dependency wait, so these stages must fit in the
+        // ring together: at most ring_slots of them.
         const int nkb = k.kb1 - k.kb0;
-        const int pre = nkb < 4 ? nkb : 4;
+        const int pre = min(min(nkb, 4), n_ring);
         int pre_slot[4];
         for (int i = 0; i < pre && ok; ++i) {
           const int rs = alloc(stage_bytes);
@@ -587,8 +570,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
       // Copies still in flight must land before the CTA may exit (error path; in the normal path
       // every issued stage has been consumed and these return at once).
       volatile int never = 0;
-      for (int i = rel; i < sseq; ++i)
-        mbar_wait(&full[i % kRingMax], static_cast<uint32_t>(i / kRingMax) & 1u, &never, p.err, kErrTimeoutProducer);
+      for (int i = sseq > n_ring ? sseq - n_ring : 0; i < sseq; ++i)
+        mbar_wait(&full[i % n_ring], static_cast<uint32_t>(i / n_ring) & 1u, &never, p.err, kErrTimeoutProducer);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -609,13 +592,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
         for (int kb = k.kb0; kb < k.kb1; ++kb) {
-          const int rs = mseq % kRingMax;
-          if (!mbar_wait(&full[rs], static_cast<uint32_t>(mseq / kRingMax) & 1u, abort_flag, p.err, kErrTimeoutMma)) {
+          const int rs = mseq % p.ring_slots;
+          if (!mbar_wait(&full[rs], static_cast<uint32_t>(mseq / p.ring_slots) & 1u, abort_flag, p.err,
+                         kErrTimeoutMma)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(smem + stage_off[rs]);
+          const uint32_t a_addr = smem_u32(smem + rs * p.slot_bytes);
           const uint64_t adesc = sdesc_sw128(a_addr, 16, 1024);
           const uint64_t bdesc = sdesc_sw128(a_addr + kABytes, 16, 1024);
 #pragma unroll
@@ -698,6 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
 
 }  // namespace
 
+int chain_ring_bytes() { return kRingBytes; }
+
 cudaError_t launch_chain(const ChainParams& p, int grid, cudaStream_t s) {
   static unsigned long long attr_set_mask = 0;
   int dev = 0;
@@ -711,13 +697,15 @@ cudaError_t launch_chain(const ChainParams& p, int grid, cudaStream_t s) {
   if (p.total_tasks <= 0) return cudaSuccess;
   if (p.n_stages < 1 || p.n_stages > kChainMaxStages || p.n_maps > kChainMaxMaps || grid <= 0)
     return cudaErrorInvalidValue;
+  if (p.ring_slots < 2 || p.ring_slots > kRingMax || p.slot_bytes % 1024 || p.ring_slots * p.slot_bytes > kRingBytes)
+    return cudaErrorInvalidValue;
 
   for (int i = 0; i < p.n_stages; ++i) {
     const ChainStage& d = p.st[i];
     if (d.bn <= 0 || d.bn > kAccCols || d.bn % 64 || d.splits < 1 || d.splits > d.kb_total ||
         (d.epi == CHAIN_QKV_HEADS && d.bn != 192) || (d.epi == CHAIN_SWIGLU && d.bn % 128) ||
         d.dep_stage >= i || (d.splits > 1 && (!d.partials || !d.arrivals)) || !d.done ||
-        kABytes + d.bn * 128 > kRingBytes / 2)
+        kABytes + d.bn * 128 > p.slot_bytes)
       return cudaErrorInvalidValue;
   }
   return launch_pdl(k_chain, dim3(grid), dim3(kThreads), SMEM, s, p);

@@ -104,11 +104,15 @@ struct ChainParams {
   CUtensorMap maps[kChainMaxMaps];
   ChainStage st[kChainMaxStages];
   int n_stages, n_maps, total_tasks;
+  int ring_slots, slot_bytes;  // operand ring: slots of slot_bytes (>= every stage's A + B bytes,
+                               // a multiple of 1024), ring_slots * slot_bytes <= chain_ring_bytes()
   float norm_inv_d, norm_eps;
   int* ticket;  // zero before the launch
   uint32_t* err;
 };
 cudaError_t launch_chain(const ChainParams& p, int grid, cudaStream_t s);
+// Shared-memory bytes of the chain kernel's operand ring.
+int chain_ring_bytes();
 
 // ---------------------------------------------------------------------------- attention
 constexpr int kMaxImages = 1024;
