@@ -237,11 +237,12 @@ def run_ours(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.Stream()
 
-    # Launches of one step: the rotary table, the first norm operand, per layer either 4 GEMMs +
-    # attention (one kernel per GEMM) or attention + one chain launch (plus layer 0's q|k|v
-    # launch), the final norm, and the aligner's window index, merged-row copy and GEMM.
+    # Launches of one step (the library's count for this batch and launch sequence): the rotary
+    # table, the first norm operand, per layer either 4 GEMMs + attention or attention + one chain
+    # launch (plus layer 0's q|k|v launch), the final norm, and the aligner's window index,
+    # merged-row copy (when the GEMM does not gather the rows itself) and GEMM.
     chain_path = A.dsv4v_tower_path(cfg, batch) == A.PATH_CHAIN
-    launches_per_step = (2 * wl.n_layers + 7) if chain_path else (5 * wl.n_layers + 6)
+    launches_per_step = A.dsv4v_step_launches(cfg, batch, True, True)
 
     def step(s):
         x.copy_(x0)

@@ -170,6 +170,12 @@ enum {
   DSV4V_PROFILE_KINDS = 6
 };
 
+/* Number of kernel launches that dsv4v_tower_forward (with a final norm when final_norm != 0)
+ * followed by dsv4v_aligner_forward (when aligner != 0) put on the stream for this config and
+ * batch under the current launch-sequence setting (host computation); -1 if the arguments are
+ * invalid. */
+int dsv4v_step_launches(const dsv4v_config* cfg, const dsv4v_batch* batch, int final_norm, int aligner);
+
 /* Launch sequence of the bf16 blocks (no effect on fp32 configs).  Both compute the same
  * block, with the same roundings: they differ in how the GEMMs' K dimension is split, so sums
  * of fp32 products may be added in another order.

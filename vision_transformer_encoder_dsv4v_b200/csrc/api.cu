@@ -277,6 +277,14 @@ Plans make_plans(const Shape& s, int sms) {
   return p;
 }
 
+// The bf16 aligner reads its window rows straight from x with TMA gather when its GEMM plan is a
+// cluster split-K whose K slices each lie within one window slot.
+bool aligner_gathers(const Shape& s, const GemmPlan& pl) {
+  const int kb_slot = s.D / 64;
+  return s.bf16 && pl.ks > 1 && pl.kb_total % pl.ks == 0 && pl.kb_total / pl.ks > 0 &&
+         kb_slot % (pl.kb_total / pl.ks) == 0 && s.P < (1ll << 31);
+}
+
 struct Layout {
   size_t cos, sin, y, qkv, attn, h, partials, counters, asrc, merged, ss1, ss2, total;
   size_t counters_bytes;
@@ -403,6 +411,10 @@ struct GemmExtra {
   int64_t lda = 0, ldb = 0;
   const float* bias = nullptr;
   int clear_counters = 0;  // zero this many split-tile counters on the stream right before the launch
+  // Gathered A (see GemmArgs): a is the source tensor [gather_rows, K / gather_r2].
+  const int32_t* gather_src = nullptr;
+  int gather_r2 = 0;
+  int64_t gather_rows = 0;
 };
 
 dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* a, int64_t M, int K, const void* b,
@@ -411,7 +423,9 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   if (M == 0) return DSV4V_OK;
   const int box_b = (epi == EPI_SWIGLU || plan.pair) ? plan.bn / 2 : plan.bn;
   CUtensorMap ta, tb, tb2, t_out, t_xw;
-  if (!bf16_map(a, M, K, 128, &ta, ex.lda) || !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
+  const bool gathered = ex.gather_src != nullptr;
+  if ((gathered ? !bf16_map(a, ex.gather_rows, K / ex.gather_r2, 1, &ta) : !bf16_map(a, M, K, 128, &ta, ex.lda)) ||
+      !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
       (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)) || !bf16_map(out, M, n_out, 32, &t_out) ||
       (nf.xw_out && !bf16_map(nf.xw_out, M, n_out, 32, &t_xw)))
     return DSV4V_ERR_CUDA;
@@ -443,6 +457,10 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.ss_out = nf.ss_out;
   g.ss_parts = nf.ss_parts;
   g.bias = ex.bias;
+  g.gather_src = ex.gather_src;
+  g.gather_r2 = ex.gather_r2;
+  g.gather_kb_per_slot = gathered ? K / ex.gather_r2 / 64 : 0;
+  g.gather_rows = static_cast<int>(ex.gather_rows);
   if (ex.clear_counters > 0 &&
       cudaMemsetAsync(g.counters, 0, static_cast<size_t>(ex.clear_counters) * sizeof(int), c.stream) != cudaSuccess)
     return DSV4V_ERR_CUDA;
@@ -836,6 +854,21 @@ const char* dsv4v_status_string(dsv4v_status s) {
   return "unknown status";
 }
 
+int dsv4v_step_launches(const dsv4v_config* cfg, const dsv4v_batch* batch, int final_norm, int aligner) {
+  Shape s;
+  if (check_all(cfg, batch, s) != DSV4V_OK) return -1;
+  const Plans pl = make_plans(s, planning_sms());
+  int n = 1;  // rotary table
+  if (s.L > 0) {
+    if (s.bf16 && pl.chain.use) n += 2 + 2 * s.L;  // first norm operand, layer 0's q|k|v, attention + chain per layer
+    else if (s.bf16) n += 1 + 5 * s.L;             // first norm operand, 4 GEMMs + attention per layer
+    else n += 8 * s.L;                              // fp32: 2 norms, 4 GEMMs, rotation, attention per layer
+  }
+  if (final_norm) n += 1;
+  if (aligner) n += (s.bf16 && aligner_gathers(s, pl.align)) ? 2 : 3;  // window index, [merged rows], GEMM
+  return n;
+}
+
 dsv4v_status dsv4v_set_tower_path(int path) {
   if (path != DSV4V_PATH_AUTO && path != DSV4V_PATH_KERNELS && path != DSV4V_PATH_CHAIN)
     return DSV4V_ERR_INVALID_ARG;
@@ -943,11 +976,21 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
                                              s.bf16 ? static_cast<int>(c.lay.counters_bytes / sizeof(int)) : 0)));
   const int K = s.r * s.r * s.D;
   if (s.bf16) {
-    // Materialise the merged window rows, then a TMA GEMM (the weights stream once; the rows
-    // are a few MB).
+    const GemmPlan& pl = c.plans.align;
+    if (aligner_gathers(s, pl)) {
+      // Each CTA of the cluster split-K takes K blocks of one window slot: its A rows come
+      // straight from x by TMA gather, four source rows per copy, no merged operand.
+      GemmExtra ex;
+      ex.gather_src = src;
+      ex.gather_r2 = s.r * s.r;
+      ex.gather_rows = s.P;
+      return gemm_bf16(c, EPI_STORE, pl, x, s.T, K, w_align, nullptr, s.E, out, nullptr, nullptr, nullptr,
+                       NormFold(), ex);
+    }
+    // Otherwise materialise the merged window rows, then a TMA GEMM.
     void* merged = c.at<uint8_t>(c.lay.merged);
     DSV4V_TRY(cuda_status(launch_merge_rows_bf16(x, src, merged, s.T, s.r * s.r, s.D, c.stream)));
-    return gemm_bf16(c, EPI_STORE, c.plans.align, merged, s.T, K, w_align, nullptr, s.E, out, nullptr);
+    return gemm_bf16(c, EPI_STORE, pl, merged, s.T, K, w_align, nullptr, s.E, out, nullptr);
   }
   float* merged = c.at<float>(c.lay.merged);
   DSV4V_TRY(cuda_status(launch_gather_f32(static_cast<const float*>(x), src, merged, s.T, s.r * s.r, s.D, c.stream)));

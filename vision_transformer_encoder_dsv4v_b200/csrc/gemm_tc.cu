@@ -48,7 +48,7 @@ struct TileCfg {
   static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : ((2 * BN <= 256) ? 256 : 512);
   static constexpr int OFF_STAGING = STAGES * STAGE;
   static constexpr int OFF_BARRIERS = OFF_STAGING + kStagingBytes;
-  static constexpr int SMEM = 1024 + OFF_BARRIERS + 512;
+  static constexpr int SMEM = 1024 + OFF_BARRIERS + 1024;
 };
 
 struct Params {
@@ -73,6 +73,11 @@ struct Params {
   float* ss_out;
   int ss_parts;
   const float* bias;
+  // Gathered A (GATHER): row r of the tile's K block kb is row src[(tile row r) * gather_r2 + slot]
+  // of the A tensor (its columns (kb % kb_per_slot) * 64 ...), slot = kb / kb_per_slot; rows
+  // past the source rows (window positions in the zero padding, tokens past the end) read zeros.
+  const int32_t* gather_src;
+  int gather_r2, gather_kb_per_slot, gather_rows;
 };
 
 // ---------------------------------------------------------------------------- stream-K ranges
@@ -253,7 +258,18 @@ __device__ __forceinline__ float* partial_slot(const Params& p, int c) {
 
 
 
-template <int BN, int EPI, bool PAIR, int KS>
+// Four rows (row0..row3) x 64 columns starting at column x of `map` (box: 64 columns x 1 row)
+// into 512 consecutive bytes of shared memory; completes 512 bytes on the mbarrier.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int r0,
+                                           int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
+template <int BN, int EPI, bool PAIR, int KS, bool GATHER = false>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
@@ -274,6 +290,7 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* ticket = reinterpret_cast<volatile int*>(tmem_holder + 2);
+  int32_t* grow = reinterpret_cast<int32_t*>(smem + C::OFF_BARRIERS + 512);  // GATHER: the tile's 128 source rows
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -332,6 +349,24 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
+    static_assert(!GATHER || (!PAIR && KS > 1), "gathered A is built for the cluster split-K plans");
+    int gslot = -1;  // window slot whose source rows are in grow
+    if constexpr (GATHER) {
+      // This CTA's K range lies in one window slot (checked by the launcher): the warp loads the
+      // tile's 128 source rows once.
+      SegmentWalker w0(p, owner);
+      Segment s0{};
+      if (w0.next(p, s0)) {
+        gslot = s0.kb0 / p.gather_kb_per_slot;
+        grid_dependency_wait();
+        for (int r = lane; r < BM; r += 32) {
+          const int t = s0.m_tile * BM + r;
+          const int src = t < p.M ? p.gather_src[static_cast<size_t>(t) * p.gather_r2 + gslot] : -1;
+          grow[r] = src >= 0 ? src : p.gather_rows;  // a row past the end reads zeros
+        }
+      }
+      __syncwarp();
+    }
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
@@ -341,7 +376,14 @@ __global__ void __launch_bounds__(192, 1)
       const bool arrives = !PAIR || rank == 0;  // posts the expected bytes of the stage
       constexpr uint32_t kStageTx = PAIR ? 2 * C::STAGE : C::STAGE;
       auto load_a = [&](uint8_t* sa, int kb, int m_tile, int s) {
-        if constexpr (PAIR)
+        if constexpr (GATHER) {
+          const int x = (kb % p.gather_kb_per_slot) * BK;
+#pragma unroll 1
+          for (int g = 0; g < BM / 4; ++g)
+            tma_gather4(sa + g * 512, &tm_a, &full[s], x, grow[4 * g], grow[4 * g + 1], grow[4 * g + 2],
+                        grow[4 * g + 3]);
+          (void)m_tile;
+        } else if constexpr (PAIR)
           tma_load_2d_pair(sa, &tm_a, full_leader + 8u * s, kb * BK, m_tile * BMT + static_cast<int>(rank) * BM);
         else
           tma_load_2d(sa, &tm_a, &full[s], kb * BK, m_tile * BM);
@@ -804,11 +846,14 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int BN, int EPI, bool PAIR = false, int KS = 1>
+template <int BN, int EPI, bool PAIR = false, int KS = 1, bool GATHER = false>
 cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   using C = TileCfg<BN, PAIR>;
   static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
-  auto kern = k_gemm_tc<BN, EPI, PAIR, KS>;
+  auto kern = k_gemm_tc<BN, EPI, PAIR, KS, GATHER>;
+  if (GATHER && (!a.gather_src || a.gather_kb_per_slot <= 0 || (plan.kb_total / KS) <= 0 ||
+                 a.gather_kb_per_slot % (plan.kb_total / KS)))
+    return cudaErrorInvalidValue;  // every CTA's K slice must lie within one window slot
   if (PAIR && (plan.grid & 1)) return cudaErrorInvalidValue;
   if (KS > 1 && (plan.grid % KS || plan.kb_total % KS || plan.grid != plan.work * KS)) return cudaErrorInvalidValue;
   int dev = 0;
@@ -846,6 +891,10 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.ss_out = a.ss_out;
   p.ss_parts = a.ss_parts;
   p.bias = a.bias;
+  p.gather_src = a.gather_src;
+  p.gather_r2 = a.gather_r2;
+  p.gather_kb_per_slot = a.gather_kb_per_slot;
+  p.gather_rows = a.gather_rows;
   const CUtensorMap& ta = *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
   const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
@@ -863,6 +912,15 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
     // Cluster split-K: 256-column residual, store and GELU tiles.
     if constexpr (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU) {
       if (plan.bn != 256 || plan.pair) return cudaErrorInvalidValue;
+      if constexpr (EPI == EPI_STORE) {
+        if (a.gather_src) {
+          switch (plan.ks) {
+            case 2: return launch_one<256, EPI, false, 2, true>(plan, a, s);
+            case 4: return launch_one<256, EPI, false, 4, true>(plan, a, s);
+            default: return cudaErrorInvalidValue;
+          }
+        }
+      }
       switch (plan.ks) {
         case 2: return launch_one<256, EPI, false, 2>(plan, a, s);
         case 4: return launch_one<256, EPI, false, 4>(plan, a, s);

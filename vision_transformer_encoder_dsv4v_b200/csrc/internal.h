@@ -66,6 +66,11 @@ struct GemmArgs {
   float* ss_out;
   int ss_parts;
   const float* bias;  // STORE: per-column fp32 bias added before rounding (NULL: none)
+  // Gathered A (STORE with a cluster split-K plan whose K slices lie within one window slot):
+  // tm_a is the source tensor [gather_rows, K / gather_r2] with a 64 x 1 box, and row r of the
+  // tile reads source row gather_src[r * gather_r2 + slot] (gather_rows when negative: zeros).
+  const int32_t* gather_src;
+  int gather_r2, gather_kb_per_slot, gather_rows;
 };
 
 cudaError_t launch_gemm_tc(int epi, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);

@@ -18,6 +18,7 @@ DSV4V_MAX_IMAGES = 1024
 
 STATUS = {0: "DSV4V_OK", 1: "DSV4V_ERR_INVALID_ARG", 2: "DSV4V_ERR_UNSUPPORTED", 3: "DSV4V_ERR_WORKSPACE",
           4: "DSV4V_ERR_CUDA", 5: "DSV4V_ERR_TIMEOUT", 6: "DSV4V_ERR_LAYOUT"}
+DSV4V_ERR_INVALID_ARG = 1
 DSV4V_ERR_TIMEOUT = 5
 DSV4V_ERR_LAYOUT = 6
 
@@ -38,7 +39,8 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_patch_merger_workspace_size", "dsv4v_patch_merger_forward", "dsv4v_image_layout",
            "dsv4v_bridge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility",
            "dsv4v_backward_workspace_size", "dsv4v_attention_backward", "dsv4v_rmsnorm_backward",
-           "dsv4v_block_backward", "dsv4v_tower_backward", "dsv4v_set_tower_path", "dsv4v_tower_path")
+           "dsv4v_block_backward", "dsv4v_tower_backward", "dsv4v_set_tower_path", "dsv4v_tower_path",
+           "dsv4v_step_launches")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -115,6 +117,7 @@ def lib() -> ctypes.CDLL:
             "dsv4v_status_string": (ctypes.c_char_p, [I]),
             "dsv4v_set_tower_path": (I, [I]),
             "dsv4v_tower_path": (I, [cfg, bat]),
+            "dsv4v_step_launches": (I, [cfg, bat, I, I]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -208,6 +211,14 @@ def dsv4v_tower_path(cfg, batch):
     r = lib().dsv4v_tower_path(ctypes.byref(cfg), ctypes.byref(batch.c))
     if r < 0:
         raise Dsv4vError(DSV4V_ERR_INVALID_ARG, "dsv4v_tower_path")
+    return r
+
+
+def dsv4v_step_launches(cfg, batch, final_norm=True, aligner=True):
+    """Kernel launches of dsv4v_tower_forward (+ final norm) followed by dsv4v_aligner_forward."""
+    r = lib().dsv4v_step_launches(ctypes.byref(cfg), ctypes.byref(batch.c), int(bool(final_norm)), int(bool(aligner)))
+    if r < 0:
+        raise Dsv4vError(DSV4V_ERR_INVALID_ARG, "dsv4v_step_launches")
     return r
 
 
