@@ -240,7 +240,7 @@ def run_ours(args):
     # Launches of one step (the library's count for this batch and launch sequence): the rotary
     # table, the first norm operand, per layer either 4 GEMMs + attention or attention + one chain
     # launch (plus layer 0's q|k|v launch), the final norm, and the aligner's window index,
-    # merged-row copy (when the GEMM does not gather the rows itself) and GEMM.
+    # merged-row copy and GEMM.
     chain_path = A.dsv4v_tower_path(cfg, batch) == A.PATH_CHAIN
     launches_per_step = A.dsv4v_step_launches(cfg, batch, True, True)
 

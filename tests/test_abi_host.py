@@ -224,17 +224,16 @@ def test_tower_path_choice_and_validation():
 def test_step_launch_count():
     """The per-step launch count the benchmark reports: rotary table, first norm operand, per
     layer 4 GEMMs + attention (or attention + one chain launch), final norm, aligner (window
-    index, merged rows unless the GEMM gathers them, GEMM)."""
+    index, merged rows, GEMM)."""
     from vision_transformer_encoder_dsv4v_b200 import dsv4v as A
     cfg = A.make_config(1024, 16, 2816, 2, 4096, 32)
     one = A.BatchRef([(28, 28)], device=None)
     try:
         A.dsv4v_set_tower_path(A.PATH_KERNELS)
-        # 196 tokens: the aligner's 4-way cluster split-K takes one window slot per CTA (gathered)
-        assert A.dsv4v_step_launches(cfg, one) == 1 + 1 + 5 * 32 + 1 + 2
+        assert A.dsv4v_step_launches(cfg, one) == 1 + 1 + 5 * 32 + 1 + 3
         assert A.dsv4v_step_launches(cfg, one, final_norm=False, aligner=False) == 1 + 1 + 5 * 32
         A.dsv4v_set_tower_path(A.PATH_CHAIN)
-        assert A.dsv4v_step_launches(cfg, one) == 1 + 2 + 2 * 32 + 1 + 2
+        assert A.dsv4v_step_launches(cfg, one) == 1 + 2 + 2 * 32 + 1 + 3
     finally:
         A.dsv4v_set_tower_path(A.PATH_AUTO)
     with pytest.raises(A.Dsv4vError):

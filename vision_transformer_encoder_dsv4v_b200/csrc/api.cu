@@ -277,14 +277,6 @@ Plans make_plans(const Shape& s, int sms) {
   return p;
 }
 
-// The bf16 aligner reads its window rows straight from x with TMA gather when its GEMM plan is a
-// cluster split-K whose K slices each lie within one window slot.
-bool aligner_gathers(const Shape& s, const GemmPlan& pl) {
-  const int kb_slot = s.D / 64;
-  return s.bf16 && pl.ks > 1 && pl.kb_total % pl.ks == 0 && pl.kb_total / pl.ks > 0 &&
-         kb_slot % (pl.kb_total / pl.ks) == 0 && s.P < (1ll << 31);
-}
-
 struct Layout {
   size_t cos, sin, y, qkv, attn, h, partials, counters, asrc, merged, ss1, ss2, total;
   size_t counters_bytes;
@@ -411,11 +403,19 @@ struct GemmExtra {
   int64_t lda = 0, ldb = 0;
   const float* bias = nullptr;
   int clear_counters = 0;  // zero this many split-tile counters on the stream right before the launch
-  // Gathered A (see GemmArgs): a is the source tensor [gather_rows, K / gather_r2].
-  const int32_t* gather_src = nullptr;
-  int gather_r2 = 0;
-  int64_t gather_rows = 0;
+  // Weights of the GEMM that follows, prefetched into L2 by this one (see GemmArgs).
+  const void* l2_next[2] = {nullptr, nullptr};
+  size_t l2_next_bytes[2] = {0, 0};
 };
+
+GemmExtra prefetching(const void* w0, size_t bytes0, const void* w1 = nullptr, size_t bytes1 = 0) {
+  GemmExtra ex;
+  ex.l2_next[0] = w0;
+  ex.l2_next_bytes[0] = w0 ? bytes0 : 0;
+  ex.l2_next[1] = w1;
+  ex.l2_next_bytes[1] = w1 ? bytes1 : 0;
+  return ex;
+}
 
 dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* a, int64_t M, int K, const void* b,
                        const void* b2, int n_out, void* out, const void* resid, const float* cos = nullptr,
@@ -423,9 +423,7 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   if (M == 0) return DSV4V_OK;
   const int box_b = (epi == EPI_SWIGLU || plan.pair) ? plan.bn / 2 : plan.bn;
   CUtensorMap ta, tb, tb2, t_out, t_xw;
-  const bool gathered = ex.gather_src != nullptr;
-  if ((gathered ? !bf16_map(a, ex.gather_rows, K / ex.gather_r2, 1, &ta) : !bf16_map(a, M, K, 128, &ta, ex.lda)) ||
-      !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
+  if (!bf16_map(a, M, K, 128, &ta, ex.lda) || !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
       (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)) || !bf16_map(out, M, n_out, 32, &t_out) ||
       (nf.xw_out && !bf16_map(nf.xw_out, M, n_out, 32, &t_xw)))
     return DSV4V_ERR_CUDA;
@@ -457,10 +455,10 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.ss_out = nf.ss_out;
   g.ss_parts = nf.ss_parts;
   g.bias = ex.bias;
-  g.gather_src = ex.gather_src;
-  g.gather_r2 = ex.gather_r2;
-  g.gather_kb_per_slot = gathered ? K / ex.gather_r2 / 64 : 0;
-  g.gather_rows = static_cast<int>(ex.gather_rows);
+  for (int r = 0; r < 2; ++r) {
+    g.l2_next[r] = ex.l2_next[r];
+    g.l2_next_bytes[r] = ex.l2_next_bytes[r];
+  }
   if (ex.clear_counters > 0 &&
       cudaMemsetAsync(g.counters, 0, static_cast<size_t>(ex.clear_counters) * sizeof(int), c.stream) != cudaSuccess)
     return DSV4V_ERR_CUDA;
@@ -529,8 +527,12 @@ dsv4v_status record(void* const* ev, int kind, int which, cudaStream_t s) {
 }
 
 dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_weights* w, const float* cos,
-                        const float* sin, void* x, bool first, const float* next_norm_w,
+                        const float* sin, void* x, bool first, const dsv4v_block_weights* next,
                         void* const* ev = nullptr) {
+  const float* next_norm_w = next ? next->norm1_w : nullptr;
+  // Each GEMM prefetches the weights of the next one into L2 (the block's weights come from HBM
+  // once per step; the next GEMM then starts on L2 hits).
+  const size_t dd = static_cast<size_t>(c.s.D) * c.s.D * 2, fd = static_cast<size_t>(c.s.F) * c.s.D * 2;
   const Shape& s = c.s;
   void* xw = c.at<void>(c.lay.y);
   void* qkv = c.at<void>(c.lay.qkv);
@@ -550,7 +552,7 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   q.stride = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_QKV, 0, c.stream));
   DSV4V_TRY(gemm_bf16(c, EPI_QKV_ROPE, c.plans.qkv, xw, s.P, s.D, w->wqkv, nullptr, 3 * s.D, qkv, nullptr, cos,
-                      sin, q));
+                      sin, q, prefetching(w->wo, dd)));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_QKV, 1, c.stream));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_ATTENTION, 0, c.stream));
   DSV4V_TRY(attention_bf16(c, b, qkv, attn));
@@ -561,7 +563,8 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   o.ss_out = ss2;
   o.ss_parts = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_OUT, 0, c.stream));
-  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x, nullptr, nullptr, o));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.out, attn, s.P, s.D, w->wo, nullptr, s.D, x, x, nullptr, nullptr, o,
+                      prefetching(w->w_gate, fd, w->w_up, fd)));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_OUT, 1, c.stream));
   NormFold m;
   m.ss = ss2;
@@ -569,7 +572,7 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
   m.stride = c.lay.ss_parts;
   DSV4V_TRY(record(ev, DSV4V_PROFILE_SWIGLU, 0, c.stream));
   DSV4V_TRY(gemm_bf16(c, EPI_SWIGLU, c.plans.gateup, xw, s.P, s.D, w->w_gate, w->w_up, s.F, h, nullptr, nullptr,
-                      nullptr, m));
+                      nullptr, m, prefetching(w->w_down, fd)));
   DSV4V_TRY(record(ev, DSV4V_PROFILE_SWIGLU, 1, c.stream));
   NormFold d;
   if (next_norm_w) {
@@ -579,7 +582,8 @@ dsv4v_status block_bf16(const Ctx& c, const dsv4v_batch* b, const dsv4v_block_we
     d.ss_parts = c.lay.ss_parts;
   }
   DSV4V_TRY(record(ev, DSV4V_PROFILE_DOWN, 0, c.stream));
-  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x, nullptr, nullptr, d));
+  DSV4V_TRY(gemm_bf16(c, EPI_RESID, c.plans.down, h, s.P, s.F, w->w_down, nullptr, s.D, x, x, nullptr, nullptr, d,
+                      prefetching(next ? next->wqkv : nullptr, 3 * dd)));
   return record(ev, DSV4V_PROFILE_DOWN, 1, c.stream);
 }
 
@@ -865,7 +869,7 @@ int dsv4v_step_launches(const dsv4v_config* cfg, const dsv4v_batch* batch, int f
     else n += 8 * s.L;                              // fp32: 2 norms, 4 GEMMs, rotation, attention per layer
   }
   if (final_norm) n += 1;
-  if (aligner) n += (s.bf16 && aligner_gathers(s, pl.align)) ? 2 : 3;  // window index, [merged rows], GEMM
+  if (aligner) n += 3;  // window index, merged rows, GEMM
   return n;
 }
 
@@ -930,11 +934,11 @@ static dsv4v_status tower_impl(const dsv4v_config* cfg, const dsv4v_batch* batch
   if (c.s.bf16 && c.plans.chain.use && c.s.L > 0) {
     DSV4V_TRY(blocks_chain(c, batch, layers, c.s.L, cos, sin, x_inout, events));
   } else {
-  for (int l = 0; l < c.s.L; ++l)
-    DSV4V_TRY(c.s.bf16 ? block_bf16(c, batch, &layers[l], cos, sin, x_inout, l == 0,
-                                    l + 1 < c.s.L ? layers[l + 1].norm1_w : nullptr,
-                                    events ? events + static_cast<size_t>(l) * DSV4V_PROFILE_KINDS * 2 : nullptr)
-                       : block_f32(c, batch, &layers[l], cos, sin, x_inout));
+    for (int l = 0; l < c.s.L; ++l)
+      DSV4V_TRY(c.s.bf16 ? block_bf16(c, batch, &layers[l], cos, sin, x_inout, l == 0,
+                                      l + 1 < c.s.L ? &layers[l + 1] : nullptr,
+                                      events ? events + static_cast<size_t>(l) * DSV4V_PROFILE_KINDS * 2 : nullptr)
+                         : block_f32(c, batch, &layers[l], cos, sin, x_inout));
   }
   if (final_norm_w)
     DSV4V_TRY(cuda_status(launch_rmsnorm(c.s.bf16, x_inout, final_norm_w, x_inout, c.s.P, c.s.D, c.eps, c.stream)));
@@ -976,21 +980,12 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
                                              s.bf16 ? static_cast<int>(c.lay.counters_bytes / sizeof(int)) : 0)));
   const int K = s.r * s.r * s.D;
   if (s.bf16) {
-    const GemmPlan& pl = c.plans.align;
-    if (aligner_gathers(s, pl)) {
-      // Each CTA of the cluster split-K takes K blocks of one window slot: its A rows come
-      // straight from x by TMA gather, four source rows per copy, no merged operand.
-      GemmExtra ex;
-      ex.gather_src = src;
-      ex.gather_r2 = s.r * s.r;
-      ex.gather_rows = s.P;
-      return gemm_bf16(c, EPI_STORE, pl, x, s.T, K, w_align, nullptr, s.E, out, nullptr, nullptr, nullptr,
-                       NormFold(), ex);
-    }
-    // Otherwise materialise the merged window rows, then a TMA GEMM.
+    // Materialise the merged window rows, then a TMA GEMM (the weights stream once; the rows
+    // are a few MB).  Gathering the rows inside the GEMM with TMA tile::gather4 (four source rows
+    // per copy) measured 2.3x slower on B200: 53 us against 5 + 23 us.
     void* merged = c.at<uint8_t>(c.lay.merged);
     DSV4V_TRY(cuda_status(launch_merge_rows_bf16(x, src, merged, s.T, s.r * s.r, s.D, c.stream)));
-    return gemm_bf16(c, EPI_STORE, pl, merged, s.T, K, w_align, nullptr, s.E, out, nullptr);
+    return gemm_bf16(c, EPI_STORE, c.plans.align, merged, s.T, K, w_align, nullptr, s.E, out, nullptr);
   }
   float* merged = c.at<float>(c.lay.merged);
   DSV4V_TRY(cuda_status(launch_gather_f32(static_cast<const float*>(x), src, merged, s.T, s.r * s.r, s.D, c.stream)));

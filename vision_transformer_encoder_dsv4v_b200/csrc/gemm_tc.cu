@@ -34,6 +34,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kMaxDynSmem = 232448;         // 227 KB per CTA
 constexpr int kStagingBytes = 4 * 2 * 4096;  // per epilogue warp: two 32-row x 128-byte staging boxes
+constexpr int kXwBytes = 256 * 4;            // the next norm's weights of a tile's columns
 
 // PAIR: the CTA is one half of a CTA pair that computes a 256 x BN tile (tcgen05 cta_group::2):
 // it holds 128 rows of A and BN / 2 rows of B per stage, and 128 x BN accumulators.
@@ -43,12 +44,13 @@ struct TileCfg {
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int RING_BUDGET = kMaxDynSmem - 1024 - 512 - kStagingBytes;
+  static constexpr int RING_BUDGET = kMaxDynSmem - 1024 - 512 - kXwBytes - kStagingBytes;
   static constexpr int STAGES = RING_BUDGET / STAGE > 8 ? 8 : RING_BUDGET / STAGE;
   static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : ((2 * BN <= 256) ? 256 : 512);
   static constexpr int OFF_STAGING = STAGES * STAGE;
   static constexpr int OFF_BARRIERS = OFF_STAGING + kStagingBytes;
-  static constexpr int SMEM = 1024 + OFF_BARRIERS + 1024;
+  static constexpr int OFF_XW = OFF_BARRIERS + 512;
+  static constexpr int SMEM = 1024 + OFF_XW + kXwBytes;
 };
 
 struct Params {
@@ -73,11 +75,8 @@ struct Params {
   float* ss_out;
   int ss_parts;
   const float* bias;
-  // Gathered A (GATHER): row r of the tile's K block kb is row src[(tile row r) * gather_r2 + slot]
-  // of the A tensor (its columns (kb % kb_per_slot) * 64 ...), slot = kb / kb_per_slot; rows
-  // past the source rows (window positions in the zero padding, tokens past the end) read zeros.
-  const int32_t* gather_src;
-  int gather_r2, gather_kb_per_slot, gather_rows;
+  const void* l2_next[2];
+  size_t l2_next_bytes[2];
 };
 
 // ---------------------------------------------------------------------------- stream-K ranges
@@ -129,8 +128,8 @@ struct SegmentWalker {
 template <int EPI, int BN, int NR>
 __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_tile, int g, float (&v)[64],
                                                const float (&rot_c)[NR], const float (&rot_s)[NR], float row_scale,
-                                               const uint4* resid, float& ss_acc, Stager& st, uint8_t* box,
-                                               uint8_t* box2) {
+                                               const uint4* resid, const float* xw_s, float& ss_acc, Stager& st,
+                                               uint8_t* box, uint8_t* box2) {
   if (row >= p.M) return;
   if constexpr (EPI == EPI_SWIGLU || EPI == EPI_QKV_ROPE) {
 #pragma unroll
@@ -207,8 +206,9 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
     }
     if constexpr (EPI == EPI_RESID) {
       if (p.xw_out) {
-        // Next RMSNorm's operand from the stored (bf16) x: bf16(x * w) and sum of x^2.
-        const float4* w4 = reinterpret_cast<const float4*>(p.xw_w + n_tile * BN + g * 64);
+        // Next RMSNorm's operand from the stored (bf16) x: bf16(x * w) and sum of x^2; w of the
+        // tile's columns was staged in shared memory before the accumulator was ready.
+        const float4* w4 = reinterpret_cast<const float4*>(xw_s + g * 64);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
@@ -258,18 +258,7 @@ __device__ __forceinline__ float* partial_slot(const Params& p, int c) {
 
 
 
-// Four rows (row0..row3) x 64 columns starting at column x of `map` (box: 64 columns x 1 row)
-// into 512 consecutive bytes of shared memory; completes 512 bytes on the mbarrier.
-__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int r0,
-                                           int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
-template <int BN, int EPI, bool PAIR, int KS, bool GATHER = false>
+template <int BN, int EPI, bool PAIR, int KS>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
@@ -287,10 +276,10 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
   uint64_t* teardown = mma_done + 1;  // one arrival per warp once its role is done
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(teardown + 1);
+  uint64_t* xchg = teardown + 1;      // cluster split-K: the peers' partial slices have landed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xchg + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* ticket = reinterpret_cast<volatile int*>(tmem_holder + 2);
-  int32_t* grow = reinterpret_cast<int32_t*>(smem + C::OFF_BARRIERS + 512);  // GATHER: the tile's 128 source rows
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -314,6 +303,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(mma_done, 1);
     mbar_init(teardown, blockDim.x / 32);
+    mbar_init(xchg, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -349,24 +339,6 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    static_assert(!GATHER || (!PAIR && KS > 1), "gathered A is built for the cluster split-K plans");
-    int gslot = -1;  // window slot whose source rows are in grow
-    if constexpr (GATHER) {
-      // This CTA's K range lies in one window slot (checked by the launcher): the warp loads the
-      // tile's 128 source rows once.
-      SegmentWalker w0(p, owner);
-      Segment s0{};
-      if (w0.next(p, s0)) {
-        gslot = s0.kb0 / p.gather_kb_per_slot;
-        grid_dependency_wait();
-        for (int r = lane; r < BM; r += 32) {
-          const int t = s0.m_tile * BM + r;
-          const int src = t < p.M ? p.gather_src[static_cast<size_t>(t) * p.gather_r2 + gslot] : -1;
-          grow[r] = src >= 0 ? src : p.gather_rows;  // a row past the end reads zeros
-        }
-      }
-      __syncwarp();
-    }
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_phase = 0;
@@ -376,14 +348,7 @@ __global__ void __launch_bounds__(192, 1)
       const bool arrives = !PAIR || rank == 0;  // posts the expected bytes of the stage
       constexpr uint32_t kStageTx = PAIR ? 2 * C::STAGE : C::STAGE;
       auto load_a = [&](uint8_t* sa, int kb, int m_tile, int s) {
-        if constexpr (GATHER) {
-          const int x = (kb % p.gather_kb_per_slot) * BK;
-#pragma unroll 1
-          for (int g = 0; g < BM / 4; ++g)
-            tma_gather4(sa + g * 512, &tm_a, &full[s], x, grow[4 * g], grow[4 * g + 1], grow[4 * g + 2],
-                        grow[4 * g + 3]);
-          (void)m_tile;
-        } else if constexpr (PAIR)
+        if constexpr (PAIR)
           tma_load_2d_pair(sa, &tm_a, full_leader + 8u * s, kb * BK, m_tile * BMT + static_cast<int>(rank) * BM);
         else
           tma_load_2d(sa, &tm_a, &full[s], kb * BK, m_tile * BM);
@@ -440,6 +405,19 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
+      // The next GEMM's weights: this CTA's share into L2 while its own stages drain.
+      if (ok) {
+        for (int r = 0; r < 2; ++r) {
+          if (!p.l2_next[r]) continue;
+          const size_t share = (p.l2_next_bytes[r] + 16 * gridDim.x - 1) / (16 * gridDim.x) * 16;
+          const size_t b0 = static_cast<size_t>(blockIdx.x) * share;
+          const size_t b1 = min(p.l2_next_bytes[r], b0 + share);
+          for (size_t o = b0; o < b1; o += 32768) {
+            const size_t piece = b1 - o < 32768 ? b1 - o : 32768;
+            prefetch_l2_bulk(static_cast<const uint8_t*>(p.l2_next[r]) + o, static_cast<uint32_t>(piece));
+          }
+        }
+      }
       // Copies still in flight must land before the CTA may exit (error path only; in the
       // normal path every issued stage was consumed already and these return at once).  The
       // second CTA of a pair has no full barrier of its own: it waits until the MMAs released
@@ -453,7 +431,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     if constexpr (KS > 1) {
       __syncwarp();
-      cluster_sync();  // the two reduce-scatter barriers of the epilogue
+      cluster_sync();  // the two cluster barriers of the epilogue
       cluster_sync();
     }
   } else if (warp == 1) {
@@ -519,7 +497,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
     if constexpr (KS > 1) {
-      cluster_sync();  // the two reduce-scatter barriers of the epilogue (this CTA's MMAs are done)
+      cluster_sync();  // the two cluster barriers of the epilogue (this CTA's MMAs are done)
       cluster_sync();
     }
   } else if (warp < 6) {
@@ -576,22 +554,26 @@ __global__ void __launch_bounds__(192, 1)
       }
       float row_scale = norm_row_scale(p, row);
       pin(row_scale);
+      float* xw_s = reinterpret_cast<float*>(smem + C::OFF_XW);
+      if (EPI == EPI_RESID && p.xw_out && have)
+        for (int i = et; i < BN; i += 128) xw_s[i] = p.xw_w[sg.n_tile * BN + i];
       float ss_acc = 0.0f;
+      // The named barrier also publishes xw_s to the four epilogue warps.
       bool got = have && mbar_wait(&tfull[0], 0, abort_flag, p.err, kErrTimeoutEpilogue);
       got = named_barrier_and(2, 128, got);
       tc_fence_after_sync();
-      // Barrier 1: every CTA of the cluster has finished its MMAs, so their TMA rings are free
-      // to receive.  Rank j's ring holds, per sending rank (slot), its partial of j's groups in
-      // the layout [slot][group][16-byte column quad][row][4], conflict-free for a warp's rows.
-      cluster_sync();
+      // Reduce-scatter through the TMA rings, free once the MMAs are done.  Each CTA's ring holds
+      // a receive area, one slot per sending rank, and a send area, one slice per peer, both in
+      // the layout [group][16-byte column quad][row][4] (conflict-free for a warp's rows).  The
+      // slices are staged locally, then moved by bulk copies that count on the peer's xchg.
+      static_assert(2 * (KS - 1) * SLOT_BYTES <= STAGES * C::STAGE, "exchange areas exceed the ring");
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+      uint8_t* send = smem + (KS - 1) * SLOT_BYTES;
       if (got) {
 #pragma unroll 1
         for (int j = 0; j < KS; ++j) {
           if (j == static_cast<int>(kslice)) continue;
-          const int slot = static_cast<int>(kslice) < j ? static_cast<int>(kslice) : static_cast<int>(kslice) - 1;
-          const uint32_t dst_base = mapa_shared(smem_u32(smem), static_cast<uint32_t>(j)) +
-                                    static_cast<uint32_t>(slot * SLOT_BYTES + row_in_tile * 16);
+          const int peer = j < static_cast<int>(kslice) ? j : j - 1;  // send slice of peer j
 #pragma unroll 1
           for (int gi = 0; gi < GPR; ++gi) {
             int c0, c1;
@@ -601,20 +583,38 @@ __global__ void __launch_bounds__(192, 1)
             tmem_ld32(t_row + c1 * 32, r1);
             tmem_ld_wait(r0);
             tmem_ld_wait(r1);
-            const uint32_t dst = dst_base + static_cast<uint32_t>(gi * 16 * BM * 16);
+            uint8_t* dst = send + peer * SLOT_BYTES + gi * 16 * BM * 16 + row_in_tile * 16;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              st_shared_cluster_v4(dst + q * (BM * 16),
-                                   make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
-                                               __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3])));
-              st_shared_cluster_v4(dst + (8 + q) * (BM * 16),
-                                   make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
-                                               __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3])));
+              *reinterpret_cast<float4*>(dst + q * (BM * 16)) =
+                  make_float4(__uint_as_float(r0[4 * q]), __uint_as_float(r0[4 * q + 1]),
+                              __uint_as_float(r0[4 * q + 2]), __uint_as_float(r0[4 * q + 3]));
+              *reinterpret_cast<float4*>(dst + (8 + q) * (BM * 16)) =
+                  make_float4(__uint_as_float(r1[4 * q]), __uint_as_float(r1[4 * q + 1]),
+                              __uint_as_float(r1[4 * q + 2]), __uint_as_float(r1[4 * q + 3]));
             }
           }
         }
       }
-      cluster_sync();  // barrier 2: every partial slice has landed
+      fence_proxy_async_smem();  // the staged slices are read by the bulk-copy (async) proxy
+      // Barrier 1: every CTA of the cluster has finished its MMAs (its receive area is free) and
+      // staged its send slices.
+      cluster_sync();
+      if (et == 0) {
+        if (have) mbar_arrive_expect_tx(xchg, (KS - 1) * SLOT_BYTES);
+        if (got) {
+          for (int j = 0; j < KS; ++j) {
+            if (j == static_cast<int>(kslice)) continue;
+            const int peer = j < static_cast<int>(kslice) ? j : j - 1;
+            const int slot = static_cast<int>(kslice) < j ? static_cast<int>(kslice) : static_cast<int>(kslice) - 1;
+            bulk_copy_to_peer(mapa_shared(smem_u32(smem + slot * SLOT_BYTES), static_cast<uint32_t>(j)),
+                              send + peer * SLOT_BYTES, SLOT_BYTES, mapa_shared(smem_u32(xchg), static_cast<uint32_t>(j)));
+          }
+        }
+      }
+      // Every peer sends its slices whenever it has a tile (the cluster shares one tile).
+      got = got && mbar_wait(xchg, 0, abort_flag, p.err, kErrTimeoutEpilogue);
+      got = named_barrier_and(2, 128, got);
       if (got) {
         uint8_t* box = nullptr;
 #pragma unroll
@@ -655,15 +655,18 @@ __global__ void __launch_bounds__(192, 1)
           if (EPI == EPI_RESID && p.xw_out) st.acquire_both(box, box2);
           else box = st.acquire();
           epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s, row_scale,
-                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? gi * 8 : 0) : nullptr, ss_acc, st,
-                                  box, box2);
+                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? gi * 8 : 0) : nullptr, xw_s, ss_acc,
+                                  st, box, box2);
           st.store(box, &tm_out, sg.n_tile * BN + g * 64, box_y, p.M);
           if (EPI == EPI_RESID && p.xw_out) st.store(box2, &tm_xw, sg.n_tile * BN + g * 64, box_y, p.M);
         }
         if (EPI == EPI_RESID && p.xw_out && row < p.M)
           p.ss_out[static_cast<size_t>(row) * p.ss_parts + sg.n_tile * KS + static_cast<int>(kslice)] = ss_acc;
       }
+      // Barrier 2: no CTA leaves while a peer's bulk copies may still read its send area.
+      cluster_sync();
     }
+    bool xw_loaded = false;
     while (KS == 1 && walk.next(p, sg)) {
       const int row0 = sg.m_tile * BMT + static_cast<int>(rank) * BM;  // this CTA's rows of the tile
       const int row = row0 + row_in_tile;
@@ -707,10 +710,17 @@ __global__ void __launch_bounds__(192, 1)
       }
       float row_scale = norm_row_scale(p, row);
       pin(row_scale);
+      float* xw_s = reinterpret_cast<float*>(smem + C::OFF_XW);
+      if (EPI == EPI_RESID && p.xw_out && finisher_or_full) {
+        // After the first tile, every warp must be done with the previous tile's weights.
+        if (xw_loaded) named_barrier_sync(3, 128);
+        for (int i = et; i < BN; i += 128) xw_s[i] = p.xw_w[sg.n_tile * BN + i];
+        xw_loaded = true;
+      }
       float ss_acc = 0.0f;
       const bool got = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, kErrTimeoutEpilogue);
       // All four epilogue warps continue or stop together (TMEM loads are warp-collective and
-      // the partial-tile path uses a named barrier).
+      // the partial-tile path uses a named barrier); the barrier also publishes xw_s.
       if (!named_barrier_and(2, 128, got)) break;
       tc_fence_after_sync();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
@@ -796,8 +806,8 @@ __global__ void __launch_bounds__(192, 1)
           if (EPI == EPI_RESID && p.xw_out) st.acquire_both(box, box2);
           else if (EPI != EPI_SWIGLU || (g & 1) == 0) box = st.acquire();
           epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s, row_scale,
-                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? (g % RG) * 8 : 0) : nullptr, ss_acc,
-                                  st, box, box2);
+                                  EPI == EPI_RESID ? resid + (EPI == EPI_RESID ? (g % RG) * 8 : 0) : nullptr, xw_s,
+                                  ss_acc, st, box, box2);
           if constexpr (EPI == EPI_RESID) {
             if (g + RG < NGROUPS) {
               const uint4* r4 = reinterpret_cast<const uint4*>(
@@ -846,14 +856,11 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int BN, int EPI, bool PAIR = false, int KS = 1, bool GATHER = false>
+template <int BN, int EPI, bool PAIR = false, int KS = 1>
 cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   using C = TileCfg<BN, PAIR>;
   static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
-  auto kern = k_gemm_tc<BN, EPI, PAIR, KS, GATHER>;
-  if (GATHER && (!a.gather_src || a.gather_kb_per_slot <= 0 || (plan.kb_total / KS) <= 0 ||
-                 a.gather_kb_per_slot % (plan.kb_total / KS)))
-    return cudaErrorInvalidValue;  // every CTA's K slice must lie within one window slot
+  auto kern = k_gemm_tc<BN, EPI, PAIR, KS>;
   if (PAIR && (plan.grid & 1)) return cudaErrorInvalidValue;
   if (KS > 1 && (plan.grid % KS || plan.kb_total % KS || plan.grid != plan.work * KS)) return cudaErrorInvalidValue;
   int dev = 0;
@@ -891,10 +898,12 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.ss_out = a.ss_out;
   p.ss_parts = a.ss_parts;
   p.bias = a.bias;
-  p.gather_src = a.gather_src;
-  p.gather_r2 = a.gather_r2;
-  p.gather_kb_per_slot = a.gather_kb_per_slot;
-  p.gather_rows = a.gather_rows;
+  for (int r = 0; r < 2; ++r) {
+    p.l2_next[r] = a.l2_next[r];
+    p.l2_next_bytes[r] = a.l2_next_bytes[r];
+    if (a.l2_next[r] && ((reinterpret_cast<uintptr_t>(a.l2_next[r]) & 15u) || (a.l2_next_bytes[r] & 15u)))
+      return cudaErrorInvalidValue;
+  }
   const CUtensorMap& ta = *a.tm_a;
   const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
   const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
@@ -912,15 +921,6 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
     // Cluster split-K: 256-column residual, store and GELU tiles.
     if constexpr (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU) {
       if (plan.bn != 256 || plan.pair) return cudaErrorInvalidValue;
-      if constexpr (EPI == EPI_STORE) {
-        if (a.gather_src) {
-          switch (plan.ks) {
-            case 2: return launch_one<256, EPI, false, 2, true>(plan, a, s);
-            case 4: return launch_one<256, EPI, false, 4, true>(plan, a, s);
-            default: return cudaErrorInvalidValue;
-          }
-        }
-      }
       switch (plan.ks) {
         case 2: return launch_one<256, EPI, false, 2>(plan, a, s);
         case 4: return launch_one<256, EPI, false, 4>(plan, a, s);

@@ -66,11 +66,10 @@ struct GemmArgs {
   float* ss_out;
   int ss_parts;
   const float* bias;  // STORE: per-column fp32 bias added before rounding (NULL: none)
-  // Gathered A (STORE with a cluster split-K plan whose K slices lie within one window slot):
-  // tm_a is the source tensor [gather_rows, K / gather_r2] with a 64 x 1 box, and row r of the
-  // tile reads source row gather_src[r * gather_r2 + slot] (gather_rows when negative: zeros).
-  const int32_t* gather_src;
-  int gather_r2, gather_kb_per_slot, gather_rows;
+  // Up to two ranges (the next GEMM's weights) that the CTAs prefetch into L2, a share each,
+  // once their own operand loads are issued (NULL: none; 16-byte aligned, bytes a multiple of 16).
+  const void* l2_next[2];
+  size_t l2_next_bytes[2];
 };
 
 cudaError_t launch_gemm_tc(int epi, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
@@ -181,9 +180,11 @@ cudaError_t launch_swiglu_bwd(const void* g, const void* u, const void* dh, void
                               int sms, cudaStream_t s);
 cudaError_t launch_rotary_bwd(void* dqkv, const float* cos, const float* sin, int64_t P, int D, int hd, int sms,
                               cudaStream_t s);
-// Image-token bridge (bridge.cu).  Positions per CTA of the merge; counts holds one int4 per
-// chunk of that many positions.
+// Image-token bridge (bridge.cu).  Positions per CTA of the merge and the visibility scan;
+// counts holds one int4 per chunk of that many positions.  Up to kBridgeFusedPositions the
+// merge is one launch and leaves counts untouched.
 constexpr int kBridgeChunk = 256;
+constexpr int64_t kBridgeFusedPositions = int64_t{1} << 16;
 cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, int4* counts, const int32_t* grid_dev,
                                 int n_images, int r, int64_t n_tokens, const void* image_tokens, const void* sentinels,
                                 void* embeds, int row_vec, uint32_t* err, cudaStream_t s);
