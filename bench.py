@@ -569,6 +569,30 @@ def patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, steps):
             "note": "standalone, 20 calls per graph replay; the alternative projector, not in value"}
 
 
+def graph_timed(torch, stream, flush, fn, steps):
+    """Average ms of fn() captured in a CUDA graph: one replay per timed interval (CUDA events on
+    the stream), each after an L2 flush outside the events; no host launch cost inside."""
+    with torch.cuda.stream(stream):
+        fn()  # warm descriptors and function attributes before the capture
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        fn()
+    out = []
+    for i in range(steps + 3):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            graph.replay()
+            ev1.record(stream)
+        stream.synchronize()
+        if i >= 3:
+            out.append(ev0.elapsed_time(ev1))
+    del graph
+    return sum(out) / len(out)
+
+
 def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
     """The image-token bridge on a language batch of n_seqs x seq_len positions holding the 16
     images of the high-resolution batch (N-layouts from dsv4v_image_layout, placed by
@@ -592,18 +616,7 @@ def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
     mask = torch.full((n_seqs, seq_len, seq_len), float("-inf"), device="cuda")
 
     def timed(fn):
-        out = []
-        for i in range(steps + 3):
-            with torch.cuda.stream(stream):
-                flush.zero_()
-                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                ev0.record(stream)
-                fn()
-                ev1.record(stream)
-            stream.synchronize()
-            if i >= 3:
-                out.append(ev0.elapsed_time(ev1))
-        return sum(out) / len(out)
+        return graph_timed(torch, stream, flush, fn, steps)
 
     merge_ms = timed(lambda: A.dsv4v_merge_image_embeddings(cfg, b, types, toks, sent, embeds, ws,
                                                             stream=stream.cuda_stream))
@@ -627,7 +640,8 @@ def bridge_timing(A, torch, cfg, stream, flush, steps, n_seqs=4, seq_len=8192):
             "visibility": {"avg_us": vis_ms * 1e3, "bytes_written": vis_bytes,
                            "gbs": vis_bytes / (vis_ms * 1e-3) / 1e9, "launches_per_call": 3},
             "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if hbm else None,
-            "note": "standalone, one call per timed interval after an L2 flush; not in value"}
+            "note": "standalone, the call captured in a CUDA graph, one replay per timed interval after an L2 "
+                    "flush; not in value"}
 
 
 def block_backward_timing(A, torch, cfg, batch, wl, lw, stream, flush, steps):
@@ -653,18 +667,7 @@ def block_backward_timing(A, torch, cfg, batch, wl, lw, stream, flush, steps):
     A.dsv4v_rope2d_table(cfg, batch, cos, sin, stream=stream.cuda_stream)
     ws = torch.empty(A.dsv4v_backward_workspace_size(cfg, batch), dtype=torch.uint8, device="cuda")
     def timed(fn):
-        out = []
-        for i in range(steps + 3):
-            with torch.cuda.stream(stream):
-                flush.zero_()
-                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                ev0.record(stream)
-                fn()
-                ev1.record(stream)
-            stream.synchronize()
-            if i >= 3:
-                out.append(ev0.elapsed_time(ev1))
-        return sum(out) / len(out)
+        return graph_timed(torch, stream, flush, fn, steps)
 
     ms = timed(lambda: A.dsv4v_block_backward(cfg, batch, lw[0], cos, sin, x, do, dx, grads, ws,
                                               stream=stream.cuda_stream))
@@ -684,8 +687,9 @@ def block_backward_timing(A, torch, cfg, batch, wl, lw, stream, flush, steps):
                                    "note": "dsv4v_attention_backward: forward attention rebuilding the row "
                                            "log-sum-exp, rowsum(do * o), dK/dV kernel, dQ kernel; flops counted "
                                            "are the backward's 8 N^2 D"},
-            "note": "standalone, one call per timed interval after an L2 flush; recompute + backward of one "
-                    "block; attention backward on tcgen05; not in value"}
+            "note": "standalone, the call's launches captured in one CUDA graph, one replay per timed interval "
+                    "after an L2 flush; recompute + backward of one block; attention backward on tcgen05; "
+                    "not in value"}
 
 
 def load_peaks():

@@ -434,9 +434,8 @@ size_t dsv4v_bridge_workspace_size(int64_t n_positions);
  * E = cfg->llm_dim; E times the element size must be a multiple of 16 bytes, and the three
  * matrices 16-byte aligned (else DSV4V_ERR_UNSUPPORTED / DSV4V_ERR_INVALID_ARG).
  * n_seqs * seq_len < 2^31.  workspace: device, 256-byte aligned, at least
- * dsv4v_bridge_workspace_size(n_seqs * seq_len) bytes (up to 65,536 positions the merge is one
- * launch and leaves it untouched; above that a count launch first writes per-chunk totals
- * there).  Types that do not fit the images (an unknown code, a pseudo token outside a span, an unclosed or nested span, a span whose
+ * dsv4v_bridge_workspace_size(n_seqs * seq_len) bytes.  Types that do not fit the images (an
+ * unknown code, a pseudo token outside a span, an unclosed or nested span, a span whose
  * feature count differs from its image's, more or fewer spans than images) are found on the
  * device: the offending rows are left as they were, and the next dsv4v_device_error returns
  * DSV4V_ERR_LAYOUT. */

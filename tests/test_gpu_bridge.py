@@ -64,13 +64,13 @@ MERGE_CASES = {
     "tiny": ([(1, 1)], 1, 5, 0, 1),
     "one_chunk_exact": ([(28, 28)], 1, 256, 1, 40),
     "many_images": ([(1 + i % 7, 2 + i % 5) for i in range(300)], 4, 1600, 5, 8),
-    # above 65,536 positions the positions before each chunk come from a count launch
-    "count_launch": ([(40 + i % 9, 30 + i % 13) for i in range(40)], 3, 24001, 3, 400),
+    # 72,003 positions: 282 chunks, long text gaps (chunks of text only)
+    "long_stream": ([(40 + i % 9, 30 + i % 13) for i in range(40)], 3, 24001, 3, 400),
 }
 
 
-# bf16 rows of 4096 (16 column slices in clusters of 8) and of 1024 (4 slices, one cluster);
-# f32 rows of 132 (one slice)
+# bf16 rows of 4096 (16 column slices) and of 1024 (4 slices); f32 rows of 132 (one slice of 33
+# vectors, not a divisor of the CTA's 256 threads)
 @pytest.mark.parametrize("name", list(MERGE_CASES))
 @pytest.mark.parametrize("dtype,llm_dim", [(A.DSV4V_BF16, 4096), (A.DSV4V_BF16, 1024), (A.DSV4V_F32, 132)])
 def test_merge_image_embeddings_bit_exact(name, dtype, llm_dim):

@@ -114,7 +114,8 @@ def test_linear_residual(rows, k):
     assert_bf16_close(to_np(xt), want, abs_floor=2e-5)
 
 
-@pytest.mark.parametrize("rows", [784, 3562, 1, 200])
+# 784, 1000 (ragged last row tile) and 1152 rows take 176-column tiles, one per CTA
+@pytest.mark.parametrize("rows", [784, 1000, 1152, 3562, 1, 200])
 def test_swiglu(rows):
     cfg = cfg_bf16()
     y = random_bf16((rows, 1024), 1.0, seed=41)

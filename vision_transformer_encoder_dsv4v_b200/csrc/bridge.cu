@@ -6,21 +6,19 @@
 // 4 image_pad.  A span runs from an image_start to the next image_end of the same sequence and
 // holds pseudo tokens only; every pseudo token lies inside one.
 //
-// Both calls work on chunks of kBridgeChunk positions.  Per chunk they need the features,
-// starts and ends over all positions before it (the exclusive prefix), then a ballot scan inside
-// the chunk.  That gives every position its feature index and its span index without any
-// serial pass, and checks the span structure.
-//  * merge: one launch up to 2^16 positions.  The `slices` CTAs that serve a chunk form
-//    clusters; the CTAs of a cluster count the positions before the chunk together, a share
-//    each, and add the shares through distributed shared memory (past 2^16 positions, where
-//    those reads grow with n^2, a count launch writes per-chunk totals first).  Each pseudo-token
-//    row is then read once (aligner token or sentinel) and written once, each CTA moving its own
-//    column slice of the chunk's rows from a table of row addresses, eight 16-byte loads in
-//    flight per thread.  The pseudo rows of a batch gather in few chunks (images sit together
-//    in a sequence), hence the column slices; for a chunk of text only, one cluster checks the
-//    layout and the other CTAs leave at once.
-//  * visibility: a count launch writes per-chunk totals, and the scan adds those of the chunks
-//    before it; the scan records each span's first and last position; then one warp per mask
+// Both calls start with the same two steps over chunks of kBridgeChunk positions: a count of
+// features, starts and ends per chunk, then, per chunk, the exclusive prefix of those counts
+// over the chunks before it plus a ballot scan inside the chunk.  That gives every position its
+// feature index and its span index without any serial pass, and checks the span structure.
+// The data movement that follows is bound by HBM:
+//  * merge: each pseudo-token row is read once (aligner token or sentinel) and written once.
+//    The pseudo rows of a batch gather in few chunks (images sit together in a sequence), so
+//    every chunk is served by `slices` CTAs, each moving its own column slice of the rows from a
+//    table of row addresses, eight 16-byte loads in flight per thread.  For a chunk of text
+//    only, the CTA of slice 0 checks the layout and the others leave at once.  (Counting the
+//    positions before each chunk inside the merge, by the CTAs of a cluster, saves the count
+//    launch but measured slower on B200: 36.3 us against 32.2 us on the 16-image stream.)
+//  * visibility: the scan records each span's first and last position; then one warp per mask
 //    row writes the zeros of its span block with 16-byte stores.
 #include "common.cuh"
 #include "internal.h"
@@ -68,7 +66,6 @@ struct PosScan {
 struct ScanSmem {
   int part[3][kWarps];
   int64_t base[3];  // features, starts, ends before the chunk
-  int share[3];     // this CTA's share of them (merge)
 };
 
 // sm.base from the per-chunk totals of the count launch.  All threads of the CTA must call it.
@@ -95,70 +92,6 @@ __device__ __forceinline__ void base_from_counts(const int4* __restrict__ counts
     sm.base[tid] = s;
   }
   __syncthreads();
-}
-
-// sm.base counted from the types by the CTAs of this CTA's cluster: rank k of the cluster
-// counts the k-th of as many shares (multiples of 4 positions) of the positions before the
-// chunk, and every CTA adds all shares, read from the others' shared memory.  All threads of
-// every CTA of the cluster must call it.  Unknown codes are not checked here (the chunk that
-// holds one reports it).
-__device__ __forceinline__ void base_from_types_cluster(const int32_t* __restrict__ types, ScanSmem& sm) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t rank = cluster_ctarank(), cs = cluster_nctarank();
-  const int64_t before = static_cast<int64_t>(blockIdx.x) * kBridgeChunk;
-  const int64_t per = ((before + 4 * cs - 1) / (4 * cs)) * 4;
-  const int64_t lo = rank * per < before ? rank * per : before;
-  const int64_t hi = before - lo < per ? before : lo + per;
-  int acc[3] = {0, 0, 0};
-  auto add = [&](int t) {
-    acc[0] += t == kTypeImage;
-    acc[1] += t == kTypeStart;
-    acc[2] += t == kTypeEnd;
-  };
-  if ((reinterpret_cast<uintptr_t>(types) & 15u) == 0) {  // lo and hi are multiples of 4
-    const int4* v = reinterpret_cast<const int4*>(types + lo);
-    const int64_t nv = (hi - lo) / 4;
-    constexpr int kLoads = 4;
-    for (int64_t q0 = tid; q0 < nv; q0 += kLoads * kBridgeChunk) {
-      int4 t[kLoads];
-#pragma unroll
-      for (int u = 0; u < kLoads; ++u) {
-        const int64_t q = q0 + u * kBridgeChunk;
-        t[u] = q < nv ? __ldg(v + q) : make_int4(kTypeText, kTypeText, kTypeText, kTypeText);
-      }
-#pragma unroll
-      for (int u = 0; u < kLoads; ++u) {
-        add(t[u].x);
-        add(t[u].y);
-        add(t[u].z);
-        add(t[u].w);
-      }
-    }
-  } else {
-    for (int64_t p = lo + tid; p < hi; p += kBridgeChunk) add(__ldg(types + p));
-  }
-#pragma unroll
-  for (int k = 0; k < 3; ++k) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
-  }
-  if (lane == 0)
-    for (int k = 0; k < 3; ++k) sm.part[k][warp] = acc[k];
-  __syncthreads();
-  if (tid < 3) {
-    int s = 0;
-    for (int w = 0; w < kWarps; ++w) s += sm.part[tid][w];
-    sm.share[tid] = s;
-  }
-  cluster_sync();  // every share is in its CTA's shared memory
-  if (tid < 3) {
-    const uint32_t addr = smem_u32(&sm.share[tid]);
-    int64_t s = 0;
-    for (uint32_t k = 0; k < static_cast<uint32_t>(cs); ++k)
-      s += static_cast<int32_t>(ld_shared_cluster_u32(mapa_shared(addr, k)));
-    sm.base[tid] = s;
-  }
-  cluster_sync();  // no CTA exits while another still reads its share; sm.base is published
 }
 
 // The ballot scan inside the chunk, from sm.base: checks that the type is known, that a
@@ -200,9 +133,8 @@ __device__ __forceinline__ PosScan chunk_scan(const int32_t* __restrict__ types,
   return r;
 }
 
-// grid (chunks, slices) in clusters of (1, cs) CTAs, cs dividing slices.  The positions before
-// the chunk are counted by the cluster, or (counts non-null) added up from the per-chunk totals
-// of a count launch.  Every CTA of a chunk scans it; the one of slice 0 reports layout errors.  Each CTA then copies columns [s * vs,
+// grid (chunks, slices).  Every CTA of a chunk with pseudo tokens scans it; the one of slice 0
+// reports layout errors (and is the only one to scan a chunk of text).  Each CTA then copies columns [s * vs,
 // (s + 1) * vs) (16-byte vectors, vs = row_vec / slices) of the chunk's pseudo rows: aligner
 // token rows for features, sentinel rows for the other pseudo types.
 __global__ void __launch_bounds__(kBridgeChunk)
@@ -222,11 +154,11 @@ __global__ void __launch_bounds__(kBridgeChunk)
   grid_dependency_wait();
   launch_dependents();
   {
-    // A chunk of text only copies nothing: one cluster of its CTAs still scans it (the layout
-    // checks need the positions before it), the others leave.  Uniform over a cluster.
+    // A chunk of text only copies nothing: slice 0 still scans it (the layout checks), the
+    // other CTAs leave.
     const int64_t p0 = static_cast<int64_t>(blockIdx.x) * kBridgeChunk + tid;
     const int t0 = p0 < n ? types[p0] : kTypeText;
-    if (!__syncthreads_or(t0 != kTypeText) && blockIdx.y >= cluster_nctarank()) return;
+    if (!__syncthreads_or(t0 != kTypeText) && blockIdx.y != 0) return;
   }
 
   if (warp == 0) {  // tok_cu by a warp-wide inclusive scan, 32 images at a time
@@ -245,8 +177,7 @@ __global__ void __launch_bounds__(kBridgeChunk)
       carry += __shfl_sync(0xffffffffu, v, 31);
     }
   }
-  if (counts) base_from_counts(counts, sm);  // their barriers publish tok_cu
-  else base_from_types_cluster(types, sm);
+  base_from_counts(counts, sm);  // its barriers publish tok_cu
   const PosScan ps = chunk_scan(types, n, seq, sm);
 
   bool bad = ps.bad;
@@ -378,32 +309,20 @@ int bridge_slices(int row_vec) {
   return s;
 }
 
-// CTAs of a merge cluster: the slices of a chunk, at most 8 (the portable cluster size).
-int bridge_cluster(int slices) { return slices < 8 ? slices : 8; }
-
 cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, int4* counts, const int32_t* grid_dev,
                                 int n_images, int r, int64_t n_tokens, const void* image_tokens, const void* sentinels,
                                 void* embeds, int row_vec, uint32_t* err, cudaStream_t s) {
   const int64_t chunks = (n + kBridgeChunk - 1) / kBridgeChunk;
   if (chunks == 0) return cudaSuccess;
+  cudaError_t e = launch_pdl(k_bridge_count, dim3(static_cast<unsigned>(chunks)), dim3(kBridgeChunk), 0, s, types, n,
+                             counts, static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr), err);
+  if (e != cudaSuccess) return e;
   const int slices = bridge_slices(row_vec);
-  const int cs = bridge_cluster(slices);
-  if (slices % cs) return cudaErrorInvalidConfiguration;
-  // Counting the positions before every chunk from the types reads about n^2 / (64 cs / slices)
-  // bytes of L2 in all; past kBridgeFusedPositions a count launch is cheaper.
-  const bool fused = n <= kBridgeFusedPositions;
-  if (!fused) {
-    const cudaError_t e = launch_pdl(k_bridge_count, dim3(static_cast<unsigned>(chunks)), dim3(kBridgeChunk), 0, s,
-                                     types, n, counts, static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr),
-                                     err);
-    if (e != cudaSuccess) return e;
-  }
-  return launch_pdl_clusters(k_bridge_merge, dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(slices)),
-                             dim3(kBridgeChunk), (n_images + 1) * sizeof(int32_t), s,
-                             dim3(1, static_cast<unsigned>(cs), 1), types, n, seq,
-                             static_cast<const int4*>(fused ? nullptr : counts), grid_dev, n_images, r, n_tokens,
-                             static_cast<const uint4*>(image_tokens), static_cast<const uint4*>(sentinels),
-                             static_cast<uint4*>(embeds), row_vec, err);
+  return launch_pdl(k_bridge_merge, dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(slices)),
+                    dim3(kBridgeChunk), (n_images + 1) * sizeof(int32_t), s, types, n, seq,
+                    static_cast<const int4*>(counts), grid_dev, n_images, r, n_tokens,
+                    static_cast<const uint4*>(image_tokens), static_cast<const uint4*>(sentinels),
+                    static_cast<uint4*>(embeds), row_vec, err);
 }
 
 cudaError_t launch_image_visibility(const int32_t* types, int64_t batch, int64_t seq, void* mask, int elem_bytes,

@@ -236,18 +236,48 @@ __device__ __forceinline__ float norm_row_scale(const Params& p, int row) {
   return 1.0f / sqrtf(acc * p.norm_inv_d + p.norm_eps);
 }
 
+// SwiGLU tiles of 352 columns: 176 gate + 176 up output columns, the gate half in TMEM columns
+// [0, 176) and the up half in [192, 368) (two MMAs of N = 176 per K step, one tile per CTA).
+template <int EPI, int BN>
+constexpr bool kSwWide = EPI == EPI_SWIGLU && BN == 352;
+// TMEM column of the up half of a SwiGLU accumulator.
+template <int BN>
+constexpr int kSwUp = BN == 352 ? 192 : BN / 2;
+
 // Accumulator chunks (32 columns each) that make up epilogue group g.
 template <int EPI, int BN>
 __device__ __forceinline__ void group_chunks(int g, int& c0, int& c1) {
   if constexpr (EPI == EPI_SWIGLU) {
     c0 = g;
-    c1 = BN / 64 + g;
+    c1 = kSwUp<BN> / 32 + g;
   } else {
     c0 = 2 * g;
     c1 = 2 * g + 1;
   }
 }
 
+
+// SwiGLU output columns [col0, col0 + n) of row `row` (n a multiple of 8) from group values v
+// (gate in v[0..31], up in v[32..63]), straight to global memory: the tail of a 176-column tile,
+// whose last 64-column box would spill into the next tile.
+__device__ __forceinline__ void swiglu_store_direct(const Params& p, int row, int col0, float (&v)[64], float row_scale,
+                                                    int n) {
+  if (row >= p.M) return;
+  __nv_bfloat16* dst = p.out + static_cast<size_t>(row) * p.ldo + col0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (8 * q >= n) break;
+    float h[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = silu(v[8 * q + i] * row_scale) * (v[32 + 8 * q + i] * row_scale);
+    uint4 o;
+    o.x = pack_bf16x2(h[0], h[1]);
+    o.y = pack_bf16x2(h[2], h[3]);
+    o.z = pack_bf16x2(h[4], h[5]);
+    o.w = pack_bf16x2(h[6], h[7]);
+    *reinterpret_cast<uint4*>(dst + 8 * q) = o;
+  }
+}
 
 // Scratch slot of CTA c (a contributor writes at most one partial: its first segment).
 // Layout [BN / 4][128 rows][4]: a warp's 32 rows of one 4-column group are 512 contiguous bytes.
@@ -444,7 +474,8 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait(mma_done, 0, &never, p.err, kErrTimeoutMma);
       }
     } else if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(BMT, BN, false);
+      constexpr bool WIDE = kSwWide<EPI, BN>;
+      constexpr uint32_t idesc = idesc_bf16(BMT, WIDE ? BN / 2 : BN, false);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -455,7 +486,7 @@ __global__ void __launch_bounds__(192, 1)
                                    : mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.err, kErrTimeoutMma);
         if (!free_acc) break;
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(WIDE ? 0 : acc * BN);  // WIDE: one tile per CTA
         for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, kErrTimeoutMma)) {
             ok = false;
@@ -469,10 +500,17 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4).
-            if constexpr (PAIR)
-              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
-            else
-              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > sg.kb0 || k > 0) ? 1u : 0u);
+            const uint32_t accum = (kb > sg.kb0 || k > 0) ? 1u : 0u;
+            if constexpr (PAIR) {
+              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+            } else if constexpr (WIDE) {
+              // gate rows [0, BN / 2) of B, then up rows (1024-byte aligned: BN / 2 is a multiple of 8)
+              const uint64_t bdesc_up = sdesc_sw128(b_addr + (BN / 2) * 128, 16, 1024);
+              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+              umma_bf16(d_tmem + kSwUp<BN>, adesc + 2 * k, bdesc_up + 2 * k, idesc, accum);
+            } else {
+              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+            }
           }
           if constexpr (PAIR) umma_commit_pair(&empty[stage]);
           else umma_commit(&empty[stage]);
@@ -723,7 +761,8 @@ __global__ void __launch_bounds__(192, 1)
       // the partial-tile path uses a named barrier); the barrier also publishes xw_s.
       if (!named_barrier_and(2, 128, got)) break;
       tc_fence_after_sync();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(kSwWide<EPI, BN> ? 0 : acc * BN);
       if (!finisher_or_full) {
         // Contributor to a tile finished by another CTA: park the partial, release it, move on.
         float* slot = partial_slot<BN>(p, blockIdx.x);
@@ -762,9 +801,11 @@ __global__ void __launch_bounds__(192, 1)
           __threadfence();
         }
         uint8_t* box = nullptr;
+        constexpr bool WIDE = kSwWide<EPI, BN>;
+        constexpr int NG = WIDE ? 6 : NGROUPS;  // WIDE: 5.5 groups of 32 output columns
         // Unrolled for the residual epilogue so that its prefetched residual row stays in registers.
 #pragma unroll(EPI == EPI_RESID ? NGROUPS : 1)
-        for (int g = 0; g < NGROUPS; ++g) {
+        for (int g = 0; g < NG; ++g) {
           int c0, c1;
           group_chunks<EPI, BN>(g, c0, c1);
           uint32_t r0[32], r1[32];
@@ -779,7 +820,7 @@ __global__ void __launch_bounds__(192, 1)
             v[32 + j] = __uint_as_float(r1[j]);
           }
 
-          if (split) {
+          if (!WIDE && split) {  // WIDE plans give every CTA one whole tile
 #pragma unroll 2
             for (int cc = c_first + 1; cc <= c_last; ++cc) {
               const float* src = partial_slot<BN>(p, PAIR ? 2 * cc + static_cast<int>(rank) : cc);
@@ -801,6 +842,11 @@ __global__ void __launch_bounds__(192, 1)
                 v[32 + 4 * q + 3] += b[q].w;
               }
             }
+          }
+          if (WIDE && g >= 4) {
+            // columns [128, 176) of the tile: a 64-column box would spill into the next tile
+            swiglu_store_direct(p, row, sg.n_tile * (BN / 2) + 32 * g, v, row_scale, g == 4 ? 32 : 16);
+            continue;
           }
           uint8_t* box2 = nullptr;
           if (EPI == EPI_RESID && p.xw_out) st.acquire_both(box, box2);
@@ -862,6 +908,8 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
   auto kern = k_gemm_tc<BN, EPI, PAIR, KS>;
   if (PAIR && (plan.grid & 1)) return cudaErrorInvalidValue;
+  if (kSwWide<EPI, BN> && (plan.grid != plan.work || plan.splits != 1 || a.n_out % (BN / 2)))
+    return cudaErrorInvalidValue;  // one whole tile per CTA (a single accumulator)
   if (KS > 1 && (plan.grid % KS || plan.kb_total % KS || plan.grid != plan.work * KS)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -955,6 +1003,7 @@ cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
     switch (plan.bn) {
       case 128: return launch_one<128, EPI>(plan, a, s);
       case 256: return launch_one<256, EPI>(plan, a, s);
+      case 352: return launch_one<352, EPI>(plan, a, s);
       default: return cudaErrorInvalidValue;
     }
   } else {
@@ -1074,6 +1123,27 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
   }
   double best_cost = 1e300;
   const int tiles_m = (M + BM - 1) / BM;
+  // SwiGLU with few row tiles: 176 output columns per tile (two MMAs of N = 176 into 352
+  // accumulator columns), one tile per CTA, when those tiles fit one wave and 128-column tiles
+  // would not (M = 784: 112 CTAs instead of 154 tiles on 77 CTAs, two each).
+  if (epi == EPI_SWIGLU && n_out % 176 == 0) {
+    const long long wide = static_cast<long long>(tiles_m) * (n_out / 176);
+    const long long narrow = static_cast<long long>(tiles_m) * ((n_out + 127) / 128);
+    if (wide <= num_sms && narrow > num_sms) {
+      best.bn = 352;
+      best.pair = 0;
+      best.ks = 1;
+      best.splits = 1;
+      best.tiles_m = tiles_m;
+      best.tiles_n = n_out / 176;
+      best.kb_total = kb_total;
+      best.work = static_cast<int>(wide);
+      best.grid = static_cast<int>(wide);
+      best.partial_bytes = 0;
+      best.counters = 0;
+      return best;
+    }
+  }
   const int cands[4] = {256, 192, 128, 64};
   for (int bn : cands) {
     // Epilogue constraints: SwiGLU stores 64-column boxes of two 32-column groups (bn / 2 a

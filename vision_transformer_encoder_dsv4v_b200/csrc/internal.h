@@ -181,10 +181,8 @@ cudaError_t launch_swiglu_bwd(const void* g, const void* u, const void* dh, void
 cudaError_t launch_rotary_bwd(void* dqkv, const float* cos, const float* sin, int64_t P, int D, int hd, int sms,
                               cudaStream_t s);
 // Image-token bridge (bridge.cu).  Positions per CTA of the merge and the visibility scan;
-// counts holds one int4 per chunk of that many positions.  Up to kBridgeFusedPositions the
-// merge is one launch and leaves counts untouched.
+// counts holds one int4 per chunk of that many positions.
 constexpr int kBridgeChunk = 256;
-constexpr int64_t kBridgeFusedPositions = int64_t{1} << 16;
 cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, int4* counts, const int32_t* grid_dev,
                                 int n_images, int r, int64_t n_tokens, const void* image_tokens, const void* sentinels,
                                 void* embeds, int row_vec, uint32_t* err, cudaStream_t s);
