@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--profile", action="store_true",
                     help="run warm-up + steps as plain C-ABI calls (no graph, no extra passes) for ncu; "
                          "prints no bench line")
+    ap.add_argument("--extra", choices=["patch_embed", "patch_merger", "bridge", "block_backward", "workload5"],
+                    help="time only this one of the bench line's extras (for a profiler) and print it; "
+                         "prints no bench line")
     return ap.parse_args()
 
 
@@ -257,6 +260,16 @@ def run_ours(args):
         print(json.dumps({"profile_run": True, "device_error": A.dsv4v_device_error(),
                           "kernels_per_step": launches_per_step,
                           "path": "chain" if chain_path else "kernels"}), flush=True)
+        return
+
+    if args.extra:
+        one = {"patch_embed": lambda: patch_embed_timing(A, torch, cfg, wl, stream, flush, args.steps),
+               "patch_merger": lambda: patch_merger_timing(A, torch, cfg, batch, wl, stream, flush, args.steps),
+               "bridge": lambda: bridge_timing(A, torch, cfg, stream, flush, args.steps),
+               "block_backward": lambda: block_backward_timing(A, torch, cfg, batch, wl, lw, stream, flush,
+                                                               args.steps),
+               "workload5": lambda: workload5_timing(A, torch, lw, fnw, wa, stream, flush, args.steps)}[args.extra]()
+        print(json.dumps({"extra": args.extra, **one}), flush=True)
         return
 
     # Capture one step (all kernels of the path, launched through the C ABI) in a CUDA graph.

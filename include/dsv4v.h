@@ -32,6 +32,11 @@
  *    kernel is launched.  A device-side check that fails (a bounded wait that gives up)
  *    records an error that dsv4v_device_error() returns after synchronising the stream.
  *  - Calls on the same workspace must not overlap on the GPU (put them on one stream).
+ *  - This library's kernels may start while earlier ones of the library on the stream still
+ *    run (dependent launch), and may read their weight arguments before those finish;
+ *    everything else they read only after.  So a weight passed to a call must not have been
+ *    written by this library's kernels since the last other kernel (or host synchronisation)
+ *    on the stream; an optimizer step in between is enough.
  *  - No call keeps device state between calls; each call may be captured in a CUDA graph
  *    (the launch geometry is taken from the host copies of the grids and offsets, which must
  *    equal the device copies).

@@ -403,6 +403,8 @@ struct GemmExtra {
   int64_t lda = 0, ldb = 0;
   const float* bias = nullptr;
   int clear_counters = 0;  // zero this many split-tile counters on the stream right before the launch
+  // B (and B2) are the caller's weights, complete before the call: see GemmArgs::b_early.
+  bool b_early = true;
   // Weights of the GEMM that follows, prefetched into L2 by this one (see GemmArgs).
   const void* l2_next[2] = {nullptr, nullptr};
   size_t l2_next_bytes[2] = {0, 0};
@@ -455,6 +457,7 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.ss_out = nf.ss_out;
   g.ss_parts = nf.ss_parts;
   g.bias = ex.bias;
+  g.b_early = ex.b_early;
   for (int r = 0; r < 2; ++r) {
     g.l2_next[r] = ex.l2_next[r];
     g.l2_next_bytes[r] = ex.l2_next_bytes[r];
@@ -1386,6 +1389,7 @@ dsv4v_status gemm_store(const Ctx& c, const void* a, int64_t M, int K, int64_t l
   GemmExtra ex;
   ex.lda = lda;
   ex.ldb = ldb;
+  ex.b_early = false;  // B is an activation or a transposed copy written earlier in the call
   return gemm_bf16(c, EPI_STORE, plan, a, M, K, b, nullptr, n_out, out, nullptr, nullptr, nullptr, NormFold(), ex);
 }
 

@@ -77,6 +77,7 @@ struct Params {
   const float* bias;
   const void* l2_next[2];
   size_t l2_next_bytes[2];
+  int b_early;
 };
 
 // ---------------------------------------------------------------------------- stream-K ranges
@@ -293,8 +294,10 @@ __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
               const __grid_constant__ CUtensorMap tm_xw, const Params p) {
-  static_assert(KS == 1 || (!PAIR && BN == 256 && (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)),
-                "cluster split-K is built for 256-column residual, store and GELU tiles");
+  static_assert(KS == 1 || (!PAIR && (BN == 256 || (BN == 128 && KS == 2)) &&
+                            (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)),
+                "cluster split-K is built for 256-column (2 or 4 ranks) and 128-column (2 ranks) residual, "
+                "store and GELU tiles");
   using C = TileCfg<BN, PAIR>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
   constexpr int STAGES = C::STAGES;
@@ -400,8 +403,9 @@ __global__ void __launch_bounds__(192, 1)
       };
       SegmentWalker walk(p, owner);
       Segment sg;
-      // The weight tiles of the first stages do not depend on the previous kernel: start them
-      // before waiting for it, then add the activation tiles.
+      // Weight tiles of the first stages do not depend on the previous kernel: start them before
+      // waiting for it (b_early), then add the activation tiles.
+      if (!p.b_early) grid_dependency_wait();
       int pre = 0;
       Segment first{};
       SegmentWalker peek = walk;
@@ -946,6 +950,7 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.ss_out = a.ss_out;
   p.ss_parts = a.ss_parts;
   p.bias = a.bias;
+  p.b_early = a.b_early ? 1 : 0;
   for (int r = 0; r < 2; ++r) {
     p.l2_next[r] = a.l2_next[r];
     p.l2_next_bytes[r] = a.l2_next_bytes[r];
@@ -966,9 +971,11 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
 template <int EPI>
 cudaError_t launch_bn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   if (plan.ks > 1) {
-    // Cluster split-K: 256-column residual, store and GELU tiles.
+    // Cluster split-K: 256-column tiles over 2 or 4 ranks, 128-column tiles over 2.
     if constexpr (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU) {
-      if (plan.bn != 256 || plan.pair) return cudaErrorInvalidValue;
+      if (plan.pair) return cudaErrorInvalidValue;
+      if (plan.bn == 128 && plan.ks == 2) return launch_one<128, EPI, false, 2>(plan, a, s);
+      if (plan.bn != 256) return cudaErrorInvalidValue;
       switch (plan.ks) {
         case 2: return launch_one<256, EPI, false, 2>(plan, a, s);
         case 4: return launch_one<256, EPI, false, 4>(plan, a, s);
@@ -1054,12 +1061,14 @@ double plan_cost(int bn, long long tiles, int kb_total, int grid, int* contrib_o
 // waves) they lose by 1-60 %, mostly to split-tile fix-ups.
 constexpr int kPairMinWaves = 5;
 
-// Cost of one partial slice exchanged through distributed shared memory in a cluster split-K
-// (128 rows x 256 / ks fp32 written to a peer's ring and summed there, with the two cluster
-// barriers and the cluster launch).  Fitted on B200 at M = 784: 4-way split of the down
-// projection (K = 2816) 15.1 us vs 16.0 us for the best single-CTA plan; of the output
-// projection (K = 1024) 12.8 us vs 9.7 us.
+// Cluster split-K costs: per 32 KB partial slice a CTA sends to a peer (staged in its ring, moved
+// by a bulk DSMEM copy, summed by the peer; DSMEM moves ~30 B/ns per SM), and per CTA for the two
+// cluster barriers and the staging.  Fitted on B200 at M = 784 (CUDA-graph step, 32 layers): the
+// down projection (K = 2816) as 128-column tiles over 2 ranks beats 256-column tiles over 4 by
+// 1.75 us per layer; the output projection (K = 1024) stays on 64-column single-CTA tiles
+// (0.3 us per layer ahead of 128 x 2 ranks, 3.3 us ahead of 256 x 4).
 constexpr double kExchangeCycles = 4200.0;
+constexpr double kClusterCycles = 1000.0;
 
 }  // namespace
 
@@ -1193,22 +1202,27 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
       }
     }
   }
-  // Cluster split-K for 256-column residual, store and GELU tiles: full-rate N = 256 MMAs even
-  // when there are too few such tiles for the SMs, without the global-memory split-tile fix-up.
-  if ((epi == EPI_RESID || epi == EPI_STORE || epi == EPI_GELU) && n_out % 256 == 0) {
-    const long long tiles = static_cast<long long>(tiles_m) * (n_out / 256);
-    for (int ks : {2, 4}) {
+  // Cluster split-K for residual, store and GELU tiles (256 columns over 2 or 4 ranks, 128 over
+  // 2): full-rate MMAs even when there are too few tiles for the SMs, without the global-memory
+  // split-tile fix-up.
+  if (epi == EPI_RESID || epi == EPI_STORE || epi == EPI_GELU) {
+    const int shapes[3][2] = {{256, 2}, {256, 4}, {128, 2}};
+    for (const auto& sh : shapes) {
+      const int bn = sh[0], ks = sh[1];
+      if (n_out % bn) continue;
+      const long long tiles = static_cast<long long>(tiles_m) * (n_out / bn);
       if (kb_total % ks || tiles * ks > num_sms) continue;
-      const double cost =
-          (kb_total / ks) * kblock_cycles(256) + 2000.0 + 12.0 * (256 / ks) + kExchangeCycles * (ks - 1);
+      const double slices = (ks - 1) * (static_cast<double>(BM) * (bn / ks) * 4.0) / 32768.0;
+      const double cost = (kb_total / ks) * kblock_cycles(bn) + 2000.0 + 12.0 * (bn / ks) +
+                          kExchangeCycles * slices + kClusterCycles;
       if (cost < best_cost - 1e-9) {
         best_cost = cost;
-        best.bn = 256;
+        best.bn = bn;
         best.pair = 0;
         best.ks = ks;
         best.splits = 1;
         best.tiles_m = tiles_m;
-        best.tiles_n = n_out / 256;
+        best.tiles_n = n_out / bn;
         best.kb_total = kb_total;
         best.work = static_cast<int>(tiles);
         best.grid = static_cast<int>(tiles * ks);

@@ -66,6 +66,10 @@ struct GemmArgs {
   float* ss_out;
   int ss_parts;
   const float* bias;  // STORE: per-column fp32 bias added before rounding (NULL: none)
+  // B (and B2) are weights that no kernel still in flight on the stream writes: their first
+  // stages may be loaded before the dependency wait.  Otherwise (B produced by an earlier kernel
+  // of the same call, as in the backward's weight gradients) every load waits.
+  bool b_early;
   // Up to two ranges (the next GEMM's weights) that the CTAs prefetch into L2, a share each,
   // once their own operand loads are issued (NULL: none; 16-byte aligned, bytes a multiple of 16).
   const void* l2_next[2];
