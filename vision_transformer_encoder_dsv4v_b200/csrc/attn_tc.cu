@@ -379,32 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = raise ? m_cand : m_used;
       const float alpha = raise ? ex2_mufu(m_used - m_new) : 1.0f;  // 0 on the first tile
       m_used = m_new;
-      if (j > 0) {
-        // P_X and O_X are free once the previous P_X V product has completed.
-        got = mbar_wait(&pv_done[x], (j - 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, raise)) {
-          uint32_t o[HD];
-          tmem_ld_cols<HD / 32>(t_o, o);
-          const uint64_t al2 = pk2(alpha, alpha);
-#pragma unroll
-          for (int c = 0; c < HD; c += 2) {
-            float a0, a1;
-            upk2(mul2(pk2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), al2), a0, a1);
-            o[c] = __float_as_uint(a0);
-            o[c + 1] = __float_as_uint(a1);
-          }
-          tmem_st32(t_o, o);
-          tmem_st32(t_o + 32, o + 32);
-        }
-      }
       // P = 2^(s c - m), some exponential pairs on the FMA pipe interleaved with the MUFU ones;
-      // the bf16 pairs are packed in place into s[0 .. TK/2) and each half of P goes to TMEM
-      // as soon as it is complete.
+      // the bf16 pairs are packed in place into s[0 .. TK/2).  They are computed before waiting
+      // for the previous P_X V product, which they overlap.
       const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(-m_new, -m_new);
       uint64_t l2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -419,9 +396,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l2[(c >> 1) & 3] = add2(l2[(c >> 1) & 3], pk2(e0, e1));
         s[c >> 1] = pack_bf16x2(e0, e1);
-        if (c == TK / 2 - 2) tmem_st32(t_p, s);
       }
+      if (j > 0) {
+        // P_X and O_X are free once the previous P_X V product has completed.
+        got = mbar_wait(&pv_done[x], (j - 1) & 1, abort_flag, p.err, kErrTimeoutEpilogue);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+      }
+      tmem_st32(t_p, s);
       tmem_st32(t_p + 32, s + 32);
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        uint32_t o[HD];
+        tmem_ld_cols<HD / 32>(t_o, o);
+        const uint64_t al2 = pk2(alpha, alpha);
+#pragma unroll
+        for (int c = 0; c < HD; c += 2) {
+          float a0, a1;
+          upk2(mul2(pk2(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), al2), a0, a1);
+          o[c] = __float_as_uint(a0);
+          o[c + 1] = __float_as_uint(a1);
+        }
+        tmem_st32(t_o, o);
+        tmem_st32(t_o + 32, o + 32);
+      }
       float la, lb, lc, ld, le, lf, lg, lh;
       upk2(l2[0], la, lb);
       upk2(l2[1], lc, ld);

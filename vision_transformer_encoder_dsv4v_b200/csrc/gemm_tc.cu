@@ -310,7 +310,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* mma_done = tempty + 2;
   uint64_t* teardown = mma_done + 1;  // one arrival per warp once its role is done
   uint64_t* xchg = teardown + 1;      // cluster split-K: the peers' partial slices have landed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xchg + 1);
+  uint64_t* sent = xchg + 1;          // cluster split-K: every peer holds this CTA's slices
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sent + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* ticket = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
@@ -337,6 +338,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(mma_done, 1);
     mbar_init(teardown, blockDim.x / 32);
     mbar_init(xchg, 1);
+    mbar_init(sent, KS > 1 ? KS - 1 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -465,8 +467,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     if constexpr (KS > 1) {
       __syncwarp();
-      cluster_sync();  // the two cluster barriers of the epilogue
-      cluster_sync();
+      cluster_sync();  // the epilogue's cluster barrier
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -538,10 +539,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(mma_done, 0, &never, p.err, kErrTimeoutMma);
     }
     __syncwarp();
-    if constexpr (KS > 1) {
-      cluster_sync();  // the two cluster barriers of the epilogue (this CTA's MMAs are done)
-      cluster_sync();
-    }
+    if constexpr (KS > 1) cluster_sync();  // the epilogue's cluster barrier (this CTA's MMAs are done)
   } else if (warp < 6) {
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) belong to this warp
@@ -657,6 +655,11 @@ __global__ void __launch_bounds__(192, 1)
       // Every peer sends its slices whenever it has a tile (the cluster shares one tile).
       got = got && mbar_wait(xchg, 0, abort_flag, p.err, kErrTimeoutEpilogue);
       got = named_barrier_and(2, 128, got);
+      // Every slice from a peer has landed, so its bulk copy no longer reads the peer's send
+      // area: tell that peer.
+      if (et == 0 && got)
+        for (int j = 0; j < KS; ++j)
+          if (j != static_cast<int>(kslice)) mbar_arrive_cluster(mapa_shared(smem_u32(sent), static_cast<uint32_t>(j)));
       if (got) {
         uint8_t* box = nullptr;
 #pragma unroll
@@ -705,8 +708,12 @@ __global__ void __launch_bounds__(192, 1)
         if (EPI == EPI_RESID && p.xw_out && row < p.M)
           p.ss_out[static_cast<size_t>(row) * p.ss_parts + sg.n_tile * KS + static_cast<int>(kslice)] = ss_acc;
       }
-      // Barrier 2: no CTA leaves while a peer's bulk copies may still read its send area.
-      cluster_sync();
+      // No CTA leaves while a peer's bulk copy may still read its send area (bounded wait: a
+      // peer that gave up never arrives).
+      if (et == 0) {
+        volatile int never = 0;
+        mbar_wait_cluster(sent, 0, &never, p.err, kErrTimeoutEpilogue);
+      }
     }
     bool xw_loaded = false;
     while (KS == 1 && walk.next(p, sg)) {
