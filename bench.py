@@ -32,11 +32,12 @@ from vision_transformer_encoder_dsv4v_b200 import synth  # noqa: E402
 
 METRIC = "ViT tower patches/sec and TFLOP/s (bf16, 1 B200) vs dense bf16 roofline"
 
-# DRAM bytes per launch of each kernel class, from one ncu launch-list capture of the benchmark
-# (dram__bytes_read.sum + dram__bytes_write.sum) of the kernels as they are now; an entry is
+# DRAM bytes per launch of each kernel class (dram__bytes_read.sum + dram__bytes_write.sum), from
+# one-kernel ncu captures of the benchmark's step (-k regex:k_gemm_tc -s 8 -c 4 for the GEMMs of
+# the third layer, -k regex:k_attn_tc -s 2 -c 1) of the kernels as they are now; an entry is
 # removed when its kernel changes.
 TRAFFIC_BYTES = {
-    (4, "down"): 11.84e6, (4, "swiglu"): 13.24e6, (4, "attention"): 4.87e6, (4, "out"): 5.37e6, (4, "qkv"): 8.20e6,
+    (4, "down"): 18.15e6, (4, "swiglu"): 19.01e6, (4, "attention"): 4.88e6, (4, "out"): 16.91e6, (4, "qkv"): 10.30e6,
 }
 UNIT = "patches/s"
 
@@ -358,7 +359,8 @@ def run_ours(args):
     traffic = TRAFFIC_BYTES.get((args.workload, dom["name"]))
     roof = {"bound": "tensor", "kernel": dom["name"], "achieved": dom["tflops"], "peak": peak, "unit": "TFLOP/s",
             "frac": dom["tflops"] / peak, "traffic": traffic,
-            "traffic_unit": "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, ncu)",
+            "traffic_unit": "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, ncu); a GEMM's "
+                            "figure includes the next GEMM's weights, which it prefetches into L2",
             "peak_source": ("MEASURED_PEAKS.json bf16_tflops, the burst cuBLAS bf16 rate (of measured)" if peaks
                             else "fallback 1.59 PF burst"),
             "peak_sustained": peaks.get("bf16_tflops_sustained"),
