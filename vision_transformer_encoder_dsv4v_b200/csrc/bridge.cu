@@ -29,6 +29,8 @@ namespace {
 
 constexpr int kTypeText = -1, kTypeImage = 0, kTypeStart = 1, kTypeEnd = 2, kTypePad = 4;
 constexpr int kWarps = kBridgeChunk / 32;
+constexpr int kBulkBufs = 4;                 // row buffers in flight per merge CTA (bulk mode)
+constexpr size_t kBulkSmemMax = 160 * 1024;  // dynamic shared memory a bulk-mode merge CTA may take
 
 __device__ __forceinline__ void record(uint32_t* err) { atomicCAS(err, 0u, static_cast<uint32_t>(kErrBridgeLayout)); }
 
@@ -141,16 +143,20 @@ __global__ void __launch_bounds__(kBridgeChunk)
     k_bridge_merge(const int32_t* __restrict__ types, int64_t n, int64_t seq, const int4* __restrict__ counts,
                    const int32_t* __restrict__ grid, int n_images, int r, int64_t n_tokens,
                    const uint4* __restrict__ image_tokens, const uint4* __restrict__ sentinels,
-                   uint4* __restrict__ embeds, int row_vec, uint32_t* err) {
-  extern __shared__ int32_t tok_cu[];  // [n_images + 1] aligner-token offsets of the images
+                   uint4* __restrict__ embeds, int row_vec, int ring_off, uint32_t* err) {
+  // Dynamic shared memory: [n_images + 1] aligner-token offsets of the images, then (bulk mode,
+  // ring_off > 0) kBulkBufs row buffers at byte offset ring_off.
+  extern __shared__ __align__(16) int32_t tok_cu[];
   __shared__ ScanSmem sm;
   __shared__ int warp_copies[kWarps];
   __shared__ int n_list;
-  // The chunk's rows to copy, in position order: where this CTA's column slice of each row is
-  // read (aligner token or sentinel) and written.
+  __shared__ __align__(8) uint64_t row_full[kBulkBufs];
+  // The chunk's rows to copy, in position order: where this CTA's part of each row is read
+  // (aligner token or sentinel) and written (a column slice, or the whole row in bulk mode).
   __shared__ const uint4* list_from[kBridgeChunk];
   __shared__ uint4* list_to[kBridgeChunk];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool bulk = ring_off > 0;
   grid_dependency_wait();
   launch_dependents();
   {
@@ -204,8 +210,12 @@ __global__ void __launch_bounds__(kBridgeChunk)
   __syncthreads();
   int slot = __popc(b_copy & ((1u << lane) - 1u));
   for (int w = 0; w < warp; ++w) slot += warp_copies[w];
-  const int vs = row_vec / static_cast<int>(gridDim.y);
-  const int col0 = static_cast<int>(blockIdx.y) * vs;
+  const int vs = bulk ? row_vec : row_vec / static_cast<int>(gridDim.y);
+  const int col0 = bulk ? 0 : static_cast<int>(blockIdx.y) * vs;
+  if (bulk && tid == 0) {
+    for (int b = 0; b < kBulkBufs; ++b) mbar_init(&row_full[b], 1);
+    fence_mbar_init();
+  }
   if (copy) {
     list_from[slot] = (s >= 0 ? image_tokens + s * row_vec : sentinels + (-s - 2) * row_vec) + col0;
     list_to[slot] = embeds + ps.p * row_vec + col0;
@@ -213,9 +223,40 @@ __global__ void __launch_bounds__(kBridgeChunk)
   if (tid == kBridgeChunk - 1) n_list = slot + (copy ? 1 : 0);
   __syncthreads();
 
+  const int nl = n_list;
+  if (bulk) {
+    // Whole rows j = y, y + slices, ... of the chunk's list by bulk (TMA) copies through a ring of
+    // kBulkBufs row buffers: one thread loads ahead, stores each row as it lands, and refills a
+    // buffer once the store issued from it one row earlier has read it.
+    if (tid != 0) return;
+    const uint32_t rb = static_cast<uint32_t>(row_vec) * 16u;
+    uint8_t* ring = reinterpret_cast<uint8_t*>(tok_cu) + ring_off;
+    const int y = static_cast<int>(blockIdx.y), step = static_cast<int>(gridDim.y);
+    const int mine = y < nl ? (nl - y + step - 1) / step : 0;
+    for (int k = 0; k < mine && k < kBulkBufs; ++k) {
+      mbar_arrive_expect_tx(&row_full[k], rb);
+      bulk_load(ring + k * rb, list_from[y + k * step], rb, &row_full[k]);
+    }
+    volatile int never = 0;
+    for (int k = 0; k < mine; ++k) {
+      const int b = k % kBulkBufs;
+      if (!mbar_wait(&row_full[b], static_cast<uint32_t>(k / kBulkBufs) & 1u, &never, err, kErrTimeoutProducer))
+        break;
+      bulk_store(list_to[y + k * step], ring + b * rb, rb);
+      bulk_commit();
+      const int kn = k - 1 + kBulkBufs;  // the next row of the previous row's buffer
+      if (k >= 1 && kn < mine) {
+        bulk_wait_read_1();  // every store but the one just issued has read its buffer
+        const int bp = (k - 1) % kBulkBufs;
+        mbar_arrive_expect_tx(&row_full[bp], rb);
+        bulk_load(ring + bp * rb, list_from[y + kn * step], rb, &row_full[bp]);
+      }
+    }
+    bulk_wait_all();
+    return;
+  }
   // Thread t copies vector column t % vs of rows t / vs, t / vs + rpp, ... (rpp rows per pass
   // of the CTA), eight independent 16-byte loads before their stores; no per-vector division.
-  const int nl = n_list;
   constexpr int kUnroll = 8;
   auto copy_rows = [&](int c, int r0, int step) {
     for (int j0 = r0; j0 < nl; j0 += step * kUnroll) {
@@ -317,12 +358,22 @@ cudaError_t launch_bridge_merge(const int32_t* types, int64_t n, int64_t seq, in
   cudaError_t e = launch_pdl(k_bridge_count, dim3(static_cast<unsigned>(chunks)), dim3(kBridgeChunk), 0, s, types, n,
                              counts, static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr), err);
   if (e != cudaSuccess) return e;
-  const int slices = bridge_slices(row_vec);
+  // Rows of 2 KB or more move by bulk copies, whole rows per CTA (16 CTAs per chunk, each taking
+  // every 16th row); narrower rows by 16-byte vectors, a column slice per CTA.
+  const size_t row_bytes = static_cast<size_t>(row_vec) * 16;
+  const size_t tok_bytes = (static_cast<size_t>(n_images) + 1) * sizeof(int32_t);
+  const size_t ring_off = (tok_bytes + 127) / 128 * 128;
+  const bool bulk = row_bytes >= 2048 && ring_off + kBulkBufs * row_bytes <= kBulkSmemMax;
+  const size_t smem = bulk ? ring_off + kBulkBufs * row_bytes : tok_bytes;
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(k_bridge_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const int slices = bulk ? 16 : bridge_slices(row_vec);
   return launch_pdl(k_bridge_merge, dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(slices)),
-                    dim3(kBridgeChunk), (n_images + 1) * sizeof(int32_t), s, types, n, seq,
-                    static_cast<const int4*>(counts), grid_dev, n_images, r, n_tokens,
-                    static_cast<const uint4*>(image_tokens), static_cast<const uint4*>(sentinels),
-                    static_cast<uint4*>(embeds), row_vec, err);
+                    dim3(kBridgeChunk), smem, s, types, n, seq, static_cast<const int4*>(counts), grid_dev, n_images,
+                    r, n_tokens, static_cast<const uint4*>(image_tokens), static_cast<const uint4*>(sentinels),
+                    static_cast<uint4*>(embeds), row_vec, bulk ? static_cast<int>(ring_off) : 0, err);
 }
 
 cudaError_t launch_image_visibility(const int32_t* types, int64_t batch, int64_t seq, void* mask, int elem_bytes,

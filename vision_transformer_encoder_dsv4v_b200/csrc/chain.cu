@@ -623,7 +623,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_chain(const __grid_constant__ C
   } else {
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
-    const int row_in_tile = quad * 32 + lane;
     const int et = threadIdx.x - 64;
     Stager1 st{smem + OFF_STAGING + (warp - 2) * 4096, lane, 0};
     grid_dependency_wait();

@@ -174,6 +174,23 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
+// Bulk copy of `bytes` (a multiple of 16, 16-byte aligned ends) from global memory into this
+// CTA's shared memory, counted on the mbarrier as it lands.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory to global memory, in the thread's current
+// bulk async-group (bulk_commit / bulk_wait_*).
+__device__ __forceinline__ void bulk_store(void* dst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
+}
+
 // Prefetch of `bytes` (a multiple of 16) at 16-byte aligned global address p into L2.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
