@@ -475,6 +475,7 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // is issued here rather than sunk past a wait that follows.
 __device__ __forceinline__ void pin(float& v) { asm volatile("" : "+f"(v)); }
 __device__ __forceinline__ void pin(uint4& v) { asm volatile("" : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)); }
+__device__ __forceinline__ void pin(uint64_t& v) { asm volatile("" : "+l"(v)); }
 // 1/x on the MUFU pipe.
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
@@ -490,6 +491,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Packed pairs of fp32 (one 64-bit register pair) for the sm_100 f32x2 arithmetic.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// The two bf16 of a packed pair as a packed fp32 pair.
+__device__ __forceinline__ uint64_t bf16x2_f2(uint32_t v) { return pk2(bf16_lo(v), bf16_hi(v)); }
 
 // Launches `kern` with programmatic stream serialization (dependent launch) allowed: the kernel
 // may begin while the previous kernel on the stream is still running, and must call

@@ -121,41 +121,55 @@ struct SegmentWalker {
 
 
 // Epilogue math of one 64-column accumulator group v[0..63] of output row `row`; the result
-// goes to the warp's staging box (the caller stores it).
+// goes to the warp's staging box (the caller stores it).  Pairs of columns use the packed fp32
+// (f32x2) arithmetic.
 //   STORE/RESID/QKV: v = accumulator columns [64g, 64g + 64) -> output columns n0 + 64g + j.
+//     QKV: rot_c / rot_s hold the row's rotation table already multiplied by the folded-norm row
+//     scale (pairs of columns, packed), so a rotated group needs no separate scaling.
 //   SWIGLU: v[0..31] = gate columns, v[32..63] = up columns of output columns n0h + 32g + j;
 //           written to chunks 4 (g & 1) .. 4 (g & 1) + 3 of the box.
 //   RESID with the next norm prepared: the second box receives bf16(x * w_next).
 template <int EPI, int BN, int NR>
 __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_tile, int g, float (&v)[64],
-                                               const float (&rot_c)[NR], const float (&rot_s)[NR], float row_scale,
-                                               const uint4* resid, const float* xw_s, float& ss_acc, Stager& st,
-                                               uint8_t* box, uint8_t* box2) {
+                                               const uint64_t (&rot_c)[NR], const uint64_t (&rot_s)[NR],
+                                               float row_scale, const uint4* resid, const float* xw_s, float& ss_acc,
+                                               Stager& st, uint8_t* box, uint8_t* box2) {
   if (row >= p.M) return;
-  if constexpr (EPI == EPI_SWIGLU || EPI == EPI_QKV_ROPE) {
-#pragma unroll
-    for (int j = 0; j < 64; ++j) v[j] *= row_scale;
-  }
+  const uint64_t rs2 = pk2(row_scale, row_scale);
   if constexpr (EPI == EPI_SWIGLU) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
+      float h[8];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        float g0, g1, u0, u1;
+        upk2(mul2(pk2(v[8 * q + i], v[8 * q + i + 1]), rs2), g0, g1);
+        upk2(mul2(pk2(v[32 + 8 * q + i], v[32 + 8 * q + i + 1]), rs2), u0, u1);
+        h[i] = silu(g0) * u0;
+        h[i + 1] = silu(g1) * u1;
+      }
       uint4 o;
-      o.x = pack_bf16x2(silu(v[8 * q + 0]) * v[32 + 8 * q + 0], silu(v[8 * q + 1]) * v[32 + 8 * q + 1]);
-      o.y = pack_bf16x2(silu(v[8 * q + 2]) * v[32 + 8 * q + 2], silu(v[8 * q + 3]) * v[32 + 8 * q + 3]);
-      o.z = pack_bf16x2(silu(v[8 * q + 4]) * v[32 + 8 * q + 4], silu(v[8 * q + 5]) * v[32 + 8 * q + 5]);
-      o.w = pack_bf16x2(silu(v[8 * q + 6]) * v[32 + 8 * q + 6], silu(v[8 * q + 7]) * v[32 + 8 * q + 7]);
+      o.x = pack_bf16x2(h[0], h[1]);
+      o.y = pack_bf16x2(h[2], h[3]);
+      o.z = pack_bf16x2(h[4], h[5]);
+      o.w = pack_bf16x2(h[6], h[7]);
       st.put(box, 4 * (g & 1) + q, o);
     }
   } else {
     if constexpr (EPI == EPI_QKV_ROPE) {
       const int col = n_tile * BN + g * 64;
       if (col < p.rot_cols) {
+        // (x1, x2) -> (x1 c - x2 s, x2 c + x1 s) for columns j and j + 32, two j at a time
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float x1 = v[j], x2 = v[32 + j];
-          v[j] = x1 * rot_c[j] - x2 * rot_s[j];
-          v[32 + j] = x2 * rot_c[j] + x1 * rot_s[j];
+        for (int j = 0; j < 32; j += 2) {
+          const uint64_t a = pk2(v[j], v[j + 1]), b = pk2(v[32 + j], v[33 + j]);
+          const uint64_t c2 = rot_c[j >> 1], s2 = rot_s[j >> 1];
+          upk2(sub2(mul2(a, c2), mul2(b, s2)), v[j], v[j + 1]);
+          upk2(fma2(a, s2, mul2(b, c2)), v[32 + j], v[33 + j]);
         }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) upk2(mul2(pk2(v[j], v[j + 1]), rs2), v[j], v[j + 1]);
       }
     }
     if constexpr (EPI == EPI_GELU) {
@@ -175,10 +189,8 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const float4 bq = b4[q];
-          v[4 * q] += bq.x;
-          v[4 * q + 1] += bq.y;
-          v[4 * q + 2] += bq.z;
-          v[4 * q + 3] += bq.w;
+          upk2(add2(pk2(v[4 * q], v[4 * q + 1]), pk2(bq.x, bq.y)), v[4 * q], v[4 * q + 1]);
+          upk2(add2(pk2(v[4 * q + 2], v[4 * q + 3]), pk2(bq.z, bq.w)), v[4 * q + 2], v[4 * q + 3]);
         }
       }
     }
@@ -186,14 +198,10 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const uint4 r = resid[q];
-        v[8 * q + 0] += bf16_lo(r.x);
-        v[8 * q + 1] += bf16_hi(r.x);
-        v[8 * q + 2] += bf16_lo(r.y);
-        v[8 * q + 3] += bf16_hi(r.y);
-        v[8 * q + 4] += bf16_lo(r.z);
-        v[8 * q + 5] += bf16_hi(r.z);
-        v[8 * q + 6] += bf16_lo(r.w);
-        v[8 * q + 7] += bf16_hi(r.w);
+        upk2(add2(pk2(v[8 * q + 0], v[8 * q + 1]), bf16x2_f2(r.x)), v[8 * q + 0], v[8 * q + 1]);
+        upk2(add2(pk2(v[8 * q + 2], v[8 * q + 3]), bf16x2_f2(r.y)), v[8 * q + 2], v[8 * q + 3]);
+        upk2(add2(pk2(v[8 * q + 4], v[8 * q + 5]), bf16x2_f2(r.z)), v[8 * q + 4], v[8 * q + 5]);
+        upk2(add2(pk2(v[8 * q + 6], v[8 * q + 7]), bf16x2_f2(r.w)), v[8 * q + 6], v[8 * q + 7]);
       }
     }
     uint4 o[8];
@@ -210,19 +218,31 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
         // Next RMSNorm's operand from the stored (bf16) x: bf16(x * w) and sum of x^2; w of the
         // tile's columns was staged in shared memory before the accumulator was ready.
         const float4* w4 = reinterpret_cast<const float4*>(xw_s + g * 64);
+        uint64_t ss2 = 0ull;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
-          const float x0 = bf16_lo(o[q].x), x1 = bf16_hi(o[q].x), x2 = bf16_lo(o[q].y), x3 = bf16_hi(o[q].y);
-          const float x4 = bf16_lo(o[q].z), x5 = bf16_hi(o[q].z), x6 = bf16_lo(o[q].w), x7 = bf16_hi(o[q].w);
-          ss_acc += ((x0 * x0 + x1 * x1) + (x2 * x2 + x3 * x3)) + ((x4 * x4 + x5 * x5) + (x6 * x6 + x7 * x7));
+          const uint64_t x01 = bf16x2_f2(o[q].x), x23 = bf16x2_f2(o[q].y), x45 = bf16x2_f2(o[q].z),
+                         x67 = bf16x2_f2(o[q].w);
+          ss2 = fma2(x01, x01, ss2);
+          ss2 = fma2(x23, x23, ss2);
+          ss2 = fma2(x45, x45, ss2);
+          ss2 = fma2(x67, x67, ss2);
+          float t0, t1, t2, t3, t4, t5, t6, t7;
+          upk2(mul2(x01, pk2(wa.x, wa.y)), t0, t1);
+          upk2(mul2(x23, pk2(wa.z, wa.w)), t2, t3);
+          upk2(mul2(x45, pk2(wb.x, wb.y)), t4, t5);
+          upk2(mul2(x67, pk2(wb.z, wb.w)), t6, t7);
           uint4 t;
-          t.x = pack_bf16x2(x0 * wa.x, x1 * wa.y);
-          t.y = pack_bf16x2(x2 * wa.z, x3 * wa.w);
-          t.z = pack_bf16x2(x4 * wb.x, x5 * wb.y);
-          t.w = pack_bf16x2(x6 * wb.z, x7 * wb.w);
+          t.x = pack_bf16x2(t0, t1);
+          t.y = pack_bf16x2(t2, t3);
+          t.z = pack_bf16x2(t4, t5);
+          t.w = pack_bf16x2(t6, t7);
           st.put(box2, q, t);
         }
+        float s0, s1;
+        upk2(ss2, s0, s1);
+        ss_acc += s0 + s1;
       }
     }
   }
@@ -566,20 +586,26 @@ __global__ void __launch_bounds__(192, 1)
       const bool have = walk.next(p, sg);
       const int row = sg.m_tile * BM + row_in_tile;
       const int box_y = sg.m_tile * BM + quad * 32;
-      float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
+      // The folded-norm row scale, and the rotation table row pre-multiplied by it (packed pairs).
+      float row_scale = norm_row_scale(p, row);
+      pin(row_scale);
+      uint64_t rot_c[EPI == EPI_QKV_ROPE ? 16 : 1], rot_s[EPI == EPI_QKV_ROPE ? 16 : 1];
       uint4 resid[EPI == EPI_RESID ? GPR * 8 : 1];
       if constexpr (EPI == EPI_QKV_ROPE) {
         const int prow = min(row, p.M - 1);
         const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(prow) * 32);
         const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(prow) * 32);
+        const uint64_t rs2 = pk2(row_scale, row_scale);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 c = c4[q], s = s4[q];
-          rot_c[4 * q] = c.x; rot_c[4 * q + 1] = c.y; rot_c[4 * q + 2] = c.z; rot_c[4 * q + 3] = c.w;
-          rot_s[4 * q] = s.x; rot_s[4 * q + 1] = s.y; rot_s[4 * q + 2] = s.z; rot_s[4 * q + 3] = s.w;
+          const float4 c = c4[q], sn = s4[q];
+          rot_c[2 * q] = mul2(pk2(c.x, c.y), rs2);
+          rot_c[2 * q + 1] = mul2(pk2(c.z, c.w), rs2);
+          rot_s[2 * q] = mul2(pk2(sn.x, sn.y), rs2);
+          rot_s[2 * q + 1] = mul2(pk2(sn.z, sn.w), rs2);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           pin(rot_c[j]);
           pin(rot_s[j]);
         }
@@ -592,8 +618,6 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int q = 0; q < GPR * 8; ++q) pin(resid[q]);
       }
-      float row_scale = norm_row_scale(p, row);
-      pin(row_scale);
       float* xw_s = reinterpret_cast<float*>(smem + C::OFF_XW);
       if (EPI == EPI_RESID && p.xw_out && have)
         for (int i = et; i < BN; i += 128) xw_s[i] = p.xw_w[sg.n_tile * BN + i];
@@ -726,7 +750,10 @@ __global__ void __launch_bounds__(192, 1)
           owner == unit_owner(p, static_cast<long long>(sg.tile) * p.kb_total);
       // Inputs of the epilogue math fetched while the MMAs run: the rotation table row and the
       // residual row of this thread's output row, and the folded-norm row scale.
-      float rot_c[EPI == EPI_QKV_ROPE ? 32 : 1], rot_s[EPI == EPI_QKV_ROPE ? 32 : 1];
+      // The folded-norm row scale, and the rotation table row pre-multiplied by it (packed pairs).
+      float row_scale = norm_row_scale(p, row);
+      pin(row_scale);
+      uint64_t rot_c[EPI == EPI_QKV_ROPE ? 16 : 1], rot_s[EPI == EPI_QKV_ROPE ? 16 : 1];
       // The residual epilogue keeps RG groups (64 columns each) of the residual row in
       // registers and refills a slot RG groups ahead once its group is done.
       constexpr int RG = NGROUPS < 2 ? NGROUPS : 2;
@@ -735,14 +762,17 @@ __global__ void __launch_bounds__(192, 1)
         const int prow = min(row, p.M - 1);
         const float4* c4 = reinterpret_cast<const float4*>(p.cos + static_cast<size_t>(prow) * 32);
         const float4* s4 = reinterpret_cast<const float4*>(p.sin + static_cast<size_t>(prow) * 32);
+        const uint64_t rs2 = pk2(row_scale, row_scale);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 c = c4[q], s = s4[q];
-          rot_c[4 * q] = c.x; rot_c[4 * q + 1] = c.y; rot_c[4 * q + 2] = c.z; rot_c[4 * q + 3] = c.w;
-          rot_s[4 * q] = s.x; rot_s[4 * q + 1] = s.y; rot_s[4 * q + 2] = s.z; rot_s[4 * q + 3] = s.w;
+          const float4 c = c4[q], sn = s4[q];
+          rot_c[2 * q] = mul2(pk2(c.x, c.y), rs2);
+          rot_c[2 * q + 1] = mul2(pk2(c.z, c.w), rs2);
+          rot_s[2 * q] = mul2(pk2(sn.x, sn.y), rs2);
+          rot_s[2 * q + 1] = mul2(pk2(sn.z, sn.w), rs2);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           pin(rot_c[j]);
           pin(rot_s[j]);
         }
@@ -757,8 +787,6 @@ __global__ void __launch_bounds__(192, 1)
           for (int q = 0; q < RG * 8; ++q) pin(resid[q]);
         }
       }
-      float row_scale = norm_row_scale(p, row);
-      pin(row_scale);
       float* xw_s = reinterpret_cast<float*>(smem + C::OFF_XW);
       if (EPI == EPI_RESID && p.xw_out && finisher_or_full) {
         // After the first tile, every warp must be done with the previous tile's weights.
