@@ -137,16 +137,18 @@ __device__ __forceinline__ void epilogue_group(const Params& p, int row, int n_t
   if (row >= p.M) return;
   const uint64_t rs2 = pk2(row_scale, row_scale);
   if constexpr (EPI == EPI_SWIGLU) {
+    // silu(g r) (u r) with a = g r / 2: (a + a tanh(a)) (u r)
+    const uint64_t hrs2 = pk2(0.5f * row_scale, 0.5f * row_scale);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       float h[8];
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
-        float g0, g1, u0, u1;
-        upk2(mul2(pk2(v[8 * q + i], v[8 * q + i + 1]), rs2), g0, g1);
-        upk2(mul2(pk2(v[32 + 8 * q + i], v[32 + 8 * q + i + 1]), rs2), u0, u1);
-        h[i] = silu(g0) * u0;
-        h[i + 1] = silu(g1) * u1;
+        const uint64_t a2 = mul2(pk2(v[8 * q + i], v[8 * q + i + 1]), hrs2);
+        const uint64_t u2 = mul2(pk2(v[32 + 8 * q + i], v[32 + 8 * q + i + 1]), rs2);
+        float a0, a1;
+        upk2(a2, a0, a1);
+        upk2(mul2(fma2(a2, pk2(tanh_approx(a0), tanh_approx(a1)), a2), u2), h[i], h[i + 1]);
       }
       uint4 o;
       o.x = pack_bf16x2(h[0], h[1]);
@@ -290,7 +292,13 @@ __device__ __forceinline__ void swiglu_store_direct(const Params& p, int row, in
     if (8 * q >= n) break;
     float h[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) h[i] = silu(v[8 * q + i] * row_scale) * (v[32 + 8 * q + i] * row_scale);
+    for (int i = 0; i < 8; i += 2) {
+      const uint64_t a2 = mul2(pk2(v[8 * q + i], v[8 * q + i + 1]), pk2(0.5f * row_scale, 0.5f * row_scale));
+      const uint64_t u2 = mul2(pk2(v[32 + 8 * q + i], v[32 + 8 * q + i + 1]), pk2(row_scale, row_scale));
+      float a0, a1;
+      upk2(a2, a0, a1);
+      upk2(mul2(fma2(a2, pk2(tanh_approx(a0), tanh_approx(a1)), a2), u2), h[i], h[i + 1]);
+    }
     uint4 o;
     o.x = pack_bf16x2(h[0], h[1]);
     o.y = pack_bf16x2(h[2], h[3]);
