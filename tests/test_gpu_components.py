@@ -22,6 +22,8 @@ GRID_SETS = {
     "tiny": [(1, 1)],
     "lines": [(1, 37), (37, 1), (3, 5)],
     "mixed": [(3, 5), (1, 1), (64, 64), (9, 14)],
+    # last key tile holding 40, 70, 96, 97, 33 and 64 keys: every 32-key chunk boundary
+    "chunks": [(5, 8), (7, 10), (12, 8), (1, 97), (3, 11), (16, 12)],
 }
 
 
@@ -86,7 +88,7 @@ def test_qkv_rope(name):
 
 
 @pytest.mark.parametrize("name,scale", [("28x28", 1.0), ("ragged4", 1.0), ("mixed", 1.0), ("lines", 1.0),
-                                        ("tiny", 1.0), ("28x28", 3.0)])
+                                        ("tiny", 1.0), ("chunks", 1.0), ("28x28", 3.0)])
 def test_attention(name, scale):
     grids = GRID_SETS[name]
     b = A.BatchRef(grids)

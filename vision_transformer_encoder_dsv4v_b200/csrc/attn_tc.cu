@@ -41,8 +41,8 @@ constexpr int OFF_Q = 0;               // Q_A, Q_B
 constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
 constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
-constexpr int OFF_XCHG = OFF_BAR + 512;  // split mode: the second warpgroup's row max and sum (128 x 2 floats)
-constexpr int SMEM_BYTES = 1024 + OFF_XCHG + 1024;
+constexpr int OFF_XCHG = OFF_BAR + 512;  // split mode: each warpgroup's row max and sum (2 x 128 x 2 floats)
+constexpr int SMEM_BYTES = 1024 + OFF_XCHG + 2048;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kFirstSoftmaxWarp = 4;
 constexpr int kRegsControl = 56;    // warpgroup 0 after setmaxnreg
@@ -353,20 +353,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 2^(s c - m), some exponential pairs on the FMA pipe interleaved with the MUFU ones;
       // the bf16 pairs are packed in place into s[0 .. TK/2).  They are computed before waiting
       // for the previous P_X V product, which they overlap.
+      // A ragged last key tile skips the 32-column chunks that hold no key (their P is zero).
       const uint64_t sc2 = pk2(p.scale_log2, p.scale_log2), nm2 = pk2(-m_new, -m_new);
       uint64_t l2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < TK; c += 2) {
-        float x0, x1, e0, e1;
-        upk2(fma2(pk2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2), x0, x1);
-        if (poly_pair(c >> 1)) {
-          ex2_poly2(x0, x1, e0, e1);
-        } else {
-          e0 = ex2_mufu(x0);
-          e1 = ex2_mufu(x1);
+      for (int ch = 0; ch < TK / 32; ++ch) {
+        if (ch > 0 && 32 * ch >= valid) {
+#pragma unroll
+          for (int c = 32 * ch; c < 32 * ch + 32; c += 2) s[c >> 1] = 0u;
+          continue;
         }
-        l2[(c >> 1) & 3] = add2(l2[(c >> 1) & 3], pk2(e0, e1));
-        s[c >> 1] = pack_bf16x2(e0, e1);
+#pragma unroll
+        for (int c = 32 * ch; c < 32 * ch + 32; c += 2) {
+          float x0, x1, e0, e1;
+          upk2(fma2(pk2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2), x0, x1);
+          if (poly_pair(c >> 1)) {
+            ex2_poly2(x0, x1, e0, e1);
+          } else {
+            e0 = ex2_mufu(x0);
+            e1 = ex2_mufu(x1);
+          }
+          l2[(c >> 1) & 3] = add2(l2[(c >> 1) & 3], pk2(e0, e1));
+          s[c >> 1] = pack_bf16x2(e0, e1);
+        }
       }
       if (j > 0) {
         // P_X and O_X are free once the previous P_X V product has completed.
@@ -409,48 +418,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float* xchg = reinterpret_cast<float*>(smem + OFF_XCHG);
     if (split) {
-      // The second group hands its row max and sum to the first through shared memory; its O
-      // stays in TMEM, where the first group's thread of the same row (same TMEM lane) reads it.
-      if (x == 1) {
-        xchg[r] = ok ? m_used : -INFINITY;
-        xchg[128 + r] = ok && n_it > 0 ? l_run : 0.0f;
-        tc_fence_before_sync();
-      }
+      // The two groups swap their row max and sum through shared memory and each writes half of
+      // the output columns, [32 x, 32 x + 32), from both groups' O (same TMEM lane = same row):
+      //   O = O_0 2^(m_0 - m) + O_1 2^(m_1 - m),  l = l_0 2^(m_0 - m) + l_1 2^(m_1 - m).
+      const bool own = ok && n_it > 0;
+      xchg[x * 256 + r] = own ? m_used : -INFINITY;
+      xchg[x * 256 + 128 + r] = own ? l_run : 0.0f;
+      tc_fence_before_sync();
       named_barrier_sync(3, 256);
-      if (x == 1) ok = false;  // the first group writes the output
-      else tc_fence_after_sync();
-    }
-    if (ok) {
+      tc_fence_after_sync();
+      const float m_b = xchg[(1 - x) * 256 + r], l_b = xchg[(1 - x) * 256 + 128 + r];
+      constexpr int HH = HD / 2;
+      const uint32_t col = static_cast<uint32_t>(x * HH);
+      uint32_t oa[HH], ob[HH];
+      if (own) tmem_ld_cols<HH / 32>(t_o + col, oa);
+      if (__any_sync(0xffffffffu, l_b > 0.0f))
+        tmem_ld_cols<HH / 32>(t_lane + T_O + static_cast<uint32_t>((1 - x) * HD) + col, ob);
+      const float m = fmaxf(own ? m_used : -INFINITY, m_b);
+      const float fa = own ? ex2_mufu(m_used - m) : 0.0f;
+      const float fb = l_b > 0.0f ? ex2_mufu(m_b - m) : 0.0f;
+      const float l_tot = (own ? l_run * fa : 0.0f) + l_b * fb;
+      const int qi = q_tile * TQ + r;
+      if (qi < len && l_tot > 0.0f) {
+        if (x == 0 && p.lse) p.lse[static_cast<int64_t>(head) * p.lse_ld + row0 + qi] = m + __log2f(l_tot);
+        const float inv_l = 1.0f / l_tot;
+        const float ga = fa * inv_l, gb = fb * inv_l;
+        float o[HH];
+#pragma unroll
+        for (int c = 0; c < HH; ++c) {
+          const float va = own ? __uint_as_float(oa[c]) * ga : 0.0f;
+          o[c] = l_b > 0.0f ? fmaf(__uint_as_float(ob[c]), gb, va) : va;
+        }
+        uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + qi) * p.vision_dim + head * HD + col);
+#pragma unroll
+        for (int q = 0; q < HH / 8; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(o[8 * q + 0], o[8 * q + 1]);
+          v.y = pack_bf16x2(o[8 * q + 2], o[8 * q + 3]);
+          v.z = pack_bf16x2(o[8 * q + 4], o[8 * q + 5]);
+          v.w = pack_bf16x2(o[8 * q + 6], o[8 * q + 7]);
+          dst[q] = v;
+        }
+      }
+    } else if (ok) {
       tc_fence_after_sync();
       uint32_t o[HD];
       tmem_ld_cols<HD / 32>(t_o, o);
-      float l_tot = l_run;
-      if (split) {
-        const float m_b = xchg[r], l_b = xchg[128 + r];
-        if (l_b > 0.0f) {
-          // O = O_A 2^(m_A - m) + O_B 2^(m_B - m), l = l_A 2^(m_A - m) + l_B 2^(m_B - m)
-          const float m = fmaxf(m_used, m_b);
-          const float fa = n_it > 0 ? ex2_mufu(m_used - m) : 0.0f, fb = ex2_mufu(m_b - m);
-          uint32_t ob[HD];
-          tmem_ld_cols<HD / 32>(t_lane + T_O + static_cast<uint32_t>(HD), ob);
-#pragma unroll
-          for (int c = 0; c < HD; ++c)
-            o[c] = __float_as_uint((n_it > 0 ? __uint_as_float(o[c]) * fa : 0.0f) + __uint_as_float(ob[c]) * fb);
-          l_tot = (n_it > 0 ? l_run * fa : 0.0f) + l_b * fb;
-        }
-      }
-      const int qi = (q_tile + (split ? 0 : x)) * TQ + r;
-      if (qi < len && p.lse) {
-        // reference max of O's accumulation: the combined max in split mode, else m_used
-        float m_ref = m_used;
-        if (split) {
-          const float m_b = xchg[r], l_b = xchg[128 + r];
-          if (l_b > 0.0f) m_ref = fmaxf(m_used, m_b);
-        }
-        p.lse[static_cast<int64_t>(head) * p.lse_ld + row0 + qi] = m_ref + __log2f(l_tot);
-      }
+      const int qi = (q_tile + x) * TQ + r;
+      if (qi < len && p.lse) p.lse[static_cast<int64_t>(head) * p.lse_ld + row0 + qi] = m_used + __log2f(l_run);
       if (qi < len) {
-        const float inv_l = 1.0f / l_tot;
+        const float inv_l = 1.0f / l_run;
         uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row0 + qi) * p.vision_dim + head * HD);
 #pragma unroll
         for (int q = 0; q < HD / 8; ++q) {
