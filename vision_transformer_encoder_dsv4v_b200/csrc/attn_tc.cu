@@ -51,7 +51,7 @@ constexpr int kThreads = (kFirstSoftmaxWarp + kSoftmaxWarps) * 32;
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t T_S = 0, T_O = 256, T_P = 384;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr int kPolyPerEight = 1;    // exponential pairs per eight computed on the FMA pipe
+constexpr int kPolyPerEight = 0;    // exponential pairs per eight computed on the FMA pipe (0: all on MUFU)
 
 // Which exponential pairs (index i = column / 2) use the FMA-pipe polynomial.
 __host__ __device__ constexpr bool poly_pair(int i) {
@@ -81,8 +81,9 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for two x <= 0 at once on the FMA pipe, used for one softmax exponential in eight so
-// that the MUFU pipe is not the only one doing them.  Range reduction x = n + f with
+// 2^x for two x <= 0 at once on the FMA pipe, used for kPolyPerEight softmax exponential pairs
+// in eight so that the MUFU pipe is not the only one doing them (none by default: with two
+// softmax warpgroups per SM the MUFU pipe alone measured faster).  Range reduction x = n + f with
 // n = round(x) (the 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2]; 2^f by a cubic fitted here
 // for minimum relative error on that interval (max 7.5e-5, far below the bf16 rounding of P);
 // 2^n is added to the exponent field.  Inputs below -125 (masked keys included) return 0.
