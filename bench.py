@@ -327,9 +327,14 @@ def run_ours(args):
     if args.workload == 4:
         extras["workload5"] = workload5_timing(A, torch, lw, fnw, wa, stream, flush, min(args.steps, 10))
 
-    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region.
+    # Serial: every step copies its input in, runs the two calls, copies its result out, and the
+    # host waits for it.  Pipelined (the reported value): the same calls and copies for K steps on
+    # a compute stream and two copy streams with two device buffer sets, so that one step's copies
+    # overlap its neighbours' kernels, as a serving loop runs; one timed interval from the first
+    # input copy to the last result copy.
     x_host = x0.cpu().pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     e2e_ms = []
     for i in range(args.warmup + args.steps):
         with torch.cuda.stream(stream):
@@ -339,17 +344,53 @@ def run_ours(args):
             x.copy_(x_host, non_blocking=True)
             A.dsv4v_tower_forward(cfg, batch, lw, fnw, x, ws, stream=stream.cuda_stream)
             A.dsv4v_aligner_forward(cfg, batch, x, wa, out, ws, stream=stream.cuda_stream)
-            out_host.copy_(out, non_blocking=True)
+            out_host[0].copy_(out, non_blocking=True)
             b.record(stream)
         stream.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_total = sum(e2e_ms)
+    e2e_serial = sum(e2e_ms)
+
+    xs, outs = [x, torch.empty_like(x)], [out, torch.empty_like(out)]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "done", "out")}
+
+    def pipelined(n):
+        for i in range(n):
+            k = i & 1
+            if i >= 2:
+                h2d.wait_event(ev["done"][k])  # step i-2 has finished reading xs[k]
+            with torch.cuda.stream(h2d):
+                xs[k].copy_(x_host, non_blocking=True)
+            ev["in"][k].record(h2d)
+            stream.wait_event(ev["in"][k])
+            if i >= 2:
+                stream.wait_event(ev["out"][k])  # step i-2's result has left outs[k]
+            A.dsv4v_tower_forward(cfg, batch, lw, fnw, xs[k], ws, stream=stream.cuda_stream)
+            A.dsv4v_aligner_forward(cfg, batch, xs[k], wa, outs[k], ws, stream=stream.cuda_stream)
+            ev["done"][k].record(stream)
+            d2h.wait_event(ev["done"][k])
+            with torch.cuda.stream(d2h):
+                out_host[k].copy_(outs[k], non_blocking=True)
+            ev["out"][k].record(d2h)
+
+    pipelined(args.warmup)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        flush()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(h2d)
+    pipelined(args.steps)
+    t1.record(d2h)
+    torch.cuda.synchronize()
+    e2e_total = t0.elapsed_time(t1)
     if dist is not None:
-        t = torch.tensor([e2e_total], device="cuda")
+        t = torch.tensor([e2e_total, e2e_serial], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+        e2e_total, e2e_serial = float(t[0].item()), float(t[1].item())
     e2e_value = patches_all * args.steps / (e2e_total / 1e3)
+    e2e_serial_value = patches_all * args.steps / (e2e_serial / 1e3)
 
     peaks = load_peaks()
     dom = kern["dominant"]
@@ -390,7 +431,11 @@ def run_ours(args):
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x0.numel() * 2,
                         "d2h_bytes_per_step": out.numel() * 2,
                         "path": "dsv4v_tower_forward + dsv4v_aligner_forward direct C-ABI calls (no graph), "
-                                "pinned host input/output copies inside the timed region"},
+                                "pinned host input/output copies of every step inside the timed region; "
+                                "copies on two copy streams overlapping the neighbouring steps' kernels "
+                                "(two device buffer sets), one interval over all steps",
+                        "serial_value": e2e_serial_value,
+                        "serial_note": "each step alone: L2 flush, copy in, calls, copy out, host wait"},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if dist is not None:
