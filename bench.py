@@ -433,7 +433,8 @@ def run_ours(args):
                 "roofline": roof, "kernels": kern["all"], "extras": extras, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x0.numel() * 2,
                         "d2h_bytes_per_step": out.numel() * 2,
-                        "path": "dsv4v_tower_forward + dsv4v_aligner_forward direct C-ABI calls (no graph), "
+                        "path": "dsv4v_tower_forward + dsv4v_aligner_forward C-ABI calls (the library replays "
+                                "each call's CUDA graph from the second identical call on), "
                                 "pinned host input/output copies of every step inside the timed region; "
                                 "copies on two copy streams overlapping the neighbouring steps' kernels "
                                 "(two device buffer sets), one interval over all steps",

@@ -167,6 +167,49 @@ def test_profiled_tower_matches_plain(path):
         A.dsv4v_set_tower_path(A.PATH_AUTO)
 
 
+def test_graph_replay_matches_direct():
+    """Repeated step calls with identical arguments on a side stream replay a CUDA graph (the
+    first call launches directly, the second captures and replays, later calls replay).  Every
+    call's tower and aligner output equals the direct launches' bitwise, also when the input
+    behind the same pointer alternates between two values (the graph reads it when it runs)."""
+    wl = synth.workload(4)
+    inp = synth.draw(wl, n_layers=3)
+    cfg = config_of(wl, n_layers=3)
+    b = A.BatchRef(wl.grids)
+    ws = workspace(cfg, b)
+    layers = upload_layers(inp)
+    keep = [A.block_weights(l) for l in layers]
+    r, D = wl.downsample_ratio, wl.vision_dim
+    fnw = f32(np.linspace(0.5, 1.5, D))
+    wa = dev(random_bf16((wl.llm_dim, r * r * D), 0.02, seed=5))
+    xs = [dev(inp.x), (dev(inp.x).float() * -0.5).to(torch.bfloat16)]
+    xbuf = torch.empty_like(xs[0])
+    out = torch.empty(A.dsv4v_aligner_tokens(cfg, b), wl.llm_dim, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+
+    def step(i):
+        with torch.cuda.stream(s):
+            xbuf.copy_(xs[i % 2])
+        A.dsv4v_tower_forward(cfg, b, keep, fnw, xbuf, ws, stream=s.cuda_stream)
+        A.dsv4v_aligner_forward(cfg, b, xbuf, wa, out, ws, stream=s.cuda_stream)
+        s.synchronize()
+        assert A.dsv4v_device_error() == 0
+        return xbuf.clone(), out.clone()
+
+    try:
+        A.dsv4v_release_graphs()
+        A.dsv4v_set_graph_replay(False)
+        ref = [step(0), step(1)]
+        A.dsv4v_set_graph_replay(True)
+        for i in range(6):
+            got = step(i)
+            assert torch.equal(got[0], ref[i % 2][0]) and torch.equal(got[1], ref[i % 2][1]), i
+        assert not torch.equal(ref[0][1], ref[1][1])
+    finally:
+        A.dsv4v_set_graph_replay(True)
+        A.dsv4v_release_graphs()
+
+
 def test_workload4_tower_aligner(workload4):
     wl, inp, tower_o, align_o = workload4
     tower_g, align_g = run_tower_and_aligner(wl, inp)

@@ -842,11 +842,132 @@ dsv4v_status linear_residual_with_scratch(const dsv4v_config* cfg, int64_t rows,
   return gemm_bf16(c, EPI_RESID, plan, a, rows, k, w, nullptr, c.s.D, x, x, nullptr, nullptr, NormFold(), ex);
 }
 
+// ----------------------------------------------------------------------------- graph replay
+// A step of the 28x28 tower is ~170 launches of ~11 us each, so launching them one by one from
+// the host costs a few percent against replaying them as one CUDA graph.  The step entry points
+// therefore keep a small cache of graph executables keyed by every argument that shapes their
+// launches (the config, the batch's host arrays and device pointers, the weight, buffer and
+// workspace pointers, the launch-sequence setting, the device).  The first call with a key runs
+// eagerly (it also warms the plan and descriptor caches); the second captures the launches on
+// the caller's stream (thread-local capture) and replays the instantiated graph, as do all
+// later calls.  Calls on the legacy default stream, or on a stream that is already being
+// captured (the caller's own graph), always launch directly.  A capture or instantiation that
+// fails leaves that key on direct launches.
+struct GraphEntry {
+  std::vector<uint64_t> key;
+  cudaGraphExec_t exec = nullptr;
+  int state = 0;  // 1: seen once, 2: graph ready, -1: direct launches only
+  uint64_t last_use = 0;
+};
+
+std::mutex g_graph_mu;
+std::vector<GraphEntry> g_graphs;
+uint64_t g_graph_clock = 0;
+std::atomic<int> g_graph_replay{1};
+constexpr size_t kMaxGraphs = 16;
+
+struct KeyBuilder {
+  std::vector<uint64_t> k;
+  void u(uint64_t v) { k.push_back(v); }
+  void p(const void* ptr) { k.push_back(reinterpret_cast<uint64_t>(ptr)); }
+  void bytes(const void* src, size_t n) {
+    const uint8_t* b = static_cast<const uint8_t*>(src);
+    for (size_t i = 0; i < n; i += 8) {
+      uint64_t v = 0;
+      memcpy(&v, b + i, std::min<size_t>(8, n - i));
+      k.push_back(v);
+    }
+  }
+};
+
+// Key prefix shared by the step entry points: which call, the device, the setting, the config
+// and the batch (host values and device pointers).
+KeyBuilder step_key(int call, const dsv4v_config* cfg, const dsv4v_batch* batch) {
+  KeyBuilder kb;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  kb.u(static_cast<uint64_t>(call));
+  kb.u(static_cast<uint64_t>(dev));
+  kb.u(static_cast<uint64_t>(g_tower_path.load()));
+  kb.bytes(cfg, sizeof(*cfg));
+  kb.u(static_cast<uint64_t>(batch->n_images));
+  kb.p(batch->grid_hw_dev);
+  kb.p(batch->cu_patches_dev);
+  kb.bytes(batch->grid_hw_host, sizeof(int32_t) * 2 * static_cast<size_t>(batch->n_images));
+  kb.bytes(batch->cu_patches_host, sizeof(int32_t) * (static_cast<size_t>(batch->n_images) + 1));
+  return kb;
+}
+
+template <class Run>
+dsv4v_status with_graph(KeyBuilder&& kb, void* stream, Run&& run) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!g_graph_replay.load() || s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread) return run();
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return run();
+  }
+  if (cs != cudaStreamCaptureStatusNone) return run();
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  GraphEntry* e = nullptr;
+  for (auto& g : g_graphs)
+    if (g.key == kb.k) {
+      e = &g;
+      break;
+    }
+  if (e == nullptr) {
+    if (g_graphs.size() >= kMaxGraphs) {
+      // evict the least recently used entry (an executable still in flight is freed when it
+      // completes)
+      auto lru = std::min_element(g_graphs.begin(), g_graphs.end(),
+                                  [](const GraphEntry& a, const GraphEntry& b) { return a.last_use < b.last_use; });
+      if (lru->exec) cudaGraphExecDestroy(lru->exec);
+      g_graphs.erase(lru);
+    }
+    g_graphs.push_back(GraphEntry{std::move(kb.k), nullptr, 1, ++g_graph_clock});
+    return run();
+  }
+  e->last_use = ++g_graph_clock;
+  if (e->state == 2) return cuda_status(cudaGraphLaunch(e->exec, s));
+  if (e->state < 0) return run();
+  // Second call with this key: capture it.
+  if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    e->state = -1;
+    return run();
+  }
+  const dsv4v_status st = run();
+  cudaGraph_t graph = nullptr;
+  const cudaError_t end = cudaStreamEndCapture(s, &graph);
+  cudaGraphExec_t exec = nullptr;
+  cudaError_t inst = cudaErrorUnknown;
+  if (st == DSV4V_OK && end == cudaSuccess && graph != nullptr) inst = cudaGraphInstantiate(&exec, graph, 0);
+  if (graph) cudaGraphDestroy(graph);
+  if (inst != cudaSuccess) {
+    // nothing of the captured call ran: run it directly
+    cudaGetLastError();
+    e->state = -1;
+    return st == DSV4V_OK ? run() : st;
+  }
+  e->exec = exec;
+  e->state = 2;
+  return cuda_status(cudaGraphLaunch(exec, s));
+}
+
 }  // namespace dsv4v
 
 using namespace dsv4v;
 
 extern "C" {
+
+void dsv4v_set_graph_replay(int enable) { g_graph_replay.store(enable ? 1 : 0); }
+
+void dsv4v_release_graphs(void) {
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  for (auto& g : g_graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  g_graphs.clear();
+}
 
 const char* dsv4v_status_string(dsv4v_status s) {
   switch (s) {
@@ -951,7 +1072,16 @@ static dsv4v_status tower_impl(const dsv4v_config* cfg, const dsv4v_batch* batch
 dsv4v_status dsv4v_tower_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const dsv4v_block_weights* layers,
                                  const float* final_norm_w, void* x_inout, void* workspace, size_t ws_bytes,
                                  void* stream) {
-  return tower_impl(cfg, batch, layers, final_norm_w, x_inout, workspace, ws_bytes, stream, nullptr);
+  auto run = [&] { return tower_impl(cfg, batch, layers, final_norm_w, x_inout, workspace, ws_bytes, stream, nullptr); };
+  Shape sh;
+  if (check_all(cfg, batch, sh) != DSV4V_OK || (cfg->n_layers > 0 && !layers)) return run();
+  KeyBuilder kb = step_key(1, cfg, batch);
+  kb.bytes(layers, sizeof(dsv4v_block_weights) * static_cast<size_t>(cfg->n_layers));
+  kb.p(final_norm_w);
+  kb.p(x_inout);
+  kb.p(workspace);
+  kb.u(ws_bytes);
+  return with_graph(std::move(kb), stream, run);
 }
 
 dsv4v_status dsv4v_tower_forward_profiled(const dsv4v_config* cfg, const dsv4v_batch* batch,
@@ -961,21 +1091,11 @@ dsv4v_status dsv4v_tower_forward_profiled(const dsv4v_config* cfg, const dsv4v_b
   return tower_impl(cfg, batch, layers, final_norm_w, x_inout, workspace, ws_bytes, stream, events);
 }
 
-dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x,
-                                   const void* w_align, void* out, int32_t* cu_tokens_host, void* workspace,
-                                   size_t ws_bytes, void* stream) {
+static dsv4v_status aligner_impl(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x,
+                                 const void* w_align, void* out, void* workspace, size_t ws_bytes, void* stream) {
   Ctx c;
   DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
   if (!x || !w_align || !out || !aligned16(x) || !aligned16(w_align) || !aligned16(out)) return DSV4V_ERR_INVALID_ARG;
-  if (cu_tokens_host) {
-    int64_t t = 0;
-    cu_tokens_host[0] = 0;
-    for (int i = 0; i < batch->n_images; ++i) {
-      const int n_h = batch->grid_hw_host[2 * i], n_w = batch->grid_hw_host[2 * i + 1];
-      t += static_cast<int64_t>((n_h + c.s.r - 1) / c.s.r) * ((n_w + c.s.r - 1) / c.s.r);
-      cu_tokens_host[i + 1] = static_cast<int32_t>(t);
-    }
-  }
   const Shape& s = c.s;
   int32_t* src = c.at<int32_t>(c.lay.asrc);
   DSV4V_TRY(cuda_status(launch_aligner_index(batch->cu_patches_dev, batch->grid_hw_dev, batch->n_images, s.r, s.T,
@@ -994,6 +1114,31 @@ dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* b
   DSV4V_TRY(cuda_status(launch_gather_f32(static_cast<const float*>(x), src, merged, s.T, s.r * s.r, s.D, c.stream)));
   return cuda_status(launch_gemm_f32(EPI_STORE, merged, static_cast<const float*>(w_align), nullptr,
                                      static_cast<float*>(out), nullptr, static_cast<int>(s.T), s.E, K, c.stream));
+}
+
+dsv4v_status dsv4v_aligner_forward(const dsv4v_config* cfg, const dsv4v_batch* batch, const void* x,
+                                   const void* w_align, void* out, int32_t* cu_tokens_host, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  Shape sh;
+  if (check_all(cfg, batch, sh) != DSV4V_OK) return aligner_impl(cfg, batch, x, w_align, out, workspace, ws_bytes, stream);
+  if (cu_tokens_host) {
+    // host output: written on every call, replayed or not
+    int64_t t = 0;
+    cu_tokens_host[0] = 0;
+    for (int i = 0; i < batch->n_images; ++i) {
+      const int n_h = batch->grid_hw_host[2 * i], n_w = batch->grid_hw_host[2 * i + 1];
+      t += static_cast<int64_t>((n_h + sh.r - 1) / sh.r) * ((n_w + sh.r - 1) / sh.r);
+      cu_tokens_host[i + 1] = static_cast<int32_t>(t);
+    }
+  }
+  KeyBuilder kb = step_key(2, cfg, batch);
+  kb.p(x);
+  kb.p(w_align);
+  kb.p(out);
+  kb.p(workspace);
+  kb.u(ws_bytes);
+  return with_graph(std::move(kb), stream,
+                    [&] { return aligner_impl(cfg, batch, x, w_align, out, workspace, ws_bytes, stream); });
 }
 
 // Scratch of the PatchMerger projector: window index [T, r^2] int32, merged rows and hidden rows

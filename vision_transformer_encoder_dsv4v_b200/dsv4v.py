@@ -40,7 +40,7 @@ EXPORTS = ("dsv4v_workspace_size", "dsv4v_rope2d_table", "dsv4v_block_forward", 
            "dsv4v_bridge_workspace_size", "dsv4v_merge_image_embeddings", "dsv4v_image_visibility",
            "dsv4v_backward_workspace_size", "dsv4v_attention_backward", "dsv4v_rmsnorm_backward",
            "dsv4v_block_backward", "dsv4v_tower_backward", "dsv4v_set_tower_path", "dsv4v_tower_path",
-           "dsv4v_step_launches")
+           "dsv4v_step_launches", "dsv4v_set_graph_replay", "dsv4v_release_graphs")
 
 DSV4V_NOALLOC_MAX_ROWS = 65536
 
@@ -118,6 +118,8 @@ def lib() -> ctypes.CDLL:
             "dsv4v_set_tower_path": (I, [I]),
             "dsv4v_tower_path": (I, [cfg, bat]),
             "dsv4v_step_launches": (I, [cfg, bat, I, I]),
+            "dsv4v_set_graph_replay": (None, [I]),
+            "dsv4v_release_graphs": (None, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -198,6 +200,18 @@ def dsv4v_tower_forward(cfg, batch, layers, final_norm_w, x_inout, workspace, st
     _check(lib().dsv4v_tower_forward(ctypes.byref(cfg), ctypes.byref(batch.c), arr, _ptr(final_norm_w),
                                      _ptr(x_inout), _ptr(workspace), workspace.numel(), _stream(stream)),
            "dsv4v_tower_forward")
+
+
+def dsv4v_set_graph_replay(enable):
+    """Process-wide switch of the step calls' graph replay (on by default): repeated
+    dsv4v_tower_forward / dsv4v_aligner_forward calls with identical arguments on a non-default
+    stream replay a CUDA graph captured on the second such call."""
+    lib().dsv4v_set_graph_replay(1 if enable else 0)
+
+
+def dsv4v_release_graphs():
+    """Destroys every cached graph executable of the step calls."""
+    lib().dsv4v_release_graphs()
 
 
 def dsv4v_set_tower_path(path):
