@@ -849,7 +849,49 @@ __global__ void __launch_bounds__(192, 1)
         }
         uint8_t* box = nullptr;
         constexpr bool WIDE = kSwWide<EPI, BN>;
-        constexpr int NG = WIDE ? 6 : NGROUPS;  // WIDE: 5.5 groups of 32 output columns
+        if constexpr (WIDE) {
+          // 5.5 groups of 32 output columns, two at a time (one 64-column box): both groups'
+          // accumulator columns are loaded together and their math is independent, so it can
+          // interleave.  Columns [128, 176) are stored directly (a 64-column box would spill
+          // into the next tile).
+#pragma unroll 1
+          for (int g = 0; g < 6; g += 2) {
+            int c0, c1, c2, c3;
+            group_chunks<EPI, BN>(g, c0, c1);
+            group_chunks<EPI, BN>(g + 1, c2, c3);
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tmem_ld32(t_row + c0 * 32, r0);
+            tmem_ld32(t_row + c1 * 32, r1);
+            tmem_ld32(t_row + c2 * 32, r2);
+            tmem_ld32(t_row + c3 * 32, r3);
+            tmem_ld_wait(r0);
+            tmem_ld_wait(r1);
+            tmem_ld_wait(r2);
+            tmem_ld_wait(r3);
+            float v[64], w[64];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              v[j] = __uint_as_float(r0[j]);
+              v[32 + j] = __uint_as_float(r1[j]);
+              w[j] = __uint_as_float(r2[j]);
+              w[32 + j] = __uint_as_float(r3[j]);
+            }
+            const int col = sg.n_tile * (BN / 2) + 32 * g;
+            if (g == 4) {
+              swiglu_store_direct(p, row, col, v, row_scale, 32);
+              swiglu_store_direct(p, row, col + 32, w, row_scale, 16);
+              continue;
+            }
+            uint8_t* box2 = nullptr;
+            box = st.acquire();
+            epilogue_group<EPI, BN>(p, row, sg.n_tile, g, v, rot_c, rot_s, row_scale, nullptr, xw_s, ss_acc, st, box,
+                                    box2);
+            epilogue_group<EPI, BN>(p, row, sg.n_tile, g + 1, w, rot_c, rot_s, row_scale, nullptr, xw_s, ss_acc, st,
+                                    box, box2);
+            st.store(box, &tm_out, col, box_y, p.M);
+          }
+        }
+        constexpr int NG = WIDE ? 0 : NGROUPS;
         // Unrolled for the residual epilogue so that its prefetched residual row stays in registers.
 #pragma unroll(EPI == EPI_RESID ? NGROUPS : 1)
         for (int g = 0; g < NG; ++g) {
@@ -889,11 +931,6 @@ __global__ void __launch_bounds__(192, 1)
                 v[32 + 4 * q + 3] += b[q].w;
               }
             }
-          }
-          if (WIDE && g >= 4) {
-            // columns [128, 176) of the tile: a 64-column box would spill into the next tile
-            swiglu_store_direct(p, row, sg.n_tile * (BN / 2) + 32 * g, v, row_scale, g == 4 ? 32 : 16);
-            continue;
           }
           uint8_t* box2 = nullptr;
           if (EPI == EPI_RESID && p.xw_out) st.acquire_both(box, box2);
