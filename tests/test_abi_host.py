@@ -170,18 +170,10 @@ def test_backward_host_checks(lib):
                                         None) == 2
     assert lib.dsv4v_block_backward(ctypes.byref(f32), ctypes.byref(b.c), None, None, None, None, None, None, None,
                                     None, 0, None) == 2
-    # the scratch grows with the patches: every activation, gradient and transpose is kept
+    # the scratch grows with the patches: every activation and gradient of the block is kept
     small = lib.dsv4v_backward_workspace_size(ctypes.byref(cfg()), ctypes.byref(HostBatch([(3, 5)]).c))
     big = lib.dsv4v_backward_workspace_size(ctypes.byref(cfg()), ctypes.byref(b.c))
     assert 0 < small < big
-
-
-def test_backward_rejects_batches_past_the_transpose_grid(lib):
-    # the transposes cover P rows in 32-row CTAs along grid.y (at most 65535): a 1500 x 1500 image
-    # (2.25 M patches) is refused on the host, before any CUDA call
-    b = HostBatch([(1500, 1500)])
-    assert lib.dsv4v_block_backward(ctypes.byref(cfg()), ctypes.byref(b.c), None, None, None, None, None, None, None,
-                                    None, 0, None) == 2
 
 
 def test_header_compiles_as_c99_and_links(lib, tmp_path):

@@ -408,6 +408,11 @@ struct GemmExtra {
   // Weights of the GEMM that follows, prefetched into L2 by this one (see GemmArgs).
   const void* l2_next[2] = {nullptr, nullptr};
   size_t l2_next_bytes[2] = {0, 0};
+  // MN-major operands (STORE only, see GemmArgs::mn_major): a_mn, A is given as its stored
+  // [K, M] matrix (row stride lda); b_mn, B as its stored [K, n_out] matrix (row stride ldb),
+  // continued along K by b2 from K row kb_split * 64 on when b2 is set.
+  bool a_mn = false, b_mn = false;
+  int kb_split = 0;
 };
 
 GemmExtra prefetching(const void* w0, size_t bytes0, const void* w1 = nullptr, size_t bytes1 = 0) {
@@ -424,9 +429,14 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
                        const float* sin = nullptr, const NormFold& nf = NormFold(), const GemmExtra& ex = GemmExtra()) {
   if (M == 0) return DSV4V_OK;
   const int box_b = (epi == EPI_SWIGLU || plan.pair) ? plan.bn / 2 : plan.bn;
+  const bool b_split = ex.b_mn && b2 != nullptr;
+  const int k_b1 = b_split ? ex.kb_split * 64 : K;  // K rows of B held by b
   CUtensorMap ta, tb, tb2, t_out, t_xw;
-  if (!bf16_map(a, M, K, 128, &ta, ex.lda) || !bf16_map(b, n_out, K, box_b, &tb, ex.ldb) ||
-      (epi == EPI_SWIGLU && !bf16_map(b2, n_out, K, box_b, &tb2)) || !bf16_map(out, M, n_out, 32, &t_out) ||
+  const bool a_ok = ex.a_mn ? bf16_map(a, K, M, 64, &ta, ex.lda) : bf16_map(a, M, K, 128, &ta, ex.lda);
+  const bool b_ok = ex.b_mn ? bf16_map(b, k_b1, n_out, 64, &tb, ex.ldb) : bf16_map(b, n_out, K, box_b, &tb, ex.ldb);
+  const bool b2_ok = b_split ? bf16_map(b2, K - k_b1, n_out, 64, &tb2, ex.ldb)
+                             : (epi != EPI_SWIGLU || bf16_map(b2, n_out, K, box_b, &tb2));
+  if (!a_ok || !b_ok || !b2_ok || !bf16_map(out, M, n_out, 32, &t_out) ||
       (nf.xw_out && !bf16_map(nf.xw_out, M, n_out, 32, &t_xw)))
     return DSV4V_ERR_CUDA;
   GemmArgs g{};
@@ -434,7 +444,9 @@ dsv4v_status gemm_bf16(const Ctx& c, int epi, const GemmPlan& plan, const void* 
   g.tm_xw = nf.xw_out ? &t_xw : nullptr;
   g.tm_a = &ta;
   g.tm_b = &tb;
-  g.tm_b2 = epi == EPI_SWIGLU ? &tb2 : nullptr;
+  g.tm_b2 = (epi == EPI_SWIGLU || b_split) ? &tb2 : nullptr;
+  g.mn_major = (ex.b_mn ? 1 : 0) | (ex.a_mn ? 2 : 0) | (b_split ? 4 : 0);
+  g.kb_split = b_split ? ex.kb_split : 0;
   g.M = static_cast<int>(M);
   g.K = K;
   g.n_out = n_out;
@@ -1449,23 +1461,17 @@ namespace {
 constexpr int kNormParts = 512;  // most CTAs of one RMSNorm backward (each leaves a [D] partial)
 
 // Scratch of the backward calls, after the forward layout (whose split-tile scratch and
-// rotation tables the recompute reuses).  Activations and gradients are bf16 [P, width];
-// transposed operands of the weight-gradient GEMMs are bf16 [width, ldp] (ldp = P rounded up to
-// a multiple of 8, 16-byte TMA rows); transposed weights; fp32 attention row statistics and
-// RMSNorm partials.
+// rotation tables the recompute reuses).  Activations and gradients are bf16 [P, width]; fp32
+// attention row statistics and RMSNorm partials.  The gradient GEMMs read every operand where
+// it lies (MN-major where needed), so there are no transposed copies.
 struct BwdLayout {
-  int64_t ldp;
   size_t y1, qkv, att, x2, y2, g, u, h, dh, dgu, dy2, dx2, datt, dqkv, dy1, dcur0, dcur1;
-  size_t dout_t, h_t, dgu_t, y2_t, dx2_t, att_t, dqkv_t, y1_t;
-  size_t wd_t, wgu_t, wo_t, wqkv_t, lse, rowdot, norm_parts, total;
+  size_t lse, rowdot, norm_parts, total;
 };
 
 BwdLayout bwd_layout(const Shape& s, size_t fwd_total) {
   BwdLayout l{};
   const size_t P = static_cast<size_t>(s.P), D = s.D, F = s.F;
-  l.ldp = (s.P + 7) / 8 * 8;
-  if (l.ldp < 8) l.ldp = 8;
-  const size_t ldp = static_cast<size_t>(l.ldp);
   size_t off = up256(fwd_total);
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -1489,18 +1495,6 @@ BwdLayout bwd_layout(const Shape& s, size_t fwd_total) {
   l.dy1 = take(P * D * 2);
   l.dcur0 = take(P * D * 2);
   l.dcur1 = take(P * D * 2);
-  l.dout_t = take(D * ldp * 2);
-  l.h_t = take(F * ldp * 2);
-  l.dgu_t = take(2 * F * ldp * 2);
-  l.y2_t = take(D * ldp * 2);
-  l.dx2_t = take(D * ldp * 2);
-  l.att_t = take(D * ldp * 2);
-  l.dqkv_t = take(3 * D * ldp * 2);
-  l.y1_t = take(D * ldp * 2);
-  l.wd_t = take(F * D * 2);
-  l.wgu_t = take(D * 2 * F * 2);
-  l.wo_t = take(D * D * 2);
-  l.wqkv_t = take(D * 3 * D * 2);
   l.lse = take(P * s.H * 4);
   l.rowdot = take(P * s.H * 4);
   l.norm_parts = take(static_cast<size_t>(kNormParts) * D * 4);
@@ -1508,12 +1502,11 @@ BwdLayout bwd_layout(const Shape& s, size_t fwd_total) {
   return l;
 }
 
-// The backward calls are bf16 only and need a grid that the transposes can cover.
+// The backward calls are bf16 only.
 dsv4v_status bwd_prepare(const dsv4v_config* cfg, const dsv4v_batch* batch, void* workspace, size_t ws_bytes,
                          void* stream, Ctx& c, BwdLayout& bl) {
   DSV4V_TRY(check_all(cfg, batch, c.s));
   if (!c.s.bf16) return DSV4V_ERR_UNSUPPORTED;
-  if ((c.s.P + 31) / 32 > 65535) return DSV4V_ERR_UNSUPPORTED;
   DSV4V_TRY(prepare(cfg, batch, workspace, ws_bytes, stream, c));
   bl = bwd_layout(c.s, c.lay.total);
   if (ws_bytes < bl.total) return DSV4V_ERR_WORKSPACE;
@@ -1538,10 +1531,23 @@ dsv4v_status gemm_store(const Ctx& c, const void* a, int64_t M, int K, int64_t l
   return gemm_bf16(c, EPI_STORE, plan, a, M, K, b, nullptr, n_out, out, nullptr, nullptr, nullptr, NormFold(), ex);
 }
 
-dsv4v_status transpose(const Ctx& c, const void* in, int64_t rows, int cols, void* out, int64_t ld_out,
-                       int64_t col0 = 0) {
-  return cuda_status(launch_transpose_bf16(in, rows, cols, cols, out, ld_out, col0, c.stream));
+// out[M, n_out] = A . B with either operand given as its stored matrix (MN-major, no transposed
+// copy): a_mn, A is stored [K, M] (row stride lda), else [M, K]; b_mn, B is stored [K, n_out]
+// (row stride ldb; with b2, its rows from kb_split * 64 on are b2's rows), else [n_out, K].
+dsv4v_status gemm_store_mn(const Ctx& c, const void* a, int64_t M, int K, int64_t lda, bool a_mn, const void* b,
+                           int64_t ldb, bool b_mn, int n_out, void* out, const void* b2 = nullptr, int kb_split = 0) {
+  const GemmPlan plan = plan_gemm_whole(static_cast<int>(M), n_out, K, c.dev.sms);
+  if (plan.bn == 0) return DSV4V_ERR_UNSUPPORTED;
+  GemmExtra ex;
+  ex.lda = lda;
+  ex.ldb = ldb;
+  ex.b_early = false;  // B may be an activation written earlier in the call
+  ex.a_mn = a_mn;
+  ex.b_mn = b_mn;
+  ex.kb_split = kb_split;
+  return gemm_bf16(c, EPI_STORE, plan, a, M, K, b, b2, n_out, out, nullptr, nullptr, nullptr, NormFold(), ex);
 }
+
 
 
 // Attention backward on tcgen05.  lse_ready: bl.lse already holds the forward's per-row
@@ -1580,7 +1586,7 @@ dsv4v_status block_backward_bf16(const Ctx& c, const BwdLayout& bl, const dsv4v_
                                  const dsv4v_block_weights* w, const float* cos, const float* sin, const void* x,
                                  const void* dout, void* dx, const dsv4v_block_grads* gr) {
   const Shape& s = c.s;
-  const int64_t P = s.P, ldp = bl.ldp;
+  const int64_t P = s.P;
   const int D = s.D, F = s.F;
   void* y1 = c.at<void>(bl.y1);
   void* qkv = c.at<void>(bl.qkv);
@@ -1597,13 +1603,7 @@ dsv4v_status block_backward_bf16(const Ctx& c, const BwdLayout& bl, const dsv4v_
   void* datt = c.at<void>(bl.datt);
   void* dqkv = c.at<void>(bl.dqkv);
   void* dy1 = c.at<void>(bl.dy1);
-  uint8_t* dgu_t = c.at<uint8_t>(bl.dgu_t);
-  // transposed weights: the input-gradient GEMMs read W^T rows
-  DSV4V_TRY(transpose(c, w->w_down, D, F, c.at<void>(bl.wd_t), D));
-  DSV4V_TRY(transpose(c, w->w_gate, F, D, c.at<void>(bl.wgu_t), 2 * F, 0));
-  DSV4V_TRY(transpose(c, w->w_up, F, D, c.at<void>(bl.wgu_t), 2 * F, F));
-  DSV4V_TRY(transpose(c, w->wo, D, D, c.at<void>(bl.wo_t), D));
-  DSV4V_TRY(transpose(c, w->wqkv, 3 * D, D, c.at<void>(bl.wqkv_t), 3 * D));
+  const int Pk = static_cast<int>(P);  // K of the weight-gradient GEMMs (they reduce over the rows)
   // recompute the block's intermediates
   DSV4V_TRY(cuda_status(launch_rmsnorm(true, x, w->norm1_w, y1, P, D, c.eps, c.stream)));
   DSV4V_TRY(reset_counters(c));
@@ -1615,33 +1615,27 @@ dsv4v_status block_backward_bf16(const Ctx& c, const BwdLayout& bl, const dsv4v_
   DSV4V_TRY(cuda_status(launch_rmsnorm(true, x2, w->norm2_w, y2, P, D, c.eps, c.stream)));
   DSV4V_TRY(gemm_store(c, y2, P, D, 0, w->w_gate, 0, F, g));
   DSV4V_TRY(gemm_store(c, y2, P, D, 0, w->w_up, 0, F, u));
-  // MLP branch
-  DSV4V_TRY(gemm_store(c, dout, P, D, 0, c.at<void>(bl.wd_t), 0, F, dh));
+  // MLP branch.  Input gradients read each weight as stored ([K, n]: MN-major B); weight
+  // gradients reduce over the rows and read both the output gradient and the activation as
+  // stored ([P, width]: MN-major A and B), so no operand is transposed.
+  DSV4V_TRY(gemm_store_mn(c, dout, P, D, 0, false, w->w_down, F, true, F, dh));  // dh = dout . w_down
   DSV4V_TRY(cuda_status(launch_swiglu_bwd(g, u, dh, dgu, h, P, F, c.dev.sms, c.stream)));
-  DSV4V_TRY(transpose(c, dout, P, D, c.at<void>(bl.dout_t), ldp));
-  DSV4V_TRY(transpose(c, h, P, F, c.at<void>(bl.h_t), ldp));
-  DSV4V_TRY(gemm_store(c, c.at<void>(bl.dout_t), D, static_cast<int>(P), ldp, c.at<void>(bl.h_t), ldp, F, gr->w_down));
-  DSV4V_TRY(gemm_store(c, dgu, P, 2 * F, 0, c.at<void>(bl.wgu_t), 0, D, dy2));
-  DSV4V_TRY(transpose(c, dgu, P, 2 * F, dgu_t, ldp));
-  DSV4V_TRY(transpose(c, y2, P, D, c.at<void>(bl.y2_t), ldp));
-  DSV4V_TRY(gemm_store(c, dgu_t, F, static_cast<int>(P), ldp, c.at<void>(bl.y2_t), ldp, D, gr->w_gate));
-  DSV4V_TRY(gemm_store(c, dgu_t + static_cast<size_t>(F) * ldp * 2, F, static_cast<int>(P), ldp,
-                       c.at<void>(bl.y2_t), ldp, D, gr->w_up));
+  DSV4V_TRY(gemm_store_mn(c, dout, D, Pk, D, true, h, F, true, F, gr->w_down));  // dout^T . h
+  // dy2 = [dg | du] . [w_gate; w_up]: B's K rows continue from w_gate into w_up (F % 64 == 0)
+  DSV4V_TRY(gemm_store_mn(c, dgu, P, 2 * F, 0, false, w->w_gate, D, true, D, dy2, w->w_up, F / 64));
+  DSV4V_TRY(gemm_store_mn(c, dgu, F, Pk, 2 * F, true, y2, D, true, D, gr->w_gate));  // dg^T . y2
+  DSV4V_TRY(gemm_store_mn(c, dgu + static_cast<size_t>(F) * 2, F, Pk, 2 * F, true, y2, D, true, D,
+                          gr->w_up));  // du^T . y2
   // norm2 and the residual
   DSV4V_TRY(rmsnorm_bwd(c, bl, x2, w->norm2_w, dy2, dout, dx2, gr->norm2_w));
   // output projection
-  DSV4V_TRY(gemm_store(c, dx2, P, D, 0, c.at<void>(bl.wo_t), 0, D, datt));
-  DSV4V_TRY(transpose(c, dx2, P, D, c.at<void>(bl.dx2_t), ldp));
-  DSV4V_TRY(transpose(c, att, P, D, c.at<void>(bl.att_t), ldp));
-  DSV4V_TRY(gemm_store(c, c.at<void>(bl.dx2_t), D, static_cast<int>(P), ldp, c.at<void>(bl.att_t), ldp, D, gr->wo));
+  DSV4V_TRY(gemm_store_mn(c, dx2, P, D, 0, false, w->wo, D, true, D, datt));      // dx2 . wo
+  DSV4V_TRY(gemm_store_mn(c, dx2, D, Pk, D, true, att, D, true, D, gr->wo));      // dx2^T . att
   // attention, rotation, fused projection
   DSV4V_TRY(attention_bwd(c, bl, batch, qkv, att, datt, dqkv, true));
   DSV4V_TRY(cuda_status(launch_rotary_bwd(dqkv, cos, sin, P, D, s.hd, c.dev.sms, c.stream)));
-  DSV4V_TRY(gemm_store(c, dqkv, P, 3 * D, 0, c.at<void>(bl.wqkv_t), 0, D, dy1));
-  DSV4V_TRY(transpose(c, dqkv, P, 3 * D, c.at<void>(bl.dqkv_t), ldp));
-  DSV4V_TRY(transpose(c, y1, P, D, c.at<void>(bl.y1_t), ldp));
-  DSV4V_TRY(gemm_store(c, c.at<void>(bl.dqkv_t), 3 * D, static_cast<int>(P), ldp, c.at<void>(bl.y1_t), ldp, D,
-                       gr->wqkv));
+  DSV4V_TRY(gemm_store_mn(c, dqkv, P, 3 * D, 0, false, w->wqkv, D, true, D, dy1));     // dqkv . wqkv
+  DSV4V_TRY(gemm_store_mn(c, dqkv, 3 * D, Pk, 3 * D, true, y1, D, true, D, gr->wqkv));  // dqkv^T . y1
   // norm1 and the residual
   return rmsnorm_bwd(c, bl, x, w->norm1_w, dy1, dx2, dx, gr->norm1_w);
 }

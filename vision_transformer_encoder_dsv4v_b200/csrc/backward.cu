@@ -1,8 +1,8 @@
 // Backward pass of the tower block ([PR], Validation: "ragged grids and backward"): the steps
 // that are neither GEMMs nor attention.  The weight and input gradients of the four projections
-// run on the tcgen05 GEMM (api.cu), fed with transposed operands from k_transpose_bf16; the
-// attention backward is attn_bwd_tc.cu; this file holds the transposes, the RMSNorm and SwiGLU
-// backward and the inverse rotation.
+// run on the tcgen05 GEMM (api.cu), which reads the activations, gradients and weights where
+// they lie (MN-major operands where needed); the attention backward is attn_bwd_tc.cu; this
+// file holds the RMSNorm and SwiGLU backward and the inverse rotation.
 #include <algorithm>
 
 #include "common.cuh"
@@ -11,31 +11,6 @@
 namespace dsv4v {
 
 namespace {
-
-// ------------------------------------------------------------------------------ transpose
-// out[c * ld_out + col0 + r] = in[r * ld_in + c] for r < rows, c < cols: a 32 x 32 tile per CTA
-// through shared memory, so that both the reads and the writes run along rows.
-__global__ void __launch_bounds__(256)
-    k_transpose_bf16(const __nv_bfloat16* __restrict__ in, int64_t rows, int cols, int64_t ld_in,
-                     __nv_bfloat16* __restrict__ out, int64_t ld_out, int64_t col0) {
-  __shared__ __nv_bfloat16 tile[32][34];
-  grid_dependency_wait();
-  launch_dependents();
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32;
-  const int c0 = blockIdx.x * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t r = r0 + i;
-    const int c = c0 + tx;
-    if (r < rows && c < cols) tile[i][tx] = in[r * ld_in + c];
-  }
-  __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int c = c0 + i;
-    const int64_t r = r0 + tx;
-    if (r < rows && c < cols) out[static_cast<int64_t>(c) * ld_out + col0 + r] = tile[tx][i];
-  }
-}
 
 // ------------------------------------------------------------------------- RMSNorm backward
 __device__ __forceinline__ void load4(const __nv_bfloat16* p, float v[4]) {
@@ -179,14 +154,6 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace
-
-cudaError_t launch_transpose_bf16(const void* in, int64_t rows, int cols, int64_t ld_in, void* out, int64_t ld_out,
-                                  int64_t col0, cudaStream_t s) {
-  if (rows == 0 || cols == 0) return cudaSuccess;
-  const dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
-  return launch_pdl(k_transpose_bf16, grid, dim3(256), 0, s, static_cast<const __nv_bfloat16*>(in), rows, cols, ld_in,
-                    static_cast<__nv_bfloat16*>(out), ld_out, col0);
-}
 
 cudaError_t launch_rmsnorm_bwd(const void* x, const float* w, const void* dy, const void* d_in, void* dx,
                                float* partial, int parts, float* dw, int64_t rows, int d, float eps, cudaStream_t s) {

@@ -386,6 +386,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool b_mn_major)
          | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
 }
 
+// The same with either operand MN-major (bit 15: A, bit 16: B).
+__host__ __device__ constexpr uint32_t idesc_bf16_mn(int m, int n, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16(m, n, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
 // D[tmem] (+)= A[tmem] * B[smem], bf16 inputs, fp32 accumulate; A holds M rows in TMEM lanes
 // with two K elements per 32-bit column.  One thread issues.
 __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,

@@ -78,6 +78,7 @@ struct Params {
   const void* l2_next[2];
   size_t l2_next_bytes[2];
   int b_early;
+  int kb_split;  // MJ bit 2: K blocks of B read from tm_b; the rest from tm_b2
 };
 
 // ---------------------------------------------------------------------------- stream-K ranges
@@ -317,7 +318,11 @@ __device__ __forceinline__ float* partial_slot(const Params& p, int c) {
 
 
 
-template <int BN, int EPI, bool PAIR, int KS>
+// MJ: operand major-ness (see GemmArgs::mn_major).  An MN-major operand tile is loaded as
+// 64 x 64 boxes of its stored [K, MN] matrix, one 128-byte-swizzled 8 KB atom column per 64
+// MN indices, the atoms 8 KB apart (the descriptor's leading byte offset) and the 8-row K groups
+// 1 KB apart (its stride byte offset); a K=16 step advances the start address by 2 KB.
+template <int BN, int EPI, bool PAIR, int KS, int MJ = 0>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ CUtensorMap tm_out,
@@ -326,6 +331,9 @@ __global__ void __launch_bounds__(192, 1)
                             (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)),
                 "cluster split-K is built for 256-column (2 or 4 ranks) and 128-column (2 ranks) residual, "
                 "store and GELU tiles");
+  static_assert(MJ == 0 || (EPI == EPI_STORE && !PAIR && KS == 1 && BN % 64 == 0),
+                "MN-major operands are built for whole-tile STORE GEMMs");
+  constexpr bool A_MN = (MJ & 2) != 0, B_MN = (MJ & 1) != 0, B_SPLIT = (MJ & 4) != 0;
   using C = TileCfg<BN, PAIR>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
   constexpr int STAGES = C::STAGES;
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
-    if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tm_b2);
+    if (EPI == EPI_SWIGLU || B_SPLIT) tma_prefetch_desc(&tm_b2);
     tma_prefetch_desc(&tm_out);
   }
   if (warp == 1) {
@@ -411,13 +419,25 @@ __global__ void __launch_bounds__(192, 1)
       const bool arrives = !PAIR || rank == 0;  // posts the expected bytes of the stage
       constexpr uint32_t kStageTx = PAIR ? 2 * C::STAGE : C::STAGE;
       auto load_a = [&](uint8_t* sa, int kb, int m_tile, int s) {
-        if constexpr (PAIR)
+        if constexpr (A_MN) {
+#pragma unroll
+          for (int j = 0; j < BM / 64; ++j) tma_load_2d(sa + j * 8192, &tm_a, &full[s], m_tile * BM + 64 * j, kb * BK);
+        } else if constexpr (PAIR)
           tma_load_2d_pair(sa, &tm_a, full_leader + 8u * s, kb * BK, m_tile * BMT + static_cast<int>(rank) * BM);
         else
           tma_load_2d(sa, &tm_a, &full[s], kb * BK, m_tile * BM);
       };
       auto load_b = [&](uint8_t* sb, int kb, int n_tile, int s) {
-        if constexpr (PAIR) {
+        if constexpr (B_MN) {
+          const CUtensorMap* mb = &tm_b;
+          int kr = kb;
+          if (B_SPLIT && kb >= p.kb_split) {
+            mb = &tm_b2;
+            kr = kb - p.kb_split;
+          }
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, mb, &full[s], n_tile * BN + 64 * j, kr * BK);
+        } else if constexpr (PAIR) {
           // The MMA's B is split along N: rank 0 holds rows [0, BN/2), rank 1 rows [BN/2, BN)
           // (SwiGLU: the gate rows and the up rows).
           if (EPI == EPI_SWIGLU)
@@ -508,7 +528,10 @@ __global__ void __launch_bounds__(192, 1)
       }
     } else if (lane == 0) {
       constexpr bool WIDE = kSwWide<EPI, BN>;
-      constexpr uint32_t idesc = idesc_bf16(BMT, WIDE ? BN / 2 : BN, false);
+      constexpr uint32_t idesc = idesc_bf16_mn(BMT, WIDE ? BN / 2 : BN, A_MN, B_MN);
+      // descriptor advance per K=16 step (address field in 16-byte units): 32 bytes inside a
+      // K-major swizzle atom, two 8-row K groups (2 KB) for an MN-major tile
+      constexpr uint64_t kStepA = A_MN ? 128 : 2, kStepB = B_MN ? 128 : 2;
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -528,8 +551,8 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after_sync();
           const uint32_t a_addr = smem_u32(smem + stage * C::STAGE);
           const uint32_t b_addr = a_addr + C::A_BYTES;
-          const uint64_t adesc = sdesc_sw128(a_addr, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(b_addr, 16, 1024);
+          const uint64_t adesc = sdesc_sw128(a_addr, A_MN ? 8192 : 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(b_addr, B_MN ? 8192 : 16, 1024);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes per K=16 step inside the 128-byte swizzle atom (encoded >> 4).
@@ -542,7 +565,7 @@ __global__ void __launch_bounds__(192, 1)
               umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
               umma_bf16(d_tmem + kSwUp<BN>, adesc + 2 * k, bdesc_up + 2 * k, idesc, accum);
             } else {
-              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, accum);
+              umma_bf16(d_tmem, adesc + kStepA * k, bdesc + kStepB * k, idesc, accum);
             }
           }
           if constexpr (PAIR) umma_commit_pair(&empty[stage]);
@@ -986,11 +1009,11 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int BN, int EPI, bool PAIR = false, int KS = 1>
+template <int BN, int EPI, bool PAIR = false, int KS = 1, int MJ = 0>
 cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   using C = TileCfg<BN, PAIR>;
   static unsigned long long attr_set_mask = 0;  // one bit per device, per instantiation
-  auto kern = k_gemm_tc<BN, EPI, PAIR, KS>;
+  auto kern = k_gemm_tc<BN, EPI, PAIR, KS, MJ>;
   if (PAIR && (plan.grid & 1)) return cudaErrorInvalidValue;
   if (kSwWide<EPI, BN> && (plan.grid != plan.work || plan.splits != 1 || a.n_out % (BN / 2)))
     return cudaErrorInvalidValue;  // one whole tile per CTA (a single accumulator)
@@ -1031,6 +1054,8 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
   p.ss_parts = a.ss_parts;
   p.bias = a.bias;
   p.b_early = a.b_early ? 1 : 0;
+  p.kb_split = a.kb_split;
+  if ((MJ & 4) && (a.kb_split <= 0 || a.kb_split >= plan.kb_total || !a.tm_b2)) return cudaErrorInvalidValue;
   for (int r = 0; r < 2; ++r) {
     p.l2_next[r] = a.l2_next[r];
     p.l2_next_bytes[r] = a.l2_next_bytes[r];
@@ -1038,7 +1063,7 @@ cudaError_t launch_one(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) 
       return cudaErrorInvalidValue;
   }
   const CUtensorMap& ta = *a.tm_a;
-  const CUtensorMap& tb2 = (EPI == EPI_SWIGLU) ? *a.tm_b2 : *a.tm_b;
+  const CUtensorMap& tb2 = (EPI == EPI_SWIGLU || (MJ & 4)) ? *a.tm_b2 : *a.tm_b;
   const CUtensorMap& txw = a.tm_xw ? *a.tm_xw : *a.tm_out;
   if constexpr (PAIR || KS > 1)
     return launch_pdl_cluster(kern, dim3(plan.grid), dim3(192), C::SMEM, s, PAIR ? 2u : static_cast<unsigned>(KS), ta,
@@ -1153,6 +1178,41 @@ constexpr double kClusterCycles = 1000.0;
 }  // namespace
 
 GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes);
+
+GemmPlan plan_gemm_whole(int M, int n_out, int K, int num_sms) {
+  // Whole tiles per CTA only (the grid divides the tile count), 64-, 128- or 256-column tiles,
+  // no cluster split-K: the plans that the MN-major STORE GEMMs are built for.
+  GemmPlan best{};
+  const int kb_total = (K + BK - 1) / BK;
+  if (kb_total <= 0 || M <= 0 || num_sms <= 0) return best;
+  const int tiles_m = (M + BM - 1) / BM;
+  double best_cost = 1e300;
+  for (int bn : {256, 128, 64}) {
+    if (n_out % bn) continue;
+    const long long tiles = static_cast<long long>(tiles_m) * (n_out / bn);
+    for (long long g = std::min<long long>(num_sms, tiles); g >= 1; --g) {
+      if (tiles % g) continue;
+      int contrib = 1;
+      const double cost = plan_cost(bn, tiles, kb_total, static_cast<int>(g), &contrib);
+      if (contrib == 1 && cost < best_cost - 1e-9) {
+        best_cost = cost;
+        best.bn = bn;
+        best.pair = 0;
+        best.ks = 1;
+        best.splits = 1;
+        best.tiles_m = tiles_m;
+        best.tiles_n = n_out / bn;
+        best.kb_total = kb_total;
+        best.work = static_cast<int>(tiles);
+        best.grid = static_cast<int>(g);
+        best.partial_bytes = 0;
+        best.counters = 0;
+      }
+      break;  // the largest divisor that fits: more CTAs only add parallelism
+    }
+  }
+  return best;
+}
 
 GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes) {
   // Plans depend only on the shape (and the scratch cap); each thread keeps the ones it has
@@ -1314,7 +1374,28 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
   return best;
 }
 
+// Whole-tile STORE GEMMs with MN-major operands (the backward's input and weight gradients).
+template <int MJ>
+cudaError_t launch_bn_mn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
+  if (plan.pair || plan.ks != 1 || plan.splits != 1) return cudaErrorInvalidValue;
+  switch (plan.bn) {
+    case 64: return launch_one<64, EPI_STORE, false, 1, MJ>(plan, a, s);
+    case 128: return launch_one<128, EPI_STORE, false, 1, MJ>(plan, a, s);
+    case 256: return launch_one<256, EPI_STORE, false, 1, MJ>(plan, a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_gemm_tc(int epi, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
+  if (a.mn_major != 0) {
+    if (epi != EPI_STORE) return cudaErrorInvalidValue;
+    switch (a.mn_major) {
+      case 1: return launch_bn_mn<1>(plan, a, s);
+      case 3: return launch_bn_mn<3>(plan, a, s);
+      case 5: return launch_bn_mn<5>(plan, a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (epi) {
     case EPI_STORE: return launch_bn<EPI_STORE>(plan, a, s);
     case EPI_RESID: return launch_bn<EPI_RESID>(plan, a, s);

@@ -35,6 +35,9 @@ inline int norm_parts_of(const GemmPlan& p) { return p.tiles_n * (p.ks > 1 ? p.k
 // Chooses tile width, CTA pairing and split count for a GEMM of this shape on `num_sms` SMs;
 // plans whose split-tile partials exceed max_partial_bytes are not considered.
 GemmPlan plan_gemm(int epi, int M, int n_out, int K, int num_sms, size_t max_partial_bytes = SIZE_MAX);
+// Whole-tile plans (the grid divides the tile count) with 64-, 128- or 256-column tiles and no
+// cluster split-K: what GemmArgs::mn_major supports.
+GemmPlan plan_gemm_whole(int M, int n_out, int K, int num_sms);
 
 struct GemmArgs {
   const CUtensorMap* tm_out;  // output [M, n_out] bf16, box 64 x 32 (TMA stores of the epilogue)
@@ -74,6 +77,12 @@ struct GemmArgs {
   // once their own operand loads are issued (NULL: none; 16-byte aligned, bytes a multiple of 16).
   const void* l2_next[2];
   size_t l2_next_bytes[2];
+  // Operand major-ness (STORE epilogue, whole-tile plans without cluster split-K only): bit 0,
+  // B is MN-major: tm_b describes the stored [K, n] matrix (n contiguous), box 64 x 64; bit 1, A
+  // is MN-major: tm_a describes the stored [K, M] matrix, box 64 x 64; bit 2 (with bit 0), the
+  // K extent of B continues in tm_b2 from K block kb_split on (B = [B1; B2] stacked along K).
+  int mn_major;
+  int kb_split;
 };
 
 cudaError_t launch_gemm_tc(int epi, const GemmPlan& plan, const GemmArgs& a, cudaStream_t s);
@@ -176,8 +185,6 @@ cudaError_t launch_ln_merge(bool bf16, const void* x, const int32_t* src, const 
 cudaError_t launch_selftest_wait(uint64_t limit_ns, uint32_t* err, cudaStream_t s);
 // Backward of the block (backward.cu).  All bf16 except the fp32 norm weights, their gradients,
 // the rotation tables and the attention row statistics.
-cudaError_t launch_transpose_bf16(const void* in, int64_t rows, int cols, int64_t ld_in, void* out, int64_t ld_out,
-                                  int64_t col0, cudaStream_t s);
 cudaError_t launch_rmsnorm_bwd(const void* x, const float* w, const void* dy, const void* d_in, void* dx,
                                float* partial, int parts, float* dw, int64_t rows, int d, float eps, cudaStream_t s);
 cudaError_t launch_swiglu_bwd(const void* g, const void* u, const void* dh, void* dgu, void* h, int64_t rows, int f,
