@@ -1536,7 +1536,12 @@ dsv4v_status gemm_store(const Ctx& c, const void* a, int64_t M, int K, int64_t l
 // (row stride ldb; with b2, its rows from kb_split * 64 on are b2's rows), else [n_out, K].
 dsv4v_status gemm_store_mn(const Ctx& c, const void* a, int64_t M, int K, int64_t lda, bool a_mn, const void* b,
                            int64_t ldb, bool b_mn, int n_out, void* out, const void* b2 = nullptr, int kb_split = 0) {
-  const GemmPlan plan = plan_gemm_whole(static_cast<int>(M), n_out, K, c.dev.sms);
+  // With A K-major (input gradients, whose K can be long) the planner's cluster split-K plans
+  // are allowed too; with an MN-major A (weight gradients, K = the packed rows) whole tiles.
+  GemmPlan plan{};
+  if (!a_mn) plan = plan_gemm(EPI_STORE, static_cast<int>(M), n_out, K, c.dev.sms, 0);
+  if (a_mn || plan.bn == 192 || plan.bn == 0 || (plan.ks > 1 && !b_mn))
+    plan = plan_gemm_whole(static_cast<int>(M), n_out, K, c.dev.sms);
   if (plan.bn == 0) return DSV4V_ERR_UNSUPPORTED;
   GemmExtra ex;
   ex.lda = lda;

@@ -33,18 +33,19 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, const float v[4]) {
 }
 
 // y = w * x * r, r = 1 / sqrt(mean(x^2) + eps).  One warp per row (grid-stride): with
-// g = dy * w, dx = r g - x r^3 (g . x) / d (+ d_in); the CTA's share of dw = sum dy * x * r is
-// summed in shared memory and stored as partial[blockIdx.x][d].  d % 128 == 0.
+// g = dy * w, dx = r g - x r^3 (g . x) / d (+ d_in).  dw = sum dy * x * r: each warp adds its
+// rows' terms into its own row of shared memory (no atomics, no contention), then the CTA sums
+// the warps' rows in warp order into partial[blockIdx.x][d].  d % 128 == 0.
 __global__ void __launch_bounds__(256)
     k_rmsnorm_bwd(const __nv_bfloat16* __restrict__ x, const float* __restrict__ w, const __nv_bfloat16* dy,
                   const __nv_bfloat16* d_in, __nv_bfloat16* dx, float* __restrict__ partial, int64_t rows, int d,
                   float eps) {
-  extern __shared__ float sdw[];  // [d]
+  extern __shared__ float sdw[];  // [warps][d]
   grid_dependency_wait();
   launch_dependents();
-  for (int c = threadIdx.x; c < d; c += blockDim.x) sdw[c] = 0.0f;
-  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+  float* my = sdw + static_cast<size_t>(warp) * d;
+  for (int c = lane * 4; c < d; c += 128) *reinterpret_cast<float4*>(my + c) = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * n_warps + warp; row < rows;
        row += static_cast<int64_t>(gridDim.x) * n_warps) {
     const __nv_bfloat16* xr = x + row * d;
@@ -73,27 +74,46 @@ __global__ void __launch_bounds__(256)
       const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
       float din[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       if (d_in) load4(d_in + row * d + c, din);
+      float4 acc = *reinterpret_cast<const float4*>(my + c);
+      acc.x += dv[0] * xv[0] * r;
+      acc.y += dv[1] * xv[1] * r;
+      acc.z += dv[2] * xv[2] * r;
+      acc.w += dv[3] * xv[3] * r;
+      *reinterpret_cast<float4*>(my + c) = acc;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        out[k] = r * dv[k] * wa[k] - xv[k] * coef + din[k];
-        atomicAdd(&sdw[c + k], dv[k] * xv[k] * r);
-      }
+      for (int k = 0; k < 4; ++k) out[k] = r * dv[k] * wa[k] - xv[k] * coef + din[k];
       store4(dx + row * d + c, out);
     }
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < d; c += blockDim.x) partial[static_cast<int64_t>(blockIdx.x) * d + c] = sdw[c];
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float t = 0.0f;
+    for (int wi = 0; wi < n_warps; ++wi) t += sdw[static_cast<size_t>(wi) * d + c];
+    partial[static_cast<int64_t>(blockIdx.x) * d + c] = t;
+  }
 }
 
-// out[c] = sum over p < parts of partial[p][c], in order.
-__global__ void k_sum_parts(const float* __restrict__ partial, int parts, int d, float* __restrict__ out) {
+// out[c] = sum over p < parts of partial[p][c] in a fixed order: warp y of a CTA of 8 warps
+// sums parts y, y + 8, y + 16, ... of 32 consecutive columns (coalesced), then the 8 warp sums
+// are added in warp order.  Deterministic.
+__global__ void __launch_bounds__(256) k_sum_parts(const float* __restrict__ partial, int parts, int d,
+                                                   float* __restrict__ out) {
+  __shared__ float part_sum[8][32];
   grid_dependency_wait();
   launch_dependents();
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= d) return;
-  float s = 0.0f;
-  for (int p = 0; p < parts; ++p) s += partial[static_cast<int64_t>(p) * d + c];
-  out[c] = s;
+  const int lane = threadIdx.x & 31, wy = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
+  float t = 0.0f;
+  if (c < d)
+    for (int p = wy; p < parts; p += 8) t += partial[static_cast<int64_t>(p) * d + c];
+  part_sum[wy][lane] = t;
+  __syncthreads();
+  if (wy == 0 && c < d) {
+    float v = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v += part_sum[k][lane];
+    out[c] = v;
+  }
 }
 
 // -------------------------------------------------------------------------- SwiGLU backward
@@ -132,24 +152,44 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------------ inverse rotation
 // In place on the q and k columns of dqkv [P, 3D]: each half-split pair (j, j + hd/2) of a head
 // is turned back by its angle: (d1, d2) <- (d1 c + d2 s, d2 c - d1 s).  cos/sin: [P, hd/2].
+// One thread per row and 8 consecutive pairs of one head (16-byte loads of each half; hd/2 is
+// a multiple of 8), CTAs striding over the rows.
 __global__ void __launch_bounds__(256)
     k_rotary_bwd(__nv_bfloat16* dqkv, const float* __restrict__ cos, const float* __restrict__ sin, int64_t P, int D,
                  int hd) {
   grid_dependency_wait();
   launch_dependents();
   const int half = hd / 2;
-  const int64_t n = P * D;  // pairs: D per row (D / 2 in q, D / 2 in k)
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t p = i / D;
-    const int j = static_cast<int>(i - p * D);
-    const int part = j / (D / 2), jj = j - part * (D / 2);
-    const int head = jj / half, e = jj - head * half;
-    const int64_t col1 = p * 3 * D + part * D + head * hd + e;
-    const float c = cos[p * half + e], s = sin[p * half + e];
-    const float d1 = __bfloat162float(dqkv[col1]), d2 = __bfloat162float(dqkv[col1 + half]);
-    dqkv[col1] = __float2bfloat16_rn(d1 * c + d2 * s);
-    dqkv[col1 + half] = __float2bfloat16_rn(d2 * c - d1 * s);
+  const int groups = D / 8;  // per row: D / 2 pairs in q and D / 2 in k, 8 per group
+  const int per_part = groups / 2;
+  for (int64_t p = blockIdx.x; p < P; p += gridDim.x) {
+    for (int gi = threadIdx.x; gi < groups; gi += blockDim.x) {
+      const int part = gi >= per_part ? 1 : 0;
+      const int jj0 = (gi - part * per_part) * 8;
+      const int head = jj0 / half, e0 = jj0 - head * half;
+      __nv_bfloat16* a = dqkv + p * 3 * D + part * D + head * hd + e0;
+      const uint4 ra = *reinterpret_cast<const uint4*>(a);
+      const uint4 rb = *reinterpret_cast<const uint4*>(a + half);
+      const float4 c0 = *reinterpret_cast<const float4*>(cos + p * half + e0);
+      const float4 c1 = *reinterpret_cast<const float4*>(cos + p * half + e0 + 4);
+      const float4 s0 = *reinterpret_cast<const float4*>(sin + p * half + e0);
+      const float4 s1 = *reinterpret_cast<const float4*>(sin + p * half + e0 + 4);
+      const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const __nv_bfloat16* va = reinterpret_cast<const __nv_bfloat16*>(&ra);
+      const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(&rb);
+      uint4 oa, ob;
+      __nv_bfloat16* wa = reinterpret_cast<__nv_bfloat16*>(&oa);
+      __nv_bfloat16* wb = reinterpret_cast<__nv_bfloat16*>(&ob);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float d1 = __bfloat162float(va[k]), d2 = __bfloat162float(vb[k]);
+        wa[k] = __float2bfloat16_rn(d1 * cs[k] + d2 * sn[k]);
+        wb[k] = __float2bfloat16_rn(d2 * cs[k] - d1 * sn[k]);
+      }
+      *reinterpret_cast<uint4*>(a) = oa;
+      *reinterpret_cast<uint4*>(a + half) = ob;
+    }
   }
 }
 
@@ -157,13 +197,25 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_rmsnorm_bwd(const void* x, const float* w, const void* dy, const void* d_in, void* dx,
                                float* partial, int parts, float* dw, int64_t rows, int d, float eps, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(d) * sizeof(float);
+  const size_t smem = static_cast<size_t>(d) * sizeof(float) * 8;  // one row of dw per warp
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
+  static int attr_dev = -1;
+  if (smem > 48 * 1024) {
+    int dev = 0;
+    cudaError_t ea = cudaGetDevice(&dev);
+    if (ea != cudaSuccess) return ea;
+    if (attr_dev != dev) {
+      ea = cudaFuncSetAttribute(k_rmsnorm_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+      if (ea != cudaSuccess) return ea;
+      attr_dev = dev;
+    }
+  }
   cudaError_t e = launch_pdl(k_rmsnorm_bwd, dim3(static_cast<unsigned>(parts)), dim3(256), smem, s,
                              static_cast<const __nv_bfloat16*>(x), w, static_cast<const __nv_bfloat16*>(dy),
                              static_cast<const __nv_bfloat16*>(d_in), static_cast<__nv_bfloat16*>(dx), partial, rows, d,
                              eps);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k_sum_parts, dim3(static_cast<unsigned>((d + 255) / 256)), dim3(256), 0, s,
+  return launch_pdl(k_sum_parts, dim3(static_cast<unsigned>((d + 31) / 32)), dim3(256), 0, s,
                     static_cast<const float*>(partial), parts, d, dw);
 }
 
@@ -180,10 +232,11 @@ cudaError_t launch_swiglu_bwd(const void* g, const void* u, const void* dh, void
 
 cudaError_t launch_rotary_bwd(void* dqkv, const float* cos, const float* sin, int64_t P, int D, int hd, int sms,
                               cudaStream_t s) {
-  const int64_t n = P * D;
-  if (n == 0) return cudaSuccess;
-  const int64_t blocks = std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(sms) * 8);
-  return launch_pdl(k_rotary_bwd, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+  if (P == 0) return cudaSuccess;
+  if (D % 16 || (hd / 2) % 8) return cudaErrorInvalidValue;
+  const int threads = std::min(256, (D / 8 + 31) / 32 * 32);
+  const int64_t blocks = std::min<int64_t>(P, static_cast<int64_t>(sms) * 8);
+  return launch_pdl(k_rotary_bwd, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, s,
                     static_cast<__nv_bfloat16*>(dqkv), cos, sin, P, D, hd);
 }
 

@@ -331,8 +331,9 @@ __global__ void __launch_bounds__(192, 1)
                             (EPI == EPI_RESID || EPI == EPI_STORE || EPI == EPI_GELU)),
                 "cluster split-K is built for 256-column (2 or 4 ranks) and 128-column (2 ranks) residual, "
                 "store and GELU tiles");
-  static_assert(MJ == 0 || (EPI == EPI_STORE && !PAIR && KS == 1 && BN % 64 == 0),
-                "MN-major operands are built for whole-tile STORE GEMMs");
+  static_assert(MJ == 0 || (EPI == EPI_STORE && !PAIR && (KS == 1 || (MJ & 2) == 0) && BN % 64 == 0),
+                "MN-major operands are built for whole-tile STORE GEMMs (with an MN-major A, without "
+                "cluster split-K)");
   constexpr bool A_MN = (MJ & 2) != 0, B_MN = (MJ & 1) != 0, B_SPLIT = (MJ & 4) != 0;
   using C = TileCfg<BN, PAIR>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
@@ -1377,7 +1378,16 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
 // Whole-tile STORE GEMMs with MN-major operands (the backward's input and weight gradients).
 template <int MJ>
 cudaError_t launch_bn_mn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
-  if (plan.pair || plan.ks != 1 || plan.splits != 1) return cudaErrorInvalidValue;
+  if (plan.pair || plan.splits != 1) return cudaErrorInvalidValue;
+  if (plan.ks > 1) {
+    // cluster split-K (input gradients with a long K): B MN-major only
+    if constexpr ((MJ & 2) == 0) {
+      if (plan.bn == 128 && plan.ks == 2) return launch_one<128, EPI_STORE, false, 2, MJ>(plan, a, s);
+      if (plan.bn == 256 && plan.ks == 2) return launch_one<256, EPI_STORE, false, 2, MJ>(plan, a, s);
+      if (plan.bn == 256 && plan.ks == 4) return launch_one<256, EPI_STORE, false, 4, MJ>(plan, a, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (plan.bn) {
     case 64: return launch_one<64, EPI_STORE, false, 1, MJ>(plan, a, s);
     case 128: return launch_one<128, EPI_STORE, false, 1, MJ>(plan, a, s);
