@@ -197,8 +197,8 @@ enum { DSV4V_PATH_AUTO = 0, DSV4V_PATH_KERNELS = 1, DSV4V_PATH_CHAIN = 2 };
  * it.  Returns DSV4V_ERR_INVALID_ARG for an unknown value. */
 dsv4v_status dsv4v_set_tower_path(int path);
 
-/* Graph replay of the step calls (dsv4v_tower_forward, dsv4v_aligner_forward).  The library
- * keeps up to 16 CUDA graph executables keyed by every argument that shapes a call's launches:
+/* Graph replay of the step calls (dsv4v_tower_forward, dsv4v_aligner_forward).  Each host
+ * thread keeps up to 16 CUDA graph executables keyed by every argument that shapes a call's launches:
  * the config and batch values, the batch's device pointers, the weight, buffer and workspace
  * pointers, the launch sequence (dsv4v_set_tower_path) and the current device.  The first call
  * with a key launches its kernels directly; the second captures them on the caller's stream
@@ -208,8 +208,9 @@ dsv4v_status dsv4v_set_tower_path(int path);
  * captured (the caller's own graph) always launch directly.  A capture or instantiation that
  * fails leaves that key on direct launches (the call still runs).
  * dsv4v_set_graph_replay(0) turns the cache off for the calls that follow (process-wide host
- * state; default on); dsv4v_release_graphs() destroys every cached executable (one still running
- * is freed when it completes).  Neither needs a GPU or fails. */
+ * state; default on); dsv4v_release_graphs() destroys the calling thread's cached executables
+ * (one still running is freed when it completes); a thread that exits without calling it leaves
+ * its executables to the driver's teardown.  Neither needs a GPU or fails. */
 void dsv4v_set_graph_replay(int enable);
 void dsv4v_release_graphs(void);
 

@@ -857,14 +857,14 @@ dsv4v_status linear_residual_with_scratch(const dsv4v_config* cfg, int64_t rows,
 // ----------------------------------------------------------------------------- graph replay
 // A step of the 28x28 tower is ~170 launches of ~11 us each, so launching them one by one from
 // the host costs a few percent against replaying them as one CUDA graph.  The step entry points
-// therefore keep a small cache of graph executables keyed by every argument that shapes their
-// launches (the config, the batch's host arrays and device pointers, the weight, buffer and
-// workspace pointers, the launch-sequence setting, the device).  The first call with a key runs
-// eagerly (it also warms the plan and descriptor caches); the second captures the launches on
-// the caller's stream (thread-local capture) and replays the instantiated graph, as do all
-// later calls.  Calls on the legacy default stream, or on a stream that is already being
-// captured (the caller's own graph), always launch directly.  A capture or instantiation that
-// fails leaves that key on direct launches.
+// therefore keep a small per-thread cache of graph executables (like the tensor-map cache)
+// keyed by every argument that shapes their launches (the config, the batch's host arrays and
+// device pointers, the weight, buffer and workspace pointers, the launch-sequence setting, the
+// device).  The first call with a key runs eagerly (it also warms the plan and descriptor
+// caches); the second captures the launches on the caller's stream (thread-local capture) and
+// replays the instantiated graph, as do all later calls.  Calls on the legacy default stream,
+// or on a stream that is already being captured (the caller's own graph), always launch
+// directly.  A capture or instantiation that fails leaves that key on direct launches.
 struct GraphEntry {
   std::vector<uint64_t> key;
   cudaGraphExec_t exec = nullptr;
@@ -872,9 +872,8 @@ struct GraphEntry {
   uint64_t last_use = 0;
 };
 
-std::mutex g_graph_mu;
-std::vector<GraphEntry> g_graphs;
-uint64_t g_graph_clock = 0;
+thread_local std::vector<GraphEntry> g_graphs;
+thread_local uint64_t g_graph_clock = 0;
 std::atomic<int> g_graph_replay{1};
 constexpr size_t kMaxGraphs = 16;
 
@@ -920,7 +919,6 @@ dsv4v_status with_graph(KeyBuilder&& kb, void* stream, Run&& run) {
     return run();
   }
   if (cs != cudaStreamCaptureStatusNone) return run();
-  std::lock_guard<std::mutex> lk(g_graph_mu);
   GraphEntry* e = nullptr;
   for (auto& g : g_graphs)
     if (g.key == kb.k) {
@@ -975,7 +973,6 @@ extern "C" {
 void dsv4v_set_graph_replay(int enable) { g_graph_replay.store(enable ? 1 : 0); }
 
 void dsv4v_release_graphs(void) {
-  std::lock_guard<std::mutex> lk(g_graph_mu);
   for (auto& g : g_graphs)
     if (g.exec) cudaGraphExecDestroy(g.exec);
   g_graphs.clear();
