@@ -338,9 +338,8 @@ const char* dsv4v_status_string(dsv4v_status s);
 /* ---------------------------------------------------------------- backward
  * The gradient of the tower ([PR], Validation: the pages train the tower and test "ragged grids
  * and backward"; no backward is printed, so each call is the chain rule through the forward
- * above).  bf16 configs only, and at most 2,097,120 patches per batch (DSV4V_ERR_UNSUPPORTED
- * otherwise): activations and gradients are bf16, norm weights and their gradients fp32, GEMMs
- * accumulate in fp32.  Every call takes the scratch of dsv4v_backward_workspace_size and writes
+ * above).  bf16 configs only (DSV4V_ERR_UNSUPPORTED otherwise): activations and gradients are
+ * bf16, norm weights and their gradients fp32, GEMMs accumulate in fp32.  Every call takes the scratch of dsv4v_backward_workspace_size and writes
  * its outputs (gradients are not accumulated into the destination). */
 
 /* Weight gradients of one block, laid out like dsv4v_block_weights: norm1_w, norm2_w fp32 [D];
