@@ -332,8 +332,8 @@ __global__ void __launch_bounds__(192, 1)
                 "cluster split-K is built for 256-column (2 or 4 ranks) and 128-column (2 ranks) residual, "
                 "store and GELU tiles");
   static_assert(MJ == 0 || (EPI == EPI_STORE && !PAIR && (KS == 1 || (MJ & 2) == 0) && BN % 64 == 0),
-                "MN-major operands are built for whole-tile STORE GEMMs (with an MN-major A, without "
-                "cluster split-K)");
+                "MN-major operands are built for STORE GEMMs without CTA pairs (with an MN-major A, "
+                "without cluster split-K)");
   constexpr bool A_MN = (MJ & 2) != 0, B_MN = (MJ & 1) != 0, B_SPLIT = (MJ & 4) != 0;
   using C = TileCfg<BN, PAIR>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // rows of an output tile
@@ -1375,7 +1375,8 @@ GemmPlan plan_gemm_uncached(int epi, int M, int n_out, int K, int num_sms, size_
   return best;
 }
 
-// Whole-tile STORE GEMMs with MN-major operands (the backward's input and weight gradients).
+// STORE GEMMs with MN-major operands (the backward's input and weight gradients): whole tiles
+// per CTA, or cluster split-K when A is K-major.
 template <int MJ>
 cudaError_t launch_bn_mn(const GemmPlan& plan, const GemmArgs& a, cudaStream_t s) {
   if (plan.pair || plan.splits != 1) return cudaErrorInvalidValue;

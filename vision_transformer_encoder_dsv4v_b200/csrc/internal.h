@@ -77,7 +77,7 @@ struct GemmArgs {
   // once their own operand loads are issued (NULL: none; 16-byte aligned, bytes a multiple of 16).
   const void* l2_next[2];
   size_t l2_next_bytes[2];
-  // Operand major-ness (STORE epilogue, whole-tile plans without cluster split-K only): bit 0,
+  // Operand major-ness (STORE epilogue; whole-tile plans, or cluster split-K when A is K-major): bit 0,
   // B is MN-major: tm_b describes the stored [K, n] matrix (n contiguous), box 64 x 64; bit 1, A
   // is MN-major: tm_a describes the stored [K, M] matrix, box 64 x 64; bit 2 (with bit 0), the
   // K extent of B continues in tm_b2 from K block kb_split on (B = [B1; B2] stacked along K).
