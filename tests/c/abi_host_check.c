@@ -34,6 +34,10 @@ int main(void) {
   check(types[0] == DSV4V_TOKEN_START && types[4] == DSV4V_TOKEN_NEWLINE && types[9] == DSV4V_TOKEN_END &&
             types[1] == DSV4V_TOKEN_IMAGE,
         "layout contents");
+  /* graph replay switch and release: host state only, no GPU needed */
+  dsv4v_set_graph_replay(0);
+  dsv4v_release_graphs();
+  dsv4v_set_graph_replay(1);
   check(strcmp(dsv4v_status_string(DSV4V_OK), "ok") == 0, "status string");
   check(dsv4v_status_string(DSV4V_ERR_LAYOUT) != NULL, "layout status string");
 

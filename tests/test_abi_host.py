@@ -213,6 +213,17 @@ def test_tower_path_choice_and_validation():
         A.dsv4v_set_tower_path(A.PATH_AUTO)
 
 
+def test_graph_replay_switch_needs_no_gpu():
+    """The step calls' graph-replay switch and the release of the calling thread's cached
+    executables are host state only: both run without a GPU, repeatedly, and in any order."""
+    from vision_transformer_encoder_dsv4v_b200 import dsv4v as A
+    for _ in range(2):
+        A.dsv4v_release_graphs()
+        A.dsv4v_set_graph_replay(False)
+        A.dsv4v_release_graphs()
+        A.dsv4v_set_graph_replay(True)
+
+
 def test_step_launch_count():
     """The per-step launch count the benchmark reports: rotary table, first norm operand, per
     layer 4 GEMMs + attention (or attention + one chain launch), final norm, aligner (window
